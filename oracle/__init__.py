@@ -1,0 +1,203 @@
+"""CPU oracle for the NVFP4 mixture-of-experts hot path (test infrastructure).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports, links or calls it.
+
+The arithmetic lives in ``nvfp4_oracle.c`` (plain C, float64 for the layer,
+IEEE FP32 for the integer-producing decisions); this module only compiles it
+with gcc and marshals numpy arrays through ctypes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nvfp4_oracle.c")
+_LIB = os.path.join(_HERE, "libnvfp4_oracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (OpenMP over tokens for the layer)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+               "-fno-fast-math", _SRC, "-o", _LIB + ".tmp", "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        _lib = ctypes.CDLL(_LIB)
+        L = _lib
+        L.orc_e2m1_value.restype = ctypes.c_double
+        L.orc_e2m1_value.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_value.restype = ctypes.c_double
+        L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.orc_e8m0_value.restype = ctypes.c_double
+        L.orc_e8m0_value.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_rne_satfinite.restype = ctypes.c_uint8
+        L.orc_e4m3_rne_satfinite.argtypes = [ctypes.c_float]
+        L.orc_e2m1_rne_sat.restype = ctypes.c_uint8
+        L.orc_e2m1_rne_sat.argtypes = [ctypes.c_float]
+        L.orc_exp_spec.restype = ctypes.c_float
+        L.orc_exp_spec.argtypes = [ctypes.c_float]
+        L.orc_sigmoid_spec.restype = ctypes.c_float
+        L.orc_sigmoid_spec.argtypes = [ctypes.c_float]
+        L.orc_float_to_bf16.restype = ctypes.c_uint16
+        L.orc_float_to_bf16.argtypes = [ctypes.c_float]
+        L.orc_transcode.restype = ctypes.c_int
+        L.orc_num_threads.restype = ctypes.c_int
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# --- scalar codecs -----------------------------------------------------------
+
+def e2m1_value(code: int) -> float:
+    return _load().orc_e2m1_value(code)
+
+
+def e4m3_value(byte: int) -> float:
+    return _load().orc_e4m3_value(byte)
+
+
+def e8m0_value(byte: int) -> float:
+    return _load().orc_e8m0_value(byte)
+
+
+def e4m3_rne_satfinite(x: float) -> int:
+    return _load().orc_e4m3_rne_satfinite(x)
+
+
+def e2m1_rne_sat(x: float) -> int:
+    return _load().orc_e2m1_rne_sat(x)
+
+
+def exp_spec(y: float) -> float:
+    return _load().orc_exp_spec(y)
+
+
+def sigmoid_spec(x: float) -> float:
+    return _load().orc_sigmoid_spec(x)
+
+
+def float_to_bf16(x: float) -> int:
+    return _load().orc_float_to_bf16(x)
+
+
+def num_threads() -> int:
+    return _load().orc_num_threads()
+
+
+# --- tensors -------------------------------------------------------------------
+
+def decode_mxfp4(codes: np.ndarray, e8m0: np.ndarray, N: int, K: int) -> np.ndarray:
+    out = np.empty((N, K), np.float64)
+    _load().orc_decode_mxfp4(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(e8m0)),
+                             ctypes.c_int64(N), ctypes.c_int64(K), _p(out))
+    return out
+
+
+def decode_nvfp4(codes: np.ndarray, e4m3: np.ndarray, global_scale: float, N: int, K: int) -> np.ndarray:
+    out = np.empty((N, K), np.float64)
+    _load().orc_decode_nvfp4(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(e4m3)),
+                             ctypes.c_float(global_scale), ctypes.c_int64(N), ctypes.c_int64(K), _p(out))
+    return out
+
+
+def transcode(codes: np.ndarray, e8m0: np.ndarray, num_tensors: int, N: int, K: int):
+    """Returns (codes_out, e4m3 [nt, N, K/16], global [nt] f32, status [nt] i32,
+    report [blocks, zero_blocks, nonrepresentable_tensors, nan_tensors], worst)."""
+    codes = np.ascontiguousarray(codes, np.uint8)
+    e8m0 = np.ascontiguousarray(e8m0, np.uint8)
+    codes_out = np.empty(num_tensors * N * K // 2, np.uint8)
+    e4m3 = np.empty((num_tensors, N, K // 16), np.uint8)
+    glob = np.empty(num_tensors, np.float32)
+    status = np.empty(num_tensors, np.int32)
+    report = np.zeros(4, np.int64)
+    worst = _load().orc_transcode(_p(codes), _p(e8m0), ctypes.c_int64(num_tensors), ctypes.c_int64(N),
+                                  ctypes.c_int64(K), _p(codes_out), _p(e4m3), _p(glob), _p(status), _p(report))
+    return codes_out.reshape(num_tensors, N, K // 2), e4m3, glob, status, report, worst
+
+
+def route(logits: np.ndarray, bias, n_group: int, topk_group: int, top_k: int, rsf: float,
+          renormalize: bool = True):
+    logits = np.ascontiguousarray(logits, np.float32)
+    T, E = logits.shape
+    ids = np.empty((T, top_k), np.int32)
+    w = np.empty((T, top_k), np.float32)
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    _load().orc_route(_p(logits), None if b is None else _p(b), ctypes.c_int(T), ctypes.c_int(E),
+                      ctypes.c_int(n_group), ctypes.c_int(topk_group), ctypes.c_int(top_k), ctypes.c_float(rsf),
+                      ctypes.c_int(int(renormalize)), _p(ids), _p(w))
+    return ids, w
+
+
+def permute(topk_ids: np.ndarray, E: int):
+    ids = np.ascontiguousarray(topk_ids, np.int32)
+    T, k = ids.shape
+    P = T * k
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    row_of_pair = np.empty(P, np.int32)
+    pair_of_row = np.empty(P, np.int32)
+    _load().orc_permute(_p(ids), ctypes.c_int(T), ctypes.c_int(k), ctypes.c_int(E), _p(counts), _p(offsets),
+                        _p(row_of_pair), _p(pair_of_row))
+    return counts, offsets, row_of_pair, pair_of_row
+
+
+def quantize_bf16(x_bits: np.ndarray, gs: float = 1.0):
+    """x_bits: uint16 BF16 bit patterns [M, K]. Returns codes [M, K/2], scales [M, K/16]."""
+    x = np.ascontiguousarray(x_bits, np.uint16)
+    M, K = x.shape
+    codes = np.empty((M, K // 2), np.uint8)
+    scales = np.empty((M, K // 16), np.uint8)
+    _load().orc_quantize_bf16(_p(x), ctypes.c_int64(M), ctypes.c_int64(K), ctypes.c_float(gs), _p(codes),
+                              _p(scales))
+    return codes, scales
+
+
+def quantize_f32(x: np.ndarray, gs: float = 1.0):
+    x = np.ascontiguousarray(x, np.float32)
+    M, K = x.shape
+    codes = np.empty((M, K // 2), np.uint8)
+    scales = np.empty((M, K // 16), np.uint8)
+    _load().orc_quantize_f32(_p(x), ctypes.c_int64(M), ctypes.c_int64(K), ctypes.c_float(gs), _p(codes),
+                             _p(scales))
+    return codes, scales
+
+
+def moe_layer(mode: int, x_bits, logits, bias, gate_codes, gate_sf, up_codes, up_sf, down_codes, down_sf,
+              w_global, act_global: float, n_group: int, topk_group: int, top_k: int, rsf: float,
+              renormalize: bool = True, tokens=None) -> np.ndarray:
+    """float64 layer output [len(tokens), H] (mode 0 = W4A16, 1 = W4A4)."""
+    x = np.ascontiguousarray(x_bits, np.uint16)
+    T, H = x.shape
+    E, I = gate_codes.shape[0], gate_codes.shape[1]
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int32)
+    tokens = np.ascontiguousarray(tokens, np.int32)
+    out = np.empty((len(tokens), H), np.float64)
+    arrs = [np.ascontiguousarray(a, np.uint8) for a in (gate_codes, gate_sf, up_codes, up_sf, down_codes, down_sf)]
+    lg = np.ascontiguousarray(logits, np.float32)
+    wg = np.ascontiguousarray(w_global, np.float32)
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    _load().orc_moe_layer(ctypes.c_int(mode), _p(x), _p(lg), None if b is None else _p(b), *[_p(a) for a in arrs],
+                          _p(wg), ctypes.c_float(act_global), ctypes.c_int(T), ctypes.c_int(H), ctypes.c_int(I),
+                          ctypes.c_int(E), ctypes.c_int(n_group), ctypes.c_int(topk_group), ctypes.c_int(top_k),
+                          ctypes.c_float(rsf), ctypes.c_int(int(renormalize)), _p(tokens), ctypes.c_int(len(tokens)),
+                          _p(out))
+    return out

@@ -1,0 +1,519 @@
+/*
+ * nvfp4_oracle.c -- plain, slow CPU oracle for the routed-expert MoE layer with
+ * 4-bit block-scaled expert weights.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls
+ * this file: only the tests, the smoke check and the CPU-baseline leg of the
+ * benchmark do.  It shares no code, header, table or constant generator with the
+ * CUDA library; every table here is built from the format definitions below.
+ *
+ * Sources (web pages; cited by page title and section):
+ *  [P1] "AxionML / MiMo-V2.6-Flash-MOPD-NVFP4" model card: introduction,
+ *       "About NVFP4 quantization", "Quantization Details / Why a unit activation
+ *       scale", "Reproduce the checkpoint".
+ *  [P2] "ProCreations/MiMo-V2.6-Flash-RL-NVFP4": "What changed", "Verification".
+ *  [P4] "MiMo-V2.6-Flash -- REAP-50": "Model Summary", "Pruning Method" section 1
+ *       (grouped sigmoid top-k router and the SwiGLU expert formula).
+ *
+ * Arithmetic: floating point decisions that produce integers (quantised codes,
+ * routing choices) are taken in IEEE FP32, exactly as written below; everything
+ * else (GEMMs, SwiGLU, the combine) is float64.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------- */
+/* Codebooks                                                                  */
+/* ------------------------------------------------------------------------- */
+
+/* E2M1 (FP4): 1 sign, 2 exponent, 1 mantissa bit; magnitudes up to 6, no NaN
+ * or Inf ([P1] "About NVFP4 quantization").  Decoded by an explicit table. */
+static const double E2M1_MAGNITUDE[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double orc_e2m1_value(uint8_t code) {
+    double m = E2M1_MAGNITUDE[code & 7];
+    return (code & 8) ? -m : m;
+}
+
+/* E4M3 (FP8) from its definition: sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits; exponent field 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN; there is
+ * no infinity, so the largest finite magnitude is 1.75 * 2^8 = 448.  NVFP4 uses
+ * it as the per-16 block scale ([P1] "About NVFP4 quantization"). */
+double orc_e4m3_value(uint8_t byte) {
+    int s = byte >> 7, e = (byte >> 3) & 15, m = byte & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* E8M0: an unsigned power-of-two exponent with bias 127; 0xFF is NaN.  The MXFP4
+ * block scale over 32 codes ([P4] "Model Summary": E2M1 + E8M0 scale, block 32). */
+double orc_e8m0_value(uint8_t byte) {
+    if (byte == 0xFF) return NAN;
+    return ldexp(1.0, (int)byte - 127);
+}
+
+/* BF16 is the upper half of an IEEE binary32. */
+float orc_bf16_to_float(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* Round an FP32 value to BF16, round-to-nearest-even (finite inputs). */
+uint16_t orc_float_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u) return (uint16_t)(u >> 16); /* inf / nan kept */
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* Nearest E4M3 byte to x, ties to the even mantissa, saturating to +-448 instead
+ * of producing NaN ("satfinite").  Plain search over the finite codes. */
+uint8_t orc_e4m3_rne_satfinite(float x) {
+    if (isnan(x)) return 0x7F;
+    double a = fabs((double)x);
+    int best = 0;
+    double best_d = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) { /* values increase with c over 0x00..0x7E */
+        double d = fabs(orc_e4m3_value((uint8_t)c) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0)) {
+            best_d = d;
+            best = c;
+        }
+    }
+    return (uint8_t)(signbit(x) ? (best | 0x80) : best);
+}
+
+/* Nearest E2M1 code to x, ties to the even mantissa bit, saturating to +-6; the
+ * sign is kept, so a negative value that rounds to zero gives code 0x8. */
+uint8_t orc_e2m1_rne_sat(float x) {
+    double a = fabs((double)x);
+    int best = 0;
+    double best_d = INFINITY;
+    for (int c = 0; c < 8; ++c) {
+        double d = fabs(E2M1_MAGNITUDE[c] - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0)) {
+            best_d = d;
+            best = c;
+        }
+    }
+    return (uint8_t)(signbit(x) ? (best | 8) : best);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Tensor decoders (used by the transcode invariant and by the layer)         */
+/* ------------------------------------------------------------------------- */
+
+static inline uint8_t nibble(const uint8_t* packed, int64_t i) {
+    /* two codes per byte; the even element is the low nibble */
+    uint8_t b = packed[i >> 1];
+    return (i & 1) ? (uint8_t)(b >> 4) : (uint8_t)(b & 15);
+}
+
+/* MXFP4 [N,K]: value = e2m1 * 2^(e8m0-127), one scale per 32 along K. */
+void orc_decode_mxfp4(const uint8_t* codes, const uint8_t* e8m0, int64_t N, int64_t K, double* out) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            out[n * K + k] = orc_e2m1_value(nibble(codes + n * (K / 2), k)) * orc_e8m0_value(e8m0[n * (K / 32) + k / 32]);
+}
+
+/* NVFP4 [N,K]: value = e2m1 * e4m3 * global, one E4M3 scale per 16 along K. */
+void orc_decode_nvfp4(const uint8_t* codes, const uint8_t* e4m3, float global, int64_t N, int64_t K, double* out) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            out[n * K + k] = orc_e2m1_value(nibble(codes + n * (K / 2), k)) *
+                             orc_e4m3_value(e4m3[n * (K / 16) + k / 16]) * (double)global;
+}
+
+/* ------------------------------------------------------------------------- */
+/* MXFP4 -> NVFP4 transcode                                                   */
+/* ------------------------------------------------------------------------- */
+/* [P1] introduction and [P2] "What changed": every E2M1 code is kept byte for
+ * byte; each E8M0 scale over 32 codes becomes two exact E4M3 scales over the two
+ * 16-code halves, times one exact power-of-two FP32 global scale per tensor;
+ * nothing is re-rounded.  [P1] "Reproduce the checkpoint" reports the count of
+ * scale blocks, of all-zero blocks and of out-of-E4M3-range blocks.
+ *
+ * Reading of the open points: the global is 2^g with g = k_max - 8 over the
+ * non-zero blocks of the tensor (the largest block maps to the scale 256); a
+ * tensor whose exponent spread k_max - k_min exceeds 17 has no exact transcode
+ * (E4M3 holds exactly the powers 2^-9 .. 2^8) and is reported, its scales
+ * zero-filled and its global 0; all-zero blocks take scale 0; a tensor with no
+ * non-zero block takes g = 0.  A NaN E8M0 scale (0xFF) on a non-zero block is
+ * reported the same way as a non-representable tensor, with its own status.
+ *
+ * Per-tensor status: 0 exact, 1 not representable, 2 NaN scale.
+ * report[0] blocks, [1] all-zero blocks, [2] non-representable tensors,
+ * [3] NaN-scale tensors.  Returns the worst status seen (2 > 1 > 0).        */
+
+static int e4m3_byte_of_power_of_two(int e) {
+    /* search the definition table for the byte whose value is exactly 2^e */
+    double target = ldexp(1.0, e);
+    for (int c = 0; c <= 0x7E; ++c)
+        if (orc_e4m3_value((uint8_t)c) == target) return c;
+    return -1;
+}
+
+int orc_transcode(const uint8_t* codes_in, const uint8_t* e8m0, int64_t num_tensors, int64_t N, int64_t K,
+                  uint8_t* codes_out, uint8_t* e4m3_out, float* global_out, int32_t* tensor_status,
+                  int64_t* report) {
+    const int64_t blocks = N * K / 32;
+    int worst = 0;
+    report[0] = report[1] = report[2] = report[3] = 0;
+    for (int64_t t = 0; t < num_tensors; ++t) {
+        const uint8_t* c = codes_in + t * blocks * 16;
+        const uint8_t* s = e8m0 + t * blocks;
+        uint8_t* so = e4m3_out + t * blocks * 2;
+        /* codes are copied byte for byte */
+        memcpy(codes_out + t * blocks * 16, c, (size_t)(blocks * 16));
+
+        int have = 0, kmin = 0, kmax = 0, nan_seen = 0;
+        for (int64_t b = 0; b < blocks; ++b) {
+            int zero = 1;
+            for (int i = 0; i < 32; ++i)
+                if (nibble(c + b * 16, i) & 7) zero = 0;
+            if (zero) {
+                report[1]++;
+                continue;
+            }
+            if (s[b] == 0xFF) {
+                nan_seen = 1;
+                continue;
+            }
+            int k = (int)s[b] - 127;
+            if (!have || k < kmin) kmin = k;
+            if (!have || k > kmax) kmax = k;
+            have = 1;
+        }
+        report[0] += blocks;
+
+        int status = 0;
+        if (nan_seen) status = 2;
+        else if (have && kmax - kmin > 17) status = 1;
+        if (status) {
+            memset(so, 0, (size_t)(blocks * 2));
+            global_out[t] = 0.0f;
+            tensor_status[t] = status;
+            report[status == 1 ? 2 : 3]++;
+            if (status > worst) worst = status;
+            continue;
+        }
+        int g = have ? kmax - 8 : 0;
+        for (int64_t b = 0; b < blocks; ++b) {
+            int zero = 1;
+            for (int i = 0; i < 32; ++i)
+                if (nibble(c + b * 16, i) & 7) zero = 0;
+            uint8_t byte = 0;
+            if (!zero) {
+                int e = (int)s[b] - 127 - g; /* in [-9, 8] */
+                int found = e4m3_byte_of_power_of_two(e);
+                byte = (uint8_t)(found < 0 ? 0 : found);
+            }
+            so[2 * b] = byte;     /* first 16-code half  */
+            so[2 * b + 1] = byte; /* second 16-code half */
+        }
+        global_out[t] = ldexpf(1.0f, g);
+        tensor_status[t] = 0;
+    }
+    return worst;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Specified FP32 exp and sigmoid                                             */
+/* ------------------------------------------------------------------------- */
+/* The router needs sigmoid ([P4] "Pruning Method" 1: grouped sigmoid top-k).
+ * The pages do not fix its rounding; to make routing choices reproducible on
+ * both sides, the exp below is specified operation by operation in IEEE FP32:
+ *   clamp y to [-87, 88]; n = rint(y * log2(e)); Cody-Waite reduction
+ *   r = fma(-n, ln2_hi, y); r = fma(-n, ln2_lo, r) with ln2_hi = ln 2 rounded to
+ *   FP32 with its 12 low mantissa bits cleared and ln2_lo = FP32(ln 2 - ln2_hi);
+ *   p = degree-7 Taylor polynomial sum r^i / i! in Horner form with fmaf, the
+ *   coefficients being FP32(1 / i!); result = p * 2^n (2^n built exactly).
+ * sigmoid(x) = 1 / (1 + exp(-x)) for x >= 0, else e / (1 + e) with e = exp(x). */
+
+static float orc_ln2_hi(void) {
+    float f = (float)0.69314718055994530942;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    u &= 0xFFFFF000u;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+float orc_exp_spec(float y) {
+    const float log2e = (float)1.44269504088896340736;
+    const float ln2_hi = orc_ln2_hi();
+    const float ln2_lo = (float)(0.69314718055994530942 - (double)ln2_hi);
+    if (y > 88.0f) y = 88.0f;
+    if (y < -87.0f) y = -87.0f;
+    float n = rintf(y * log2e);
+    float r = fmaf(-n, ln2_hi, y);
+    r = fmaf(-n, ln2_lo, r);
+    float p = (float)(1.0 / 5040.0);
+    p = fmaf(p, r, (float)(1.0 / 720.0));
+    p = fmaf(p, r, (float)(1.0 / 120.0));
+    p = fmaf(p, r, (float)(1.0 / 24.0));
+    p = fmaf(p, r, (float)(1.0 / 6.0));
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    int ni = (int)n; /* in [-126, 127] */
+    uint32_t bits = (uint32_t)(ni + 127) << 23;
+    float two_n;
+    memcpy(&two_n, &bits, 4);
+    return p * two_n;
+}
+
+float orc_sigmoid_spec(float x) {
+    if (x >= 0.0f) return 1.0f / (1.0f + orc_exp_spec(-x));
+    float e = orc_exp_spec(x);
+    return e / (1.0f + e);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Grouped sigmoid top-k routing                                              */
+/* ------------------------------------------------------------------------- */
+/* [P4] "Model Summary" and "Pruning Method" 1: n_routed_experts experts are
+ * reshaped into [n_group, n_routed_experts / n_group]; topk_group groups are
+ * kept, top-k experts are chosen inside them, and the weights are scaled by
+ * routed_scaling_factor.  A selection-only correction bias exists
+ * (e_score_correction_bias).  Readings: s = sigmoid(logit); c = s + bias (bias 0
+ * when absent) decides the selection; a group's score is the sum of its two
+ * largest c (its largest when a group has one expert); groups and experts are
+ * taken by descending value, ties to the lower index; the output order is the
+ * selection order.  With renormalize: S = sum of the chosen s in output order
+ * (sequential FP32 adds), w_j = (s_j / S) * rsf; without: w_j = s_j * rsf.   */
+void orc_route(const float* logits, const float* bias, int T, int E, int n_group, int topk_group, int top_k,
+               float rsf, int renormalize, int32_t* topk_ids, float* topk_weights) {
+    const int gsize = E / n_group;
+    float* s = (float*)malloc(sizeof(float) * (size_t)E);
+    float* c = (float*)malloc(sizeof(float) * (size_t)E);
+    float* gscore = (float*)malloc(sizeof(float) * (size_t)n_group);
+    char* gsel = (char*)malloc((size_t)n_group);
+    char* taken = (char*)malloc((size_t)E);
+    for (int t = 0; t < T; ++t) {
+        const float* lg = logits + (int64_t)t * E;
+        for (int e = 0; e < E; ++e) {
+            s[e] = orc_sigmoid_spec(lg[e]);
+            c[e] = s[e] + (bias ? bias[e] : 0.0f);
+        }
+        for (int g = 0; g < n_group; ++g) {
+            int i1 = -1, i2 = -1;
+            for (int e = g * gsize; e < (g + 1) * gsize; ++e)
+                if (i1 < 0 || c[e] > c[i1]) i1 = e;
+            for (int e = g * gsize; e < (g + 1) * gsize; ++e)
+                if (e != i1 && (i2 < 0 || c[e] > c[i2])) i2 = e;
+            gscore[g] = (i2 < 0) ? c[i1] : c[i1] + c[i2];
+            gsel[g] = 0;
+        }
+        for (int r = 0; r < topk_group; ++r) {
+            int best = -1;
+            for (int g = 0; g < n_group; ++g)
+                if (!gsel[g] && (best < 0 || gscore[g] > gscore[best])) best = g;
+            gsel[best] = 1;
+        }
+        for (int e = 0; e < E; ++e) taken[e] = 0;
+        for (int j = 0; j < top_k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e)
+                if (gsel[e / gsize] && !taken[e] && (best < 0 || c[e] > c[best])) best = e;
+            taken[best] = 1;
+            topk_ids[(int64_t)t * top_k + j] = best;
+        }
+        float S = 0.0f;
+        for (int j = 0; j < top_k; ++j) S = S + s[topk_ids[(int64_t)t * top_k + j]];
+        for (int j = 0; j < top_k; ++j) {
+            float sj = s[topk_ids[(int64_t)t * top_k + j]];
+            topk_weights[(int64_t)t * top_k + j] = renormalize ? (sj / S) * rsf : sj * rsf;
+        }
+    }
+    free(s);
+    free(c);
+    free(gscore);
+    free(gsel);
+    free(taken);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Token permutation                                                          */
+/* ------------------------------------------------------------------------- */
+/* Groups the (token, slot) pairs by expert so each expert's rows are contiguous
+ * ("grouped" experts: [P1] "Deploy" runs a fused grouped MoE; [P5] "Speed v4"
+ * names an exact grouped kernel).  Order inside an expert: by token, then slot.
+ * counts[E], offsets[E+1] (exclusive prefix sums), row_of_pair[T*k],
+ * pair_of_row[T*k]; pair index = t * k + j.                                  */
+void orc_permute(const int32_t* topk_ids, int T, int top_k, int E, int32_t* counts, int32_t* offsets,
+                 int32_t* row_of_pair, int32_t* pair_of_row) {
+    const int64_t P = (int64_t)T * top_k;
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t p = 0; p < P; ++p) counts[topk_ids[p]]++;
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int64_t row = 0;
+    for (int e = 0; e < E; ++e)
+        for (int64_t p = 0; p < P; ++p)
+            if (topk_ids[p] == e) {
+                row_of_pair[p] = (int32_t)row;
+                pair_of_row[row] = (int32_t)p;
+                row++;
+            }
+}
+
+/* ------------------------------------------------------------------------- */
+/* NVFP4 quantisation                                                         */
+/* ------------------------------------------------------------------------- */
+/* [P1] "About NVFP4 quantization" (E2M1 codes with an E4M3 scale per 16) and
+ * "Why a unit activation scale" (one activation global scale, set to 1).
+ * Per 16-element block of a row, with gs the dequantisation global scale:
+ *   amax = max |x|;  sf = E4M3_rne_satfinite((amax / 6) / gs)  (IEEE FP32);
+ *   if value(sf) == 0 every code is 0x0;
+ *   else q_i = E2M1_rne_sat(x_i / (value(sf) * gs))            (IEEE FP32).
+ * Codes are packed two per byte (even element in the low nibble); scales are
+ * row-major [M, K/16].                                                       */
+void orc_quantize_f32(const float* x, int64_t M, int64_t K, float gs, uint8_t* codes, uint8_t* scales) {
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t b = 0; b < K / 16; ++b) {
+            const float* xb = x + m * K + b * 16;
+            float amax = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float a = fabsf(xb[i]);
+                if (a > amax) amax = a;
+            }
+            float v = amax / 6.0f;
+            v = v / gs;
+            uint8_t sf = orc_e4m3_rne_satfinite(v);
+            scales[m * (K / 16) + b] = sf;
+            double sfv = orc_e4m3_value(sf);
+            uint8_t q[16];
+            if (sfv == 0.0) {
+                for (int i = 0; i < 16; ++i) q[i] = 0;
+            } else {
+                float denom = (float)sfv * gs;
+                for (int i = 0; i < 16; ++i) q[i] = orc_e2m1_rne_sat(xb[i] / denom);
+            }
+            for (int i = 0; i < 8; ++i) codes[m * (K / 2) + b * 8 + i] = (uint8_t)(q[2 * i] | (q[2 * i + 1] << 4));
+        }
+    }
+}
+
+void orc_quantize_bf16(const uint16_t* x, int64_t M, int64_t K, float gs, uint8_t* codes, uint8_t* scales) {
+    float* xf = (float*)malloc(sizeof(float) * (size_t)K);
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k) xf[k] = orc_bf16_to_float(x[m * K + k]);
+        orc_quantize_f32(xf, 1, K, gs, codes + m * (K / 2), scales + m * (K / 16));
+    }
+    free(xf);
+}
+
+/* ------------------------------------------------------------------------- */
+/* The MoE layer                                                              */
+/* ------------------------------------------------------------------------- */
+/* Expert MLP ([P4] "Pruning Method" 1, the expert output inside the saliency
+ * formula): y_j = W_down,j( SiLU(W_gate,j h) (.) (W_up,j h) ), combined as
+ * sum_j g_{t,j} y_j over the token's selected experts.
+ * Modes ([P1] "Usage"/"Accuracy"): W4A16 keeps the activations in BF16 (the
+ * SwiGLU output is rounded FP32 -> BF16 before the down projection); W4A4
+ * quantises the activations to NVFP4 with the unit global scale ([P1] "Why a
+ * unit activation scale") and requantises the SwiGLU output per 16 the same way.
+ * Weights: NVFP4, gate/up [E, I, H] and down [E, H, I] (out x in), scales per 16
+ * along the input dimension, w_global[E][3] = gate, up, down global scales.
+ * Everything after decoding is float64; out is [n_tokens, H] for the listed
+ * tokens (tokens are independent, so a sample of tokens is exact for them).  */
+
+static double silu(double g) { return g / (1.0 + exp(-g)); }
+
+static void decode_row(const uint8_t* codes, const uint8_t* sf, double global, int64_t K, double* out) {
+    for (int64_t k = 0; k < K; ++k)
+        out[k] = orc_e2m1_value(nibble(codes, k)) * orc_e4m3_value(sf[k / 16]) * global;
+}
+
+void orc_moe_layer(int mode, const uint16_t* x, const float* logits, const float* bias, const uint8_t* gate_codes,
+                   const uint8_t* gate_sf, const uint8_t* up_codes, const uint8_t* up_sf, const uint8_t* down_codes,
+                   const uint8_t* down_sf, const float* w_global, float act_global, int T, int H, int I, int E,
+                   int n_group, int topk_group, int top_k, float rsf, int renormalize, const int32_t* tokens,
+                   int n_tokens, double* out) {
+    (void)T;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int it = 0; it < n_tokens; ++it) {
+        const int t = tokens[it];
+        int32_t ids[64];
+        float wts[64];
+        orc_route(logits + (int64_t)t * E, bias, 1, E, n_group, topk_group, top_k, rsf, renormalize, ids, wts);
+
+        double* xd = (double*)malloc(sizeof(double) * (size_t)H);
+        double* wrow = (double*)malloc(sizeof(double) * (size_t)(H > I ? H : I));
+        double* a = (double*)malloc(sizeof(double) * (size_t)I);
+        float* a32 = (float*)malloc(sizeof(float) * (size_t)I);
+        uint8_t* aq = (uint8_t*)malloc((size_t)I / 2);
+        uint8_t* as = (uint8_t*)malloc((size_t)I / 16);
+        double* o = out + (int64_t)it * H;
+        for (int h = 0; h < H; ++h) o[h] = 0.0;
+
+        if (mode == 1) {
+            uint8_t* xq = (uint8_t*)malloc((size_t)H / 2);
+            uint8_t* xs = (uint8_t*)malloc((size_t)H / 16);
+            orc_quantize_bf16(x + (int64_t)t * H, 1, H, act_global, xq, xs);
+            for (int h = 0; h < H; ++h)
+                xd[h] = orc_e2m1_value(nibble(xq, h)) * orc_e4m3_value(xs[h / 16]) * (double)act_global;
+            free(xq);
+            free(xs);
+        } else {
+            for (int h = 0; h < H; ++h) xd[h] = (double)orc_bf16_to_float(x[(int64_t)t * H + h]);
+        }
+
+        for (int j = 0; j < top_k; ++j) {
+            const int e = ids[j];
+            const double gg = w_global[e * 3 + 0], gu = w_global[e * 3 + 1], gd = w_global[e * 3 + 2];
+            for (int i = 0; i < I; ++i) {
+                const int64_t r = (int64_t)e * I + i;
+                double g = 0.0, u = 0.0;
+                decode_row(gate_codes + r * (H / 2), gate_sf + r * (H / 16), gg, H, wrow);
+                for (int h = 0; h < H; ++h) g += xd[h] * wrow[h];
+                decode_row(up_codes + r * (H / 2), up_sf + r * (H / 16), gu, H, wrow);
+                for (int h = 0; h < H; ++h) u += xd[h] * wrow[h];
+                a[i] = silu(g) * u;
+            }
+            if (mode == 1) {
+                for (int i = 0; i < I; ++i) a32[i] = (float)a[i];
+                orc_quantize_f32(a32, 1, I, act_global, aq, as);
+                for (int i = 0; i < I; ++i)
+                    a[i] = orc_e2m1_value(nibble(aq, i)) * orc_e4m3_value(as[i / 16]) * (double)act_global;
+            } else {
+                for (int i = 0; i < I; ++i) a[i] = (double)orc_bf16_to_float(orc_float_to_bf16((float)a[i]));
+            }
+            for (int h = 0; h < H; ++h) {
+                const int64_t r = (int64_t)e * H + h;
+                decode_row(down_codes + r * (I / 2), down_sf + r * (I / 16), gd, I, wrow);
+                double y = 0.0;
+                for (int i = 0; i < I; ++i) y += a[i] * wrow[i];
+                o[h] += (double)wts[j] * y;
+            }
+        }
+        free(xd);
+        free(wrow);
+        free(a);
+        free(a32);
+        free(aq);
+        free(as);
+    }
+}
+
+/* Routing weights/ids for a subset of tokens, for the sampled-token checks. */
+int orc_num_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,419 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself:
+values printed on the pages (golden files), format definitions, closed forms,
+library routines (torch FP8 casts, numpy float64 matmul) and brute force on
+tiny inputs.  CPU only."""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nvfp4_mixture_experts_grouped_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+# ---------------------------------------------------------------------------
+# codebooks
+# ---------------------------------------------------------------------------
+
+def test_e2m1_codebook_matches_pages():
+    rows = _rows("e2m1_codebook.txt")
+    for code, mag in rows:
+        c = int(code)
+        assert oracle.e2m1_value(c) == float(mag)
+        assert oracle.e2m1_value(c | 8) == -float(mag)
+    assert {oracle.e2m1_value(c) for c in range(8)} == {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0}
+    # no NaN / Inf encodings, max magnitude 6
+    assert max(abs(oracle.e2m1_value(c)) for c in range(16)) == 6.0
+
+
+def test_e4m3_points_and_structure():
+    for byte, val in _rows("e4m3_points.txt"):
+        v = oracle.e4m3_value(int(byte, 16))
+        if val == "nan":
+            assert math.isnan(v)
+        else:
+            assert v == float(val) and math.copysign(1, v) == math.copysign(1, float(val))
+    vals = [oracle.e4m3_value(b) for b in range(256)]
+    assert sum(math.isnan(v) for v in vals) == 2
+    pos = vals[:0x7F]
+    assert all(a < b for a, b in zip(pos, pos[1:]))  # monotone over 0x00..0x7E
+    assert max(pos) == 448.0
+    # every finite value has at most 4 significant bits
+    for v in pos[1:]:
+        m, e = math.frexp(v)
+        assert (m * 16) == int(m * 16)
+
+
+def test_e4m3_table_matches_torch_fp8():
+    # independent library decode of every finite byte
+    b = torch.arange(256, dtype=torch.uint8)
+    ref = b.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for i in range(256):
+        v = oracle.e4m3_value(i)
+        if math.isnan(ref[i]):
+            assert math.isnan(v)
+        else:
+            assert v == ref[i]
+
+
+def test_e8m0():
+    assert oracle.e8m0_value(127) == 1.0
+    assert oracle.e8m0_value(0) == 2.0 ** -127
+    assert oracle.e8m0_value(254) == 2.0 ** 127
+    assert math.isnan(oracle.e8m0_value(255))
+
+
+def test_e4m3_rounding_against_torch_cast():
+    rng = np.random.default_rng(7)
+    xs = np.concatenate([
+        rng.uniform(0, 448, 3000), np.exp(rng.uniform(-14, 6, 3000)),
+        # exact midpoints between neighbours
+        np.array([(oracle.e4m3_value(c) + oracle.e4m3_value(c + 1)) / 2 for c in range(0, 0x7E)]),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(xs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_rne_satfinite(float(x)) for x in xs], np.uint8)
+    assert np.array_equal(got, ref)
+    # satfinite: beyond 448 the result is the largest finite code, not NaN
+    for x in (448.0, 460.0, 464.0, 1e6, 3.0e38):
+        assert oracle.e4m3_rne_satfinite(x) == 0x7E
+
+
+def test_e2m1_rounding_golden():
+    for ratio, code in _rows("e2m1_rounding.txt"):
+        assert oracle.e2m1_rne_sat(float(ratio)) == int(code), ratio
+
+
+def test_e2m1_rounding_is_nearest():
+    rng = np.random.default_rng(3)
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    for x in rng.uniform(-8, 8, 2000).astype(np.float32):
+        c = oracle.e2m1_rne_sat(float(x))
+        d = abs(abs(float(x)) - mags[c & 7])
+        assert d <= np.min(np.abs(abs(float(x)) - mags)) + 0.0
+
+
+def test_page_count_identities():
+    d = {k: int(v) for k, v in _rows("page_counts.txt")}
+    # blocks x block size == verified values; values == matrices x 4096*2048
+    assert d["scale_blocks"] * d["mxfp4_block"] == d["expert_values"]
+    assert d["values_per_matrix"] == 4096 * 2048
+    assert d["expert_values"] % d["values_per_matrix"] == 0
+    # unit-scale clip point == E2M1 max x E4M3 max
+    assert d["unit_scale_clip"] == oracle.e2m1_value(7) * oracle.e4m3_value(0x7E)
+
+
+# ---------------------------------------------------------------------------
+# transcode
+# ---------------------------------------------------------------------------
+
+def _mx(num, N, K, lo, hi, seed=11):
+    rng = np.random.default_rng(seed)
+    return inputs.mxfp4_tensors(rng, num, N, K, lo, hi)
+
+
+@pytest.mark.parametrize("lo,hi", [(-8, -3), (-20, -3), (0, 17), (-127, -110), (110, 127), (5, 5)])
+def test_transcode_decode_equality(lo, hi):
+    num, N, K = 3, 8, 128
+    codes, e8 = _mx(num, N, K, lo, hi)
+    # one all-zero block (codes 0x0 and 0x8 only) in tensor 0
+    codes[0, 1, 0:16] = np.array([0x00, 0x88, 0x08, 0x80] * 4, np.uint8)
+    c2, e4, g, st, rep, worst = oracle.transcode(codes, e8, num, N, K)
+    assert worst == 0 and np.all(st == 0)
+    assert np.array_equal(c2, codes)  # codes byte for byte
+    assert rep[0] == num * N * K // 32 and rep[1] >= 1
+    for t in range(num):
+        ref = oracle.decode_mxfp4(codes[t], e8[t], N, K)
+        got = oracle.decode_nvfp4(c2[t], e4[t], float(g[t]), N, K)
+        assert np.array_equal(ref, got)
+        m, _ = math.frexp(float(g[t]))
+        assert m == 0.5  # exact power of two
+        # two equal scales per 32-block, each a finite exact power of two
+        s = e4[t].reshape(-1, 2)
+        assert np.all(s[:, 0] == s[:, 1])
+        for b in np.unique(s):
+            v = oracle.e4m3_value(int(b))
+            assert not math.isnan(v)
+            if v:
+                assert math.frexp(v)[0] == 0.5
+    assert e4[0, 1, 0] == 0 and e4[0, 1, 1] == 0  # the all-zero block
+
+
+def test_transcode_spread_boundary():
+    N, K = 4, 64
+    codes, e8 = _mx(2, N, K, 0, 0)
+    codes[:] = 0x11
+    e8[0] = 127
+    e8[0, 0, 0] = 127 + 17  # spread 17: representable
+    e8[1] = 127
+    e8[1, 0, 0] = 127 + 18  # spread 18: not representable
+    _, e4, g, st, rep, worst = oracle.transcode(codes, e8, 2, N, K)
+    assert list(st) == [0, 1] and worst == 1 and rep[2] == 1
+    assert g[1] == 0.0 and np.all(e4[1] == 0)
+    assert g[0] == 2.0 ** 9 and e4[0, 0, 0] == 0x78 and e4[0, 0, 2] == 0x01  # 2^8 and 2^-9
+
+
+def test_transcode_nan_scale_and_empty_tensor():
+    codes, e8 = _mx(2, 2, 64, 0, 0)
+    e8[0, 0, 1] = 0xFF
+    codes[1] = 0x00  # tensor with no non-zero block
+    _, e4, g, st, rep, _ = oracle.transcode(codes, e8, 2, 2, 64)
+    assert st[0] == 2 and rep[3] == 1
+    assert st[1] == 0 and g[1] == 1.0 and np.all(e4[1] == 0)
+
+
+def test_transcode_adversarial_tensor_of_the_layer_recipe():
+    rng = np.random.default_rng(inputs.TRANSCODE_SEED)
+    adv_codes, adv_e8 = inputs.mxfp4_tensors(rng, 1, 64, 128, -9, 9)
+    adv_codes[0, 0, :16] = 0x77
+    adv_codes[0, 1, :16] = 0x77
+    adv_e8[0, 0, 0] = 127 - 9
+    adv_e8[0, 1, 0] = 127 + 9
+    *_, st, rep, worst = oracle.transcode(adv_codes, adv_e8, 1, 64, 128)
+    assert st[0] == 1 and worst == 1
+
+
+# ---------------------------------------------------------------------------
+# sigmoid / exp specification
+# ---------------------------------------------------------------------------
+
+def _ulp_diff(a: np.float32, b: float) -> float:
+    return abs(float(a) - b) / float(np.spacing(np.float32(abs(b)) if b else np.float32(1e-45)))
+
+
+def test_exp_and_sigmoid_within_2ulp():
+    rng = np.random.default_rng(5)
+    xs = np.concatenate([rng.uniform(-20, 20, 4000), rng.normal(0, 1, 2000), np.linspace(-87, 88, 500)])
+    for x in xs.astype(np.float32):
+        e = oracle.exp_spec(float(x))
+        assert _ulp_diff(np.float32(e), math.exp(float(x))) <= 2.0, x
+        s = oracle.sigmoid_spec(float(x))
+        assert _ulp_diff(np.float32(s), 1.0 / (1.0 + math.exp(-float(x)))) <= 2.0, x
+    assert oracle.sigmoid_spec(0.0) == 0.5
+
+
+# ---------------------------------------------------------------------------
+# router
+# ---------------------------------------------------------------------------
+
+def _route_bruteforce(logits, bias, ng, tg, k, rsf, renorm):
+    T, E = logits.shape
+    gsz = E // ng
+    ids = np.zeros((T, k), np.int64)
+    w = np.zeros((T, k), np.float32)
+    for t in range(T):
+        s = np.array([oracle.sigmoid_spec(float(v)) for v in logits[t]], np.float32)
+        c = s + (bias if bias is not None else np.zeros(E, np.float32))
+        c = c.astype(np.float32)
+        score = []
+        for g in range(ng):
+            grp = sorted(c[g * gsz:(g + 1) * gsz], reverse=True)
+            score.append(np.float32(grp[0]) + np.float32(grp[1]) if gsz > 1 else np.float32(grp[0]))
+        # best subset of tg groups: enumerate all subsets, rank by (sorted scores desc, then indices)
+        best = None
+        for sub in itertools.combinations(range(ng), tg):
+            key = sorted(((-score[g], g) for g in sub))
+            # a subset is the top-tg set iff every member outranks every non-member
+            others = [(-score[g], g) for g in range(ng) if g not in sub]
+            if all(a < b for a in key for b in others):
+                best = sub
+        cand = [e for e in range(E) if e // gsz in best]
+        order = sorted(cand, key=lambda e: (-c[e], e))[:k]
+        ids[t] = order
+        S = np.float32(0)
+        for e in order:
+            S = np.float32(S + s[e])
+        for j, e in enumerate(order):
+            w[t, j] = np.float32(np.float32(s[e] / S) * np.float32(rsf)) if renorm else np.float32(s[e] * np.float32(rsf))
+    return ids, w
+
+
+@pytest.mark.parametrize("E,ng,tg,k", [(16, 4, 2, 4), (32, 8, 4, 8), (12, 3, 2, 3), (8, 8, 3, 3), (8, 1, 1, 2)])
+@pytest.mark.parametrize("ties", [False, True])
+def test_route_bruteforce(E, ng, tg, k, ties):
+    rng = np.random.default_rng(E * 7 + ng)
+    T = 24
+    if ties:  # few distinct values so that scores and groups tie
+        logits = rng.integers(-2, 3, size=(T, E)).astype(np.float32)
+    else:
+        logits = rng.standard_normal((T, E)).astype(np.float32)
+    bias = (rng.standard_normal(E) * 0.1).astype(np.float32) if not ties else None
+    for renorm in (True, False):
+        ids, w = oracle.route(logits, bias, ng, tg, k, 2.827, renorm)
+        rid, rw = _route_bruteforce(logits, bias, ng, tg, k, 2.827, renorm)
+        assert np.array_equal(ids, rid)
+        assert np.array_equal(w.view(np.uint32), rw.view(np.uint32))
+
+
+def test_route_single_group_is_plain_topk_and_weights_sum():
+    rng = np.random.default_rng(99)
+    logits = rng.standard_normal((64, 32)).astype(np.float32)
+    ids, w = oracle.route(logits, None, 1, 1, 8, 2.827, True)
+    s = np.vectorize(oracle.sigmoid_spec, otypes=[np.float32])(logits)
+    ref = np.argsort(-s, axis=1, kind="stable")[:, :8]
+    assert np.array_equal(ids, ref)
+    assert np.allclose(w.sum(1), 2.827, rtol=3e-6)
+
+
+# ---------------------------------------------------------------------------
+# permutation
+# ---------------------------------------------------------------------------
+
+def test_permute_is_stable_grouping():
+    rng = np.random.default_rng(1)
+    logits = rng.standard_normal((50, 16)).astype(np.float32)
+    ids, _ = oracle.route(logits, None, 4, 2, 4, 1.0)
+    counts, offsets, rop, por = oracle.permute(ids, 16)
+    pairs = sorted(range(ids.size), key=lambda p: (ids.reshape(-1)[p], p))
+    assert list(por) == pairs
+    assert np.array_equal(np.bincount(ids.reshape(-1), minlength=16), counts)
+    assert offsets[0] == 0 and np.array_equal(np.diff(offsets), counts)
+    assert np.array_equal(rop[por], np.arange(ids.size))
+
+
+# ---------------------------------------------------------------------------
+# quantiser
+# ---------------------------------------------------------------------------
+
+def _bits(x):
+    return inputs.bf16_bits(np.asarray(x, np.float32))
+
+
+def test_quantize_midpoints_with_unit_scale():
+    # block max 6 -> scale E4M3(1.0) = 0x38; every other entry a golden ratio
+    rows = [r for r in _rows("e2m1_rounding.txt") if abs(float(r[0])) <= 6.0]
+    ratios = [float(r[0]) for r in rows]
+    codes_ref = [int(r[1]) for r in rows]
+    for i in range(0, len(ratios), 15):
+        blk = [6.0] + ratios[i:i + 15]
+        blk += [0.0] * (16 - len(blk))
+        ref = [7] + codes_ref[i:i + 15] + [0] * (16 - 1 - len(codes_ref[i:i + 15]))
+        c, s = oracle.quantize_f32(np.array([blk], np.float32))
+        assert s[0, 0] == 0x38
+        got = [(c[0, j // 2] >> (4 * (j % 2))) & 15 for j in range(16)]
+        assert got == ref
+
+
+def test_quantize_saturation_and_zero_block():
+    x = np.zeros((2, 32), np.float32)
+    x[0, 0] = 3.0e5  # >= 2688: scale saturates at 448, code saturates at 6
+    x[0, 1] = -2688.0
+    x[0, 2] = 1000.0
+    c, s = oracle.quantize_f32(x)
+    assert s[0, 0] == 0x7E
+    assert c[0, 0] == (0x7 | (0xF << 4))
+    assert s[0, 1] == 0 and np.all(c[1] == 0) and np.all(s[1] == 0)
+    # 2688 is exactly representable: 6 x 448
+    assert oracle.e2m1_value(0xF) * oracle.e4m3_value(s[0, 0]) == -2688.0
+
+
+def test_quantize_roundtrip_of_representable_blocks():
+    rng = np.random.default_rng(8)
+    for _ in range(200):
+        sfb = int(rng.integers(0x08, 0x70))
+        sfv = oracle.e4m3_value(sfb)
+        q = rng.integers(0, 16, 16)
+        q[0] = 7  # block max = 6 * scale, so the scale is recovered exactly
+        x = np.array([oracle.e2m1_value(int(v)) * sfv for v in q], np.float32)
+        c, s = oracle.quantize_f32(x[None, :])
+        assert s[0, 0] == sfb
+        dec = [oracle.e2m1_value(int((c[0, j // 2] >> (4 * (j % 2))) & 15)) * sfv for j in range(16)]
+        assert np.array_equal(np.array(dec, np.float32), x)
+
+
+def test_quantize_scale_against_torch_fp8():
+    rng = np.random.default_rng(4)
+    x = (rng.standard_normal((64, 256)) * np.exp(rng.uniform(-6, 6, (64, 1)))).astype(np.float32)
+    c, s = oracle.quantize_f32(x)
+    amax = np.abs(x.reshape(64, 16, 16)).max(-1)
+    ref = torch.from_numpy((amax / np.float32(6)).astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(s, ref)
+
+
+# ---------------------------------------------------------------------------
+# GEMM exactness and the layer
+# ---------------------------------------------------------------------------
+
+def test_fp4_products_exact_in_fp32():
+    rng = np.random.default_rng(0)
+    lut = np.array([oracle.e2m1_value(c) for c in range(16)])
+    for K in (16, 64, 4096):
+        a = lut[rng.integers(0, 16, (8, K))]
+        b = lut[rng.integers(0, 16, (8, K))]
+        r64 = a @ b.T
+        r32 = a.astype(np.float32) @ b.T.astype(np.float32)
+        assert np.array_equal(r64, r32.astype(np.float64))
+        assert np.all(np.mod(r64 * 4, 1) == 0)  # multiples of 0.25
+
+
+def _np_decode(codes, sf, glob):
+    """Independent numpy decode ([N, K/2] codes, [N, K/16] E4M3) via torch FP8."""
+    lut = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.0, -0.5, -1, -1.5, -2, -3, -4, -6])
+    lo = lut[codes & 15]
+    hi = lut[codes >> 4]
+    vals = np.stack([lo, hi], -1).reshape(codes.shape[0], -1)
+    s = torch.from_numpy(sf).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return vals * np.repeat(s, 16, axis=1) * float(glob)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_layer_reduces_to_dense_swiglu(mode):
+    rng = np.random.default_rng(21 + mode)
+    T, H, I = 5, 64, 32
+    gc, gs, _ = inputs.nvfp4_tensors(rng, 1, I, H)
+    uc, us, _ = inputs.nvfp4_tensors(rng, 1, I, H)
+    dc, ds, _ = inputs.nvfp4_tensors(rng, 1, H, I)
+    wg = np.array([[0.5, 0.25, 2.0]], np.float32)
+    x = inputs.activations(rng, T, H)
+    logits = rng.standard_normal((T, 1)).astype(np.float32)
+    out = oracle.moe_layer(mode, x, logits, None, gc, gs, uc, us, dc, ds, wg, 1.0, 1, 1, 1, 1.0)
+    Wg = _np_decode(gc[0], gs[0], 0.5)
+    Wu = _np_decode(uc[0], us[0], 0.25)
+    Wd = _np_decode(dc[0], ds[0], 2.0)
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    if mode == 1:
+        qc, qs = oracle.quantize_bf16(x)
+        xf = _np_decode(qc, qs, 1.0)
+    G = xf @ Wg.T
+    U = xf @ Wu.T
+    A = G / (1 + np.exp(-G)) * U
+    if mode == 1:
+        ac, as_ = oracle.quantize_f32(A.astype(np.float32))
+        A = _np_decode(ac, as_, 1.0)
+    else:
+        A = torch.from_numpy(A.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    Y = A @ Wd.T
+    assert np.allclose(out, Y, rtol=1e-12, atol=1e-12 * np.abs(Y).max())
+
+
+def test_layer_combines_two_experts_with_routing_weights():
+    rng = np.random.default_rng(33)
+    T, H, I, E = 4, 32, 16, 2
+    gc, gs, _ = inputs.nvfp4_tensors(rng, E, I, H)
+    uc, us, _ = inputs.nvfp4_tensors(rng, E, I, H)
+    dc, ds, _ = inputs.nvfp4_tensors(rng, E, H, I)
+    wg = np.ones((E, 3), np.float32)
+    x = inputs.activations(rng, T, H)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    both = oracle.moe_layer(0, x, logits, None, gc, gs, uc, us, dc, ds, wg, 1.0, 2, 2, 2, 2.827)
+    ids, w = oracle.route(logits, None, 2, 2, 2, 2.827)
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    for t in range(T):
+        acc = np.zeros(H)
+        for j in range(2):
+            e = ids[t, j]
+            G = _np_decode(gc[e], gs[e], 1) @ xf[t]
+            U = _np_decode(uc[e], us[e], 1) @ xf[t]
+            A = G / (1 + np.exp(-G)) * U
+            A = torch.from_numpy(A.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+            acc += float(w[t, j]) * (_np_decode(dc[e], ds[e], 1) @ A)
+        assert np.allclose(both[t], acc, rtol=1e-12, atol=1e-12 * np.abs(acc).max())
