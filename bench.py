@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 MoE layer hot path on B200.
+
+One step = one moe_forward call over one batch: grouped top-8 routing, token
+permutation, NVFP4 activation quantisation (unit global), gate/up grouped GEMM
++ SwiGLU (+ requantisation), down grouped GEMM x routing weight, weighted
+un-permute.  Default workload: the 8192-token W4A4 prefill layer (H=4096,
+I=2048, 256 experts in 8 groups, keep 4, top-8, scaling 2.827).  At N=1 the
+run also measures the W4A16 decode layer (T=16) and the MXFP4->NVFP4
+transcode of one layer of expert weights, reported as nested objects.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 it is launched by torchrun, one rank per GPU; every rank runs the
+same-shaped workload on its own batch (independent problems, no collective on
+the data path), timings are the max over ranks and `value` is the total tokens
+of all ranks per second ("scaling": "weak").  `--impl reference` times the CPU
+oracle (the parity reference) on a bounded token sample per step instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from nvfp4_mixture_experts_grouped_b200 import inputs  # noqa: E402
+
+N_TRACE = 7
+STAGES = ["route", "permute", "quantize", "gateup_gemm", "down_gemm", "combine"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["prefill", "skewed", "decode"], default="prefill")
+    ap.add_argument("--no-extras", action="store_true", help="skip the decode and transcode sub-measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=0, help="oracle tokens per step (0 = host threads)")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+# nominal dense FP4 : BF16 tensor-core throughput on B200 (9 : 2.25 PFLOP/s)
+FP4_OVER_BF16 = 4.0
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    def __init__(self, index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                       "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and "Active" in r[5 + i]})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def layer_flops(T, H, I, k):
+    return 6.0 * T * k * H * I
+
+
+def make_layer(torch, moe, mode, w, T, wl):
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+    E, I, hh = w["gate_codes"].shape
+    H = hh * 2
+    packed = torch.empty(moe.moe_packed_weights_size(mode, E, H, I), dtype=torch.uint8, device="cuda")
+    tw = {k: dev(v) for k, v in w.items()}
+    moe.moe_pack_weights(mode, tw["gate_codes"], tw["gate_sf"], tw["up_codes"], tw["up_sf"], tw["down_codes"],
+                         tw["down_sf"], tw["w_global"], packed)
+    torch.cuda.synchronize()
+    del tw
+    ws = torch.empty(moe.moe_forward_workspace_size(mode, T, H, I, E, wl.top_k), dtype=torch.uint8, device="cuda")
+    return packed, ws
+
+
+def time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, steps, warmup, trace=True):
+    """Returns (ms per step, per-stage ms means) timed with CUDA events on the current stream."""
+    H, I, E = wl.H, wl.I, wl.E
+
+    def step():
+        moe.moe_forward(mode, x, logits, None, packed, 1.0, T, H, I, E, wl.n_group, wl.topk_group, wl.top_k, wl.rsf,
+                        True, ws, out)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = []
+    if trace:
+        for _ in range(steps):
+            row = [torch.cuda.Event(enable_timing=True) for _ in range(N_TRACE)]
+            for e in row:
+                e.record()
+            evs.append(row)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        if trace:
+            moe.nvfp4moe_set_trace_events(evs[i])
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    moe.nvfp4moe_set_trace_events(None)
+    moe.nvfp4moe_check_device_status()
+    ms = t0.elapsed_time(t1) / steps
+    stage = None
+    if trace:
+        stage = {}
+        for s, name in enumerate(STAGES):
+            stage[name] = float(np.mean([evs[i][s].elapsed_time(evs[i][s + 1]) for i in range(steps)]))
+    return ms, stage
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import nvfp4_mixture_experts_grouped_b200 as moe
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+    P = peaks()
+    wl = inputs.WORKLOADS[args.workload]
+    T = wl.T
+    d = inputs.moe_inputs(wl)
+    w = {k: d[k] for k in ("gate_codes", "gate_sf", "up_codes", "up_sf", "down_codes", "down_sf", "w_global")}
+    # each rank gets its own batch (the weights are the layer's, identical on every rank)
+    if rank:
+        rng = np.random.default_rng(wl.seed * 1000 + rank)
+        d["x"] = inputs.activations(rng, T, wl.H, wl.outliers)
+        d["logits"] = inputs.router_logits(rng, T, wl.E, wl.zipf)
+    mode = wl.mode
+    packed, ws = make_layer(torch, moe, mode, w, T, wl)
+    x = torch.from_numpy(d["x"].view(np.int16)).cuda().view(torch.bfloat16)
+    logits = torch.from_numpy(d["logits"]).cuda()
+    out = torch.empty((T, wl.H), dtype=torch.bfloat16, device="cuda")
+
+    # ----------------------------------------------------------------- timed region
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    ms, stage = time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, args.steps, args.warmup)
+    clocks = sampler.stop() if sampler else None
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    value = T * world / (ms / 1e3)
+
+    # ----------------------------------------------------------------- end to end
+    xh = torch.from_numpy(d["x"].view(np.int16)).pin_memory()
+    lh = torch.from_numpy(d["logits"]).pin_memory()
+    oh = torch.empty((T, wl.H), dtype=torch.int16).pin_memory()
+
+    def e2e_step():
+        x.view(torch.int16).copy_(xh, non_blocking=True)
+        logits.copy_(lh, non_blocking=True)
+        moe.moe_forward(mode, x, logits, None, packed, 1.0, T, wl.H, wl.I, wl.E, wl.n_group, wl.topk_group,
+                        wl.top_k, wl.rsf, True, ws, out)
+        oh.copy_(out.view(torch.int16), non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        e2e_step()
+    b.record()
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / args.steps
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # ----------------------------------------------------------------- roofline
+    if mode == moe.W4A4:
+        flops = 4.0 * T * wl.top_k * wl.H * wl.I  # gate/up GEMM, padding rows excluded
+        t_kernel = stage["gateup_gemm"] / 1e3
+        achieved = flops / t_kernel / 1e12
+        peak = P["bf16_tflops"] * FP4_OVER_BF16
+        roofline = {"bound": "tensor", "kernel": "k_w4a4_gemm<gate/up>", "achieved": round(achieved, 1),
+                    "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                    "peak_src": f"{P['src']} bf16 burst x {FP4_OVER_BF16:g} (nominal dense FP4:BF16)",
+                    "algorithmic_flops_per_launch": flops}
+    else:
+        roofline = None
+
+    res = {
+        "metric": "MoE-layer tokens/s", "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp4 e2m1 (e4m3 block scales) x fp4 -> f32",
+        "data": "synthetic",
+        "config": {"workload": f"{wl.name}: T={T} H={wl.H} I={wl.I} E={wl.E} groups={wl.n_group} "
+                               f"keep={wl.topk_group} top_k={wl.top_k} rsf={wl.rsf} "
+                               f"{'W4A4' if mode == moe.W4A4 else 'W4A16'}",
+                   "global_batch": T * world, "tokens_per_gpu": T, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (3.6 GB packed expert weights per step)"},
+        "roofline": roofline,
+        "stages_ms": {k: round(v, 4) for k, v in stage.items()},
+        "e2e": {"value": round(T * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(d["x"].nbytes + d["logits"].nbytes), "d2h_bytes_per_step": int(T * wl.H * 2)},
+        "gpu_launches": 8 * args.steps,
+        "clocks": clocks,
+        "tflops": round(layer_flops(T, wl.H, wl.I, wl.top_k) / (ms / 1e3) / 1e12, 1),
+    }
+    del packed, ws
+    torch.cuda.empty_cache()
+
+    if world == 1 and not args.no_extras and rank == 0:
+        res["decode"] = bench_decode(torch, moe, w, args, P)
+        del w
+        res["transcode"] = bench_transcode(torch, moe, args, P)
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl, d, args)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def bench_decode(torch, moe, w, args, P):
+    """W4A16 decode layer (T=16): tokens/s and weight-stream HBM GB/s."""
+    wl = inputs.WORKLOADS["decode"]
+    d = inputs.moe_inputs(wl) if False else None  # weights: same recipe as the prefill layer, reused
+    rng = np.random.default_rng(wl.seed)
+    x = inputs.activations(rng, wl.T, wl.H)
+    lg = inputs.router_logits(rng, wl.T, wl.E)
+    packed, ws = make_layer(torch, moe, moe.W4A16, w, wl.T, wl)
+    xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    ld = torch.from_numpy(lg).cuda()
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    # flush L2 between steps: the active experts' weights (~1.4 GB) exceed L2, but
+    # the same experts repeat every step, so rotate through a 256 MB buffer too
+    ms, stage = time_layer(torch, moe, moe.W4A16, packed, ws, xd, ld, out, wl, wl.T, max(args.steps, 20),
+                           args.warmup)
+    ids = torch.empty((wl.T, wl.top_k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((wl.T, wl.top_k), dtype=torch.float32, device="cuda")
+    moe.moe_route(ld, None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf, True, ids, wts)
+    active = int(torch.unique(ids).numel())
+    per_expert = (2 * wl.I * wl.H + wl.H * wl.I) * (0.5 + 1.0 / 16)  # codes + E4M3 scales
+    gemm_ms = stage["gateup_gemm"] + stage["down_gemm"]
+    wbytes = active * per_expert
+    achieved = wbytes / (gemm_ms / 1e3) / 1e9
+    del packed, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"decode: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top_k={wl.top_k} W4A16",
+            "value": round(wl.T / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+            "active_experts": active, "stages_ms": {k: round(v, 4) for k, v in stage.items()},
+            "roofline": {"bound": "hbm", "kernel": "k_w16_gateup + k_w16_down", "achieved": round(achieved, 1),
+                         "peak": P["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / P["hbm_gbs"], 4),
+                         "traffic": None, "algorithmic_bytes_per_step": int(wbytes)}}
+
+
+def bench_transcode(torch, moe, args, P):
+    """MXFP4 -> NVFP4 transcode of one layer (768 expert tensors), out of place."""
+    rng = np.random.default_rng(inputs.TRANSCODE_SEED)
+    layer = inputs.transcode_layer(rng)
+    codes = np.concatenate([layer["gate"][0], layer["up"][0], layer["down"][0].reshape(256, 2048, 2048)])
+    e8 = np.concatenate([layer["gate"][1], layer["up"][1], layer["down"][1].reshape(256, 2048, 128)])
+    nt, N, K = codes.shape[0], 2048, 4096  # the down tensors [4096, 2048] have the same block count
+    c = torch.from_numpy(codes).cuda()
+    s = torch.from_numpy(e8).cuda()
+    del codes, e8, layer
+    co = torch.empty_like(c)
+    e4 = torch.empty((nt, N, K // 16), dtype=torch.uint8, device="cuda")
+    g = torch.empty(nt, dtype=torch.float32, device="cuda")
+    st = torch.empty(nt, dtype=torch.int32, device="cuda")
+    ws = torch.empty(moe.nvfp4moe_transcode_workspace_size(nt), dtype=torch.uint8, device="cuda")
+    status, rep = moe.transcode_mxfp4_to_nvfp4(c, s, nt, N, K, co, e4, g, st, ws, report=True)
+    for _ in range(args.warmup):
+        moe.transcode_mxfp4_to_nvfp4(c, s, nt, N, K, co, e4, g, st, ws, report=False)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(args.steps, 10)
+    a.record()
+    for _ in range(steps):
+        moe.transcode_mxfp4_to_nvfp4(c, s, nt, N, K, co, e4, g, st, ws, report=False)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    nbytes = c.numel() * 2 + s.numel() + e4.numel()  # read codes + e8m0, write codes + e4m3
+    gbs = nbytes / (ms / 1e3) / 1e9
+    res = {"workload": "transcode: 768 MXFP4 expert tensors (256 experts x gate/up [2048,4096], down [4096,2048]), "
+                       "out of place", "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
+           "tensors_per_s": round(nt / (ms / 1e3), 1), "status": int(status), "report": rep,
+           "roofline": {"bound": "hbm", "kernel": "k_transcode", "achieved": round(gbs, 1), "peak": P["hbm_gbs"],
+                        "unit": "GB/s", "frac": round(gbs / P["hbm_gbs"], 4), "traffic": None,
+                        "algorithmic_bytes_per_launch": int(nbytes)}}
+    # in place (codes aliased): scales only
+    a.record()
+    for _ in range(steps):
+        moe.transcode_mxfp4_to_nvfp4(c, s, nt, N, K, c, e4, g, st, ws, report=False)
+    b.record()
+    torch.cuda.synchronize()
+    ms2 = a.elapsed_time(b) / steps
+    nb2 = c.numel() + s.numel() + e4.numel()
+    res["in_place"] = {"ms": round(ms2, 4), "GB/s": round(nb2 / (ms2 / 1e3) / 1e9, 1)}
+    del c, s, co, e4
+    torch.cuda.empty_cache()
+    return res
+
+
+def cpu_baseline(wl, d, args, steps=1):
+    """The oracle as it stands, on a bounded token sample of the same workload."""
+    import oracle
+
+    threads = oracle.num_threads()
+    n = args.cpu_sample_tokens or threads
+    toks = np.arange(n, dtype=np.int32)
+    w = {k: d[k] for k in ("gate_codes", "gate_sf", "up_codes", "up_sf", "down_codes", "down_sf", "w_global")}
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.moe_layer(wl.mode, d["x"], d["logits"], None, w["gate_codes"], w["gate_sf"], w["up_codes"], w["up_sf"],
+                         w["down_codes"], w["down_sf"], w["w_global"], 1.0, wl.n_group, wl.topk_group, wl.top_k,
+                         wl.rsf, True, toks)
+    dt = (time.perf_counter() - t0) / steps
+    return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} tokens of the {wl.name} workload per step (float64 C oracle, OpenMP over tokens)",
+            "seconds_per_step": round(dt, 3)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = inputs.WORKLOADS[args.workload]
+    d = inputs.moe_inputs(wl)
+    import oracle
+
+    oracle.build()
+    for _ in range(min(args.warmup, 1)):
+        cpu_baseline(wl, d, args)
+    vals = [cpu_baseline(wl, d, args) for _ in range(max(1, min(args.steps, 5)))]
+    v = float(np.mean([r["value"] for r in vals]))
+    dt = float(np.mean([r["seconds_per_step"] for r in vals]))
+    out = {"impl": "reference", "metric": "MoE-layer tokens/s", "value": round(v, 3), "unit": "tokens/s",
+           "n_gpus": world, "steps": len(vals), "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top_k={wl.top_k} "
+                                  f"{'W4A4' if wl.mode else 'W4A16'}"},
+           "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "kind": "oracle", "cores": vals[0]["cores"],
+                            "sample": vals[0]["sample"]},
+           "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if "WORLD_SIZE" not in os.environ:
+        world = 1  # without torchrun there is one process
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

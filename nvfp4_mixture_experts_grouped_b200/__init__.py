@@ -1,1 +1,218 @@
+"""B200 (sm_100a) routed-expert MoE layer with NVFP4 expert weights.
 
+Thin ctypes binding of ``libnvfp4moe.so`` (declared in ``include/nvfp4moe.h``).
+Every function takes ``torch`` tensors that already live on the GPU, checks
+nothing beyond what ctypes needs, and passes raw device pointers and sizes to
+the C ABI; all arithmetic runs in the library's CUDA kernels.  PyTorch is used
+for device memory and streams only.  There is no CPU fallback: if the shared
+library cannot be loaded every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "W4A16", "W4A4", "NVFP4MoEError", "library_path", "load",
+    "transcode_mxfp4_to_nvfp4", "nvfp4moe_transcode_workspace_size", "moe_route", "quantize_nvfp4",
+    "moe_packed_weights_size", "moe_pack_weights", "moe_forward_workspace_size", "moe_forward",
+    "moe_forward_routed", "nvfp4moe_check_device_status", "nvfp4moe_version", "moe_permute",
+    "moe_permute_workspace_size", "nvfp4moe_set_trace_events",
+]
+
+W4A16 = 0
+W4A4 = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libnvfp4moe.so")
+_lib = None
+
+STATUS_NAMES = {
+    0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_ALIGNMENT", 3: "ERR_UNSUPPORTED_SHAPE", 4: "ERR_NAN_SCALE",
+    5: "ERR_NOT_REPRESENTABLE", 6: "ERR_WORKSPACE_TOO_SMALL", 7: "ERR_CUDA", 8: "ERR_TIMEOUT",
+    9: "ERR_UNSUPPORTED_DEVICE",
+}
+
+
+class NVFP4MoEError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class TranscodeReport(ctypes.Structure):
+    _fields_ = [("blocks", ctypes.c_int64), ("zero_blocks", ctypes.c_int64),
+                ("nonrepresentable_tensors", ctypes.c_int64), ("nan_scale_tensors", ctypes.c_int64)]
+
+
+class ExpertWeights(ctypes.Structure):
+    _fields_ = [("gate_codes", ctypes.c_void_p), ("gate_sf", ctypes.c_void_p), ("up_codes", ctypes.c_void_p),
+                ("up_sf", ctypes.c_void_p), ("down_codes", ctypes.c_void_p), ("down_sf", ctypes.c_void_p),
+                ("w_global", ctypes.c_void_p), ("E", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m nvfp4_mixture_experts_grouped_b200.build`")
+    L = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    L.nvfp4moe_last_error_string.restype = ctypes.c_char_p
+    L.nvfp4moe_version.restype = i32
+    L.nvfp4moe_transcode_workspace_size.restype = sz
+    L.nvfp4moe_transcode_workspace_size.argtypes = [i64]
+    L.transcode_mxfp4_to_nvfp4.restype = ctypes.c_int
+    L.transcode_mxfp4_to_nvfp4.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp, vp, sz, ctypes.POINTER(TranscodeReport),
+                                           vp]
+    L.moe_route.restype = ctypes.c_int
+    L.moe_route.argtypes = [vp, vp, i32, i32, i32, i32, i32, f32, i32, vp, vp, vp]
+    L.quantize_nvfp4.restype = ctypes.c_int
+    L.quantize_nvfp4.argtypes = [vp, i64, i64, f32, vp, vp, vp]
+    L.moe_packed_weights_size.restype = sz
+    L.moe_packed_weights_size.argtypes = [ctypes.c_int, i32, i32, i32]
+    L.moe_pack_weights.restype = ctypes.c_int
+    L.moe_pack_weights.argtypes = [ctypes.c_int, ctypes.POINTER(ExpertWeights), vp, vp]
+    L.moe_forward_workspace_size.restype = sz
+    L.moe_forward_workspace_size.argtypes = [ctypes.c_int, i32, i32, i32, i32, i32]
+    L.moe_forward.restype = ctypes.c_int
+    L.moe_forward.argtypes = [ctypes.c_int, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, i32, i32, f32, i32, vp, sz, vp,
+                              i32, vp, vp, vp]
+    L.moe_forward_routed.restype = ctypes.c_int
+    L.moe_forward_routed.argtypes = [ctypes.c_int, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, vp, sz, vp, i32, vp]
+    L.moe_permute_workspace_size.restype = sz
+    L.moe_permute_workspace_size.argtypes = [i32, i32, i32, i32]
+    L.moe_permute.restype = ctypes.c_int
+    L.moe_permute.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+    L.nvfp4moe_set_trace_events.restype = ctypes.c_int
+    L.nvfp4moe_set_trace_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
+    L.nvfp4moe_check_device_status.restype = ctypes.c_int
+    L.nvfp4moe_check_device_status.argtypes = [vp]
+    _lib = L
+    return L
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int):
+    if status != 0:
+        raise NVFP4MoEError(status, load().nvfp4moe_last_error_string().decode())
+
+
+def nvfp4moe_version() -> int:
+    return load().nvfp4moe_version()
+
+
+def nvfp4moe_transcode_workspace_size(num_tensors: int) -> int:
+    return load().nvfp4moe_transcode_workspace_size(num_tensors)
+
+
+def transcode_mxfp4_to_nvfp4(codes_in, e8m0_in, num_tensors, N, K, codes_out, e4m3_out, global_scale_out,
+                             tensor_status_out, workspace, report: bool = True, stream=None, raise_on_error=False):
+    """Returns (status, report dict or None).  With report=True the call is synchronous."""
+    rep = TranscodeReport()
+    st = load().transcode_mxfp4_to_nvfp4(
+        _ptr(codes_in), _ptr(e8m0_in), num_tensors, N, K, _ptr(codes_out), _ptr(e4m3_out), _ptr(global_scale_out),
+        _ptr(tensor_status_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        ctypes.byref(rep) if report else None, _stream(stream))
+    if st not in (0, 4, 5) or (raise_on_error and st != 0):
+        _check(st)
+    out = None
+    if report:
+        out = {f: getattr(rep, f) for f, _ in TranscodeReport._fields_}
+    return st, out
+
+
+def moe_route(logits, bias, n_group, topk_group, top_k, routed_scaling_factor, renormalize, topk_ids, topk_weights,
+              stream=None):
+    T, E = logits.shape
+    _check(load().moe_route(_ptr(logits), _ptr(bias), T, E, n_group, topk_group, top_k, routed_scaling_factor,
+                            int(renormalize), _ptr(topk_ids), _ptr(topk_weights), _stream(stream)))
+
+
+def quantize_nvfp4(x_bf16, gs, codes, e4m3_scales, stream=None):
+    M, K = x_bf16.shape
+    _check(load().quantize_nvfp4(_ptr(x_bf16), M, K, gs, _ptr(codes), _ptr(e4m3_scales), _stream(stream)))
+
+
+def moe_permute_workspace_size(T, E, top_k, pad) -> int:
+    return load().moe_permute_workspace_size(T, E, top_k, pad)
+
+
+def moe_permute(topk_ids, E, pad, counts_out, pad_offsets_out, row_of_pair_out, workspace, stream=None):
+    T, k = topk_ids.shape
+    _check(load().moe_permute(_ptr(topk_ids), T, E, k, pad, _ptr(counts_out), _ptr(pad_offsets_out),
+                              _ptr(row_of_pair_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)))
+
+
+def moe_packed_weights_size(mode, E, H, I) -> int:
+    return load().moe_packed_weights_size(mode, E, H, I)
+
+
+def moe_pack_weights(mode, gate_codes, gate_sf, up_codes, up_sf, down_codes, down_sf, w_global, packed, stream=None):
+    E, I = gate_codes.shape[0], gate_codes.shape[1]
+    H = down_codes.shape[1]
+    w = ExpertWeights(gate_codes.data_ptr(), gate_sf.data_ptr(), up_codes.data_ptr(), up_sf.data_ptr(),
+                      down_codes.data_ptr(), down_sf.data_ptr(), w_global.data_ptr(), E, H, I)
+    _check(load().moe_pack_weights(mode, ctypes.byref(w), _ptr(packed), _stream(stream)))
+
+
+def moe_forward_workspace_size(mode, T, H, I, E, top_k) -> int:
+    return load().moe_forward_workspace_size(mode, T, H, I, E, top_k)
+
+
+def moe_forward(mode, x, router_logits, bias, packed_weights, act_global, T, H, I, E, n_group, topk_group, top_k,
+                routed_scaling_factor, renormalize, workspace, out, topk_ids_out=None, topk_weights_out=None,
+                stream=None):
+    import torch
+
+    out_f32 = 1 if out.dtype == torch.float32 else 0
+    _check(load().moe_forward(mode, _ptr(x), _ptr(router_logits), _ptr(bias), _ptr(packed_weights), act_global, T, H,
+                              I, E, n_group, topk_group, top_k, routed_scaling_factor, int(renormalize),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), out_f32,
+                              _ptr(topk_ids_out), _ptr(topk_weights_out), _stream(stream)))
+
+
+def moe_forward_routed(mode, x, topk_ids, topk_weights, packed_weights, act_global, T, H, I, E, top_k, workspace, out,
+                       stream=None):
+    import torch
+
+    out_f32 = 1 if out.dtype == torch.float32 else 0
+    _check(load().moe_forward_routed(mode, _ptr(x), _ptr(topk_ids), _ptr(topk_weights), _ptr(packed_weights),
+                                     act_global, T, H, I, E, top_k, _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _ptr(out), out_f32,
+                                     _stream(stream)))
+
+
+def nvfp4moe_set_trace_events(events) -> None:
+    """events: None (tracing off) or 7 torch.cuda.Event(enable_timing=True) objects
+    (each already created, e.g. recorded once)."""
+    if events is None:
+        _check(load().nvfp4moe_set_trace_events(None, 0))
+        return
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _check(load().nvfp4moe_set_trace_events(arr, len(events)))
+
+
+def nvfp4moe_check_device_status(stream=None):
+    _check(load().nvfp4moe_check_device_status(_stream(stream)))

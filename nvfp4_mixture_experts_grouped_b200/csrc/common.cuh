@@ -1,0 +1,52 @@
+// common.cuh -- shared host/device plumbing of the sm_100a MoE library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nvfp4moe.h"
+
+namespace nvfp4moe {
+
+// ---------------------------------------------------------------------------
+// Host-side error reporting
+// ---------------------------------------------------------------------------
+void set_error(const char* fmt, ...);
+
+#define NVFP4MOE_CHECK_LAUNCH(what)                                                            \
+    do {                                                                                        \
+        cudaError_t _e = cudaGetLastError();                                                    \
+        if (_e != cudaSuccess) {                                                                \
+            ::nvfp4moe::set_error("%s: %s", what, cudaGetErrorString(_e));                      \
+            return NVFP4MOE_ERR_CUDA;                                                           \
+        }                                                                                       \
+    } while (0)
+
+#define NVFP4MOE_CUDA(call)                                                                    \
+    do {                                                                                        \
+        cudaError_t _e = (call);                                                                \
+        if (_e != cudaSuccess) {                                                                \
+            ::nvfp4moe::set_error("%s: %s", #call, cudaGetErrorString(_e));                     \
+            return NVFP4MOE_ERR_CUDA;                                                           \
+        }                                                                                       \
+    } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+// Device error word set by bounded waits that give up (never trapped).
+enum : int32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1 };
+int32_t* device_error_word();  // device address of the word (current device)
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
+__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+
+}  // namespace nvfp4moe

@@ -1,0 +1,69 @@
+// moe_internal.cuh -- declarations shared by the kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace nvfp4moe {
+
+constexpr int PERM_CHUNK = 256;  // tokens per permutation chunk (one CTA)
+constexpr int PERM_WARPS = PERM_CHUNK / 32;
+constexpr int MTILE = 128;       // rows of one tcgen05 M-tile
+
+__device__ __forceinline__ int64_t round_up_dev(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+// Device pointers (inside the workspace) describing one routing of T tokens.
+struct RoutingPlan {
+    int32_t* ids;           // [T*k] expert of each pair (pair = t*k + j)
+    float* wts;             // [T*k] routing weight of each pair
+    int32_t* chunk_counts;  // [n_chunks*E] per-chunk counts, then per-chunk rank bases
+    int32_t* counts;        // [E]
+    int32_t* offsets;       // [E+1] unpadded row offsets
+    int32_t* pad_offsets;   // [E+1] row offsets with every segment padded to `pad`
+    int32_t* row_of_pair;   // [T*k]
+    int32_t* pair_of_row;   // [rows_max]
+    int4* tiles;            // [max_tiles] {expert, first padded row, valid rows, m-tile index}
+    int32_t* n_tiles;       // [1]
+    int32_t* active;        // [E] experts with at least one row
+    int32_t* n_active;      // [1]
+};
+
+// transcode.cu
+size_t transcode_ws_size(int64_t num_tensors);
+nvfp4moe_status launch_transcode(const uint8_t* codes_in, const uint8_t* e8m0_in, int64_t num_tensors, int64_t N,
+                                 int64_t K, uint8_t* codes_out, uint8_t* e4m3_out, float* global_out,
+                                 int32_t* status_out, void* workspace, cudaStream_t stream);
+nvfp4moe_status read_transcode_report(const void* workspace, nvfp4moe_transcode_report* out, cudaStream_t stream);
+
+// route.cu
+nvfp4moe_status launch_route(const float* logits, const float* bias, int T, int E, int n_group, int topk_group,
+                             int top_k, float rsf, int renorm, int32_t* ids, float* wts, cudaStream_t stream);
+
+// permute.cu
+nvfp4moe_status launch_permute(const int32_t* ids, int T, int k, int E, int pad, RoutingPlan& plan,
+                               cudaStream_t stream);
+nvfp4moe_status launch_quantize_linear(const uint16_t* x, int64_t M, int64_t K, float gs, uint8_t* codes,
+                                       uint8_t* scales, cudaStream_t stream);
+nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H, float gs, uint8_t* codes,
+                                        uint8_t* scales, const int32_t* row_of_pair, int k, cudaStream_t stream);
+nvfp4moe_status launch_combine(const uint16_t* Y, const int32_t* row_of_pair, int64_t T, int H, int k, void* out,
+                               bool out_f32, cudaStream_t stream);
+
+// w4a16.cu
+size_t w4a16_packed_size(int E, int H, int I);
+nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream);
+nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T, int H, int I, int E, int k,
+                                   const RoutingPlan& plan, uint16_t* A2, uint16_t* Y, cudaStream_t stream,
+                                   cudaEvent_t mid_event);
+
+// w4a4.cu
+size_t w4a4_packed_size(int E, int H, int I);
+nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream);
+nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E, int k, float act_global,
+                                  int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
+                                  const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, uint16_t* Y, cudaStream_t stream,
+                                  cudaEvent_t mid_event);
+
+}  // namespace nvfp4moe

@@ -1,0 +1,270 @@
+// permute.cu -- token permutation (grouping (token, slot) pairs by expert),
+// activation quantise-and-scatter, and the weighted un-permute (combine).
+//
+// Grouped experts: "AxionML / MiMo-V2.6-Flash-MOPD-NVFP4", "Usage" (fused
+// grouped MoE backend); "MiMo-V2.6-Flash-MOPD on one RTX PRO 6000", "Speed v4"
+// (exact grouped kernel).  Combine: "MiMo-V2.6-Flash -- REAP-50", "Pruning
+// Method" 1 (the layer output is the g_{t,j}-weighted sum of the selected
+// experts' outputs).
+//
+// Rows of expert e occupy [pad_off[e], pad_off[e] + count[e]) of the permuted
+// buffers, ordered by token then slot (deterministic, no sort).  pad_off rounds
+// every expert's segment up to `pad` rows so that GEMM M-tiles never straddle
+// two experts (pad = 128 for the tcgen05 path, 1 for the W4A16 path).
+#include "common.cuh"
+#include "formats.cuh"
+#include "moe_internal.cuh"
+
+namespace nvfp4moe {
+
+// ---------------------------------------------------------------------------
+// 1. per-chunk expert histogram (chunks of PERM_CHUNK tokens)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(PERM_CHUNK)
+    k_count_chunks(const int32_t* __restrict__ ids, int T, int k, int E, int32_t* __restrict__ chunk_counts) {
+    extern __shared__ int s_hist[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+    __syncthreads();
+    const int t = blockIdx.x * PERM_CHUNK + threadIdx.x;
+    if (t < T)
+        for (int j = 0; j < k; ++j) atomicAdd(&s_hist[ids[(int64_t)t * k + j]], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[(int64_t)blockIdx.x * E + e] = s_hist[e];
+}
+
+// ---------------------------------------------------------------------------
+// 2. per-expert scan over chunks, expert offsets, M-tile list, active list
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int& total) {
+    // blockDim.x == 1024
+    const int tid = threadIdx.x;
+    s_tmp[tid] = v;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+        const int add = tid >= o ? s_tmp[tid - o] : 0;
+        __syncthreads();
+        s_tmp[tid] += add;
+        __syncthreads();
+    }
+    total = s_tmp[1023];
+    const int incl = s_tmp[tid];
+    __syncthreads();
+    return incl - v;
+}
+
+__global__ void __launch_bounds__(1024)
+    k_scan_experts(int n_chunks, int E, int pad, int32_t* __restrict__ chunk_counts, RoutingPlan plan) {
+    __shared__ int s_tmp[1024];
+    const int e = threadIdx.x;
+    int cnt = 0;
+    if (e < E) {
+        for (int c = 0; c < n_chunks; ++c) {
+            const int v = chunk_counts[(int64_t)c * E + e];
+            chunk_counts[(int64_t)c * E + e] = cnt;  // becomes the rank base of chunk c
+            cnt += v;
+        }
+    }
+    int total;
+    const int off = block_exclusive_scan(cnt, s_tmp, total);
+    const int padded = e < E ? (int)round_up_dev(cnt, pad) : 0;
+    int ptotal;
+    const int poff = block_exclusive_scan(padded, s_tmp, ptotal);
+    const int tiles = e < E ? (cnt + MTILE - 1) / MTILE : 0;
+    int ttotal;
+    const int toff = block_exclusive_scan(tiles, s_tmp, ttotal);
+    int atotal;
+    const int aoff = block_exclusive_scan(e < E && cnt > 0 ? 1 : 0, s_tmp, atotal);
+    if (e < E) {
+        plan.counts[e] = cnt;
+        plan.offsets[e] = off;
+        plan.pad_offsets[e] = poff;
+        for (int j = 0; j < tiles; ++j) {
+            int4 ti;
+            ti.x = e;
+            ti.y = poff + j * MTILE;
+            ti.z = min(MTILE, cnt - j * MTILE);
+            ti.w = j;
+            plan.tiles[toff + j] = ti;
+        }
+        if (cnt > 0) plan.active[aoff] = e;
+    }
+    if (e == 0) {
+        plan.offsets[E] = total;
+        plan.pad_offsets[E] = ptotal;
+        plan.n_tiles[0] = ttotal;
+        plan.n_active[0] = atotal;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 3. stable scatter: row of every (token, slot) pair
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(PERM_CHUNK)
+    k_scatter(const int32_t* __restrict__ ids, int T, int k, int E, const int32_t* __restrict__ chunk_base,
+              RoutingPlan plan) {
+    extern __shared__ int s_wh[];  // [PERM_WARPS][E]
+    const int warp = warp_id(), lane = lane_id();
+    for (int i = threadIdx.x; i < PERM_WARPS * E; i += blockDim.x) s_wh[i] = 0;
+    __syncthreads();
+    const int t0 = blockIdx.x * PERM_CHUNK + warp * 32;
+    {
+        const int t = t0 + lane;
+        if (t < T)
+            for (int j = 0; j < k; ++j) atomicAdd(&s_wh[warp * E + ids[(int64_t)t * k + j]], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = chunk_base[(int64_t)blockIdx.x * E + e];
+        for (int w = 0; w < PERM_WARPS; ++w) {
+            const int v = s_wh[w * E + e];
+            s_wh[w * E + e] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    // tokens of this warp in order; a token's k experts are distinct, so the
+    // k lanes never touch the same counter in one step
+    for (int i = 0; i < 32; ++i) {
+        const int t = t0 + i;
+        if (t >= T) break;
+        if (lane < k) {
+            const int64_t p = (int64_t)t * k + lane;
+            const int e = ids[p];
+            const int r = s_wh[warp * E + e]++;
+            const int row = plan.pad_offsets[e] + r;
+            plan.row_of_pair[p] = row;
+            plan.pair_of_row[row] = (int32_t)p;
+        }
+        __syncwarp();
+    }
+}
+
+nvfp4moe_status launch_permute(const int32_t* ids, int T, int k, int E, int pad, RoutingPlan& plan,
+                               cudaStream_t stream) {
+    const int n_chunks = (int)ceil_div(T, PERM_CHUNK);
+    k_count_chunks<<<n_chunks, PERM_CHUNK, E * sizeof(int), stream>>>(ids, T, k, E, plan.chunk_counts);
+    NVFP4MOE_CHECK_LAUNCH("permute count kernel");
+    k_scan_experts<<<1, 1024, 0, stream>>>(n_chunks, E, pad, plan.chunk_counts, plan);
+    NVFP4MOE_CHECK_LAUNCH("permute scan kernel");
+    k_scatter<<<n_chunks, PERM_CHUNK, PERM_WARPS * E * sizeof(int), stream>>>(ids, T, k, E, plan.chunk_counts, plan);
+    NVFP4MOE_CHECK_LAUNCH("permute scatter kernel");
+    return NVFP4MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// 4. NVFP4 quantisation (one warp per row, a 16-element block per lane step)
+// ---------------------------------------------------------------------------
+// Linear layout (quantize_nvfp4): codes [M, K/2], scales [M, K/16].
+// Scatter layout (moe_forward W4A4): the token's codes go to the k permuted
+// rows of its pairs; scales go to the tcgen05 block-scale atom layout.
+template <bool SCATTER>
+__global__ void __launch_bounds__(256)
+    k_quantize(const uint16_t* __restrict__ x, int64_t M, int64_t K, float gs, uint8_t* __restrict__ codes,
+               uint8_t* __restrict__ scales, const int32_t* __restrict__ row_of_pair, int k) {
+    const int64_t m = (int64_t)blockIdx.x * 8 + warp_id();
+    if (m >= M) return;
+    const int lane = lane_id();
+    const int64_t nb = K / 16;
+    const uint16_t* xr = x + m * K;
+    int rows[32];
+    int nrows = 1;
+    if (SCATTER) {
+        nrows = k;
+        for (int j = 0; j < k; ++j) rows[j] = row_of_pair[m * k + j];
+    }
+    for (int64_t b = lane; b < nb; b += 32) {
+        const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(xr + b * 16));
+        const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(xr + b * 16 + 8));
+        float f[16];
+        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            f[2 * i] = bf16_bits_to_float(w[i] & 0xFFFFu);
+            f[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+        }
+        uint32_t c0, c1;
+        const uint32_t sf = quantize_block16(f, gs, c0, c1);
+        if (!SCATTER) {
+            *reinterpret_cast<uint2*>(codes + m * (K / 2) + b * 8) = make_uint2(c0, c1);
+            scales[m * nb + b] = (uint8_t)sf;
+        } else {
+            for (int j = 0; j < nrows; ++j) {
+                const int64_t row = rows[j];
+                *reinterpret_cast<uint2*>(codes + row * (K / 2) + b * 8) = make_uint2(c0, c1);
+                scales[sf_atom_offset(row, b, nb)] = (uint8_t)sf;
+            }
+        }
+    }
+}
+
+nvfp4moe_status launch_quantize_linear(const uint16_t* x, int64_t M, int64_t K, float gs, uint8_t* codes,
+                                       uint8_t* scales, cudaStream_t stream) {
+    if (M == 0) return NVFP4MOE_OK;
+    k_quantize<false><<<(unsigned)ceil_div(M, 8), 256, 0, stream>>>(x, M, K, gs, codes, scales, nullptr, 1);
+    NVFP4MOE_CHECK_LAUNCH("quantize kernel");
+    return NVFP4MOE_OK;
+}
+
+nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H, float gs, uint8_t* codes,
+                                        uint8_t* scales, const int32_t* row_of_pair, int k, cudaStream_t stream) {
+    if (T == 0) return NVFP4MOE_OK;
+    k_quantize<true><<<(unsigned)ceil_div(T, 8), 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k);
+    NVFP4MOE_CHECK_LAUNCH("quantize-scatter kernel");
+    return NVFP4MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// 5. weighted un-permute: out[t] = sum_j Y[row_of_pair(t, j)] (weights already
+//    applied by the down GEMM), FP32 in slot order, one rounding.
+// ---------------------------------------------------------------------------
+template <bool OUT_F32>
+__global__ void __launch_bounds__(256)
+    k_combine(const uint16_t* __restrict__ Y, const int32_t* __restrict__ row_of_pair, int64_t T, int H, int k,
+              void* __restrict__ out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // one 8-element vector
+    const int64_t per_row = H / 8;
+    if (i >= T * per_row) return;
+    const int64_t t = i / per_row;
+    const int64_t h8 = (i - t * per_row) * 8;
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        const int64_t row = __ldg(row_of_pair + t * k + j);
+        const uint4 v = __ldcs(reinterpret_cast<const uint4*>(Y + row * H + h8));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            acc[2 * q] = __fadd_rn(acc[2 * q], bf16_bits_to_float(w[q] & 0xFFFFu));
+            acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16_bits_to_float(w[q] >> 16));
+        }
+    }
+    if (OUT_F32) {
+        float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + t * H + h8);
+        __stcs(o, make_float4(acc[0], acc[1], acc[2], acc[3]));
+        __stcs(o + 1, make_float4(acc[4], acc[5], acc[6], acc[7]));
+    } else {
+        uint32_t p[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+            p[q] = *reinterpret_cast<uint32_t*>(&b);
+        }
+        __stcs(reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + t * H + h8), make_uint4(p[0], p[1], p[2], p[3]));
+    }
+}
+
+nvfp4moe_status launch_combine(const uint16_t* Y, const int32_t* row_of_pair, int64_t T, int H, int k, void* out,
+                               bool out_f32, cudaStream_t stream) {
+    if (T == 0) return NVFP4MOE_OK;
+    const int64_t n = T * (H / 8);
+    const unsigned grid = (unsigned)ceil_div(n, 256);
+    if (out_f32)
+        k_combine<true><<<grid, 256, 0, stream>>>(Y, row_of_pair, T, H, k, out);
+    else
+        k_combine<false><<<grid, 256, 0, stream>>>(Y, row_of_pair, T, H, k, out);
+    NVFP4MOE_CHECK_LAUNCH("combine kernel");
+    return NVFP4MOE_OK;
+}
+
+}  // namespace nvfp4moe

@@ -1,0 +1,415 @@
+// w4a4.cu -- W4A4 grouped expert GEMMs on the sm_100a 5th-generation tensor
+// cores: NVFP4 activations x NVFP4 weights with tcgen05.mma kind::mxf4nvf4
+// (E4M3 block scale per 16 elements, FP32 accumulators in tensor memory).
+//
+// Mode: "AxionML / MiMo-V2.6-Flash-MOPD-NVFP4", introduction (routed experts as
+// W4A4 NVFP4 on native FP4 tensor cores) and "Why a unit activation scale".
+// Expert MLP: "MiMo-V2.6-Flash -- REAP-50", "Pruning Method" 1.
+//
+// One persistent kernel per projection, one CTA per SM, 128 x 256 output tiles:
+//   warp 0      TMA producer: A/B code tiles (SWIZZLE_128B tensor maps, never
+//               multicast) and their block-scale atoms (1-D bulk copies) into a
+//               4-stage shared-memory ring guarded by mbarriers;
+//   warp 1      MMA issuer: copies the stage's scale factors into TMEM
+//               (tcgen05.cp 32x128b.warpx4) and issues four K=64 block-scaled
+//               MMAs per stage into a 128 x 256 FP32 TMEM accumulator;
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quadrant, then
+//               gate/up: SiLU(gate) * up and NVFP4 requantisation per 16 (the
+//                        down GEMM's A operand, written straight into its
+//                        block-scale layout);
+//               down:    x global scale x routing weight, BF16 per-pair rows.
+// Rows of an expert are padded to 128 by the permutation, so an M-tile never
+// straddles two experts; padding rows are computed and never stored.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "formats.cuh"
+#include "moe_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace nvfp4moe {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 256;  // BK in elements (128 bytes of codes)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK / 2;
+constexpr int B_BYTES = BN * BK / 2;
+constexpr int SFA_BYTES = BM * BK / 16;
+constexpr int SFB_BYTES = BN * BK / 16;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_SF = 256;      // scale-factor columns after the 256 accumulator columns
+constexpr uint32_t TM_SF_STRIDE = 48;  // per buffer: 16 (A: 4 k-steps x 4) + 32 (B: 4 x 8)
+constexpr int THREADS = 192;
+
+enum { EPI_GATEUP = 0, EPI_DOWN = 1 };
+
+struct W4Layout {
+    int64_t gu_codes, gu_sf, d_codes, d_sf, globals, total;
+};
+
+inline int64_t a256(int64_t v) { return (v + 255) / 256 * 256; }
+
+W4Layout w4_layout(int E, int H, int I) {
+    W4Layout L;
+    L.gu_codes = 0;
+    L.gu_sf = a256(L.gu_codes + (int64_t)E * 2 * I * H / 2);
+    L.d_codes = a256(L.gu_sf + (int64_t)E * 2 * I * H / 16);
+    L.d_sf = a256(L.d_codes + (int64_t)E * H * I / 2);
+    L.globals = a256(L.d_sf + (int64_t)E * H * I / 16);
+    L.total = a256(L.globals + (int64_t)E * 3 * 4);
+    return L;
+}
+
+struct GemmParams {
+    int K;                   // reduction length (elements)
+    int n_ntiles;            // N / 256
+    int64_t b_rows_per_expert;
+    const int4* tiles;       // M-tile list
+    const int32_t* n_tiles;  // number of M-tiles (device)
+    const uint8_t* sfa;      // A block scales, atom layout
+    const uint8_t* sfb;      // B block scales, atom layout
+    const float* globals;    // [E, 3]
+    float act_global;
+    uint8_t* out_codes;      // gate/up: intermediate codes [rows, I/2]
+    uint8_t* out_sf;         // gate/up: intermediate scales, atom layout
+    int out_k;               // gate/up: I
+    uint16_t* Y;             // down: [rows, H] BF16
+    int ldy;                 // down: H
+    const float* wts;        // down: routing weight of each pair
+    const int32_t* pair_of_row;
+    int32_t* err;
+};
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_w4a4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;
+    uint64_t* acc_empty = acc_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+
+    const int warp = warp_id(), lane = lane_id();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        tc::mbar_init(acc_full, 1);
+        tc::mbar_init(acc_empty, 4);
+        tc::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tc::prefetch_tmap(&tmA);
+        tc::prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int total = p.n_tiles[0] * p.n_ntiles;
+    const int k64_total = p.K / 64;
+    const int ks_count = (k64_total + 3) / 4;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int it = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                const int m = tile / p.n_ntiles, n = tile - m * p.n_ntiles;
+                const int4 ti = p.tiles[m];
+                const int64_t b_row0 = (int64_t)ti.x * p.b_rows_per_expert + (int64_t)n * BN;
+                for (int ks = 0; ks < ks_count; ++ks, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    if (!tc::mbar_wait(&empty[s], ph ^ 1u, p.err)) goto done;
+                    const int n64 = min(4, k64_total - ks * 4);
+                    uint8_t* st = smem + s * STAGE_BYTES;
+                    tc::mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES + 3 * n64 * 512);
+                    tc::tma_load_2d(st, &tmA, ks * 128, ti.y, &full[s]);
+                    tc::tma_load_2d(st + A_BYTES, &tmB, ks * 128, (int32_t)b_row0, &full[s]);
+                    const uint8_t* sfa = p.sfa + ((int64_t)(ti.y / 128) * k64_total + ks * 4) * 512;
+                    tc::bulk_load(st + A_BYTES + B_BYTES, sfa, n64 * 512, &full[s]);
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const uint8_t* sfb = p.sfb + ((b_row0 / 128 + r) * k64_total + ks * 4) * 512;
+                        tc::bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES + r * 2048, sfb, n64 * 512, &full[s]);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = tc::idesc_mxf4nvf4(BM, BN);
+            int it = 0, tl = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tl) {
+                if (!tc::mbar_wait(acc_empty, ((uint32_t)tl & 1u) ^ 1u, p.err)) goto done;
+                tc::tc_fence_after();
+                for (int ks = 0; ks < ks_count; ++ks, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    if (!tc::mbar_wait(&full[s], ph, p.err)) goto done;
+                    tc::tc_fence_after();
+                    const int n64 = min(4, k64_total - ks * 4);
+                    uint8_t* st = smem + s * STAGE_BYTES;
+                    const uint32_t sf_col = tmem + TM_SF + (uint32_t)(it & 1) * TM_SF_STRIDE;
+                    for (int j = 0; j < n64; ++j) {
+                        tc::tmem_cp_32x128_x4(sf_col + 4 * j, tc::desc_sf(st + A_BYTES + B_BYTES + j * 512));
+                        tc::tmem_cp_32x128_x4(sf_col + 16 + 8 * j,
+                                              tc::desc_sf(st + A_BYTES + B_BYTES + SFA_BYTES + j * 512));
+                        tc::tmem_cp_32x128_x4(sf_col + 16 + 8 * j + 4,
+                                              tc::desc_sf(st + A_BYTES + B_BYTES + SFA_BYTES + 2048 + j * 512));
+                    }
+                    const uint64_t adesc = tc::desc_sw128(st);
+                    const uint64_t bdesc = tc::desc_sw128(st + A_BYTES);
+                    for (int j = 0; j < n64; ++j)
+                        tc::mma_mxf4nvf4(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j,
+                                         sf_col + 16 + 8 * j, (ks | j) != 0);
+                    tc::tc_commit(&empty[s]);
+                }
+                tc::tc_commit(acc_full);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        const int r_in = q * 32 + lane;
+        const uint32_t t_row = tmem + ((uint32_t)(q * 32) << 16);
+        int tl = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tl) {
+            const int m = tile / p.n_ntiles, n = tile - m * p.n_ntiles;
+            const int4 ti = p.tiles[m];
+            const bool valid = r_in < ti.z;
+            const int64_t row = (int64_t)ti.y + r_in;
+            if (!tc::mbar_wait(acc_full, (uint32_t)tl & 1u, p.err)) goto done;
+            tc::tc_fence_after();
+            if (EPI == EPI_GATEUP) {
+                const float ag = p.globals[ti.x * 3 + 0] * p.act_global;
+                const float au = p.globals[ti.x * 3 + 1] * p.act_global;
+                const int i0 = n * (BN / 2);
+                const int nkb = p.out_k / 16;
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    float gv[16], uv[16];
+                    tc::tmem_ld16x2(t_row + 16 * c, t_row + 128 + 16 * c, gv, uv);
+                    if (valid) {
+                        float a[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) a[i] = silu(gv[i] * ag) * (uv[i] * au);
+                        uint32_t w0, w1;
+                        const uint32_t sf = quantize_block16(a, p.act_global, w0, w1);
+                        const int col = i0 + 16 * c;
+                        *reinterpret_cast<uint2*>(p.out_codes + row * (p.out_k / 2) + col / 2) = make_uint2(w0, w1);
+                        p.out_sf[sf_atom_offset(row, col / 16, nkb)] = (uint8_t)sf;
+                    }
+                }
+            } else {
+                const float f = valid ? p.globals[ti.x * 3 + 2] * p.act_global * p.wts[p.pair_of_row[row]] : 0.0f;
+                uint16_t* yrow = p.Y + row * p.ldy + (int64_t)n * BN;
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    float v0[16], v1[16];
+                    tc::tmem_ld16x2(t_row + 32 * c, t_row + 32 * c + 16, v0, v1);
+                    if (valid) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            __nv_bfloat162 b0 = __floats2bfloat162_rn(v0[2 * i] * f, v0[2 * i + 1] * f);
+                            __nv_bfloat162 b1 = __floats2bfloat162_rn(v1[2 * i] * f, v1[2 * i + 1] * f);
+                            pk[i] = *reinterpret_cast<uint32_t*>(&b0);
+                            pk[8 + i] = *reinterpret_cast<uint32_t*>(&b1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(yrow + 32 * c);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    }
+                }
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(acc_empty);
+        }
+    }
+done:
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// pack: gate/up rows interleaved per 128 (a 256-row N-tile = 128 gate rows then
+// the same 128 intermediates' up rows), block scales into the atom layout.
+// ---------------------------------------------------------------------------
+__global__ void k_w4_pack_codes(const uint8_t* __restrict__ src0, const uint8_t* __restrict__ src1, int64_t rows,
+                                int64_t row_bytes, int interleave, int64_t rows_per_expert_src,
+                                uint8_t* __restrict__ dst) {
+    const int64_t vec_per_row = row_bytes / 16;
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= rows * vec_per_row) return;
+    const int64_t prow = idx / vec_per_row, v = idx - prow * vec_per_row;
+    const uint8_t* src = src0;
+    int64_t srow = prow;
+    if (interleave) {
+        const int64_t per_e = 2 * rows_per_expert_src;
+        const int64_t e = prow / per_e, p = prow - e * per_e;
+        const int64_t b = p / 256, w = p % 256;
+        src = w < 128 ? src0 : src1;
+        srow = e * rows_per_expert_src + b * 128 + (w & 127);
+    }
+    reinterpret_cast<uint4*>(dst)[idx] = reinterpret_cast<const uint4*>(src + srow * row_bytes)[v];
+}
+
+__global__ void k_w4_pack_sf(const uint8_t* __restrict__ src0, const uint8_t* __restrict__ src1, int64_t rows,
+                             int64_t nkb, int interleave, int64_t rows_per_expert_src, uint8_t* __restrict__ dst) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= rows * nkb) return;
+    const int64_t prow = idx / nkb, kb = idx - prow * nkb;
+    const uint8_t* src = src0;
+    int64_t srow = prow;
+    if (interleave) {
+        const int64_t per_e = 2 * rows_per_expert_src;
+        const int64_t e = prow / per_e, p = prow - e * per_e;
+        const int64_t b = p / 256, w = p % 256;
+        src = w < 128 ? src0 : src1;
+        srow = e * rows_per_expert_src + b * 128 + (w & 127);
+    }
+    const int64_t off = ((prow >> 7) * (nkb >> 2) + (kb >> 2)) * 512 + (prow & 31) * 16 + ((prow >> 5) & 3) * 4 + (kb & 3);
+    dst[off] = src[srow * nkb + kb];
+}
+
+// ---------------------------------------------------------------------------
+// host: tensor maps and launches
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D uint8 map over [rows, row_bytes] with a box of 128 bytes x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t row_bytes, int64_t rows, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) {
+        set_error("cuTensorMapEncodeTiled is not available from the driver");
+        return false;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d) for a [%lld x %lld] map", (int)r, (long long)rows,
+                  (long long)row_bytes);
+        return false;
+    }
+    return true;
+}
+
+}  // namespace
+
+size_t w4a4_packed_size(int E, int H, int I) { return (size_t)w4_layout(E, H, I).total; }
+
+nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream) {
+    const int E = w.E, H = w.H, I = w.I;
+    const W4Layout L = w4_layout(E, H, I);
+    uint8_t* p = static_cast<uint8_t*>(packed);
+    const int64_t gu_rows = (int64_t)E * 2 * I, d_rows = (int64_t)E * H;
+    k_w4_pack_codes<<<(unsigned)ceil_div(gu_rows * (H / 32), 256), 256, 0, stream>>>(
+        w.gate_codes, w.up_codes, gu_rows, H / 2, 1, I, p + L.gu_codes);
+    k_w4_pack_sf<<<(unsigned)ceil_div(gu_rows * (H / 16), 256), 256, 0, stream>>>(w.gate_sf, w.up_sf, gu_rows, H / 16,
+                                                                                   1, I, p + L.gu_sf);
+    k_w4_pack_codes<<<(unsigned)ceil_div(d_rows * (I / 32), 256), 256, 0, stream>>>(w.down_codes, nullptr, d_rows,
+                                                                                     I / 2, 0, H, p + L.d_codes);
+    k_w4_pack_sf<<<(unsigned)ceil_div(d_rows * (I / 16), 256), 256, 0, stream>>>(w.down_sf, nullptr, d_rows, I / 16, 0,
+                                                                                   H, p + L.d_sf);
+    NVFP4MOE_CHECK_LAUNCH("w4a4 pack");
+    NVFP4MOE_CUDA(cudaMemcpyAsync(p + L.globals, w.w_global, (size_t)E * 3 * sizeof(float), cudaMemcpyDeviceToDevice,
+                                  stream));
+    return NVFP4MOE_OK;
+}
+
+nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E, int k, float act_global,
+                                  int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
+                                  const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, uint16_t* Y, cudaStream_t stream,
+                                  cudaEvent_t mid_event) {
+    (void)T;
+    (void)k;
+    const W4Layout L = w4_layout(E, H, I);
+    const uint8_t* pk = static_cast<const uint8_t*>(packed);
+    NVFP4MOE_CUDA(
+        cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w4a4_gemm<EPI_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    CUtensorMap mA1, mGU, mA2, mD;
+    if (!make_map(&mA1, A1c, H / 2, rows_max, BM) || !make_map(&mGU, pk + L.gu_codes, H / 2, (int64_t)E * 2 * I, BN) ||
+        !make_map(&mA2, A2c, I / 2, rows_max, BM) || !make_map(&mD, pk + L.d_codes, I / 2, (int64_t)E * H, BN))
+        return NVFP4MOE_ERR_CUDA;
+    const int sms = num_sms();
+    GemmParams g{};
+    g.tiles = plan.tiles;
+    g.n_tiles = plan.n_tiles;
+    g.globals = reinterpret_cast<const float*>(pk + L.globals);
+    g.act_global = act_global;
+    g.err = device_error_word();
+    g.wts = plan.wts;
+    g.pair_of_row = plan.pair_of_row;
+    // gate/up + SwiGLU + requantise
+    g.K = H;
+    g.n_ntiles = (2 * I) / BN;
+    g.b_rows_per_expert = 2 * I;
+    g.sfa = A1s;
+    g.sfb = pk + L.gu_sf;
+    g.out_codes = A2c;
+    g.out_sf = A2s;
+    g.out_k = I;
+    {
+        const int grid = (int)std::min<int64_t>(sms, (int64_t)max_tiles * g.n_ntiles);
+        k_w4a4_gemm<EPI_GATEUP><<<grid, THREADS, SMEM_BYTES, stream>>>(mA1, mGU, g);
+        NVFP4MOE_CHECK_LAUNCH("w4a4 gate/up kernel");
+    }
+    if (mid_event) cudaEventRecord(mid_event, stream);
+    // down x routing weight
+    g.K = I;
+    g.n_ntiles = H / BN;
+    g.b_rows_per_expert = H;
+    g.sfa = A2s;
+    g.sfb = pk + L.d_sf;
+    g.Y = Y;
+    g.ldy = H;
+    {
+        const int grid = (int)std::min<int64_t>(sms, (int64_t)max_tiles * g.n_ntiles);
+        k_w4a4_gemm<EPI_DOWN><<<grid, THREADS, SMEM_BYTES, stream>>>(mA2, mD, g);
+        NVFP4MOE_CHECK_LAUNCH("w4a4 down kernel");
+    }
+    return NVFP4MOE_OK;
+}
+
+}  // namespace nvfp4moe

@@ -1,0 +1,117 @@
+"""The C ABI library: it loads, exports every function include/nvfp4moe.h
+declares, and its host-side validation rejects bad arguments before touching
+the GPU.  CPU only (no kernel is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_mixture_experts_grouped_b200 as moe
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "nvfp4moe.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w ]*?[\s\*]+([A-Za-z_]\w*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+def test_header_declares_the_hot_path_calls():
+    names = declared_functions()
+    for n in ("transcode_mxfp4_to_nvfp4", "moe_route", "quantize_nvfp4", "moe_forward", "moe_pack_weights",
+              "moe_permute", "moe_forward_routed"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = moe.load()
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_version_and_sizes():
+    assert moe.nvfp4moe_version() >> 16 == 1
+    assert moe.nvfp4moe_transcode_workspace_size(768) >= 32
+    E, H, I = 256, 4096, 2048
+    # W4A4 packed weights hold exactly the checkpoint bytes (codes + E4M3 scales + globals)
+    exact = E * (2 * I * H + H * I) // 2 + E * (2 * I * H + H * I) // 16 + E * 3 * 4
+    assert exact <= moe.moe_packed_weights_size(moe.W4A4, E, H, I) <= exact + 1024
+    assert exact <= moe.moe_packed_weights_size(moe.W4A16, E, H, I) <= exact + 1024
+    ws = moe.moe_forward_workspace_size(moe.W4A4, 8192, H, I, E, 8)
+    assert ws > 8192 * 8 * H * 2  # holds the per-pair BF16 rows at least
+    assert moe.moe_forward_workspace_size(moe.W4A4, -1, H, I, E, 8) == 0
+
+
+def _status(call):
+    return call
+
+
+@pytest.mark.parametrize("args,expect", [
+    # T, E, n_group, topk_group, top_k
+    ((4, 0, 1, 1, 1), 3),
+    ((4, 256, 7, 4, 8), 3),     # E % n_group
+    ((4, 256, 8, 9, 8), 3),     # topk_group > n_group
+    ((4, 256, 8, 4, 33), 3),    # top_k > 32
+    ((4, 16, 4, 1, 5), 3),      # top_k > experts in the kept groups
+    ((-1, 256, 8, 4, 8), 1),    # negative T
+    ((4, 256, 64, 4, 8), 3),    # n_group > 32
+])
+def test_route_rejects_bad_shapes_before_launch(args, expect):
+    lib = moe.load()
+    T, E, ng, tg, k = args
+    st = lib.moe_route(ctypes.c_void_p(16), None, T, E, ng, tg, k, 2.827, 1, ctypes.c_void_p(16),
+                       ctypes.c_void_p(16), None)
+    assert st == expect, lib.nvfp4moe_last_error_string()
+
+
+def test_route_rejects_misaligned_pointer():
+    lib = moe.load()
+    st = lib.moe_route(ctypes.c_void_p(24), None, 4, 256, 8, 4, 8, 2.827, 1, ctypes.c_void_p(16),
+                       ctypes.c_void_p(16), None)
+    assert st == 2
+
+
+def test_quantize_and_transcode_validation():
+    lib = moe.load()
+    assert lib.quantize_nvfp4(ctypes.c_void_p(16), 4, 24, 1.0, ctypes.c_void_p(16), ctypes.c_void_p(16), None) == 3
+    assert lib.quantize_nvfp4(ctypes.c_void_p(16), 4, 32, 0.0, ctypes.c_void_p(16), ctypes.c_void_p(16), None) == 1
+    assert lib.quantize_nvfp4(ctypes.c_void_p(16), 4, 32, float("nan"), ctypes.c_void_p(16), ctypes.c_void_p(16),
+                              None) == 1
+    p = ctypes.c_void_p(4096)
+    # K not a multiple of 32
+    assert lib.transcode_mxfp4_to_nvfp4(p, p, 1, 4, 48, p, p, p, p, p, 64, None, None) == 3
+    # workspace too small
+    assert lib.transcode_mxfp4_to_nvfp4(p, p, 1, 4, 64, p, p, p, p, p, 1, None, None) == 6
+    # overlapping but unequal code buffers
+    assert lib.transcode_mxfp4_to_nvfp4(p, p, 1, 4, 64, ctypes.c_void_p(4096 + 16), p, p, p, p, 64, None,
+                                        None) == 1
+
+
+def test_forward_validation():
+    lib = moe.load()
+    p = ctypes.c_void_p(4096)
+    args = dict(T=4, H=4096, I=2048, E=256, ng=8, tg=4, k=8)
+
+    def call(mode=1, ws_bytes=1 << 40, **kw):
+        a = {**args, **kw}
+        return lib.moe_forward(mode, p, p, None, p, 1.0, a["T"], a["H"], a["I"], a["E"], a["ng"], a["tg"], a["k"],
+                               2.827, 1, p, ws_bytes, p, 0, None, None, None)
+
+    assert call(mode=3) == 1
+    assert call(H=4000) == 3
+    assert call(I=200) == 3
+    assert call(ws_bytes=16) == 6
+    assert lib.moe_forward(1, p, p, None, p, 0.0, 4, 4096, 2048, 256, 8, 4, 8, 2.827, 1, p, 1 << 40, p, 0, None,
+                           None, None) == 1
+    # T == 0 is a no-op even with null pointers
+    assert lib.moe_forward(1, None, None, None, None, 1.0, 0, 4096, 2048, 256, 8, 4, 8, 2.827, 1, None, 0, None, 0,
+                           None, None, None) == 0
+
+
+def test_error_string_is_text():
+    lib = moe.load()
+    lib.moe_route(ctypes.c_void_p(16), None, 4, 0, 1, 1, 1, 1.0, 1, ctypes.c_void_p(16), ctypes.c_void_p(16), None)
+    assert b"E=0" in lib.nvfp4moe_last_error_string()

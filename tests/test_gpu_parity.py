@@ -1,0 +1,330 @@
+"""GPU parity: every step of the CUDA path against the CPU oracle, through the
+C ABI.  Integer results (transcode codes/scales/globals, routing ids, routing
+weights as bits, quantised codes and scales, permutation) must be bit-exact;
+layer outputs must be within rel-L2 2e-3 and max-abs 1e-2 * rms(out) of the
+float64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_mixture_experts_grouped_b200 as moe
+import oracle
+from nvfp4_mixture_experts_grouped_b200 import inputs
+
+from helpers import (GpuLayer, bf16_tensor, compare_layer, dev, gpu_transcode, host, nvfp4_weights_from_inputs,
+                     oracle_layer, out_to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+# ---------------------------------------------------------------------------
+# transcode
+# ---------------------------------------------------------------------------
+
+def _assert_transcode_equal(codes, e8m0, in_place=False):
+    nt, N, kh = codes.shape
+    rc, re4, rg, rst, rrep, rworst = oracle.transcode(codes, e8m0, nt, N, kh * 2)
+    gc, ge4, gg, gst, grep, gstatus = gpu_transcode(codes, e8m0, in_place=in_place)
+    assert np.array_equal(gst, rst)
+    assert np.array_equal(gc.reshape(-1), rc.reshape(-1))
+    assert np.array_equal(ge4, re4)
+    assert np.array_equal(gg.view(np.uint32), rg.view(np.uint32))
+    assert grep["blocks"] == rrep[0] and grep["zero_blocks"] == rrep[1]
+    assert grep["nonrepresentable_tensors"] == rrep[2] and grep["nan_scale_tensors"] == rrep[3]
+    expect_status = {0: 0, 1: 5, 2: 4}[rworst]
+    assert gstatus == expect_status
+
+
+def test_transcode_tiny_layer_weights():
+    d = inputs.moe_inputs(inputs.WORKLOADS["tiny"])
+    for name in ("gate", "up", "down"):
+        _assert_transcode_equal(*d["mx"][name])
+
+
+@pytest.mark.parametrize("in_place", [False, True])
+def test_transcode_windows_edges_and_failures(in_place):
+    rng = np.random.default_rng(77)
+    nt, N, K = 12, 64, 256
+    lo = rng.integers(-30, 20, nt)
+    w = rng.integers(0, 18, nt)
+    codes, e8 = inputs.mxfp4_tensors(rng, nt, N, K, lo, lo + w)
+    e8[0] = 127 - 120  # extreme but uniform exponents
+    e8[1, 0, 0] = 127 + 17
+    e8[1, 1:] = 127  # spread 17: exact
+    e8[2, 0, 0] = 127 + 18
+    e8[2, 1:] = 127  # spread 18: not representable
+    codes[3] = 0x88  # all blocks +-0
+    e8[4, 5, 3] = 0xFF  # NaN scale on a non-zero block
+    codes[5, 7, 0:16] = 0x80  # one all-zero block whose E8M0 is NaN: ignored
+    e8[5, 7, 0] = 0xFF
+    _assert_transcode_equal(codes, e8, in_place=in_place)
+
+
+def test_transcode_large_tensor_uncached_path():
+    # 2^21+ blocks per tensor: more than the per-CTA shared-memory cache holds
+    rng = np.random.default_rng(5)
+    codes, e8 = inputs.mxfp4_tensors(rng, 1, 8192, 8448, -12, 3)
+    _assert_transcode_equal(codes, e8)
+
+
+def test_transcode_full_layer_sampled():
+    """The full transcode workload (768 expert tensors + the adversarial one) on
+    the GPU; a seeded sample of tensors is checked against the oracle."""
+    rng = np.random.default_rng(inputs.TRANSCODE_SEED)
+    layer = inputs.transcode_layer(rng)
+    gate_c, gate_s = layer["gate"]
+    codes = np.concatenate([gate_c, layer["adversarial"][0]])
+    e8 = np.concatenate([gate_s, layer["adversarial"][1]])
+    gc, ge4, gg, gst, grep, gstatus = gpu_transcode(codes, e8)
+    assert gstatus == 5 and grep["nonrepresentable_tensors"] == 1 and gst[-1] == 1
+    assert np.all(gst[:-1] == 0)
+    pick = sorted(set(np.random.default_rng(1).choice(256, 6, replace=False).tolist()) | {0, 255, 256})
+    for t in pick:
+        rc, re4, rg, rst, _, _ = oracle.transcode(codes[t:t + 1], e8[t:t + 1], 1, 2048, 4096)
+        assert np.array_equal(ge4[t], re4[0]) and gg[t] == rg[0] and gst[t] == rst[0]
+    assert np.array_equal(gc, codes)
+    down_c, down_s = layer["down"]
+    gc2, ge42, gg2, gst2, _, st2 = gpu_transcode(down_c, down_s, in_place=True)
+    assert st2 == 0 and np.all(gst2 == 0)
+    for t in (0, 128, 255):
+        rc, re4, rg, _, _, _ = oracle.transcode(down_c[t:t + 1], down_s[t:t + 1], 1, 4096, 2048)
+        assert np.array_equal(ge42[t], re4[0]) and gg2[t] == rg[0]
+
+
+# ---------------------------------------------------------------------------
+# routing
+# ---------------------------------------------------------------------------
+
+def _gpu_route(logits, bias, ng, tg, k, rsf, renorm=True):
+    T, E = logits.shape
+    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    moe.moe_route(dev(logits), None if bias is None else dev(bias), ng, tg, k, rsf, renorm, ids, w)
+    torch.cuda.synchronize()
+    return host(ids), host(w)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "skewed"])
+def test_route_workloads_bit_exact(name):
+    wl = inputs.WORKLOADS[name]
+    rng = np.random.default_rng(wl.seed)
+    logits = inputs.router_logits(rng, wl.T, wl.E, wl.zipf)
+    gi, gw = _gpu_route(logits, None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf)
+    ri, rw = oracle.route(logits, None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf)
+    assert np.array_equal(gi, ri)
+    assert np.array_equal(gw.view(np.uint32), rw.view(np.uint32))
+
+
+@pytest.mark.parametrize("E,ng,tg,k", [(16, 4, 2, 4), (256, 8, 4, 8), (128, 8, 4, 8), (64, 1, 1, 6), (96, 3, 2, 5),
+                                       (1024, 32, 8, 32), (32, 32, 32, 32), (8, 8, 3, 3)])
+@pytest.mark.parametrize("ties", [False, True])
+def test_route_shapes_ties_bias(E, ng, tg, k, ties):
+    rng = np.random.default_rng(E + ng + k)
+    T = 97
+    if ties:
+        logits = rng.integers(-3, 4, size=(T, E)).astype(np.float32) * 0.5
+        bias = None
+    else:
+        logits = (rng.standard_normal((T, E)) * 3).astype(np.float32)
+        logits[0, :] = 0.0  # every expert ties
+        bias = (rng.standard_normal(E) * 0.05).astype(np.float32)
+    for renorm in (True, False):
+        gi, gw = _gpu_route(logits, bias, ng, tg, k, 2.827, renorm)
+        ri, rw = oracle.route(logits, bias, ng, tg, k, 2.827, renorm)
+        assert np.array_equal(gi, ri)
+        assert np.array_equal(gw.view(np.uint32), rw.view(np.uint32))
+
+
+def test_route_extreme_logits():
+    rng = np.random.default_rng(3)
+    logits = rng.uniform(-120, 120, size=(64, 256)).astype(np.float32)
+    gi, gw = _gpu_route(logits, None, 8, 4, 8, 2.827)
+    ri, rw = oracle.route(logits, None, 8, 4, 8, 2.827)
+    assert np.array_equal(gi, ri) and np.array_equal(gw.view(np.uint32), rw.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# permutation
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,E,k,pad", [(32, 16, 4, 128), (16, 256, 8, 1), (1000, 64, 6, 128), (8192, 256, 8, 128),
+                                       (3, 8, 8, 1), (600, 1024, 32, 1)])
+def test_permute_against_oracle(T, E, k, pad):
+    rng = np.random.default_rng(T + E)
+    ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    poff = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    rop = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    ws = torch.empty(moe.moe_permute_workspace_size(T, E, k, pad), dtype=torch.uint8, device="cuda")
+    assert moe.load().moe_permute(None, 4, E, k, pad, None, None, None, None, 0, None) != 0  # null pointers
+    moe.moe_permute(dev(ids), E, pad, counts, poff, rop, ws)
+    torch.cuda.synchronize()
+    rc, ro, rrop, _ = oracle.permute(ids, E)
+    gc, gpo, grop = host(counts), host(poff), host(rop)
+    assert np.array_equal(gc, rc)
+    padded = ((rc + pad - 1) // pad) * pad
+    assert np.array_equal(gpo, np.concatenate([[0], np.cumsum(padded)]).astype(np.int32))
+    e_of = ids.reshape(-1)
+    assert np.array_equal(grop - gpo[e_of], rrop - ro[e_of])  # identical rank inside each expert
+
+
+# ---------------------------------------------------------------------------
+# quantisation
+# ---------------------------------------------------------------------------
+
+def _gpu_quant(xbits, gs=1.0):
+    M, K = xbits.shape
+    c = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    s = torch.empty((M, K // 16), dtype=torch.uint8, device="cuda")
+    moe.quantize_nvfp4(bf16_tensor(xbits), gs, c, s)
+    torch.cuda.synchronize()
+    return host(c), host(s)
+
+
+@pytest.mark.parametrize("gs", [1.0, 0.375, 3.0])
+def test_quantize_random_and_outliers_bit_exact(gs):
+    rng = np.random.default_rng(int(gs * 8))
+    x = inputs.activations(rng, 257, 4096, outliers=True)
+    gc, gsf = _gpu_quant(x, gs)
+    rc, rs = oracle.quantize_bf16(x, gs)
+    assert np.array_equal(gsf, rs)
+    assert np.array_equal(gc, rc)
+
+
+def test_quantize_ties_signed_zeros_subnormal_scales():
+    blocks = []
+    mags = [0.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 7.0]
+    for s in (1.0, 0.5, 2.0 ** -8, 2.0 ** -10, 448.0, 2 ** -12):  # block scales incl. E4M3 subnormals
+        for sign in (1.0, -1.0):
+            b = np.array(mags, np.float32) * np.float32(s) * sign
+            b[0] = 6.0 * s  # pins the scale
+            blocks.append(b)
+    blocks.append(np.array([-0.0] * 16, np.float32))
+    blocks.append(np.array([1e-30, -1e-30] * 8, np.float32))
+    blocks.append(np.array([3e5, -3e5] + [1.0] * 14, np.float32))
+    x = inputs.bf16_bits(np.concatenate(blocks).reshape(-1, 32))
+    gc, gsf = _gpu_quant(x)
+    rc, rs = oracle.quantize_bf16(x)
+    assert np.array_equal(gsf, rs)
+    assert np.array_equal(gc, rc)
+
+
+def test_quantize_exhaustive_bf16_ratios():
+    # every positive BF16 bit pattern in [2^-12, 2^9), fifteen per block after a 6
+    vals = np.arange(0x3980, 0x4400, dtype=np.uint32)  # bit patterns
+    f = (vals << 16).view(np.float32)
+    n = (len(f) // 15) * 15
+    body = f[:n].reshape(-1, 15)
+    x = np.concatenate([np.full((body.shape[0], 1), 6.0, np.float32), body], axis=1)
+    x = np.concatenate([x, -x], axis=0)
+    xb = inputs.bf16_bits(x.reshape(-1, 32))
+    gc, gsf = _gpu_quant(xb)
+    rc, rs = oracle.quantize_bf16(xb)
+    assert np.array_equal(gsf, rs) and np.array_equal(gc, rc)
+
+
+# ---------------------------------------------------------------------------
+# the layer
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [moe.W4A4, moe.W4A16])
+def test_layer_tiny_all_tokens(mode):
+    wl = inputs.WORKLOADS["tiny"]
+    d = inputs.moe_inputs(wl)
+    w_gpu = nvfp4_weights_from_inputs(d, use_oracle_transcode=False)
+    w_ref = nvfp4_weights_from_inputs(d, use_oracle_transcode=True)
+    for k in w_ref:
+        assert np.array_equal(w_gpu[k].view(np.uint8), w_ref[k].view(np.uint8))
+    layer = GpuLayer(mode, w_gpu, wl.T, wl.n_group, wl.topk_group, wl.top_k)
+    out, ids, wts = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]))
+    ref = oracle_layer(mode, d, w_ref, wl)
+    ri, rw = oracle.route(d["logits"], None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf)
+    assert np.array_equal(host(ids), ri) and np.array_equal(host(wts).view(np.uint32), rw.view(np.uint32))
+    compare_layer(out_to_f64(out), ref)
+    out32, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), out_fp32=True)
+    compare_layer(out_to_f64(out32), ref)
+
+
+def test_layer_decode_w4a16_full():
+    wl = inputs.WORKLOADS["decode"]
+    d = inputs.moe_inputs(wl)
+    w = nvfp4_weights_from_inputs(d, False)
+    layer = GpuLayer(moe.W4A16, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
+    out, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]))
+    ref = oracle_layer(moe.W4A16, d, w, wl)
+    compare_layer(out_to_f64(out), ref)
+
+
+def _sample_tokens(ids: np.ndarray, n: int, seed: int):
+    rng = np.random.default_rng(seed)
+    T = ids.shape[0]
+    heavy = np.bincount(ids.reshape(-1)).argmax()
+    on_heavy = np.where((ids == heavy).any(1))[0]
+    pick = set(rng.choice(T, n, replace=False).tolist()) | set(on_heavy[:2].tolist()) | {0, T - 1}
+    return np.array(sorted(pick), np.int32)
+
+
+@pytest.mark.parametrize("name", ["prefill", "skewed"])
+def test_layer_w4a4_full_size_sampled(name):
+    wl = inputs.WORKLOADS[name]
+    d = inputs.moe_inputs(wl)
+    w = nvfp4_weights_from_inputs(d, False)
+    layer = GpuLayer(wl.mode, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
+    out, ids, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]))
+    toks = _sample_tokens(host(ids), 12, wl.seed)
+    ref = oracle_layer(wl.mode, d, w, wl, tokens=toks)
+    compare_layer(out_to_f64(out)[toks], ref)
+    # also the W4A16 path on a decode-sized slice of the same weights
+    del layer
+    torch.cuda.empty_cache()
+
+
+def test_layer_edge_cases():
+    wl = inputs.WORKLOADS["tiny"]
+    d = inputs.moe_inputs(wl)
+    w = nvfp4_weights_from_inputs(d, False)
+    for mode in (moe.W4A4, moe.W4A16):
+        layer = GpuLayer(mode, w, 1, wl.n_group, wl.topk_group, wl.top_k)
+        # T = 1
+        out, _, _ = layer.forward(bf16_tensor(d["x"][:1]), dev(d["logits"][:1]))
+        compare_layer(out_to_f64(out), oracle_layer(mode, {"x": d["x"][:1], "logits": d["logits"][:1]}, w, wl))
+        # every token routed to the same experts (one expert gets > 2 M-tiles of rows)
+        T = 300
+        rng = np.random.default_rng(9)
+        x = inputs.activations(rng, T, wl.H)
+        lg = np.full((T, wl.E), -8.0, np.float32)
+        lg[:, [0, 1, 2, 3]] = 8.0
+        lg += rng.standard_normal((T, wl.E)).astype(np.float32) * 0.01
+        out, ids, _ = layer.forward(bf16_tensor(x), dev(lg))
+        assert set(np.unique(host(ids)).tolist()) == {0, 1, 2, 3}
+        ref = oracle_layer(mode, {"x": x, "logits": lg}, w, wl)
+        compare_layer(out_to_f64(out), ref)
+        # T = 0 is a no-op
+        empty = torch.empty((0, wl.H), dtype=torch.bfloat16, device="cuda")
+        moe.moe_forward(mode, empty, torch.empty((0, wl.E), device="cuda"), None, layer.packed, 1.0, 0, wl.H, wl.I,
+                        wl.E, wl.n_group, wl.topk_group, wl.top_k, wl.rsf, True, layer.ws, empty)
+
+
+def test_layer_deterministic_and_routed_entry_point():
+    wl = inputs.WORKLOADS["tiny"]
+    d = inputs.moe_inputs(wl, T=200)
+    w = nvfp4_weights_from_inputs(d, False)
+    layer = GpuLayer(moe.W4A4, w, 200, wl.n_group, wl.topk_group, wl.top_k)
+    x, lg = bf16_tensor(d["x"]), dev(d["logits"])
+    a, ids, wts = layer.forward(x, lg)
+    b, _, _ = layer.forward(x, lg)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    out = torch.empty_like(a)
+    moe.moe_forward_routed(moe.W4A4, x, ids, wts, layer.packed, 1.0, 200, wl.H, wl.I, wl.E, wl.top_k, layer.ws, out)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), a.view(torch.int16))
+
+
+def test_layer_non_unit_activation_global():
+    wl = inputs.WORKLOADS["tiny"]
+    d = inputs.moe_inputs(wl)
+    w = nvfp4_weights_from_inputs(d, False)
+    layer = GpuLayer(moe.W4A4, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
+    out, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), act_global=0.25)
+    ref = oracle_layer(moe.W4A4, d, w, wl, act_global=0.25)
+    compare_layer(out_to_f64(out), ref)
