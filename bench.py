@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-extras", action="store_true", help="skip the decode and transcode sub-measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=0, help="oracle tokens per step (0 = host threads)")
+    ap.add_argument("--tokens", type=int, default=0, help="override T (smaller cases for profiling)")
+    ap.add_argument("--experts", type=int, default=0, help="override E (smaller cases for profiling)")
     return ap.parse_args()
 
 
@@ -98,6 +100,17 @@ class ClockSampler:
         reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and "Active" in r[5 + i]})
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(rows)}
+
+
+def workload(args):
+    import dataclasses
+
+    wl = inputs.WORKLOADS[args.workload]
+    if args.tokens:
+        wl = dataclasses.replace(wl, T=args.tokens)
+    if args.experts:
+        wl = dataclasses.replace(wl, E=args.experts)
+    return wl
 
 
 def layer_flops(T, H, I, k):
@@ -171,7 +184,7 @@ def run_ours(args, rank, world, local_rank):
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
     P = peaks()
-    wl = inputs.WORKLOADS[args.workload]
+    wl = workload(args)
     T = wl.T
     d = inputs.moe_inputs(wl)
     w = {k: d[k] for k in ("gate_codes", "gate_sf", "up_codes", "up_sf", "down_codes", "down_sf", "w_global")}
@@ -251,7 +264,8 @@ def run_ours(args, rank, world, local_rank):
                                f"keep={wl.topk_group} top_k={wl.top_k} rsf={wl.rsf} "
                                f"{'W4A4' if mode == moe.W4A4 else 'W4A16'}",
                    "global_batch": T * world, "tokens_per_gpu": T, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (3.6 GB packed expert weights per step)"},
+                   "l2": f"inputs larger than L2 ({moe.moe_packed_weights_size(mode, wl.E, wl.H, wl.I) / 1e9:.2f} GB "
+                         f"packed expert weights per step)"},
         "roofline": roofline,
         "stages_ms": {k: round(v, 4) for k, v in stage.items()},
         "e2e": {"value": round(T * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
@@ -279,7 +293,6 @@ def run_ours(args, rank, world, local_rank):
 def bench_decode(torch, moe, w, args, P):
     """W4A16 decode layer (T=16): tokens/s and weight-stream HBM GB/s."""
     wl = inputs.WORKLOADS["decode"]
-    d = inputs.moe_inputs(wl) if False else None  # weights: same recipe as the prefill layer, reused
     rng = np.random.default_rng(wl.seed)
     x = inputs.activations(rng, wl.T, wl.H)
     lg = inputs.router_logits(rng, wl.T, wl.E)
@@ -380,7 +393,7 @@ def cpu_baseline(wl, d, args, steps=1):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    wl = inputs.WORKLOADS[args.workload]
+    wl = workload(args)
     d = inputs.moe_inputs(wl)
     import oracle
 

@@ -93,7 +93,7 @@ struct ForwardLayout {
     // byte offsets
     int64_t ids, wts, chunk_counts, counts, offsets, pad_offsets, row_of_pair, pair_of_row, tiles, n_tiles, active,
         n_active;
-    int64_t a1c, a1s, a2c, a2s, a2bf, y;
+    int64_t a1c, a1s, a2c, a2s, a2bf, y, ys;
     int64_t total;
 };
 
@@ -131,11 +131,13 @@ static ForwardLayout forward_layout(nvfp4moe_mode mode, int64_t T, int64_t H, in
         L.a2c = take(L.rows_max * I / 2);
         L.a2s = take(L.rows_max * I / 16);
         L.a2bf = -1;
+        L.y = take(L.rows_max * H * 2);          // FP16 staged rows
+        L.ys = take(L.rows_max * (H / 256) * 4);  // their power-of-two scales
     } else {
-        L.a1c = L.a1s = L.a2c = L.a2s = -1;
+        L.a1c = L.a1s = L.a2c = L.a2s = L.ys = -1;
         L.a2bf = take(L.rows_max * I * 2);
+        L.y = take(L.rows_max * H * 4);  // FP32 staged rows
     }
-    L.y = take(L.rows_max * H * 2);
     L.total = o;
     return L;
 }
@@ -371,21 +373,23 @@ static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, con
     trace(1, st);
     RETURN_IF(launch_permute(plan.ids, T, top_k, E, L.pad, plan, st));
     trace(2, st);
-    uint16_t* Y = reinterpret_cast<uint16_t*>(ws + L.y);
+    void* Y = ws + L.y;
+    float* ys = mode == NVFP4MOE_W4A4 ? reinterpret_cast<float*>(ws + L.ys) : nullptr;
     if (mode == NVFP4MOE_W4A4) {
         uint8_t* a1c = ws + L.a1c;
         uint8_t* a1s = ws + L.a1s;
         RETURN_IF(launch_quantize_scatter(x, T, H, act_global, a1c, a1s, plan.row_of_pair, top_k, st));
         trace(3, st);
         RETURN_IF(launch_w4a4_layer(packed, T, H, I, E, top_k, act_global, L.rows_max, (int)L.max_tiles, plan, a1c,
-                                    a1s, ws + L.a2c, ws + L.a2s, Y, st, g_trace_on ? g_trace[4] : nullptr));
+                                    a1s, ws + L.a2c, ws + L.a2s, static_cast<__half*>(Y), ys, st,
+                                    g_trace_on ? g_trace[4] : nullptr));
     } else {
         trace(3, st);
-        RETURN_IF(launch_w4a16_layer(x, packed, T, H, I, E, top_k, plan, reinterpret_cast<uint16_t*>(ws + L.a2bf), Y,
-                                     st, g_trace_on ? g_trace[4] : nullptr));
+        RETURN_IF(launch_w4a16_layer(x, packed, T, H, I, E, top_k, plan, reinterpret_cast<uint16_t*>(ws + L.a2bf),
+                                     static_cast<float*>(Y), st, g_trace_on ? g_trace[4] : nullptr));
     }
     trace(5, st);
-    RETURN_IF(launch_combine(Y, plan.row_of_pair, T, H, top_k, out, out_is_fp32 != 0, st));
+    RETURN_IF(launch_combine(Y, ys, plan.row_of_pair, T, H, top_k, out, out_is_fp32 != 0, st));
     trace(6, st);
     if (ids_out) NVFP4MOE_CUDA(cudaMemcpyAsync(ids_out, plan.ids, (size_t)L.P * 4, cudaMemcpyDeviceToDevice, st));
     if (wts_out) NVFP4MOE_CUDA(cudaMemcpyAsync(wts_out, plan.wts, (size_t)L.P * 4, cudaMemcpyDeviceToDevice, st));

@@ -1,6 +1,7 @@
 // moe_internal.cuh -- declarations shared by the kernels and the C-ABI layer.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -48,14 +49,16 @@ nvfp4moe_status launch_quantize_linear(const uint16_t* x, int64_t M, int64_t K, 
                                        uint8_t* scales, cudaStream_t stream);
 nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H, float gs, uint8_t* codes,
                                         uint8_t* scales, const int32_t* row_of_pair, int k, cudaStream_t stream);
-nvfp4moe_status launch_combine(const uint16_t* Y, const int32_t* row_of_pair, int64_t T, int H, int k, void* out,
-                               bool out_f32, cudaStream_t stream);
+// Y staged as FP16 rows with a power-of-two scale per 256 columns (y_scale != nullptr,
+// W4A4) or as FP32 rows (y_scale == nullptr, W4A16).
+nvfp4moe_status launch_combine(const void* Y, const float* y_scale, const int32_t* row_of_pair, int64_t T, int H,
+                               int k, void* out, bool out_f32, cudaStream_t stream);
 
 // w4a16.cu
 size_t w4a16_packed_size(int E, int H, int I);
 nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream);
 nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T, int H, int I, int E, int k,
-                                   const RoutingPlan& plan, uint16_t* A2, uint16_t* Y, cudaStream_t stream,
+                                   const RoutingPlan& plan, uint16_t* A2, float* Y, cudaStream_t stream,
                                    cudaEvent_t mid_event);
 
 // w4a4.cu
@@ -63,7 +66,7 @@ size_t w4a4_packed_size(int E, int H, int I);
 nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream);
 nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E, int k, float act_global,
                                   int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
-                                  const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, uint16_t* Y, cudaStream_t stream,
-                                  cudaEvent_t mid_event);
+                                  const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, __half* Y, float* y_scale,
+                                  cudaStream_t stream, cudaEvent_t mid_event);
 
 }  // namespace nvfp4moe

@@ -214,13 +214,14 @@ nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H,
 }
 
 // ---------------------------------------------------------------------------
-// 5. weighted un-permute: out[t] = sum_j Y[row_of_pair(t, j)] (weights already
-//    applied by the down GEMM), FP32 in slot order, one rounding.
+// 5. weighted un-permute: out[t] = sum_j Y[row_of_pair(t, j)] (routing weights
+//    already applied by the down GEMM), FP32 in slot order, one rounding.
+//    Y is FP16 with a power-of-two scale per 256 columns (W4A4) or FP32 (W4A16).
 // ---------------------------------------------------------------------------
-template <bool OUT_F32>
+template <bool Y_F16, bool OUT_F32>
 __global__ void __launch_bounds__(256)
-    k_combine(const uint16_t* __restrict__ Y, const int32_t* __restrict__ row_of_pair, int64_t T, int H, int k,
-              void* __restrict__ out) {
+    k_combine(const void* __restrict__ Yv, const float* __restrict__ y_scale, const int32_t* __restrict__ row_of_pair,
+              int64_t T, int H, int k, void* __restrict__ out) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // one 8-element vector
     const int64_t per_row = H / 8;
     if (i >= T * per_row) return;
@@ -231,12 +232,22 @@ __global__ void __launch_bounds__(256)
     for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
     for (int j = 0; j < k; ++j) {
         const int64_t row = __ldg(row_of_pair + t * k + j);
-        const uint4 v = __ldcs(reinterpret_cast<const uint4*>(Y + row * H + h8));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        if (Y_F16) {
+            const float s = __ldg(y_scale + row * (H / 256) + h8 / 256);
+            const uint4 v = __ldcs(reinterpret_cast<const uint4*>(static_cast<const __half*>(Yv) + row * H + h8));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            acc[2 * q] = __fadd_rn(acc[2 * q], bf16_bits_to_float(w[q] & 0xFFFFu));
-            acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16_bits_to_float(w[q] >> 16));
+            for (int q = 0; q < 4; ++q) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[q]));
+                acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(f.x, s));
+                acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(f.y, s));
+            }
+        } else {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(Yv) + row * H + h8);
+            const float4 a = __ldcs(src), b = __ldcs(src + 1);
+            const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = __fadd_rn(acc[q], f[q]);
         }
     }
     if (OUT_F32) {
@@ -254,15 +265,22 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-nvfp4moe_status launch_combine(const uint16_t* Y, const int32_t* row_of_pair, int64_t T, int H, int k, void* out,
-                               bool out_f32, cudaStream_t stream) {
+nvfp4moe_status launch_combine(const void* Y, const float* y_scale, const int32_t* row_of_pair, int64_t T, int H,
+                               int k, void* out, bool out_f32, cudaStream_t stream) {
     if (T == 0) return NVFP4MOE_OK;
     const int64_t n = T * (H / 8);
     const unsigned grid = (unsigned)ceil_div(n, 256);
-    if (out_f32)
-        k_combine<true><<<grid, 256, 0, stream>>>(Y, row_of_pair, T, H, k, out);
-    else
-        k_combine<false><<<grid, 256, 0, stream>>>(Y, row_of_pair, T, H, k, out);
+    if (y_scale) {
+        if (out_f32)
+            k_combine<true, true><<<grid, 256, 0, stream>>>(Y, y_scale, row_of_pair, T, H, k, out);
+        else
+            k_combine<true, false><<<grid, 256, 0, stream>>>(Y, y_scale, row_of_pair, T, H, k, out);
+    } else {
+        if (out_f32)
+            k_combine<false, true><<<grid, 256, 0, stream>>>(Y, y_scale, row_of_pair, T, H, k, out);
+        else
+            k_combine<false, false><<<grid, 256, 0, stream>>>(Y, y_scale, row_of_pair, T, H, k, out);
+    }
     NVFP4MOE_CHECK_LAUNCH("combine kernel");
     return NVFP4MOE_OK;
 }

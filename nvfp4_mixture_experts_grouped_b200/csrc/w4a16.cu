@@ -22,6 +22,7 @@
 //   * the FP32 accumulator is multiplied by 2^8 * global in the epilogue.
 // Gate and up rows of the same 16 intermediates are streamed by the same warp,
 // so SwiGLU is applied on the accumulators and only BF16 SwiGLU rows are stored.
+// The down GEMM stages its weighted per-pair rows in FP32 (a few MB at decode).
 #include <algorithm>
 
 #include "common.cuh"
@@ -290,7 +291,7 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(W16_WARPS * 32)
     k_w16_down(const uint8_t* __restrict__ packed, W16Layout L, int H, int I, RoutingPlan plan,
-               const uint16_t* __restrict__ A2, uint16_t* __restrict__ Y) {
+               const uint16_t* __restrict__ A2, float* __restrict__ Y) {
     const int lane = lane_id();
     const int g = lane >> 2, c = lane & 3;
     const int hblocks = H / 32;
@@ -334,10 +335,8 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
 #pragma unroll
                     for (int u = 0; u < 2; ++u)
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const __nv_bfloat16 v = __float2bfloat16_rn(acc[u][nt][2 * h + j] * w);
-                            Y[(int64_t)row * H + hb * 32 + u * 16 + g + 8 * h] = *reinterpret_cast<const uint16_t*>(&v);
-                        }
+                        for (int h = 0; h < 2; ++h)
+                            Y[(int64_t)row * H + hb * 32 + u * 16 + g + 8 * h] = acc[u][nt][2 * h + j] * w;
                 }
             }
         }
@@ -374,7 +373,7 @@ nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed
 }
 
 nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T, int H, int I, int E, int k,
-                                   const RoutingPlan& plan, uint16_t* A2, uint16_t* Y, cudaStream_t stream,
+                                   const RoutingPlan& plan, uint16_t* A2, float* Y, cudaStream_t stream,
                                    cudaEvent_t mid_event) {
     const W16Layout L = w16_layout(E, H, I);
     const uint8_t* p = static_cast<const uint8_t*>(packed);

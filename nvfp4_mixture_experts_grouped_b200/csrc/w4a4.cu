@@ -17,7 +17,8 @@
 //               gate/up: SiLU(gate) * up and NVFP4 requantisation per 16 (the
 //                        down GEMM's A operand, written straight into its
 //                        block-scale layout);
-//               down:    x global scale x routing weight, BF16 per-pair rows.
+//               down:    x global scale x routing weight, per-pair rows staged
+//                        as FP16 with a power-of-two scale per 256 columns.
 // Rows of an expert are padded to 128 by the permutation, so an M-tile never
 // straddles two experts; padding rows are computed and never stored.
 #include <cuda.h>
@@ -80,7 +81,8 @@ struct GemmParams {
     uint8_t* out_codes;      // gate/up: intermediate codes [rows, I/2]
     uint8_t* out_sf;         // gate/up: intermediate scales, atom layout
     int out_k;               // gate/up: I
-    uint16_t* Y;             // down: [rows, H] BF16
+    __half* Y;               // down: [rows, H] FP16 staged rows
+    float* y_scale;          // down: [rows, H / 256] power-of-two scale of each staged row tile
     int ldy;                 // down: H
     const float* wts;        // down: routing weight of each pair
     const int32_t* pair_of_row;
@@ -221,8 +223,25 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
             } else {
+                // y = acc * global * routing weight, staged as FP16 with one power-of-two
+                // scale per (row, 256-column tile): pass 1 finds the row's max, pass 2
+                // writes y / scale (exact scaling, then one FP16 rounding).
                 const float f = valid ? p.globals[ti.x * 3 + 2] * p.act_global * p.wts[p.pair_of_row[row]] : 0.0f;
-                uint16_t* yrow = p.Y + row * p.ldy + (int64_t)n * BN;
+                float amax = 0.0f;
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    float v0[16], v1[16];
+                    tc::tmem_ld16x2(t_row + 32 * c, t_row + 32 * c + 16, v0, v1);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fmaxf(fabsf(v0[i]), fabsf(v1[i])));
+                }
+                amax *= fabsf(f);
+                // scale = 2^(e - 14) with amax in [2^e, 2^(e+1)): staged magnitudes stay below 2^15
+                int e = 0;
+                if (amax > 0.0f && isfinite(amax)) e = ((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+                e = max(min(e - 14, 100), -100);
+                const float g = ldexpf(f, -e);
+                __half* yrow = p.Y + row * p.ldy + (int64_t)n * BN;
 #pragma unroll 1
                 for (int c = 0; c < 8; ++c) {
                     float v0[16], v1[16];
@@ -231,8 +250,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                         uint32_t pk[16];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            __nv_bfloat162 b0 = __floats2bfloat162_rn(v0[2 * i] * f, v0[2 * i + 1] * f);
-                            __nv_bfloat162 b1 = __floats2bfloat162_rn(v1[2 * i] * f, v1[2 * i + 1] * f);
+                            __half2 b0 = __floats2half2_rn(v0[2 * i] * g, v0[2 * i + 1] * g);
+                            __half2 b1 = __floats2half2_rn(v1[2 * i] * g, v1[2 * i + 1] * g);
                             pk[i] = *reinterpret_cast<uint32_t*>(&b0);
                             pk[8 + i] = *reinterpret_cast<uint32_t*>(&b1);
                         }
@@ -241,6 +260,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                     }
                 }
+                if (valid) p.y_scale[row * p.n_ntiles + n] = ldexpf(1.0f, e);
             }
             tc::tc_fence_before();
             __syncwarp();
@@ -359,8 +379,8 @@ nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed,
 
 nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E, int k, float act_global,
                                   int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
-                                  const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, uint16_t* Y, cudaStream_t stream,
-                                  cudaEvent_t mid_event) {
+                                  const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, __half* Y, float* y_scale,
+                                  cudaStream_t stream, cudaEvent_t mid_event) {
     (void)T;
     (void)k;
     const W4Layout L = w4_layout(E, H, I);
@@ -403,6 +423,7 @@ nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E
     g.sfa = A2s;
     g.sfb = pk + L.d_sf;
     g.Y = Y;
+    g.y_scale = y_scale;
     g.ldy = H;
     {
         const int grid = (int)std::min<int64_t>(sms, (int64_t)max_tiles * g.n_ntiles);

@@ -202,7 +202,7 @@ def test_quantize_ties_signed_zeros_subnormal_scales():
     blocks.append(np.array([-0.0] * 16, np.float32))
     blocks.append(np.array([1e-30, -1e-30] * 8, np.float32))
     blocks.append(np.array([3e5, -3e5] + [1.0] * 14, np.float32))
-    x = inputs.bf16_bits(np.concatenate(blocks).reshape(-1, 32))
+    x = inputs.bf16_bits(np.concatenate(blocks).reshape(-1, 16))
     gc, gsf = _gpu_quant(x)
     rc, rs = oracle.quantize_bf16(x)
     assert np.array_equal(gsf, rs)
