@@ -18,7 +18,7 @@
 //                        down GEMM's A operand, written straight into its
 //                        block-scale layout);
 //               down:    x global scale x routing weight, per-pair rows staged
-//                        as FP16 with a power-of-two scale per 256 columns.
+//                        as FP16 with a power-of-two scale per 128 columns.
 // Rows of an expert are padded to 128 by the permutation, so an M-tile never
 // straddles two experts; padding rows are computed and never stored.
 #include <cuda.h>
@@ -47,7 +47,8 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_SF = 256;      // scale-factor columns after the 256 accumulator columns
 constexpr uint32_t TM_SF_STRIDE = 48;  // per buffer: 16 (A: 4 k-steps x 4) + 32 (B: 4 x 8)
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;  // two warps per TMEM lane quadrant, each on half the columns
+constexpr int THREADS = 64 + EPI_WARPS * 32;
 
 enum { EPI_GATEUP = 0, EPI_DOWN = 1 };
 
@@ -82,14 +83,34 @@ struct GemmParams {
     uint8_t* out_sf;         // gate/up: intermediate scales, atom layout
     int out_k;               // gate/up: I
     __half* Y;               // down: [rows, H] FP16 staged rows
-    float* y_scale;          // down: [rows, H / 256] power-of-two scale of each staged row tile
+    float* y_scale;          // down: [rows, H / 128] power-of-two scale of each 128 staged columns
     int ldy;                 // down: H
     const float* wts;        // down: routing weight of each pair
     const int32_t* pair_of_row;
     int32_t* err;
 };
 
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+// SiLU with the hardware exp2 and a fast divide (the layer is checked against the
+// float64 oracle with a tolerance; these are not bit-exact steps).
+__device__ __forceinline__ float silu_fast(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
+// NVFP4 requantisation of 16 SwiGLU outputs held by one thread: the block scale
+// is decided exactly as the standalone quantiser does ((amax / 6) / gs with IEEE
+// divisions, E4M3 round-to-nearest-even), the codes use x * (1 / (value(sf) * gs)).
+__device__ __forceinline__ uint32_t requant_block16(const float* x, float gs, uint32_t& w0, uint32_t& w1) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    const uint32_t sf = f32x2_to_e4m3x2(__fdiv_rn(__fdiv_rn(amax, 6.0f), gs), 0.0f) & 0xFFu;
+    const float sfv = e4m3_to_float(sf);
+    const float r = sfv != 0.0f ? __frcp_rn(sfv * gs) : 0.0f;
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = x[i] * r;
+    w0 = f32x8_to_e2m1x8(q);
+    w1 = f32x8_to_e2m1x8(q + 8);
+    return sf;
+}
 
 template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -109,7 +130,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::mbar_init(&empty[s], 1);
         }
         tc::mbar_init(acc_full, 1);
-        tc::mbar_init(acc_empty, 4);
+        tc::mbar_init(acc_empty, EPI_WARPS);
         tc::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -191,7 +212,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        // warps 2..9: warp w reads TMEM lane quadrant w % 4 (the hardware rule) and
+        // column half (w - 2) / 4 of the tile.
+        const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int r_in = q * 32 + lane;
         const uint32_t t_row = tmem + ((uint32_t)(q * 32) << 16);
         int tl = 0;
@@ -203,35 +227,43 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!tc::mbar_wait(acc_full, (uint32_t)tl & 1u, p.err)) goto done;
             tc::tc_fence_after();
             if (EPI == EPI_GATEUP) {
+                // columns [0,128) gate, [128,256) up, for intermediates n*128 .. n*128+127
                 const float ag = p.globals[ti.x * 3 + 0] * p.act_global;
                 const float au = p.globals[ti.x * 3 + 1] * p.act_global;
-                const int i0 = n * (BN / 2);
+                const int i0 = n * (BN / 2) + half * 64;  // first intermediate of this warp
                 const int nkb = p.out_k / 16;
-#pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
-                    float gv[16], uv[16];
-                    tc::tmem_ld16x2(t_row + 16 * c, t_row + 128 + 16 * c, gv, uv);
-                    if (valid) {
-                        float a[16];
+                uint32_t codes[8], sfw = 0;
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) a[i] = silu(gv[i] * ag) * (uv[i] * au);
-                        uint32_t w0, w1;
-                        const uint32_t sf = quantize_block16(a, p.act_global, w0, w1);
-                        const int col = i0 + 16 * c;
-                        *reinterpret_cast<uint2*>(p.out_codes + row * (p.out_k / 2) + col / 2) = make_uint2(w0, w1);
-                        p.out_sf[sf_atom_offset(row, col / 16, nkb)] = (uint8_t)sf;
-                    }
+                for (int c = 0; c < 4; ++c) {
+                    float gv[16], uv[16];
+                    tc::tmem_ld16x2(t_row + half * 64 + 16 * c, t_row + 128 + half * 64 + 16 * c, gv, uv);
+                    float a[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) a[i] = silu_fast(gv[i] * ag) * (uv[i] * au);
+                    const uint32_t sf = requant_block16(a, p.act_global, codes[2 * c], codes[2 * c + 1]);
+                    sfw |= sf << (8 * c);
+                }
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(acc_empty);  // accumulator drained by this warp
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(p.out_codes + row * (p.out_k / 2) + i0 / 2);
+                    dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                    dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+                    // the 4 block scales of this row are 4 consecutive bytes of one atom row
+                    *reinterpret_cast<uint32_t*>(p.out_sf + sf_atom_offset(row, i0 / 16, nkb)) = sfw;
                 }
             } else {
                 // y = acc * global * routing weight, staged as FP16 with one power-of-two
-                // scale per (row, 256-column tile): pass 1 finds the row's max, pass 2
-                // writes y / scale (exact scaling, then one FP16 rounding).
+                // scale per (row, 128 columns): pass 1 finds the max, pass 2 writes
+                // y / scale (exact power-of-two scaling, then one FP16 rounding).
                 const float f = valid ? p.globals[ti.x * 3 + 2] * p.act_global * p.wts[p.pair_of_row[row]] : 0.0f;
+                const uint32_t t_col = t_row + half * 128;
                 float amax = 0.0f;
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 4; ++c) {
                     float v0[16], v1[16];
-                    tc::tmem_ld16x2(t_row + 32 * c, t_row + 32 * c + 16, v0, v1);
+                    tc::tmem_ld16x2(t_col + 32 * c, t_col + 32 * c + 16, v0, v1);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fmaxf(fabsf(v0[i]), fabsf(v1[i])));
                 }
@@ -241,11 +273,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (amax > 0.0f && isfinite(amax)) e = ((__float_as_uint(amax) >> 23) & 0xFF) - 127;
                 e = max(min(e - 14, 100), -100);
                 const float g = ldexpf(f, -e);
-                __half* yrow = p.Y + row * p.ldy + (int64_t)n * BN;
+                __half* yrow = p.Y + row * p.ldy + (int64_t)n * BN + half * 128;
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 4; ++c) {
                     float v0[16], v1[16];
-                    tc::tmem_ld16x2(t_row + 32 * c, t_row + 32 * c + 16, v0, v1);
+                    tc::tmem_ld16x2(t_col + 32 * c, t_col + 32 * c + 16, v0, v1);
+                    if (c == 3) {
+                        tc::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(acc_empty);
+                    }
                     if (valid) {
                         uint32_t pk[16];
 #pragma unroll
@@ -260,11 +297,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                         for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                     }
                 }
-                if (valid) p.y_scale[row * p.n_ntiles + n] = ldexpf(1.0f, e);
+                if (valid) p.y_scale[row * (p.ldy / 128) + n * 2 + half] = ldexpf(1.0f, e);
             }
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(acc_empty);
         }
     }
 done:

@@ -240,7 +240,7 @@ def test_layer_tiny_all_tokens(mode):
     ref = oracle_layer(mode, d, w_ref, wl)
     ri, rw = oracle.route(d["logits"], None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf)
     assert np.array_equal(host(ids), ri) and np.array_equal(host(wts).view(np.uint32), rw.view(np.uint32))
-    compare_layer(out_to_f64(out), ref)
+    compare_layer(out_to_f64(out), ref, bf16_output=True)
     out32, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), out_fp32=True)
     compare_layer(out_to_f64(out32), ref)
 
@@ -250,9 +250,11 @@ def test_layer_decode_w4a16_full():
     d = inputs.moe_inputs(wl)
     w = nvfp4_weights_from_inputs(d, False)
     layer = GpuLayer(moe.W4A16, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
-    out, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]))
+    out, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), out_fp32=True)
     ref = oracle_layer(moe.W4A16, d, w, wl)
     compare_layer(out_to_f64(out), ref)
+    out16, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]))
+    compare_layer(out_to_f64(out16), ref, bf16_output=True)
 
 
 def _sample_tokens(ids: np.ndarray, n: int, seed: int):
@@ -270,10 +272,12 @@ def test_layer_w4a4_full_size_sampled(name):
     d = inputs.moe_inputs(wl)
     w = nvfp4_weights_from_inputs(d, False)
     layer = GpuLayer(wl.mode, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
-    out, ids, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]))
+    out, ids, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), out_fp32=True)
     toks = _sample_tokens(host(ids), 12, wl.seed)
     ref = oracle_layer(wl.mode, d, w, wl, tokens=toks)
     compare_layer(out_to_f64(out)[toks], ref)
+    out16, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]))
+    compare_layer(out_to_f64(out16)[toks], ref, bf16_output=True)
     # also the W4A16 path on a decode-sized slice of the same weights
     del layer
     torch.cuda.empty_cache()
@@ -286,7 +290,7 @@ def test_layer_edge_cases():
     for mode in (moe.W4A4, moe.W4A16):
         layer = GpuLayer(mode, w, 1, wl.n_group, wl.topk_group, wl.top_k)
         # T = 1
-        out, _, _ = layer.forward(bf16_tensor(d["x"][:1]), dev(d["logits"][:1]))
+        out, _, _ = layer.forward(bf16_tensor(d["x"][:1]), dev(d["logits"][:1]), out_fp32=True)
         compare_layer(out_to_f64(out), oracle_layer(mode, {"x": d["x"][:1], "logits": d["logits"][:1]}, w, wl))
         # every token routed to the same experts (one expert gets > 2 M-tiles of rows)
         T = 300
@@ -295,7 +299,7 @@ def test_layer_edge_cases():
         lg = np.full((T, wl.E), -8.0, np.float32)
         lg[:, [0, 1, 2, 3]] = 8.0
         lg += rng.standard_normal((T, wl.E)).astype(np.float32) * 0.01
-        out, ids, _ = layer.forward(bf16_tensor(x), dev(lg))
+        out, ids, _ = layer.forward(bf16_tensor(x), dev(lg), out_fp32=True)
         assert set(np.unique(host(ids)).tolist()) == {0, 1, 2, 3}
         ref = oracle_layer(mode, {"x": x, "logits": lg}, w, wl)
         compare_layer(out_to_f64(out), ref)
@@ -325,6 +329,6 @@ def test_layer_non_unit_activation_global():
     d = inputs.moe_inputs(wl)
     w = nvfp4_weights_from_inputs(d, False)
     layer = GpuLayer(moe.W4A4, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
-    out, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), act_global=0.25)
+    out, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), act_global=0.25, out_fp32=True)
     ref = oracle_layer(moe.W4A4, d, w, wl, act_global=0.25)
     compare_layer(out_to_f64(out), ref)
