@@ -28,6 +28,7 @@
 #include "common.cuh"
 #include "formats.cuh"
 #include "moe_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace nvfp4moe {
 
@@ -176,109 +177,167 @@ __device__ __forceinline__ void mma_bf16(float d[4], const uint32_t a[4], uint32
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
 // ---------------------------------------------------------------------------
-// gate/up GEMM + SwiGLU: one warp per (active expert, 16 intermediates)
+// Weight streaming: every warp owns a ring of W16_STAGES shared-memory stages;
+// lane 0 fills a stage with 1-D bulk copies (cp.async.bulk, completion counted
+// on the stage's mbarrier) W16_STAGES groups ahead of the consumer, so each SM
+// keeps ~200 KB of the weight stream in flight without holding it in registers.
+// A stage holds W16_CH consecutive 64-column chunks of both 16-row tiles.
 // ---------------------------------------------------------------------------
-template <int NTILE_TILES>
-__device__ __forceinline__ void w16_stream(const uint4* __restrict__ codes[NTILE_TILES],
-                                           const uint2* __restrict__ scales[NTILE_TILES], int chunks,
-                                           const uint16_t* const bptr[W16_MAX_NT], int nt_count, int c,
-                                           float acc[NTILE_TILES][W16_MAX_NT][4]) {
-    uint4 qn[NTILE_TILES];
-    uint2 sn[NTILE_TILES];
+constexpr int W16_STAGES = 4;
+constexpr int W16_CH = 4;
+constexpr int W16_STAGE_CODES = 2 * W16_CH * 512;
+constexpr int W16_STAGE_SCALES = 2 * W16_CH * 64;
+constexpr int W16_STAGE = W16_STAGE_CODES + W16_STAGE_SCALES;
+constexpr int W16_WARP_SMEM = W16_STAGES * W16_STAGE;
+constexpr int W16_SMEM = W16_WARPS * (W16_WARP_SMEM + W16_STAGES * 8);
+
+struct Ring {
+    uint8_t* buf;   // W16_STAGES stages
+    uint64_t* bar;  // W16_STAGES mbarriers
+    uint32_t ctr;   // groups consumed so far (stage = ctr % S, parity = ctr / S)
+};
+
+__device__ __forceinline__ void ring_issue(Ring& r, int stage, const uint8_t* const codes[2],
+                                           const uint8_t* const scales[2], int grp, int ch) {
+    uint8_t* st = r.buf + stage * W16_STAGE;
+    tc::mbar_arrive_expect_tx(&r.bar[stage], 2 * ch * (512 + 64));
 #pragma unroll
-    for (int u = 0; u < NTILE_TILES; ++u) {
-        qn[u] = __ldcs(codes[u]);
-        sn[u] = __ldcs(scales[u]);
-    }
-    for (int ch = 0; ch < chunks; ++ch) {
-        uint4 q[NTILE_TILES];
-        uint2 sc[NTILE_TILES];
-#pragma unroll
-        for (int u = 0; u < NTILE_TILES; ++u) {
-            q[u] = qn[u];
-            sc[u] = sn[u];
-        }
-        if (ch + 1 < chunks) {
-#pragma unroll
-            for (int u = 0; u < NTILE_TILES; ++u) {
-                qn[u] = __ldcs(codes[u] + (ch + 1) * 32);
-                sn[u] = __ldcs(scales[u] + (ch + 1) * 8);
-            }
-        }
-#pragma unroll
-        for (int st = 0; st < 4; ++st) {
-            const int kb = ch * 64 + st * 16;
-            uint32_t b0[W16_MAX_NT], b1[W16_MAX_NT];
-#pragma unroll
-            for (int nt = 0; nt < W16_MAX_NT; ++nt) {
-                b0[nt] = b1[nt] = 0;
-                if (nt < nt_count && bptr[nt]) {
-                    b0[nt] = __ldg(reinterpret_cast<const uint32_t*>(bptr[nt] + kb + 2 * c));
-                    b1[nt] = __ldg(reinterpret_cast<const uint32_t*>(bptr[nt] + kb + 2 * c + 8));
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < NTILE_TILES; ++u) {
-                const uint32_t qw = st == 0 ? q[u].x : st == 1 ? q[u].y : st == 2 ? q[u].z : q[u].w;
-                const uint32_t sw = st < 2 ? sc[u].x : sc[u].y;
-                const uint32_t m = scale_mult2((st & 1) ? (sw >> 16) : (sw & 0xFFFFu));
-                uint32_t a[4];
-                dequant_step(qw, m, 0, a);
-#pragma unroll
-                for (int nt = 0; nt < W16_MAX_NT; ++nt)
-                    if (nt < nt_count) mma_bf16(acc[u][nt], a, b0[nt], b1[nt]);
-            }
-        }
+    for (int u = 0; u < 2; ++u) {
+        tc::bulk_load(st + u * W16_CH * 512, codes[u] + (int64_t)grp * ch * 512, ch * 512, &r.bar[stage]);
+        tc::bulk_load(st + W16_STAGE_CODES + u * W16_CH * 64, scales[u] + (int64_t)grp * ch * 64, ch * 64,
+                      &r.bar[stage]);
     }
 }
 
+// Streams `chunks` 64-column chunks of two 16-row tiles and accumulates their
+// products with up to W16_MAX_NT 8-token B tiles.  Returns false on a timeout.
+__device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2], const uint8_t* const scales[2],
+                                           int chunks, const uint16_t* const bptr[W16_MAX_NT], int nt_count,
+                                           float acc[2][W16_MAX_NT][4], int32_t* err) {
+    const int lane = lane_id();
+    const int g = lane >> 2, c = lane & 3;
+    const int ch = (chunks % W16_CH == 0) ? W16_CH : 2;
+    const int groups = chunks / ch;
+    const uint32_t base = r.ctr;
+    if (lane == 0)
+        for (int i = 0; i < W16_STAGES && i < groups; ++i) ring_issue(r, (base + i) % W16_STAGES, codes, scales, i, ch);
+    __syncwarp();
+    for (int grp = 0; grp < groups; ++grp) {
+        const uint32_t n = base + grp;
+        const int stage = n % W16_STAGES;
+        if (!tc::mbar_wait(&r.bar[stage], (n / W16_STAGES) & 1u, err)) return false;
+        const uint8_t* st = r.buf + stage * W16_STAGE;
+        for (int cc = 0; cc < ch; ++cc) {
+            uint4 q[2];
+            uint2 sc[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                q[u] = *reinterpret_cast<const uint4*>(st + u * W16_CH * 512 + cc * 512 + lane * 16);
+                sc[u] = *reinterpret_cast<const uint2*>(st + W16_STAGE_CODES + u * W16_CH * 64 + cc * 64 + g * 8);
+            }
+            const int kbase = (grp * ch + cc) * 64;
+#pragma unroll
+            for (int stp = 0; stp < 4; ++stp) {
+                const int kb = kbase + stp * 16;
+                uint32_t b0[W16_MAX_NT], b1[W16_MAX_NT];
+#pragma unroll
+                for (int nt = 0; nt < W16_MAX_NT; ++nt) {
+                    b0[nt] = b1[nt] = 0;
+                    if (nt < nt_count && bptr[nt]) {
+                        b0[nt] = __ldg(reinterpret_cast<const uint32_t*>(bptr[nt] + kb + 2 * c));
+                        b1[nt] = __ldg(reinterpret_cast<const uint32_t*>(bptr[nt] + kb + 2 * c + 8));
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const uint32_t qw = stp == 0 ? q[u].x : stp == 1 ? q[u].y : stp == 2 ? q[u].z : q[u].w;
+                    const uint32_t sw = stp < 2 ? sc[u].x : sc[u].y;
+                    const uint32_t m = scale_mult2((stp & 1) ? (sw >> 16) : (sw & 0xFFFFu));
+                    uint32_t a[4];
+                    dequant_step(qw, m, 0, a);
+#pragma unroll
+                    for (int nt = 0; nt < W16_MAX_NT; ++nt)
+                        if (nt < nt_count) mma_bf16(acc[u][nt], a, b0[nt], b1[nt]);
+                }
+            }
+        }
+        __syncwarp();  // every lane has read the stage
+        if (lane == 0 && grp + W16_STAGES < groups) {
+            tc::fence_proxy_async_smem();
+            ring_issue(r, stage, codes, scales, grp + W16_STAGES, ch);
+        }
+    }
+    r.ctr = base + groups;
+    return true;
+}
+
+__device__ __forceinline__ Ring make_ring(uint8_t* smem) {
+    Ring r;
+    const int w = warp_id();
+    r.buf = smem + w * W16_WARP_SMEM;
+    r.bar = reinterpret_cast<uint64_t*>(smem + W16_WARPS * W16_WARP_SMEM) + w * W16_STAGES;
+    r.ctr = 0;
+    if (lane_id() == 0) {
+        for (int i = 0; i < W16_STAGES; ++i) tc::mbar_init(&r.bar[i], 1);
+        tc::fence_mbar_init();
+    }
+    __syncwarp();
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// gate/up GEMM + SwiGLU: warps loop over (active expert, 16 intermediates)
+// ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(W16_WARPS * 32)
     k_w16_gateup(const uint16_t* __restrict__ x, const uint8_t* __restrict__ packed, W16Layout L, int H, int I, int k,
-                 RoutingPlan plan, uint16_t* __restrict__ A2) {
+                 RoutingPlan plan, uint16_t* __restrict__ A2, int32_t* err) {
+    extern __shared__ __align__(128) uint8_t w16_smem[];
+    Ring ring = make_ring(w16_smem);
     const int lane = lane_id();
     const int g = lane >> 2, c = lane & 3;
     const int iblocks = I / 16;
-    const int64_t wid = (int64_t)blockIdx.x * W16_WARPS + warp_id();
-    const int a_idx = (int)(wid / iblocks);
-    const int ib = (int)(wid % iblocks);
-    if (a_idx >= plan.n_active[0]) return;
-    const int e = plan.active[a_idx];
-    const int n_e = plan.counts[e];
-    const int row0 = plan.offsets[e];
     const int chunks = H / 64;
+    const int64_t items = (int64_t)plan.n_active[0] * iblocks;
     const float* glob = reinterpret_cast<const float*>(packed + L.globals);
-    const float ag = glob[e * 3 + 0] * 256.0f, au = glob[e * 3 + 1] * 256.0f;
-    const int64_t tile0 = ((int64_t)e * iblocks + ib) * 2;
-    const uint4* cbase[2];
-    const uint2* sbase[2];
+    for (int64_t item = (int64_t)blockIdx.x * W16_WARPS + warp_id(); item < items;
+         item += (int64_t)gridDim.x * W16_WARPS) {
+        const int e = plan.active[item / iblocks];
+        const int ib = (int)(item % iblocks);
+        const int n_e = plan.counts[e];
+        const int row0 = plan.offsets[e];
+        const float ag = glob[e * 3 + 0] * 256.0f, au = glob[e * 3 + 1] * 256.0f;
+        const int64_t tile0 = ((int64_t)e * iblocks + ib) * 2;
+        const uint8_t* cb[2];
+        const uint8_t* sb[2];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        cbase[u] = reinterpret_cast<const uint4*>(packed + L.gu_codes + (tile0 + u) * chunks * 512) + lane;
-        sbase[u] = reinterpret_cast<const uint2*>(packed + L.gu_scales + (tile0 + u) * chunks * 64) + g;
-    }
-    for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
-        const int nt_count = min(W16_MAX_NT, (n_e - n0 + 7) / 8);
-        const uint16_t* bptr[W16_MAX_NT];
-#pragma unroll
-        for (int nt = 0; nt < W16_MAX_NT; ++nt) {
-            const int n = n0 + nt * 8 + g;
-            bptr[nt] = (nt < nt_count && n < n_e) ? x + (int64_t)(plan.pair_of_row[row0 + n] / k) * H : nullptr;
+        for (int u = 0; u < 2; ++u) {
+            cb[u] = packed + L.gu_codes + (tile0 + u) * chunks * 512;
+            sb[u] = packed + L.gu_scales + (tile0 + u) * chunks * 64;
         }
-        float acc[2][W16_MAX_NT][4] = {};
-        w16_stream<2>(cbase, sbase, chunks, bptr, nt_count, c, acc);
+        for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
+            const int nt_count = min(W16_MAX_NT, (n_e - n0 + 7) / 8);
+            const uint16_t* bptr[W16_MAX_NT];
 #pragma unroll
-        for (int nt = 0; nt < W16_MAX_NT; ++nt) {
-            if (nt >= nt_count) break;
+            for (int nt = 0; nt < W16_MAX_NT; ++nt) {
+                const int n = n0 + nt * 8 + g;
+                bptr[nt] = (nt < nt_count && n < n_e) ? x + (int64_t)(plan.pair_of_row[row0 + n] / k) * H : nullptr;
+            }
+            float acc[2][W16_MAX_NT][4] = {};
+            if (!w16_stream(ring, cb, sb, chunks, bptr, nt_count, acc, err)) return;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {      // rows g, g + 8
+            for (int nt = 0; nt < W16_MAX_NT; ++nt) {
+                if (nt >= nt_count) break;
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {  // tokens 2c, 2c + 1
-                    const int n = n0 + nt * 8 + 2 * c + j;
-                    if (n < n_e) {
-                        const float gv = acc[0][nt][2 * h + j] * ag;
-                        const float uv = acc[1][nt][2 * h + j] * au;
-                        const __nv_bfloat16 v = __float2bfloat16_rn(silu(gv) * uv);
-                        A2[(int64_t)(row0 + n) * I + ib * 16 + g + 8 * h] = *reinterpret_cast<const uint16_t*>(&v);
+                for (int h = 0; h < 2; ++h) {      // rows g, g + 8
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {  // tokens 2c, 2c + 1
+                        const int n = n0 + nt * 8 + 2 * c + j;
+                        if (n < n_e) {
+                            const float gv = acc[0][nt][2 * h + j] * ag;
+                            const float uv = acc[1][nt][2 * h + j] * au;
+                            const __nv_bfloat16 v = __float2bfloat16_rn(silu(gv) * uv);
+                            A2[(int64_t)(row0 + n) * I + ib * 16 + g + 8 * h] = *reinterpret_cast<const uint16_t*>(&v);
+                        }
                     }
                 }
             }
@@ -287,56 +346,59 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
 }
 
 // ---------------------------------------------------------------------------
-// down GEMM x routing weight: one warp per (active expert, 32 hidden rows)
+// down GEMM x routing weight: warps loop over (active expert, 32 hidden rows)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(W16_WARPS * 32)
     k_w16_down(const uint8_t* __restrict__ packed, W16Layout L, int H, int I, RoutingPlan plan,
-               const uint16_t* __restrict__ A2, float* __restrict__ Y) {
+               const uint16_t* __restrict__ A2, float* __restrict__ Y, int32_t* err) {
+    extern __shared__ __align__(128) uint8_t w16_smem[];
+    Ring ring = make_ring(w16_smem);
     const int lane = lane_id();
     const int g = lane >> 2, c = lane & 3;
     const int hblocks = H / 32;
-    const int64_t wid = (int64_t)blockIdx.x * W16_WARPS + warp_id();
-    const int a_idx = (int)(wid / hblocks);
-    const int hb = (int)(wid % hblocks);
-    if (a_idx >= plan.n_active[0]) return;
-    const int e = plan.active[a_idx];
-    const int n_e = plan.counts[e];
-    const int row0 = plan.offsets[e];
     const int chunks = I / 64;
+    const int64_t items = (int64_t)plan.n_active[0] * hblocks;
     const float* glob = reinterpret_cast<const float*>(packed + L.globals);
-    const float ad = glob[e * 3 + 2] * 256.0f;
-    const int64_t tile0 = (int64_t)e * (H / 16) + hb * 2;
-    const uint4* cbase[2];
-    const uint2* sbase[2];
+    for (int64_t item = (int64_t)blockIdx.x * W16_WARPS + warp_id(); item < items;
+         item += (int64_t)gridDim.x * W16_WARPS) {
+        const int e = plan.active[item / hblocks];
+        const int hb = (int)(item % hblocks);
+        const int n_e = plan.counts[e];
+        const int row0 = plan.offsets[e];
+        const float ad = glob[e * 3 + 2] * 256.0f;
+        const int64_t tile0 = (int64_t)e * (H / 16) + hb * 2;
+        const uint8_t* cb[2];
+        const uint8_t* sb[2];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        cbase[u] = reinterpret_cast<const uint4*>(packed + L.d_codes + (tile0 + u) * chunks * 512) + lane;
-        sbase[u] = reinterpret_cast<const uint2*>(packed + L.d_scales + (tile0 + u) * chunks * 64) + g;
-    }
-    for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
-        const int nt_count = min(W16_MAX_NT, (n_e - n0 + 7) / 8);
-        const uint16_t* bptr[W16_MAX_NT];
-#pragma unroll
-        for (int nt = 0; nt < W16_MAX_NT; ++nt) {
-            const int n = n0 + nt * 8 + g;
-            bptr[nt] = (nt < nt_count && n < n_e) ? A2 + (int64_t)(row0 + n) * I : nullptr;
+        for (int u = 0; u < 2; ++u) {
+            cb[u] = packed + L.d_codes + (tile0 + u) * chunks * 512;
+            sb[u] = packed + L.d_scales + (tile0 + u) * chunks * 64;
         }
-        float acc[2][W16_MAX_NT][4] = {};
-        w16_stream<2>(cbase, sbase, chunks, bptr, nt_count, c, acc);
+        for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
+            const int nt_count = min(W16_MAX_NT, (n_e - n0 + 7) / 8);
+            const uint16_t* bptr[W16_MAX_NT];
 #pragma unroll
-        for (int nt = 0; nt < W16_MAX_NT; ++nt) {
-            if (nt >= nt_count) break;
+            for (int nt = 0; nt < W16_MAX_NT; ++nt) {
+                const int n = n0 + nt * 8 + g;
+                bptr[nt] = (nt < nt_count && n < n_e) ? A2 + (int64_t)(row0 + n) * I : nullptr;
+            }
+            float acc[2][W16_MAX_NT][4] = {};
+            if (!w16_stream(ring, cb, sb, chunks, bptr, nt_count, acc, err)) return;
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int n = n0 + nt * 8 + 2 * c + j;
-                if (n < n_e) {
-                    const int row = row0 + n;
-                    const float w = plan.wts[plan.pair_of_row[row]] * ad;
+            for (int nt = 0; nt < W16_MAX_NT; ++nt) {
+                if (nt >= nt_count) break;
 #pragma unroll
-                    for (int u = 0; u < 2; ++u)
+                for (int j = 0; j < 2; ++j) {
+                    const int n = n0 + nt * 8 + 2 * c + j;
+                    if (n < n_e) {
+                        const int row = row0 + n;
+                        const float w = plan.wts[plan.pair_of_row[row]] * ad;
 #pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            Y[(int64_t)row * H + hb * 32 + u * 16 + g + 8 * h] = acc[u][nt][2 * h + j] * w;
+                        for (int u = 0; u < 2; ++u)
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+                                Y[(int64_t)row * H + hb * 32 + u * 16 + g + 8 * h] = acc[u][nt][2 * h + j] * w;
+                    }
                 }
             }
         }
@@ -377,17 +439,22 @@ nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T,
                                    cudaEvent_t mid_event) {
     const W16Layout L = w16_layout(E, H, I);
     const uint8_t* p = static_cast<const uint8_t*>(packed);
-    // experts with rows <= min(E, T*k); grids cover that bound, extra warps exit
+    // experts with rows <= min(E, T*k): grids cover that bound; warps loop over
+    // the (expert, row block) items the device-side active list holds
     const int64_t max_active = std::min<int64_t>(E, (int64_t)T * k);
+    const int64_t max_ctas = (int64_t)num_sms() * 3;
+    int32_t* err = device_error_word();
+    NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));
+    NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_down, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));
     {
-        const int64_t warps = max_active * (I / 16);
-        k_w16_gateup<<<(unsigned)ceil_div(warps, W16_WARPS), W16_WARPS * 32, 0, stream>>>(x, p, L, H, I, k, plan, A2);
+        const int64_t ctas = std::min<int64_t>(ceil_div(max_active * (I / 16), W16_WARPS), max_ctas);
+        k_w16_gateup<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(x, p, L, H, I, k, plan, A2, err);
         NVFP4MOE_CHECK_LAUNCH("w4a16 gate/up kernel");
     }
     if (mid_event) cudaEventRecord(mid_event, stream);
     {
-        const int64_t warps = max_active * (H / 32);
-        k_w16_down<<<(unsigned)ceil_div(warps, W16_WARPS), W16_WARPS * 32, 0, stream>>>(p, L, H, I, plan, A2, Y);
+        const int64_t ctas = std::min<int64_t>(ceil_div(max_active * (H / 32), W16_WARPS), max_ctas);
+        k_w16_down<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(p, L, H, I, plan, A2, Y, err);
         NVFP4MOE_CHECK_LAUNCH("w4a16 down kernel");
     }
     return NVFP4MOE_OK;
