@@ -149,6 +149,29 @@ nvfp4moe_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t E, int32
                             int32_t* counts_out, int32_t* pad_offsets_out, int32_t* row_of_pair_out, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/* moe_permute without a workspace.  The pages have no counterpart to this call:
+ * it exists for callers that cannot allocate device memory, such as a plugin
+ * inside an inference engine that owns every device buffer and hands the plugin
+ * only its inputs and outputs, or a latency-critical path where cudaMalloc
+ * (which may synchronise the device) is not allowed.  Same operation, arguments
+ * and outputs as moe_permute, minus the workspace: the scratch is one static
+ * device array of NVFP4MOE_NOALLOC_SCRATCH_BYTES (1 MiB) inside the library,
+ * held on every GPU that loads the library until the process exits.
+ *   - Sizes whose moe_permute_workspace_size() exceeds that array are rejected
+ *     with NVFP4MOE_ERR_UNSUPPORTED_SHAPE before anything is launched;
+ *     T * top_k <= 65536 with E <= 256 always fits.
+ *   - The first call on a device looks up the array's device address (with that
+ *     device current); make that first call before any stream capture.
+ *   - No call allocates or frees device memory.
+ *   - All calls share the one array and it keeps the last call's contents:
+ *     calls whose work overlaps on the GPU (other streams, other host threads)
+ *     race; serialise them.  Nothing in the array needs clearing between calls. */
+#define NVFP4MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+nvfp4moe_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, int32_t E, int32_t top_k, int32_t pad,
+                                    int32_t* counts_out, int32_t* pad_offsets_out, int32_t* row_of_pair_out,
+                                    void* stream);
+
 /* ------------------------------------------------------------------------- */
 /* NVFP4 activation quantisation                                              */
 /* ------------------------------------------------------------------------- */

@@ -17,7 +17,7 @@ __all__ = [
     "transcode_mxfp4_to_nvfp4", "nvfp4moe_transcode_workspace_size", "moe_route", "quantize_nvfp4",
     "moe_packed_weights_size", "moe_pack_weights", "moe_forward_workspace_size", "moe_forward",
     "moe_forward_routed", "nvfp4moe_check_device_status", "nvfp4moe_version", "moe_permute",
-    "moe_permute_workspace_size", "nvfp4moe_set_trace_events",
+    "moe_permute_workspace_size", "nvfp4moe_set_trace_events", "moe_permute_noalloc",
 ]
 
 W4A16 = 0
@@ -91,6 +91,8 @@ def load():
     L.moe_permute_workspace_size.argtypes = [i32, i32, i32, i32]
     L.moe_permute.restype = ctypes.c_int
     L.moe_permute.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+    L.moe_permute_noalloc.restype = ctypes.c_int
+    L.moe_permute_noalloc.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
     L.nvfp4moe_set_trace_events.restype = ctypes.c_int
     L.nvfp4moe_set_trace_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     L.nvfp4moe_check_device_status.restype = ctypes.c_int
@@ -163,6 +165,14 @@ def moe_permute(topk_ids, E, pad, counts_out, pad_offsets_out, row_of_pair_out, 
     _check(load().moe_permute(_ptr(topk_ids), T, E, k, pad, _ptr(counts_out), _ptr(pad_offsets_out),
                               _ptr(row_of_pair_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
                               _stream(stream)))
+
+
+def moe_permute_noalloc(topk_ids, E, pad, counts_out, pad_offsets_out, row_of_pair_out, stream=None):
+    """moe_permute for callers that cannot allocate device memory: the scratch is
+    a fixed 1 MiB device array inside the library (see include/nvfp4moe.h)."""
+    T, k = topk_ids.shape
+    _check(load().moe_permute_noalloc(_ptr(topk_ids), T, E, k, pad, _ptr(counts_out), _ptr(pad_offsets_out),
+                                      _ptr(row_of_pair_out), _stream(stream)))
 
 
 def moe_packed_weights_size(mode, E, H, I) -> int:
