@@ -38,6 +38,7 @@ namespace {
 
 constexpr int BM = 128, BN = 256, BK = 256;  // BK in elements (128 bytes of codes)
 constexpr int STAGES = 4;
+constexpr int PREFETCH_AHEAD = 8;  // k-stages of L2 prefetch in front of the shared-memory ring
 constexpr int A_BYTES = BM * BK / 2;
 constexpr int B_BYTES = BN * BK / 2;
 constexpr int SFA_BYTES = BM * BK / 16;
@@ -154,11 +155,32 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int it = 0;
+            // L2 prefetch cursor, PREFETCH_AHEAD k-stages in front of the loads, so
+            // that weight tiles coming from HBM are L2 hits when the ring loads them
+            int pf_tile = blockIdx.x, pf_ks = 0;
+            auto prefetch_next = [&]() {
+                if (pf_tile >= total) return;
+                const int pm = pf_tile / p.n_ntiles, pn = pf_tile - pm * p.n_ntiles;
+                const int4 pti = p.tiles[pm];
+                const int64_t pb = (int64_t)pti.x * p.b_rows_per_expert + (int64_t)pn * BN;
+                const int n64 = min(4, k64_total - pf_ks * 4);
+                tc::tma_prefetch_2d(&tmA, pf_ks * 128, pti.y);
+                tc::tma_prefetch_2d(&tmB, pf_ks * 128, (int32_t)pb);
+                tc::bulk_prefetch_l2(p.sfa + ((int64_t)(pti.y / 128) * k64_total + pf_ks * 4) * 512, n64 * 512);
+                tc::bulk_prefetch_l2(p.sfb + ((pb / 128) * k64_total + pf_ks * 4) * 512, n64 * 512);
+                tc::bulk_prefetch_l2(p.sfb + ((pb / 128 + 1) * k64_total + pf_ks * 4) * 512, n64 * 512);
+                if (++pf_ks == ks_count) {
+                    pf_ks = 0;
+                    pf_tile += gridDim.x;
+                }
+            };
+            for (int i = 0; i < PREFETCH_AHEAD; ++i) prefetch_next();
             for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
                 const int m = tile / p.n_ntiles, n = tile - m * p.n_ntiles;
                 const int4 ti = p.tiles[m];
                 const int64_t b_row0 = (int64_t)ti.x * p.b_rows_per_expert + (int64_t)n * BN;
                 for (int ks = 0; ks < ks_count; ++ks, ++it) {
+                    prefetch_next();
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                     if (!tc::mbar_wait(&empty[s], ph ^ 1u, p.err)) goto done;
@@ -227,26 +249,32 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!tc::mbar_wait(acc_full, (uint32_t)tl & 1u, p.err)) goto done;
             tc::tc_fence_after();
             if (EPI == EPI_GATEUP) {
-                // columns [0,128) gate, [128,256) up, for intermediates n*128 .. n*128+127
-                const float ag = p.globals[ti.x * 3 + 0] * p.act_global;
-                const float au = p.globals[ti.x * 3 + 1] * p.act_global;
+                // columns [0,128) gate, [128,256) up, for intermediates n*128 .. n*128+127.
+                // All of this warp's accumulator values are pulled into registers first
+                // and the accumulator is released before any arithmetic, so the MMA
+                // warp only waits for the TMEM reads.
                 const int i0 = n * (BN / 2) + half * 64;  // first intermediate of this warp
-                const int nkb = p.out_k / 16;
-                uint32_t codes[8], sfw = 0;
+                float gv[64], uv[64];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float gv[16], uv[16];
-                    tc::tmem_ld16x2(t_row + half * 64 + 16 * c, t_row + 128 + half * 64 + 16 * c, gv, uv);
-                    float a[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) a[i] = silu_fast(gv[i] * ag) * (uv[i] * au);
-                    const uint32_t sf = requant_block16(a, p.act_global, codes[2 * c], codes[2 * c + 1]);
-                    sfw |= sf << (8 * c);
-                }
+                for (int c = 0; c < 4; ++c)
+                    tc::tmem_ld16x2(t_row + half * 64 + 16 * c, t_row + 128 + half * 64 + 16 * c, gv + 16 * c,
+                                    uv + 16 * c);
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(acc_empty);  // accumulator drained by this warp
+                if (lane == 0) tc::mbar_arrive(acc_empty);
                 if (valid) {
+                    const float ag = p.globals[ti.x * 3 + 0] * p.act_global;
+                    const float au = p.globals[ti.x * 3 + 1] * p.act_global;
+                    const int nkb = p.out_k / 16;
+                    uint32_t codes[8], sfw = 0;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float a[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) a[i] = silu_fast(gv[16 * c + i] * ag) * (uv[16 * c + i] * au);
+                        const uint32_t sf = requant_block16(a, p.act_global, codes[2 * c], codes[2 * c + 1]);
+                        sfw |= sf << (8 * c);
+                    }
                     uint4* dst = reinterpret_cast<uint4*>(p.out_codes + row * (p.out_k / 2) + i0 / 2);
                     dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
                     dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
@@ -255,49 +283,41 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             } else {
                 // y = acc * global * routing weight, staged as FP16 with one power-of-two
-                // scale per (row, 128 columns): pass 1 finds the max, pass 2 writes
-                // y / scale (exact power-of-two scaling, then one FP16 rounding).
-                const float f = valid ? p.globals[ti.x * 3 + 2] * p.act_global * p.wts[p.pair_of_row[row]] : 0.0f;
+                // scale per (row, 128 columns).  The warp's 128 accumulator columns are
+                // read into registers and released first; then the max picks the
+                // scale and y / scale is written (exact power-of-two scaling, one FP16
+                // rounding).
+                float v[128];
                 const uint32_t t_col = t_row + half * 128;
-                float amax = 0.0f;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float v0[16], v1[16];
-                    tc::tmem_ld16x2(t_col + 32 * c, t_col + 32 * c + 16, v0, v1);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fmaxf(fabsf(v0[i]), fabsf(v1[i])));
-                }
-                amax *= fabsf(f);
-                // scale = 2^(e - 14) with amax in [2^e, 2^(e+1)): staged magnitudes stay below 2^15
-                int e = 0;
-                if (amax > 0.0f && isfinite(amax)) e = ((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-                e = max(min(e - 14, 100), -100);
-                const float g = ldexpf(f, -e);
-                __half* yrow = p.Y + row * p.ldy + (int64_t)n * BN + half * 128;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float v0[16], v1[16];
-                    tc::tmem_ld16x2(t_col + 32 * c, t_col + 32 * c + 16, v0, v1);
-                    if (c == 3) {
-                        tc::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(acc_empty);
-                    }
-                    if (valid) {
-                        uint32_t pk[16];
+                for (int c = 0; c < 4; ++c) tc::tmem_ld16x2(t_col + 32 * c, t_col + 32 * c + 16, v + 32 * c, v + 32 * c + 16);
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(acc_empty);
+                if (valid) {
+                    const float f = p.globals[ti.x * 3 + 2] * p.act_global * p.wts[p.pair_of_row[row]];
+                    float amax = 0.0f;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            __half2 b0 = __floats2half2_rn(v0[2 * i] * g, v0[2 * i + 1] * g);
-                            __half2 b1 = __floats2half2_rn(v1[2 * i] * g, v1[2 * i + 1] * g);
-                            pk[i] = *reinterpret_cast<uint32_t*>(&b0);
-                            pk[8 + i] = *reinterpret_cast<uint32_t*>(&b1);
+                    for (int i = 0; i < 128; ++i) amax = fmaxf(amax, fabsf(v[i]));
+                    amax *= fabsf(f);
+                    // scale = 2^(e - 14) with amax in [2^e, 2^(e+1)): staged magnitudes stay below 2^15
+                    int e = 0;
+                    if (amax > 0.0f && isfinite(amax)) e = ((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+                    e = max(min(e - 14, 100), -100);
+                    const float g = ldexpf(f, -e);
+                    uint4* dst = reinterpret_cast<uint4*>(p.Y + row * p.ldy + (int64_t)n * BN + half * 128);
+#pragma unroll
+                    for (int q8 = 0; q8 < 16; ++q8) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            __half2 b = __floats2half2_rn(v[8 * q8 + 2 * i] * g, v[8 * q8 + 2 * i + 1] * g);
+                            pk[i] = *reinterpret_cast<uint32_t*>(&b);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(yrow + 32 * c);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                        dst[q8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     }
+                    p.y_scale[row * (p.ldy / 128) + n * 2 + half] = ldexpf(1.0f, e);
                 }
-                if (valid) p.y_scale[row * (p.ldy / 128) + n * 2 + half] = ldexpf(1.0f, e);
             }
         }
     }
