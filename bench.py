@@ -253,7 +253,18 @@ def run_ours(args, rank, world, local_rank):
                     "peak_src": f"{P['src']} bf16 burst x {FP4_OVER_BF16:g} (nominal dense FP4:BF16)",
                     "algorithmic_flops_per_launch": flops}
     else:
-        roofline = None
+        # W4A16 weight stream: every active expert's codes + E4M3 scales read once
+        ids_t = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+        w_t = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+        moe.moe_route(logits, None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf, True, ids_t, w_t)
+        active = int(torch.unique(ids_t).numel())
+        wbytes = active * (2 * wl.I * wl.H + wl.H * wl.I) * (0.5 + 1.0 / 16)
+        t_kernel = (stage["gateup_gemm"] + stage["down_gemm"]) / 1e3
+        achieved = wbytes / t_kernel / 1e9
+        roofline = {"bound": "hbm", "kernel": "k_w16_gateup + k_w16_down", "achieved": round(achieved, 1),
+                    "peak": P["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / P["hbm_gbs"], 4), "traffic": None,
+                    "peak_src": f"{P['src']} copy bandwidth", "algorithmic_bytes_per_step": int(wbytes),
+                    "active_experts": active}
 
     res = {
         "metric": "MoE-layer tokens/s", "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -272,7 +283,7 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": int(d["x"].nbytes + d["logits"].nbytes), "d2h_bytes_per_step": int(T * wl.H * 2)},
         "gpu_launches": 8 * args.steps,
         "clocks": clocks,
-        "tflops": round(layer_flops(T, wl.H, wl.I, wl.top_k) / (ms / 1e3) / 1e12, 1),
+        "tflops": round(layer_flops(T, wl.H, wl.I, wl.top_k) / (ms / 1e3) / 1e12, 2),
     }
     del packed, ws
     torch.cuda.empty_cache()

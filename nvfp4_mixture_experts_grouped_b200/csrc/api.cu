@@ -93,7 +93,7 @@ struct ForwardLayout {
     // byte offsets
     int64_t ids, wts, chunk_counts, counts, offsets, pad_offsets, row_of_pair, pair_of_row, tiles, n_tiles, active,
         n_active;
-    int64_t a1c, a1s, a2c, a2s, a2bf, y, ys;
+    int64_t a1c, a1s, a2c, a2s, a2bf, y, ys, w16s;
     int64_t total;
 };
 
@@ -137,6 +137,7 @@ static ForwardLayout forward_layout(nvfp4moe_mode mode, int64_t T, int64_t H, in
         L.a1c = L.a1s = L.a2c = L.a2s = L.ys = -1;
         L.a2bf = take(L.rows_max * I * 2);
         L.y = take(L.rows_max * H * 4);  // FP32 staged rows
+        L.w16s = take((int64_t)w4a16_scratch_size((int)T, (int)H, (int)I, (int)k));
     }
     L.total = o;
     return L;
@@ -386,7 +387,7 @@ static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, con
     } else {
         trace(3, st);
         RETURN_IF(launch_w4a16_layer(x, packed, T, H, I, E, top_k, plan, reinterpret_cast<uint16_t*>(ws + L.a2bf),
-                                     static_cast<float*>(Y), st, g_trace_on ? g_trace[4] : nullptr));
+                                     static_cast<float*>(Y), ws + L.w16s, st, g_trace_on ? g_trace[4] : nullptr));
     }
     trace(5, st);
     RETURN_IF(launch_combine(Y, ys, plan.row_of_pair, T, H, top_k, out, out_is_fp32 != 0, st));

@@ -57,9 +57,10 @@ nvfp4moe_status launch_combine(const void* Y, const float* y_scale, const int32_
 // w4a16.cu
 size_t w4a16_packed_size(int E, int H, int I);
 nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream);
+size_t w4a16_scratch_size(int T, int H, int I, int k);  // FP16 copies of the activations + row scales
 nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T, int H, int I, int E, int k,
-                                   const RoutingPlan& plan, uint16_t* A2, float* Y, cudaStream_t stream,
-                                   cudaEvent_t mid_event);
+                                   const RoutingPlan& plan, uint16_t* A2, float* Y, void* scratch,
+                                   cudaStream_t stream, cudaEvent_t mid_event);
 
 // w4a4.cu
 size_t w4a4_packed_size(int E, int H, int I);

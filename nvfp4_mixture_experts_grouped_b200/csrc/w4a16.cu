@@ -1,4 +1,4 @@
-// w4a16.cu -- the W4A16 (BF16 activations x NVFP4 weights) expert GEMMs for
+// w4a16.cu -- the W4A16 (16-bit activations x NVFP4 weights) expert GEMMs for
 // decode-sized batches on sm_100a.
 //
 // Mode: "AxionML / MiMo-V2.6-Flash-MOPD-NVFP4", "Usage" (BF16-activation,
@@ -6,23 +6,23 @@
 // REAP-50", "Pruning Method" 1 (down(SiLU(gate h) * up h)).
 //
 // At decode an expert sees ~1-2 tokens, so the layer is a weight stream: every
-// active expert's codes and scales are read from HBM exactly once.  Weights are
-// the MMA "A" operand (16 weight rows per mma.sync.m16n8k16), tokens the "B"
-// operand (8 per n-tile).  Weights are dequantised in registers to BF16:
-//   * one 32-bit word holds the 8 codes a lane needs for one k16 step, with
-//     their bits pre-placed by the pack step so that each BF16x2 fragment
-//     register is one or two shift/AND operations away: a code (s e1 e0 m)
-//     whose 3 magnitude bits land on BF16 bits 8..6 and whose sign lands on bit
-//     15 is exactly the E2M1 value times 2^-126 (the 0.5 code becomes the BF16
-//     subnormal 2^-127);
-//   * the E4M3 block scale becomes the BF16 multiplier scale * 2^118 (through
-//     the exact E4M3->F16 conversion and an exponent re-bias), so one BF16x2
-//     multiply yields value * scale * 2^-8 exactly (at most 5 significant bits,
-//     range [2^-18, 10.5]);
-//   * the FP32 accumulator is multiplied by 2^8 * global in the epilogue.
-// Gate and up rows of the same 16 intermediates are streamed by the same warp,
-// so SwiGLU is applied on the accumulators and only BF16 SwiGLU rows are stored.
-// The down GEMM stages its weighted per-pair rows in FP32 (a few MB at decode).
+// active expert's codes and scales are read from HBM once and dequantised in
+// registers, which makes the instruction count per weight the limit.  Weights
+// are the mma.sync.m16n8k16 "A" operand (16 weight rows), tokens the "B"
+// operand (8 per n-tile), both FP16:
+//   * E2M1 codes become exact FP16 values with the hardware e2m1x2->f16x2
+//     conversion (one instruction per pair), E4M3 block scales with the
+//     e4m3x2->f16x2 conversion, and one FP16x2 multiply gives value * scale
+//     exactly (at most 5 significant bits, range [2^-10, 2688]);
+//   * the BF16 activations (the layer input, and the SwiGLU output rounded to
+//     BF16) are rescaled per row by a power of two 2^s that puts the row's
+//     largest magnitude in [2^14, 2^15) and converted to FP16: every element
+//     within 2^29 of the row's largest keeps its exact BF16 value, smaller ones
+//     round below 2^-40 of the largest; the accumulator is scaled back by 2^-s.
+// Weight bytes reach shared memory through per-warp cp.async.bulk rings (see
+// w16_stream); gate and up rows of the same 16 intermediates are streamed by
+// one warp so SwiGLU is applied on the accumulators.  The down GEMM stages its
+// weighted per-pair rows in FP32 (a few MB at decode).
 #include <algorithm>
 
 #include "common.cuh"
@@ -55,34 +55,26 @@ __host__ __device__ inline W16Layout w16_layout(int E, int H, int I) {
 }
 
 // ---------------------------------------------------------------------------
-// pack
+// pack: per 16-row tile and 64-column chunk, 512 bytes in fragment order (lane
+// l holds 16 bytes: one 32-bit word per k16 step); inside a word byte j holds
+// the two consecutive-column codes of A-fragment register j (low nibble = even
+// column): j=0 row g cols 2c,2c+1; j=1 row g+8; j=2 row g cols 2c+8,2c+9; j=3
+// row g+8.  Scales: 64 bytes per chunk, 8 per row pair g: [s(g,k16 step t),
+// s(g+8,t)] for t = 0..3.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t code_at(const uint8_t* codes, const uint8_t* sf, int64_t r, int64_t k, int64_t K) {
-    if (sf[r * (K / 16) + k / 16] == 0) return 0;  // a zero-scale block decodes to 0 whatever its codes
+__device__ __forceinline__ uint32_t code_at(const uint8_t* codes, int64_t r, int64_t k, int64_t K) {
     const uint32_t b = codes[r * (K / 2) + k / 2];
     return (k & 1) ? (b >> 4) : (b & 15u);
 }
 
-// Fragment word of lane (g, c) for k16 step at column kb of a 16-row tile at r0.
-__device__ uint32_t pack_word(const uint8_t* codes, const uint8_t* sf, int64_t r0, int64_t kb, int g, int c,
-                              int64_t K) {
+__device__ uint32_t pack_word(const uint8_t* codes, int64_t r0, int64_t kb, int g, int c, int64_t K) {
     const int64_t ra = r0 + g, rb = r0 + g + 8;
     const int64_t k0 = kb + 2 * c, k1 = kb + 2 * c + 8;
-    const uint32_t q0l = code_at(codes, sf, ra, k0, K), q0h = code_at(codes, sf, ra, k0 + 1, K);
-    const uint32_t q1l = code_at(codes, sf, rb, k0, K), q1h = code_at(codes, sf, rb, k0 + 1, K);
-    const uint32_t q2l = code_at(codes, sf, ra, k1, K), q2h = code_at(codes, sf, ra, k1 + 1, K);
-    const uint32_t q3l = code_at(codes, sf, rb, k1, K), q3h = code_at(codes, sf, rb, k1 + 1, K);
-    uint32_t w = 0;
-    // register 0: magnitude at 6..8 / 22..24, sign at 15 / 31
-    w |= ((q0l & 7u) << 6) | ((q0l >> 3) << 15) | ((q0h & 7u) << 22) | ((q0h >> 3) << 31);
-    // register 1: stored 3 bits lower
-    w |= ((q1l & 7u) << 3) | ((q1l >> 3) << 12) | ((q1h & 7u) << 19) | ((q1h >> 3) << 28);
-    // register 2: stored 6 bits lower
-    w |= ((q2l & 7u) << 0) | ((q2l >> 3) << 9) | ((q2h & 7u) << 16) | ((q2h >> 3) << 25);
-    // register 3: m -> 10, e0 -> 11, e1 -> 13, sign -> 14 (and +16 for the odd element)
-    w |= ((q3l & 1u) << 10) | (((q3l >> 1) & 1u) << 11) | (((q3l >> 2) & 1u) << 13) | ((q3l >> 3) << 14);
-    w |= ((q3h & 1u) << 26) | (((q3h >> 1) & 1u) << 27) | (((q3h >> 2) & 1u) << 29) | ((q3h >> 3) << 30);
-    return w;
+    const uint32_t b0 = code_at(codes, ra, k0, K) | (code_at(codes, ra, k0 + 1, K) << 4);
+    const uint32_t b1 = code_at(codes, rb, k0, K) | (code_at(codes, rb, k0 + 1, K) << 4);
+    const uint32_t b2 = code_at(codes, ra, k1, K) | (code_at(codes, ra, k1 + 1, K) << 4);
+    const uint32_t b3 = code_at(codes, rb, k1, K) | (code_at(codes, rb, k1 + 1, K) << 4);
+    return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
 }
 
 // One thread per (tile, k64 chunk, lane): 16 code bytes, plus 8 scale bytes for lanes with c == 0.
@@ -96,7 +88,6 @@ __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __r
     const int lane = (int)(idx & 31);
     const int64_t chunk = (idx >> 5) % chunks;
     const int64_t tile = (idx >> 5) / chunks;  // packed tile index
-    // source tensor and its first row
     const uint8_t* c = codes;
     const uint8_t* s = sf;
     int64_t r0;
@@ -105,70 +96,113 @@ __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __r
         const int64_t tiles_per_expert = rows_per_expert / 16 * 2;
         const int64_t e = tile / tiles_per_expert;
         const int64_t rem = tile % tiles_per_expert;
-        const int64_t ib = rem / 2;
         if (rem & 1) {
             c = codes2;
             s = sf2;
         }
-        r0 = e * rows_per_expert + ib * 16;
+        r0 = e * rows_per_expert + (rem / 2) * 16;
     } else {
         r0 = tile * 16;
     }
     const int g = lane >> 2, cc = lane & 3;
     uint32_t w[4];
 #pragma unroll
-    for (int st = 0; st < 4; ++st) w[st] = pack_word(c, s, r0, chunk * 64 + st * 16, g, cc, K);
+    for (int st = 0; st < 4; ++st) w[st] = pack_word(c, r0, chunk * 64 + st * 16, g, cc, K);
     *reinterpret_cast<uint4*>(out_codes + (tile * chunks + chunk) * 512 + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
     if (cc == 0) {
-        uint8_t b[8];
+        uint32_t b[8];
 #pragma unroll
         for (int st = 0; st < 4; ++st) {
-            const int64_t kb = (chunk * 64 + st * 16) / 16;
+            const int64_t kb = chunk * 4 + st;
             b[2 * st] = s[(r0 + g) * (K / 16) + kb];
             b[2 * st + 1] = s[(r0 + g + 8) * (K / 16) + kb];
         }
         uint2 v;
-        v.x = b[0] | (b[1] << 8) | (b[2] << 16) | ((uint32_t)b[3] << 24);
-        v.y = b[4] | (b[5] << 8) | (b[6] << 16) | ((uint32_t)b[7] << 24);
+        v.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+        v.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
         *reinterpret_cast<uint2*>(out_scales + (tile * chunks + chunk) * 64 + g * 8) = v;
     }
 }
 
 // ---------------------------------------------------------------------------
-// dequantisation helpers
+// BF16 rows -> FP16 rows with a per-row power-of-two scale (one warp per row)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+__global__ void __launch_bounds__(256)
+    k_rows_to_f16(const uint16_t* __restrict__ src, int64_t rows, int K, __half* __restrict__ dst,
+                  float* __restrict__ inv_scale) {
+    const int64_t r = (int64_t)blockIdx.x * 8 + warp_id();
+    if (r >= rows) return;
+    const int lane = lane_id();
+    const uint4* s = reinterpret_cast<const uint4*>(src + r * K);
+    float amax = 0.0f;
+    for (int i = lane; i < K / 8; i += 32) {
+        const uint4 v = s[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            amax = fmaxf(amax, fmaxf(fabsf(bf16_bits_to_float(w[q] & 0xFFFFu)), fabsf(bf16_bits_to_float(w[q] >> 16))));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int sh = 0;
+    if (amax > 0.0f && isfinite(amax)) {
+        int e;
+        frexpf(amax, &e);  // amax in [2^(e-1), 2^e)
+        sh = 15 - e;       // amax * 2^sh in [2^14, 2^15)
+    }
+    uint4* d = reinterpret_cast<uint4*>(dst + r * K);
+    for (int i = lane; i < K / 8; i += 32) {
+        const uint4 v = s[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const __half2 h = __floats2half2_rn(ldexpf(bf16_bits_to_float(w[q] & 0xFFFFu), sh),
+                                                ldexpf(bf16_bits_to_float(w[q] >> 16), sh));
+            o[q] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        d[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (lane == 0) inv_scale[r] = ldexpf(1.0f, -sh);
+}
+
+// ---------------------------------------------------------------------------
+// dequantisation and MMA helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
     uint32_t d;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
-// Two E4M3 scales (bytes lo, hi of `pair`) -> BF16x2 multipliers scale * 2^118.
-__device__ __forceinline__ uint32_t scale_mult2(uint32_t pair) {
+// Two E4M3 scales (bytes lo, hi of `pair`) -> FP16x2 (exact).
+__device__ __forceinline__ uint32_t scales_f16x2(uint32_t pair) {
     uint32_t h;
     asm("{\n\t.reg .b16 t;\n\tmov.b16 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "h"((uint16_t)pair));
-    return ((h >> 3) & 0x0FFF0FFFu) + 0x73007300u;
+    return h;
 }
 
-// 8 codes of one k16 step -> four BF16x2 A-fragment registers scaled by the
-// multipliers of rows g (mg) and g + 8 (mg8).
-__device__ __forceinline__ void dequant_step(uint32_t q, uint32_t mg, uint32_t mg8, uint32_t a[4]) {
-    const uint32_t P = 0x81C081C0u;
-    const uint32_t r0 = q & P;
-    const uint32_t r1 = (q << 3) & P;
-    const uint32_t r2 = (q << 6) & P;
-    const uint32_t r3 = ((q >> 4) & 0x00C000C0u) | ((q >> 5) & 0x01000100u) | ((q << 1) & 0x80008000u);
-    const uint32_t dg = __byte_perm(mg, mg, 0x1010), dg8 = __byte_perm(mg, mg, 0x3232);
-    (void)mg8;
-    a[0] = bf16x2_mul(r0, dg);
-    a[1] = bf16x2_mul(r1, dg8);
-    a[2] = bf16x2_mul(r2, dg);
-    a[3] = bf16x2_mul(r3, dg8);
+// 8 codes of one k16 step -> the four FP16x2 A-fragment registers, scaled by
+// the block scales of rows g and g + 8 (m = FP16x2 {scale g, scale g+8}).
+__device__ __forceinline__ void dequant_step(uint32_t q, uint32_t m, uint32_t a[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+        : "r"(q));
+    const uint32_t dg = __byte_perm(m, m, 0x1010), dg8 = __byte_perm(m, m, 0x3232);
+    a[0] = f16x2_mul(a[0], dg);
+    a[1] = f16x2_mul(a[1], dg8);
+    a[2] = f16x2_mul(a[2], dg);
+    a[3] = f16x2_mul(a[3], dg8);
 }
 
-__device__ __forceinline__ void mma_bf16(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_f16(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -179,12 +213,12 @@ __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 // ---------------------------------------------------------------------------
 // Weight streaming: every warp owns a ring of W16_STAGES shared-memory stages;
 // lane 0 fills a stage with 1-D bulk copies (cp.async.bulk, completion counted
-// on the stage's mbarrier) W16_STAGES groups ahead of the consumer, so each SM
-// keeps ~200 KB of the weight stream in flight without holding it in registers.
-// A stage holds W16_CH consecutive 64-column chunks of both 16-row tiles.
+// on the stage's mbarrier) W16_STAGES groups ahead of the consumer, so the
+// weight stream stays in flight without occupying registers.  A stage holds
+// W16_CH consecutive 64-column chunks of both 16-row tiles of the warp.
 // ---------------------------------------------------------------------------
 constexpr int W16_STAGES = 4;
-constexpr int W16_CH = 4;
+constexpr int W16_CH = 2;
 constexpr int W16_STAGE_CODES = 2 * W16_CH * 512;
 constexpr int W16_STAGE_SCALES = 2 * W16_CH * 64;
 constexpr int W16_STAGE = W16_STAGE_CODES + W16_STAGE_SCALES;
@@ -198,36 +232,37 @@ struct Ring {
 };
 
 __device__ __forceinline__ void ring_issue(Ring& r, int stage, const uint8_t* const codes[2],
-                                           const uint8_t* const scales[2], int grp, int ch) {
+                                           const uint8_t* const scales[2], int grp) {
     uint8_t* st = r.buf + stage * W16_STAGE;
-    tc::mbar_arrive_expect_tx(&r.bar[stage], 2 * ch * (512 + 64));
+    tc::mbar_arrive_expect_tx(&r.bar[stage], W16_STAGE);
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-        tc::bulk_load(st + u * W16_CH * 512, codes[u] + (int64_t)grp * ch * 512, ch * 512, &r.bar[stage]);
-        tc::bulk_load(st + W16_STAGE_CODES + u * W16_CH * 64, scales[u] + (int64_t)grp * ch * 64, ch * 64,
+        tc::bulk_load(st + u * W16_CH * 512, codes[u] + (int64_t)grp * W16_CH * 512, W16_CH * 512, &r.bar[stage]);
+        tc::bulk_load(st + W16_STAGE_CODES + u * W16_CH * 64, scales[u] + (int64_t)grp * W16_CH * 64, W16_CH * 64,
                       &r.bar[stage]);
     }
 }
 
 // Streams `chunks` 64-column chunks of two 16-row tiles and accumulates their
-// products with up to W16_MAX_NT 8-token B tiles.  Returns false on a timeout.
+// products with up to W16_MAX_NT 8-token B tiles (FP16 rows).  Returns false on
+// a timeout.
 __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2], const uint8_t* const scales[2],
-                                           int chunks, const uint16_t* const bptr[W16_MAX_NT], int nt_count,
+                                           int chunks, const __half* const bptr[W16_MAX_NT], int nt_count,
                                            float acc[2][W16_MAX_NT][4], int32_t* err) {
     const int lane = lane_id();
     const int g = lane >> 2, c = lane & 3;
-    const int ch = (chunks % W16_CH == 0) ? W16_CH : 2;
-    const int groups = chunks / ch;
+    const int groups = chunks / W16_CH;
     const uint32_t base = r.ctr;
     if (lane == 0)
-        for (int i = 0; i < W16_STAGES && i < groups; ++i) ring_issue(r, (base + i) % W16_STAGES, codes, scales, i, ch);
+        for (int i = 0; i < W16_STAGES && i < groups; ++i) ring_issue(r, (base + i) % W16_STAGES, codes, scales, i);
     __syncwarp();
     for (int grp = 0; grp < groups; ++grp) {
         const uint32_t n = base + grp;
         const int stage = n % W16_STAGES;
         if (!tc::mbar_wait(&r.bar[stage], (n / W16_STAGES) & 1u, err)) return false;
         const uint8_t* st = r.buf + stage * W16_STAGE;
-        for (int cc = 0; cc < ch; ++cc) {
+#pragma unroll
+        for (int cc = 0; cc < W16_CH; ++cc) {
             uint4 q[2];
             uint2 sc[2];
 #pragma unroll
@@ -235,7 +270,7 @@ __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2
                 q[u] = *reinterpret_cast<const uint4*>(st + u * W16_CH * 512 + cc * 512 + lane * 16);
                 sc[u] = *reinterpret_cast<const uint2*>(st + W16_STAGE_CODES + u * W16_CH * 64 + cc * 64 + g * 8);
             }
-            const int kbase = (grp * ch + cc) * 64;
+            const int kbase = (grp * W16_CH + cc) * 64;
 #pragma unroll
             for (int stp = 0; stp < 4; ++stp) {
                 const int kb = kbase + stp * 16;
@@ -252,19 +287,18 @@ __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2
                 for (int u = 0; u < 2; ++u) {
                     const uint32_t qw = stp == 0 ? q[u].x : stp == 1 ? q[u].y : stp == 2 ? q[u].z : q[u].w;
                     const uint32_t sw = stp < 2 ? sc[u].x : sc[u].y;
-                    const uint32_t m = scale_mult2((stp & 1) ? (sw >> 16) : (sw & 0xFFFFu));
                     uint32_t a[4];
-                    dequant_step(qw, m, 0, a);
+                    dequant_step(qw, scales_f16x2((stp & 1) ? (sw >> 16) : (sw & 0xFFFFu)), a);
 #pragma unroll
                     for (int nt = 0; nt < W16_MAX_NT; ++nt)
-                        if (nt < nt_count) mma_bf16(acc[u][nt], a, b0[nt], b1[nt]);
+                        if (nt < nt_count) mma_f16(acc[u][nt], a, b0[nt], b1[nt]);
                 }
             }
         }
         __syncwarp();  // every lane has read the stage
         if (lane == 0 && grp + W16_STAGES < groups) {
             tc::fence_proxy_async_smem();
-            ring_issue(r, stage, codes, scales, grp + W16_STAGES, ch);
+            ring_issue(r, stage, codes, scales, grp + W16_STAGES);
         }
     }
     r.ctr = base + groups;
@@ -289,8 +323,8 @@ __device__ __forceinline__ Ring make_ring(uint8_t* smem) {
 // gate/up GEMM + SwiGLU: warps loop over (active expert, 16 intermediates)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(W16_WARPS * 32)
-    k_w16_gateup(const uint16_t* __restrict__ x, const uint8_t* __restrict__ packed, W16Layout L, int H, int I, int k,
-                 RoutingPlan plan, uint16_t* __restrict__ A2, int32_t* err) {
+    k_w16_gateup(const __half* __restrict__ x16, const float* __restrict__ x_inv, const uint8_t* __restrict__ packed,
+                 W16Layout L, int H, int I, int k, RoutingPlan plan, uint16_t* __restrict__ A2, int32_t* err) {
     extern __shared__ __align__(128) uint8_t w16_smem[];
     Ring ring = make_ring(w16_smem);
     const int lane = lane_id();
@@ -305,7 +339,7 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
         const int ib = (int)(item % iblocks);
         const int n_e = plan.counts[e];
         const int row0 = plan.offsets[e];
-        const float ag = glob[e * 3 + 0] * 256.0f, au = glob[e * 3 + 1] * 256.0f;
+        const float ag = glob[e * 3 + 0], au = glob[e * 3 + 1];
         const int64_t tile0 = ((int64_t)e * iblocks + ib) * 2;
         const uint8_t* cb[2];
         const uint8_t* sb[2];
@@ -316,11 +350,11 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
         }
         for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
             const int nt_count = min(W16_MAX_NT, (n_e - n0 + 7) / 8);
-            const uint16_t* bptr[W16_MAX_NT];
+            const __half* bptr[W16_MAX_NT];
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
                 const int n = n0 + nt * 8 + g;
-                bptr[nt] = (nt < nt_count && n < n_e) ? x + (int64_t)(plan.pair_of_row[row0 + n] / k) * H : nullptr;
+                bptr[nt] = (nt < nt_count && n < n_e) ? x16 + (int64_t)(plan.pair_of_row[row0 + n] / k) * H : nullptr;
             }
             float acc[2][W16_MAX_NT][4] = {};
             if (!w16_stream(ring, cb, sb, chunks, bptr, nt_count, acc, err)) return;
@@ -328,13 +362,14 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
                 if (nt >= nt_count) break;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {      // rows g, g + 8
+                for (int j = 0; j < 2; ++j) {  // tokens 2c, 2c + 1
+                    const int n = n0 + nt * 8 + 2 * c + j;
+                    if (n < n_e) {
+                        const float inv = x_inv[plan.pair_of_row[row0 + n] / k];
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {  // tokens 2c, 2c + 1
-                        const int n = n0 + nt * 8 + 2 * c + j;
-                        if (n < n_e) {
-                            const float gv = acc[0][nt][2 * h + j] * ag;
-                            const float uv = acc[1][nt][2 * h + j] * au;
+                        for (int h = 0; h < 2; ++h) {  // rows g, g + 8
+                            const float gv = acc[0][nt][2 * h + j] * inv * ag;
+                            const float uv = acc[1][nt][2 * h + j] * inv * au;
                             const __nv_bfloat16 v = __float2bfloat16_rn(silu(gv) * uv);
                             A2[(int64_t)(row0 + n) * I + ib * 16 + g + 8 * h] = *reinterpret_cast<const uint16_t*>(&v);
                         }
@@ -350,7 +385,7 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(W16_WARPS * 32)
     k_w16_down(const uint8_t* __restrict__ packed, W16Layout L, int H, int I, RoutingPlan plan,
-               const uint16_t* __restrict__ A2, float* __restrict__ Y, int32_t* err) {
+               const __half* __restrict__ A16, const float* __restrict__ a_inv, float* __restrict__ Y, int32_t* err) {
     extern __shared__ __align__(128) uint8_t w16_smem[];
     Ring ring = make_ring(w16_smem);
     const int lane = lane_id();
@@ -365,7 +400,7 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
         const int hb = (int)(item % hblocks);
         const int n_e = plan.counts[e];
         const int row0 = plan.offsets[e];
-        const float ad = glob[e * 3 + 2] * 256.0f;
+        const float ad = glob[e * 3 + 2];
         const int64_t tile0 = (int64_t)e * (H / 16) + hb * 2;
         const uint8_t* cb[2];
         const uint8_t* sb[2];
@@ -376,11 +411,11 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
         }
         for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
             const int nt_count = min(W16_MAX_NT, (n_e - n0 + 7) / 8);
-            const uint16_t* bptr[W16_MAX_NT];
+            const __half* bptr[W16_MAX_NT];
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
                 const int n = n0 + nt * 8 + g;
-                bptr[nt] = (nt < nt_count && n < n_e) ? A2 + (int64_t)(row0 + n) * I : nullptr;
+                bptr[nt] = (nt < nt_count && n < n_e) ? A16 + (int64_t)(row0 + n) * I : nullptr;
             }
             float acc[2][W16_MAX_NT][4] = {};
             if (!w16_stream(ring, cb, sb, chunks, bptr, nt_count, acc, err)) return;
@@ -392,7 +427,7 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
                     const int n = n0 + nt * 8 + 2 * c + j;
                     if (n < n_e) {
                         const int row = row0 + n;
-                        const float w = plan.wts[plan.pair_of_row[row]] * ad;
+                        const float w = plan.wts[plan.pair_of_row[row]] * ad * a_inv[row];
 #pragma unroll
                         for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -408,6 +443,11 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
 }  // namespace
 
 size_t w4a16_packed_size(int E, int H, int I) { return (size_t)w16_layout(E, H, I).total; }
+
+size_t w4a16_scratch_size(int T, int H, int I, int k) {
+    return (size_t)(align256((int64_t)T * H * 2) + align256((int64_t)T * 4) + align256((int64_t)T * k * I * 2) +
+                    align256((int64_t)T * k * 4));
+}
 
 nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream) {
     const int E = w.E, H = w.H, I = w.I;
@@ -435,26 +475,37 @@ nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed
 }
 
 nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T, int H, int I, int E, int k,
-                                   const RoutingPlan& plan, uint16_t* A2, float* Y, cudaStream_t stream,
-                                   cudaEvent_t mid_event) {
+                                   const RoutingPlan& plan, uint16_t* A2, float* Y, void* scratch,
+                                   cudaStream_t stream, cudaEvent_t mid_event) {
     const W16Layout L = w16_layout(E, H, I);
     const uint8_t* p = static_cast<const uint8_t*>(packed);
+    uint8_t* sc = static_cast<uint8_t*>(scratch);
+    __half* x16 = reinterpret_cast<__half*>(sc);
+    float* x_inv = reinterpret_cast<float*>(sc + align256((int64_t)T * H * 2));
+    __half* a16 = reinterpret_cast<__half*>(sc + align256((int64_t)T * H * 2) + align256((int64_t)T * 4));
+    float* a_inv = reinterpret_cast<float*>(sc + align256((int64_t)T * H * 2) + align256((int64_t)T * 4) +
+                                            align256((int64_t)T * k * I * 2));
+    const int64_t P = (int64_t)T * k;
     // experts with rows <= min(E, T*k): grids cover that bound; warps loop over
     // the (expert, row block) items the device-side active list holds
-    const int64_t max_active = std::min<int64_t>(E, (int64_t)T * k);
-    const int64_t max_ctas = (int64_t)num_sms() * 3;
+    const int64_t max_active = std::min<int64_t>(E, P);
+    const int64_t max_ctas = (int64_t)num_sms() * 4;
     int32_t* err = device_error_word();
     NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));
     NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_down, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));
+    k_rows_to_f16<<<(unsigned)ceil_div(T, 8), 256, 0, stream>>>(x, T, H, x16, x_inv);
+    NVFP4MOE_CHECK_LAUNCH("w4a16 activation conversion");
     {
         const int64_t ctas = std::min<int64_t>(ceil_div(max_active * (I / 16), W16_WARPS), max_ctas);
-        k_w16_gateup<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(x, p, L, H, I, k, plan, A2, err);
+        k_w16_gateup<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(x16, x_inv, p, L, H, I, k, plan, A2, err);
         NVFP4MOE_CHECK_LAUNCH("w4a16 gate/up kernel");
     }
     if (mid_event) cudaEventRecord(mid_event, stream);
+    k_rows_to_f16<<<(unsigned)ceil_div(P, 8), 256, 0, stream>>>(A2, P, I, a16, a_inv);
+    NVFP4MOE_CHECK_LAUNCH("w4a16 intermediate conversion");
     {
         const int64_t ctas = std::min<int64_t>(ceil_div(max_active * (H / 32), W16_WARPS), max_ctas);
-        k_w16_down<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(p, L, H, I, plan, A2, Y, err);
+        k_w16_down<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(p, L, H, I, plan, a16, a_inv, Y, err);
         NVFP4MOE_CHECK_LAUNCH("w4a16 down kernel");
     }
     return NVFP4MOE_OK;
