@@ -35,7 +35,8 @@ namespace nvfp4moe {
 namespace {
 
 constexpr int W16_WARPS = 4;
-constexpr int W16_MAX_NT = 4;  // n-tiles (of 8 tokens) per pass over the weights
+constexpr int W16_MAX_NT = 2;  // n-tiles (of 8 tokens) per pass over the weights
+constexpr int W16_MIN_CTAS = 5;  // CTAs per SM the register budget is sized for
 
 struct W16Layout {
     int64_t gu_codes, gu_scales, d_codes, d_scales, globals, total;
@@ -322,7 +323,7 @@ __device__ __forceinline__ Ring make_ring(uint8_t* smem) {
 // ---------------------------------------------------------------------------
 // gate/up GEMM + SwiGLU: warps loop over (active expert, 16 intermediates)
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(W16_WARPS * 32)
+__global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
     k_w16_gateup(const __half* __restrict__ x16, const float* __restrict__ x_inv, const uint8_t* __restrict__ packed,
                  W16Layout L, int H, int I, int k, RoutingPlan plan, uint16_t* __restrict__ A2, int32_t* err) {
     extern __shared__ __align__(128) uint8_t w16_smem[];
@@ -383,7 +384,7 @@ __global__ void __launch_bounds__(W16_WARPS * 32)
 // ---------------------------------------------------------------------------
 // down GEMM x routing weight: warps loop over (active expert, 32 hidden rows)
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(W16_WARPS * 32)
+__global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
     k_w16_down(const uint8_t* __restrict__ packed, W16Layout L, int H, int I, RoutingPlan plan,
                const __half* __restrict__ A16, const float* __restrict__ a_inv, float* __restrict__ Y, int32_t* err) {
     extern __shared__ __align__(128) uint8_t w16_smem[];
@@ -489,7 +490,7 @@ nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T,
     // experts with rows <= min(E, T*k): grids cover that bound; warps loop over
     // the (expert, row block) items the device-side active list holds
     const int64_t max_active = std::min<int64_t>(E, P);
-    const int64_t max_ctas = (int64_t)num_sms() * 4;
+    const int64_t max_ctas = (int64_t)num_sms() * W16_MIN_CTAS;
     int32_t* err = device_error_word();
     NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));
     NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_down, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));

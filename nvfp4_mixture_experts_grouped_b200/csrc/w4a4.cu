@@ -155,20 +155,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int it = 0;
-            // L2 prefetch cursor, PREFETCH_AHEAD k-stages in front of the loads, so
-            // that weight tiles coming from HBM are L2 hits when the ring loads them
+            // L2 prefetch cursor, PREFETCH_AHEAD k-stages in front of the loads.  Only
+            // the weight tiles of an expert's first M-tile are prefetched: they are
+            // the HBM misses; every other tile is an L2 hit, where a prefetch would
+            // only spend L2 bandwidth.
             int pf_tile = blockIdx.x, pf_ks = 0;
             auto prefetch_next = [&]() {
                 if (pf_tile >= total) return;
                 const int pm = pf_tile / p.n_ntiles, pn = pf_tile - pm * p.n_ntiles;
                 const int4 pti = p.tiles[pm];
-                const int64_t pb = (int64_t)pti.x * p.b_rows_per_expert + (int64_t)pn * BN;
-                const int n64 = min(4, k64_total - pf_ks * 4);
-                tc::tma_prefetch_2d(&tmA, pf_ks * 128, pti.y);
-                tc::tma_prefetch_2d(&tmB, pf_ks * 128, (int32_t)pb);
-                tc::bulk_prefetch_l2(p.sfa + ((int64_t)(pti.y / 128) * k64_total + pf_ks * 4) * 512, n64 * 512);
-                tc::bulk_prefetch_l2(p.sfb + ((pb / 128) * k64_total + pf_ks * 4) * 512, n64 * 512);
-                tc::bulk_prefetch_l2(p.sfb + ((pb / 128 + 1) * k64_total + pf_ks * 4) * 512, n64 * 512);
+                if (pti.w == 0) {
+                    const int64_t pb = (int64_t)pti.x * p.b_rows_per_expert + (int64_t)pn * BN;
+                    const int n64 = min(4, k64_total - pf_ks * 4);
+                    tc::tma_prefetch_2d(&tmB, pf_ks * 128, (int32_t)pb);
+                    tc::bulk_prefetch_l2(p.sfb + ((pb / 128) * k64_total + pf_ks * 4) * 512, n64 * 512);
+                    tc::bulk_prefetch_l2(p.sfb + ((pb / 128 + 1) * k64_total + pf_ks * 4) * 512, n64 * 512);
+                }
                 if (++pf_ks == ks_count) {
                     pf_ks = 0;
                     pf_tile += gridDim.x;
