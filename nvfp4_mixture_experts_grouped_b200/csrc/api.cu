@@ -132,7 +132,7 @@ static ForwardLayout forward_layout(nvfp4moe_mode mode, int64_t T, int64_t H, in
         L.a2s = take(L.rows_max * I / 16);
         L.a2bf = -1;
         L.y = take(L.rows_max * H * 2);          // FP16 staged rows
-        L.ys = take(L.rows_max * (H / 128) * 4);  // their power-of-two scales
+        L.ys = take(L.rows_max * (H / 64) * 4);  // their power-of-two scales
     } else {
         L.a1c = L.a1s = L.a2c = L.a2s = L.ys = -1;
         L.a2bf = take(L.rows_max * I * 2);

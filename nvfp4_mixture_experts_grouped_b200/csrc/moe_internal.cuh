@@ -49,7 +49,7 @@ nvfp4moe_status launch_quantize_linear(const uint16_t* x, int64_t M, int64_t K, 
                                        uint8_t* scales, cudaStream_t stream);
 nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H, float gs, uint8_t* codes,
                                         uint8_t* scales, const int32_t* row_of_pair, int k, cudaStream_t stream);
-// Y staged as FP16 rows with a power-of-two scale per 128 columns (y_scale != nullptr,
+// Y staged as FP16 rows with a power-of-two scale per 64 columns (y_scale != nullptr,
 // W4A4) or as FP32 rows (y_scale == nullptr, W4A16).
 nvfp4moe_status launch_combine(const void* Y, const float* y_scale, const int32_t* row_of_pair, int64_t T, int H,
                                int k, void* out, bool out_f32, cudaStream_t stream);

@@ -216,7 +216,7 @@ nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H,
 // ---------------------------------------------------------------------------
 // 5. weighted un-permute: out[t] = sum_j Y[row_of_pair(t, j)] (routing weights
 //    already applied by the down GEMM), FP32 in slot order, one rounding.
-//    Y is FP16 with a power-of-two scale per 128 columns (W4A4) or FP32 (W4A16).
+//    Y is FP16 with a power-of-two scale per 64 columns (W4A4) or FP32 (W4A16).
 // ---------------------------------------------------------------------------
 template <bool Y_F16, bool OUT_F32>
 __global__ void __launch_bounds__(256)
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(256)
     for (int j = 0; j < k; ++j) {
         const int64_t row = __ldg(row_of_pair + t * k + j);
         if (Y_F16) {
-            const float s = __ldg(y_scale + row * (H / 128) + h8 / 128);
+            const float s = __ldg(y_scale + row * (H / 64) + h8 / 64);
             const uint4 v = __ldcs(reinterpret_cast<const uint4*>(static_cast<const __half*>(Yv) + row * H + h8));
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll

@@ -10,15 +10,18 @@
 //   warp 0      TMA producer: A/B code tiles (SWIZZLE_128B tensor maps, never
 //               multicast) and their block-scale atoms (1-D bulk copies) into a
 //               4-stage shared-memory ring guarded by mbarriers;
-//   warp 1      MMA issuer: copies the stage's scale factors into TMEM
-//               (tcgen05.cp 32x128b.warpx4) and issues four K=64 block-scaled
-//               MMAs per stage into a 128 x 256 FP32 TMEM accumulator;
-//   warps 2..5  epilogue: tcgen05.ld of their 32-lane quadrant, then
+//   warp 1      MMA issuer: four K=64 block-scaled MMAs per stage into a
+//               128 x 256 FP32 TMEM accumulator, nothing else (a tcgen05.cp
+//               costs the tensor pipe ~60-80 cycles whatever its size, so twelve
+//               scale copies per stage would cost more than the stage's MMAs);
+//   warps 18..21 scale warps: tcgen05.st of each stage's scale factors into the
+//               stage's TMEM scale columns, one warp per lane quadrant;
+//   warps 2..17 epilogue: tcgen05.ld of their 32-lane quadrant, then
 //               gate/up: SiLU(gate) * up and NVFP4 requantisation per 16 (the
 //                        down GEMM's A operand, written straight into its
 //                        block-scale layout);
 //               down:    x global scale x routing weight, per-pair rows staged
-//                        as FP16 with a power-of-two scale per 128 columns.
+//                        as FP16 with a power-of-two scale per 64 columns.
 // Rows of an expert are padded to 128 by the permutation, so an M-tile never
 // straddles two experts; padding rows are computed and never stored.
 #include <cuda.h>
@@ -45,11 +48,13 @@ constexpr int SFA_BYTES = BM * BK / 16;
 constexpr int SFB_BYTES = BN * BK / 16;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+static_assert(256 + STAGES * 48 <= 512, "accumulator + per-slot scale columns must fit the TMEM allocation");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_SF = 256;      // scale-factor columns after the 256 accumulator columns
-constexpr uint32_t TM_SF_STRIDE = 48;  // per buffer: 16 (A: 4 k-steps x 4) + 32 (B: 4 x 8)
-constexpr int EPI_WARPS = 8;  // two warps per TMEM lane quadrant, each on half the columns
-constexpr int THREADS = 64 + EPI_WARPS * 32;
+constexpr uint32_t TM_SF_STRIDE = 48;  // per ring slot: 16 (A: 4 k-steps x 4) + 32 (B: 4 x 8)
+constexpr int EPI_WARPS = 16;  // four warps per TMEM lane quadrant, each on a quarter of the columns
+constexpr int SF_WARPS = 4;    // one warp per TMEM lane quadrant writes the scale factors
+constexpr int THREADS = (2 + EPI_WARPS + SF_WARPS) * 32;
 
 enum { EPI_GATEUP = 0, EPI_DOWN = 1 };
 
@@ -84,7 +89,7 @@ struct GemmParams {
     uint8_t* out_sf;         // gate/up: intermediate scales, atom layout
     int out_k;               // gate/up: I
     __half* Y;               // down: [rows, H] FP16 staged rows
-    float* y_scale;          // down: [rows, H / 128] power-of-two scale of each 128 staged columns
+    float* y_scale;          // down: [rows, H / 64] power-of-two scale of each 64 staged columns
     int ldy;                 // down: H
     const float* wts;        // down: routing weight of each pair
     const int32_t* pair_of_row;
@@ -119,7 +124,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-    uint64_t* empty = full + STAGES;
+    uint64_t* sf_ready = full + STAGES;
+    uint64_t* empty = sf_ready + STAGES;
     uint64_t* acc_full = empty + STAGES;
     uint64_t* acc_empty = acc_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
@@ -128,6 +134,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&sf_ready[s], SF_WARPS);
             tc::mbar_init(&empty[s], 1);
         }
         tc::mbar_init(acc_full, 1);
@@ -203,6 +210,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Scale factors are already in TMEM (the scale warps put them there), so
+        // this thread issues nothing but the block-scaled MMAs.
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_mxf4nvf4(BM, BN);
             int it = 0, tl = 0;
@@ -212,18 +221,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int ks = 0; ks < ks_count; ++ks, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!tc::mbar_wait(&full[s], ph, p.err)) goto done;
+                    if (!tc::mbar_wait(&sf_ready[s], ph, p.err)) goto done;
                     tc::tc_fence_after();
                     const int n64 = min(4, k64_total - ks * 4);
                     uint8_t* st = smem + s * STAGE_BYTES;
-                    const uint32_t sf_col = tmem + TM_SF + (uint32_t)(it & 1) * TM_SF_STRIDE;
-                    for (int j = 0; j < n64; ++j) {
-                        tc::tmem_cp_32x128_x4(sf_col + 4 * j, tc::desc_sf(st + A_BYTES + B_BYTES + j * 512));
-                        tc::tmem_cp_32x128_x4(sf_col + 16 + 8 * j,
-                                              tc::desc_sf(st + A_BYTES + B_BYTES + SFA_BYTES + j * 512));
-                        tc::tmem_cp_32x128_x4(sf_col + 16 + 8 * j + 4,
-                                              tc::desc_sf(st + A_BYTES + B_BYTES + SFA_BYTES + 2048 + j * 512));
-                    }
+                    const uint32_t sf_col = tmem + TM_SF + (uint32_t)s * TM_SF_STRIDE;
                     const uint64_t adesc = tc::desc_sw128(st);
                     const uint64_t bdesc = tc::desc_sw128(st + A_BYTES);
                     for (int j = 0; j < n64; ++j)
@@ -234,12 +236,48 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc::tc_commit(acc_full);
             }
         }
+    } else if (warp >= 2 + EPI_WARPS) {
+        // ------------------------------------------------------------ scale warps
+        // Warp w writes the scale factors of every stage into TMEM lane quadrant
+        // w % 4 with tcgen05.st, in the replicated atom layout the MMA reads: lane
+        // (32q + l), column c of an atom's 4 holds word c of the atom's 16-byte row
+        // l.  Each ring slot has its own scale columns, rewritten only after the
+        // slot's MMAs completed (the slot is refilled only after `empty`).
+        const int q = warp & 3;
+        const uint32_t t_q = tmem + ((uint32_t)(q * 32) << 16);
+        int it = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            for (int ks = 0; ks < ks_count; ++ks, ++it) {
+                const int s = it % STAGES;
+                const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                if (!tc::mbar_wait(&full[s], ph, p.err)) goto done;
+                const uint8_t* st = smem + s * STAGE_BYTES + A_BYTES + B_BYTES;
+                uint32_t v[48];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(st + j * 512 + lane * 16);
+                    const uint4 b0 = *reinterpret_cast<const uint4*>(st + SFA_BYTES + j * 512 + lane * 16);
+                    const uint4 b1 = *reinterpret_cast<const uint4*>(st + SFA_BYTES + 2048 + j * 512 + lane * 16);
+                    v[4 * j + 0] = a.x, v[4 * j + 1] = a.y, v[4 * j + 2] = a.z, v[4 * j + 3] = a.w;
+                    v[16 + 8 * j + 0] = b0.x, v[16 + 8 * j + 1] = b0.y, v[16 + 8 * j + 2] = b0.z, v[16 + 8 * j + 3] = b0.w;
+                    v[16 + 8 * j + 4] = b1.x, v[16 + 8 * j + 5] = b1.y, v[16 + 8 * j + 6] = b1.z, v[16 + 8 * j + 7] = b1.w;
+                }
+                const uint32_t col = t_q + TM_SF + (uint32_t)s * TM_SF_STRIDE;
+                tc::tmem_st16(col, v);
+                tc::tmem_st16(col + 16, v + 16);
+                tc::tmem_st16(col + 32, v + 32);
+                tc::tmem_st_wait();
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&sf_ready[s]);
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue
-        // warps 2..9: warp w reads TMEM lane quadrant w % 4 (the hardware rule) and
-        // column half (w - 2) / 4 of the tile.
+        // warps 2..17: warp w reads TMEM lane quadrant w % 4 (the hardware rule) and
+        // column quarter (w - 2) / 4 of the tile.
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;
+        const int quarter = (warp - 2) >> 2;
         const int r_in = q * 32 + lane;
         const uint32_t t_row = tmem + ((uint32_t)(q * 32) << 16);
         int tl = 0;
@@ -251,15 +289,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!tc::mbar_wait(acc_full, (uint32_t)tl & 1u, p.err)) goto done;
             tc::tc_fence_after();
             if (EPI == EPI_GATEUP) {
-                // columns [0,128) gate, [128,256) up, for intermediates n*128 .. n*128+127.
-                // All of this warp's accumulator values are pulled into registers first
-                // and the accumulator is released before any arithmetic, so the MMA
-                // warp only waits for the TMEM reads.
-                const int i0 = n * (BN / 2) + half * 64;  // first intermediate of this warp
-                float gv[64], uv[64];
+                // columns [0,128) gate, [128,256) up, for intermediates n*128 .. n*128+127;
+                // this warp: 32 intermediates.  All of its accumulator values are read
+                // and the accumulator released before the arithmetic, so the MMA warp
+                // only waits for the TMEM reads.
+                const int i0 = n * (BN / 2) + quarter * 32;
+                float gv[32], uv[32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    tc::tmem_ld16x2(t_row + half * 64 + 16 * c, t_row + 128 + half * 64 + 16 * c, gv + 16 * c,
+                for (int c = 0; c < 2; ++c)
+                    tc::tmem_ld16x2(t_row + quarter * 32 + 16 * c, t_row + 128 + quarter * 32 + 16 * c, gv + 16 * c,
                                     uv + 16 * c);
                 tc::tc_fence_before();
                 __syncwarp();
@@ -268,31 +306,29 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const float ag = p.globals[ti.x * 3 + 0] * p.act_global;
                     const float au = p.globals[ti.x * 3 + 1] * p.act_global;
                     const int nkb = p.out_k / 16;
-                    uint32_t codes[8], sfw = 0;
+                    uint32_t codes[4], sfw = 0;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < 2; ++c) {
                         float a[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) a[i] = silu_fast(gv[16 * c + i] * ag) * (uv[16 * c + i] * au);
                         const uint32_t sf = requant_block16(a, p.act_global, codes[2 * c], codes[2 * c + 1]);
                         sfw |= sf << (8 * c);
                     }
-                    uint4* dst = reinterpret_cast<uint4*>(p.out_codes + row * (p.out_k / 2) + i0 / 2);
-                    dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                    dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-                    // the 4 block scales of this row are 4 consecutive bytes of one atom row
-                    *reinterpret_cast<uint32_t*>(p.out_sf + sf_atom_offset(row, i0 / 16, nkb)) = sfw;
+                    *reinterpret_cast<uint4*>(p.out_codes + row * (p.out_k / 2) + i0 / 2) =
+                        make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                    // the 2 block scales of this row are 2 consecutive bytes of one atom row
+                    *reinterpret_cast<uint16_t*>(p.out_sf + sf_atom_offset(row, i0 / 16, nkb)) = (uint16_t)sfw;
                 }
             } else {
                 // y = acc * global * routing weight, staged as FP16 with one power-of-two
-                // scale per (row, 128 columns).  The warp's 128 accumulator columns are
-                // read into registers and released first; then the max picks the
-                // scale and y / scale is written (exact power-of-two scaling, one FP16
-                // rounding).
-                float v[128];
-                const uint32_t t_col = t_row + half * 128;
+                // scale per (row, 64 columns).  The warp's 64 accumulator columns are
+                // read and released first; then the max picks the scale and y / scale
+                // is written (exact power-of-two scaling, one FP16 rounding).
+                float v[64];
+                const uint32_t t_col = t_row + quarter * 64;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tc::tmem_ld16x2(t_col + 32 * c, t_col + 32 * c + 16, v + 32 * c, v + 32 * c + 16);
+                for (int c = 0; c < 2; ++c) tc::tmem_ld16x2(t_col + 32 * c, t_col + 32 * c + 16, v + 32 * c, v + 32 * c + 16);
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(acc_empty);
@@ -300,16 +336,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const float f = p.globals[ti.x * 3 + 2] * p.act_global * p.wts[p.pair_of_row[row]];
                     float amax = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < 128; ++i) amax = fmaxf(amax, fabsf(v[i]));
+                    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
                     amax *= fabsf(f);
                     // scale = 2^(e - 14) with amax in [2^e, 2^(e+1)): staged magnitudes stay below 2^15
                     int e = 0;
                     if (amax > 0.0f && isfinite(amax)) e = ((__float_as_uint(amax) >> 23) & 0xFF) - 127;
                     e = max(min(e - 14, 100), -100);
                     const float g = ldexpf(f, -e);
-                    uint4* dst = reinterpret_cast<uint4*>(p.Y + row * p.ldy + (int64_t)n * BN + half * 128);
+                    uint4* dst = reinterpret_cast<uint4*>(p.Y + row * p.ldy + (int64_t)n * BN + quarter * 64);
 #pragma unroll
-                    for (int q8 = 0; q8 < 16; ++q8) {
+                    for (int q8 = 0; q8 < 8; ++q8) {
                         uint32_t pk[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
@@ -318,7 +354,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         }
                         dst[q8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     }
-                    p.y_scale[row * (p.ldy / 128) + n * 2 + half] = ldexpf(1.0f, e);
+                    p.y_scale[row * (p.ldy / 64) + n * 4 + quarter] = ldexpf(1.0f, e);
                 }
             }
         }
