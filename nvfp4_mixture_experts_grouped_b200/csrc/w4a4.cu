@@ -324,7 +324,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 // y = acc * global * routing weight, staged as FP16 with one power-of-two
                 // scale per (row, 64 columns).  The warp's 64 accumulator columns are
                 // read and released first; then the max picks the scale and y / scale
-                // is written (exact power-of-two scaling, one FP16 rounding).
+                // is converted (exact power-of-two scaling, one FP16 rounding).
                 float v[64];
                 const uint32_t t_col = t_row + quarter * 64;
 #pragma unroll
@@ -332,29 +332,53 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(acc_empty);
-                if (valid) {
-                    const float f = p.globals[ti.x * 3 + 2] * p.act_global * p.wts[p.pair_of_row[row]];
-                    float amax = 0.0f;
+                // rows past the tile's valid count hold padding: weight 0, never stored
+                const float f = valid ? p.globals[ti.x * 3 + 2] * p.act_global * p.wts[p.pair_of_row[row]] : 0.0f;
+                float amax = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
-                    amax *= fabsf(f);
-                    // scale = 2^(e - 14) with amax in [2^e, 2^(e+1)): staged magnitudes stay below 2^15
-                    int e = 0;
-                    if (amax > 0.0f && isfinite(amax)) e = ((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-                    e = max(min(e - 14, 100), -100);
-                    const float g = ldexpf(f, -e);
-                    uint4* dst = reinterpret_cast<uint4*>(p.Y + row * p.ldy + (int64_t)n * BN + quarter * 64);
+                for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
+                amax *= fabsf(f);
+                // scale = 2^(e - 14) with amax in [2^e, 2^(e+1)): staged magnitudes stay below 2^15
+                int e = 0;
+                if (amax > 0.0f && isfinite(amax)) e = ((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+                e = max(min(e - 14, 100), -100);
+                const float g = ldexpf(f, -e);
+                // pk: this row's 64 FP16 values as 8 chunks of 16 bytes (4 words each)
+                uint32_t pk[32];
 #pragma unroll
-                    for (int q8 = 0; q8 < 8; ++q8) {
-                        uint32_t pk[4];
+                for (int i = 0; i < 32; ++i) {
+                    __half2 b = __floats2half2_rn(v[2 * i] * g, v[2 * i + 1] * g);
+                    pk[i] = *reinterpret_cast<uint32_t*>(&b);
+                }
+                if (valid) p.y_scale[row * (p.ldy / 64) + n * 4 + quarter] = ldexpf(1.0f, e);
+                // Transpose the 8 x 8 chunk matrix of each group of 8 lanes (rows), a
+                // butterfly over lane bits 1, 2, 4: afterwards lane 8G + c holds chunk c
+                // of the group's rows 8G + 0..7, so one store instruction writes 4 whole
+                // 128-byte row segments instead of 32 scattered 16-byte pieces.
+                const int c8 = lane & 7, g8 = lane >> 3;
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            __half2 b = __floats2half2_rn(v[8 * q8 + 2 * i] * g, v[8 * q8 + 2 * i + 1] * g);
-                            pk[i] = *reinterpret_cast<uint32_t*>(&b);
+                for (int b = 0; b < 3; ++b) {
+                    const int m = 1 << b;
+                    const bool hi = (c8 & m) != 0;
+#pragma unroll
+                    for (int k0 = 0; k0 < 8; ++k0) {
+                        if (k0 & m) continue;
+                        const int k1 = k0 | m;
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const uint32_t send = hi ? pk[4 * k0 + w] : pk[4 * k1 + w];
+                            const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
+                            if (hi) pk[4 * k0 + w] = recv;
+                            else pk[4 * k1 + w] = recv;
                         }
-                        dst[q8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     }
-                    p.y_scale[row * (p.ldy / 64) + n * 4 + quarter] = ldexpf(1.0f, e);
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int r_j = q * 32 + g8 * 8 + j;
+                    if (r_j < ti.z)
+                        *reinterpret_cast<uint4*>(p.Y + ((int64_t)ti.y + r_j) * p.ldy + (int64_t)n * BN + quarter * 64 +
+                                                  c8 * 8) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
                 }
             }
         }
