@@ -11,7 +11,8 @@ namespace nvfp4moe {
 
 constexpr int PERM_CHUNK = 256;  // tokens per permutation chunk (one CTA)
 constexpr int PERM_WARPS = PERM_CHUNK / 32;
-constexpr int MTILE = 128;       // rows of one tcgen05 M-tile
+constexpr int MTILE = 128;       // rows of one tcgen05 M-tile per CTA (the row padding of the W4A4 path)
+constexpr int PAIR_ROWS = 256;   // rows of one tile of a CTA pair (the tile list's unit)
 
 __device__ __forceinline__ int64_t round_up_dev(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
@@ -25,7 +26,7 @@ struct RoutingPlan {
     int32_t* pad_offsets;   // [E+1] row offsets with every segment padded to `pad`
     int32_t* row_of_pair;   // [T*k]
     int32_t* pair_of_row;   // [rows_max]
-    int4* tiles;            // [max_tiles] {expert, first padded row, valid rows, m-tile index}
+    int4* tiles;            // [max_tiles] {expert, first padded row, valid rows (<= 256), tile index in expert}
     int32_t* n_tiles;       // [1]
     int32_t* active;        // [E] experts with at least one row
     int32_t* n_active;      // [1]

@@ -33,7 +33,8 @@ __global__ void __launch_bounds__(PERM_CHUNK)
 }
 
 // ---------------------------------------------------------------------------
-// 2. per-expert scan over chunks, expert offsets, M-tile list, active list
+// 2. per-expert scan over chunks, expert offsets, tile list (256-row pair tiles
+//    of the tcgen05 path), active list
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int& total) {
     // blockDim.x == 1024
@@ -69,7 +70,7 @@ __global__ void __launch_bounds__(1024)
     const int padded = e < E ? (int)round_up_dev(cnt, pad) : 0;
     int ptotal;
     const int poff = block_exclusive_scan(padded, s_tmp, ptotal);
-    const int tiles = e < E ? (cnt + MTILE - 1) / MTILE : 0;
+    const int tiles = e < E ? (cnt + PAIR_ROWS - 1) / PAIR_ROWS : 0;
     int ttotal;
     const int toff = block_exclusive_scan(tiles, s_tmp, ttotal);
     int atotal;
@@ -81,8 +82,8 @@ __global__ void __launch_bounds__(1024)
         for (int j = 0; j < tiles; ++j) {
             int4 ti;
             ti.x = e;
-            ti.y = poff + j * MTILE;
-            ti.z = min(MTILE, cnt - j * MTILE);
+            ti.y = poff + j * PAIR_ROWS;
+            ti.z = min(PAIR_ROWS, cnt - j * PAIR_ROWS);
             ti.w = j;
             plan.tiles[toff + j] = ti;
         }

@@ -6,14 +6,18 @@
 // W4A4 NVFP4 on native FP4 tensor cores) and "Why a unit activation scale".
 // Expert MLP: "MiMo-V2.6-Flash -- REAP-50", "Pruning Method" 1.
 //
-// One persistent kernel per projection, one CTA per SM, 128 x 256 output tiles:
-//   warp 0      TMA producer: A/B code tiles (SWIZZLE_128B tensor maps, never
-//               multicast) and their block-scale atoms (1-D bulk copies) into a
-//               4-stage shared-memory ring guarded by mbarriers;
-//   warp 1      MMA issuer: four K=64 block-scaled MMAs per stage into a
-//               128 x 256 FP32 TMEM accumulator, nothing else (a tcgen05.cp
-//               costs the tensor pipe ~60-80 cycles whatever its size, so twelve
-//               scale copies per stage would cost more than the stage's MMAs);
+// One persistent kernel per projection.  CTA pairs (2-CTA clusters, one CTA per
+// SM) compute 256 x 256 output tiles with the pair form of the MMA (cta_group::2):
+// each CTA loads half of A's rows and half of B's rows, so a CTA moves 2/3 of the
+// operand bytes a single-CTA 128 x 256 tile needs for the same FLOPs.  Per CTA:
+//   warp 0      TMA producer: its A/B code half-tiles (SWIZZLE_128B tensor maps,
+//               never multicast) and block-scale atoms (1-D bulk copies) into a
+//               5-stage shared-memory ring guarded by mbarriers;
+//   warp 1      (even CTA) MMA issuer: four K=64 block-scaled M=256 x N=256 MMAs
+//               per stage into the pair's FP32 TMEM accumulators, nothing else
+//               (a tcgen05.cp costs the tensor pipe ~60-80 cycles whatever its
+//               size, so twelve scale copies per stage would cost more than the
+//               stage's MMAs);
 //   warps 18..21 scale warps: tcgen05.st of each stage's scale factors into the
 //               stage's TMEM scale columns, one warp per lane quadrant;
 //   warps 2..17 epilogue: tcgen05.ld of their 32-lane quadrant, then
@@ -22,8 +26,9 @@
 //                        block-scale layout);
 //               down:    x global scale x routing weight, per-pair rows staged
 //                        as FP16 with a power-of-two scale per 64 columns.
-// Rows of an expert are padded to 128 by the permutation, so an M-tile never
-// straddles two experts; padding rows are computed and never stored.
+// Rows of an expert are padded to 128 by the permutation and its rows are cut
+// into 256-row pair tiles, so a tile never straddles two experts; padding rows
+// are computed and never stored.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -39,15 +44,18 @@ namespace nvfp4moe {
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 256;  // BK in elements (128 bytes of codes)
-constexpr int STAGES = 4;
-constexpr int PREFETCH_AHEAD = 8;  // k-stages of L2 prefetch in front of the shared-memory ring
+// A CTA pair computes a 256 x 256 tile: each CTA holds 128 rows of A, 128 rows
+// (N) of B, the scale factors of its A rows and of all 256 B rows.
+constexpr int BM = 128, BN = 256, BK = 256;  // BM per CTA, BN per pair, BK in elements (128 bytes of codes)
+constexpr int STAGES = 5;
 constexpr int A_BYTES = BM * BK / 2;
-constexpr int B_BYTES = BN * BK / 2;
+constexpr int B_BYTES = (BN / 2) * BK / 2;
 constexpr int SFA_BYTES = BM * BK / 16;
 constexpr int SFB_BYTES = BN * BK / 16;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+static_assert(SMEM_BYTES <= 232448, "shared-memory ring above the 227 KB a CTA may use");
+static_assert(STAGE_BYTES % 1024 == 0, "128-byte-swizzled operand tiles need 1024-byte alignment");
 static_assert(256 + STAGES * 48 <= 512, "accumulator + per-slot scale columns must fit the TMEM allocation");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_SF = 256;      // scale-factor columns after the 256 accumulator columns
@@ -119,26 +127,27 @@ __device__ __forceinline__ uint32_t requant_block16(const float* x, float gs, ui
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     k_w4a4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-    uint64_t* sf_ready = full + STAGES;
-    uint64_t* empty = sf_ready + STAGES;
-    uint64_t* acc_full = empty + STAGES;
-    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* sf_ready = full + STAGES;   // even CTA only: both CTAs' scale warps
+    uint64_t* empty = sf_ready + STAGES;  // both CTAs: the even CTA's MMA commits
+    uint64_t* acc_full = empty + STAGES;  // both CTAs: the even CTA's MMA commits
+    uint64_t* acc_empty = acc_full + 1;   // even CTA only: both CTAs' epilogue warps
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
 
+    const uint32_t rank = tc::cluster_ctarank();  // 0: issues the MMAs of the pair
     const int warp = warp_id(), lane = lane_id();
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             tc::mbar_init(&full[s], 1);
-            tc::mbar_init(&sf_ready[s], SF_WARPS);
+            tc::mbar_init(&sf_ready[s], 2 * SF_WARPS);
             tc::mbar_init(&empty[s], 1);
         }
         tc::mbar_init(acc_full, 1);
-        tc::mbar_init(acc_empty, EPI_WARPS);
+        tc::mbar_init(acc_empty, 2 * EPI_WARPS);
         tc::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -146,82 +155,77 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::prefetch_tmap(&tmB);
     }
     if (warp == 1) {
-        tc::tmem_alloc(tmem_slot, TMEM_COLS);
-        tc::tmem_relinquish();
+        tc::tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tc::tmem_relinquish_pair();
     }
+    // barriers initialised and TMEM allocated in both CTAs before either uses the other's
     tc::tc_fence_before();
-    __syncthreads();
+    tc::cluster_sync();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
     const int total = p.n_tiles[0] * p.n_ntiles;
     const int k64_total = p.K / 64;
     const int ks_count = (k64_total + 3) / 4;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        // This CTA's half of the pair tile: A rows [128 rank, +128) and B (N) rows
+        // [128 rank, +128); the scale factors of its A rows and of all 256 N rows.
         if (lane == 0) {
+            // No L2 prefetch: every TMA instruction costs this thread ~85 cycles of
+            // issue (a prefetch ~270), and with five copies per stage the issue
+            // time, not the memory system, would bound the MMA rate.
             int it = 0;
-            // L2 prefetch cursor, PREFETCH_AHEAD k-stages in front of the loads.  Only
-            // the weight tiles of an expert's first M-tile are prefetched: they are
-            // the HBM misses; every other tile is an L2 hit, where a prefetch would
-            // only spend L2 bandwidth.
-            int pf_tile = blockIdx.x, pf_ks = 0;
-            auto prefetch_next = [&]() {
-                if (pf_tile >= total) return;
-                const int pm = pf_tile / p.n_ntiles, pn = pf_tile - pm * p.n_ntiles;
-                const int4 pti = p.tiles[pm];
-                if (pti.w == 0) {
-                    const int64_t pb = (int64_t)pti.x * p.b_rows_per_expert + (int64_t)pn * BN;
-                    const int n64 = min(4, k64_total - pf_ks * 4);
-                    tc::tma_prefetch_2d(&tmB, pf_ks * 128, (int32_t)pb);
-                    tc::bulk_prefetch_l2(p.sfb + ((pb / 128) * k64_total + pf_ks * 4) * 512, n64 * 512);
-                    tc::bulk_prefetch_l2(p.sfb + ((pb / 128 + 1) * k64_total + pf_ks * 4) * 512, n64 * 512);
-                }
-                if (++pf_ks == ks_count) {
-                    pf_ks = 0;
-                    pf_tile += gridDim.x;
-                }
-            };
-            for (int i = 0; i < PREFETCH_AHEAD; ++i) prefetch_next();
-            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            for (int tile = pair; tile < total; tile += n_pairs) {
                 const int m = tile / p.n_ntiles, n = tile - m * p.n_ntiles;
                 const int4 ti = p.tiles[m];
-                const int64_t b_row0 = (int64_t)ti.x * p.b_rows_per_expert + (int64_t)n * BN;
+                // rows of this CTA's half that hold pairs; none in the odd half of an
+                // expert's last pair tile when its count leaves it empty (then its A
+                // operand is not loaded: those accumulator rows are never stored)
+                const bool a_live = ti.z > BM * (int)rank;
+                const int a_row = ti.y + BM * (int)rank;
+                const int64_t b_tile0 = (int64_t)ti.x * p.b_rows_per_expert + (int64_t)n * BN;
                 for (int ks = 0; ks < ks_count; ++ks, ++it) {
-                    prefetch_next();
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!tc::mbar_wait(&empty[s], ph ^ 1u, p.err)) goto done;
+                    if (!tc::mbar_wait<true>(&empty[s], ph ^ 1u, p.err)) goto done;
                     const int n64 = min(4, k64_total - ks * 4);
                     uint8_t* st = smem + s * STAGE_BYTES;
-                    tc::mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES + 3 * n64 * 512);
-                    tc::tma_load_2d(st, &tmA, ks * 128, ti.y, &full[s]);
-                    tc::tma_load_2d(st + A_BYTES, &tmB, ks * 128, (int32_t)b_row0, &full[s]);
-                    const uint8_t* sfa = p.sfa + ((int64_t)(ti.y / 128) * k64_total + ks * 4) * 512;
-                    tc::bulk_load(st + A_BYTES + B_BYTES, sfa, n64 * 512, &full[s]);
+                    tc::mbar_arrive_expect_tx(&full[s], B_BYTES + 2 * n64 * 512 + (a_live ? A_BYTES + n64 * 512 : 0));
+                    if (a_live) {
+                        tc::tma_load_2d(st, &tmA, ks * 128, a_row, &full[s]);
+                        const uint8_t* sfa = p.sfa + ((int64_t)(a_row / 128) * k64_total + ks * 4) * 512;
+                        tc::bulk_load(st + A_BYTES + B_BYTES, sfa, n64 * 512, &full[s]);
+                    }
+                    tc::tma_load_2d(st + A_BYTES, &tmB, ks * 128, (int32_t)(b_tile0 + BM * rank), &full[s]);
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
-                        const uint8_t* sfb = p.sfb + ((b_row0 / 128 + r) * k64_total + ks * 4) * 512;
+                        const uint8_t* sfb = p.sfb + ((b_tile0 / 128 + r) * k64_total + ks * 4) * 512;
                         tc::bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES + r * 2048, sfb, n64 * 512, &full[s]);
                     }
                 }
             }
+            // wait for the MMA's release of every slot still in use, so that no
+            // completion signal of the other CTA lands after this CTA has finished
+            for (int i = it; i < it + STAGES; ++i)
+                if (!tc::mbar_wait<true>(&empty[i % STAGES], ((uint32_t)(i / STAGES) & 1u) ^ 1u, p.err)) goto done;
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // Scale factors are already in TMEM (the scale warps put them there), so
-        // this thread issues nothing but the block-scaled MMAs.
-        if (lane == 0) {
-            const uint32_t idesc = tc::idesc_mxf4nvf4(BM, BN);
+        // One thread of the even CTA issues the pair's M=256 x N=256 MMAs; scale
+        // factors are already in both CTAs' TMEM (the scale warps put them there).
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = tc::idesc_mxf4nvf4(2 * BM, BN);
             int it = 0, tl = 0;
-            for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tl) {
-                if (!tc::mbar_wait(acc_empty, ((uint32_t)tl & 1u) ^ 1u, p.err)) goto done;
+            for (int tile = pair; tile < total; tile += n_pairs, ++tl) {
+                if (!tc::mbar_wait<true>(acc_empty, ((uint32_t)tl & 1u) ^ 1u, p.err)) goto done;
                 tc::tc_fence_after();
                 for (int ks = 0; ks < ks_count; ++ks, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!tc::mbar_wait(&sf_ready[s], ph, p.err)) goto done;
+                    if (!tc::mbar_wait<true>(&sf_ready[s], ph, p.err)) goto done;
                     tc::tc_fence_after();
                     const int n64 = min(4, k64_total - ks * 4);
                     uint8_t* st = smem + s * STAGE_BYTES;
@@ -229,24 +233,25 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint64_t adesc = tc::desc_sw128(st);
                     const uint64_t bdesc = tc::desc_sw128(st + A_BYTES);
                     for (int j = 0; j < n64; ++j)
-                        tc::mma_mxf4nvf4(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j,
-                                         sf_col + 16 + 8 * j, (ks | j) != 0);
-                    tc::tc_commit(&empty[s]);
+                        tc::mma_mxf4nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j,
+                                              sf_col + 16 + 8 * j, (ks | j) != 0);
+                    tc::tc_commit_pair(&empty[s], 0x3);
                 }
-                tc::tc_commit(acc_full);
+                tc::tc_commit_pair(acc_full, 0x3);
             }
         }
     } else if (warp >= 2 + EPI_WARPS) {
         // ------------------------------------------------------------ scale warps
         // Warp w writes the scale factors of every stage into TMEM lane quadrant
-        // w % 4 with tcgen05.st, in the replicated atom layout the MMA reads: lane
-        // (32q + l), column c of an atom's 4 holds word c of the atom's 16-byte row
-        // l.  Each ring slot has its own scale columns, rewritten only after the
-        // slot's MMAs completed (the slot is refilled only after `empty`).
+        // w % 4 of its own CTA with tcgen05.st, in the replicated atom layout the
+        // MMA reads: lane (32q + l), column c of an atom's 4 holds word c of the
+        // atom's 16-byte row l.  Each ring slot has its own scale columns, rewritten
+        // only after the slot's MMAs completed (the slot is refilled only after
+        // `empty`).  The even CTA's MMA thread waits for all eight scale warps.
         const int q = warp & 3;
         const uint32_t t_q = tmem + ((uint32_t)(q * 32) << 16);
         int it = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        for (int tile = pair; tile < total; tile += n_pairs) {
             for (int ks = 0; ks < ks_count; ++ks, ++it) {
                 const int s = it % STAGES;
                 const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -269,7 +274,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc::tmem_st_wait();
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&sf_ready[s]);
+                if (lane == 0) tc::mbar_arrive_remote_relaxed(tc::cluster_addr(&sf_ready[s], 0));
             }
         }
     } else {
@@ -280,13 +285,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int quarter = (warp - 2) >> 2;
         const int r_in = q * 32 + lane;
         const uint32_t t_row = tmem + ((uint32_t)(q * 32) << 16);
+        const uint32_t acc_empty_leader = tc::cluster_addr(acc_empty, 0);
         int tl = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tl) {
+        for (int tile = pair; tile < total; tile += n_pairs, ++tl) {
             const int m = tile / p.n_ntiles, n = tile - m * p.n_ntiles;
             const int4 ti = p.tiles[m];
-            const bool valid = r_in < ti.z;
-            const int64_t row = (int64_t)ti.y + r_in;
-            if (!tc::mbar_wait(acc_full, (uint32_t)tl & 1u, p.err)) goto done;
+            // this CTA's 128 rows of the pair tile
+            const int n_valid = ti.z - BM * (int)rank;
+            const int64_t row0 = (int64_t)ti.y + BM * (int)rank;
+            const bool valid = r_in < n_valid;
+            const int64_t row = row0 + r_in;
+            if (!tc::mbar_wait<true>(acc_full, (uint32_t)tl & 1u, p.err)) goto done;
             tc::tc_fence_after();
             if (EPI == EPI_GATEUP) {
                 // columns [0,128) gate, [128,256) up, for intermediates n*128 .. n*128+127;
@@ -301,7 +310,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                                     uv + 16 * c);
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(acc_empty);
+                if (lane == 0) tc::mbar_arrive_remote_relaxed(acc_empty_leader);
                 if (valid) {
                     const float ag = p.globals[ti.x * 3 + 0] * p.act_global;
                     const float au = p.globals[ti.x * 3 + 1] * p.act_global;
@@ -331,7 +340,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int c = 0; c < 2; ++c) tc::tmem_ld16x2(t_col + 32 * c, t_col + 32 * c + 16, v + 32 * c, v + 32 * c + 16);
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(acc_empty);
+                if (lane == 0) tc::mbar_arrive_remote_relaxed(acc_empty_leader);
                 // rows past the tile's valid count hold padding: weight 0, never stored
                 const float f = valid ? p.globals[ti.x * 3 + 2] * p.act_global * p.wts[p.pair_of_row[row]] : 0.0f;
                 float amax = 0.0f;
@@ -376,18 +385,21 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int r_j = q * 32 + g8 * 8 + j;
-                    if (r_j < ti.z)
-                        *reinterpret_cast<uint4*>(p.Y + ((int64_t)ti.y + r_j) * p.ldy + (int64_t)n * BN + quarter * 64 +
+                    if (r_j < n_valid)
+                        *reinterpret_cast<uint4*>(p.Y + (row0 + r_j) * p.ldy + (int64_t)n * BN + quarter * 64 +
                                                   c8 * 8) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
                 }
             }
         }
     }
 done:
+    // neither CTA frees its TMEM or exits while the other may still signal it
     __syncthreads();
+    tc::tc_fence_before();
+    tc::cluster_sync();
     if (warp == 1) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem, TMEM_COLS);
+        tc::tmem_dealloc_pair(tmem, TMEM_COLS);
     }
 }
 
@@ -470,6 +482,37 @@ bool make_map(CUtensorMap* m, const void* base, int64_t row_bytes, int64_t rows,
     return true;
 }
 
+// CTA pairs that fit on the device at once (1 CTA per SM), per device, cached.
+int max_resident_pairs() {
+    static std::mutex mu;
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        set_error("w4a4: no usable current CUDA device");
+        return 0;
+    }
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev] == 0) {
+        if (cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+            cudaSuccess) {
+            set_error("w4a4: cannot raise the shared-memory limit to %d bytes", SMEM_BYTES);
+            return 0;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * 74, 1, 1);
+        cfg.blockDim = dim3(THREADS, 1, 1);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        int n = 0;
+        const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, k_w4a4_gemm<EPI_GATEUP>, &cfg);
+        if (e != cudaSuccess || n <= 0) {
+            (void)cudaGetLastError();
+            n = num_sms() / 2;  // one CTA per SM, two SMs per pair
+        }
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 }  // namespace
 
 size_t w4a4_packed_size(int E, int H, int I) { return (size_t)w4_layout(E, H, I).total; }
@@ -505,10 +548,12 @@ nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E
         cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
     NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w4a4_gemm<EPI_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
     CUtensorMap mA1, mGU, mA2, mD;
-    if (!make_map(&mA1, A1c, H / 2, rows_max, BM) || !make_map(&mGU, pk + L.gu_codes, H / 2, (int64_t)E * 2 * I, BN) ||
-        !make_map(&mA2, A2c, I / 2, rows_max, BM) || !make_map(&mD, pk + L.d_codes, I / 2, (int64_t)E * H, BN))
+    if (!make_map(&mA1, A1c, H / 2, rows_max, BM) ||
+        !make_map(&mGU, pk + L.gu_codes, H / 2, (int64_t)E * 2 * I, BN / 2) ||
+        !make_map(&mA2, A2c, I / 2, rows_max, BM) || !make_map(&mD, pk + L.d_codes, I / 2, (int64_t)E * H, BN / 2))
         return NVFP4MOE_ERR_CUDA;
-    const int sms = num_sms();
+    const int pairs = max_resident_pairs();
+    if (pairs <= 0) return NVFP4MOE_ERR_CUDA;
     GemmParams g{};
     g.tiles = plan.tiles;
     g.n_tiles = plan.n_tiles;
@@ -527,7 +572,7 @@ nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E
     g.out_sf = A2s;
     g.out_k = I;
     {
-        const int grid = (int)std::min<int64_t>(sms, (int64_t)max_tiles * g.n_ntiles);
+        const int grid = 2 * (int)std::min<int64_t>(pairs, (int64_t)max_tiles * g.n_ntiles);
         k_w4a4_gemm<EPI_GATEUP><<<grid, THREADS, SMEM_BYTES, stream>>>(mA1, mGU, g);
         NVFP4MOE_CHECK_LAUNCH("w4a4 gate/up kernel");
     }
@@ -542,7 +587,7 @@ nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E
     g.y_scale = y_scale;
     g.ldy = H;
     {
-        const int grid = (int)std::min<int64_t>(sms, (int64_t)max_tiles * g.n_ntiles);
+        const int grid = 2 * (int)std::min<int64_t>(pairs, (int64_t)max_tiles * g.n_ntiles);
         k_w4a4_gemm<EPI_DOWN><<<grid, THREADS, SMEM_BYTES, stream>>>(mA2, mD, g);
         NVFP4MOE_CHECK_LAUNCH("w4a4 down kernel");
     }
