@@ -216,28 +216,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------ MMA issuer
         // One thread of the even CTA issues the pair's M=256 x N=256 MMAs; scale
         // factors are already in both CTAs' TMEM (the scale warps put them there).
+        // The tensor pipe accepts few MMAs ahead of the one it executes (an issue
+        // returns ~140 cycles after the previous one), so whatever this thread does
+        // between stages is pipe idle time.  The wait for the next stage is
+        // therefore made before the current stage's last MMA is issued, and
+        // overlaps the MMAs still queued.
         if (lane == 0 && rank == 0) {
             const uint32_t idesc = tc::idesc_mxf4nvf4(2 * BM, BN);
-            int it = 0, tl = 0;
-            for (int tile = pair; tile < total; tile += n_pairs, ++tl) {
-                if (!tc::mbar_wait<true>(acc_empty, ((uint32_t)tl & 1u) ^ 1u, p.err)) goto done;
+            const int n_tiles_mine = pair < total ? (total - pair + n_pairs - 1) / n_pairs : 0;
+            const int n_it = n_tiles_mine * ks_count;
+            if (n_it > 0) {
+                if (!tc::mbar_wait<true>(acc_empty, 1u, p.err)) goto done;
+                if (!tc::mbar_wait<true>(&sf_ready[0], 0u, p.err)) goto done;
                 tc::tc_fence_after();
-                for (int ks = 0; ks < ks_count; ++ks, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!tc::mbar_wait<true>(&sf_ready[s], ph, p.err)) goto done;
-                    tc::tc_fence_after();
-                    const int n64 = min(4, k64_total - ks * 4);
-                    uint8_t* st = smem + s * STAGE_BYTES;
-                    const uint32_t sf_col = tmem + TM_SF + (uint32_t)s * TM_SF_STRIDE;
-                    const uint64_t adesc = tc::desc_sw128(st);
-                    const uint64_t bdesc = tc::desc_sw128(st + A_BYTES);
-                    for (int j = 0; j < n64; ++j)
-                        tc::mma_mxf4nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j,
-                                              sf_col + 16 + 8 * j, (ks | j) != 0);
-                    tc::tc_commit_pair(&empty[s], 0x3);
+            }
+            int ks = 0, tl = 0;
+            for (int it = 0; it < n_it; ++it) {
+                const int s = it % STAGES;
+                const int n64 = min(4, k64_total - ks * 4);
+                uint8_t* st = smem + s * STAGE_BYTES;
+                const uint32_t sf_col = tmem + TM_SF + (uint32_t)s * TM_SF_STRIDE;
+                const uint64_t adesc = tc::desc_sw128(st);
+                const uint64_t bdesc = tc::desc_sw128(st + A_BYTES);
+                for (int j = 0; j < n64 - 1; ++j)
+                    tc::mma_mxf4nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j,
+                                          sf_col + 16 + 8 * j, (ks | j) != 0);
+                const int nx = it + 1;
+                const bool tile_end = ks + 1 == ks_count;
+                // next stage of the same tile: its scale factors (and so its operands)
+                bool ok = true;
+                if (nx < n_it && !tile_end)
+                    ok = tc::mbar_wait<true>(&sf_ready[nx % STAGES], (uint32_t)(nx / STAGES) & 1u, p.err);
+                {
+                    const int j = n64 - 1;
+                    tc::mma_mxf4nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j,
+                                          sf_col + 16 + 8 * j, (ks | j) != 0);
                 }
-                tc::tc_commit_pair(acc_full, 0x3);
+                tc::tc_commit_pair(&empty[s], 0x3);
+                if (tile_end) {
+                    tc::tc_commit_pair(acc_full, 0x3);
+                    ks = 0;
+                    ++tl;
+                    if (nx < n_it) {
+                        // the single accumulator: the epilogues must have read it
+                        ok = ok && tc::mbar_wait<true>(acc_empty, ((uint32_t)tl & 1u) ^ 1u, p.err);
+                        ok = ok && tc::mbar_wait<true>(&sf_ready[nx % STAGES], (uint32_t)(nx / STAGES) & 1u, p.err);
+                    }
+                } else {
+                    ++ks;
+                }
+                if (!ok) goto done;
+                tc::tc_fence_after();
             }
         }
     } else if (warp >= 2 + EPI_WARPS) {
