@@ -247,10 +247,14 @@ def run_ours(args, rank, world, local_rank):
         flops = 4.0 * T * wl.top_k * wl.H * wl.I  # gate/up GEMM, padding rows excluded
         t_kernel = stage["gateup_gemm"] / 1e3
         achieved = flops / t_kernel / 1e12
-        peak = P["bf16_tflops"] * FP4_OVER_BF16
+        # The GEMM runs inside a long loop of steps and draws the board to its power
+        # cap (its SM clock falls to ~1.4-1.6 GHz), so the denominator is the
+        # sustained bf16 figure, scaled to FP4 by the nominal dense ratio.
+        peak = P["bf16_tflops_sustained"] * FP4_OVER_BF16
         roofline = {"bound": "tensor", "kernel": "k_w4a4_gemm<gate/up>", "achieved": round(achieved, 1),
                     "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
-                    "peak_src": f"{P['src']} bf16 burst x {FP4_OVER_BF16:g} (nominal dense FP4:BF16)",
+                    "peak_src": f"{P['src']} bf16 sustained x {FP4_OVER_BF16:g} (nominal dense FP4:BF16); "
+                                f"burst would be {P['bf16_tflops'] * FP4_OVER_BF16:.0f}",
                     "algorithmic_flops_per_launch": flops}
     else:
         # W4A16 weight stream: every active expert's codes + E4M3 scales read once
