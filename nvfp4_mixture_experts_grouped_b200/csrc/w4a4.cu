@@ -220,33 +220,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // returns ~140 cycles after the previous one), so whatever this thread does
         // between stages is pipe idle time.  The wait for the next stage is
         // therefore made before the current stage's last MMA is issued, and
-        // overlaps the MMAs still queued.
+        // overlaps the MMAs still queued.  The loop carries slot, phase, descriptors
+        // and scale column forward instead of recomputing them: its own
+        // instructions are pipe idle time too.
         if (lane == 0 && rank == 0) {
             const uint32_t idesc = tc::idesc_mxf4nvf4(2 * BM, BN);
             const int n_tiles_mine = pair < total ? (total - pair + n_pairs - 1) / n_pairs : 0;
             const int n_it = n_tiles_mine * ks_count;
+            const uint64_t adesc0 = tc::desc_sw128(smem);
+            constexpr uint64_t STAGE_DESC = STAGE_BYTES >> 4, B_DESC = A_BYTES >> 4;
             if (n_it > 0) {
                 if (!tc::mbar_wait<true>(acc_empty, 1u, p.err)) goto done;
                 if (!tc::mbar_wait<true>(&sf_ready[0], 0u, p.err)) goto done;
                 tc::tc_fence_after();
             }
-            int ks = 0, tl = 0;
+            int ks = 0, tl = 0, s = 0;
+            uint32_t ph = 0;
+            uint64_t adesc = adesc0;
+            uint32_t sf_col = tmem + TM_SF;
             for (int it = 0; it < n_it; ++it) {
-                const int s = it % STAGES;
-                const int n64 = min(4, k64_total - ks * 4);
-                uint8_t* st = smem + s * STAGE_BYTES;
-                const uint32_t sf_col = tmem + TM_SF + (uint32_t)s * TM_SF_STRIDE;
-                const uint64_t adesc = tc::desc_sw128(st);
-                const uint64_t bdesc = tc::desc_sw128(st + A_BYTES);
-                for (int j = 0; j < n64 - 1; ++j)
-                    tc::mma_mxf4nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j,
-                                          sf_col + 16 + 8 * j, (ks | j) != 0);
-                const int nx = it + 1;
+                const int n64 = ks + 1 < ks_count ? 4 : k64_total - ks * 4;
+                const uint64_t bdesc = adesc + B_DESC;
+                const uint32_t acc0 = ks != 0;
+                if (n64 == 4) {
+                    tc::mma_mxf4nvf4_pair(tmem, adesc, bdesc, idesc, sf_col, sf_col + 16, acc0);
+                    tc::mma_mxf4nvf4_pair(tmem, adesc + 2, bdesc + 2, idesc, sf_col + 4, sf_col + 24, 1u);
+                    tc::mma_mxf4nvf4_pair(tmem, adesc + 4, bdesc + 4, idesc, sf_col + 8, sf_col + 32, 1u);
+                } else {
+                    for (int j = 0; j < n64 - 1; ++j)
+                        tc::mma_mxf4nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j,
+                                              sf_col + 16 + 8 * j, (ks | j) != 0);
+                }
+                const int ns = s + 1 == STAGES ? 0 : s + 1;
+                const uint32_t nph = ns == 0 ? ph ^ 1u : ph;
                 const bool tile_end = ks + 1 == ks_count;
+                const bool more = it + 1 < n_it;
                 // next stage of the same tile: its scale factors (and so its operands)
                 bool ok = true;
-                if (nx < n_it && !tile_end)
-                    ok = tc::mbar_wait<true>(&sf_ready[nx % STAGES], (uint32_t)(nx / STAGES) & 1u, p.err);
+                if (more && !tile_end) ok = tc::mbar_wait<true>(&sf_ready[ns], nph, p.err);
                 {
                     const int j = n64 - 1;
                     tc::mma_mxf4nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j,
@@ -257,16 +268,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     tc::tc_commit_pair(acc_full, 0x3);
                     ks = 0;
                     ++tl;
-                    if (nx < n_it) {
+                    if (more) {
                         // the single accumulator: the epilogues must have read it
                         ok = ok && tc::mbar_wait<true>(acc_empty, ((uint32_t)tl & 1u) ^ 1u, p.err);
-                        ok = ok && tc::mbar_wait<true>(&sf_ready[nx % STAGES], (uint32_t)(nx / STAGES) & 1u, p.err);
+                        ok = ok && tc::mbar_wait<true>(&sf_ready[ns], nph, p.err);
                     }
                 } else {
                     ++ks;
                 }
                 if (!ok) goto done;
                 tc::tc_fence_after();
+                s = ns;
+                ph = nph;
+                adesc = ns == 0 ? adesc0 : adesc + STAGE_DESC;
+                sf_col = ns == 0 ? tmem + TM_SF : sf_col + TM_SF_STRIDE;
             }
         }
     } else if (warp >= 2 + EPI_WARPS) {
