@@ -152,6 +152,126 @@ __global__ void __launch_bounds__(RT_WARPS * 32)
     }
 }
 
+// Fast path for the common group shapes: group size G a power of two <= 32
+// (a group is an aligned run of G lanes of one register row) or a multiple of
+// 32 (a group is G/32 whole register rows).  Group scores come from a
+// segmented warp reduction of (largest, second largest) instead of a
+// sequential scan, and every element's group bit is computed once.  Same
+// arithmetic and tie rules as k_route: the group score is the FP32 sum of the
+// two largest values, which does not depend on which of equal values is taken.
+template <int NPL>
+__global__ void __launch_bounds__(RT_WARPS * 32)
+    k_route_fast(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int n_group,
+                 int topk_group, int top_k, float rsf, int renorm, ExpSpecConsts kc, int32_t* __restrict__ ids,
+                 float* __restrict__ wts) {
+    __shared__ float s_score[RT_WARPS][32];
+    const int warp = warp_id(), lane = lane_id();
+    const int t = blockIdx.x * RT_WARPS + warp;
+    if (t >= T) return;
+    const int gsz = E / n_group;
+    const float* lg = logits + (int64_t)t * E;
+    float s[NPL], c[NPL];
+    uint32_t gbit[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            s[i] = sigmoid_spec(__ldg(lg + e), kc);
+            c[i] = __fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f);
+            gbit[i] = 1u << (e / gsz);
+        } else {
+            s[i] = 0.0f;
+            c[i] = -INFINITY;
+            gbit[i] = 0u;
+        }
+    }
+    if (gsz <= 32) {
+        // per row: segments of gsz lanes
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            float a = c[i], b = -INFINITY;
+            for (int o = gsz >> 1; o; o >>= 1) {
+                const float pa = __shfl_xor_sync(0xffffffffu, a, o);
+                const float pb = __shfl_xor_sync(0xffffffffu, b, o);
+                b = fmaxf(fminf(a, pa), fmaxf(b, pb));
+                a = fmaxf(a, pa);
+            }
+            const int e = lane + 32 * i;
+            if ((lane & (gsz - 1)) == 0 && e < E) s_score[warp][e / gsz] = __fadd_rn(a, b);
+        }
+    } else {
+        // per group: its rows, then the whole warp
+        const int rows = gsz >> 5;
+        for (int g = 0; g < n_group; ++g) {
+            float a = -INFINITY, b = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+                if (i >= g * rows && i < (g + 1) * rows) {
+                    b = fmaxf(b, fminf(a, c[i]));
+                    a = fmaxf(a, c[i]);
+                }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                const float pa = __shfl_xor_sync(0xffffffffu, a, o);
+                const float pb = __shfl_xor_sync(0xffffffffu, b, o);
+                b = fmaxf(fminf(a, pa), fmaxf(b, pb));
+                a = fmaxf(a, pa);
+            }
+            if (lane == 0) s_score[warp][g] = __fadd_rn(a, b);
+        }
+    }
+    __syncwarp();
+    const float score = lane < n_group ? s_score[warp][lane] : -INFINITY;
+    // keep topk_group groups
+    uint32_t chosen = 0;
+    for (int r = 0; r < topk_group; ++r) {
+        float v = (lane < n_group && !((chosen >> lane) & 1u)) ? score : -INFINITY;
+        int idx = (lane < n_group && !((chosen >> lane) & 1u)) ? lane : 0x7fffffff;
+        warp_argmax(v, idx);
+        chosen |= 1u << idx;
+    }
+    // top_k experts inside the chosen groups
+    float cand[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) cand[i] = (chosen & gbit[i]) ? c[i] : -INFINITY;
+    int my_id = 0;
+    float my_s = 0.0f;
+    for (int j = 0; j < top_k; ++j) {
+        float v = -INFINITY;
+        int idx = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            if (cand[i] != -INFINITY && better(cand[i], e, v, idx)) {
+                v = cand[i];
+                idx = e;
+            }
+        }
+        warp_argmax(v, idx);
+        float sv = 0.0f;
+        if ((idx & 31) == lane) {
+            const int hit = idx >> 5;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+                if (i == hit) {
+                    sv = s[i];
+                    cand[i] = -INFINITY;
+                }
+        }
+        sv = __shfl_sync(0xffffffffu, sv, idx & 31);
+        if (lane == j) {
+            my_id = idx;
+            my_s = sv;
+        }
+    }
+    float S = 0.0f;
+    for (int j = 0; j < top_k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, my_s, j));
+    if (lane < top_k) {
+        ids[(int64_t)t * top_k + lane] = my_id;
+        wts[(int64_t)t * top_k + lane] = renorm ? __fmul_rn(__fdiv_rn(my_s, S), rsf) : __fmul_rn(my_s, rsf);
+    }
+}
+
 static ExpSpecConsts exp_spec_consts() {
     // ln2_hi = ln 2 rounded to FP32 with its 12 low mantissa bits cleared;
     // ln2_lo = FP32(ln 2 - ln2_hi); log2e = FP32(log2 e).
@@ -174,9 +294,17 @@ nvfp4moe_status launch_route(const float* logits, const float* bias, int T, int 
     const ExpSpecConsts kc = exp_spec_consts();
     const dim3 grid((unsigned)ceil_div(T, RT_WARPS));
     const int npl = (int)ceil_div(E, 32);
-#define RT_LAUNCH(N)                                                                                           \
-    k_route<N><<<grid, RT_WARPS * 32, 0, stream>>>(logits, bias, T, E, n_group, topk_group, top_k, rsf, renorm, \
-                                                   kc, ids, wts)
+    const int gsz = E / n_group;
+    const bool fast = n_group <= 32 && gsz >= 2 && ((gsz <= 32 && (gsz & (gsz - 1)) == 0) || gsz % 32 == 0);
+#define RT_LAUNCH(N)                                                                                              \
+    do {                                                                                                          \
+        if (fast)                                                                                                 \
+            k_route_fast<N><<<grid, RT_WARPS * 32, 0, stream>>>(logits, bias, T, E, n_group, topk_group, top_k,  \
+                                                                rsf, renorm, kc, ids, wts);                       \
+        else                                                                                                      \
+            k_route<N><<<grid, RT_WARPS * 32, 0, stream>>>(logits, bias, T, E, n_group, topk_group, top_k, rsf,  \
+                                                           renorm, kc, ids, wts);                                 \
+    } while (0)
     if (npl <= 1)
         RT_LAUNCH(1);
     else if (npl <= 2)
