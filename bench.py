@@ -117,6 +117,29 @@ def layer_flops(T, H, I, k):
     return 6.0 * T * k * H * I
 
 
+def max_over_ranks(torch, dist, ms, device):
+    """The slowest rank's time: the job is done only when every rank is."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank, world, ms):
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (ms / 1e3)
+
+
+def rank_batch(wl, d, rank):
+    """Rank r > 0 gets its own seeded batch (activations, logits); the layer's
+    weights are the same on every rank."""
+    if rank == 0:
+        return d["x"], d["logits"]
+    rng = np.random.default_rng(wl.seed * 1000 + rank)
+    return inputs.activations(rng, wl.T, wl.H, wl.outliers), inputs.router_logits(rng, wl.T, wl.E, wl.zipf)
+
+
 def make_layer(torch, moe, mode, w, T, wl):
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
     E, I, hh = w["gate_codes"].shape
@@ -188,11 +211,7 @@ def run_ours(args, rank, world, local_rank):
     T = wl.T
     d = inputs.moe_inputs(wl)
     w = {k: d[k] for k in ("gate_codes", "gate_sf", "up_codes", "up_sf", "down_codes", "down_sf", "w_global")}
-    # each rank gets its own batch (the weights are the layer's, identical on every rank)
-    if rank:
-        rng = np.random.default_rng(wl.seed * 1000 + rank)
-        d["x"] = inputs.activations(rng, T, wl.H, wl.outliers)
-        d["logits"] = inputs.router_logits(rng, T, wl.E, wl.zipf)
+    d["x"], d["logits"] = rank_batch(wl, d, rank)
     mode = wl.mode
     packed, ws = make_layer(torch, moe, mode, w, T, wl)
     x = torch.from_numpy(d["x"].view(np.int16)).cuda().view(torch.bfloat16)
@@ -206,12 +225,10 @@ def run_ours(args, rank, world, local_rank):
     sampler = ClockSampler(local_rank) if rank == 0 else None
     ms, stage = time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, args.steps, args.warmup)
     clocks = sampler.stop() if sampler else None
+    ms = max_over_ranks(torch, dist, ms, "cuda")
     if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
-    value = T * world / (ms / 1e3)
+    value = job_tokens_per_s(T, world, ms)
 
     # ----------------------------------------------------------------- end to end
     xh = torch.from_numpy(d["x"].view(np.int16)).pin_memory()
@@ -237,10 +254,7 @@ def run_ours(args, rank, world, local_rank):
     b.record()
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / args.steps
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(torch, dist, e2e_ms, "cuda")
 
     # ----------------------------------------------------------------- roofline
     if mode == moe.W4A4:
@@ -283,7 +297,7 @@ def run_ours(args, rank, world, local_rank):
                          f"packed expert weights per step)"},
         "roofline": roofline,
         "stages_ms": {k: round(v, 4) for k, v in stage.items()},
-        "e2e": {"value": round(T * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(job_tokens_per_s(T, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(d["x"].nbytes + d["logits"].nbytes), "d2h_bytes_per_step": int(T * wl.H * 2)},
         "gpu_launches": 8 * args.steps,
         "clocks": clocks,
