@@ -167,15 +167,19 @@ __global__ void __launch_bounds__(256)
     const int lane = lane_id();
     const int64_t nb = K / 16;
     const uint16_t* xr = x + m * K;
-    int rows[32];
-    int nrows = 1;
-    if (SCATTER) {
-        nrows = k;
-        for (int j = 0; j < k; ++j) rows[j] = row_of_pair[m * k + j];
-    }
-    for (int64_t b = lane; b < nb; b += 32) {
-        const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(xr + b * 16));
-        const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(xr + b * 16 + 8));
+    // destination rows of this token's k pairs, one per lane (k <= 32), broadcast below
+    const int my_row = SCATTER && lane < k ? row_of_pair[m * k + lane] : 0;
+    // every lane runs every iteration (the shuffles below need all 32); lanes past
+    // the row's last block only skip their loads and stores.  The scatter form
+    // needs nb % 4 == 0 (K % 64 == 0) so that a lane quad is all in or all out.
+    for (int64_t b0 = 0; b0 < nb; b0 += 32) {
+        const int64_t b = b0 + lane;
+        const bool active = b < nb;
+        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+        if (active) {
+            v0 = __ldg(reinterpret_cast<const uint4*>(xr + b * 16));
+            v1 = __ldg(reinterpret_cast<const uint4*>(xr + b * 16 + 8));
+        }
         float f[16];
         const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
@@ -186,13 +190,22 @@ __global__ void __launch_bounds__(256)
         uint32_t c0, c1;
         const uint32_t sf = quantize_block16(f, gs, c0, c1);
         if (!SCATTER) {
-            *reinterpret_cast<uint2*>(codes + m * (K / 2) + b * 8) = make_uint2(c0, c1);
-            scales[m * nb + b] = (uint8_t)sf;
+            if (active) {
+                *reinterpret_cast<uint2*>(codes + m * (K / 2) + b * 8) = make_uint2(c0, c1);
+                scales[m * nb + b] = (uint8_t)sf;
+            }
         } else {
-            for (int j = 0; j < nrows; ++j) {
-                const int64_t row = rows[j];
-                *reinterpret_cast<uint2*>(codes + row * (K / 2) + b * 8) = make_uint2(c0, c1);
-                scales[sf_atom_offset(row, b, nb)] = (uint8_t)sf;
+            // lanes 4q..4q+3 hold the scales of blocks b..b+3 (b % 4 == 0 at lane 4q):
+            // four consecutive bytes of one atom row, stored as one word by lane 4q
+            uint32_t sfw = sf << (8 * (lane & 3));
+            sfw |= __shfl_xor_sync(0xffffffffu, sfw, 1);
+            sfw |= __shfl_xor_sync(0xffffffffu, sfw, 2);
+            for (int j = 0; j < k; ++j) {
+                const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
+                if (active) {
+                    *reinterpret_cast<uint2*>(codes + row * (K / 2) + b * 8) = make_uint2(c0, c1);
+                    if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(scales + sf_atom_offset(row, b, nb)) = sfw;
+                }
             }
         }
     }
