@@ -77,9 +77,22 @@ class ClockSampler:
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                                       "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+                                       "-lms", "20"], stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.p = None
+
+    def wait_ready(self, timeout_s: float = 10.0):
+        """Block until nvidia-smi has written its first sample (its start-up takes
+        longer than a short timed region)."""
+        t0 = time.time()
+        while self.p is not None and time.time() - t0 < timeout_s:
+            if os.path.getsize(self.f.name) > 0:
+                return
+            time.sleep(0.02)
+
+    def mark(self):
+        """Samples before this point (start-up, warm-up) are not reported."""
+        self.offset = os.path.getsize(self.f.name) if self.p is not None else 0
 
     def stop(self):
         if self.p is None:
@@ -90,7 +103,12 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.p.kill()
         self.f.seek(0)
-        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        text = self.f.read()
+        during = text[getattr(self, "offset", 0):]
+        # a timed region shorter than the sampling interval may hold no sample:
+        # then the last one taken before its end stands for it
+        lines = [r for r in during.strip().splitlines() if r.strip()] or text.strip().splitlines()[-1:]
+        rows = [r.split(",") for r in lines if r.strip()]
         os.unlink(self.f.name)
         if not rows:
             return None
@@ -154,7 +172,7 @@ def make_layer(torch, moe, mode, w, T, wl):
     return packed, ws
 
 
-def time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, steps, warmup, trace=True):
+def time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, steps, warmup, trace=True, on_start=None):
     """Returns (ms per step, per-stage ms means) timed with CUDA events on the current stream."""
     H, I, E = wl.H, wl.I, wl.E
 
@@ -173,6 +191,8 @@ def time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, steps, warmu
                 e.record()
             evs.append(row)
     torch.cuda.synchronize()
+    if on_start:
+        on_start()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
@@ -191,6 +211,57 @@ def time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, steps, warmu
         for s, name in enumerate(STAGES):
             stage[name] = float(np.mean([evs[i][s].elapsed_time(evs[i][s + 1]) for i in range(steps)]))
     return ms, stage
+
+
+def time_e2e(torch, moe, mode, packed, ws, d, wl, T, steps, warmup):
+    """ms per step of the pipelined host-buffer loop (see run_ours)."""
+    xh = torch.from_numpy(d["x"].view(np.int16)).pin_memory()
+    lh = torch.from_numpy(d["logits"]).pin_memory()
+    oh = [torch.empty((T, wl.H), dtype=torch.int16).pin_memory() for _ in range(2)]
+    xd = [torch.empty((T, wl.H), dtype=torch.int16, device="cuda") for _ in range(2)]
+    ld = [torch.empty((T, wl.E), dtype=torch.float32, device="cuda") for _ in range(2)]
+    od = [torch.empty((T, wl.H), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    up, ran, down = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    used = [False, False]
+
+    def step(i):
+        b = i & 1
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(ran[b])  # the layer of step i-2 has read these inputs
+            xd[b].copy_(xh, non_blocking=True)
+            ld[b].copy_(lh, non_blocking=True)
+            up[b].record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(up[b])
+            if used[b]:
+                s_run.wait_event(down[b])  # step i-2's output has left the device
+            moe.moe_forward(mode, xd[b].view(torch.bfloat16), ld[b], None, packed, 1.0, T, wl.H, wl.I, wl.E,
+                            wl.n_group, wl.topk_group, wl.top_k, wl.rsf, True, ws, od[b], stream=s_run)
+            ran[b].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ran[b])
+            oh[b].copy_(od[b].view(torch.int16), non_blocking=True)
+            down[b].record(s_out)
+        used[b] = True
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s_in)
+    for i in range(steps):
+        step(warmup + i)
+    # the last step's download ends the region
+    s_out.wait_event(down[(warmup + steps - 1) & 1])
+    z.record(s_out)
+    torch.cuda.synchronize()
+    # every step really produced its output on the host
+    ref = od[(warmup + steps - 1) & 1].view(torch.int16).cpu()
+    assert torch.equal(oh[(warmup + steps - 1) & 1], ref)
+    return a.elapsed_time(z) / steps
 
 
 def run_ours(args, rank, world, local_rank):
@@ -223,7 +294,10 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(local_rank) if rank == 0 else None
-    ms, stage = time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, args.steps, args.warmup)
+    if sampler:
+        sampler.wait_ready()
+    ms, stage = time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, args.steps, args.warmup,
+                           on_start=sampler.mark if sampler else None)
     clocks = sampler.stop() if sampler else None
     ms = max_over_ranks(torch, dist, ms, "cuda")
     if dist:
@@ -231,29 +305,14 @@ def run_ours(args, rank, world, local_rank):
     value = job_tokens_per_s(T, world, ms)
 
     # ----------------------------------------------------------------- end to end
-    xh = torch.from_numpy(d["x"].view(np.int16)).pin_memory()
-    lh = torch.from_numpy(d["logits"]).pin_memory()
-    oh = torch.empty((T, wl.H), dtype=torch.int16).pin_memory()
-
-    def e2e_step():
-        x.view(torch.int16).copy_(xh, non_blocking=True)
-        logits.copy_(lh, non_blocking=True)
-        moe.moe_forward(mode, x, logits, None, packed, 1.0, T, wl.H, wl.I, wl.E, wl.n_group, wl.topk_group,
-                        wl.top_k, wl.rsf, True, ws, out)
-        oh.copy_(out.view(torch.int16), non_blocking=True)
-
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(args.steps):
-        e2e_step()
-    b.record()
-    torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b) / args.steps
+    # A stream of batches through the public API with host buffers: every step
+    # uploads its x and logits from pinned host memory, runs moe_forward and
+    # downloads its output to pinned host memory, all inside the timed region.
+    # Uploads, layer and downloads run on three streams with double-buffered
+    # device inputs and outputs, so step i+1's upload and step i-1's download
+    # overlap step i's layer (PCIe is full duplex); the layer calls are ordered on
+    # one stream and share one workspace.
+    e2e_ms = time_e2e(torch, moe, mode, packed, ws, d, wl, T, args.steps, args.warmup)
     e2e_ms = max_over_ranks(torch, dist, e2e_ms, "cuda")
 
     # ----------------------------------------------------------------- roofline
