@@ -464,7 +464,7 @@ def cpu_baseline(wl, d, args, steps=1):
     import oracle
 
     threads = oracle.num_threads()
-    n = args.cpu_sample_tokens or threads
+    n = args.cpu_sample_tokens or 4 * threads  # ~10 s of oracle work on a 16-thread host
     toks = np.arange(n, dtype=np.int32)
     w = {k: d[k] for k in ("gate_codes", "gate_sf", "up_codes", "up_sf", "down_codes", "down_sf", "w_global")}
     t0 = time.perf_counter()
