@@ -126,7 +126,11 @@ __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __r
 }
 
 // ---------------------------------------------------------------------------
-// BF16 rows -> FP16 rows with a per-row power-of-two scale (one warp per row)
+// BF16 rows -> FP16 rows with a per-row power-of-two scale (one warp per row),
+// written in MMA B-fragment order: inside every 64-column chunk, lane quad c's
+// sixteen values (k = 16 t + 2c, 2c+1, 2c+8, 2c+9 for the chunk's four k16 steps
+// t) are 32 consecutive bytes, so a lane fetches a step's B fragment (b0, b1)
+// with one 8-byte load.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
     k_rows_to_f16(const uint16_t* __restrict__ src, int64_t rows, int K, __half* __restrict__ dst,
@@ -151,7 +155,7 @@ __global__ void __launch_bounds__(256)
         frexpf(amax, &e);  // amax in [2^(e-1), 2^e)
         sh = 15 - e;       // amax * 2^sh in [2^14, 2^15)
     }
-    uint4* d = reinterpret_cast<uint4*>(dst + r * K);
+    uint32_t* d = reinterpret_cast<uint32_t*>(dst + r * K);
     for (int i = lane; i < K / 8; i += 32) {
         const uint4 v = s[i];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -162,7 +166,11 @@ __global__ void __launch_bounds__(256)
                                                 ldexpf(bf16_bits_to_float(w[q] >> 16), sh));
             o[q] = *reinterpret_cast<const uint32_t*>(&h);
         }
-        d[i] = make_uint4(o[0], o[1], o[2], o[3]);
+        // elements 8i .. 8i+7: chunk i / 8, k16 step (i / 2) % 4, fragment register i % 2;
+        // pair j belongs to lane quad j
+        const int64_t wbase = (int64_t)(i >> 3) * 32 + ((i >> 1) & 3) * 2 + (i & 1);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) d[wbase + q * 8] = o[q];
     }
     if (lane == 0) inv_scale[r] = ldexpf(1.0f, -sh);
 }
@@ -245,10 +253,12 @@ __device__ __forceinline__ void ring_issue(Ring& r, int stage, const uint8_t* co
 }
 
 // Streams `chunks` 64-column chunks of two 16-row tiles and accumulates their
-// products with up to W16_MAX_NT 8-token B tiles (FP16 rows).  Returns false on
-// a timeout.
+// products with NT 8-token B tiles (FP16 rows in fragment order; every lane's
+// pointer is valid, lanes past the expert's tokens read a real row and their
+// results are dropped).  Returns false on a timeout.
+template <int NT>
 __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2], const uint8_t* const scales[2],
-                                           int chunks, const __half* const bptr[W16_MAX_NT], int nt_count,
+                                           int chunks, const __half* const bptr[W16_MAX_NT],
                                            float acc[2][W16_MAX_NT][4], int32_t* err) {
     const int lane = lane_id();
     const int g = lane >> 2, c = lane & 3;
@@ -271,19 +281,16 @@ __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2
                 q[u] = *reinterpret_cast<const uint4*>(st + u * W16_CH * 512 + cc * 512 + lane * 16);
                 sc[u] = *reinterpret_cast<const uint2*>(st + W16_STAGE_CODES + u * W16_CH * 64 + cc * 64 + g * 8);
             }
-            const int kbase = (grp * W16_CH + cc) * 64;
+            // this lane's B fragments of the chunk: (b0, b1) of step t at 8 t bytes
+            const uint2* bp[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                bp[nt] = reinterpret_cast<const uint2*>(bptr[nt] + (int64_t)(grp * W16_CH + cc) * 64 + c * 16);
 #pragma unroll
             for (int stp = 0; stp < 4; ++stp) {
-                const int kb = kbase + stp * 16;
-                uint32_t b0[W16_MAX_NT], b1[W16_MAX_NT];
+                uint2 bw[NT];
 #pragma unroll
-                for (int nt = 0; nt < W16_MAX_NT; ++nt) {
-                    b0[nt] = b1[nt] = 0;
-                    if (nt < nt_count && bptr[nt]) {
-                        b0[nt] = __ldg(reinterpret_cast<const uint32_t*>(bptr[nt] + kb + 2 * c));
-                        b1[nt] = __ldg(reinterpret_cast<const uint32_t*>(bptr[nt] + kb + 2 * c + 8));
-                    }
-                }
+                for (int nt = 0; nt < NT; ++nt) bw[nt] = __ldg(bp[nt] + stp);
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     const uint32_t qw = stp == 0 ? q[u].x : stp == 1 ? q[u].y : stp == 2 ? q[u].z : q[u].w;
@@ -291,8 +298,7 @@ __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2
                     uint32_t a[4];
                     dequant_step(qw, scales_f16x2((stp & 1) ? (sw >> 16) : (sw & 0xFFFFu)), a);
 #pragma unroll
-                    for (int nt = 0; nt < W16_MAX_NT; ++nt)
-                        if (nt < nt_count) mma_f16(acc[u][nt], a, b0[nt], b1[nt]);
+                    for (int nt = 0; nt < NT; ++nt) mma_f16(acc[u][nt], a, bw[nt].x, bw[nt].y);
                 }
             }
         }
@@ -355,10 +361,12 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
                 const int n = n0 + nt * 8 + g;
-                bptr[nt] = (nt < nt_count && n < n_e) ? x16 + (int64_t)(plan.pair_of_row[row0 + n] / k) * H : nullptr;
+                bptr[nt] = x16 + (int64_t)(plan.pair_of_row[row0 + (n < n_e ? n : n0)] / k) * H;
             }
             float acc[2][W16_MAX_NT][4] = {};
-            if (!w16_stream(ring, cb, sb, chunks, bptr, nt_count, acc, err)) return;
+            const bool ok = nt_count == 1 ? w16_stream<1>(ring, cb, sb, chunks, bptr, acc, err)
+                                          : w16_stream<2>(ring, cb, sb, chunks, bptr, acc, err);
+            if (!ok) return;
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
                 if (nt >= nt_count) break;
@@ -416,10 +424,12 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
                 const int n = n0 + nt * 8 + g;
-                bptr[nt] = (nt < nt_count && n < n_e) ? A16 + (int64_t)(row0 + n) * I : nullptr;
+                bptr[nt] = A16 + (int64_t)(row0 + (n < n_e ? n : n0)) * I;
             }
             float acc[2][W16_MAX_NT][4] = {};
-            if (!w16_stream(ring, cb, sb, chunks, bptr, nt_count, acc, err)) return;
+            const bool ok = nt_count == 1 ? w16_stream<1>(ring, cb, sb, chunks, bptr, acc, err)
+                                          : w16_stream<2>(ring, cb, sb, chunks, bptr, acc, err);
+            if (!ok) return;
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
                 if (nt >= nt_count) break;
