@@ -66,6 +66,12 @@ def peaks():
 # nominal dense FP4 : BF16 tensor-core throughput on B200 (9 : 2.25 PFLOP/s)
 FP4_OVER_BF16 = 4.0
 
+# DRAM bytes (read + write) of one k_w4a4_gemm<gate/up> launch, from ncu
+# (profiles/k_w4a4_gemm_prefill2k_e64.txt: 652.8 MB read + 22.6 MB written at
+# T=2048, E=64), scaled x4 to T=8192, E=256 (weights and activations both grow
+# 4x).  Valid for this kernel version and the default prefill workload only.
+GATEUP_TRAFFIC_T8192_E256 = 4 * (652.802560e6 + 22.621184e6)
+
 
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
@@ -324,8 +330,10 @@ def run_ours(args, rank, world, local_rank):
         # cap (its SM clock falls to ~1.4-1.6 GHz), so the denominator is the
         # sustained bf16 figure, scaled to FP4 by the nominal dense ratio.
         peak = P["bf16_tflops_sustained"] * FP4_OVER_BF16
+        traffic = GATEUP_TRAFFIC_T8192_E256 if (T, wl.E, wl.H, wl.I) == (8192, 256, 4096, 2048) else None
         roofline = {"bound": "tensor", "kernel": "k_w4a4_gemm<gate/up>", "achieved": round(achieved, 1),
-                    "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                    "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "traffic": traffic, "traffic_unit": "bytes per launch (ncu dram read+write)",
                     "peak_src": f"{P['src']} bf16 sustained x {FP4_OVER_BF16:g} (nominal dense FP4:BF16); "
                                 f"burst would be {P['bf16_tflops'] * FP4_OVER_BF16:.0f}",
                     "algorithmic_flops_per_launch": flops}
