@@ -95,6 +95,12 @@ def router_logits(rng: np.random.Generator, T: int, E: int, zipf: bool = False) 
     return lg
 
 
+def router_weights(rng: np.random.Generator, E: int, H: int) -> np.ndarray:
+    """FP32 router rows [E, H] ~ N(0, 1/H): with N(0,1) hidden rows the logits are
+    ~N(0,1), the scale of the logit recipe above."""
+    return (rng.standard_normal((E, H), dtype=np.float32) / np.float32(np.sqrt(H))).astype(np.float32)
+
+
 def random_codes(rng: np.random.Generator, shape) -> np.ndarray:
     """Packed E2M1 bytes: both nibbles uniform over all 16 codes."""
     return rng.integers(0, 256, size=shape, dtype=np.uint8)

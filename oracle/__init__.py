@@ -146,6 +146,20 @@ def route(logits: np.ndarray, bias, n_group: int, topk_group: int, top_k: int, r
     return ids, w
 
 
+def router_logits(x_bits: np.ndarray, w: np.ndarray):
+    """FP32 router logits of BF16 rows x_bits [T,H] (uint16) against FP32 router
+    rows w [E,H], float64 dot products rounded once; also the float64 sums of
+    |x_h w_h| (the scale of each logit's rounding error bound)."""
+    x = np.ascontiguousarray(x_bits, np.uint16)
+    wr = np.ascontiguousarray(w, np.float32)
+    T, H = x.shape
+    E = wr.shape[0]
+    out = np.empty((T, E), np.float32)
+    mag = np.empty((T, E), np.float64)
+    _load().orc_router_logits(_p(x), _p(wr), ctypes.c_int(T), ctypes.c_int(H), ctypes.c_int(E), _p(out), _p(mag))
+    return out, mag
+
+
 def permute(topk_ids: np.ndarray, E: int):
     ids = np.ascontiguousarray(topk_ids, np.int32)
     T, k = ids.shape

@@ -14,6 +14,10 @@
  *  [P2] "ProCreations/MiMo-V2.6-Flash-RL-NVFP4": "What changed", "Verification".
  *  [P4] "MiMo-V2.6-Flash -- REAP-50": "Model Summary", "Pruning Method" section 1
  *       (grouped sigmoid top-k router and the SwiGLU expert formula).
+ *  [P3] "baekpica MiMo-V2.6-Flash-RL mixed-quant GGUF": tensor precision table
+ *       (routers kept in F32).
+ *  [P5] "MiMo-V2.6-Flash-MOPD on one RTX PRO 6000": "Speed v6" and "What makes it
+ *       fast" (the router's matmul followed by a fused top-k).
  *
  * Arithmetic: floating point decisions that produce integers (quantised codes,
  * routing choices) are taken in IEEE FP32, exactly as written below; everything
@@ -352,6 +356,29 @@ void orc_route(const float* logits, const float* bias, int T, int E, int n_group
  * names an exact grouped kernel).  Order inside an expert: by token, then slot.
  * counts[E], offsets[E+1] (exclusive prefix sums), row_of_pair[T*k],
  * pair_of_row[T*k]; pair index = t * k + j.                                  */
+/* ------------------------------------------------------------------------- */
+/* Router projection [P3 precision table; P5 "What makes it fast"]: the gate   */
+/* logits of each token are the dot products of its BF16 hidden row with the   */
+/* FP32 router rows: logits[t][e] = sum_h x[t][h] * w[e][h], computed here in   */
+/* float64 in h order and rounded once to FP32.  The routing of those logits   */
+/* is orc_route.                                                               */
+/* ------------------------------------------------------------------------- */
+void orc_router_logits(const uint16_t* x, const float* w, int T, int H, int E, float* logits_out,
+                       double* abs_sum_out) {
+    for (int t = 0; t < T; ++t)
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0, mag = 0.0;
+            for (int h = 0; h < H; ++h) {
+                const double a = (double)orc_bf16_to_float(x[(int64_t)t * H + h]);
+                const double b = (double)w[(int64_t)e * H + h];
+                acc += a * b;
+                mag += fabs(a * b);
+            }
+            logits_out[(int64_t)t * E + e] = (float)acc;
+            if (abs_sum_out) abs_sum_out[(int64_t)t * E + e] = mag;
+        }
+}
+
 void orc_permute(const int32_t* topk_ids, int T, int top_k, int E, int32_t* counts, int32_t* offsets,
                  int32_t* row_of_pair, int32_t* pair_of_row) {
     const int64_t P = (int64_t)T * top_k;

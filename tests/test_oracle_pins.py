@@ -417,3 +417,48 @@ def test_layer_combines_two_experts_with_routing_weights():
             A = torch.from_numpy(A.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
             acc += float(w[t, j]) * (_np_decode(dc[e], ds[e], 1) @ A)
         assert np.allclose(both[t], acc, rtol=1e-12, atol=1e-12 * np.abs(acc).max())
+
+
+# ---------------------------------------------------------------------------
+# router projection ("MiMo-V2.6-Flash-MOPD on one RTX PRO 6000", "What makes it
+# fast": the router's matmul; routers kept in F32 per the mixed-quant GGUF
+# page's precision table)
+# ---------------------------------------------------------------------------
+def _bf16_bits(a):
+    return inputs.bf16_bits(np.asarray(a, np.float32))
+
+
+def test_router_logits_one_hot_rows_copy_the_input():
+    rng = np.random.default_rng(7)
+    T, H, E = 5, 64, 48
+    x = _bf16_bits(rng.standard_normal((T, H)).astype(np.float32) * 3)
+    w = np.zeros((E, H), np.float32)
+    w[np.arange(E), np.arange(E)] = 1.0
+    logits, mag = oracle.router_logits(x, w)
+    xf = (x.astype(np.uint32) << 16).view(np.float32)
+    assert np.array_equal(logits, xf[:, :E])
+    assert np.array_equal(mag, np.abs(xf[:, :E]).astype(np.float64))
+
+
+def test_router_logits_exact_integers():
+    rng = np.random.default_rng(8)
+    T, H, E = 7, 256, 16
+    xi = rng.integers(-8, 9, size=(T, H))
+    wi = rng.integers(-50, 51, size=(E, H))
+    logits, mag = oracle.router_logits(_bf16_bits(xi), wi.astype(np.float32))
+    ref = xi.astype(np.int64) @ wi.astype(np.int64).T  # |sum| < 2^24: exact in FP32
+    assert np.array_equal(logits, ref.astype(np.float32))
+    assert np.array_equal(mag, np.abs(xi)[:, None, :].__mul__(np.abs(wi)[None, :, :]).sum(-1).astype(np.float64))
+
+
+def test_router_logits_match_float64_matmul():
+    rng = np.random.default_rng(9)
+    T, H, E = 6, 4096, 32
+    x = _bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    w = (rng.standard_normal((E, H)) * 0.02).astype(np.float32)
+    logits, _ = oracle.router_logits(x, w)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ref = xf @ w.astype(np.float64).T
+    # the only difference is the float64 summation order: at most one FP32 rounding apart
+    ulp = np.spacing(np.abs(ref).astype(np.float32))
+    assert np.all(np.abs(logits.astype(np.float64) - ref) <= ulp)
