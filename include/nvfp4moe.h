@@ -130,6 +130,32 @@ nvfp4moe_status moe_route(const float* logits, const float* bias, int32_t T, int
                           int32_t* topk_ids, float* topk_weights, void* stream);
 
 /* ------------------------------------------------------------------------- */
+/* Router projection fused with the grouped top-k                             */
+/* ------------------------------------------------------------------------- */
+/* Operation ("MiMo-V2.6-Flash-MOPD on one RTX PRO 6000", "Speed v6" and "What
+ * makes it fast": the router's matmul followed by a fused top-k; routers kept
+ * in F32 per the tensor precision table of "baekpica MiMo-V2.6-Flash-RL
+ * mixed-quant GGUF"): logits[t][e] = sum_h x[t][h] * w_router[e][h] in FP32
+ * arithmetic (BF16 hidden rows, FP32 router rows; each logit summed in a fixed
+ * order, so repeated calls give the same bits), written to logits_out, then
+ * routed exactly as moe_route routes logits_out (same ids and weight bits).
+ * One kernel launch (plus a 4-byte-per-16-tokens clear of the workspace).
+ *   x_bf16 [T, H] bf16 bits; w_router [E, H] f32; bias [E] f32 or NULL;
+ *   logits_out [T, E] f32; topk_ids [T, top_k] i32; topk_weights [T, top_k]
+ *   f32 (caller-owned device memory); workspace: device, at least
+ *   moe_router_topk_workspace_size(T) bytes, caller-owned, left all-zero on
+ *   return; calls sharing one workspace must be ordered (one stream).
+ * Constraints: as moe_route, plus H >= 256 with H % 256 == 0 and E % 4 == 0;
+ * all pointers 16-byte aligned.  Meant for decode-sized T (the router is read
+ * once per 16 tokens).                                                        */
+size_t moe_router_topk_workspace_size(int32_t T);
+nvfp4moe_status moe_router_topk(const uint16_t* x_bf16, const float* w_router, const float* bias, int32_t T,
+                                int32_t H, int32_t E, int32_t n_group, int32_t topk_group, int32_t top_k,
+                                float routed_scaling_factor, int32_t renormalize, float* logits_out,
+                                int32_t* topk_ids, float* topk_weights, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* ------------------------------------------------------------------------- */
 /* Token permutation                                                          */
 /* ------------------------------------------------------------------------- */
 /* Operation (grouped experts: "AxionML ... NVFP4", "Usage", fused grouped MoE

@@ -14,7 +14,8 @@ import os
 
 __all__ = [
     "W4A16", "W4A4", "NVFP4MoEError", "library_path", "load",
-    "transcode_mxfp4_to_nvfp4", "nvfp4moe_transcode_workspace_size", "moe_route", "quantize_nvfp4",
+    "transcode_mxfp4_to_nvfp4", "nvfp4moe_transcode_workspace_size", "moe_route", "moe_router_topk",
+    "moe_router_topk_workspace_size", "quantize_nvfp4",
     "moe_packed_weights_size", "moe_pack_weights", "moe_forward_workspace_size", "moe_forward",
     "moe_forward_routed", "nvfp4moe_check_device_status", "nvfp4moe_version", "moe_permute",
     "moe_permute_workspace_size", "nvfp4moe_set_trace_events", "moe_permute_noalloc",
@@ -74,6 +75,10 @@ def load():
                                            vp]
     L.moe_route.restype = ctypes.c_int
     L.moe_route.argtypes = [vp, vp, i32, i32, i32, i32, i32, f32, i32, vp, vp, vp]
+    L.moe_router_topk_workspace_size.restype = sz
+    L.moe_router_topk_workspace_size.argtypes = [i32]
+    L.moe_router_topk.restype = ctypes.c_int
+    L.moe_router_topk.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp, vp, vp, sz, vp]
     L.quantize_nvfp4.restype = ctypes.c_int
     L.quantize_nvfp4.argtypes = [vp, i64, i64, f32, vp, vp, vp]
     L.moe_packed_weights_size.restype = sz
@@ -149,6 +154,20 @@ def moe_route(logits, bias, n_group, topk_group, top_k, routed_scaling_factor, r
     T, E = logits.shape
     _check(load().moe_route(_ptr(logits), _ptr(bias), T, E, n_group, topk_group, top_k, routed_scaling_factor,
                             int(renormalize), _ptr(topk_ids), _ptr(topk_weights), _stream(stream)))
+
+
+def moe_router_topk_workspace_size(T) -> int:
+    return load().moe_router_topk_workspace_size(T)
+
+
+def moe_router_topk(x_bf16, w_router, bias, n_group, topk_group, top_k, routed_scaling_factor, renormalize,
+                    logits_out, topk_ids, topk_weights, workspace, stream=None):
+    T, H = x_bf16.shape
+    E = w_router.shape[0]
+    _check(load().moe_router_topk(_ptr(x_bf16), _ptr(w_router), _ptr(bias), T, H, E, n_group, topk_group, top_k,
+                                  routed_scaling_factor, int(renormalize), _ptr(logits_out), _ptr(topk_ids),
+                                  _ptr(topk_weights), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream)))
 
 
 def quantize_nvfp4(x_bf16, gs, codes, e4m3_scales, stream=None):

@@ -237,6 +237,32 @@ nvfp4moe_status moe_route(const float* logits, const float* bias, int32_t T, int
                         topk_weights, static_cast<cudaStream_t>(stream));
 }
 
+size_t moe_router_topk_workspace_size(int32_t T) { return T > 0 ? router_ws_size(T) : 0; }
+
+nvfp4moe_status moe_router_topk(const uint16_t* x_bf16, const float* w_router, const float* bias, int32_t T,
+                                int32_t H, int32_t E, int32_t n_group, int32_t topk_group, int32_t top_k,
+                                float routed_scaling_factor, int32_t renormalize, float* logits_out,
+                                int32_t* topk_ids, float* topk_weights, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+    REQUIRE(T >= 0, NVFP4MOE_ERR_INVALID_ARG, "T=%d is negative", T);
+    RETURN_IF(validate_routing(E, n_group, topk_group, top_k));
+    REQUIRE(E % 4 == 0, NVFP4MOE_ERR_UNSUPPORTED_SHAPE, "E=%d is not a multiple of 4", E);
+    REQUIRE(H >= 256 && H % 256 == 0, NVFP4MOE_ERR_UNSUPPORTED_SHAPE, "H=%d must be a positive multiple of 256", H);
+    REQUIRE(std::isfinite(routed_scaling_factor), NVFP4MOE_ERR_INVALID_ARG, "routed_scaling_factor is not finite");
+    if (T == 0) return NVFP4MOE_OK;
+    REQUIRE(x_bf16 && w_router && logits_out && topk_ids && topk_weights && workspace, NVFP4MOE_ERR_INVALID_ARG,
+            "null pointer");
+    REQUIRE(workspace_bytes >= router_ws_size(T), NVFP4MOE_ERR_WORKSPACE_TOO_SMALL,
+            "workspace of %zu bytes, %zu needed", workspace_bytes, router_ws_size(T));
+    REQUIRE(aligned16(x_bf16) && aligned16(w_router) && aligned16(logits_out) && aligned16(topk_ids) &&
+                aligned16(topk_weights) && aligned16(workspace) && (!bias || aligned16(bias)),
+            NVFP4MOE_ERR_ALIGNMENT, "a pointer is not 16-byte aligned");
+    RETURN_IF(check_device());
+    return launch_router_topk(x_bf16, w_router, bias, T, H, E, n_group, topk_group, top_k, routed_scaling_factor,
+                              renormalize, logits_out, topk_ids, topk_weights, workspace,
+                              static_cast<cudaStream_t>(stream));
+}
+
 nvfp4moe_status quantize_nvfp4(const uint16_t* x_bf16, int64_t M, int64_t K, float gs, uint8_t* codes,
                                uint8_t* e4m3_scales, void* stream) {
     REQUIRE(M >= 0 && K >= 16, NVFP4MOE_ERR_INVALID_ARG, "bad sizes M=%lld K=%lld", (long long)M, (long long)K);

@@ -43,6 +43,12 @@ nvfp4moe_status read_transcode_report(const void* workspace, nvfp4moe_transcode_
 nvfp4moe_status launch_route(const float* logits, const float* bias, int T, int E, int n_group, int topk_group,
                              int top_k, float rsf, int renorm, int32_t* ids, float* wts, cudaStream_t stream);
 
+// router.cu
+size_t router_ws_size(int T);
+nvfp4moe_status launch_router_topk(const uint16_t* x, const float* w, const float* bias, int T, int H, int E,
+                                   int n_group, int topk_group, int top_k, float rsf, int renorm, float* logits,
+                                   int32_t* ids, float* wts, void* workspace, cudaStream_t stream);
+
 // permute.cu
 nvfp4moe_status launch_permute(const int32_t* ids, int T, int k, int E, int pad, RoutingPlan& plan,
                                cudaStream_t stream);

@@ -1,0 +1,303 @@
+// route_token.cuh -- grouped sigmoid top-k routing of one token by one warp,
+// shared by the routing kernel and the fused router-projection kernel.
+//
+// "MiMo-V2.6-Flash -- REAP-50", "Model Summary" and "Pruning Method" 1: experts
+// reshaped to [n_group, E / n_group], keep topk_group groups, top-k experts
+// inside them, weights scaled by routed_scaling_factor; an
+// e_score_correction_bias steers the selection only.  Group score = sum of the
+// group's two largest biased scores; ties go to the lower index; output order is
+// selection order; weights w_j = (s_j / sum s) * rsf (renormalised) or s_j * rsf.
+//
+// Every floating point operation that decides an id or produces a weight is an
+// explicit IEEE FP32 intrinsic (no contraction), and sigmoid uses the specified
+// exp below, so ids and weights are bit-reproducible.  Files including this one
+// are built with -fmad=false.
+#pragma once
+
+#include <cstring>
+
+#include "common.cuh"
+
+namespace nvfp4moe {
+
+struct ExpSpecConsts {
+    float log2e, ln2_hi, ln2_lo;
+};
+
+// Specified FP32 exp: clamp to [-87, 88]; n = rint(y * log2e); Cody-Waite
+// r = fma(-n, ln2_hi, y), r = fma(-n, ln2_lo, r); p = degree-7 Taylor series of
+// e^r in Horner form with fma, coefficients FP32(1/i!); result p * 2^n with 2^n
+// assembled from its exponent bits (n in [-126, 127], always a normal float).
+__device__ __forceinline__ float exp_spec(float y, const ExpSpecConsts& k) {
+    y = fminf(fmaxf(y, -87.0f), 88.0f);
+    const float n = rintf(__fmul_rn(y, k.log2e));
+    float r = __fmaf_rn(-n, k.ln2_hi, y);
+    r = __fmaf_rn(-n, k.ln2_lo, r);
+    float p = (float)(1.0 / 5040.0);
+    p = __fmaf_rn(p, r, (float)(1.0 / 720.0));
+    p = __fmaf_rn(p, r, (float)(1.0 / 120.0));
+    p = __fmaf_rn(p, r, (float)(1.0 / 24.0));
+    p = __fmaf_rn(p, r, (float)(1.0 / 6.0));
+    p = __fmaf_rn(p, r, 0.5f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    const float two_n = __uint_as_float((uint32_t)((int)n + 127) << 23);
+    return __fmul_rn(p, two_n);
+}
+
+__device__ __forceinline__ float sigmoid_spec(float x, const ExpSpecConsts& k) {
+    if (x >= 0.0f) return __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_spec(-x, k)));
+    const float e = exp_spec(x, k);
+    return __fdiv_rn(e, __fadd_rn(1.0f, e));
+}
+
+// (value desc, index asc) lexicographic "better than"
+__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+
+__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+        if (better(ov, oi, v, i)) {
+            v = ov;
+            i = oi;
+        }
+    }
+}
+
+constexpr int RT_WARPS = 8;
+constexpr int RT_MAX_E = 1024;
+constexpr int RT_MAX_NPL = RT_MAX_E / 32;
+
+// Logits written by other CTAs of the same launch are read through L2 (COHERENT);
+// logits that are inputs of the launch through the read-only path.
+template <bool COHERENT>
+__device__ __forceinline__ float load_logit(const float* p) {
+    return COHERENT ? __ldcg(p) : __ldg(p);
+}
+
+// Any group shape.  s_c: this warp's shared scratch of RT_MAX_E + 32 floats.
+template <int NPL, bool COHERENT>
+__device__ __forceinline__ void route_token_general(const float* __restrict__ lg, const float* __restrict__ bias,
+                                                    int64_t t, int E, int n_group, int topk_group, int top_k,
+                                                    float rsf, int renorm, const ExpSpecConsts& kc,
+                                                    int32_t* __restrict__ ids, float* __restrict__ wts, float* s_c) {
+    // biased scores laid out group by group with one pad word per group
+    const int lane = lane_id();
+    const int gsz = E / n_group;
+    float s[NPL], c[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            s[i] = sigmoid_spec(load_logit<COHERENT>(lg + e), kc);
+            c[i] = __fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f);
+            const int g = e / gsz;
+            s_c[g * (gsz + 1) + (e - g * gsz)] = c[i];
+        } else {
+            s[i] = 0.0f;
+            c[i] = -INFINITY;
+        }
+    }
+    __syncwarp();
+    // group scores: lane g scans group g
+    float score = -INFINITY;
+    if (lane < n_group) {
+        const float* gp = &s_c[lane * (gsz + 1)];
+        int i1 = 0;
+        for (int j = 1; j < gsz; ++j)
+            if (gp[j] > gp[i1]) i1 = j;
+        int i2 = -1;
+        for (int j = 0; j < gsz; ++j)
+            if (j != i1 && (i2 < 0 || gp[j] > gp[i2])) i2 = j;
+        score = i2 < 0 ? gp[i1] : __fadd_rn(gp[i1], gp[i2]);
+    }
+    // keep topk_group groups
+    uint32_t chosen = 0;
+    for (int r = 0; r < topk_group; ++r) {
+        float v = (lane < n_group && !((chosen >> lane) & 1u)) ? score : -INFINITY;
+        int idx = (lane < n_group && !((chosen >> lane) & 1u)) ? lane : 0x7fffffff;
+        warp_argmax(v, idx);
+        chosen |= 1u << idx;
+    }
+    // top_k experts inside the chosen groups
+    uint32_t taken = 0;
+    int my_id = 0;
+    float my_s = 0.0f;
+    for (int j = 0; j < top_k; ++j) {
+        float v = -INFINITY;
+        int idx = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && ((chosen >> (e / gsz)) & 1u) && !((taken >> i) & 1u) && better(c[i], e, v, idx)) {
+                v = c[i];
+                idx = e;
+            }
+        }
+        warp_argmax(v, idx);
+        float sv = 0.0f;
+        if ((idx & 31) == lane) {
+            const int i = idx >> 5;
+            taken |= 1u << i;
+#pragma unroll
+            for (int ii = 0; ii < NPL; ++ii)
+                if (ii == i) sv = s[ii];
+        }
+        sv = __shfl_sync(0xffffffffu, sv, idx & 31);
+        if (lane == j) {
+            my_id = idx;
+            my_s = sv;
+        }
+    }
+    float S = 0.0f;
+    for (int j = 0; j < top_k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, my_s, j));
+    if (lane < top_k) {
+        ids[(int64_t)t * top_k + lane] = my_id;
+        wts[(int64_t)t * top_k + lane] = renorm ? __fmul_rn(__fdiv_rn(my_s, S), rsf) : __fmul_rn(my_s, rsf);
+    }
+}
+
+// Fast path for the common group shapes: group size G a power of two <= 32
+// (a group is an aligned run of G lanes of one register row) or a multiple of
+// 32 (a group is G/32 whole register rows).  Group scores come from a
+// segmented warp reduction of (largest, second largest) instead of a
+// sequential scan, and every element's group bit is computed once.  Same
+// arithmetic and tie rules as k_route: the group score is the FP32 sum of the
+// two largest values, which does not depend on which of equal values is taken.
+// s_score: this warp's shared scratch of 32 floats.
+template <int NPL, bool COHERENT>
+__device__ __forceinline__ void route_token_fast(const float* __restrict__ lg, const float* __restrict__ bias,
+                                                 int64_t t, int E, int n_group, int topk_group, int top_k, float rsf,
+                                                 int renorm, const ExpSpecConsts& kc, int32_t* __restrict__ ids,
+                                                 float* __restrict__ wts, float* s_score) {
+    const int lane = lane_id();
+    const int gsz = E / n_group;
+    float s[NPL], c[NPL];
+    uint32_t gbit[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            s[i] = sigmoid_spec(load_logit<COHERENT>(lg + e), kc);
+            c[i] = __fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f);
+            gbit[i] = 1u << (e / gsz);
+        } else {
+            s[i] = 0.0f;
+            c[i] = -INFINITY;
+            gbit[i] = 0u;
+        }
+    }
+    if (gsz <= 32) {
+        // per row: segments of gsz lanes
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            float a = c[i], b = -INFINITY;
+            for (int o = gsz >> 1; o; o >>= 1) {
+                const float pa = __shfl_xor_sync(0xffffffffu, a, o);
+                const float pb = __shfl_xor_sync(0xffffffffu, b, o);
+                b = fmaxf(fminf(a, pa), fmaxf(b, pb));
+                a = fmaxf(a, pa);
+            }
+            const int e = lane + 32 * i;
+            if ((lane & (gsz - 1)) == 0 && e < E) s_score[e / gsz] = __fadd_rn(a, b);
+        }
+    } else {
+        // per group: its rows, then the whole warp
+        const int rows = gsz >> 5;
+        for (int g = 0; g < n_group; ++g) {
+            float a = -INFINITY, b = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+                if (i >= g * rows && i < (g + 1) * rows) {
+                    b = fmaxf(b, fminf(a, c[i]));
+                    a = fmaxf(a, c[i]);
+                }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                const float pa = __shfl_xor_sync(0xffffffffu, a, o);
+                const float pb = __shfl_xor_sync(0xffffffffu, b, o);
+                b = fmaxf(fminf(a, pa), fmaxf(b, pb));
+                a = fmaxf(a, pa);
+            }
+            if (lane == 0) s_score[g] = __fadd_rn(a, b);
+        }
+    }
+    __syncwarp();
+    const float score = lane < n_group ? s_score[lane] : -INFINITY;
+    // keep topk_group groups
+    uint32_t chosen = 0;
+    for (int r = 0; r < topk_group; ++r) {
+        float v = (lane < n_group && !((chosen >> lane) & 1u)) ? score : -INFINITY;
+        int idx = (lane < n_group && !((chosen >> lane) & 1u)) ? lane : 0x7fffffff;
+        warp_argmax(v, idx);
+        chosen |= 1u << idx;
+    }
+    // top_k experts inside the chosen groups
+    float cand[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) cand[i] = (chosen & gbit[i]) ? c[i] : -INFINITY;
+    int my_id = 0;
+    float my_s = 0.0f;
+    for (int j = 0; j < top_k; ++j) {
+        float v = -INFINITY;
+        int idx = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int e = lane + 32 * i;
+            if (cand[i] != -INFINITY && better(cand[i], e, v, idx)) {
+                v = cand[i];
+                idx = e;
+            }
+        }
+        warp_argmax(v, idx);
+        float sv = 0.0f;
+        if ((idx & 31) == lane) {
+            const int hit = idx >> 5;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+                if (i == hit) {
+                    sv = s[i];
+                    cand[i] = -INFINITY;
+                }
+        }
+        sv = __shfl_sync(0xffffffffu, sv, idx & 31);
+        if (lane == j) {
+            my_id = idx;
+            my_s = sv;
+        }
+    }
+    float S = 0.0f;
+    for (int j = 0; j < top_k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, my_s, j));
+    if (lane < top_k) {
+        ids[(int64_t)t * top_k + lane] = my_id;
+        wts[(int64_t)t * top_k + lane] = renorm ? __fmul_rn(__fdiv_rn(my_s, S), rsf) : __fmul_rn(my_s, rsf);
+    }
+}
+
+// The fast path applies: group size a power of two <= 32, or a multiple of 32.
+inline bool route_fast_shape(int E, int n_group) {
+    const int gsz = E / n_group;
+    return n_group <= 32 && gsz >= 2 && ((gsz <= 32 && (gsz & (gsz - 1)) == 0) || gsz % 32 == 0);
+}
+
+inline ExpSpecConsts exp_spec_consts() {
+    // ln2_hi = ln 2 rounded to FP32 with its 12 low mantissa bits cleared;
+    // ln2_lo = FP32(ln 2 - ln2_hi); log2e = FP32(log2 e).
+    const double ln2 = 0.69314718055994530942;
+    float hi = (float)ln2;
+    uint32_t u;
+    memcpy(&u, &hi, 4);
+    u &= 0xFFFFF000u;
+    memcpy(&hi, &u, 4);
+    ExpSpecConsts k;
+    k.log2e = (float)1.44269504088896340736;
+    k.ln2_hi = hi;
+    k.ln2_lo = (float)(ln2 - (double)hi);
+    return k;
+}
+
+}  // namespace nvfp4moe

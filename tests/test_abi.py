@@ -115,3 +115,31 @@ def test_error_string_is_text():
     lib = moe.load()
     lib.moe_route(ctypes.c_void_p(16), None, 4, 0, 1, 1, 1, 1.0, 1, ctypes.c_void_p(16), ctypes.c_void_p(16), None)
     assert b"E=0" in lib.nvfp4moe_last_error_string()
+
+
+@pytest.mark.parametrize("args,expect", [
+    # T, H, E, n_group, topk_group, top_k, workspace bytes
+    ((16, 4096, 254, 2, 1, 8, 64), 3),   # E % 4
+    ((16, 4000, 256, 8, 4, 8, 64), 3),   # H % 256
+    ((16, 128, 256, 8, 4, 8, 64), 3),    # H < 256
+    ((16, 4096, 256, 7, 4, 8, 64), 3),   # E % n_group
+    ((16, 4096, 256, 8, 4, 33, 64), 3),  # top_k > 32
+    ((-2, 4096, 256, 8, 4, 8, 64), 1),   # negative T
+    ((33, 4096, 256, 8, 4, 8, 8), 6),    # workspace below 4 bytes per 16 tokens
+])
+def test_router_topk_rejects_bad_arguments_before_launch(args, expect):
+    T, H, E, ng, tg, k, wsb = args
+    lib = moe.load()
+    fake = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: validation fails first
+    st = lib.moe_router_topk(fake, fake, None, T, H, E, ng, tg, k, ctypes.c_float(2.827), 1, fake, fake, fake, fake,
+                             wsb, None)
+    assert st == expect, moe.load().nvfp4moe_last_error_string()
+
+
+def test_router_topk_zero_tokens_and_sizes():
+    lib = moe.load()
+    assert lib.moe_router_topk(None, None, None, 0, 4096, 256, 8, 4, 8, ctypes.c_float(1.0), 1, None, None, None,
+                               None, 0, None) == 0
+    assert moe.moe_router_topk_workspace_size(16) == 4
+    assert moe.moe_router_topk_workspace_size(17) == 8
+    assert moe.moe_router_topk_workspace_size(0) == 0
