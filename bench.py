@@ -377,6 +377,7 @@ def run_ours(args, rank, world, local_rank):
         res["decode"] = bench_decode(torch, moe, w, args, P)
         del w
         res["transcode"] = bench_transcode(torch, moe, args, P)
+        res["router"] = bench_router(torch, moe, args, P)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(wl, d, args)
     if rank == 0:
@@ -416,6 +417,68 @@ def bench_decode(torch, moe, w, args, P):
             "roofline": {"bound": "hbm", "kernel": "k_w16_gateup + k_w16_down", "achieved": round(achieved, 1),
                          "peak": P["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / P["hbm_gbs"], 4),
                          "traffic": None, "algorithmic_bytes_per_step": int(wbytes)}}
+
+
+def bench_router(torch, moe, args, P):
+    """Router projection + grouped top-k (moe_router_topk) at the decode shape:
+    T=16 BF16 hidden rows x an FP32 router [256, 4096].  Successive calls use the
+    routers of 47 distinct layers (188 MB > L2), as a model stepping through its
+    MoE layers does, so every call reads its router from HBM."""
+    wl = inputs.WORKLOADS["decode"]
+    T, H, E, layers = wl.T, wl.H, wl.E, 47
+    rng = np.random.default_rng(wl.seed + 100)
+    x = torch.from_numpy(inputs.bf16_bits(rng.standard_normal((T, H), dtype=np.float32)).view(np.int16)).cuda()
+    w = torch.empty((layers, E, H), dtype=torch.float32, device="cuda")
+    for l in range(layers):
+        w[l].copy_(torch.from_numpy(inputs.router_weights(rng, E, H)))
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    ids = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(16, moe.moe_router_topk_workspace_size(T)), dtype=torch.uint8, device="cuda")
+
+    def call(l):
+        moe.moe_router_topk(x, w[l], None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf, True, logits, ids, wts, ws)
+
+    for l in range(layers):
+        call(l)
+    torch.cuda.synchronize()
+    reps = max(args.steps, 20)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # eager: one library call per layer from Python (host-bound at this size)
+    a.record()
+    for i in range(reps * layers):
+        call(i % layers)
+    b.record()
+    torch.cuda.synchronize()
+    eager_us = a.elapsed_time(b) / (reps * layers) * 1e3
+    # device time: the 47 calls captured once in a CUDA graph, as a decode step is
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=cs):
+        for l in range(layers):
+            call(l)
+    g.replay()
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    moe.nvfp4moe_check_device_status()
+    us = a.elapsed_time(b) / (reps * layers) * 1e3
+    del g
+    nbytes = E * H * 4 + T * H * 2 + T * E * 4 + T * wl.top_k * 8
+    gbs = nbytes / (us / 1e6) / 1e9
+    del w
+    torch.cuda.empty_cache()
+    return {"workload": f"router: T={T} H={H} E={E} groups={wl.n_group} keep={wl.topk_group} top_k={wl.top_k}, "
+                        f"FP32 router, {layers} layers' routers rotated (> L2)",
+            "value": round(us, 2), "unit": "us per layer (CUDA graph of 47 layers' calls)",
+            "higher_is_better": False, "eager_us_per_call": round(eager_us, 2),
+            "roofline": {"bound": "hbm", "kernel": "k_router_topk", "achieved": round(gbs, 1), "peak": P["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / P["hbm_gbs"], 4), "traffic": None,
+                         "algorithmic_bytes_per_launch": int(nbytes)}}
 
 
 def bench_transcode(torch, moe, args, P):

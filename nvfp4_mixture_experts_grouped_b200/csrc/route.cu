@@ -18,6 +18,17 @@ __global__ void __launch_bounds__(RT_WARPS * 32)
 
 template <int NPL>
 __global__ void __launch_bounds__(RT_WARPS * 32)
+    k_route_rows(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int n_group,
+                 int topk_group, int top_k, float rsf, int renorm, ExpSpecConsts kc, int32_t* __restrict__ ids,
+                 float* __restrict__ wts) {
+    const int t = blockIdx.x * RT_WARPS + warp_id();
+    if (t >= T) return;
+    route_token_rows<NPL, false>(logits + (int64_t)t * E, bias, t, E, n_group, topk_group, top_k, rsf, renorm, kc, ids,
+                                 wts);
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(RT_WARPS * 32)
     k_route_fast(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int n_group,
                  int topk_group, int top_k, float rsf, int renorm, ExpSpecConsts kc, int32_t* __restrict__ ids,
                  float* __restrict__ wts) {
@@ -35,10 +46,13 @@ nvfp4moe_status launch_route(const float* logits, const float* bias, int T, int 
     const ExpSpecConsts kc = exp_spec_consts();
     const dim3 grid((unsigned)ceil_div(T, RT_WARPS));
     const int npl = (int)ceil_div(E, 32);
-    const bool fast = route_fast_shape(E, n_group);
+    const RouteShape shape = route_shape(E, n_group);
 #define RT_LAUNCH(N)                                                                                              \
     do {                                                                                                          \
-        if (fast)                                                                                                 \
+        if (shape == ROUTE_ROWS)                                                                                  \
+            k_route_rows<N><<<grid, RT_WARPS * 32, 0, stream>>>(logits, bias, T, E, n_group, topk_group, top_k,  \
+                                                                rsf, renorm, kc, ids, wts);                       \
+        else if (shape == ROUTE_SEGMENTS)                                                                         \
             k_route_fast<N><<<grid, RT_WARPS * 32, 0, stream>>>(logits, bias, T, E, n_group, topk_group, top_k,  \
                                                                 rsf, renorm, kc, ids, wts);                       \
         else                                                                                                      \

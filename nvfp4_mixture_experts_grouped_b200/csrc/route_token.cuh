@@ -14,6 +14,7 @@
 // are built with -fmad=false.
 #pragma once
 
+#include <climits>
 #include <cstring>
 
 #include "common.cuh"
@@ -89,11 +90,14 @@ __device__ __forceinline__ void route_token_general(const float* __restrict__ lg
     const int lane = lane_id();
     const int gsz = E / n_group;
     float s[NPL], c[NPL];
+    // all of the lane's logits are loaded before any sigmoid, so the loads overlap
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) s[i] = lane + 32 * i < E ? load_logit<COHERENT>(lg + lane + 32 * i) : 0.0f;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
         if (e < E) {
-            s[i] = sigmoid_spec(load_logit<COHERENT>(lg + e), kc);
+            s[i] = sigmoid_spec(s[i], kc);
             c[i] = __fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f);
             const int g = e / gsz;
             s_c[g * (gsz + 1) + (e - g * gsz)] = c[i];
@@ -178,11 +182,14 @@ __device__ __forceinline__ void route_token_fast(const float* __restrict__ lg, c
     const int gsz = E / n_group;
     float s[NPL], c[NPL];
     uint32_t gbit[NPL];
+    // all of the lane's logits are loaded before any sigmoid, so the loads overlap
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) s[i] = lane + 32 * i < E ? load_logit<COHERENT>(lg + lane + 32 * i) : 0.0f;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
         if (e < E) {
-            s[i] = sigmoid_spec(load_logit<COHERENT>(lg + e), kc);
+            s[i] = sigmoid_spec(s[i], kc);
             c[i] = __fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f);
             gbit[i] = 1u << (e / gsz);
         } else {
@@ -278,10 +285,136 @@ __device__ __forceinline__ void route_token_fast(const float* __restrict__ lg, c
     }
 }
 
-// The fast path applies: group size a power of two <= 32, or a multiple of 32.
-inline bool route_fast_shape(int E, int n_group) {
+// Order-preserving int key of a float (larger float -> larger key; -0 and NaN
+// do not occur here: c = sigmoid + bias).  KEY_NONE is below every key.
+__device__ __forceinline__ int32_t okey(float v) {
+    const int32_t b = __float_as_int(v);
+    return b >= 0 ? b : b ^ 0x7FFFFFFF;
+}
+__device__ __forceinline__ float okey_value(int32_t k) { return __int_as_float(k >= 0 ? k : k ^ 0x7FFFFFFF); }
+constexpr int32_t KEY_NONE = INT32_MIN;
+
+// Group size a multiple of 32 (a group is whole register rows): the same
+// selections as route_token_fast, with every warp-wide arg-max done by two
+// warp reductions -- the largest key, then the lowest index holding it (the
+// lower-index tie rule) -- instead of shuffle butterflies.
+template <int NPL, bool COHERENT>
+__device__ __forceinline__ void route_token_rows(const float* __restrict__ lg, const float* __restrict__ bias,
+                                                 int64_t t, int E, int n_group, int topk_group, int top_k, float rsf,
+                                                 int renorm, const ExpSpecConsts& kc, int32_t* __restrict__ ids,
+                                                 float* __restrict__ wts) {
+    const int lane = lane_id();
+    const int rows = (E / n_group) >> 5;  // register rows per group
+    float s[NPL];
+    int32_t key[NPL];
+    // all of the lane's logits are loaded before any sigmoid, so the loads overlap
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) s[i] = lane + 32 * i < E ? load_logit<COHERENT>(lg + lane + 32 * i) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            s[i] = sigmoid_spec(s[i], kc);
+            key[i] = okey(__fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f));
+        } else {
+            s[i] = 0.0f;
+            key[i] = KEY_NONE;
+        }
+    }
+    // group scores: the group's largest and second largest c (equal values count twice)
+    int32_t gkey = KEY_NONE;  // lane g: key of group g's score
+    if (rows == 1) {
+        // one register row per group: the rows' reductions are independent and overlap
+#pragma unroll
+        for (int g = 0; g < NPL; ++g)
+            if (g < n_group) {
+                const int32_t m1 = __reduce_max_sync(0xffffffffu, key[g]);
+                const uint32_t holders = __ballot_sync(0xffffffffu, key[g] == m1);
+                const int32_t m2 = __popc(holders) >= 2
+                                       ? m1
+                                       : __reduce_max_sync(0xffffffffu, (holders >> lane) & 1u ? KEY_NONE : key[g]);
+                if (lane == g) gkey = okey(__fadd_rn(okey_value(m1), okey_value(m2)));
+            }
+    } else {
+        for (int g = 0; g < n_group; ++g) {
+            int32_t a = KEY_NONE, b = KEY_NONE;  // this lane's largest, second largest in the group
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+                if (i >= g * rows && i < (g + 1) * rows) {
+                    const int32_t k = key[i];
+                    b = max(b, min(a, k));
+                    a = max(a, k);
+                }
+            const int32_t m1 = __reduce_max_sync(0xffffffffu, a);
+            const uint32_t holders = __ballot_sync(0xffffffffu, a == m1);
+            int32_t m2;
+            if (__popc(holders) >= 2)
+                m2 = m1;
+            else
+                m2 = __reduce_max_sync(0xffffffffu, (holders >> lane) & 1u ? b : a);
+            if (lane == g) gkey = okey(__fadd_rn(okey_value(m1), okey_value(m2)));
+        }
+    }
+    // keep topk_group groups: largest score, ties to the lower group
+    uint32_t chosen = 0;
+    for (int r = 0; r < topk_group; ++r) {
+        const bool elig = lane < n_group && !((chosen >> lane) & 1u);
+        const int32_t m = __reduce_max_sync(0xffffffffu, elig ? gkey : KEY_NONE);
+        const uint32_t g = __reduce_min_sync(0xffffffffu, elig && gkey == m ? (uint32_t)lane : 32u);
+        chosen |= 1u << g;
+    }
+    // top_k experts inside the chosen groups: largest c, ties to the lower expert
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+        if (!((chosen >> (i / rows)) & 1u)) key[i] = KEY_NONE;
+    int my_id = 0;
+    float my_s = 0.0f;
+    for (int j = 0; j < top_k; ++j) {
+        int32_t lk = KEY_NONE;
+        int li = 0;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+            if (key[i] > lk) {  // strict: the lower row (lower expert) keeps a tie
+                lk = key[i];
+                li = i;
+            }
+        const int32_t m = __reduce_max_sync(0xffffffffu, lk);
+        const uint32_t idx =
+            __reduce_min_sync(0xffffffffu, lk == m && lk != KEY_NONE ? (uint32_t)(lane + 32 * li) : 0x7fffffffu);
+        float sv = 0.0f;
+        if ((int)(idx & 31) == lane) {
+            const int hit = (int)(idx >> 5);
+#pragma unroll
+            for (int i = 0; i < NPL; ++i)
+                if (i == hit) {
+                    sv = s[i];
+                    key[i] = KEY_NONE;
+                }
+        }
+        sv = __shfl_sync(0xffffffffu, sv, idx & 31);
+        if (lane == j) {
+            my_id = (int)idx;
+            my_s = sv;
+        }
+    }
+    float S = 0.0f;
+    for (int j = 0; j < top_k; ++j) S = __fadd_rn(S, __shfl_sync(0xffffffffu, my_s, j));
+    if (lane < top_k) {
+        ids[t * top_k + lane] = my_id;
+        wts[t * top_k + lane] = renorm ? __fmul_rn(__fdiv_rn(my_s, S), rsf) : __fmul_rn(my_s, rsf);
+    }
+}
+
+// Which per-token routine a group shape takes: whole register rows per group
+// (group size a multiple of 32), segments of one row (a power of two <= 32), or
+// the general one.
+enum RouteShape { ROUTE_GENERAL = 0, ROUTE_SEGMENTS = 1, ROUTE_ROWS = 2 };
+inline RouteShape route_shape(int E, int n_group) {
     const int gsz = E / n_group;
-    return n_group <= 32 && gsz >= 2 && ((gsz <= 32 && (gsz & (gsz - 1)) == 0) || gsz % 32 == 0);
+    if (n_group > 32) return ROUTE_GENERAL;
+    if (gsz % 32 == 0) return ROUTE_ROWS;
+    if (gsz >= 2 && gsz <= 32 && (gsz & (gsz - 1)) == 0) return ROUTE_SEGMENTS;
+    return ROUTE_GENERAL;
 }
 
 inline ExpSpecConsts exp_spec_consts() {
