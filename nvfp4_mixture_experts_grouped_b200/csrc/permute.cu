@@ -37,20 +37,30 @@ __global__ void __launch_bounds__(PERM_CHUNK)
 //    of the tcgen05 path), active list
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int& total) {
-    // blockDim.x == 1024
-    const int tid = threadIdx.x;
-    s_tmp[tid] = v;
-    __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-        const int add = tid >= o ? s_tmp[tid - o] : 0;
-        __syncthreads();
-        s_tmp[tid] += add;
-        __syncthreads();
+    // blockDim.x == 1024: a shuffle scan inside each warp, then over the 32 warp totals
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
     }
-    total = s_tmp[1023];
-    const int incl = s_tmp[tid];
+    if (lane == 31) s_tmp[warp] = x;
     __syncthreads();
-    return incl - v;
+    if (warp == 0) {
+        int w = s_tmp[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        s_tmp[lane] = w;
+    }
+    __syncthreads();
+    const int before = warp > 0 ? s_tmp[warp - 1] : 0;
+    total = s_tmp[31];
+    __syncthreads();  // s_tmp is reused by the next scan
+    return before + x - v;
 }
 
 __global__ void __launch_bounds__(1024)
@@ -140,8 +150,82 @@ __global__ void __launch_bounds__(PERM_CHUNK)
     }
 }
 
+// ---------------------------------------------------------------------------
+// 1-3 in one CTA for up to PERM_FUSED_MAX_PAIRS pairs and E <= 256: per-warp
+// histograms over contiguous pair chunks, the same scans as k_scan_experts,
+// then stable ranks from match_any over 32-pair batches (a warp's chunk in pair
+// order, warps in order), so every output equals the three-kernel path's.
+// ---------------------------------------------------------------------------
+constexpr int PERM_FUSED_MAX_E = 256;
+constexpr int PERM_FUSED_MAX_PAIRS = 8192;  // one CTA beats three launches below ~10K pairs
+
+__global__ void __launch_bounds__(1024)
+    k_permute_fused(const int32_t* __restrict__ ids, int T, int k, int E, int pad, RoutingPlan plan) {
+    __shared__ int s_wc[32 * PERM_FUSED_MAX_E];  // per-warp counts, then per-warp rank bases
+    __shared__ int s_tmp[1024];
+    __shared__ int s_poff[PERM_FUSED_MAX_E];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int P = T * k;
+    const int chunk = (P + 31) / 32;
+    const int p0 = min(P, warp * chunk), p1 = min(P, p0 + chunk);
+    for (int i = tid; i < 32 * E; i += 1024) s_wc[i] = 0;
+    __syncthreads();
+    for (int p = p0 + lane; p < p1; p += 32) atomicAdd(&s_wc[warp * E + ids[p]], 1);
+    __syncthreads();
+    int cnt = 0;
+    if (tid < E) {
+        for (int w = 0; w < 32; ++w) {
+            const int v = s_wc[w * E + tid];
+            s_wc[w * E + tid] = cnt;
+            cnt += v;
+        }
+    }
+    int total, ptotal, ttotal, atotal;
+    const int off = block_exclusive_scan(cnt, s_tmp, total);
+    const int padded = tid < E ? (int)round_up_dev(cnt, pad) : 0;
+    const int poff = block_exclusive_scan(padded, s_tmp, ptotal);
+    const int tiles = tid < E ? (cnt + PAIR_ROWS - 1) / PAIR_ROWS : 0;
+    const int toff = block_exclusive_scan(tiles, s_tmp, ttotal);
+    const int aoff = block_exclusive_scan(tid < E && cnt > 0 ? 1 : 0, s_tmp, atotal);
+    if (tid < E) {
+        plan.counts[tid] = cnt;
+        plan.offsets[tid] = off;
+        plan.pad_offsets[tid] = poff;
+        s_poff[tid] = poff;
+        for (int j = 0; j < tiles; ++j)
+            plan.tiles[toff + j] = make_int4(tid, poff + j * PAIR_ROWS, min(PAIR_ROWS, cnt - j * PAIR_ROWS), j);
+        if (cnt > 0) plan.active[aoff] = tid;
+    }
+    if (tid == 0) {
+        plan.offsets[E] = total;
+        plan.pad_offsets[E] = ptotal;
+        plan.n_tiles[0] = ttotal;
+        plan.n_active[0] = atotal;
+    }
+    __syncthreads();
+    for (int b = p0; b < p1; b += 32) {
+        const int p = b + lane;
+        const bool valid = p < p1;
+        const int e = valid ? ids[p] : -1 - lane;  // lanes past the chunk: keys of their own
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        if (valid) {
+            const int row = s_poff[e] + s_wc[warp * E + e] + __popc(same & ((1u << lane) - 1u));
+            plan.row_of_pair[p] = row;
+            plan.pair_of_row[row] = p;
+        }
+        __syncwarp();
+        if (valid && lane == __ffs(same) - 1) s_wc[warp * E + e] += __popc(same);
+        __syncwarp();
+    }
+}
+
 nvfp4moe_status launch_permute(const int32_t* ids, int T, int k, int E, int pad, RoutingPlan& plan,
                                cudaStream_t stream) {
+    if (E <= PERM_FUSED_MAX_E && (int64_t)T * k <= PERM_FUSED_MAX_PAIRS) {
+        k_permute_fused<<<1, 1024, 0, stream>>>(ids, T, k, E, pad, plan);
+        NVFP4MOE_CHECK_LAUNCH("permute kernel");
+        return NVFP4MOE_OK;
+    }
     const int n_chunks = (int)ceil_div(T, PERM_CHUNK);
     k_count_chunks<<<n_chunks, PERM_CHUNK, E * sizeof(int), stream>>>(ids, T, k, E, plan.chunk_counts);
     NVFP4MOE_CHECK_LAUNCH("permute count kernel");
