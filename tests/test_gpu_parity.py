@@ -148,7 +148,9 @@ def test_route_extreme_logits():
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("T,E,k,pad", [(32, 16, 4, 128), (16, 256, 8, 1), (1000, 64, 6, 128), (8192, 256, 8, 128),
-                                       (3, 8, 8, 1), (600, 1024, 32, 1)])
+                                       (3, 8, 8, 1), (600, 1024, 32, 1),
+                                       # both sides of the one-CTA path's limit (8192 pairs, E <= 256)
+                                       (1024, 256, 8, 128), (1025, 256, 8, 128), (2048, 256, 4, 1), (64, 257, 8, 1)])
 def test_permute_against_oracle(T, E, k, pad):
     rng = np.random.default_rng(T + E)
     ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
