@@ -196,8 +196,10 @@ def quantize_f32(x: np.ndarray, gs: float = 1.0):
 
 def moe_layer(mode: int, x_bits, logits, bias, gate_codes, gate_sf, up_codes, up_sf, down_codes, down_sf,
               w_global, act_global: float, n_group: int, topk_group: int, top_k: int, rsf: float,
-              renormalize: bool = True, tokens=None) -> np.ndarray:
-    """float64 layer output [len(tokens), H] (mode 0 = W4A16, 1 = W4A4)."""
+              renormalize: bool = True, tokens=None, act_global_mid=None) -> np.ndarray:
+    """float64 layer output [len(tokens), H] (mode 0 = W4A16, 1 = W4A4).  act_global
+    scales the layer input's quantisation, act_global_mid (default: the same) the
+    down-projection input's."""
     x = np.ascontiguousarray(x_bits, np.uint16)
     T, H = x.shape
     E, I = gate_codes.shape[0], gate_codes.shape[1]
@@ -209,9 +211,10 @@ def moe_layer(mode: int, x_bits, logits, bias, gate_codes, gate_sf, up_codes, up
     lg = np.ascontiguousarray(logits, np.float32)
     wg = np.ascontiguousarray(w_global, np.float32)
     b = None if bias is None else np.ascontiguousarray(bias, np.float32)
-    _load().orc_moe_layer(ctypes.c_int(mode), _p(x), _p(lg), None if b is None else _p(b), *[_p(a) for a in arrs],
-                          _p(wg), ctypes.c_float(act_global), ctypes.c_int(T), ctypes.c_int(H), ctypes.c_int(I),
-                          ctypes.c_int(E), ctypes.c_int(n_group), ctypes.c_int(topk_group), ctypes.c_int(top_k),
-                          ctypes.c_float(rsf), ctypes.c_int(int(renormalize)), _p(tokens), ctypes.c_int(len(tokens)),
-                          _p(out))
+    mid = act_global if act_global_mid is None else act_global_mid
+    _load().orc_moe_layer2(ctypes.c_int(mode), _p(x), _p(lg), None if b is None else _p(b), *[_p(a) for a in arrs],
+                           _p(wg), ctypes.c_float(act_global), ctypes.c_float(mid), ctypes.c_int(T), ctypes.c_int(H),
+                           ctypes.c_int(I), ctypes.c_int(E), ctypes.c_int(n_group), ctypes.c_int(topk_group),
+                           ctypes.c_int(top_k), ctypes.c_float(rsf), ctypes.c_int(int(renormalize)), _p(tokens),
+                           ctypes.c_int(len(tokens)), _p(out))
     return out

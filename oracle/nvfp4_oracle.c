@@ -464,11 +464,15 @@ static void decode_row(const uint8_t* codes, const uint8_t* sf, double global, i
         out[k] = orc_e2m1_value(nibble(codes, k)) * orc_e4m3_value(sf[k / 16]) * global;
 }
 
-void orc_moe_layer(int mode, const uint16_t* x, const float* logits, const float* bias, const uint8_t* gate_codes,
-                   const uint8_t* gate_sf, const uint8_t* up_codes, const uint8_t* up_sf, const uint8_t* down_codes,
-                   const uint8_t* down_sf, const float* w_global, float act_global, int T, int H, int I, int E,
-                   int n_group, int topk_group, int top_k, float rsf, int renormalize, const int32_t* tokens,
-                   int n_tokens, double* out) {
+/* The layer with separate activation global scales for the layer input
+ * (act_global) and the down-projection input (act_global_mid): [P1] "Why a unit
+ * activation scale" compares calibrated per-layer scales, the down-projection
+ * input's scale capped at 2688, and a unit scale everywhere. */
+void orc_moe_layer2(int mode, const uint16_t* x, const float* logits, const float* bias, const uint8_t* gate_codes,
+                    const uint8_t* gate_sf, const uint8_t* up_codes, const uint8_t* up_sf, const uint8_t* down_codes,
+                    const uint8_t* down_sf, const float* w_global, float act_global, float act_global_mid, int T,
+                    int H, int I, int E, int n_group, int topk_group, int top_k, float rsf, int renormalize,
+                    const int32_t* tokens, int n_tokens, double* out) {
     (void)T;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int it = 0; it < n_tokens; ++it) {
@@ -512,9 +516,9 @@ void orc_moe_layer(int mode, const uint16_t* x, const float* logits, const float
             }
             if (mode == 1) {
                 for (int i = 0; i < I; ++i) a32[i] = (float)a[i];
-                orc_quantize_f32(a32, 1, I, act_global, aq, as);
+                orc_quantize_f32(a32, 1, I, act_global_mid, aq, as);
                 for (int i = 0; i < I; ++i)
-                    a[i] = orc_e2m1_value(nibble(aq, i)) * orc_e4m3_value(as[i / 16]) * (double)act_global;
+                    a[i] = orc_e2m1_value(nibble(aq, i)) * orc_e4m3_value(as[i / 16]) * (double)act_global_mid;
             } else {
                 for (int i = 0; i < I; ++i) a[i] = (double)orc_bf16_to_float(orc_float_to_bf16((float)a[i]));
             }
@@ -533,6 +537,17 @@ void orc_moe_layer(int mode, const uint16_t* x, const float* logits, const float
         free(aq);
         free(as);
     }
+}
+
+/* One activation global scale for both quantisations (the pages' unit scale). */
+void orc_moe_layer(int mode, const uint16_t* x, const float* logits, const float* bias, const uint8_t* gate_codes,
+                   const uint8_t* gate_sf, const uint8_t* up_codes, const uint8_t* up_sf, const uint8_t* down_codes,
+                   const uint8_t* down_sf, const float* w_global, float act_global, int T, int H, int I, int E,
+                   int n_group, int topk_group, int top_k, float rsf, int renormalize, const int32_t* tokens,
+                   int n_tokens, double* out) {
+    orc_moe_layer2(mode, x, logits, bias, gate_codes, gate_sf, up_codes, up_sf, down_codes, down_sf, w_global,
+                   act_global, act_global, T, H, I, E, n_group, topk_group, top_k, rsf, renormalize, tokens, n_tokens,
+                   out);
 }
 
 /* Routing weights/ids for a subset of tokens, for the sampled-token checks. */

@@ -395,6 +395,36 @@ def test_layer_reduces_to_dense_swiglu(mode):
     assert np.allclose(out, Y, rtol=1e-12, atol=1e-12 * np.abs(Y).max())
 
 
+@pytest.mark.parametrize("gs_in,gs_mid", [(0.37, 2.5), (116.0, 1.0), (1.0, 0.03125)])
+def test_layer_separate_input_and_intermediate_scales(gs_in, gs_mid):
+    # "Why a unit activation scale": calibrated per-layer scales, the down input's
+    # capped at 2688, or unit.  Dense reduction (E=1, k=1, rsf=1) against the
+    # quantiser pins: x quantised with gs_in, the SwiGLU output with gs_mid.
+    rng = np.random.default_rng(41)
+    T, H, I = 4, 64, 32
+    gc, gs, _ = inputs.nvfp4_tensors(rng, 1, I, H)
+    uc, us, _ = inputs.nvfp4_tensors(rng, 1, I, H)
+    dc, ds, _ = inputs.nvfp4_tensors(rng, 1, H, I)
+    wg = np.array([[0.5, 0.25, 2.0]], np.float32)
+    x = inputs.activations(rng, T, H, outliers=True)
+    logits = rng.standard_normal((T, 1)).astype(np.float32)
+    out = oracle.moe_layer(1, x, logits, None, gc, gs, uc, us, dc, ds, wg, gs_in, 1, 1, 1, 1.0,
+                           act_global_mid=gs_mid)
+    qc, qs = oracle.quantize_bf16(x, gs_in)
+    xf = _np_decode(qc, qs, gs_in)
+    G = xf @ _np_decode(gc[0], gs[0], 0.5).T
+    U = xf @ _np_decode(uc[0], us[0], 0.25).T
+    A = G / (1 + np.exp(-G)) * U
+    ac, as_ = oracle.quantize_f32(A.astype(np.float32), gs_mid)
+    Y = _np_decode(ac, as_, gs_mid) @ _np_decode(dc[0], ds[0], 2.0).T
+    assert np.allclose(out, Y, rtol=1e-12, atol=1e-12 * np.abs(Y).max())
+    # the two scales are not interchangeable
+    if gs_in != gs_mid:
+        swapped = oracle.moe_layer(1, x, logits, None, gc, gs, uc, us, dc, ds, wg, gs_mid, 1, 1, 1, 1.0,
+                                   act_global_mid=gs_in)
+        assert not np.allclose(swapped, Y, rtol=1e-6)
+
+
 def test_layer_combines_two_experts_with_routing_weights():
     rng = np.random.default_rng(33)
     T, H, I, E = 4, 32, 16, 2
