@@ -224,7 +224,8 @@ nvfp4moe_status quantize_nvfp4(const uint16_t* x_bf16, int64_t M, int64_t K, flo
  *                   to BF16.  Meant for decode-sized batches.
  *   NVFP4MOE_W4A4:  activations quantised to NVFP4 with global act_global (1.0
  *                   in the pages' recipe); FP4 x FP4 block-scaled tcgen05 MMA;
- *                   SwiGLU output requantised per 16 with the same global.
+ *                   SwiGLU output requantised per 16 with the same global
+ *                   (moe_forward_ex takes a separate global for it).
  * FP32 accumulation throughout; the combine adds the k weighted expert rows of a
  * token in slot order in FP32 and rounds once to the output type.
  *
@@ -283,6 +284,27 @@ nvfp4moe_status moe_forward_routed(nvfp4moe_mode mode, const uint16_t* x, const 
                                    const float* topk_weights, const void* packed_weights, float act_global, int32_t T,
                                    int32_t H, int32_t I, int32_t E, int32_t top_k, void* workspace,
                                    size_t workspace_bytes, void* out, int32_t out_is_fp32, void* stream);
+
+/* moe_forward with one activation global scale per GEMM input
+ * ("AxionML / MiMo-V2.6-Flash-MOPD-NVFP4", "Why a unit activation scale": a
+ * calibrated scale per layer, optionally with the down-projection input's
+ * amax capped, is the alternative to the shipped unit scale).
+ *   act_global_in:  global of the layer input's NVFP4 codes (W4A4): the input is
+ *                   quantised as x / act_global_in per 16-element block and the
+ *                   gate/up products are scaled back by it.
+ *   act_global_mid: global of the SwiGLU output's NVFP4 codes, the
+ *                   down-projection input (W4A4).
+ * Both finite and > 0 (also in W4A16 mode, where they are not used: that mode
+ * keeps its activations in BF16).  moe_forward(..., g, ...) is
+ * moe_forward_ex(..., g, g, ...).  A unit global covers magnitudes up to
+ * 6 * 448 = 2688 (largest E2M1 code times largest E4M3 block scale); a
+ * calibrated global is amax / 2688 of the tensor it quantises.              */
+nvfp4moe_status moe_forward_ex(nvfp4moe_mode mode, const uint16_t* x, const float* router_logits, const float* bias,
+                               const void* packed_weights, float act_global_in, float act_global_mid, int32_t T,
+                               int32_t H, int32_t I, int32_t E, int32_t n_group, int32_t topk_group, int32_t top_k,
+                               float routed_scaling_factor, int32_t renormalize, void* workspace,
+                               size_t workspace_bytes, void* out, int32_t out_is_fp32, int32_t* topk_ids_out,
+                               float* topk_weights_out, void* stream);
 
 /* Stage tracing.  When `events` is non-NULL, every later moe_forward /
  * moe_forward_routed call on this host thread records the cudaEvent_t handles

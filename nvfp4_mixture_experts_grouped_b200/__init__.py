@@ -17,7 +17,7 @@ __all__ = [
     "transcode_mxfp4_to_nvfp4", "nvfp4moe_transcode_workspace_size", "moe_route", "moe_router_topk",
     "moe_router_topk_workspace_size", "quantize_nvfp4",
     "moe_packed_weights_size", "moe_pack_weights", "moe_forward_workspace_size", "moe_forward",
-    "moe_forward_routed", "nvfp4moe_check_device_status", "nvfp4moe_version", "moe_permute",
+    "moe_forward_ex", "moe_forward_routed", "nvfp4moe_check_device_status", "nvfp4moe_version", "moe_permute",
     "moe_permute_workspace_size", "nvfp4moe_set_trace_events", "moe_permute_noalloc",
 ]
 
@@ -90,6 +90,9 @@ def load():
     L.moe_forward.restype = ctypes.c_int
     L.moe_forward.argtypes = [ctypes.c_int, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, i32, i32, f32, i32, vp, sz, vp,
                               i32, vp, vp, vp]
+    L.moe_forward_ex.restype = ctypes.c_int
+    L.moe_forward_ex.argtypes = [ctypes.c_int, vp, vp, vp, vp, f32, f32, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+                                 vp, sz, vp, i32, vp, vp, vp]
     L.moe_forward_routed.restype = ctypes.c_int
     L.moe_forward_routed.argtypes = [ctypes.c_int, vp, vp, vp, vp, f32, i32, i32, i32, i32, i32, vp, sz, vp, i32, vp]
     L.moe_permute_workspace_size.restype = sz
@@ -220,6 +223,18 @@ def moe_forward(mode, x, router_logits, bias, packed_weights, act_global, T, H, 
                               I, E, n_group, topk_group, top_k, routed_scaling_factor, int(renormalize),
                               _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), out_f32,
                               _ptr(topk_ids_out), _ptr(topk_weights_out), _stream(stream)))
+
+
+def moe_forward_ex(mode, x, router_logits, bias, packed_weights, act_global_in, act_global_mid, T, H, I, E, n_group,
+                   topk_group, top_k, routed_scaling_factor, renormalize, workspace, out, topk_ids_out=None,
+                   topk_weights_out=None, stream=None):
+    import torch
+
+    out_f32 = 1 if out.dtype == torch.float32 else 0
+    _check(load().moe_forward_ex(mode, _ptr(x), _ptr(router_logits), _ptr(bias), _ptr(packed_weights), act_global_in,
+                                 act_global_mid, T, H, I, E, n_group, topk_group, top_k, routed_scaling_factor,
+                                 int(renormalize), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _ptr(out), out_f32, _ptr(topk_ids_out), _ptr(topk_weights_out), _stream(stream)))
 
 
 def moe_forward_routed(mode, x, topk_ids, topk_weights, packed_weights, act_global, T, H, I, E, top_k, workspace, out,

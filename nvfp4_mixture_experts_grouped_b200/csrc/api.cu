@@ -361,7 +361,8 @@ size_t moe_forward_workspace_size(nvfp4moe_mode mode, int32_t T, int32_t H, int3
 
 static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, const float* logits, const float* bias,
                                       const int32_t* ids_in, const float* wts_in, const void* packed,
-                                      float act_global, int32_t T, int32_t H, int32_t I, int32_t E, int32_t n_group,
+                                      float act_global, float act_global_mid, int32_t T, int32_t H, int32_t I,
+                                      int32_t E, int32_t n_group,
                                       int32_t topk_group, int32_t top_k, float rsf, int32_t renorm, void* workspace,
                                       size_t workspace_bytes, void* out, int32_t out_is_fp32, int32_t* ids_out,
                                       float* wts_out, void* stream) {
@@ -376,6 +377,8 @@ static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, con
     }
     REQUIRE(std::isfinite(act_global) && act_global > 0.0f, NVFP4MOE_ERR_INVALID_ARG,
             "act_global must be finite and > 0");
+    REQUIRE(std::isfinite(act_global_mid) && act_global_mid > 0.0f, NVFP4MOE_ERR_INVALID_ARG,
+            "act_global_mid must be finite and > 0");
     REQUIRE(std::isfinite(rsf), NVFP4MOE_ERR_INVALID_ARG, "routed_scaling_factor is not finite");
     if (T == 0) return NVFP4MOE_OK;
     REQUIRE(x && packed && workspace && out, NVFP4MOE_ERR_INVALID_ARG, "null pointer");
@@ -407,7 +410,7 @@ static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, con
         uint8_t* a1s = ws + L.a1s;
         RETURN_IF(launch_quantize_scatter(x, T, H, act_global, a1c, a1s, plan.row_of_pair, top_k, st));
         trace(3, st);
-        RETURN_IF(launch_w4a4_layer(packed, T, H, I, E, top_k, act_global, L.rows_max, (int)L.max_tiles, plan, a1c,
+        RETURN_IF(launch_w4a4_layer(packed, T, H, I, E, top_k, act_global, act_global_mid, L.rows_max, (int)L.max_tiles, plan, a1c,
                                     a1s, ws + L.a2c, ws + L.a2s, static_cast<__half*>(Y), ys, st,
                                     g_trace_on ? g_trace[4] : nullptr));
     } else {
@@ -429,9 +432,21 @@ nvfp4moe_status moe_forward(nvfp4moe_mode mode, const uint16_t* x, const float* 
                             int32_t renormalize, void* workspace, size_t workspace_bytes, void* out,
                             int32_t out_is_fp32, int32_t* topk_ids_out, float* topk_weights_out, void* stream) {
     if (T > 0 && !router_logits) return fail(NVFP4MOE_ERR_INVALID_ARG, "router_logits is null");
-    return forward_common(mode, x, router_logits, bias, nullptr, nullptr, packed_weights, act_global, T, H, I, E,
-                          n_group, topk_group, top_k, routed_scaling_factor, renormalize, workspace, workspace_bytes,
-                          out, out_is_fp32, topk_ids_out, topk_weights_out, stream);
+    return forward_common(mode, x, router_logits, bias, nullptr, nullptr, packed_weights, act_global, act_global, T,
+                          H, I, E, n_group, topk_group, top_k, routed_scaling_factor, renormalize, workspace,
+                          workspace_bytes, out, out_is_fp32, topk_ids_out, topk_weights_out, stream);
+}
+
+nvfp4moe_status moe_forward_ex(nvfp4moe_mode mode, const uint16_t* x, const float* router_logits, const float* bias,
+                               const void* packed_weights, float act_global_in, float act_global_mid, int32_t T,
+                               int32_t H, int32_t I, int32_t E, int32_t n_group, int32_t topk_group, int32_t top_k,
+                               float routed_scaling_factor, int32_t renormalize, void* workspace,
+                               size_t workspace_bytes, void* out, int32_t out_is_fp32, int32_t* topk_ids_out,
+                               float* topk_weights_out, void* stream) {
+    if (T > 0 && !router_logits) return fail(NVFP4MOE_ERR_INVALID_ARG, "router_logits is null");
+    return forward_common(mode, x, router_logits, bias, nullptr, nullptr, packed_weights, act_global_in,
+                          act_global_mid, T, H, I, E, n_group, topk_group, top_k, routed_scaling_factor, renormalize,
+                          workspace, workspace_bytes, out, out_is_fp32, topk_ids_out, topk_weights_out, stream);
 }
 
 nvfp4moe_status moe_forward_routed(nvfp4moe_mode mode, const uint16_t* x, const int32_t* topk_ids,
@@ -439,8 +454,8 @@ nvfp4moe_status moe_forward_routed(nvfp4moe_mode mode, const uint16_t* x, const 
                                    int32_t H, int32_t I, int32_t E, int32_t top_k, void* workspace,
                                    size_t workspace_bytes, void* out, int32_t out_is_fp32, void* stream) {
     if (T > 0 && (!topk_ids || !topk_weights)) return fail(NVFP4MOE_ERR_INVALID_ARG, "routing input is null");
-    return forward_common(mode, x, nullptr, nullptr, topk_ids, topk_weights, packed_weights, act_global, T, H, I, E, 1,
-                          1, top_k, 1.0f, 0, workspace, workspace_bytes, out, out_is_fp32, nullptr, nullptr, stream);
+    return forward_common(mode, x, nullptr, nullptr, topk_ids, topk_weights, packed_weights, act_global, act_global, T,
+                          H, I, E, 1, 1, top_k, 1.0f, 0, workspace, workspace_bytes, out, out_is_fp32, nullptr, nullptr, stream);
 }
 
 nvfp4moe_status nvfp4moe_set_trace_events(void* const* events, int32_t n_events) {

@@ -72,8 +72,8 @@ nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T,
 // w4a4.cu
 size_t w4a4_packed_size(int E, int H, int I);
 nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream);
-nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E, int k, float act_global,
-                                  int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
+nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E, int k, float act_global_in,
+                                  float act_global_mid, int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
                                   const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, __half* Y, float* y_scale,
                                   cudaStream_t stream, cudaEvent_t mid_event);
 

@@ -92,7 +92,8 @@ struct GemmParams {
     const uint8_t* sfa;      // A block scales, atom layout
     const uint8_t* sfb;      // B block scales, atom layout
     const float* globals;    // [E, 3]
-    float act_global;
+    float act_global;        // global scale of the A operand's NVFP4 codes
+    float out_global;        // gate/up: global scale the intermediate is requantised with
     uint8_t* out_codes;      // gate/up: intermediate codes [rows, I/2]
     uint8_t* out_sf;         // gate/up: intermediate scales, atom layout
     int out_k;               // gate/up: I
@@ -365,7 +366,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         float a[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) a[i] = silu_fast(gv[16 * c + i] * ag) * (uv[16 * c + i] * au);
-                        const uint32_t sf = requant_block16(a, p.act_global, codes[2 * c], codes[2 * c + 1]);
+                        const uint32_t sf = requant_block16(a, p.out_global, codes[2 * c], codes[2 * c + 1]);
                         sfw |= sf << (8 * c);
                     }
                     *reinterpret_cast<uint4*>(p.out_codes + row * (p.out_k / 2) + i0 / 2) =
@@ -580,8 +581,8 @@ nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed,
     return NVFP4MOE_OK;
 }
 
-nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E, int k, float act_global,
-                                  int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
+nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E, int k, float act_global_in,
+                                  float act_global_mid, int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
                                   const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, __half* Y, float* y_scale,
                                   cudaStream_t stream, cudaEvent_t mid_event) {
     (void)T;
@@ -602,11 +603,12 @@ nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E
     g.tiles = plan.tiles;
     g.n_tiles = plan.n_tiles;
     g.globals = reinterpret_cast<const float*>(pk + L.globals);
-    g.act_global = act_global;
     g.err = device_error_word();
     g.wts = plan.wts;
     g.pair_of_row = plan.pair_of_row;
-    // gate/up + SwiGLU + requantise
+    // gate/up + SwiGLU + requantise: inputs carry act_global_in, the intermediate act_global_mid
+    g.act_global = act_global_in;
+    g.out_global = act_global_mid;
     g.K = H;
     g.n_ntiles = (2 * I) / BN;
     g.b_rows_per_expert = 2 * I;
@@ -622,6 +624,7 @@ nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E
     }
     if (mid_event) cudaEventRecord(mid_event, stream);
     // down x routing weight
+    g.act_global = act_global_mid;
     g.K = I;
     g.n_ntiles = H / BN;
     g.b_rows_per_expert = H;

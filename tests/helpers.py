@@ -87,15 +87,20 @@ class GpuLayer:
                                                                       self.top_k)), dtype=torch.uint8, device="cuda")
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor, rsf: float = 2.827, act_global: float = 1.0,
-                bias=None, out_fp32: bool = False, renormalize: bool = True):
+                bias=None, out_fp32: bool = False, renormalize: bool = True, act_global_mid: float | None = None):
         T = x.shape[0]
         if T != self.T:
             self.resize(T)
         out = torch.empty((T, self.H), dtype=torch.float32 if out_fp32 else torch.bfloat16, device="cuda")
         ids = torch.empty((T, self.top_k), dtype=torch.int32, device="cuda")
         wts = torch.empty((T, self.top_k), dtype=torch.float32, device="cuda")
-        moe.moe_forward(self.mode, x, logits, bias, self.packed, act_global, T, self.H, self.I, self.E, self.n_group,
-                        self.topk_group, self.top_k, rsf, renormalize, self.ws, out, ids, wts)
+        if act_global_mid is None:
+            moe.moe_forward(self.mode, x, logits, bias, self.packed, act_global, T, self.H, self.I, self.E,
+                            self.n_group, self.topk_group, self.top_k, rsf, renormalize, self.ws, out, ids, wts)
+        else:
+            moe.moe_forward_ex(self.mode, x, logits, bias, self.packed, act_global, act_global_mid, T, self.H, self.I,
+                               self.E, self.n_group, self.topk_group, self.top_k, rsf, renormalize, self.ws, out, ids,
+                               wts)
         moe.nvfp4moe_check_device_status()
         return out, ids, wts
 
@@ -125,10 +130,11 @@ def compare_layer(got: np.ndarray, ref: np.ndarray, rel_l2: float = REL_L2, max_
     return rel, float(err.max()) / rms
 
 
-def oracle_layer(mode: int, d: dict, w: dict, wl, tokens=None, act_global: float = 1.0, renormalize: bool = True):
+def oracle_layer(mode: int, d: dict, w: dict, wl, tokens=None, act_global: float = 1.0, renormalize: bool = True,
+                 act_global_mid: float | None = None):
     return oracle.moe_layer(mode, d["x"], d["logits"], None, w["gate_codes"], w["gate_sf"], w["up_codes"], w["up_sf"],
                             w["down_codes"], w["down_sf"], w["w_global"], act_global, wl.n_group, wl.topk_group,
-                            wl.top_k, wl.rsf, renormalize, tokens)
+                            wl.top_k, wl.rsf, renormalize, tokens, act_global_mid=act_global_mid)
 
 
 def out_to_f64(out: torch.Tensor) -> np.ndarray:

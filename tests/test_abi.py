@@ -22,7 +22,7 @@ def declared_functions():
 def test_header_declares_the_hot_path_calls():
     names = declared_functions()
     for n in ("transcode_mxfp4_to_nvfp4", "moe_route", "quantize_nvfp4", "moe_forward", "moe_pack_weights",
-              "moe_permute", "moe_forward_routed"):
+              "moe_permute", "moe_forward_routed", "moe_forward_ex"):
         assert n in names
 
 
@@ -109,6 +109,23 @@ def test_forward_validation():
     # T == 0 is a no-op even with null pointers
     assert lib.moe_forward(1, None, None, None, None, 1.0, 0, 4096, 2048, 256, 8, 4, 8, 2.827, 1, None, 0, None, 0,
                            None, None, None) == 0
+
+
+@pytest.mark.parametrize("g_in,g_mid", [(0.0, 1.0), (1.0, 0.0), (1.0, -2.0), (float("nan"), 1.0),
+                                        (1.0, float("inf"))])
+def test_forward_ex_rejects_bad_activation_globals(g_in, g_mid):
+    lib = moe.load()
+    p = ctypes.c_void_p(4096)
+    for mode in (0, 1):
+        assert lib.moe_forward_ex(mode, p, p, None, p, g_in, g_mid, 4, 4096, 2048, 256, 8, 4, 8, 2.827, 1, p, 1 << 40,
+                                  p, 0, None, None, None) == 1
+    assert "act_global" in moe.load().nvfp4moe_last_error_string().decode()
+
+
+def test_forward_ex_zero_tokens_is_a_no_op():
+    lib = moe.load()
+    assert lib.moe_forward_ex(1, None, None, None, None, 0.5, 2.0, 0, 4096, 2048, 256, 8, 4, 8, 2.827, 1, None, 0,
+                              None, 0, None, None, None) == 0
 
 
 def test_error_string_is_text():

@@ -334,3 +334,55 @@ def test_layer_non_unit_activation_global():
     out, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), act_global=0.25, out_fp32=True)
     ref = oracle_layer(moe.W4A4, d, w, wl, act_global=0.25)
     compare_layer(out_to_f64(out), ref)
+
+
+@pytest.mark.parametrize("g_in,g_mid", [("calibrated", 1.0), (1.0, 0.03125), (0.37, 2.5), ("calibrated", 0.125)])
+def test_layer_separate_input_and_intermediate_globals(g_in, g_mid):
+    # moe_forward_ex: the layer input quantised with g_in, the SwiGLU output
+    # (down-projection input) requantised with g_mid.  "calibrated" is the
+    # input's amax / 2688, the global that maps it onto the largest E4M3 block
+    # scale times the largest E2M1 code.
+    wl = inputs.WORKLOADS["tiny"]
+    d = inputs.moe_inputs(wl)
+    w = nvfp4_weights_from_inputs(d, False)
+    if g_in == "calibrated":
+        amax = float(np.abs((d["x"].astype(np.uint32) << 16).view(np.float32)).max())
+        g_in = float(np.float32(amax / 2688.0))
+    layer = GpuLayer(moe.W4A4, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
+    x, lg = bf16_tensor(d["x"]), dev(d["logits"])
+    out, _, _ = layer.forward(x, lg, act_global=g_in, act_global_mid=g_mid, out_fp32=True)
+    ref = oracle_layer(moe.W4A4, d, w, wl, act_global=g_in, act_global_mid=g_mid)
+    compare_layer(out_to_f64(out), ref)
+    # the single-global entry point is the same call with both globals equal
+    a, _, _ = layer.forward(x, lg, act_global=g_in, act_global_mid=g_in)
+    b, _, _ = layer.forward(x, lg, act_global=g_in)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_layer_w4a16_ignores_activation_globals():
+    wl = inputs.WORKLOADS["tiny"]
+    d = inputs.moe_inputs(wl)
+    w = nvfp4_weights_from_inputs(d, False)
+    layer = GpuLayer(moe.W4A16, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
+    x, lg = bf16_tensor(d["x"]), dev(d["logits"])
+    a, _, _ = layer.forward(x, lg, act_global=0.3, act_global_mid=7.0)
+    b, _, _ = layer.forward(x, lg)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_layer_prefill_calibrated_globals_sampled():
+    # full prefill size, input global calibrated from the input, the
+    # down-projection input's global capped at 1 (amax capped at 2688)
+    wl = inputs.WORKLOADS["prefill"]
+    d = inputs.moe_inputs(wl)
+    w = nvfp4_weights_from_inputs(d, False)
+    amax = float(np.abs((d["x"].astype(np.uint32) << 16).view(np.float32)).max())
+    g_in = float(np.float32(amax / 2688.0))
+    layer = GpuLayer(moe.W4A4, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
+    out, ids, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), act_global=g_in, act_global_mid=0.5,
+                                out_fp32=True)
+    toks = _sample_tokens(host(ids), 8, wl.seed + 1)
+    ref = oracle_layer(moe.W4A4, d, w, wl, tokens=toks, act_global=g_in, act_global_mid=0.5)
+    compare_layer(out_to_f64(out)[toks], ref)
+    del layer
+    torch.cuda.empty_cache()
