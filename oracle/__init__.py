@@ -118,6 +118,29 @@ def decode_nvfp4(codes: np.ndarray, e4m3: np.ndarray, global_scale: float, N: in
     return out
 
 
+def compact_scales(codes: np.ndarray, e4m3: np.ndarray, rows: int, K: int):
+    """NVFP4 rows -> compact scales.  Returns (nib [rows, K/64] u8, row_exp [rows]
+    i8, status [rows] i32, number of rows that are not representable)."""
+    codes = np.ascontiguousarray(codes, np.uint8)
+    e4m3 = np.ascontiguousarray(e4m3, np.uint8)
+    nib = np.empty((rows, K // 64), np.uint8)
+    rexp = np.empty(rows, np.int8)
+    status = np.empty(rows, np.int32)
+    L = _load()
+    L.orc_compact_scales.restype = ctypes.c_int64
+    bad = L.orc_compact_scales(_p(codes), _p(e4m3), ctypes.c_int64(rows), ctypes.c_int64(K), _p(nib), _p(rexp),
+                               _p(status))
+    return nib, rexp, status, int(bad)
+
+
+def compact_decode(nib: np.ndarray, row_exp: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """Scale of every 32-code block [rows, K/32] (float64) of compact rows."""
+    out = np.empty((rows, K // 32), np.float64)
+    _load().orc_compact_decode(_p(np.ascontiguousarray(nib, np.uint8)), _p(np.ascontiguousarray(row_exp, np.int8)),
+                               ctypes.c_int64(rows), ctypes.c_int64(K), _p(out))
+    return out
+
+
 def transcode(codes: np.ndarray, e8m0: np.ndarray, num_tensors: int, N: int, K: int):
     """Returns (codes_out, e4m3 [nt, N, K/16], global [nt] f32, status [nt] i32,
     report [blocks, zero_blocks, nonrepresentable_tensors, nan_tensors], worst)."""

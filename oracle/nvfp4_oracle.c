@@ -17,7 +17,8 @@
  *  [P3] "baekpica MiMo-V2.6-Flash-RL mixed-quant GGUF": tensor precision table
  *       (routers kept in F32).
  *  [P5] "MiMo-V2.6-Flash-MOPD on one RTX PRO 6000": "Speed v6" and "What makes it
- *       fast" (the router's matmul followed by a fused top-k).
+ *       fast" (the router's matmul followed by a fused top-k; the compact
+ *       4.125-bit expert encoding).
  *
  * Arithmetic: floating point decisions that produce integers (quantised codes,
  * routing choices) are taken in IEEE FP32, exactly as written below; everything
@@ -230,6 +231,102 @@ int orc_transcode(const uint8_t* codes_in, const uint8_t* e8m0, int64_t num_tens
         tensor_status[t] = 0;
     }
     return worst;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Compact scales: 4.125 bits per weight                                      */
+/* ------------------------------------------------------------------------- */
+/* [P5] "Speed v6" lists a lossless compact expert encoding ("nvfp4c": 4.125
+ * instead of 4.5 bits per weight, the same values).  It is possible because of
+ * [P1] introduction: after the transcode, the two E4M3 scales of every 32 codes
+ * are the same power of two.  The pages give no layout; the reading here:
+ *
+ *   per row of K codes one exponent r (int8) and per 32 codes one 4-bit field
+ *   n; the block's scale is 2^(r - n) for n = 0..14 and 0 for n = 15.
+ *
+ * 4 bits per 32 codes = 0.125 bits per weight (plus 8 bits per row).  A row is
+ * representable when, in every 32-code block, the two E4M3 scales have equal
+ * value and that value is either 0 (then all 32 codes must be +-0, so the
+ * block decodes to zeros whatever its scale) or an exact positive power of two
+ * 2^e; then r is the largest e of the row's non-zero-scale blocks (0 if none)
+ * and every such block needs r - e <= 14.
+ *
+ * Outputs: nib [rows, K/64] (byte j: low nibble = block 2j, high nibble =
+ * block 2j+1), row_exp [rows], status [rows] (0 representable, 1 not).  A row
+ * that is not representable gets nibbles 0xFF and r = 0.  Returns the number
+ * of rows that are not representable.                                       */
+static int power_of_two_exponent(double v, int* e) {
+    /* v = 2^e exactly, v > 0 */
+    if (!(v > 0.0)) return 0;
+    int ex;
+    double m = frexp(v, &ex); /* v = m * 2^ex, m in [0.5, 1) */
+    if (m != 0.5) return 0;
+    *e = ex - 1;
+    return 1;
+}
+
+int64_t orc_compact_scales(const uint8_t* codes, const uint8_t* e4m3, int64_t rows, int64_t K, uint8_t* nib,
+                           int8_t* row_exp, int32_t* status) {
+    const int64_t nb = K / 32;
+    int64_t bad = 0;
+    int* e_of = (int*)malloc(sizeof(int) * (size_t)(nb > 0 ? nb : 1));
+    int* zero_of = (int*)malloc(sizeof(int) * (size_t)(nb > 0 ? nb : 1));
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint8_t* c = codes + r * (K / 2);
+        const uint8_t* s = e4m3 + r * (K / 16);
+        int ok = 1, have = 0, emax = 0;
+        for (int64_t b = 0; b < nb; ++b) {
+            double v0 = orc_e4m3_value(s[2 * b]), v1 = orc_e4m3_value(s[2 * b + 1]);
+            zero_of[b] = 0;
+            if (!(v0 == v1)) { /* unequal, or NaN */
+                ok = 0;
+                continue;
+            }
+            if (v0 == 0.0) {
+                for (int i = 0; i < 32; ++i)
+                    if (nibble(c + b * 16, i) & 7) ok = 0;
+                zero_of[b] = 1;
+                continue;
+            }
+            int e;
+            if (!power_of_two_exponent(v0, &e)) {
+                ok = 0;
+                continue;
+            }
+            e_of[b] = e;
+            if (!have || e > emax) emax = e;
+            have = 1;
+        }
+        if (ok)
+            for (int64_t b = 0; b < nb; ++b)
+                if (!zero_of[b] && emax - e_of[b] > 14) ok = 0;
+        status[r] = ok ? 0 : 1;
+        if (!ok) {
+            ++bad;
+            row_exp[r] = 0;
+            memset(nib + r * (K / 64), 0xFF, (size_t)(K / 64));
+            continue;
+        }
+        row_exp[r] = (int8_t)(have ? emax : 0);
+        for (int64_t j = 0; j < K / 64; ++j) {
+            int lo = zero_of[2 * j] ? 15 : emax - e_of[2 * j];
+            int hi = zero_of[2 * j + 1] ? 15 : emax - e_of[2 * j + 1];
+            nib[r * (K / 64) + j] = (uint8_t)(lo | (hi << 4));
+        }
+    }
+    free(e_of);
+    free(zero_of);
+    return bad;
+}
+
+/* The scale of every 32-code block of a compact row: 2^(r - n), or 0 for n = 15. */
+void orc_compact_decode(const uint8_t* nib, const int8_t* row_exp, int64_t rows, int64_t K, double* scale_out) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < K / 32; ++b) {
+            const uint8_t byte = nib[r * (K / 64) + b / 2];
+            const int n = (b & 1) ? (byte >> 4) : (byte & 15);
+            scale_out[r * (K / 32) + b] = n == 15 ? 0.0 : ldexp(1.0, (int)row_exp[r] - n);
+        }
 }
 
 /* ------------------------------------------------------------------------- */

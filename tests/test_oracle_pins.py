@@ -183,6 +183,102 @@ def test_transcode_adversarial_tensor_of_the_layer_recipe():
 
 
 # ---------------------------------------------------------------------------
+# compact scales (4.125 bits per weight)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("lo,hi", [(-8, -3), (-20, -6), (3, 17), (-9, 8)])
+def test_compact_of_a_transcode_is_the_e8m0_exponent_distance(lo, hi):
+    # after the transcode every block scale is 2^(k - g); the compact field of a
+    # block is then (row max of k) - k, computed here from the E8M0 bytes alone
+    num, N, K = 2, 16, 256
+    codes, e8 = _mx(num, N, K, lo, hi, seed=5)
+    codes[0, 3, 0:16] = 0x80  # an all-zero block (codes +-0)
+    codes[1, 7, :] = 0x08     # an all-zero row
+    c2, e4, g, st, _, worst = oracle.transcode(codes, e8, num, N, K)
+    spread_ok = hi - lo <= 14
+    assert worst == 0
+    for t in range(num):
+        nib, rexp, status, bad = oracle.compact_scales(c2[t], e4[t], N, K)
+        k = e8[t].astype(np.int64) - 127
+        zero = np.array([[not np.any(codes[t, r, 16 * b:16 * b + 16] & 0x77) for b in range(K // 32)]
+                         for r in range(N)])
+        gexp = math.frexp(float(g[t]))[1] - 1
+        for r in range(N):
+            live = ~zero[r]
+            if not live.any():
+                assert status[r] == 0 and rexp[r] == 0 and np.all(nib[r] == 0xFF)
+                continue
+            kmax = int(k[r][live].max())
+            ok = kmax - int(k[r][live].min()) <= 14
+            assert status[r] == (0 if ok else 1)
+            if not ok:
+                continue
+            assert rexp[r] == kmax - gexp
+            want = np.where(live, kmax - k[r], 15)
+            got = np.stack([nib[r] & 15, nib[r] >> 4], 1).reshape(-1)
+            assert np.array_equal(got, want)
+        if spread_ok:
+            assert bad == 0
+        else:
+            assert bad == int(np.sum(status))
+
+
+def test_compact_values_equal_the_mxfp4_values():
+    num, N, K = 1, 8, 512
+    codes, e8 = _mx(num, N, K, -9, 4, seed=6)
+    c2, e4, g, *_ = oracle.transcode(codes, e8, num, N, K)
+    nib, rexp, status, bad = oracle.compact_scales(c2[0], e4[0], N, K)
+    assert bad == 0
+    scale = oracle.compact_decode(nib, rexp, N, K)
+    e2m1 = oracle.decode_nvfp4(c2[0], np.full((N, K // 16), 0x38, np.uint8), 1.0, N, K)  # E4M3 0x38 = 1.0
+    got = e2m1 * np.repeat(scale, 32, axis=1) * float(g[0])
+    assert np.array_equal(got, oracle.decode_mxfp4(codes[0], e8[0], N, K))
+
+
+def _sf_row(pairs):
+    """One row of E4M3 scale bytes: a byte b stands for the pair (b, b)."""
+    return np.array([x for p in pairs for x in (p if isinstance(p, tuple) else (p, p))], np.uint8)[None, :]
+
+
+def test_compact_hand_example():
+    # blocks: 2^0 (E4M3 0x38), 2^-3 (0x20), zero (codes +-0), 2^2 (0x48)
+    codes = np.full((1, 64), 0x11, np.uint8)
+    codes[0, 32:48] = 0x08
+    nib, rexp, status, bad = oracle.compact_scales(codes, _sf_row([0x38, 0x20, 0x00, 0x48]), 1, 128)
+    assert bad == 0 and status[0] == 0 and rexp[0] == 2
+    assert list(nib[0]) == [0x52, 0x0F]  # n = 2, 5 | 15, 0
+    assert list(oracle.compact_decode(nib, rexp, 1, 128)[0]) == [1.0, 0.125, 0.0, 4.0]
+
+
+def test_compact_spread_and_subnormal_boundaries():
+    codes = np.full((2, 64), 0x22, np.uint8)
+    # row 0: 2^8 (0x78) and 2^-6 (0x08): spread 14, representable; row 1: 2^8 and 2^-7 (subnormal 0x04)
+    sf = np.concatenate([_sf_row([0x78, 0x08, 0x78, 0x78]), _sf_row([0x78, 0x04, 0x78, 0x78])])
+    nib, rexp, status, bad = oracle.compact_scales(codes, sf, 2, 128)
+    assert list(status) == [0, 1] and bad == 1
+    assert rexp[0] == 8 and nib[0, 0] == 0xE0
+    assert rexp[1] == 0 and np.all(nib[1] == 0xFF)
+    # subnormal powers of two are accepted: 2^-9 (0x01), 2^-8 (0x02), 2^-7 (0x04), 2^-6 (0x08)
+    nib, rexp, status, _ = oracle.compact_scales(codes[:1], _sf_row([0x01, 0x02, 0x04, 0x08]), 1, 128)
+    assert status[0] == 0 and rexp[0] == -6 and list(nib[0]) == [0x23, 0x01]
+
+
+@pytest.mark.parametrize("pair,zero_codes", [((0x38, 0x30), True), ((0x39, 0x39), True), ((0x7F, 0x7F), True),
+                                             ((0xB8, 0xB8), True), ((0x00, 0x00), False), ((0x00, 0x80), True)])
+def test_compact_rejections(pair, zero_codes):
+    # unequal halves, not a power of two, NaN, negative, zero scale over
+    # non-zero codes; and +0 / -0 halves, which have equal value (accepted)
+    codes = np.full((1, 64), 0x11, np.uint8)
+    if zero_codes:
+        codes[0, 0:16] = 0x00
+    nib, rexp, status, bad = oracle.compact_scales(codes, _sf_row([pair, 0x38, 0x38, 0x38]), 1, 128)
+    expect_ok = pair == (0x00, 0x80)
+    assert status[0] == (0 if expect_ok else 1) and bad == (0 if expect_ok else 1)
+    if expect_ok:
+        assert rexp[0] == 0 and list(nib[0]) == [0x0F, 0x00]
+
+
+# ---------------------------------------------------------------------------
 # sigmoid / exp specification
 # ---------------------------------------------------------------------------
 
