@@ -376,6 +376,7 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_extras and rank == 0:
         res["decode"] = bench_decode(torch, moe, w, args, P)
         del w
+        res["decode_compact"] = bench_decode(torch, moe, None, args, P, compact=True)
         res["transcode"] = bench_transcode(torch, moe, args, P)
         res["router"] = bench_router(torch, moe, args, P)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -387,33 +388,57 @@ def run_ours(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
-def bench_decode(torch, moe, w, args, P):
-    """W4A16 decode layer (T=16): tokens/s and weight-stream HBM GB/s."""
-    wl = inputs.WORKLOADS["decode"]
-    rng = np.random.default_rng(wl.seed)
-    x = inputs.activations(rng, wl.T, wl.H)
-    lg = inputs.router_logits(rng, wl.T, wl.E)
-    packed, ws = make_layer(torch, moe, moe.W4A16, w, wl.T, wl)
+def bench_decode(torch, moe, w, args, P, compact=False):
+    """W4A16 decode layer (T=16): tokens/s and weight-stream HBM GB/s.  compact:
+    the same layer on weights with the transcode's scale structure, stored with
+    compact scales (mode W4A16C, 4.125 bits per weight)."""
+    mode = moe.W4A16C if compact else moe.W4A16
+    if compact:
+        wl = inputs.WORKLOADS["decode_pow2"]
+        d = inputs.moe_inputs(wl)
+        w = {k: d[k] for k in ("gate_codes", "gate_sf", "up_codes", "up_sf", "down_codes", "down_sf", "w_global")}
+        x, lg = d["x"], d["logits"]
+        del d
+    else:
+        wl = inputs.WORKLOADS["decode"]
+        rng = np.random.default_rng(wl.seed)
+        x = inputs.activations(rng, wl.T, wl.H)
+        lg = inputs.router_logits(rng, wl.T, wl.E)
     xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
     ld = torch.from_numpy(lg).cuda()
     out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    same_weights = None
+    if compact:
+        # the plain W4A16 form of the same weights, for comparison (same outputs bit for bit)
+        packed, ws = make_layer(torch, moe, moe.W4A16, w, wl.T, wl)
+        ms16, _ = time_layer(torch, moe, moe.W4A16, packed, ws, xd, ld, out, wl, wl.T, max(args.steps, 20),
+                             args.warmup, trace=False)
+        same_weights = {"mode": "W4A16", "ms_per_step": round(ms16, 4)}
+        del packed, ws
+        torch.cuda.empty_cache()
+    packed, ws = make_layer(torch, moe, mode, w, wl.T, wl)
+    del w
     # flush L2 between steps: the active experts' weights (~1.4 GB) exceed L2, but
     # the same experts repeat every step, so rotate through a 256 MB buffer too
-    ms, stage = time_layer(torch, moe, moe.W4A16, packed, ws, xd, ld, out, wl, wl.T, max(args.steps, 20),
-                           args.warmup)
+    ms, stage = time_layer(torch, moe, mode, packed, ws, xd, ld, out, wl, wl.T, max(args.steps, 20), args.warmup)
     ids = torch.empty((wl.T, wl.top_k), dtype=torch.int32, device="cuda")
     wts = torch.empty((wl.T, wl.top_k), dtype=torch.float32, device="cuda")
     moe.moe_route(ld, None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf, True, ids, wts)
     active = int(torch.unique(ids).numel())
-    per_expert = (2 * wl.I * wl.H + wl.H * wl.I) * (0.5 + 1.0 / 16)  # codes + E4M3 scales
+    if compact:  # codes + a 4-bit field per 32 weights + an exponent byte per row
+        per_expert = (2 * wl.I * wl.H + wl.H * wl.I) * (0.5 + 1.0 / 64) + (2 * wl.I + wl.H)
+    else:  # codes + E4M3 scales
+        per_expert = (2 * wl.I * wl.H + wl.H * wl.I) * (0.5 + 1.0 / 16)
     gemm_ms = stage["gateup_gemm"] + stage["down_gemm"]
     wbytes = active * per_expert
     achieved = wbytes / (gemm_ms / 1e3) / 1e9
     del packed, ws
     torch.cuda.empty_cache()
-    return {"workload": f"decode: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top_k={wl.top_k} W4A16",
+    name = "W4A16 compact scales (4.125 bits per weight)" if compact else "W4A16"
+    return {"workload": f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top_k={wl.top_k} {name}",
             "value": round(wl.T / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
             "active_experts": active, "stages_ms": {k: round(v, 4) for k, v in stage.items()},
+            **({"same_weights": same_weights} if same_weights else {}),
             "roofline": {"bound": "hbm", "kernel": "k_w16_gateup + k_w16_down", "achieved": round(achieved, 1),
                          "peak": P["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / P["hbm_gbs"], 4),
                          "traffic": None, "algorithmic_bytes_per_step": int(wbytes)}}

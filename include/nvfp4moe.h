@@ -104,6 +104,30 @@ nvfp4moe_status transcode_mxfp4_to_nvfp4(const uint8_t* codes_in, const uint8_t*
                                          void* stream);
 
 /* ------------------------------------------------------------------------- */
+/* Compact scales (4.125 bits per weight)                                     */
+/* ------------------------------------------------------------------------- */
+/* Operation ("MiMo-V2.6-Flash-MOPD on one RTX PRO 6000", "Speed v6": a lossless
+ * compact expert encoding of 4.125 instead of 4.5 bits per weight; "AxionML ...
+ * NVFP4", introduction: a transcode's two E4M3 scales per 32 codes are the
+ * same power of two).  Per row of K codes: one exponent r and one 4-bit field
+ * n per 32 codes; the block's scale is 2^(r - n) for n = 0..14, 0 for n = 15.
+ * A row has a compact form when every 32-code block's two E4M3 scales have
+ * equal value and that value is an exact positive power of two 2^e, or 0 with
+ * all 32 codes +-0; r = the largest such e of the row (0 if none), and each
+ * block needs r - e <= 14.
+ *   codes      uint8 [rows, K/2] E2M1 (read only for zero-scale blocks)
+ *   e4m3_sf    uint8 [rows, K/16]
+ *   nib_out    uint8 [rows, K/64]: byte j = field of block 2j (low nibble) |
+ *              field of block 2j+1 << 4; 0xFF for a row without compact form
+ *   row_exp_out int8 [rows]: r (0 for a row without compact form)
+ *   row_status_out int32 [rows]: 0 compact form exists, 1 not
+ *   n_bad_out  int32 [1] or NULL: the number of rows without compact form
+ * Constraints: K % 64 == 0, rows >= 0 (0 is a no-op).  Asynchronous.        */
+nvfp4moe_status nvfp4_compact_scales(const uint8_t* codes, const uint8_t* e4m3_sf, int64_t rows, int64_t K,
+                                     uint8_t* nib_out, int8_t* row_exp_out, int32_t* row_status_out,
+                                     int32_t* n_bad_out, void* stream);
+
+/* ------------------------------------------------------------------------- */
 /* Grouped sigmoid top-k routing                                              */
 /* ------------------------------------------------------------------------- */
 /* Operation ("MiMo-V2.6-Flash -- REAP-50", "Model Summary" and "Pruning Method"
@@ -222,6 +246,11 @@ nvfp4moe_status quantize_nvfp4(const uint16_t* x_bf16, int64_t M, int64_t K, flo
  *   NVFP4MOE_W4A16: BF16 activations x NVFP4 weights (weights dequantised in
  *                   registers to BF16 tensor-core MMA); SwiGLU output rounded
  *                   to BF16.  Meant for decode-sized batches.
+ *   NVFP4MOE_W4A16C: NVFP4MOE_W4A16 arithmetic on weights stored with compact
+ *                   scales (see nvfp4_compact_scales): 4.125 instead of 4.5
+ *                   bits per weight, the same values, the same outputs bit for
+ *                   bit.  Needs weights whose scale pairs are equal powers of
+ *                   two (the MXFP4 transcode gives exactly that).
  *   NVFP4MOE_W4A4:  activations quantised to NVFP4 with global act_global (1.0
  *                   in the pages' recipe); FP4 x FP4 block-scaled tcgen05 MMA;
  *                   SwiGLU output requantised per 16 with the same global
@@ -233,7 +262,7 @@ nvfp4moe_status quantize_nvfp4(const uint16_t* x_bf16, int64_t M, int64_t K, flo
  * projection), which moe_pack_weights rearranges once into the layout the GEMM
  * kernels read:
  */
-typedef enum nvfp4moe_mode { NVFP4MOE_W4A16 = 0, NVFP4MOE_W4A4 = 1 } nvfp4moe_mode;
+typedef enum nvfp4moe_mode { NVFP4MOE_W4A16 = 0, NVFP4MOE_W4A4 = 1, NVFP4MOE_W4A16C = 2 } nvfp4moe_mode;
 
 typedef struct nvfp4moe_expert_weights {
     const uint8_t* gate_codes; /* [E, I, H/2]  */
@@ -253,7 +282,10 @@ size_t moe_packed_weights_size(nvfp4moe_mode mode, int32_t E, int32_t H, int32_t
  * moe_packed_weights_size bytes, owned by the caller).  Values are unchanged:
  * the packed buffer holds the same codes, scales and globals, reordered (gate and
  * up rows interleaved, MMA scale-factor layout for W4A4, fragment order for
- * W4A16).  Constraints: H % 128 == 0, I % 128 == 0, E >= 1.                 */
+ * W4A16).  Constraints: H % 128 == 0, I % 128 == 0, E >= 1.
+ * NVFP4MOE_W4A16C re-encodes the scales (nvfp4_compact_scales) and is
+ * SYNCHRONOUS: it waits for `stream` and returns NVFP4MOE_ERR_NOT_REPRESENTABLE
+ * when any weight row has no compact form (the packed buffer is then unusable). */
 nvfp4moe_status moe_pack_weights(nvfp4moe_mode mode, const nvfp4moe_expert_weights* weights_host_struct,
                                  void* packed, void* stream);
 

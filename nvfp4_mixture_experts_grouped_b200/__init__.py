@@ -18,11 +18,13 @@ __all__ = [
     "moe_router_topk_workspace_size", "quantize_nvfp4",
     "moe_packed_weights_size", "moe_pack_weights", "moe_forward_workspace_size", "moe_forward",
     "moe_forward_ex", "moe_forward_routed", "nvfp4moe_check_device_status", "nvfp4moe_version", "moe_permute",
-    "moe_permute_workspace_size", "nvfp4moe_set_trace_events", "moe_permute_noalloc",
+    "moe_permute_workspace_size", "nvfp4moe_set_trace_events", "moe_permute_noalloc", "W4A16C",
+    "nvfp4_compact_scales",
 ]
 
 W4A16 = 0
 W4A4 = 1
+W4A16C = 2  # W4A16 on weights with compact (4.125-bit) scales
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libnvfp4moe.so")
@@ -73,6 +75,8 @@ def load():
     L.transcode_mxfp4_to_nvfp4.restype = ctypes.c_int
     L.transcode_mxfp4_to_nvfp4.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp, vp, sz, ctypes.POINTER(TranscodeReport),
                                            vp]
+    L.nvfp4_compact_scales.restype = ctypes.c_int
+    L.nvfp4_compact_scales.argtypes = [vp, vp, i64, i64, vp, vp, vp, vp, vp]
     L.moe_route.restype = ctypes.c_int
     L.moe_route.argtypes = [vp, vp, i32, i32, i32, i32, i32, f32, i32, vp, vp, vp]
     L.moe_router_topk_workspace_size.restype = sz
@@ -195,6 +199,12 @@ def moe_permute_noalloc(topk_ids, E, pad, counts_out, pad_offsets_out, row_of_pa
     T, k = topk_ids.shape
     _check(load().moe_permute_noalloc(_ptr(topk_ids), T, E, k, pad, _ptr(counts_out), _ptr(pad_offsets_out),
                                       _ptr(row_of_pair_out), _stream(stream)))
+
+
+def nvfp4_compact_scales(codes, e4m3_sf, rows, K, nib_out, row_exp_out, row_status_out, n_bad_out=None,
+                         stream=None):
+    _check(load().nvfp4_compact_scales(_ptr(codes), _ptr(e4m3_sf), rows, K, _ptr(nib_out), _ptr(row_exp_out),
+                                       _ptr(row_status_out), _ptr(n_bad_out), _stream(stream)))
 
 
 def moe_packed_weights_size(mode, E, H, I) -> int:

@@ -222,6 +222,23 @@ nvfp4moe_status transcode_mxfp4_to_nvfp4(const uint8_t* codes_in, const uint8_t*
     return NVFP4MOE_OK;
 }
 
+nvfp4moe_status nvfp4_compact_scales(const uint8_t* codes, const uint8_t* e4m3_sf, int64_t rows, int64_t K,
+                                     uint8_t* nib_out, int8_t* row_exp_out, int32_t* row_status_out,
+                                     int32_t* n_bad_out, void* stream) {
+    REQUIRE(rows >= 0 && K >= 64, NVFP4MOE_ERR_INVALID_ARG, "bad sizes rows=%lld K=%lld", (long long)rows,
+            (long long)K);
+    REQUIRE(K % 64 == 0, NVFP4MOE_ERR_UNSUPPORTED_SHAPE, "K=%lld is not a multiple of 64", (long long)K);
+    if (rows == 0) return NVFP4MOE_OK;
+    REQUIRE(codes && e4m3_sf && nib_out && row_exp_out && row_status_out, NVFP4MOE_ERR_INVALID_ARG,
+            "null tensor pointer");
+    const void* al16[] = {codes, e4m3_sf, nib_out, row_exp_out, row_status_out, n_bad_out};
+    for (const void* q : al16) REQUIRE(!q || aligned16(q), NVFP4MOE_ERR_ALIGNMENT, "a pointer is not 16-byte aligned");
+    RETURN_IF(check_device());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n_bad_out) NVFP4MOE_CUDA(cudaMemsetAsync(n_bad_out, 0, sizeof(int32_t), st));
+    return launch_compact_rows(codes, e4m3_sf, rows, K, row_exp_out, nib_out, row_status_out, n_bad_out, st);
+}
+
 nvfp4moe_status moe_route(const float* logits, const float* bias, int32_t T, int32_t E, int32_t n_group,
                           int32_t topk_group, int32_t top_k, float routed_scaling_factor, int32_t renormalize,
                           int32_t* topk_ids, float* topk_weights, void* stream) {
@@ -334,13 +351,17 @@ nvfp4moe_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t E, int32
     return launch_permute(topk_ids, T, top_k, E, pad, plan, st);
 }
 
+static bool valid_mode(nvfp4moe_mode mode) {
+    return mode == NVFP4MOE_W4A16 || mode == NVFP4MOE_W4A4 || mode == NVFP4MOE_W4A16C;
+}
+
 size_t moe_packed_weights_size(nvfp4moe_mode mode, int32_t E, int32_t H, int32_t I) {
-    if (E < 1 || H < 1 || I < 1) return 0;
-    return mode == NVFP4MOE_W4A4 ? w4a4_packed_size(E, H, I) : w4a16_packed_size(E, H, I);
+    if (E < 1 || H < 1 || I < 1 || !valid_mode(mode)) return 0;
+    return mode == NVFP4MOE_W4A4 ? w4a4_packed_size(E, H, I) : w4a16_packed_size(E, H, I, mode == NVFP4MOE_W4A16C);
 }
 
 nvfp4moe_status moe_pack_weights(nvfp4moe_mode mode, const nvfp4moe_expert_weights* w, void* packed, void* stream) {
-    REQUIRE(mode == NVFP4MOE_W4A16 || mode == NVFP4MOE_W4A4, NVFP4MOE_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
+    REQUIRE(valid_mode(mode), NVFP4MOE_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
     REQUIRE(w && packed, NVFP4MOE_ERR_INVALID_ARG, "null pointer");
     RETURN_IF(validate_layer_shape(w->H, w->I, w->E));
     const void* ptrs[7] = {w->gate_codes, w->gate_sf, w->up_codes, w->up_sf, w->down_codes, w->down_sf, w->w_global};
@@ -351,7 +372,8 @@ nvfp4moe_status moe_pack_weights(nvfp4moe_mode mode, const nvfp4moe_expert_weigh
     REQUIRE(aligned16(packed), NVFP4MOE_ERR_ALIGNMENT, "packed buffer is not 16-byte aligned");
     RETURN_IF(check_device());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return mode == NVFP4MOE_W4A4 ? launch_w4a4_pack(*w, packed, st) : launch_w4a16_pack(*w, packed, st);
+    return mode == NVFP4MOE_W4A4 ? launch_w4a4_pack(*w, packed, st)
+                                 : launch_w4a16_pack(*w, packed, mode == NVFP4MOE_W4A16C, st);
 }
 
 size_t moe_forward_workspace_size(nvfp4moe_mode mode, int32_t T, int32_t H, int32_t I, int32_t E, int32_t top_k) {
@@ -366,7 +388,7 @@ static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, con
                                       int32_t topk_group, int32_t top_k, float rsf, int32_t renorm, void* workspace,
                                       size_t workspace_bytes, void* out, int32_t out_is_fp32, int32_t* ids_out,
                                       float* wts_out, void* stream) {
-    REQUIRE(mode == NVFP4MOE_W4A16 || mode == NVFP4MOE_W4A4, NVFP4MOE_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
+    REQUIRE(valid_mode(mode), NVFP4MOE_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
     REQUIRE(T >= 0, NVFP4MOE_ERR_INVALID_ARG, "T=%d is negative", T);
     RETURN_IF(validate_layer_shape(H, I, E));
     if (logits) {
@@ -415,7 +437,7 @@ static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, con
                                     g_trace_on ? g_trace[4] : nullptr));
     } else {
         trace(3, st);
-        RETURN_IF(launch_w4a16_layer(x, packed, T, H, I, E, top_k, plan, reinterpret_cast<uint16_t*>(ws + L.a2bf),
+        RETURN_IF(launch_w4a16_layer(x, packed, mode == NVFP4MOE_W4A16C, T, H, I, E, top_k, plan, reinterpret_cast<uint16_t*>(ws + L.a2bf),
                                      static_cast<float*>(Y), ws + L.w16s, st, g_trace_on ? g_trace[4] : nullptr));
     }
     trace(5, st);

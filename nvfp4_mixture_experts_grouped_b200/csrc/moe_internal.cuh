@@ -61,12 +61,19 @@ nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H,
 nvfp4moe_status launch_combine(const void* Y, const float* y_scale, const int32_t* row_of_pair, int64_t T, int H,
                                int k, void* out, bool out_f32, cudaStream_t stream);
 
+// compact.cu: compact scales of NVFP4 rows (row_exp [rows]; nib [rows, K/64],
+// row_status [rows] and the failure counter n_bad are optional).  K % 64 == 0.
+nvfp4moe_status launch_compact_rows(const uint8_t* codes, const uint8_t* sf, int64_t rows, int64_t K,
+                                    int8_t* row_exp, uint8_t* nib, int32_t* row_status, int32_t* n_bad,
+                                    cudaStream_t stream);
+
 // w4a16.cu
-size_t w4a16_packed_size(int E, int H, int I);
-nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream);
+// compact = the 4.125-bit scale form (mode NVFP4MOE_W4A16C)
+size_t w4a16_packed_size(int E, int H, int I, bool compact);
+nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed, bool compact, cudaStream_t stream);
 size_t w4a16_scratch_size(int T, int H, int I, int k);  // FP16 copies of the activations + row scales
-nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T, int H, int I, int E, int k,
-                                   const RoutingPlan& plan, uint16_t* A2, float* Y, void* scratch,
+nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, bool compact, int T, int H, int I,
+                                   int E, int k, const RoutingPlan& plan, uint16_t* A2, float* Y, void* scratch,
                                    cudaStream_t stream, cudaEvent_t mid_event);
 
 // w4a4.cu

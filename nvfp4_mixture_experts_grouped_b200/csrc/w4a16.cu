@@ -38,22 +38,41 @@ constexpr int W16_WARPS = 4;
 constexpr int W16_MAX_NT = 2;  // n-tiles (of 8 tokens) per pass over the weights
 constexpr int W16_MIN_CTAS = 5;  // CTAs per SM the register budget is sized for
 
+// Scale bytes per 16-row tile and 64-column chunk: 64 E4M3 bytes, or 16 bytes
+// of 4-bit compact fields (one byte per row).
+__host__ __device__ constexpr int w16_chunk_scale_bytes(bool compact) { return compact ? 16 : 64; }
+
 struct W16Layout {
-    int64_t gu_codes, gu_scales, d_codes, d_scales, globals, total;
+    int64_t gu_codes, gu_scales, d_codes, d_scales, globals;
+    int64_t rexp_g, rexp_u, rexp_d, status;  // compact form only: row exponents [E, I], [E, I], [E, H]; failures
+    int64_t total;
 };
 
 __host__ __device__ inline int64_t align256(int64_t v) { return (v + 255) / 256 * 256; }
 
-__host__ __device__ inline W16Layout w16_layout(int E, int H, int I) {
+__host__ __device__ inline W16Layout w16_layout(int E, int H, int I, bool compact) {
+    const int64_t per64 = w16_chunk_scale_bytes(compact) / 16;  // scale bytes per row per 64 columns
     W16Layout L;
     L.gu_codes = 0;
     L.gu_scales = align256(L.gu_codes + (int64_t)E * I * H);
-    L.d_codes = align256(L.gu_scales + (int64_t)E * I * H / 8);
+    L.d_codes = align256(L.gu_scales + (int64_t)E * 2 * I * (H / 64) * per64);
     L.d_scales = align256(L.d_codes + (int64_t)E * H * I / 2);
-    L.globals = align256(L.d_scales + (int64_t)E * H * I / 16);
-    L.total = align256(L.globals + (int64_t)E * 3 * 4);
+    L.globals = align256(L.d_scales + (int64_t)E * H * (I / 64) * per64);
+    int64_t end = L.globals + (int64_t)E * 3 * 4;
+    L.rexp_g = L.rexp_u = L.rexp_d = L.status = -1;
+    if (compact) {
+        L.rexp_g = align256(end);
+        L.rexp_u = align256(L.rexp_g + (int64_t)E * I);
+        L.rexp_d = align256(L.rexp_u + (int64_t)E * I);
+        L.status = align256(L.rexp_d + (int64_t)E * H);
+        end = L.status + 16;
+    }
+    L.total = align256(end);
     return L;
 }
+
+// 2^k as FP32 for k in [-126, 127]
+__device__ __forceinline__ float pow2f(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
 
 // ---------------------------------------------------------------------------
 // pack: per 16-row tile and 64-column chunk, 512 bytes in fragment order (lane
@@ -61,7 +80,9 @@ __host__ __device__ inline W16Layout w16_layout(int E, int H, int I) {
 // the two consecutive-column codes of A-fragment register j (low nibble = even
 // column): j=0 row g cols 2c,2c+1; j=1 row g+8; j=2 row g cols 2c+8,2c+9; j=3
 // row g+8.  Scales: 64 bytes per chunk, 8 per row pair g: [s(g,k16 step t),
-// s(g+8,t)] for t = 0..3.
+// s(g+8,t)] for t = 0..3.  Compact form: 16 bytes per chunk, byte 2g for row g
+// and 2g+1 for row g+8, each holding the 4-bit fields of the chunk's two
+// 32-column blocks (low nibble first); the row exponents stay in row order.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t code_at(const uint8_t* codes, int64_t r, int64_t k, int64_t K) {
     const uint32_t b = codes[r * (K / 2) + k / 2];
@@ -78,11 +99,15 @@ __device__ uint32_t pack_word(const uint8_t* codes, int64_t r0, int64_t kb, int 
     return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
 }
 
-// One thread per (tile, k64 chunk, lane): 16 code bytes, plus 8 scale bytes for lanes with c == 0.
+// One thread per (tile, k64 chunk, lane): 16 code bytes, plus the scale bytes
+// of rows g, g + 8 for lanes with c == 0.  rexp/rexp2: row exponents of the
+// compact form (COMPACT only).
+template <bool COMPACT>
 __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf, int64_t n_tiles,
                            int64_t K, int interleave_gu, const uint8_t* __restrict__ codes2,
                            const uint8_t* __restrict__ sf2, uint8_t* __restrict__ out_codes,
-                           uint8_t* __restrict__ out_scales, int64_t rows_per_expert) {
+                           uint8_t* __restrict__ out_scales, int64_t rows_per_expert, const int8_t* __restrict__ rexp,
+                           const int8_t* __restrict__ rexp2) {
     const int64_t chunks = K / 64;
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= n_tiles * chunks * 32) return;
@@ -91,6 +116,7 @@ __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __r
     const int64_t tile = (idx >> 5) / chunks;  // packed tile index
     const uint8_t* c = codes;
     const uint8_t* s = sf;
+    const int8_t* rx = rexp;
     int64_t r0;
     if (interleave_gu) {
         // packed tile order per expert: (iblock, {gate, up}); rows_per_expert = I
@@ -100,6 +126,7 @@ __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __r
         if (rem & 1) {
             c = codes2;
             s = sf2;
+            rx = rexp2;
         }
         r0 = e * rows_per_expert + (rem / 2) * 16;
     } else {
@@ -110,7 +137,24 @@ __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __r
 #pragma unroll
     for (int st = 0; st < 4; ++st) w[st] = pack_word(c, r0, chunk * 64 + st * 16, g, cc, K);
     *reinterpret_cast<uint4*>(out_codes + (tile * chunks + chunk) * 512 + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-    if (cc == 0) {
+    if (COMPACT && cc == 0) {
+        uint32_t v = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int64_t row = r0 + g + 8 * h;
+            const int re = rx[row];
+            uint32_t byte = 0;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int64_t b = chunk * 2 + half;  // 32-column block
+                int e = 0;
+                const int kind = compact_block_kind(s[row * (K / 16) + 2 * b], s[row * (K / 16) + 2 * b + 1], e);
+                byte |= (uint32_t)((kind == 0 ? re - e : 15) & 15) << (4 * half);
+            }
+            v |= byte << (8 * h);
+        }
+        *reinterpret_cast<uint16_t*>(out_scales + (tile * chunks + chunk) * 16 + g * 2) = (uint16_t)v;
+    } else if (!COMPACT && cc == 0) {
         uint32_t b[8];
 #pragma unroll
         for (int st = 0; st < 4; ++st) {
@@ -229,8 +273,8 @@ __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 constexpr int W16_STAGES = 4;
 constexpr int W16_CH = 2;
 constexpr int W16_STAGE_CODES = 2 * W16_CH * 512;
-constexpr int W16_STAGE_SCALES = 2 * W16_CH * 64;
-constexpr int W16_STAGE = W16_STAGE_CODES + W16_STAGE_SCALES;
+__host__ __device__ constexpr int w16_stage_scales(bool compact) { return 2 * W16_CH * w16_chunk_scale_bytes(compact); }
+constexpr int W16_STAGE = W16_STAGE_CODES + w16_stage_scales(false);  // stage stride (the larger form)
 constexpr int W16_WARP_SMEM = W16_STAGES * W16_STAGE;
 constexpr int W16_SMEM = W16_WARPS * (W16_WARP_SMEM + W16_STAGES * 8);
 
@@ -240,14 +284,16 @@ struct Ring {
     uint32_t ctr;   // groups consumed so far (stage = ctr % S, parity = ctr / S)
 };
 
+template <bool COMPACT>
 __device__ __forceinline__ void ring_issue(Ring& r, int stage, const uint8_t* const codes[2],
                                            const uint8_t* const scales[2], int grp) {
+    constexpr int SCB = w16_chunk_scale_bytes(COMPACT);
     uint8_t* st = r.buf + stage * W16_STAGE;
-    tc::mbar_arrive_expect_tx(&r.bar[stage], W16_STAGE);
+    tc::mbar_arrive_expect_tx(&r.bar[stage], W16_STAGE_CODES + w16_stage_scales(COMPACT));
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
         tc::bulk_load(st + u * W16_CH * 512, codes[u] + (int64_t)grp * W16_CH * 512, W16_CH * 512, &r.bar[stage]);
-        tc::bulk_load(st + W16_STAGE_CODES + u * W16_CH * 64, scales[u] + (int64_t)grp * W16_CH * 64, W16_CH * 64,
+        tc::bulk_load(st + W16_STAGE_CODES + u * W16_CH * SCB, scales[u] + (int64_t)grp * W16_CH * SCB, W16_CH * SCB,
                       &r.bar[stage]);
     }
 }
@@ -255,8 +301,11 @@ __device__ __forceinline__ void ring_issue(Ring& r, int stage, const uint8_t* co
 // Streams `chunks` 64-column chunks of two 16-row tiles and accumulates their
 // products with NT 8-token B tiles (FP16 rows in fragment order; every lane's
 // pointer is valid, lanes past the expert's tokens read a real row and their
-// results are dropped).  Returns false on a timeout.
-template <int NT>
+// results are dropped).  Returns false on a timeout.  COMPACT: the scales are
+// 4-bit fields n and each block's FP16 multiplier is 2^(13 - n) (the row
+// factor 2^(r - 13) is applied to the accumulators by the caller): bits
+// (28 - n) << 10, for rows g and g + 8 at once in the two halves of a word.
+template <int NT, bool COMPACT>
 __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2], const uint8_t* const scales[2],
                                            int chunks, const __half* const bptr[W16_MAX_NT],
                                            float acc[2][W16_MAX_NT][4], int32_t* err) {
@@ -265,7 +314,8 @@ __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2
     const int groups = chunks / W16_CH;
     const uint32_t base = r.ctr;
     if (lane == 0)
-        for (int i = 0; i < W16_STAGES && i < groups; ++i) ring_issue(r, (base + i) % W16_STAGES, codes, scales, i);
+        for (int i = 0; i < W16_STAGES && i < groups; ++i)
+            ring_issue<COMPACT>(r, (base + i) % W16_STAGES, codes, scales, i);
     __syncwarp();
     for (int grp = 0; grp < groups; ++grp) {
         const uint32_t n = base + grp;
@@ -275,11 +325,19 @@ __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2
 #pragma unroll
         for (int cc = 0; cc < W16_CH; ++cc) {
             uint4 q[2];
-            uint2 sc[2];
+            uint2 sc[2];  // E4M3 pairs of steps 0, 1 (x) and 2, 3 (y), or the compact multipliers
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 q[u] = *reinterpret_cast<const uint4*>(st + u * W16_CH * 512 + cc * 512 + lane * 16);
-                sc[u] = *reinterpret_cast<const uint2*>(st + W16_STAGE_CODES + u * W16_CH * 64 + cc * 64 + g * 8);
+                if (COMPACT) {
+                    const uint32_t w =
+                        *reinterpret_cast<const uint16_t*>(st + W16_STAGE_CODES + u * W16_CH * 16 + cc * 16 + g * 2);
+                    const uint32_t t = __byte_perm(w, 0u, 0x4140);  // [row g, 0, row g + 8, 0]
+                    sc[u].x = (0x001C001Cu - (t & 0x000F000Fu)) << 10;         // blocks of steps 0, 1
+                    sc[u].y = (0x001C001Cu - ((t >> 4) & 0x000F000Fu)) << 10;  // steps 2, 3
+                } else {
+                    sc[u] = *reinterpret_cast<const uint2*>(st + W16_STAGE_CODES + u * W16_CH * 64 + cc * 64 + g * 8);
+                }
             }
             // this lane's B fragments of the chunk: (b0, b1) of step t at 8 t bytes
             const uint2* bp[NT];
@@ -296,7 +354,7 @@ __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2
                     const uint32_t qw = stp == 0 ? q[u].x : stp == 1 ? q[u].y : stp == 2 ? q[u].z : q[u].w;
                     const uint32_t sw = stp < 2 ? sc[u].x : sc[u].y;
                     uint32_t a[4];
-                    dequant_step(qw, scales_f16x2((stp & 1) ? (sw >> 16) : (sw & 0xFFFFu)), a);
+                    dequant_step(qw, COMPACT ? sw : scales_f16x2((stp & 1) ? (sw >> 16) : (sw & 0xFFFFu)), a);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) mma_f16(acc[u][nt], a, bw[nt].x, bw[nt].y);
                 }
@@ -305,7 +363,7 @@ __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2
         __syncwarp();  // every lane has read the stage
         if (lane == 0 && grp + W16_STAGES < groups) {
             tc::fence_proxy_async_smem();
-            ring_issue(r, stage, codes, scales, grp + W16_STAGES);
+            ring_issue<COMPACT>(r, stage, codes, scales, grp + W16_STAGES);
         }
     }
     r.ctr = base + groups;
@@ -329,6 +387,7 @@ __device__ __forceinline__ Ring make_ring(uint8_t* smem) {
 // ---------------------------------------------------------------------------
 // gate/up GEMM + SwiGLU: warps loop over (active expert, 16 intermediates)
 // ---------------------------------------------------------------------------
+template <bool COMPACT>
 __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
     k_w16_gateup(const __half* __restrict__ x16, const float* __restrict__ x_inv, const uint8_t* __restrict__ packed,
                  W16Layout L, int H, int I, int k, RoutingPlan plan, uint16_t* __restrict__ A2, int32_t* err) {
@@ -347,13 +406,24 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
         const int n_e = plan.counts[e];
         const int row0 = plan.offsets[e];
         const float ag = glob[e * 3 + 0], au = glob[e * 3 + 1];
+        float ph[2][2] = {{1.0f, 1.0f}, {1.0f, 1.0f}};  // [gate, up][rows g, g + 8]: compact row factors
+        if (COMPACT) {
+            const int64_t r = (int64_t)e * I + ib * 16 + g;
+            const int8_t* rg = reinterpret_cast<const int8_t*>(packed + L.rexp_g);
+            const int8_t* ru = reinterpret_cast<const int8_t*>(packed + L.rexp_u);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                ph[0][h] = pow2f(rg[r + 8 * h] - 13);
+                ph[1][h] = pow2f(ru[r + 8 * h] - 13);
+            }
+        }
         const int64_t tile0 = ((int64_t)e * iblocks + ib) * 2;
         const uint8_t* cb[2];
         const uint8_t* sb[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             cb[u] = packed + L.gu_codes + (tile0 + u) * chunks * 512;
-            sb[u] = packed + L.gu_scales + (tile0 + u) * chunks * 64;
+            sb[u] = packed + L.gu_scales + (tile0 + u) * chunks * w16_chunk_scale_bytes(COMPACT);
         }
         for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
             const int nt_count = min(W16_MAX_NT, (n_e - n0 + 7) / 8);
@@ -364,8 +434,8 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
                 bptr[nt] = x16 + (int64_t)(plan.pair_of_row[row0 + (n < n_e ? n : n0)] / k) * H;
             }
             float acc[2][W16_MAX_NT][4] = {};
-            const bool ok = nt_count == 1 ? w16_stream<1>(ring, cb, sb, chunks, bptr, acc, err)
-                                          : w16_stream<2>(ring, cb, sb, chunks, bptr, acc, err);
+            const bool ok = nt_count == 1 ? w16_stream<1, COMPACT>(ring, cb, sb, chunks, bptr, acc, err)
+                                          : w16_stream<2, COMPACT>(ring, cb, sb, chunks, bptr, acc, err);
             if (!ok) return;
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
@@ -377,8 +447,8 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
                         const float inv = x_inv[plan.pair_of_row[row0 + n] / k];
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {  // rows g, g + 8
-                            const float gv = acc[0][nt][2 * h + j] * inv * ag;
-                            const float uv = acc[1][nt][2 * h + j] * inv * au;
+                            const float gv = acc[0][nt][2 * h + j] * inv * (ag * ph[0][h]);
+                            const float uv = acc[1][nt][2 * h + j] * inv * (au * ph[1][h]);
                             const __nv_bfloat16 v = __float2bfloat16_rn(silu(gv) * uv);
                             A2[(int64_t)(row0 + n) * I + ib * 16 + g + 8 * h] = *reinterpret_cast<const uint16_t*>(&v);
                         }
@@ -392,6 +462,7 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
 // ---------------------------------------------------------------------------
 // down GEMM x routing weight: warps loop over (active expert, 32 hidden rows)
 // ---------------------------------------------------------------------------
+template <bool COMPACT>
 __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
     k_w16_down(const uint8_t* __restrict__ packed, W16Layout L, int H, int I, RoutingPlan plan,
                const __half* __restrict__ A16, const float* __restrict__ a_inv, float* __restrict__ Y, int32_t* err) {
@@ -410,13 +481,21 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
         const int n_e = plan.counts[e];
         const int row0 = plan.offsets[e];
         const float ad = glob[e * 3 + 2];
+        float ph[2][2] = {{1.0f, 1.0f}, {1.0f, 1.0f}};  // [tile u][rows g, g + 8]: compact row factors
+        if (COMPACT) {
+            const int8_t* rd = reinterpret_cast<const int8_t*>(packed + L.rexp_d) + (int64_t)e * H + hb * 32 + g;
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) ph[u][h] = pow2f(rd[u * 16 + 8 * h] - 13);
+        }
         const int64_t tile0 = (int64_t)e * (H / 16) + hb * 2;
         const uint8_t* cb[2];
         const uint8_t* sb[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             cb[u] = packed + L.d_codes + (tile0 + u) * chunks * 512;
-            sb[u] = packed + L.d_scales + (tile0 + u) * chunks * 64;
+            sb[u] = packed + L.d_scales + (tile0 + u) * chunks * w16_chunk_scale_bytes(COMPACT);
         }
         for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
             const int nt_count = min(W16_MAX_NT, (n_e - n0 + 7) / 8);
@@ -427,8 +506,8 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
                 bptr[nt] = A16 + (int64_t)(row0 + (n < n_e ? n : n0)) * I;
             }
             float acc[2][W16_MAX_NT][4] = {};
-            const bool ok = nt_count == 1 ? w16_stream<1>(ring, cb, sb, chunks, bptr, acc, err)
-                                          : w16_stream<2>(ring, cb, sb, chunks, bptr, acc, err);
+            const bool ok = nt_count == 1 ? w16_stream<1, COMPACT>(ring, cb, sb, chunks, bptr, acc, err)
+                                          : w16_stream<2, COMPACT>(ring, cb, sb, chunks, bptr, acc, err);
             if (!ok) return;
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
@@ -443,7 +522,8 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
                         for (int u = 0; u < 2; ++u)
 #pragma unroll
                             for (int h = 0; h < 2; ++h)
-                                Y[(int64_t)row * H + hb * 32 + u * 16 + g + 8 * h] = acc[u][nt][2 * h + j] * w;
+                                Y[(int64_t)row * H + hb * 32 + u * 16 + g + 8 * h] =
+                                    acc[u][nt][2 * h + j] * (w * ph[u][h]);
                     }
                 }
             }
@@ -453,42 +533,80 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
 
 }  // namespace
 
-size_t w4a16_packed_size(int E, int H, int I) { return (size_t)w16_layout(E, H, I).total; }
+size_t w4a16_packed_size(int E, int H, int I, bool compact) { return (size_t)w16_layout(E, H, I, compact).total; }
 
 size_t w4a16_scratch_size(int T, int H, int I, int k) {
     return (size_t)(align256((int64_t)T * H * 2) + align256((int64_t)T * 4) + align256((int64_t)T * k * I * 2) +
                     align256((int64_t)T * k * 4));
 }
 
-nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream) {
+template <bool COMPACT>
+static nvfp4moe_status pack_tiles(const nvfp4moe_expert_weights& w, uint8_t* p, const W16Layout& L,
+                                  cudaStream_t stream) {
     const int E = w.E, H = w.H, I = w.I;
-    const W16Layout L = w16_layout(E, H, I);
-    uint8_t* p = static_cast<uint8_t*>(packed);
+    const int8_t* rg = COMPACT ? reinterpret_cast<const int8_t*>(p + L.rexp_g) : nullptr;
+    const int8_t* ru = COMPACT ? reinterpret_cast<const int8_t*>(p + L.rexp_u) : nullptr;
+    const int8_t* rd = COMPACT ? reinterpret_cast<const int8_t*>(p + L.rexp_d) : nullptr;
     {
         const int64_t n_tiles = (int64_t)E * (I / 16) * 2;
         const int64_t threads = n_tiles * (H / 64) * 32;
-        k_w16_pack<<<(unsigned)ceil_div(threads, 256), 256, 0, stream>>>(w.gate_codes, w.gate_sf, n_tiles, H, 1,
-                                                                         w.up_codes, w.up_sf, p + L.gu_codes,
-                                                                         p + L.gu_scales, I);
+        k_w16_pack<COMPACT><<<(unsigned)ceil_div(threads, 256), 256, 0, stream>>>(
+            w.gate_codes, w.gate_sf, n_tiles, H, 1, w.up_codes, w.up_sf, p + L.gu_codes, p + L.gu_scales, I, rg, ru);
         NVFP4MOE_CHECK_LAUNCH("w4a16 pack (gate/up)");
     }
     {
         const int64_t n_tiles = (int64_t)E * (H / 16);
         const int64_t threads = n_tiles * (I / 64) * 32;
-        k_w16_pack<<<(unsigned)ceil_div(threads, 256), 256, 0, stream>>>(w.down_codes, w.down_sf, n_tiles, I, 0,
-                                                                         nullptr, nullptr, p + L.d_codes,
-                                                                         p + L.d_scales, H);
+        k_w16_pack<COMPACT><<<(unsigned)ceil_div(threads, 256), 256, 0, stream>>>(
+            w.down_codes, w.down_sf, n_tiles, I, 0, nullptr, nullptr, p + L.d_codes, p + L.d_scales, H, rd, nullptr);
         NVFP4MOE_CHECK_LAUNCH("w4a16 pack (down)");
     }
-    NVFP4MOE_CUDA(cudaMemcpyAsync(p + L.globals, w.w_global, (size_t)E * 3 * sizeof(float), cudaMemcpyDeviceToDevice,
-                                  stream));
     return NVFP4MOE_OK;
 }
 
-nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T, int H, int I, int E, int k,
-                                   const RoutingPlan& plan, uint16_t* A2, float* Y, void* scratch,
+nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed, bool compact, cudaStream_t stream) {
+    const int E = w.E, H = w.H, I = w.I;
+    const W16Layout L = w16_layout(E, H, I, compact);
+    uint8_t* p = static_cast<uint8_t*>(packed);
+    if (compact) {
+        // row exponents and the count of rows without a compact form, then the tiles
+        int32_t* n_bad = reinterpret_cast<int32_t*>(p + L.status);
+        NVFP4MOE_CUDA(cudaMemsetAsync(n_bad, 0, sizeof(int32_t), stream));
+        int8_t* rg = reinterpret_cast<int8_t*>(p + L.rexp_g);
+        int8_t* ru = reinterpret_cast<int8_t*>(p + L.rexp_u);
+        int8_t* rd = reinterpret_cast<int8_t*>(p + L.rexp_d);
+        const nvfp4moe_status st[3] = {
+            launch_compact_rows(w.gate_codes, w.gate_sf, (int64_t)E * I, H, rg, nullptr, nullptr, n_bad, stream),
+            launch_compact_rows(w.up_codes, w.up_sf, (int64_t)E * I, H, ru, nullptr, nullptr, n_bad, stream),
+            launch_compact_rows(w.down_codes, w.down_sf, (int64_t)E * H, I, rd, nullptr, nullptr, n_bad, stream)};
+        for (nvfp4moe_status s : st)
+            if (s != NVFP4MOE_OK) return s;
+        const nvfp4moe_status s = pack_tiles<true>(w, p, L, stream);
+        if (s != NVFP4MOE_OK) return s;
+    } else {
+        const nvfp4moe_status s = pack_tiles<false>(w, p, L, stream);
+        if (s != NVFP4MOE_OK) return s;
+    }
+    NVFP4MOE_CUDA(cudaMemcpyAsync(p + L.globals, w.w_global, (size_t)E * 3 * sizeof(float), cudaMemcpyDeviceToDevice,
+                                  stream));
+    if (compact) {
+        int32_t bad = 0;
+        NVFP4MOE_CUDA(cudaMemcpyAsync(&bad, p + L.status, sizeof(bad), cudaMemcpyDeviceToHost, stream));
+        NVFP4MOE_CUDA(cudaStreamSynchronize(stream));
+        if (bad != 0) {
+            set_error("moe_pack_weights: %d weight rows have no compact scale form (unequal or non-power-of-two "
+                      "scale pairs, a zero scale over non-zero codes, or an exponent spread above 14)",
+                      bad);
+            return NVFP4MOE_ERR_NOT_REPRESENTABLE;
+        }
+    }
+    return NVFP4MOE_OK;
+}
+
+nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, bool compact, int T, int H, int I,
+                                   int E, int k, const RoutingPlan& plan, uint16_t* A2, float* Y, void* scratch,
                                    cudaStream_t stream, cudaEvent_t mid_event) {
-    const W16Layout L = w16_layout(E, H, I);
+    const W16Layout L = w16_layout(E, H, I, compact);
     const uint8_t* p = static_cast<const uint8_t*>(packed);
     uint8_t* sc = static_cast<uint8_t*>(scratch);
     __half* x16 = reinterpret_cast<__half*>(sc);
@@ -502,13 +620,15 @@ nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T,
     const int64_t max_active = std::min<int64_t>(E, P);
     const int64_t max_ctas = (int64_t)num_sms() * W16_MIN_CTAS;
     int32_t* err = device_error_word();
-    NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));
-    NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_down, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));
+    auto gateup = compact ? k_w16_gateup<true> : k_w16_gateup<false>;
+    auto down = compact ? k_w16_down<true> : k_w16_down<false>;
+    NVFP4MOE_CUDA(cudaFuncSetAttribute(gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));
+    NVFP4MOE_CUDA(cudaFuncSetAttribute(down, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));
     k_rows_to_f16<<<(unsigned)ceil_div(T, 8), 256, 0, stream>>>(x, T, H, x16, x_inv);
     NVFP4MOE_CHECK_LAUNCH("w4a16 activation conversion");
     {
         const int64_t ctas = std::min<int64_t>(ceil_div(max_active * (I / 16), W16_WARPS), max_ctas);
-        k_w16_gateup<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(x16, x_inv, p, L, H, I, k, plan, A2, err);
+        gateup<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(x16, x_inv, p, L, H, I, k, plan, A2, err);
         NVFP4MOE_CHECK_LAUNCH("w4a16 gate/up kernel");
     }
     if (mid_event) cudaEventRecord(mid_event, stream);
@@ -516,7 +636,7 @@ nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, int T,
     NVFP4MOE_CHECK_LAUNCH("w4a16 intermediate conversion");
     {
         const int64_t ctas = std::min<int64_t>(ceil_div(max_active * (H / 32), W16_WARPS), max_ctas);
-        k_w16_down<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(p, L, H, I, plan, a16, a_inv, Y, err);
+        down<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(p, L, H, I, plan, a16, a_inv, Y, err);
         NVFP4MOE_CHECK_LAUNCH("w4a16 down kernel");
     }
     return NVFP4MOE_OK;

@@ -24,6 +24,11 @@ keeps 16 experts per group):
 * ``skewed``    T=65536, E=128 (8 groups x 16), otherwise as ``prefill``; router
                 logits N(0,1) plus a per-expert Zipf(1.1) bias -1.1*ln(r_e), r a
                 seeded permutation of 1..E.
+* ``decode_pow2`` as ``decode``, but with the scale structure of a transcoded
+                MXFP4 checkpoint: per 32 codes one E4M3 byte drawn uniformly
+                from the zero-mantissa codes 0x08, 0x10, .., 0x48 (2^-6 .. 2^2),
+                the same byte for both 16-code halves; W4A16 with compact
+                scales.
 
 Activations are BF16 N(0,1) (drawn in float32, stored as BF16 bit patterns);
 router logits are float32 N(0,1).  Seeds are 1234 + the workload's index.
@@ -47,8 +52,8 @@ class Workload:
     topk_group: int
     top_k: int
     rsf: float
-    mode: int  # 0 = W4A16, 1 = W4A4
-    weights: str  # "mxfp4_tiny" | "nvfp4"
+    mode: int  # 0 = W4A16, 1 = W4A4, 2 = W4A16 with compact scales
+    weights: str  # "mxfp4_tiny" | "nvfp4" | "nvfp4_pow2"
     outliers: bool = False
     zipf: bool = False
 
@@ -62,6 +67,7 @@ WORKLOADS = {
     "decode": Workload("decode", 2, 16, 4096, 2048, 256, 8, 4, 8, 2.827, 0, "nvfp4"),
     "prefill": Workload("prefill", 3, 8192, 4096, 2048, 256, 8, 4, 8, 2.827, 1, "nvfp4", outliers=True),
     "skewed": Workload("skewed", 4, 65536, 4096, 2048, 128, 8, 4, 8, 2.827, 1, "nvfp4", outliers=True, zipf=True),
+    "decode_pow2": Workload("decode_pow2", 5, 16, 4096, 2048, 256, 8, 4, 8, 2.827, 2, "nvfp4_pow2"),
 }
 
 TRANSCODE_SEED = 1234 + 1
@@ -127,6 +133,17 @@ def nvfp4_tensors(rng: np.random.Generator, num: int, N: int, K: int):
     return codes, scales, glob
 
 
+def nvfp4_pow2_tensors(rng: np.random.Generator, num: int, N: int, K: int):
+    """NVFP4 tensors [num, N, K] whose two scales per 32 codes are one E4M3 byte
+    drawn from the zero-mantissa codes 0x08 .. 0x48 (values 2^-6 .. 2^2); codes
+    uniform; global 2^-4 per tensor."""
+    codes = random_codes(rng, (num, N, K // 2))
+    pick = rng.integers(1, 10, size=(num, N, K // 32), dtype=np.uint8) * np.uint8(8)
+    scales = np.repeat(pick, 2, axis=2)
+    glob = np.full(num, 2.0 ** -4, np.float32)
+    return codes, scales, glob
+
+
 def transcode_layer(rng: np.random.Generator, E: int = 256, H: int = 4096, I: int = 2048):
     """One MoE layer of MXFP4 expert weights plus one adversarial tensor.
 
@@ -165,9 +182,10 @@ def moe_inputs(wl: Workload, T: int | None = None):
             "down": mxfp4_tensors(rng, E, H, I, -8, -3),
         }
     else:
-        gc, gs, gg = nvfp4_tensors(rng, E, I, H)
-        uc, us, ug = nvfp4_tensors(rng, E, I, H)
-        dc, ds, dg = nvfp4_tensors(rng, E, H, I)
+        gen = nvfp4_pow2_tensors if wl.weights == "nvfp4_pow2" else nvfp4_tensors
+        gc, gs, gg = gen(rng, E, I, H)
+        uc, us, ug = gen(rng, E, I, H)
+        dc, ds, dg = gen(rng, E, H, I)
         out.update(gate_codes=gc, gate_sf=gs, up_codes=uc, up_sf=us, down_codes=dc, down_sf=ds,
                    w_global=np.stack([gg, ug, dg], axis=1).astype(np.float32))
     out["x"] = activations(rng, T, H, wl.outliers)

@@ -22,7 +22,7 @@ def declared_functions():
 def test_header_declares_the_hot_path_calls():
     names = declared_functions()
     for n in ("transcode_mxfp4_to_nvfp4", "moe_route", "quantize_nvfp4", "moe_forward", "moe_pack_weights",
-              "moe_permute", "moe_forward_routed", "moe_forward_ex"):
+              "moe_permute", "moe_forward_routed", "moe_forward_ex", "nvfp4_compact_scales"):
         assert n in names
 
 
@@ -40,6 +40,12 @@ def test_version_and_sizes():
     exact = E * (2 * I * H + H * I) // 2 + E * (2 * I * H + H * I) // 16 + E * 3 * 4
     assert exact <= moe.moe_packed_weights_size(moe.W4A4, E, H, I) <= exact + 1024
     assert exact <= moe.moe_packed_weights_size(moe.W4A16, E, H, I) <= exact + 1024
+    # compact scales: codes + one byte per 64 weights + one exponent byte per row + globals + a status word
+    compact = E * (2 * I * H + H * I) // 2 + E * (2 * I * H + H * I) // 64 + E * (2 * I + H) + E * 3 * 4 + 16
+    assert compact <= moe.moe_packed_weights_size(moe.W4A16C, E, H, I) <= compact + 2048
+    bits = 8 * moe.moe_packed_weights_size(moe.W4A16C, E, H, I) / (E * 3 * I * H)
+    assert 4.125 < bits < 4.13
+    assert moe.moe_packed_weights_size(3, E, H, I) == 0  # unknown mode
     ws = moe.moe_forward_workspace_size(moe.W4A4, 8192, H, I, E, 8)
     assert ws > 8192 * 8 * H * 2  # holds the per-pair BF16 rows at least
     assert moe.moe_forward_workspace_size(moe.W4A4, -1, H, I, E, 8) == 0
@@ -160,3 +166,15 @@ def test_router_topk_zero_tokens_and_sizes():
     assert moe.moe_router_topk_workspace_size(16) == 4
     assert moe.moe_router_topk_workspace_size(17) == 8
     assert moe.moe_router_topk_workspace_size(0) == 0
+
+
+def test_compact_scales_validation():
+    lib = moe.load()
+    p = ctypes.c_void_p(4096)
+    q = ctypes.c_void_p(4100)  # not 16-byte aligned
+    assert lib.nvfp4_compact_scales(p, p, 8, 96, p, p, p, None, None) == 3   # K % 64
+    assert lib.nvfp4_compact_scales(p, p, 8, 32, p, p, p, None, None) == 1   # K < 64
+    assert lib.nvfp4_compact_scales(p, p, -1, 128, p, p, p, None, None) == 1
+    assert lib.nvfp4_compact_scales(p, None, 8, 128, p, p, p, None, None) == 1
+    assert lib.nvfp4_compact_scales(p, p, 8, 128, q, p, p, None, None) == 2
+    assert lib.nvfp4_compact_scales(None, None, 0, 128, None, None, None, None, None) == 0  # no-op
