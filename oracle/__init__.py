@@ -217,10 +217,30 @@ def quantize_f32(x: np.ndarray, gs: float = 1.0):
     return codes, scales
 
 
+def quantize_mxfp8_f32(x: np.ndarray):
+    """MXFP8 of FP32 rows [M, K]: E4M3 codes [M, K] and E8M0 scales [M, K/32]."""
+    x = np.ascontiguousarray(x, np.float32)
+    M, K = x.shape
+    codes = np.empty((M, K), np.uint8)
+    scales = np.empty((M, K // 32), np.uint8)
+    _load().orc_quantize_mxfp8_f32(_p(x), ctypes.c_int64(M), ctypes.c_int64(K), _p(codes), _p(scales))
+    return codes, scales
+
+
+def quantize_mxfp8_bf16(x_bits: np.ndarray):
+    x = np.ascontiguousarray(x_bits, np.uint16)
+    M, K = x.shape
+    codes = np.empty((M, K), np.uint8)
+    scales = np.empty((M, K // 32), np.uint8)
+    _load().orc_quantize_mxfp8_bf16(_p(x), ctypes.c_int64(M), ctypes.c_int64(K), _p(codes), _p(scales))
+    return codes, scales
+
+
 def moe_layer(mode: int, x_bits, logits, bias, gate_codes, gate_sf, up_codes, up_sf, down_codes, down_sf,
               w_global, act_global: float, n_group: int, topk_group: int, top_k: int, rsf: float,
               renormalize: bool = True, tokens=None, act_global_mid=None) -> np.ndarray:
-    """float64 layer output [len(tokens), H] (mode 0 = W4A16, 1 = W4A4).  act_global
+    """float64 layer output [len(tokens), H] (mode 0 = W4A16, 1 = W4A4, 3 = W4A8:
+    MXFP8 activations, which takes no activation global).  act_global
     scales the layer input's quantisation, act_global_mid (default: the same) the
     down-projection input's."""
     x = np.ascontiguousarray(x_bits, np.uint16)

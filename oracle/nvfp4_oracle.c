@@ -540,6 +540,57 @@ void orc_quantize_bf16(const uint16_t* x, int64_t M, int64_t K, float gs, uint8_
 }
 
 /* ------------------------------------------------------------------------- */
+/* MXFP8 quantisation                                                         */
+/* ------------------------------------------------------------------------- */
+/* [P5] "Speed v5.2" and "Quantization, context and quality": prefill expert
+ * GEMMs take MXFP8 activations, E4M3 elements with one power-of-two scale per 32
+ * values, on the block-scaled FP8 x FP4 tensor cores.  The pages do not spell
+ * out the scale choice; the reading here is the OCP microscaling one: per 32
+ * elements of a row, with amax = max |x|,
+ *   X = floor(log2 amax) - 8   (8 = exponent of the largest E4M3 normal),
+ *   clamped to [-127, 127]; amax == 0 gives X = -127;
+ *   scale byte = X + 127 (E8M0);  q_i = E4M3_rne_satfinite(x_i / 2^X).
+ * x_i / 2^X is exact in FP32 (a power-of-two step that stays in range), so the
+ * only rounding is the E4M3 one.  codes [M, K] (one byte each), scales
+ * [M, K/32].                                                                 */
+void orc_quantize_mxfp8_f32(const float* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* scales) {
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t b = 0; b < K / 32; ++b) {
+            const float* xb = x + m * K + b * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double a = fabs((double)xb[i]);
+                if (a > amax) amax = a;
+            }
+            int X = -127;
+            if (amax > 0.0) {
+                int ex;
+                frexp(amax, &ex); /* amax = f * 2^ex, f in [0.5, 1): floor(log2 amax) = ex - 1 */
+                X = ex - 1 - 8;
+                if (X < -127) X = -127;
+                if (X > 127) X = 127;
+            }
+            scales[m * (K / 32) + b] = (uint8_t)(X + 127);
+            for (int i = 0; i < 32; ++i) codes[m * K + b * 32 + i] = orc_e4m3_rne_satfinite(ldexpf(xb[i], -X));
+        }
+    }
+}
+
+void orc_quantize_mxfp8_bf16(const uint16_t* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* scales) {
+    float* xf = (float*)malloc(sizeof(float) * (size_t)K);
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k) xf[k] = orc_bf16_to_float(x[m * K + k]);
+        orc_quantize_mxfp8_f32(xf, 1, K, codes + m * K, scales + m * (K / 32));
+    }
+    free(xf);
+}
+
+/* value of element k of an MXFP8 row */
+static double mxfp8_value(const uint8_t* codes, const uint8_t* scales, int64_t k) {
+    return orc_e4m3_value(codes[k]) * orc_e8m0_value(scales[k / 32]);
+}
+
+/* ------------------------------------------------------------------------- */
 /* The MoE layer                                                              */
 /* ------------------------------------------------------------------------- */
 /* Expert MLP ([P4] "Pruning Method" 1, the expert output inside the saliency
@@ -548,7 +599,9 @@ void orc_quantize_bf16(const uint16_t* x, int64_t M, int64_t K, float gs, uint8_
  * Modes ([P1] "Usage"/"Accuracy"): W4A16 keeps the activations in BF16 (the
  * SwiGLU output is rounded FP32 -> BF16 before the down projection); W4A4
  * quantises the activations to NVFP4 with the unit global scale ([P1] "Why a
- * unit activation scale") and requantises the SwiGLU output per 16 the same way.
+ * unit activation scale") and requantises the SwiGLU output per 16 the same way;
+ * W4A8 (mode 3, [P5] "Speed v5.2") quantises the layer input and the SwiGLU
+ * output to MXFP8 (above) and keeps the NVFP4 weights.
  * Weights: NVFP4, gate/up [E, I, H] and down [E, H, I] (out x in), scales per 16
  * along the input dimension, w_global[E][3] = gate, up, down global scales.
  * Everything after decoding is float64; out is [n_tokens, H] for the listed
@@ -587,7 +640,14 @@ void orc_moe_layer2(int mode, const uint16_t* x, const float* logits, const floa
         double* o = out + (int64_t)it * H;
         for (int h = 0; h < H; ++h) o[h] = 0.0;
 
-        if (mode == 1) {
+        if (mode == 3) {
+            uint8_t* xq = (uint8_t*)malloc((size_t)H);
+            uint8_t* xs = (uint8_t*)malloc((size_t)H / 32);
+            orc_quantize_mxfp8_bf16(x + (int64_t)t * H, 1, H, xq, xs);
+            for (int h = 0; h < H; ++h) xd[h] = mxfp8_value(xq, xs, h);
+            free(xq);
+            free(xs);
+        } else if (mode == 1) {
             uint8_t* xq = (uint8_t*)malloc((size_t)H / 2);
             uint8_t* xs = (uint8_t*)malloc((size_t)H / 16);
             orc_quantize_bf16(x + (int64_t)t * H, 1, H, act_global, xq, xs);
@@ -611,7 +671,15 @@ void orc_moe_layer2(int mode, const uint16_t* x, const float* logits, const floa
                 for (int h = 0; h < H; ++h) u += xd[h] * wrow[h];
                 a[i] = silu(g) * u;
             }
-            if (mode == 1) {
+            if (mode == 3) {
+                uint8_t* mq = (uint8_t*)malloc((size_t)I);
+                uint8_t* ms = (uint8_t*)malloc((size_t)I / 32);
+                for (int i = 0; i < I; ++i) a32[i] = (float)a[i];
+                orc_quantize_mxfp8_f32(a32, 1, I, mq, ms);
+                for (int i = 0; i < I; ++i) a[i] = mxfp8_value(mq, ms, i);
+                free(mq);
+                free(ms);
+            } else if (mode == 1) {
                 for (int i = 0; i < I; ++i) a32[i] = (float)a[i];
                 orc_quantize_f32(a32, 1, I, act_global_mid, aq, as);
                 for (int i = 0; i < I; ++i)

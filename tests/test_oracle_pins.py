@@ -546,6 +546,79 @@ def test_layer_combines_two_experts_with_routing_weights():
 
 
 # ---------------------------------------------------------------------------
+# MXFP8 activations ("MiMo-V2.6-Flash-MOPD on one RTX PRO 6000", "Speed v5.2":
+# E4M3 with a power-of-two scale per 32 values; OCP scale choice)
+# ---------------------------------------------------------------------------
+
+def _mx8_reference(x: np.ndarray):
+    """Independent MXFP8 of FP32 rows with numpy frexp and torch's E4M3 cast."""
+    M, K = x.shape
+    blocks = x.astype(np.float64).reshape(M, K // 32, 32)
+    amax = np.abs(blocks).max(-1)
+    X = np.where(amax > 0, np.frexp(amax)[1] - 1 - 8, -127).clip(-127, 127)
+    scaled = blocks * np.exp2(-X.astype(np.float64))[..., None]
+    codes = torch.from_numpy(np.clip(scaled, -448, 448).reshape(M, K)).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.numpy(), (X + 127).astype(np.uint8)
+
+
+def _mx8_decode(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    v = torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return v * np.repeat(np.exp2(scales.astype(np.float64) - 127), 32, axis=1)
+
+
+def test_mxfp8_matches_frexp_and_torch_e4m3():
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal((48, 256)) * np.exp(rng.uniform(-30, 30, (48, 1)))).astype(np.float32)
+    x[3, 32:64] = 0.0                  # zero block
+    x[4, 5] = 3.0e38                   # near the FP32 maximum
+    x[5, 0:32] = 1e-42                 # FP32 subnormals
+    x[6, 64:96] = np.float32(2.0 ** -3)  # power-of-two amax
+    codes, scales = oracle.quantize_mxfp8_f32(x)
+    rc, rs = _mx8_reference(x)
+    assert np.array_equal(scales, rs)
+    same = (codes == rc) | ((codes & 0x7F) == 0) & ((rc & 0x7F) == 0)  # +-0 either way
+    assert same.all()
+    assert scales[3, 1] == 0 and np.all(codes[3, 32:64] & 0x7F == 0)
+
+
+def test_mxfp8_hand_values():
+    x = np.zeros((1, 32), np.float32)
+    x[0, :6] = [1.0, 0.3, -1.9, 2.0 ** -9, 1.875, 0.0]
+    codes, scales = oracle.quantize_mxfp8_f32(x)
+    # amax 1.9: X = 0 - 8, scale byte 119; elements x * 256
+    assert scales[0, 0] == 119
+    assert codes[0, 0] == 0x78          # 256 = 2^8
+    assert codes[0, 1] == 0x6A          # 76.8 -> 80 = 1.25 * 2^6
+    assert codes[0, 2] == 0xFE          # -486.4 saturates to -448
+    assert codes[0, 3] == 0x30          # 2^-9 * 2^8 = 2^-1
+    assert codes[0, 4] == 0x7E          # 480 saturates to 448
+    assert codes[0, 5] == 0x00
+
+
+def test_layer_w4a8_reduces_to_dense_swiglu():
+    # mode 3: MXFP8 layer input and SwiGLU output, NVFP4 weights (E=1, k=1, rsf=1)
+    rng = np.random.default_rng(25)
+    T, H, I = 5, 64, 64
+    gc, gs, _ = inputs.nvfp4_tensors(rng, 1, I, H)
+    uc, us, _ = inputs.nvfp4_tensors(rng, 1, I, H)
+    dc, ds, _ = inputs.nvfp4_tensors(rng, 1, H, I)
+    wg = np.array([[0.5, 0.25, 2.0]], np.float32)
+    x = inputs.activations(rng, T, H, outliers=True)
+    logits = rng.standard_normal((T, 1)).astype(np.float32)
+    out = oracle.moe_layer(3, x, logits, None, gc, gs, uc, us, dc, ds, wg, 1.0, 1, 1, 1, 1.0)
+    xf = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(torch.float32).numpy()
+    xc, xs = _mx8_reference(xf)
+    xq = _mx8_decode(xc, xs)
+    G = xq @ _np_decode(gc[0], gs[0], 0.5).T
+    U = xq @ _np_decode(uc[0], us[0], 0.25).T
+    A = G / (1 + np.exp(-G)) * U
+    ac, as_ = _mx8_reference(A.astype(np.float32))
+    Y = _mx8_decode(ac, as_) @ _np_decode(dc[0], ds[0], 2.0).T
+    assert np.allclose(out, Y, rtol=1e-12, atol=1e-12 * np.abs(Y).max())
+    # and it is not the W4A4 or W4A16 layer
+    assert not np.allclose(out, oracle.moe_layer(1, x, logits, None, gc, gs, uc, us, dc, ds, wg, 1.0, 1, 1, 1, 1.0),
+                           rtol=1e-6)
+# ---------------------------------------------------------------------------
 # router projection ("MiMo-V2.6-Flash-MOPD on one RTX PRO 6000", "What makes it
 # fast": the router's matmul; routers kept in F32 per the mixed-quant GGUF
 # page's precision table)
