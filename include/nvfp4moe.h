@@ -237,6 +237,19 @@ nvfp4moe_status moe_permute_noalloc(const int32_t* topk_ids, int32_t T, int32_t 
 nvfp4moe_status quantize_nvfp4(const uint16_t* x_bf16, int64_t M, int64_t K, float gs, uint8_t* codes,
                                uint8_t* e4m3_scales, void* stream);
 
+/* MXFP8 activation quantisation ("MiMo-V2.6-Flash-MOPD on one RTX PRO 6000",
+ * "Speed v5.2" and "Quantization, context and quality": E4M3 elements with one
+ * power-of-two scale per 32 values, the prefill activations of the W4A8 mode).
+ * Scale choice (the OCP microscaling one; the pages do not spell it out): per 32
+ * consecutive elements of a row, X = floor(log2 amax) - 8 clamped to
+ * [-127, 127] (-127 when amax is 0 or below the FP32 normal range); scale byte
+ * X + 127 (E8M0); element E4M3 round-to-nearest-even, saturating to +-448, of
+ * x * 2^-X (the sign of a zero result is kept).
+ *   x_bf16 [M, K] BF16 bit patterns; codes [M, K] E4M3 bytes; e8m0_scales
+ *   [M, K/32].  Constraints: K % 32 == 0, M >= 0 (0 is a no-op).            */
+nvfp4moe_status quantize_mxfp8(const uint16_t* x_bf16, int64_t M, int64_t K, uint8_t* codes, uint8_t* e8m0_scales,
+                               void* stream);
+
 /* ------------------------------------------------------------------------- */
 /* The MoE layer                                                              */
 /* ------------------------------------------------------------------------- */
@@ -255,6 +268,13 @@ nvfp4moe_status quantize_nvfp4(const uint16_t* x_bf16, int64_t M, int64_t K, flo
  *                   in the pages' recipe); FP4 x FP4 block-scaled tcgen05 MMA;
  *                   SwiGLU output requantised per 16 with the same global
  *                   (moe_forward_ex takes a separate global for it).
+ *   NVFP4MOE_W4A8:  activations (layer input and SwiGLU output) quantised to
+ *                   MXFP8 (see quantize_mxfp8) on the block-scaled FP8 x FP4
+ *                   tcgen05 MMA ("MiMo-V2.6-Flash-MOPD on one RTX PRO 6000",
+ *                   "Speed v5.2"); the weights keep their E2M1 codes and take
+ *                   each 32-code block's power-of-two scale as E8M0, so they
+ *                   must have that form (the MXFP4 transcode gives it); the
+ *                   activation globals are not used.
  * FP32 accumulation throughout; the combine adds the k weighted expert rows of a
  * token in slot order in FP32 and rounds once to the output type.
  *
@@ -262,7 +282,12 @@ nvfp4moe_status quantize_nvfp4(const uint16_t* x_bf16, int64_t M, int64_t K, flo
  * projection), which moe_pack_weights rearranges once into the layout the GEMM
  * kernels read:
  */
-typedef enum nvfp4moe_mode { NVFP4MOE_W4A16 = 0, NVFP4MOE_W4A4 = 1, NVFP4MOE_W4A16C = 2 } nvfp4moe_mode;
+typedef enum nvfp4moe_mode {
+    NVFP4MOE_W4A16 = 0,
+    NVFP4MOE_W4A4 = 1,
+    NVFP4MOE_W4A16C = 2,
+    NVFP4MOE_W4A8 = 3
+} nvfp4moe_mode;
 
 typedef struct nvfp4moe_expert_weights {
     const uint8_t* gate_codes; /* [E, I, H/2]  */
@@ -285,7 +310,11 @@ size_t moe_packed_weights_size(nvfp4moe_mode mode, int32_t E, int32_t H, int32_t
  * W4A16).  Constraints: H % 128 == 0, I % 128 == 0, E >= 1.
  * NVFP4MOE_W4A16C re-encodes the scales (nvfp4_compact_scales) and is
  * SYNCHRONOUS: it waits for `stream` and returns NVFP4MOE_ERR_NOT_REPRESENTABLE
- * when any weight row has no compact form (the packed buffer is then unusable). */
+ * when any weight row has no compact form (the packed buffer is then unusable).
+ * NVFP4MOE_W4A8 stores each code in a byte-per-element padded form (twice the
+ * code bytes) with E8M0 scales, and is SYNCHRONOUS in the same way: a row whose
+ * 32-code blocks do not each have one power-of-two scale (or zero scale over
+ * zero codes) makes it return NVFP4MOE_ERR_NOT_REPRESENTABLE.               */
 nvfp4moe_status moe_pack_weights(nvfp4moe_mode mode, const nvfp4moe_expert_weights* weights_host_struct,
                                  void* packed, void* stream);
 

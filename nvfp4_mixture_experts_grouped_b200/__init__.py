@@ -18,13 +18,14 @@ __all__ = [
     "moe_router_topk_workspace_size", "quantize_nvfp4",
     "moe_packed_weights_size", "moe_pack_weights", "moe_forward_workspace_size", "moe_forward",
     "moe_forward_ex", "moe_forward_routed", "nvfp4moe_check_device_status", "nvfp4moe_version", "moe_permute",
-    "moe_permute_workspace_size", "nvfp4moe_set_trace_events", "moe_permute_noalloc", "W4A16C",
-    "nvfp4_compact_scales",
+    "moe_permute_workspace_size", "nvfp4moe_set_trace_events", "moe_permute_noalloc", "W4A16C", "W4A8",
+    "nvfp4_compact_scales", "quantize_mxfp8",
 ]
 
 W4A16 = 0
 W4A4 = 1
 W4A16C = 2  # W4A16 on weights with compact (4.125-bit) scales
+W4A8 = 3  # MXFP8 activations x FP4 weights (prefill)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libnvfp4moe.so")
@@ -83,6 +84,8 @@ def load():
     L.moe_router_topk_workspace_size.argtypes = [i32]
     L.moe_router_topk.restype = ctypes.c_int
     L.moe_router_topk.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp, vp, vp, sz, vp]
+    L.quantize_mxfp8.restype = ctypes.c_int
+    L.quantize_mxfp8.argtypes = [vp, i64, i64, vp, vp, vp]
     L.quantize_nvfp4.restype = ctypes.c_int
     L.quantize_nvfp4.argtypes = [vp, i64, i64, f32, vp, vp, vp]
     L.moe_packed_weights_size.restype = sz
@@ -175,6 +178,10 @@ def moe_router_topk(x_bf16, w_router, bias, n_group, topk_group, top_k, routed_s
                                   routed_scaling_factor, int(renormalize), _ptr(logits_out), _ptr(topk_ids),
                                   _ptr(topk_weights), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream)))
+
+
+def quantize_mxfp8(x, M, K, codes, e8m0_scales, stream=None):
+    _check(load().quantize_mxfp8(_ptr(x), M, K, _ptr(codes), _ptr(e8m0_scales), _stream(stream)))
 
 
 def quantize_nvfp4(x_bf16, gs, codes, e4m3_scales, stream=None):

@@ -102,9 +102,10 @@ static int64_t al(int64_t v) { return (v + 255) / 256 * 256; }
 static ForwardLayout forward_layout(nvfp4moe_mode mode, int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
     ForwardLayout L{};
     L.P = T * k;
-    L.pad = mode == NVFP4MOE_W4A4 ? MTILE : 1;
+    const bool tc = mode == NVFP4MOE_W4A4 || mode == NVFP4MOE_W4A8;  // tcgen05 GEMMs on 128-row tiles
+    L.pad = tc ? MTILE : 1;
     const int64_t occupied = std::min<int64_t>(E, L.P);
-    L.rows_max = mode == NVFP4MOE_W4A4 ? round_up(L.P + occupied * (MTILE - 1), MTILE) : std::max<int64_t>(L.P, 1);
+    L.rows_max = tc ? round_up(L.P + occupied * (MTILE - 1), MTILE) : std::max<int64_t>(L.P, 1);
     L.n_chunks = std::max<int64_t>(ceil_div(T, PERM_CHUNK), 1);
     L.max_tiles = ceil_div(L.P, MTILE) + occupied + 1;
     int64_t o = 0;
@@ -125,14 +126,21 @@ static ForwardLayout forward_layout(nvfp4moe_mode mode, int64_t T, int64_t H, in
     L.n_tiles = take(4);
     L.active = take(E * 4);
     L.n_active = take(4);
-    if (mode == NVFP4MOE_W4A4) {
-        L.a1c = take(L.rows_max * H / 2);
-        L.a1s = take(L.rows_max * H / 16);
-        L.a2c = take(L.rows_max * I / 2);
-        L.a2s = take(L.rows_max * I / 16);
+    if (tc) {
+        // W4A4: NVFP4 codes + E4M3 per 16; W4A8: E4M3 elements + E8M0 per 32
+        const bool mx = mode == NVFP4MOE_W4A8;
+        L.a1c = take(mx ? L.rows_max * H : L.rows_max * H / 2);
+        L.a1s = take(L.rows_max * H / (mx ? 32 : 16));
+        L.a2c = take(mx ? L.rows_max * I : L.rows_max * I / 2);
+        L.a2s = take(L.rows_max * I / (mx ? 32 : 16));
         L.a2bf = -1;
-        L.y = take(L.rows_max * H * 2);          // FP16 staged rows
-        L.ys = take(L.rows_max * (H / 64) * 4);  // their power-of-two scales
+        if (mx) {
+            L.y = take(L.rows_max * H * 4);  // FP32 staged rows
+            L.ys = -1;
+        } else {
+            L.y = take(L.rows_max * H * 2);          // FP16 staged rows
+            L.ys = take(L.rows_max * (H / 64) * 4);  // their power-of-two scales
+        }
     } else {
         L.a1c = L.a1s = L.a2c = L.a2s = L.ys = -1;
         L.a2bf = take(L.rows_max * I * 2);
@@ -293,6 +301,18 @@ nvfp4moe_status quantize_nvfp4(const uint16_t* x_bf16, int64_t M, int64_t K, flo
     return launch_quantize_linear(x_bf16, M, K, gs, codes, e4m3_scales, static_cast<cudaStream_t>(stream));
 }
 
+nvfp4moe_status quantize_mxfp8(const uint16_t* x_bf16, int64_t M, int64_t K, uint8_t* codes, uint8_t* e8m0_scales,
+                               void* stream) {
+    REQUIRE(M >= 0 && K >= 32, NVFP4MOE_ERR_INVALID_ARG, "bad sizes M=%lld K=%lld", (long long)M, (long long)K);
+    REQUIRE(K % 32 == 0, NVFP4MOE_ERR_UNSUPPORTED_SHAPE, "K=%lld is not a multiple of 32", (long long)K);
+    if (M == 0) return NVFP4MOE_OK;
+    REQUIRE(x_bf16 && codes && e8m0_scales, NVFP4MOE_ERR_INVALID_ARG, "null tensor pointer");
+    REQUIRE(aligned16(x_bf16) && aligned16(codes) && aligned16(e8m0_scales), NVFP4MOE_ERR_ALIGNMENT,
+            "a tensor pointer is not 16-byte aligned");
+    RETURN_IF(check_device());
+    return launch_quantize_mx8_linear(x_bf16, M, K, codes, e8m0_scales, static_cast<cudaStream_t>(stream));
+}
+
 size_t moe_permute_workspace_size(int32_t T, int32_t E, int32_t top_k, int32_t pad) {
     if (T < 0 || E < 1 || top_k < 1 || pad < 1) return 0;
     const int64_t P = (int64_t)T * top_k;
@@ -352,12 +372,13 @@ nvfp4moe_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t E, int32
 }
 
 static bool valid_mode(nvfp4moe_mode mode) {
-    return mode == NVFP4MOE_W4A16 || mode == NVFP4MOE_W4A4 || mode == NVFP4MOE_W4A16C;
+    return mode == NVFP4MOE_W4A16 || mode == NVFP4MOE_W4A4 || mode == NVFP4MOE_W4A16C || mode == NVFP4MOE_W4A8;
 }
 
 size_t moe_packed_weights_size(nvfp4moe_mode mode, int32_t E, int32_t H, int32_t I) {
     if (E < 1 || H < 1 || I < 1 || !valid_mode(mode)) return 0;
-    return mode == NVFP4MOE_W4A4 ? w4a4_packed_size(E, H, I) : w4a16_packed_size(E, H, I, mode == NVFP4MOE_W4A16C);
+    if (mode == NVFP4MOE_W4A4 || mode == NVFP4MOE_W4A8) return w4a4_packed_size(E, H, I, mode == NVFP4MOE_W4A8);
+    return w4a16_packed_size(E, H, I, mode == NVFP4MOE_W4A16C);
 }
 
 nvfp4moe_status moe_pack_weights(nvfp4moe_mode mode, const nvfp4moe_expert_weights* w, void* packed, void* stream) {
@@ -372,8 +393,8 @@ nvfp4moe_status moe_pack_weights(nvfp4moe_mode mode, const nvfp4moe_expert_weigh
     REQUIRE(aligned16(packed), NVFP4MOE_ERR_ALIGNMENT, "packed buffer is not 16-byte aligned");
     RETURN_IF(check_device());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return mode == NVFP4MOE_W4A4 ? launch_w4a4_pack(*w, packed, st)
-                                 : launch_w4a16_pack(*w, packed, mode == NVFP4MOE_W4A16C, st);
+    if (mode == NVFP4MOE_W4A4 || mode == NVFP4MOE_W4A8) return launch_w4a4_pack(*w, packed, mode == NVFP4MOE_W4A8, st);
+    return launch_w4a16_pack(*w, packed, mode == NVFP4MOE_W4A16C, st);
 }
 
 size_t moe_forward_workspace_size(nvfp4moe_mode mode, int32_t T, int32_t H, int32_t I, int32_t E, int32_t top_k) {
@@ -426,13 +447,17 @@ static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, con
     RETURN_IF(launch_permute(plan.ids, T, top_k, E, L.pad, plan, st));
     trace(2, st);
     void* Y = ws + L.y;
-    float* ys = mode == NVFP4MOE_W4A4 ? reinterpret_cast<float*>(ws + L.ys) : nullptr;
-    if (mode == NVFP4MOE_W4A4) {
+    const bool tc = mode == NVFP4MOE_W4A4 || mode == NVFP4MOE_W4A8;
+    float* ys = mode == NVFP4MOE_W4A4 ? reinterpret_cast<float*>(ws + L.ys) : nullptr;  // else FP32 rows
+    if (tc) {
         uint8_t* a1c = ws + L.a1c;
         uint8_t* a1s = ws + L.a1s;
-        RETURN_IF(launch_quantize_scatter(x, T, H, act_global, a1c, a1s, plan.row_of_pair, top_k, st));
+        if (mode == NVFP4MOE_W4A8)
+            RETURN_IF(launch_quantize_mx8_scatter(x, T, H, a1c, a1s, plan.row_of_pair, top_k, st));
+        else
+            RETURN_IF(launch_quantize_scatter(x, T, H, act_global, a1c, a1s, plan.row_of_pair, top_k, st));
         trace(3, st);
-        RETURN_IF(launch_w4a4_layer(packed, T, H, I, E, top_k, act_global, act_global_mid, L.rows_max, (int)L.max_tiles, plan, a1c,
+        RETURN_IF(launch_w4a4_layer(packed, mode == NVFP4MOE_W4A8, T, H, I, E, top_k, act_global, act_global_mid, L.rows_max, (int)L.max_tiles, plan, a1c,
                                     a1s, ws + L.a2c, ws + L.a2s, static_cast<__half*>(Y), ys, st,
                                     g_trace_on ? g_trace[4] : nullptr));
     } else {

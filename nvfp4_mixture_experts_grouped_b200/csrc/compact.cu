@@ -10,6 +10,10 @@
 // weight streams, so the 0.4375 bits per weight saved on scales are ~8% of
 // their HBM bytes.
 //
+// The same check with no spread limit (max_spread large) tells whether a row's
+// scales have an E8M0 form (one power of two per 32 codes), which the W4A8
+// weights need.
+//
 // One warp per row: pass 1 classifies the row's blocks (lane j takes blocks 2j
 // and 2j+1 of every 64 columns, one 32-bit load of their four scale bytes; the
 // codes are read only for zero-scale blocks) and reduces max / min exponent and
@@ -38,7 +42,7 @@ __device__ __forceinline__ int block_kind(const uint8_t* codes_row, uint32_t s0,
 __global__ void __launch_bounds__(CP_WARPS * 32)
     k_compact_rows(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf, int64_t rows, int64_t K,
                    int8_t* __restrict__ row_exp, uint8_t* __restrict__ nib, int32_t* __restrict__ row_status,
-                   int32_t* __restrict__ n_bad) {
+                   int32_t* __restrict__ n_bad, int max_spread) {
     const int64_t r = (int64_t)blockIdx.x * CP_WARPS + warp_id();
     if (r >= rows) return;
     const int lane = lane_id();
@@ -61,7 +65,7 @@ __global__ void __launch_bounds__(CP_WARPS * 32)
     }
     emax = __reduce_max_sync(0xffffffffu, emax);
     emin = __reduce_min_sync(0xffffffffu, emin);
-    const bool ok = !__any_sync(0xffffffffu, bad) && (emax == -128 || emax - emin <= 14);
+    const bool ok = !__any_sync(0xffffffffu, bad) && (emax == -128 || emax - emin <= max_spread);
     const int re = (ok && emax != -128) ? emax : 0;
     if (nib) {
         for (int64_t j = lane; j < n64; j += 32) {
@@ -81,7 +85,7 @@ __global__ void __launch_bounds__(CP_WARPS * 32)
         }
     }
     if (lane == 0) {
-        row_exp[r] = (int8_t)re;
+        if (row_exp) row_exp[r] = (int8_t)re;
         if (row_status) row_status[r] = ok ? 0 : 1;
         if (!ok && n_bad) atomicAdd(n_bad, 1);
     }
@@ -91,10 +95,10 @@ __global__ void __launch_bounds__(CP_WARPS * 32)
 
 nvfp4moe_status launch_compact_rows(const uint8_t* codes, const uint8_t* sf, int64_t rows, int64_t K,
                                     int8_t* row_exp, uint8_t* nib, int32_t* row_status, int32_t* n_bad,
-                                    cudaStream_t stream) {
+                                    cudaStream_t stream, int max_spread) {
     if (rows == 0) return NVFP4MOE_OK;
     k_compact_rows<<<(unsigned)ceil_div(rows, CP_WARPS), CP_WARPS * 32, 0, stream>>>(codes, sf, rows, K, row_exp, nib,
-                                                                                     row_status, n_bad);
+                                                                                     row_status, n_bad, max_spread);
     NVFP4MOE_CHECK_LAUNCH("compact scales kernel");
     return NVFP4MOE_OK;
 }

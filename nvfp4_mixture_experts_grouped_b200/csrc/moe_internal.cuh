@@ -56,16 +56,25 @@ nvfp4moe_status launch_quantize_linear(const uint16_t* x, int64_t M, int64_t K, 
                                        uint8_t* scales, cudaStream_t stream);
 nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H, float gs, uint8_t* codes,
                                         uint8_t* scales, const int32_t* row_of_pair, int k, cudaStream_t stream);
+// MXFP8 (E4M3 + E8M0 per 32): linear [M, K] codes / [M, K/32] scales, and the
+// scatter into permuted rows with atom-layout scales (K % 128 == 0)
+nvfp4moe_status launch_quantize_mx8_linear(const uint16_t* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* scales,
+                                           cudaStream_t stream);
+nvfp4moe_status launch_quantize_mx8_scatter(const uint16_t* x, int64_t T, int64_t H, uint8_t* codes, uint8_t* scales,
+                                            const int32_t* row_of_pair, int k, cudaStream_t stream);
 // Y staged as FP16 rows with a power-of-two scale per 64 columns (y_scale != nullptr,
 // W4A4) or as FP32 rows (y_scale == nullptr, W4A16).
 nvfp4moe_status launch_combine(const void* Y, const float* y_scale, const int32_t* row_of_pair, int64_t T, int H,
                                int k, void* out, bool out_f32, cudaStream_t stream);
 
-// compact.cu: compact scales of NVFP4 rows (row_exp [rows]; nib [rows, K/64],
-// row_status [rows] and the failure counter n_bad are optional).  K % 64 == 0.
+// compact.cu: compact scales of NVFP4 rows (row_exp [rows], nib [rows, K/64],
+// row_status [rows] and the failure counter n_bad, each optional).  K % 64 == 0.
+// max_spread: 14 for the compact form; larger only checks that every 32-code
+// block's scale is one power of two (the E8M0 form).
+constexpr int COMPACT_MAX_SPREAD = 14;
 nvfp4moe_status launch_compact_rows(const uint8_t* codes, const uint8_t* sf, int64_t rows, int64_t K,
                                     int8_t* row_exp, uint8_t* nib, int32_t* row_status, int32_t* n_bad,
-                                    cudaStream_t stream);
+                                    cudaStream_t stream, int max_spread = COMPACT_MAX_SPREAD);
 
 // w4a16.cu
 // compact = the 4.125-bit scale form (mode NVFP4MOE_W4A16C)
@@ -76,12 +85,13 @@ nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, bool c
                                    int E, int k, const RoutingPlan& plan, uint16_t* A2, float* Y, void* scratch,
                                    cudaStream_t stream, cudaEvent_t mid_event);
 
-// w4a4.cu
-size_t w4a4_packed_size(int E, int H, int I);
-nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream);
-nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E, int k, float act_global_in,
-                                  float act_global_mid, int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
-                                  const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, __half* Y, float* y_scale,
-                                  cudaStream_t stream, cudaEvent_t mid_event);
+// w4a4.cu: the tcgen05 pair GEMMs; mx8 selects W4A8 (MXFP8 activations x FP4
+// weights held in the padded form with E8M0 scales) instead of W4A4
+size_t w4a4_packed_size(int E, int H, int I, bool mx8);
+nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed, bool mx8, cudaStream_t stream);
+nvfp4moe_status launch_w4a4_layer(const void* packed, bool mx8, int T, int H, int I, int E, int k,
+                                  float act_global_in, float act_global_mid, int64_t rows_max, int max_tiles,
+                                  const RoutingPlan& plan, const uint8_t* A1c, const uint8_t* A1s, uint8_t* A2c,
+                                  uint8_t* A2s, __half* Y, float* y_scale, cudaStream_t stream, cudaEvent_t mid_event);
 
 }  // namespace nvfp4moe

@@ -311,6 +311,83 @@ nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H,
     return NVFP4MOE_OK;
 }
 
+// MXFP8 of BF16 rows (W4A8 layer input): one warp per row, four lanes per
+// 32-element block (8 elements each: one 16-byte load, an amax shuffle within
+// the quad, 8 code bytes), so a warp instruction covers 8 blocks = 512 contiguous
+// input bytes.  SCATTER writes each token's codes to its k permuted rows and the
+// scales in the block-scale atom layout (K % 128 == 0: the four blocks of an
+// atom word are in one half-warp); the linear form writes [M, K] codes and
+// row-major [M, K/32] scales.
+template <bool SCATTER>
+__global__ void __launch_bounds__(256)
+    k_quantize_mx8(const uint16_t* __restrict__ x, int64_t M, int64_t K, uint8_t* __restrict__ codes,
+                   uint8_t* __restrict__ scales, const int32_t* __restrict__ row_of_pair, int k) {
+    const int64_t m = (int64_t)blockIdx.x * 8 + warp_id();
+    if (m >= M) return;
+    const int lane = lane_id();
+    const int64_t nb = K / 32;
+    const uint16_t* xr = x + m * K;
+    const int my_row = SCATTER && lane < k ? row_of_pair[m * k + lane] : 0;
+    for (int64_t b0 = 0; b0 < nb; b0 += 8) {
+        const int64_t b = b0 + (lane >> 2);  // this lane's block; it holds elements 8 (lane % 4) .. +7
+        const bool active = b < nb;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (active) v = __ldg(reinterpret_cast<const uint4*>(xr + b * 32 + (lane & 3) * 8));
+        float f[8];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = bf16_bits_to_float(w[i] & 0xFFFFu);
+            f[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const int X = mx8_exponent(amax);
+        const float r = pow2_f32(-X);
+        const uint2 c = make_uint2(f32x4_to_e4m3x4(f[0] * r, f[1] * r, f[2] * r, f[3] * r),
+                                   f32x4_to_e4m3x4(f[4] * r, f[5] * r, f[6] * r, f[7] * r));
+        const uint32_t sf = (uint32_t)(X + 127);
+        if (!SCATTER) {
+            if (active) {
+                *reinterpret_cast<uint2*>(codes + m * K + b * 32 + (lane & 3) * 8) = c;
+                if ((lane & 3) == 0) scales[m * nb + b] = (uint8_t)sf;
+            }
+        } else {
+            // lanes 16h + 4j (j = 0..3) hold the scales of blocks b0 + 4h + j: one
+            // atom word, assembled in lane 16h
+            uint32_t sfw = sf << (8 * ((lane >> 2) & 3));
+            sfw |= __shfl_xor_sync(0xffffffffu, sfw, 4);
+            sfw |= __shfl_xor_sync(0xffffffffu, sfw, 8);
+            for (int j = 0; j < k; ++j) {
+                const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
+                if (active) {
+                    *reinterpret_cast<uint2*>(codes + row * K + b * 32 + (lane & 3) * 8) = c;
+                    if ((lane & 15) == 0) *reinterpret_cast<uint32_t*>(scales + sf_atom_offset(row, b, nb)) = sfw;
+                }
+            }
+        }
+    }
+}
+
+nvfp4moe_status launch_quantize_mx8_linear(const uint16_t* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* scales,
+                                           cudaStream_t stream) {
+    if (M == 0) return NVFP4MOE_OK;
+    k_quantize_mx8<false><<<(unsigned)ceil_div(M, 8), 256, 0, stream>>>(x, M, K, codes, scales, nullptr, 1);
+    NVFP4MOE_CHECK_LAUNCH("mxfp8 quantize kernel");
+    return NVFP4MOE_OK;
+}
+
+nvfp4moe_status launch_quantize_mx8_scatter(const uint16_t* x, int64_t T, int64_t H, uint8_t* codes, uint8_t* scales,
+                                            const int32_t* row_of_pair, int k, cudaStream_t stream) {
+    if (T == 0) return NVFP4MOE_OK;
+    k_quantize_mx8<true><<<(unsigned)ceil_div(T, 8), 256, 0, stream>>>(x, T, H, codes, scales, row_of_pair, k);
+    NVFP4MOE_CHECK_LAUNCH("mxfp8 quantize-scatter kernel");
+    return NVFP4MOE_OK;
+}
+
 // ---------------------------------------------------------------------------
 // 5. weighted un-permute: out[t] = sum_j Y[row_of_pair(t, j)] (routing weights
 //    already applied by the down GEMM), FP32 in slot order, one rounding.

@@ -239,6 +239,32 @@ __device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t d_tmem, uint64_t ades
         : "memory");
 }
 
+// Instruction descriptor of kind::mxf8f6f4 with UE8M0 block scales (one per 32
+// elements, scale_vec::1X): A E4M3, B E2M1 (held in shared memory in the padded
+// form: each 16 codes packed in 8 bytes followed by 8 bytes of padding), K-major,
+// FP32 accumulate.  The four bytes of a row's scale word in TMEM serve four
+// consecutive K=32 MMAs; scale_id (0..3) selects the byte, for A and B alike.
+__host__ __device__ constexpr uint32_t idesc_mxf8f6f4_e4m3_e2m1(int M, int N, uint32_t scale_id) {
+    return (scale_id << 4)                 // B scale factor byte
+           | (0u << 7)                     // A format: E4M3
+           | (5u << 10)                    // B format: E2M1
+           | ((uint32_t)(N >> 3) << 17)    // N / 8
+           | (1u << 23)                    // scale format: UE8M0
+           | ((uint32_t)(M >> 4) << 24)    // M / 16
+           | (scale_id << 29);             // A scale factor byte
+}
+
+__device__ __forceinline__ void mma_mxf8f6f4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
 // Copy a 32-row x 128-bit block from shared memory to TMEM, replicated into the
 // four 32-lane quadrants.
 __device__ __forceinline__ void tmem_cp_32x128_x4(uint32_t taddr, uint64_t sdesc) {
@@ -271,6 +297,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t v[16]) 
         "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
         "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
         : "memory");
+}
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t v[4]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t v[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+                 "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 

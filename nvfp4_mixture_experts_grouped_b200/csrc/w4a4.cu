@@ -45,21 +45,57 @@ namespace nvfp4moe {
 namespace {
 
 // A CTA pair computes a 256 x 256 tile: each CTA holds 128 rows of A, 128 rows
-// (N) of B, the scale factors of its A rows and of all 256 B rows.
-constexpr int BM = 128, BN = 256, BK = 256;  // BM per CTA, BN per pair, BK in elements (128 bytes of codes)
-constexpr int STAGES = 5;
-constexpr int A_BYTES = BM * BK / 2;
-constexpr int B_BYTES = (BN / 2) * BK / 2;
-constexpr int SFA_BYTES = BM * BK / 16;
-constexpr int SFB_BYTES = BN * BK / 16;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
-static_assert(SMEM_BYTES <= 232448, "shared-memory ring above the 227 KB a CTA may use");
-static_assert(STAGE_BYTES % 1024 == 0, "128-byte-swizzled operand tiles need 1024-byte alignment");
-static_assert(256 + STAGES * 48 <= 512, "accumulator + per-slot scale columns must fit the TMEM allocation");
+// (N) of B, the scale factors of its A rows and of all 256 B rows.  Two operand
+// kinds share the kernel:
+//   KIND_NVF4  W4A4: A and B E2M1 with E4M3 scales per 16, kind::mxf4nvf4
+//              (scale_vec::4X, K=64 per MMA); a stage is 256 K elements.
+//   KIND_MXF8  W4A8: A E4M3 with E8M0 scales per 32 (MXFP8), B E2M1 in the padded
+//              shared-memory form with E8M0 scales per 32, kind::mxf8f6f4
+//              (scale_vec::1X, K=32 per MMA); a stage is 128 K elements.
+// Either way an operand row of a stage is 128 bytes (one SWIZZLE_128B row) and a
+// stage holds four MMAs.
+constexpr int BM = 128, BN = 256;  // BM per CTA, BN per pair
+enum { KIND_NVF4 = 0, KIND_MXF8 = 1 };
+
+template <int KIND>
+struct Cfg;
+template <>
+struct Cfg<KIND_NVF4> {
+    static constexpr int BK = 256;        // K elements per stage
+    static constexpr int STAGES = 5;
+    static constexpr int SF_ELEMS = 16;   // elements per scale
+    static constexpr int SFA_ATOMS = 4;   // scale atoms (128 rows x 4 scales) per 128 rows per stage
+    static constexpr uint32_t SF_STRIDE = 48;  // TMEM scale columns per ring slot: A 4 x 4, B 4 x 8
+    static constexpr uint32_t SFB_COL = 16;    // B's first scale column within a slot
+};
+template <>
+struct Cfg<KIND_MXF8> {
+    static constexpr int BK = 128;
+    static constexpr int STAGES = 6;
+    static constexpr int SF_ELEMS = 32;
+    static constexpr int SFA_ATOMS = 1;
+    static constexpr uint32_t SF_STRIDE = 12;  // A 4, B 8 (one word per row holds the stage's four scales)
+    static constexpr uint32_t SFB_COL = 4;
+};
+constexpr int A_BYTES = BM * 128;         // 128 rows x 128 bytes
+constexpr int B_BYTES = (BN / 2) * 128;
+template <int KIND>
+__host__ __device__ constexpr int sfa_bytes() { return Cfg<KIND>::SFA_ATOMS * 512; }
+template <int KIND>
+__host__ __device__ constexpr int sfb_bytes() { return 2 * Cfg<KIND>::SFA_ATOMS * 512; }
+template <int KIND>
+__host__ __device__ constexpr int stage_bytes() {  // padded to the 1024-byte alignment of swizzled tiles
+    return (A_BYTES + B_BYTES + sfa_bytes<KIND>() + sfb_bytes<KIND>() + 1023) / 1024 * 1024;
+}
+template <int KIND>
+__host__ __device__ constexpr int smem_bytes() { return Cfg<KIND>::STAGES * stage_bytes<KIND>() + 1024 + 256; }
+static_assert(smem_bytes<KIND_NVF4>() <= 232448 && smem_bytes<KIND_MXF8>() <= 232448,
+              "shared-memory ring above the 227 KB a CTA may use");
+static_assert(256 + Cfg<KIND_NVF4>::STAGES * Cfg<KIND_NVF4>::SF_STRIDE <= 512 &&
+                  256 + Cfg<KIND_MXF8>::STAGES * Cfg<KIND_MXF8>::SF_STRIDE <= 512,
+              "accumulator + per-slot scale columns must fit the TMEM allocation");
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_SF = 256;      // scale-factor columns after the 256 accumulator columns
-constexpr uint32_t TM_SF_STRIDE = 48;  // per ring slot: 16 (A: 4 k-steps x 4) + 32 (B: 4 x 8)
+constexpr uint32_t TM_SF = 256;  // scale-factor columns after the 256 accumulator columns
 constexpr int EPI_WARPS = 16;  // four warps per TMEM lane quadrant, each on a quarter of the columns
 constexpr int SF_WARPS = 4;    // one warp per TMEM lane quadrant writes the scale factors
 constexpr int THREADS = (2 + EPI_WARPS + SF_WARPS) * 32;
@@ -67,19 +103,25 @@ constexpr int THREADS = (2 + EPI_WARPS + SF_WARPS) * 32;
 enum { EPI_GATEUP = 0, EPI_DOWN = 1 };
 
 struct W4Layout {
-    int64_t gu_codes, gu_sf, d_codes, d_sf, globals, total;
+    int64_t gu_codes, gu_sf, d_codes, d_sf, globals, status, total;
 };
 
 inline int64_t a256(int64_t v) { return (v + 255) / 256 * 256; }
 
-W4Layout w4_layout(int E, int H, int I) {
+// W4A4: codes 4 bits and an E4M3 scale per 16 elements (the checkpoint's bytes).
+// W4A8: codes in the padded form (16 codes in 8 bytes + 8 bytes of padding, so
+// one byte per element) and an E8M0 scale per 32; a status word for the pack.
+W4Layout w4_layout(int E, int H, int I, bool mx8 = false) {
+    const int64_t n = (int64_t)E * 3 * I * H;  // weights of the layer
+    const int64_t gu = (int64_t)E * 2 * I * H;
     W4Layout L;
     L.gu_codes = 0;
-    L.gu_sf = a256(L.gu_codes + (int64_t)E * 2 * I * H / 2);
-    L.d_codes = a256(L.gu_sf + (int64_t)E * 2 * I * H / 16);
-    L.d_sf = a256(L.d_codes + (int64_t)E * H * I / 2);
-    L.globals = a256(L.d_sf + (int64_t)E * H * I / 16);
-    L.total = a256(L.globals + (int64_t)E * 3 * 4);
+    L.gu_sf = a256(L.gu_codes + (mx8 ? gu : gu / 2));
+    L.d_codes = a256(L.gu_sf + (mx8 ? gu / 32 : gu / 16));
+    L.d_sf = a256(L.d_codes + (mx8 ? (n - gu) : (n - gu) / 2));
+    L.globals = a256(L.d_sf + (mx8 ? (n - gu) / 32 : (n - gu) / 16));
+    L.status = a256(L.globals + (int64_t)E * 3 * 4);
+    L.total = mx8 ? a256(L.status + 16) : L.status;
     return L;
 }
 
@@ -97,7 +139,8 @@ struct GemmParams {
     uint8_t* out_codes;      // gate/up: intermediate codes [rows, I/2]
     uint8_t* out_sf;         // gate/up: intermediate scales, atom layout
     int out_k;               // gate/up: I
-    __half* Y;               // down: [rows, H] FP16 staged rows
+    __half* Y;               // down: [rows, H] FP16 staged rows (W4A4)
+    float* Yf;               // down: [rows, H] FP32 staged rows (W4A8)
     float* y_scale;          // down: [rows, H / 64] power-of-two scale of each 64 staged columns
     int ldy;                 // down: H
     const float* wts;        // down: routing weight of each pair
@@ -127,9 +170,53 @@ __device__ __forceinline__ uint32_t requant_block16(const float* x, float gs, ui
     return sf;
 }
 
-template <int EPI>
+// Transposes the 8 x 8 matrix of 16-byte chunks held by each group of 8 lanes
+// (pk: a lane's 8 chunks of 4 words), a butterfly over lane bits 1, 2, 4:
+// afterwards lane 8G + c holds chunk c of the group's rows 8G + 0..7, so one
+// store instruction writes whole 128-byte row segments.
+template <typename T>
+__device__ __forceinline__ void transpose_chunks8(T* pk, int lane) {
+    const int c8 = lane & 7;
+#pragma unroll
+    for (int b = 0; b < 3; ++b) {
+        const int m = 1 << b;
+        const bool hi = (c8 & m) != 0;
+#pragma unroll
+        for (int k0 = 0; k0 < 8; ++k0) {
+            if (k0 & m) continue;
+            const int k1 = k0 | m;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const T send = hi ? pk[4 * k0 + w] : pk[4 * k1 + w];
+                const T recv = __shfl_xor_sync(0xffffffffu, send, m);
+                if (hi) pk[4 * k0 + w] = recv;
+                else pk[4 * k1 + w] = recv;
+            }
+        }
+    }
+}
+
+// One stage's MMA j (of four): K=64 block-scaled FP4 (four E4M3 scales per row
+// and MMA, own TMEM columns) or K=32 FP8 x FP4 (one E8M0 scale per row and MMA,
+// byte j of the stage's scale word).
+template <int KIND>
+__device__ __forceinline__ void stage_mma(uint32_t tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t sf_col, int j, uint32_t accumulate) {
+    if (KIND == KIND_NVF4)
+        tc::mma_mxf4nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j, sf_col + 16 + 8 * j,
+                              accumulate);
+    else
+        tc::mma_mxf8f6f4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4),
+                              sf_col, sf_col + Cfg<KIND>::SFB_COL, accumulate);
+}
+
+template <int EPI, int KIND>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     k_w4a4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
+    constexpr int STAGES = Cfg<KIND>::STAGES;
+    constexpr int STAGE_BYTES = stage_bytes<KIND>();
+    constexpr int SFA_BYTES = sfa_bytes<KIND>();
+    constexpr uint32_t TM_SF_STRIDE = Cfg<KIND>::SF_STRIDE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
@@ -167,8 +254,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
     const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
     const int total = p.n_tiles[0] * p.n_ntiles;
-    const int k64_total = p.K / 64;
-    const int ks_count = (k64_total + 3) / 4;
+    // MMA steps (K=64 FP4 or K=32 FP8) and stages of four; scale atoms per 128 rows
+    const int ksub_total = KIND == KIND_NVF4 ? p.K / 64 : p.K / 32;
+    const int ks_count = (ksub_total + 3) / 4;
+    const int atoms_per_row = p.K / Cfg<KIND>::SF_ELEMS / 4;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -192,19 +281,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                     if (!tc::mbar_wait<true>(&empty[s], ph ^ 1u, p.err)) goto done;
-                    const int n64 = min(4, k64_total - ks * 4);
+                    // scale atoms of this stage per 128 rows (a partial last stage: W4A4 only)
+                    const int na = KIND == KIND_NVF4 ? min(4, ksub_total - ks * 4) : 1;
                     uint8_t* st = smem + s * STAGE_BYTES;
-                    tc::mbar_arrive_expect_tx(&full[s], B_BYTES + 2 * n64 * 512 + (a_live ? A_BYTES + n64 * 512 : 0));
+                    tc::mbar_arrive_expect_tx(&full[s], B_BYTES + 2 * na * 512 + (a_live ? A_BYTES + na * 512 : 0));
                     if (a_live) {
                         tc::tma_load_2d(st, &tmA, ks * 128, a_row, &full[s]);
-                        const uint8_t* sfa = p.sfa + ((int64_t)(a_row / 128) * k64_total + ks * 4) * 512;
-                        tc::bulk_load(st + A_BYTES + B_BYTES, sfa, n64 * 512, &full[s]);
+                        const uint8_t* sfa =
+                            p.sfa + ((int64_t)(a_row / 128) * atoms_per_row + ks * Cfg<KIND>::SFA_ATOMS) * 512;
+                        tc::bulk_load(st + A_BYTES + B_BYTES, sfa, na * 512, &full[s]);
                     }
                     tc::tma_load_2d(st + A_BYTES, &tmB, ks * 128, (int32_t)(b_tile0 + BM * rank), &full[s]);
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
-                        const uint8_t* sfb = p.sfb + ((b_tile0 / 128 + r) * k64_total + ks * 4) * 512;
-                        tc::bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES + r * 2048, sfb, n64 * 512, &full[s]);
+                        const uint8_t* sfb =
+                            p.sfb + ((b_tile0 / 128 + r) * atoms_per_row + ks * Cfg<KIND>::SFA_ATOMS) * 512;
+                        tc::bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES + r * SFA_BYTES, sfb, na * 512, &full[s]);
                     }
                 }
             }
@@ -225,7 +317,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // and scale column forward instead of recomputing them: its own
         // instructions are pipe idle time too.
         if (lane == 0 && rank == 0) {
-            const uint32_t idesc = tc::idesc_mxf4nvf4(2 * BM, BN);
+            const uint32_t idesc = KIND == KIND_NVF4 ? tc::idesc_mxf4nvf4(2 * BM, BN)
+                                                     : tc::idesc_mxf8f6f4_e4m3_e2m1(2 * BM, BN, 0);
             const int n_tiles_mine = pair < total ? (total - pair + n_pairs - 1) / n_pairs : 0;
             const int n_it = n_tiles_mine * ks_count;
             const uint64_t adesc0 = tc::desc_sw128(smem);
@@ -240,17 +333,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             uint64_t adesc = adesc0;
             uint32_t sf_col = tmem + TM_SF;
             for (int it = 0; it < n_it; ++it) {
-                const int n64 = ks + 1 < ks_count ? 4 : k64_total - ks * 4;
+                const int n64 = ks + 1 < ks_count ? 4 : ksub_total - ks * 4;
                 const uint64_t bdesc = adesc + B_DESC;
                 const uint32_t acc0 = ks != 0;
                 if (n64 == 4) {
-                    tc::mma_mxf4nvf4_pair(tmem, adesc, bdesc, idesc, sf_col, sf_col + 16, acc0);
-                    tc::mma_mxf4nvf4_pair(tmem, adesc + 2, bdesc + 2, idesc, sf_col + 4, sf_col + 24, 1u);
-                    tc::mma_mxf4nvf4_pair(tmem, adesc + 4, bdesc + 4, idesc, sf_col + 8, sf_col + 32, 1u);
+                    stage_mma<KIND>(tmem, adesc, bdesc, idesc, sf_col, 0, acc0);
+                    stage_mma<KIND>(tmem, adesc, bdesc, idesc, sf_col, 1, 1u);
+                    stage_mma<KIND>(tmem, adesc, bdesc, idesc, sf_col, 2, 1u);
                 } else {
                     for (int j = 0; j < n64 - 1; ++j)
-                        tc::mma_mxf4nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j,
-                                              sf_col + 16 + 8 * j, (ks | j) != 0);
+                        stage_mma<KIND>(tmem, adesc, bdesc, idesc, sf_col, j, (ks | j) != 0);
                 }
                 const int ns = s + 1 == STAGES ? 0 : s + 1;
                 const uint32_t nph = ns == 0 ? ph ^ 1u : ph;
@@ -259,11 +351,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 // next stage of the same tile: its scale factors (and so its operands)
                 bool ok = true;
                 if (more && !tile_end) ok = tc::mbar_wait<true>(&sf_ready[ns], nph, p.err);
-                {
-                    const int j = n64 - 1;
-                    tc::mma_mxf4nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j,
-                                          sf_col + 16 + 8 * j, (ks | j) != 0);
-                }
+                stage_mma<KIND>(tmem, adesc, bdesc, idesc, sf_col, n64 - 1, (ks | (n64 - 1)) != 0);
                 tc::tc_commit_pair(&empty[s], 0x3);
                 if (tile_end) {
                     tc::tc_commit_pair(acc_full, 0x3);
@@ -302,20 +390,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                 if (!tc::mbar_wait(&full[s], ph, p.err)) goto done;
                 const uint8_t* st = smem + s * STAGE_BYTES + A_BYTES + B_BYTES;
-                uint32_t v[48];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint4 a = *reinterpret_cast<const uint4*>(st + j * 512 + lane * 16);
-                    const uint4 b0 = *reinterpret_cast<const uint4*>(st + SFA_BYTES + j * 512 + lane * 16);
-                    const uint4 b1 = *reinterpret_cast<const uint4*>(st + SFA_BYTES + 2048 + j * 512 + lane * 16);
-                    v[4 * j + 0] = a.x, v[4 * j + 1] = a.y, v[4 * j + 2] = a.z, v[4 * j + 3] = a.w;
-                    v[16 + 8 * j + 0] = b0.x, v[16 + 8 * j + 1] = b0.y, v[16 + 8 * j + 2] = b0.z, v[16 + 8 * j + 3] = b0.w;
-                    v[16 + 8 * j + 4] = b1.x, v[16 + 8 * j + 5] = b1.y, v[16 + 8 * j + 6] = b1.z, v[16 + 8 * j + 7] = b1.w;
-                }
                 const uint32_t col = t_q + TM_SF + (uint32_t)s * TM_SF_STRIDE;
-                tc::tmem_st16(col, v);
-                tc::tmem_st16(col + 16, v + 16);
-                tc::tmem_st16(col + 32, v + 32);
+                if (KIND == KIND_NVF4) {
+                    uint32_t v[48];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 a = *reinterpret_cast<const uint4*>(st + j * 512 + lane * 16);
+                        const uint4 b0 = *reinterpret_cast<const uint4*>(st + SFA_BYTES + j * 512 + lane * 16);
+                        const uint4 b1 = *reinterpret_cast<const uint4*>(st + 2 * SFA_BYTES + j * 512 + lane * 16);
+                        v[4 * j + 0] = a.x, v[4 * j + 1] = a.y, v[4 * j + 2] = a.z, v[4 * j + 3] = a.w;
+                        v[16 + 8 * j + 0] = b0.x, v[16 + 8 * j + 1] = b0.y, v[16 + 8 * j + 2] = b0.z,
+                                       v[16 + 8 * j + 3] = b0.w;
+                        v[16 + 8 * j + 4] = b1.x, v[16 + 8 * j + 5] = b1.y, v[16 + 8 * j + 6] = b1.z,
+                                       v[16 + 8 * j + 7] = b1.w;
+                    }
+                    tc::tmem_st16(col, v);
+                    tc::tmem_st16(col + 16, v + 16);
+                    tc::tmem_st16(col + 32, v + 32);
+                } else {
+                    // one atom of A (columns 0..3) and the two of B (4..7: N rows 0..127, 8..11: 128..255)
+                    const uint4 a = *reinterpret_cast<const uint4*>(st + lane * 16);
+                    const uint4 b0 = *reinterpret_cast<const uint4*>(st + SFA_BYTES + lane * 16);
+                    const uint4 b1 = *reinterpret_cast<const uint4*>(st + 2 * SFA_BYTES + lane * 16);
+                    const uint32_t va[4] = {a.x, a.y, a.z, a.w};
+                    const uint32_t vb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                    tc::tmem_st4(col, va);
+                    tc::tmem_st8(col + 4, vb);
+                }
                 tc::tmem_st_wait();
                 tc::tc_fence_before();
                 __syncwarp();
@@ -359,26 +460,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 if (valid) {
                     const float ag = p.globals[ti.x * 3 + 0] * p.act_global;
                     const float au = p.globals[ti.x * 3 + 1] * p.act_global;
-                    const int nkb = p.out_k / 16;
-                    uint32_t codes[4], sfw = 0;
+                    if (KIND == KIND_NVF4) {
+                        const int nkb = p.out_k / 16;
+                        uint32_t codes[4], sfw = 0;
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float a[16];
+                        for (int c = 0; c < 2; ++c) {
+                            float a[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) a[i] = silu_fast(gv[16 * c + i] * ag) * (uv[16 * c + i] * au);
-                        const uint32_t sf = requant_block16(a, p.out_global, codes[2 * c], codes[2 * c + 1]);
-                        sfw |= sf << (8 * c);
+                            for (int i = 0; i < 16; ++i) a[i] = silu_fast(gv[16 * c + i] * ag) * (uv[16 * c + i] * au);
+                            const uint32_t sf = requant_block16(a, p.out_global, codes[2 * c], codes[2 * c + 1]);
+                            sfw |= sf << (8 * c);
+                        }
+                        *reinterpret_cast<uint4*>(p.out_codes + row * (p.out_k / 2) + i0 / 2) =
+                            make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                        // the 2 block scales of this row are 2 consecutive bytes of one atom row
+                        *reinterpret_cast<uint16_t*>(p.out_sf + sf_atom_offset(row, i0 / 16, nkb)) = (uint16_t)sfw;
+                    } else {
+                        // the warp's 32 intermediates are one MXFP8 block of this row
+                        float a[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) a[i] = silu_fast(gv[i] * ag) * (uv[i] * au);
+                        uint32_t w[8];
+                        const uint32_t sf = quantize_block32_mx8(a, w);
+                        uint4* dst = reinterpret_cast<uint4*>(p.out_codes + row * p.out_k + i0);
+                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                        p.out_sf[sf_atom_offset(row, i0 / 32, p.out_k / 32)] = (uint8_t)sf;
                     }
-                    *reinterpret_cast<uint4*>(p.out_codes + row * (p.out_k / 2) + i0 / 2) =
-                        make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                    // the 2 block scales of this row are 2 consecutive bytes of one atom row
-                    *reinterpret_cast<uint16_t*>(p.out_sf + sf_atom_offset(row, i0 / 16, nkb)) = (uint16_t)sfw;
                 }
             } else {
-                // y = acc * global * routing weight, staged as FP16 with one power-of-two
-                // scale per (row, 64 columns).  The warp's 64 accumulator columns are
-                // read and released first; then the max picks the scale and y / scale
-                // is converted (exact power-of-two scaling, one FP16 rounding).
+                // y = acc * global * routing weight.  W4A4: staged as FP16 with one
+                // power-of-two scale per (row, 64 columns): the warp's 64 accumulator
+                // columns are read and released first; then the max picks the scale and
+                // y / scale is converted (exact power-of-two scaling, one FP16 rounding).
+                // W4A8: staged as FP32 (its MXFP8 activations carry outliers unclipped,
+                // so a row's values can sit far above the layer's rms, where an FP16
+                // rounding would exceed the output tolerance).
                 float v[64];
                 const uint32_t t_col = t_row + quarter * 64;
 #pragma unroll
@@ -388,51 +505,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 if (lane == 0) tc::mbar_arrive_remote_relaxed(acc_empty_leader);
                 // rows past the tile's valid count hold padding: weight 0, never stored
                 const float f = valid ? p.globals[ti.x * 3 + 2] * p.act_global * p.wts[p.pair_of_row[row]] : 0.0f;
-                float amax = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
-                amax *= fabsf(f);
-                // scale = 2^(e - 14) with amax in [2^e, 2^(e+1)): staged magnitudes stay below 2^15
-                int e = 0;
-                if (amax > 0.0f && isfinite(amax)) e = ((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-                e = max(min(e - 14, 100), -100);
-                const float g = ldexpf(f, -e);
-                // pk: this row's 64 FP16 values as 8 chunks of 16 bytes (4 words each)
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    __half2 b = __floats2half2_rn(v[2 * i] * g, v[2 * i + 1] * g);
-                    pk[i] = *reinterpret_cast<uint32_t*>(&b);
-                }
-                if (valid) p.y_scale[row * (p.ldy / 64) + n * 4 + quarter] = ldexpf(1.0f, e);
-                // Transpose the 8 x 8 chunk matrix of each group of 8 lanes (rows), a
-                // butterfly over lane bits 1, 2, 4: afterwards lane 8G + c holds chunk c
-                // of the group's rows 8G + 0..7, so one store instruction writes 4 whole
-                // 128-byte row segments instead of 32 scattered 16-byte pieces.
                 const int c8 = lane & 7, g8 = lane >> 3;
+                if (KIND == KIND_MXF8) {
 #pragma unroll
-                for (int b = 0; b < 3; ++b) {
-                    const int m = 1 << b;
-                    const bool hi = (c8 & m) != 0;
+                    for (int i = 0; i < 64; ++i) v[i] *= f;
 #pragma unroll
-                    for (int k0 = 0; k0 < 8; ++k0) {
-                        if (k0 & m) continue;
-                        const int k1 = k0 | m;
+                    for (int h = 0; h < 2; ++h) {
+                        float* pk = v + 32 * h;  // 8 chunks of 4 values, transposed in place
+                        transpose_chunks8(pk, lane);
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const uint32_t send = hi ? pk[4 * k0 + w] : pk[4 * k1 + w];
-                            const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
-                            if (hi) pk[4 * k0 + w] = recv;
-                            else pk[4 * k1 + w] = recv;
+                        for (int j = 0; j < 8; ++j) {
+                            const int r_j = q * 32 + g8 * 8 + j;
+                            if (r_j < n_valid)
+                                *reinterpret_cast<float4*>(p.Yf + (row0 + r_j) * p.ldy + (int64_t)n * BN +
+                                                           quarter * 64 + h * 32 + c8 * 4) =
+                                    make_float4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
                         }
                     }
-                }
+                } else {
+                    float amax = 0.0f;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int r_j = q * 32 + g8 * 8 + j;
-                    if (r_j < n_valid)
-                        *reinterpret_cast<uint4*>(p.Y + (row0 + r_j) * p.ldy + (int64_t)n * BN + quarter * 64 +
-                                                  c8 * 8) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(v[i]));
+                    amax *= fabsf(f);
+                    // scale = 2^(e - 14) with amax in [2^e, 2^(e+1)): staged magnitudes stay below 2^15
+                    int e = 0;
+                    if (amax > 0.0f && isfinite(amax)) e = ((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+                    e = max(min(e - 14, 100), -100);
+                    const float g = ldexpf(f, -e);
+                    // pk: this row's 64 FP16 values as 8 chunks of 16 bytes (4 words each)
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        __half2 b = __floats2half2_rn(v[2 * i] * g, v[2 * i + 1] * g);
+                        pk[i] = *reinterpret_cast<uint32_t*>(&b);
+                    }
+                    if (valid) p.y_scale[row * (p.ldy / 64) + n * 4 + quarter] = ldexpf(1.0f, e);
+                    transpose_chunks8(pk, lane);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int r_j = q * 32 + g8 * 8 + j;
+                        if (r_j < n_valid)
+                            *reinterpret_cast<uint4*>(p.Y + (row0 + r_j) * p.ldy + (int64_t)n * BN + quarter * 64 +
+                                                      c8 * 8) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2],
+                                                                           pk[4 * j + 3]);
+                    }
                 }
             }
         }
@@ -489,6 +605,53 @@ __global__ void k_w4_pack_sf(const uint8_t* __restrict__ src0, const uint8_t* __
     dst[off] = src[srow * nkb + kb];
 }
 
+// W4A8 weights: codes in the padded form the FP8 x FP4 MMA reads (each 8 bytes
+// of 16 codes followed by 8 zero bytes), rows interleaved as above.  One thread
+// per 8 source bytes.
+__global__ void k_w8_pack_codes(const uint8_t* __restrict__ src0, const uint8_t* __restrict__ src1, int64_t rows,
+                                int64_t row_bytes, int interleave, int64_t rows_per_expert_src,
+                                uint8_t* __restrict__ dst) {
+    const int64_t per_row = row_bytes / 8;
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= rows * per_row) return;
+    const int64_t prow = idx / per_row, v = idx - prow * per_row;
+    const uint8_t* src = src0;
+    int64_t srow = prow;
+    if (interleave) {
+        const int64_t per_e = 2 * rows_per_expert_src;
+        const int64_t e = prow / per_e, p = prow - e * per_e;
+        const int64_t b = p / 256, w = p % 256;
+        src = w < 128 ? src0 : src1;
+        srow = e * rows_per_expert_src + b * 128 + (w & 127);
+    }
+    const uint2 c = reinterpret_cast<const uint2*>(src + srow * row_bytes)[v];
+    reinterpret_cast<uint4*>(dst)[idx] = make_uint4(c.x, c.y, 0u, 0u);
+}
+
+// W4A8 weight scales: the E8M0 scale per 32 of each block whose two E4M3 scales
+// are one power of two 2^e (byte e + 127); a zero-scale block (all codes +-0)
+// takes 2^0.  Rows without that form are counted by the compact-form check
+// before this runs.  Atom layout with K/32 columns.
+__global__ void k_w8_pack_sf(const uint8_t* __restrict__ src0, const uint8_t* __restrict__ src1, int64_t rows,
+                             int64_t nkb32, int interleave, int64_t rows_per_expert_src, uint8_t* __restrict__ dst) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= rows * nkb32) return;
+    const int64_t prow = idx / nkb32, kb = idx - prow * nkb32;
+    const uint8_t* src = src0;
+    int64_t srow = prow;
+    if (interleave) {
+        const int64_t per_e = 2 * rows_per_expert_src;
+        const int64_t e = prow / per_e, p = prow - e * per_e;
+        const int64_t b = p / 256, w = p % 256;
+        src = w < 128 ? src0 : src1;
+        srow = e * rows_per_expert_src + b * 128 + (w & 127);
+    }
+    const uint8_t* s = src + srow * (2 * nkb32) + 2 * kb;
+    int e = 0;
+    const int kind = compact_block_kind(s[0], s[1], e);
+    dst[sf_atom_offset(prow, kb, nkb32)] = (uint8_t)(kind == 0 ? e + 127 : 127);
+}
+
 // ---------------------------------------------------------------------------
 // host: tensor maps and launches
 // ---------------------------------------------------------------------------
@@ -527,8 +690,10 @@ bool make_map(CUtensorMap* m, const void* base, int64_t row_bytes, int64_t rows,
     return true;
 }
 
-// CTA pairs that fit on the device at once (1 CTA per SM), per device, cached.
+// CTA pairs that fit on the device at once (1 CTA per SM), per device and kind, cached.
+template <int KIND>
 int max_resident_pairs() {
+    constexpr int SMEM_BYTES = smem_bytes<KIND>();
     static std::mutex mu;
     static int cache[64] = {};
     int dev = 0;
@@ -538,7 +703,8 @@ int max_resident_pairs() {
     }
     std::lock_guard<std::mutex> lk(mu);
     if (cache[dev] == 0) {
-        if (cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+        if (cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM_BYTES) !=
             cudaSuccess) {
             set_error("w4a4: cannot raise the shared-memory limit to %d bytes", SMEM_BYTES);
             return 0;
@@ -548,7 +714,7 @@ int max_resident_pairs() {
         cfg.blockDim = dim3(THREADS, 1, 1);
         cfg.dynamicSmemBytes = SMEM_BYTES;
         int n = 0;
-        const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, k_w4a4_gemm<EPI_GATEUP>, &cfg);
+        const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, k_w4a4_gemm<EPI_GATEUP, KIND>, &cfg);
         if (e != cudaSuccess || n <= 0) {
             (void)cudaGetLastError();
             n = num_sms() / 2;  // one CTA per SM, two SMs per pair
@@ -560,13 +726,48 @@ int max_resident_pairs() {
 
 }  // namespace
 
-size_t w4a4_packed_size(int E, int H, int I) { return (size_t)w4_layout(E, H, I).total; }
+size_t w4a4_packed_size(int E, int H, int I, bool mx8) { return (size_t)w4_layout(E, H, I, mx8).total; }
 
-nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed, cudaStream_t stream) {
+nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed, bool mx8, cudaStream_t stream) {
     const int E = w.E, H = w.H, I = w.I;
-    const W4Layout L = w4_layout(E, H, I);
+    const W4Layout L = w4_layout(E, H, I, mx8);
     uint8_t* p = static_cast<uint8_t*>(packed);
     const int64_t gu_rows = (int64_t)E * 2 * I, d_rows = (int64_t)E * H;
+    if (mx8) {
+        // the E8M0 form needs every weight row's scale pairs to be one power of two
+        int32_t* n_bad = reinterpret_cast<int32_t*>(p + L.status);
+        NVFP4MOE_CUDA(cudaMemsetAsync(n_bad, 0, sizeof(int32_t), stream));
+        const nvfp4moe_status st[3] = {
+            launch_compact_rows(w.gate_codes, w.gate_sf, (int64_t)E * I, H, nullptr, nullptr, nullptr, n_bad, stream,
+                                1 << 20),
+            launch_compact_rows(w.up_codes, w.up_sf, (int64_t)E * I, H, nullptr, nullptr, nullptr, n_bad, stream,
+                                1 << 20),
+            launch_compact_rows(w.down_codes, w.down_sf, d_rows, I, nullptr, nullptr, nullptr, n_bad, stream,
+                                1 << 20)};
+        for (nvfp4moe_status x : st)
+            if (x != NVFP4MOE_OK) return x;
+        k_w8_pack_codes<<<(unsigned)ceil_div(gu_rows * (H / 16), 256), 256, 0, stream>>>(
+            w.gate_codes, w.up_codes, gu_rows, H / 2, 1, I, p + L.gu_codes);
+        k_w8_pack_sf<<<(unsigned)ceil_div(gu_rows * (H / 32), 256), 256, 0, stream>>>(w.gate_sf, w.up_sf, gu_rows,
+                                                                                       H / 32, 1, I, p + L.gu_sf);
+        k_w8_pack_codes<<<(unsigned)ceil_div(d_rows * (I / 16), 256), 256, 0, stream>>>(w.down_codes, nullptr, d_rows,
+                                                                                         I / 2, 0, H, p + L.d_codes);
+        k_w8_pack_sf<<<(unsigned)ceil_div(d_rows * (I / 32), 256), 256, 0, stream>>>(w.down_sf, nullptr, d_rows, I / 32,
+                                                                                       0, H, p + L.d_sf);
+        NVFP4MOE_CHECK_LAUNCH("w4a8 pack");
+        NVFP4MOE_CUDA(cudaMemcpyAsync(p + L.globals, w.w_global, (size_t)E * 3 * sizeof(float),
+                                      cudaMemcpyDeviceToDevice, stream));
+        int32_t bad = 0;
+        NVFP4MOE_CUDA(cudaMemcpyAsync(&bad, n_bad, sizeof(bad), cudaMemcpyDeviceToHost, stream));
+        NVFP4MOE_CUDA(cudaStreamSynchronize(stream));
+        if (bad != 0) {
+            set_error("moe_pack_weights: %d weight rows have no E8M0 scale form (the two E4M3 scales of a 32-code "
+                      "block must be one power of two, or zero over zero codes)",
+                      bad);
+            return NVFP4MOE_ERR_NOT_REPRESENTABLE;
+        }
+        return NVFP4MOE_OK;
+    }
     k_w4_pack_codes<<<(unsigned)ceil_div(gu_rows * (H / 32), 256), 256, 0, stream>>>(
         w.gate_codes, w.up_codes, gu_rows, H / 2, 1, I, p + L.gu_codes);
     k_w4_pack_sf<<<(unsigned)ceil_div(gu_rows * (H / 16), 256), 256, 0, stream>>>(w.gate_sf, w.up_sf, gu_rows, H / 16,
@@ -581,23 +782,26 @@ nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed,
     return NVFP4MOE_OK;
 }
 
-nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E, int k, float act_global_in,
-                                  float act_global_mid, int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
-                                  const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, __half* Y, float* y_scale,
-                                  cudaStream_t stream, cudaEvent_t mid_event) {
-    (void)T;
-    (void)k;
-    const W4Layout L = w4_layout(E, H, I);
+template <int KIND>
+static nvfp4moe_status run_layer(const void* packed, int H, int I, int E, float act_global_in, float act_global_mid,
+                                 int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
+                                 const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, __half* Y, float* y_scale,
+                                 cudaStream_t stream, cudaEvent_t mid_event) {
+    constexpr bool MX8 = KIND == KIND_MXF8;
+    constexpr int SMEM_BYTES = smem_bytes<KIND>();
+    const W4Layout L = w4_layout(E, H, I, MX8);
     const uint8_t* pk = static_cast<const uint8_t*>(packed);
     NVFP4MOE_CUDA(
-        cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w4a4_gemm<EPI_DOWN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+        cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    NVFP4MOE_CUDA(
+        cudaFuncSetAttribute(k_w4a4_gemm<EPI_DOWN, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    // operand rows in bytes: FP4 two codes per byte; FP8 and padded FP4 one element per byte
+    const int64_t hb = MX8 ? H : H / 2, ib = MX8 ? I : I / 2;
     CUtensorMap mA1, mGU, mA2, mD;
-    if (!make_map(&mA1, A1c, H / 2, rows_max, BM) ||
-        !make_map(&mGU, pk + L.gu_codes, H / 2, (int64_t)E * 2 * I, BN / 2) ||
-        !make_map(&mA2, A2c, I / 2, rows_max, BM) || !make_map(&mD, pk + L.d_codes, I / 2, (int64_t)E * H, BN / 2))
+    if (!make_map(&mA1, A1c, hb, rows_max, BM) || !make_map(&mGU, pk + L.gu_codes, hb, (int64_t)E * 2 * I, BN / 2) ||
+        !make_map(&mA2, A2c, ib, rows_max, BM) || !make_map(&mD, pk + L.d_codes, ib, (int64_t)E * H, BN / 2))
         return NVFP4MOE_ERR_CUDA;
-    const int pairs = max_resident_pairs();
+    const int pairs = max_resident_pairs<KIND>();
     if (pairs <= 0) return NVFP4MOE_ERR_CUDA;
     GemmParams g{};
     g.tiles = plan.tiles;
@@ -607,8 +811,9 @@ nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E
     g.wts = plan.wts;
     g.pair_of_row = plan.pair_of_row;
     // gate/up + SwiGLU + requantise: inputs carry act_global_in, the intermediate act_global_mid
-    g.act_global = act_global_in;
-    g.out_global = act_global_mid;
+    // (MXFP8 activations carry their own power-of-two scales: no global)
+    g.act_global = MX8 ? 1.0f : act_global_in;
+    g.out_global = MX8 ? 1.0f : act_global_mid;
     g.K = H;
     g.n_ntiles = (2 * I) / BN;
     g.b_rows_per_expert = 2 * I;
@@ -619,26 +824,39 @@ nvfp4moe_status launch_w4a4_layer(const void* packed, int T, int H, int I, int E
     g.out_k = I;
     {
         const int grid = 2 * (int)std::min<int64_t>(pairs, (int64_t)max_tiles * g.n_ntiles);
-        k_w4a4_gemm<EPI_GATEUP><<<grid, THREADS, SMEM_BYTES, stream>>>(mA1, mGU, g);
-        NVFP4MOE_CHECK_LAUNCH("w4a4 gate/up kernel");
+        k_w4a4_gemm<EPI_GATEUP, KIND><<<grid, THREADS, SMEM_BYTES, stream>>>(mA1, mGU, g);
+        NVFP4MOE_CHECK_LAUNCH(MX8 ? "w4a8 gate/up kernel" : "w4a4 gate/up kernel");
     }
     if (mid_event) cudaEventRecord(mid_event, stream);
     // down x routing weight
-    g.act_global = act_global_mid;
+    g.act_global = MX8 ? 1.0f : act_global_mid;
     g.K = I;
     g.n_ntiles = H / BN;
     g.b_rows_per_expert = H;
     g.sfa = A2s;
     g.sfb = pk + L.d_sf;
     g.Y = Y;
+    g.Yf = reinterpret_cast<float*>(Y);  // W4A8 stages FP32 rows in the same buffer
     g.y_scale = y_scale;
     g.ldy = H;
     {
         const int grid = 2 * (int)std::min<int64_t>(pairs, (int64_t)max_tiles * g.n_ntiles);
-        k_w4a4_gemm<EPI_DOWN><<<grid, THREADS, SMEM_BYTES, stream>>>(mA2, mD, g);
-        NVFP4MOE_CHECK_LAUNCH("w4a4 down kernel");
+        k_w4a4_gemm<EPI_DOWN, KIND><<<grid, THREADS, SMEM_BYTES, stream>>>(mA2, mD, g);
+        NVFP4MOE_CHECK_LAUNCH(MX8 ? "w4a8 down kernel" : "w4a4 down kernel");
     }
     return NVFP4MOE_OK;
+}
+
+nvfp4moe_status launch_w4a4_layer(const void* packed, bool mx8, int T, int H, int I, int E, int k,
+                                  float act_global_in, float act_global_mid, int64_t rows_max, int max_tiles,
+                                  const RoutingPlan& plan, const uint8_t* A1c, const uint8_t* A1s, uint8_t* A2c,
+                                  uint8_t* A2s, __half* Y, float* y_scale, cudaStream_t stream, cudaEvent_t mid_event) {
+    (void)T;
+    (void)k;
+    return mx8 ? run_layer<KIND_MXF8>(packed, H, I, E, act_global_in, act_global_mid, rows_max, max_tiles, plan, A1c,
+                                      A1s, A2c, A2s, Y, y_scale, stream, mid_event)
+               : run_layer<KIND_NVF4>(packed, H, I, E, act_global_in, act_global_mid, rows_max, max_tiles, plan, A1c,
+                                      A1s, A2c, A2s, Y, y_scale, stream, mid_event);
 }
 
 }  // namespace nvfp4moe

@@ -29,6 +29,8 @@ keeps 16 experts per group):
                 from the zero-mantissa codes 0x08, 0x10, .., 0x48 (2^-6 .. 2^2),
                 the same byte for both 16-code halves; W4A16 with compact
                 scales.
+* ``prefill_pow2`` as ``prefill`` (outliers included) with the weights of
+                ``decode_pow2``; W4A8 (MXFP8 activations).
 
 Activations are BF16 N(0,1) (drawn in float32, stored as BF16 bit patterns);
 router logits are float32 N(0,1).  Seeds are 1234 + the workload's index.
@@ -52,7 +54,7 @@ class Workload:
     topk_group: int
     top_k: int
     rsf: float
-    mode: int  # 0 = W4A16, 1 = W4A4, 2 = W4A16 with compact scales
+    mode: int  # 0 = W4A16, 1 = W4A4, 2 = W4A16 with compact scales, 3 = W4A8
     weights: str  # "mxfp4_tiny" | "nvfp4" | "nvfp4_pow2"
     outliers: bool = False
     zipf: bool = False
@@ -68,6 +70,8 @@ WORKLOADS = {
     "prefill": Workload("prefill", 3, 8192, 4096, 2048, 256, 8, 4, 8, 2.827, 1, "nvfp4", outliers=True),
     "skewed": Workload("skewed", 4, 65536, 4096, 2048, 128, 8, 4, 8, 2.827, 1, "nvfp4", outliers=True, zipf=True),
     "decode_pow2": Workload("decode_pow2", 5, 16, 4096, 2048, 256, 8, 4, 8, 2.827, 2, "nvfp4_pow2"),
+    "prefill_pow2": Workload("prefill_pow2", 6, 8192, 4096, 2048, 256, 8, 4, 8, 2.827, 3, "nvfp4_pow2",
+                             outliers=True),
 }
 
 TRANSCODE_SEED = 1234 + 1

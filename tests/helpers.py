@@ -132,7 +132,8 @@ def compare_layer(got: np.ndarray, ref: np.ndarray, rel_l2: float = REL_L2, max_
 
 def oracle_layer(mode: int, d: dict, w: dict, wl, tokens=None, act_global: float = 1.0, renormalize: bool = True,
                  act_global_mid: float | None = None):
-    # the compact-scale mode computes W4A16 on the same weight values
+    # the compact-scale mode computes W4A16 on the same weight values; W4A8 is the
+    # oracle's mode 3 (its numbering matches the library's)
     mode = moe.W4A16 if mode == moe.W4A16C else mode
     return oracle.moe_layer(mode, d["x"], d["logits"], None, w["gate_codes"], w["gate_sf"], w["up_codes"], w["up_sf"],
                             w["down_codes"], w["down_sf"], w["w_global"], act_global, wl.n_group, wl.topk_group,

@@ -22,7 +22,7 @@ def declared_functions():
 def test_header_declares_the_hot_path_calls():
     names = declared_functions()
     for n in ("transcode_mxfp4_to_nvfp4", "moe_route", "quantize_nvfp4", "moe_forward", "moe_pack_weights",
-              "moe_permute", "moe_forward_routed", "moe_forward_ex", "nvfp4_compact_scales"):
+              "moe_permute", "moe_forward_routed", "moe_forward_ex", "nvfp4_compact_scales", "quantize_mxfp8"):
         assert n in names
 
 
@@ -45,7 +45,12 @@ def test_version_and_sizes():
     assert compact <= moe.moe_packed_weights_size(moe.W4A16C, E, H, I) <= compact + 2048
     bits = 8 * moe.moe_packed_weights_size(moe.W4A16C, E, H, I) / (E * 3 * I * H)
     assert 4.125 < bits < 4.13
-    assert moe.moe_packed_weights_size(3, E, H, I) == 0  # unknown mode
+    # W4A8: codes one byte per element (padded form) + an E8M0 scale per 32 + globals + a status word
+    w8 = E * (2 * I * H + H * I) + E * (2 * I * H + H * I) // 32 + E * 3 * 4 + 16
+    assert w8 <= moe.moe_packed_weights_size(moe.W4A8, E, H, I) <= w8 + 2048
+    assert moe.moe_packed_weights_size(4, E, H, I) == 0  # unknown mode
+    ws8 = moe.moe_forward_workspace_size(moe.W4A8, 8192, H, I, E, 8)
+    assert ws8 > moe.moe_forward_workspace_size(moe.W4A4, 8192, H, I, E, 8)
     ws = moe.moe_forward_workspace_size(moe.W4A4, 8192, H, I, E, 8)
     assert ws > 8192 * 8 * H * 2  # holds the per-pair BF16 rows at least
     assert moe.moe_forward_workspace_size(moe.W4A4, -1, H, I, E, 8) == 0
@@ -106,7 +111,7 @@ def test_forward_validation():
         return lib.moe_forward(mode, p, p, None, p, 1.0, a["T"], a["H"], a["I"], a["E"], a["ng"], a["tg"], a["k"],
                                2.827, 1, p, ws_bytes, p, 0, None, None, None)
 
-    assert call(mode=3) == 1
+    assert call(mode=4) == 1  # unknown mode
     assert call(H=4000) == 3
     assert call(I=200) == 3
     assert call(ws_bytes=16) == 6
@@ -178,3 +183,14 @@ def test_compact_scales_validation():
     assert lib.nvfp4_compact_scales(p, None, 8, 128, p, p, p, None, None) == 1
     assert lib.nvfp4_compact_scales(p, p, 8, 128, q, p, p, None, None) == 2
     assert lib.nvfp4_compact_scales(None, None, 0, 128, None, None, None, None, None) == 0  # no-op
+
+
+def test_quantize_mxfp8_validation():
+    lib = moe.load()
+    p = ctypes.c_void_p(4096)
+    assert lib.quantize_mxfp8(p, 4, 48, p, p, None) == 3    # K % 32
+    assert lib.quantize_mxfp8(p, -1, 64, p, p, None) == 1
+    assert lib.quantize_mxfp8(p, 4, 16, p, p, None) == 1    # K < 32
+    assert lib.quantize_mxfp8(p, 4, 64, None, p, None) == 1
+    assert lib.quantize_mxfp8(p, 4, 64, ctypes.c_void_p(4104), p, None) == 2
+    assert lib.quantize_mxfp8(None, 0, 64, None, None, None) == 0
