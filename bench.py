@@ -44,7 +44,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill", "skewed", "decode"], default="prefill")
+    ap.add_argument("--workload", choices=["prefill", "skewed", "decode", "decode_pow2", "prefill_pow2"],
+                    default="prefill")
     ap.add_argument("--no-extras", action="store_true", help="skip the decode and transcode sub-measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=0, help="oracle tokens per step (0 = host threads)")
@@ -63,8 +64,15 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
 
 
-# nominal dense FP4 : BF16 tensor-core throughput on B200 (9 : 2.25 PFLOP/s)
+# nominal dense FP4 : BF16 and FP8 : BF16 tensor-core throughput on B200 (9 : 4.5 : 2.25 PFLOP/s)
 FP4_OVER_BF16 = 4.0
+FP8_OVER_BF16 = 2.0
+
+MODE_NAMES = {0: "W4A16", 1: "W4A4", 2: "W4A16 compact scales", 3: "W4A8 (MXFP8 x FP4)"}
+MODE_DTYPES = {0: "bf16 activations x fp4 e2m1 weights (e4m3 block scales), fp16 mma -> f32",
+               1: "fp4 e2m1 (e4m3 block scales) x fp4 -> f32",
+               2: "bf16 activations x fp4 e2m1 weights (compact power-of-two scales), fp16 mma -> f32",
+               3: "fp8 e4m3 (e8m0 block scales) x fp4 e2m1 (e8m0 block scales) -> f32"}
 
 # DRAM bytes (read + write) of one k_w4a4_gemm<gate/up> launch, from ncu
 # (profiles/k_w4a4_gemm_prefill2k_e64.txt: 652.8 MB read + 22.6 MB written at
@@ -322,20 +330,23 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = max_over_ranks(torch, dist, e2e_ms, "cuda")
 
     # ----------------------------------------------------------------- roofline
-    if mode == moe.W4A4:
+    if mode in (moe.W4A4, moe.W4A8):
         flops = 4.0 * T * wl.top_k * wl.H * wl.I  # gate/up GEMM, padding rows excluded
         t_kernel = stage["gateup_gemm"] / 1e3
         achieved = flops / t_kernel / 1e12
         # The GEMM runs inside a long loop of steps and draws the board to its power
         # cap (its SM clock falls to ~1.4-1.6 GHz), so the denominator is the
-        # sustained bf16 figure, scaled to FP4 by the nominal dense ratio.
-        peak = P["bf16_tflops_sustained"] * FP4_OVER_BF16
-        traffic = GATEUP_TRAFFIC_T8192_E256 if (T, wl.E, wl.H, wl.I) == (8192, 256, 4096, 2048) else None
+        # sustained bf16 figure, scaled to FP4 (FP8 for W4A8) by the nominal dense ratio.
+        ratio = FP4_OVER_BF16 if mode == moe.W4A4 else FP8_OVER_BF16
+        peak = P["bf16_tflops_sustained"] * ratio
+        traffic = (GATEUP_TRAFFIC_T8192_E256 if mode == moe.W4A4 and (T, wl.E, wl.H, wl.I) == (8192, 256, 4096, 2048)
+                   else None)
         roofline = {"bound": "tensor", "kernel": "k_w4a4_gemm<gate/up>", "achieved": round(achieved, 1),
                     "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                     "traffic": traffic, "traffic_unit": "bytes per launch (ncu dram read+write)",
-                    "peak_src": f"{P['src']} bf16 sustained x {FP4_OVER_BF16:g} (nominal dense FP4:BF16); "
-                                f"burst would be {P['bf16_tflops'] * FP4_OVER_BF16:.0f}",
+                    "peak_src": f"{P['src']} bf16 sustained x {ratio:g} (nominal dense "
+                                f"{'FP4' if mode == moe.W4A4 else 'FP8'}:BF16); "
+                                f"burst would be {P['bf16_tflops'] * ratio:.0f}",
                     "algorithmic_flops_per_launch": flops}
     else:
         # W4A16 weight stream: every active expert's codes + E4M3 scales read once
@@ -343,7 +354,10 @@ def run_ours(args, rank, world, local_rank):
         w_t = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
         moe.moe_route(logits, None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf, True, ids_t, w_t)
         active = int(torch.unique(ids_t).numel())
-        wbytes = active * (2 * wl.I * wl.H + wl.H * wl.I) * (0.5 + 1.0 / 16)
+        if mode == moe.W4A16C:  # codes + a 4-bit field per 32 weights + an exponent byte per row
+            wbytes = active * ((2 * wl.I * wl.H + wl.H * wl.I) * (0.5 + 1.0 / 64) + (2 * wl.I + wl.H))
+        else:
+            wbytes = active * (2 * wl.I * wl.H + wl.H * wl.I) * (0.5 + 1.0 / 16)
         t_kernel = (stage["gateup_gemm"] + stage["down_gemm"]) / 1e3
         achieved = wbytes / t_kernel / 1e9
         roofline = {"bound": "hbm", "kernel": "k_w16_gateup + k_w16_down", "achieved": round(achieved, 1),
@@ -354,11 +368,11 @@ def run_ours(args, rank, world, local_rank):
     res = {
         "metric": "MoE-layer tokens/s", "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp4 e2m1 (e4m3 block scales) x fp4 -> f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": MODE_DTYPES[mode],
         "data": "synthetic",
         "config": {"workload": f"{wl.name}: T={T} H={wl.H} I={wl.I} E={wl.E} groups={wl.n_group} "
                                f"keep={wl.topk_group} top_k={wl.top_k} rsf={wl.rsf} "
-                               f"{'W4A4' if mode == moe.W4A4 else 'W4A16'}",
+                               f"{MODE_NAMES[mode]}",
                    "global_batch": T * world, "tokens_per_gpu": T, "parallelism": f"replicas{world}",
                    "l2": f"inputs larger than L2 ({moe.moe_packed_weights_size(mode, wl.E, wl.H, wl.I) / 1e9:.2f} GB "
                          f"packed expert weights per step)"},
@@ -377,6 +391,7 @@ def run_ours(args, rank, world, local_rank):
         res["decode"] = bench_decode(torch, moe, w, args, P)
         del w
         res["decode_compact"] = bench_decode(torch, moe, None, args, P, compact=True)
+        res["prefill_w4a8"] = bench_w4a8(torch, moe, args, P)
         res["transcode"] = bench_transcode(torch, moe, args, P)
         res["router"] = bench_router(torch, moe, args, P)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -442,6 +457,39 @@ def bench_decode(torch, moe, w, args, P, compact=False):
             "roofline": {"bound": "hbm", "kernel": "k_w16_gateup + k_w16_down", "achieved": round(achieved, 1),
                          "peak": P["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / P["hbm_gbs"], 4),
                          "traffic": None, "algorithmic_bytes_per_step": int(wbytes)}}
+
+
+def bench_w4a8(torch, moe, args, P):
+    """W4A8 prefill layer (MXFP8 activations x FP4 weights, T=8192) on weights with
+    the transcode's scale structure; the W4A4 layer on the same weights beside it.
+    The FP8 x FP4 MMA runs at the FP8 rate, so the denominator is the FP8 peak."""
+    wl = inputs.WORKLOADS["prefill_pow2"]
+    d = inputs.moe_inputs(wl)
+    w = {k: d[k] for k in ("gate_codes", "gate_sf", "up_codes", "up_sf", "down_codes", "down_sf", "w_global")}
+    xd = torch.from_numpy(d["x"].view(np.int16)).cuda().view(torch.bfloat16)
+    ld = torch.from_numpy(d["logits"]).cuda()
+    del d
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    packed, ws = make_layer(torch, moe, moe.W4A4, w, wl.T, wl)
+    ms4, _ = time_layer(torch, moe, moe.W4A4, packed, ws, xd, ld, out, wl, wl.T, args.steps, args.warmup, trace=False)
+    del packed, ws
+    torch.cuda.empty_cache()
+    packed, ws = make_layer(torch, moe, moe.W4A8, w, wl.T, wl)
+    del w
+    ms, stage = time_layer(torch, moe, moe.W4A8, packed, ws, xd, ld, out, wl, wl.T, args.steps, args.warmup)
+    del packed, ws
+    torch.cuda.empty_cache()
+    flops = 4.0 * wl.T * wl.top_k * wl.H * wl.I
+    achieved = flops / (stage["gateup_gemm"] / 1e3) / 1e12
+    peak = P["bf16_tflops_sustained"] * FP8_OVER_BF16
+    return {"workload": f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top_k={wl.top_k} W4A8 (MXFP8 x FP4)",
+            "value": round(wl.T / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+            "stages_ms": {k: round(v, 4) for k, v in stage.items()},
+            "same_weights": {"mode": "W4A4", "ms_per_step": round(ms4, 4)},
+            "roofline": {"bound": "tensor", "kernel": "k_w4a4_gemm<gate/up, FP8 x FP4>", "achieved": round(achieved, 1),
+                         "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                         "peak_src": f"{P['src']} bf16 sustained x {FP8_OVER_BF16:g} (nominal dense FP8:BF16)",
+                         "algorithmic_flops_per_launch": flops}}
 
 
 def bench_router(torch, moe, args, P):

@@ -36,28 +36,34 @@ namespace {
 
 constexpr int W16_WARPS = 4;
 constexpr int W16_MAX_NT = 2;  // n-tiles (of 8 tokens) per pass over the weights
-constexpr int W16_MIN_CTAS = 5;  // CTAs per SM the register budget is sized for
 
 // Scale bytes per 16-row tile and 64-column chunk: 64 E4M3 bytes, or 16 bytes
 // of 4-bit compact fields (one byte per row).
 __host__ __device__ constexpr int w16_chunk_scale_bytes(bool compact) { return compact ? 16 : 64; }
+// 64-column chunks per streamed group: 4 when H and I allow it (fewer, larger
+// copies: the copy count, not the bytes, limited the stream with 2), else 2.
+inline int w16_ch(int H, int I) { return (H % 256 == 0 && I % 256 == 0) ? 4 : 2; }
+// Bytes of one 16-row tile's group of CH chunks: the codes, then the scales,
+// contiguous, so that one bulk copy moves both.
+__host__ __device__ constexpr int w16_group_bytes(bool compact, int CH) {
+    return CH * 512 + CH * w16_chunk_scale_bytes(compact);
+}
 
 struct W16Layout {
-    int64_t gu_codes, gu_scales, d_codes, d_scales, globals;
+    int64_t gu, d, globals;                  // gate/up and down tiles (codes + scales per group)
     int64_t rexp_g, rexp_u, rexp_d, status;  // compact form only: row exponents [E, I], [E, I], [E, H]; failures
     int64_t total;
 };
 
 __host__ __device__ inline int64_t align256(int64_t v) { return (v + 255) / 256 * 256; }
 
-__host__ __device__ inline W16Layout w16_layout(int E, int H, int I, bool compact) {
-    const int64_t per64 = w16_chunk_scale_bytes(compact) / 16;  // scale bytes per row per 64 columns
+inline W16Layout w16_layout(int E, int H, int I, bool compact) {
+    const int ch = w16_ch(H, I);
+    const int64_t gb = w16_group_bytes(compact, ch);
     W16Layout L;
-    L.gu_codes = 0;
-    L.gu_scales = align256(L.gu_codes + (int64_t)E * I * H);
-    L.d_codes = align256(L.gu_scales + (int64_t)E * 2 * I * (H / 64) * per64);
-    L.d_scales = align256(L.d_codes + (int64_t)E * H * I / 2);
-    L.globals = align256(L.d_scales + (int64_t)E * H * (I / 64) * per64);
+    L.gu = 0;
+    L.d = align256(L.gu + (int64_t)E * (2 * I / 16) * (H / (64 * ch)) * gb);
+    L.globals = align256(L.d + (int64_t)E * (H / 16) * (I / (64 * ch)) * gb);
     int64_t end = L.globals + (int64_t)E * 3 * 4;
     L.rexp_g = L.rexp_u = L.rexp_d = L.status = -1;
     if (compact) {
@@ -74,15 +80,28 @@ __host__ __device__ inline W16Layout w16_layout(int E, int H, int I, bool compac
 // 2^k as FP32 for k in [-126, 127]
 __device__ __forceinline__ float pow2f(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
 
+// A row exponent, loaded where it is written in the code: issued before the
+// weight stream so that its latency is not paid in the epilogue.
+__device__ __forceinline__ int ld_rexp(const int8_t* p) {
+    int v;
+    asm volatile("ld.global.nc.s8 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 // ---------------------------------------------------------------------------
 // pack: per 16-row tile and 64-column chunk, 512 bytes in fragment order (lane
 // l holds 16 bytes: one 32-bit word per k16 step); inside a word byte j holds
 // the two consecutive-column codes of A-fragment register j (low nibble = even
 // column): j=0 row g cols 2c,2c+1; j=1 row g+8; j=2 row g cols 2c+8,2c+9; j=3
 // row g+8.  Scales: 64 bytes per chunk, 8 per row pair g: [s(g,k16 step t),
-// s(g+8,t)] for t = 0..3.  Compact form: 16 bytes per chunk, byte 2g for row g
-// and 2g+1 for row g+8, each holding the 4-bit fields of the chunk's two
-// 32-column blocks (low nibble first); the row exponents stay in row order.
+// s(g+8,t)] for t = 0..3.  Compact form: 32 bytes per pair of chunks, one word
+// per row pair g whose byte p (chunk 2j + p) holds row g's two 4-bit fields
+// (the chunk's 32-column blocks, low nibble first) and byte 2 + p row g + 8's,
+// so a shift and a mask put row g's field in the low half and row g + 8's in
+// the high half; the row exponents stay in row order.  A tile's chunks are
+// stored in groups of two, codes then scales, and the groups of a tile pair
+// (gate and up of 16 intermediates, or two 16-row down tiles) alternate, so one
+// copy moves both tiles' group.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t code_at(const uint8_t* codes, int64_t r, int64_t k, int64_t K) {
     const uint32_t b = codes[r * (K / 2) + k / 2];
@@ -102,12 +121,11 @@ __device__ uint32_t pack_word(const uint8_t* codes, int64_t r0, int64_t kb, int 
 // One thread per (tile, k64 chunk, lane): 16 code bytes, plus the scale bytes
 // of rows g, g + 8 for lanes with c == 0.  rexp/rexp2: row exponents of the
 // compact form (COMPACT only).
-template <bool COMPACT>
+template <bool COMPACT, int CH>
 __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sf, int64_t n_tiles,
                            int64_t K, int interleave_gu, const uint8_t* __restrict__ codes2,
-                           const uint8_t* __restrict__ sf2, uint8_t* __restrict__ out_codes,
-                           uint8_t* __restrict__ out_scales, int64_t rows_per_expert, const int8_t* __restrict__ rexp,
-                           const int8_t* __restrict__ rexp2) {
+                           const uint8_t* __restrict__ sf2, uint8_t* __restrict__ out, int64_t rows_per_expert,
+                           const int8_t* __restrict__ rexp, const int8_t* __restrict__ rexp2) {
     const int64_t chunks = K / 64;
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= n_tiles * chunks * 32) return;
@@ -136,7 +154,13 @@ __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __r
     uint32_t w[4];
 #pragma unroll
     for (int st = 0; st < 4; ++st) w[st] = pack_word(c, r0, chunk * 64 + st * 16, g, cc, K);
-    *reinterpret_cast<uint4*>(out_codes + (tile * chunks + chunk) * 512 + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    // this chunk's place: tiles are stored in pairs (the two a warp streams together),
+    // group by group, the pair's two groups adjacent; in a group the codes at
+    // (chunk % CH) * 512, the scales after the codes
+    constexpr int GB = w16_group_bytes(COMPACT, CH);
+    uint8_t* grp = out + ((tile >> 1) * (chunks / CH) + chunk / CH) * 2 * GB + (tile & 1) * GB;
+    const int sub = (int)(chunk % CH);
+    *reinterpret_cast<uint4*>(grp + sub * 512 + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
     if (COMPACT && cc == 0) {
         uint32_t v = 0;
 #pragma unroll
@@ -153,7 +177,11 @@ __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __r
             }
             v |= byte << (8 * h);
         }
-        *reinterpret_cast<uint16_t*>(out_scales + (tile * chunks + chunk) * 16 + g * 2) = (uint16_t)v;
+        // one 32-bit word per row pair g and chunk pair: byte (sub & 1) for row g, byte
+        // 2 + (sub & 1) for row g + 8
+        uint8_t* wd = grp + CH * 512 + (sub >> 1) * 32 + g * 4 + (sub & 1);
+        wd[0] = (uint8_t)(v & 0xFFu);
+        wd[2] = (uint8_t)(v >> 8);
     } else if (!COMPACT && cc == 0) {
         uint32_t b[8];
 #pragma unroll
@@ -165,7 +193,7 @@ __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __r
         uint2 v;
         v.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
         v.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
-        *reinterpret_cast<uint2*>(out_scales + (tile * chunks + chunk) * 64 + g * 8) = v;
+        *reinterpret_cast<uint2*>(grp + CH * 512 + sub * 64 + g * 8) = v;
     }
 }
 
@@ -228,11 +256,11 @@ __device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
     return d;
 }
 
-// Two E4M3 scales (bytes lo, hi of `pair`) -> FP16x2 (exact).
-__device__ __forceinline__ uint32_t scales_f16x2(uint32_t pair) {
-    uint32_t h;
-    asm("{\n\t.reg .b16 t;\n\tmov.b16 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "h"((uint16_t)pair));
-    return h;
+// Four E4M3 scales (bytes 0..3 of `w`) -> two FP16x2 (exact): bytes 0, 1 and 2, 3.
+__device__ __forceinline__ void scales_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 // 8 codes of one k16 step -> the four FP16x2 A-fragment registers, scaled by
@@ -246,11 +274,39 @@ __device__ __forceinline__ void dequant_step(uint32_t q, uint32_t m, uint32_t a[
         "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
         : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
         : "r"(q));
-    const uint32_t dg = __byte_perm(m, m, 0x1010), dg8 = __byte_perm(m, m, 0x3232);
-    a[0] = f16x2_mul(a[0], dg);
-    a[1] = f16x2_mul(a[1], dg8);
-    a[2] = f16x2_mul(a[2], dg);
-    a[3] = f16x2_mul(a[3], dg8);
+    // each scale broadcast to both halves: as half2 operations, which the multiply
+    // can take as an operand swizzle instead of a separate byte permute
+    __half2 mh;
+    memcpy(&mh, &m, 4);
+    const __half2 dg = __low2half2(mh), dg8 = __high2half2(mh);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __half2 v;
+        memcpy(&v, &a[i], 4);
+        v = __hmul2(v, (i & 1) ? dg8 : dg);
+        memcpy(&a[i], &v, 4);
+    }
+}
+
+// 8 codes of one k16 step -> the four FP16x2 A-fragment registers, unscaled.
+__device__ __forceinline__ void codes_step(uint32_t q, uint32_t a[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+        : "r"(q));
+}
+
+// d = A B (no accumulator input)
+__device__ __forceinline__ void mma_f16_first(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
 __device__ __forceinline__ void mma_f16(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
@@ -264,120 +320,162 @@ __device__ __forceinline__ void mma_f16(float d[4], const uint32_t a[4], uint32_
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
 // ---------------------------------------------------------------------------
-// Weight streaming: every warp owns a ring of W16_STAGES shared-memory stages;
+// Weight streaming: every warp owns a ring of STAGES shared-memory stages;
 // lane 0 fills a stage with 1-D bulk copies (cp.async.bulk, completion counted
-// on the stage's mbarrier) W16_STAGES groups ahead of the consumer, so the
+// on the stage's mbarrier) STAGES groups ahead of the consumer, so the
 // weight stream stays in flight without occupying registers.  A stage holds
-// W16_CH consecutive 64-column chunks of both 16-row tiles of the warp.
+// CH consecutive 64-column chunks of both 16-row tiles of the warp.
 // ---------------------------------------------------------------------------
-constexpr int W16_STAGES = 4;
-constexpr int W16_CH = 2;
-constexpr int W16_STAGE_CODES = 2 * W16_CH * 512;
-__host__ __device__ constexpr int w16_stage_scales(bool compact) { return 2 * W16_CH * w16_chunk_scale_bytes(compact); }
-constexpr int W16_STAGE = W16_STAGE_CODES + w16_stage_scales(false);  // stage stride (the larger form)
-constexpr int W16_WARP_SMEM = W16_STAGES * W16_STAGE;
-constexpr int W16_SMEM = W16_WARPS * (W16_WARP_SMEM + W16_STAGES * 8);
+template <int CH>
+struct W16Cfg {
+    static constexpr int STAGES = CH == 4 ? 3 : 4;
+    static constexpr int MIN_CTAS = CH == 4 ? 4 : 5;       // CTAs per SM the register budget is sized for
+    static constexpr int STAGE = 2 * w16_group_bytes(false, CH);  // stage stride (the larger form)
+    static constexpr int WARP_SMEM = STAGES * STAGE;
+    static constexpr int SMEM = W16_WARPS * (WARP_SMEM + STAGES * 8);
+};
+static_assert(W16Cfg<4>::SMEM * W16Cfg<4>::MIN_CTAS <= 228 * 1024 && W16Cfg<2>::SMEM * W16Cfg<2>::MIN_CTAS <= 228 * 1024,
+              "the rings of the CTAs an SM is sized for must fit its shared memory");
 
 struct Ring {
-    uint8_t* buf;   // W16_STAGES stages
-    uint64_t* bar;  // W16_STAGES mbarriers
+    uint8_t* buf;   // STAGES stages
+    uint64_t* bar;  // STAGES mbarriers
     uint32_t ctr;   // groups consumed so far (stage = ctr % S, parity = ctr / S)
 };
 
-template <bool COMPACT>
-__device__ __forceinline__ void ring_issue(Ring& r, int stage, const uint8_t* const codes[2],
-                                           const uint8_t* const scales[2], int grp) {
-    constexpr int SCB = w16_chunk_scale_bytes(COMPACT);
-    uint8_t* st = r.buf + stage * W16_STAGE;
-    tc::mbar_arrive_expect_tx(&r.bar[stage], W16_STAGE_CODES + w16_stage_scales(COMPACT));
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        tc::bulk_load(st + u * W16_CH * 512, codes[u] + (int64_t)grp * W16_CH * 512, W16_CH * 512, &r.bar[stage]);
-        tc::bulk_load(st + W16_STAGE_CODES + u * W16_CH * SCB, scales[u] + (int64_t)grp * W16_CH * SCB, W16_CH * SCB,
-                      &r.bar[stage]);
-    }
+template <bool COMPACT, int CH>
+__device__ __forceinline__ void ring_issue(Ring& r, int stage, const uint8_t* pair, int grp) {
+    constexpr int GB2 = 2 * w16_group_bytes(COMPACT, CH);
+    uint8_t* st = r.buf + stage * W16Cfg<CH>::STAGE;
+    tc::mbar_arrive_expect_tx(&r.bar[stage], GB2);
+    tc::bulk_load(st, pair + (int64_t)grp * GB2, GB2, &r.bar[stage]);
 }
 
 // Streams `chunks` 64-column chunks of two 16-row tiles and accumulates their
 // products with NT 8-token B tiles (FP16 rows in fragment order; every lane's
 // pointer is valid, lanes past the expert's tokens read a real row and their
 // results are dropped).  Returns false on a timeout.  COMPACT: the scales are
-// 4-bit fields n and each block's FP16 multiplier is 2^(13 - n) (the row
-// factor 2^(r - 13) is applied to the accumulators by the caller): bits
-// (28 - n) << 10, for rows g and g + 8 at once in the two halves of a word.
-template <int NT, bool COMPACT>
-__device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* const codes[2], const uint8_t* const scales[2],
-                                           int chunks, const __half* const bptr[W16_MAX_NT],
+// 4-bit fields n, one per 32 columns; the codes enter the MMA unscaled and each
+// 32-column block's FP32 product is added to the accumulator times 2^(13 - n)
+// (the row factor 2^(r - 13) is applied by the caller).
+template <int NT, bool COMPACT, int CH>
+__device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* pair, int chunks, const __half* const bptr[W16_MAX_NT],
                                            float acc[2][W16_MAX_NT][4], int32_t* err) {
     const int lane = lane_id();
     const int g = lane >> 2, c = lane & 3;
-    const int groups = chunks / W16_CH;
+    constexpr int STAGES = W16Cfg<CH>::STAGES;
+    constexpr int GB = w16_group_bytes(COMPACT, CH);
+    const int groups = chunks / CH;
     const uint32_t base = r.ctr;
     if (lane == 0)
-        for (int i = 0; i < W16_STAGES && i < groups; ++i)
-            ring_issue<COMPACT>(r, (base + i) % W16_STAGES, codes, scales, i);
+        for (int i = 0; i < STAGES && i < groups; ++i) ring_issue<COMPACT, CH>(r, (base + i) % STAGES, pair, i);
     __syncwarp();
     for (int grp = 0; grp < groups; ++grp) {
         const uint32_t n = base + grp;
-        const int stage = n % W16_STAGES;
-        if (!tc::mbar_wait(&r.bar[stage], (n / W16_STAGES) & 1u, err)) return false;
-        const uint8_t* st = r.buf + stage * W16_STAGE;
+        const int stage = n % STAGES;
+        if (!tc::mbar_wait(&r.bar[stage], (n / STAGES) & 1u, err)) return false;
+        const uint8_t* st = r.buf + stage * W16Cfg<CH>::STAGE;
 #pragma unroll
-        for (int cc = 0; cc < W16_CH; ++cc) {
-            uint4 q[2];
-            uint2 sc[2];  // E4M3 pairs of steps 0, 1 (x) and 2, 3 (y), or the compact multipliers
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                q[u] = *reinterpret_cast<const uint4*>(st + u * W16_CH * 512 + cc * 512 + lane * 16);
-                if (COMPACT) {
-                    const uint32_t w =
-                        *reinterpret_cast<const uint16_t*>(st + W16_STAGE_CODES + u * W16_CH * 16 + cc * 16 + g * 2);
-                    const uint32_t t = __byte_perm(w, 0u, 0x4140);  // [row g, 0, row g + 8, 0]
-                    sc[u].x = (0x001C001Cu - (t & 0x000F000Fu)) << 10;         // blocks of steps 0, 1
-                    sc[u].y = (0x001C001Cu - ((t >> 4) & 0x000F000Fu)) << 10;  // steps 2, 3
-                } else {
-                    sc[u] = *reinterpret_cast<const uint2*>(st + W16_STAGE_CODES + u * W16_CH * 64 + cc * 64 + g * 8);
-                }
-            }
+        for (int cc = 0; cc < CH; ++cc) {
             // this lane's B fragments of the chunk: (b0, b1) of step t at 8 t bytes
             const uint2* bp[NT];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
-                bp[nt] = reinterpret_cast<const uint2*>(bptr[nt] + (int64_t)(grp * W16_CH + cc) * 64 + c * 16);
+                bp[nt] = reinterpret_cast<const uint2*>(bptr[nt] + (int64_t)(grp * CH + cc) * 64 + c * 16);
+            uint4 q[2];
 #pragma unroll
-            for (int stp = 0; stp < 4; ++stp) {
-                uint2 bw[NT];
+            for (int u = 0; u < 2; ++u)
+                q[u] = *reinterpret_cast<const uint4*>(st + u * GB + cc * 512 + lane * 16);
+            if (COMPACT) {
+                // One power-of-two scale per 32 columns: the two k16 steps of a block
+                // accumulate unscaled codes into a block product, which joins the
+                // accumulator with one FP32 multiply-add per value:
+                // acc += product * 2^(13 - n) (the row factor 2^(r - 13) is applied
+                // at the end).  FP32 bits of 2^(13 - n): (140 - n) << 23.
+                static_assert(CH % 2 == 0, "a compact scale word covers two chunks");
+                uint32_t sw[2];  // the scale word of this chunk pair, each tile
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) bw[nt] = __ldg(bp[nt] + stp);
+                for (int u = 0; u < 2; ++u)
+                    sw[u] = *reinterpret_cast<const uint32_t*>(st + u * GB + CH * 512 + (cc >> 1) * 32 + g * 4);
+#pragma unroll
+                for (int blk = 0; blk < 2; ++blk) {
+                    float prod[2][NT][4];
+#pragma unroll
+                    for (int s2 = 0; s2 < 2; ++s2) {
+                        const int stp = 2 * blk + s2;
+                        uint2 bw[NT];
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) bw[nt] = __ldg(bp[nt] + stp);
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const uint32_t qw = stp == 0 ? q[u].x : stp == 1 ? q[u].y : stp == 2 ? q[u].z : q[u].w;
+                            uint32_t a[4];
+                            codes_step(qw, a);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) {
+                                if (s2 == 0) mma_f16_first(prod[u][nt], a, bw[nt].x, bw[nt].y);
+                                else mma_f16(prod[u][nt], a, bw[nt].x, bw[nt].y);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const uint32_t nf = sw[u] >> (8 * (cc & 1) + 4 * blk);  // row g's field in bits 0..3, g + 8's in 16..19
+                        const float s_g = __uint_as_float(0x46000000u - (nf & 15u) * 0x00800000u);
+                        const float s_g8 = __uint_as_float(0x46000000u - ((nf >> 16) & 15u) * 0x00800000u);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            acc[u][nt][0] = __fmaf_rn(prod[u][nt][0], s_g, acc[u][nt][0]);
+                            acc[u][nt][1] = __fmaf_rn(prod[u][nt][1], s_g, acc[u][nt][1]);
+                            acc[u][nt][2] = __fmaf_rn(prod[u][nt][2], s_g8, acc[u][nt][2]);
+                            acc[u][nt][3] = __fmaf_rn(prod[u][nt][3], s_g8, acc[u][nt][3]);
+                        }
+                    }
+                }
+            } else {
+                uint32_t m[2][4];  // FP16x2 {scale g, scale g + 8} of each k16 step
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    const uint32_t qw = stp == 0 ? q[u].x : stp == 1 ? q[u].y : stp == 2 ? q[u].z : q[u].w;
-                    const uint32_t sw = stp < 2 ? sc[u].x : sc[u].y;
-                    uint32_t a[4];
-                    dequant_step(qw, COMPACT ? sw : scales_f16x2((stp & 1) ? (sw >> 16) : (sw & 0xFFFFu)), a);
+                    const uint2 sc = *reinterpret_cast<const uint2*>(st + u * GB + CH * 512 + cc * 64 + g * 8);
+                    scales_f16x2x2(sc.x, m[u][0], m[u][1]);
+                    scales_f16x2x2(sc.y, m[u][2], m[u][3]);
+                }
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_f16(acc[u][nt], a, bw[nt].x, bw[nt].y);
+                for (int stp = 0; stp < 4; ++stp) {
+                    uint2 bw[NT];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) bw[nt] = __ldg(bp[nt] + stp);
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const uint32_t qw = stp == 0 ? q[u].x : stp == 1 ? q[u].y : stp == 2 ? q[u].z : q[u].w;
+                        uint32_t a[4];
+                        dequant_step(qw, m[u][stp], a);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_f16(acc[u][nt], a, bw[nt].x, bw[nt].y);
+                    }
                 }
             }
         }
         __syncwarp();  // every lane has read the stage
-        if (lane == 0 && grp + W16_STAGES < groups) {
+        if (lane == 0 && grp + STAGES < groups) {
             tc::fence_proxy_async_smem();
-            ring_issue<COMPACT>(r, stage, codes, scales, grp + W16_STAGES);
+            ring_issue<COMPACT, CH>(r, stage, pair, grp + STAGES);
         }
     }
     r.ctr = base + groups;
     return true;
 }
 
+template <int CH>
 __device__ __forceinline__ Ring make_ring(uint8_t* smem) {
+    constexpr int STAGES = W16Cfg<CH>::STAGES;
     Ring r;
     const int w = warp_id();
-    r.buf = smem + w * W16_WARP_SMEM;
-    r.bar = reinterpret_cast<uint64_t*>(smem + W16_WARPS * W16_WARP_SMEM) + w * W16_STAGES;
+    r.buf = smem + w * W16Cfg<CH>::WARP_SMEM;
+    r.bar = reinterpret_cast<uint64_t*>(smem + W16_WARPS * W16Cfg<CH>::WARP_SMEM) + w * STAGES;
     r.ctr = 0;
     if (lane_id() == 0) {
-        for (int i = 0; i < W16_STAGES; ++i) tc::mbar_init(&r.bar[i], 1);
+        for (int i = 0; i < STAGES; ++i) tc::mbar_init(&r.bar[i], 1);
         tc::fence_mbar_init();
     }
     __syncwarp();
@@ -387,12 +485,12 @@ __device__ __forceinline__ Ring make_ring(uint8_t* smem) {
 // ---------------------------------------------------------------------------
 // gate/up GEMM + SwiGLU: warps loop over (active expert, 16 intermediates)
 // ---------------------------------------------------------------------------
-template <bool COMPACT>
-__global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
+template <bool COMPACT, int CH>
+__global__ void __launch_bounds__(W16_WARPS * 32, W16Cfg<CH>::MIN_CTAS)
     k_w16_gateup(const __half* __restrict__ x16, const float* __restrict__ x_inv, const uint8_t* __restrict__ packed,
                  W16Layout L, int H, int I, int k, RoutingPlan plan, uint16_t* __restrict__ A2, int32_t* err) {
     extern __shared__ __align__(128) uint8_t w16_smem[];
-    Ring ring = make_ring(w16_smem);
+    Ring ring = make_ring<CH>(w16_smem);
     const int lane = lane_id();
     const int g = lane >> 2, c = lane & 3;
     const int iblocks = I / 16;
@@ -413,18 +511,12 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
             const int8_t* ru = reinterpret_cast<const int8_t*>(packed + L.rexp_u);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                ph[0][h] = pow2f(rg[r + 8 * h] - 13);
-                ph[1][h] = pow2f(ru[r + 8 * h] - 13);
+                ph[0][h] = pow2f(ld_rexp(rg + r + 8 * h) - 13);
+                ph[1][h] = pow2f(ld_rexp(ru + r + 8 * h) - 13);
             }
         }
-        const int64_t tile0 = ((int64_t)e * iblocks + ib) * 2;
-        const uint8_t* cb[2];
-        const uint8_t* sb[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            cb[u] = packed + L.gu_codes + (tile0 + u) * chunks * 512;
-            sb[u] = packed + L.gu_scales + (tile0 + u) * chunks * w16_chunk_scale_bytes(COMPACT);
-        }
+        const int64_t pair = (int64_t)e * iblocks + ib;  // tiles 2 pair (gate) and 2 pair + 1 (up)
+        const uint8_t* tb = packed + L.gu + pair * (chunks / CH) * 2 * w16_group_bytes(COMPACT, CH);
         for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
             const int nt_count = min(W16_MAX_NT, (n_e - n0 + 7) / 8);
             const __half* bptr[W16_MAX_NT];
@@ -434,8 +526,8 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
                 bptr[nt] = x16 + (int64_t)(plan.pair_of_row[row0 + (n < n_e ? n : n0)] / k) * H;
             }
             float acc[2][W16_MAX_NT][4] = {};
-            const bool ok = nt_count == 1 ? w16_stream<1, COMPACT>(ring, cb, sb, chunks, bptr, acc, err)
-                                          : w16_stream<2, COMPACT>(ring, cb, sb, chunks, bptr, acc, err);
+            const bool ok = nt_count == 1 ? w16_stream<1, COMPACT, CH>(ring, tb, chunks, bptr, acc, err)
+                                          : w16_stream<2, COMPACT, CH>(ring, tb, chunks, bptr, acc, err);
             if (!ok) return;
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
@@ -462,12 +554,12 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
 // ---------------------------------------------------------------------------
 // down GEMM x routing weight: warps loop over (active expert, 32 hidden rows)
 // ---------------------------------------------------------------------------
-template <bool COMPACT>
-__global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
+template <bool COMPACT, int CH>
+__global__ void __launch_bounds__(W16_WARPS * 32, W16Cfg<CH>::MIN_CTAS)
     k_w16_down(const uint8_t* __restrict__ packed, W16Layout L, int H, int I, RoutingPlan plan,
                const __half* __restrict__ A16, const float* __restrict__ a_inv, float* __restrict__ Y, int32_t* err) {
     extern __shared__ __align__(128) uint8_t w16_smem[];
-    Ring ring = make_ring(w16_smem);
+    Ring ring = make_ring<CH>(w16_smem);
     const int lane = lane_id();
     const int g = lane >> 2, c = lane & 3;
     const int hblocks = H / 32;
@@ -487,16 +579,10 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
 #pragma unroll
             for (int u = 0; u < 2; ++u)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) ph[u][h] = pow2f(rd[u * 16 + 8 * h] - 13);
+                for (int h = 0; h < 2; ++h) ph[u][h] = pow2f(ld_rexp(rd + u * 16 + 8 * h) - 13);
         }
-        const int64_t tile0 = (int64_t)e * (H / 16) + hb * 2;
-        const uint8_t* cb[2];
-        const uint8_t* sb[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            cb[u] = packed + L.d_codes + (tile0 + u) * chunks * 512;
-            sb[u] = packed + L.d_scales + (tile0 + u) * chunks * w16_chunk_scale_bytes(COMPACT);
-        }
+        const int64_t pair = (int64_t)e * (H / 32) + hb;  // 16-row tiles 2 pair, 2 pair + 1
+        const uint8_t* tb = packed + L.d + pair * (chunks / CH) * 2 * w16_group_bytes(COMPACT, CH);
         for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
             const int nt_count = min(W16_MAX_NT, (n_e - n0 + 7) / 8);
             const __half* bptr[W16_MAX_NT];
@@ -506,8 +592,8 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16_MIN_CTAS)
                 bptr[nt] = A16 + (int64_t)(row0 + (n < n_e ? n : n0)) * I;
             }
             float acc[2][W16_MAX_NT][4] = {};
-            const bool ok = nt_count == 1 ? w16_stream<1, COMPACT>(ring, cb, sb, chunks, bptr, acc, err)
-                                          : w16_stream<2, COMPACT>(ring, cb, sb, chunks, bptr, acc, err);
+            const bool ok = nt_count == 1 ? w16_stream<1, COMPACT, CH>(ring, tb, chunks, bptr, acc, err)
+                                          : w16_stream<2, COMPACT, CH>(ring, tb, chunks, bptr, acc, err);
             if (!ok) return;
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
@@ -540,7 +626,7 @@ size_t w4a16_scratch_size(int T, int H, int I, int k) {
                     align256((int64_t)T * k * 4));
 }
 
-template <bool COMPACT>
+template <bool COMPACT, int CH>
 static nvfp4moe_status pack_tiles(const nvfp4moe_expert_weights& w, uint8_t* p, const W16Layout& L,
                                   cudaStream_t stream) {
     const int E = w.E, H = w.H, I = w.I;
@@ -550,15 +636,15 @@ static nvfp4moe_status pack_tiles(const nvfp4moe_expert_weights& w, uint8_t* p, 
     {
         const int64_t n_tiles = (int64_t)E * (I / 16) * 2;
         const int64_t threads = n_tiles * (H / 64) * 32;
-        k_w16_pack<COMPACT><<<(unsigned)ceil_div(threads, 256), 256, 0, stream>>>(
-            w.gate_codes, w.gate_sf, n_tiles, H, 1, w.up_codes, w.up_sf, p + L.gu_codes, p + L.gu_scales, I, rg, ru);
+        k_w16_pack<COMPACT, CH><<<(unsigned)ceil_div(threads, 256), 256, 0, stream>>>(
+            w.gate_codes, w.gate_sf, n_tiles, H, 1, w.up_codes, w.up_sf, p + L.gu, I, rg, ru);
         NVFP4MOE_CHECK_LAUNCH("w4a16 pack (gate/up)");
     }
     {
         const int64_t n_tiles = (int64_t)E * (H / 16);
         const int64_t threads = n_tiles * (I / 64) * 32;
-        k_w16_pack<COMPACT><<<(unsigned)ceil_div(threads, 256), 256, 0, stream>>>(
-            w.down_codes, w.down_sf, n_tiles, I, 0, nullptr, nullptr, p + L.d_codes, p + L.d_scales, H, rd, nullptr);
+        k_w16_pack<COMPACT, CH><<<(unsigned)ceil_div(threads, 256), 256, 0, stream>>>(
+            w.down_codes, w.down_sf, n_tiles, I, 0, nullptr, nullptr, p + L.d, H, rd, nullptr);
         NVFP4MOE_CHECK_LAUNCH("w4a16 pack (down)");
     }
     return NVFP4MOE_OK;
@@ -581,10 +667,12 @@ nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed
             launch_compact_rows(w.down_codes, w.down_sf, (int64_t)E * H, I, rd, nullptr, nullptr, n_bad, stream)};
         for (nvfp4moe_status s : st)
             if (s != NVFP4MOE_OK) return s;
-        const nvfp4moe_status s = pack_tiles<true>(w, p, L, stream);
+        const nvfp4moe_status s =
+            w16_ch(H, I) == 4 ? pack_tiles<true, 4>(w, p, L, stream) : pack_tiles<true, 2>(w, p, L, stream);
         if (s != NVFP4MOE_OK) return s;
     } else {
-        const nvfp4moe_status s = pack_tiles<false>(w, p, L, stream);
+        const nvfp4moe_status s =
+            w16_ch(H, I) == 4 ? pack_tiles<false, 4>(w, p, L, stream) : pack_tiles<false, 2>(w, p, L, stream);
         if (s != NVFP4MOE_OK) return s;
     }
     NVFP4MOE_CUDA(cudaMemcpyAsync(p + L.globals, w.w_global, (size_t)E * 3 * sizeof(float), cudaMemcpyDeviceToDevice,
@@ -603,12 +691,11 @@ nvfp4moe_status launch_w4a16_pack(const nvfp4moe_expert_weights& w, void* packed
     return NVFP4MOE_OK;
 }
 
-nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, bool compact, int T, int H, int I,
-                                   int E, int k, const RoutingPlan& plan, uint16_t* A2, float* Y, void* scratch,
-                                   cudaStream_t stream, cudaEvent_t mid_event) {
-    const W16Layout L = w16_layout(E, H, I, compact);
-    const uint8_t* p = static_cast<const uint8_t*>(packed);
-    uint8_t* sc = static_cast<uint8_t*>(scratch);
+template <bool COMPACT, int CH>
+static nvfp4moe_status run_w16(const uint16_t* x, const uint8_t* p, const W16Layout& L, int T, int H, int I, int E,
+                               int k, const RoutingPlan& plan, uint16_t* A2, float* Y, uint8_t* sc, cudaStream_t stream,
+                               cudaEvent_t mid_event) {
+    constexpr int SMEM = W16Cfg<CH>::SMEM;
     __half* x16 = reinterpret_cast<__half*>(sc);
     float* x_inv = reinterpret_cast<float*>(sc + align256((int64_t)T * H * 2));
     __half* a16 = reinterpret_cast<__half*>(sc + align256((int64_t)T * H * 2) + align256((int64_t)T * 4));
@@ -618,17 +705,16 @@ nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, bool c
     // experts with rows <= min(E, T*k): grids cover that bound; warps loop over
     // the (expert, row block) items the device-side active list holds
     const int64_t max_active = std::min<int64_t>(E, P);
-    const int64_t max_ctas = (int64_t)num_sms() * W16_MIN_CTAS;
+    const int64_t max_ctas = (int64_t)num_sms() * W16Cfg<CH>::MIN_CTAS;
     int32_t* err = device_error_word();
-    auto gateup = compact ? k_w16_gateup<true> : k_w16_gateup<false>;
-    auto down = compact ? k_w16_down<true> : k_w16_down<false>;
-    NVFP4MOE_CUDA(cudaFuncSetAttribute(gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));
-    NVFP4MOE_CUDA(cudaFuncSetAttribute(down, cudaFuncAttributeMaxDynamicSharedMemorySize, W16_SMEM));
+    NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_gateup<COMPACT, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM));
+    NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_down<COMPACT, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM));
     k_rows_to_f16<<<(unsigned)ceil_div(T, 8), 256, 0, stream>>>(x, T, H, x16, x_inv);
     NVFP4MOE_CHECK_LAUNCH("w4a16 activation conversion");
     {
         const int64_t ctas = std::min<int64_t>(ceil_div(max_active * (I / 16), W16_WARPS), max_ctas);
-        gateup<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(x16, x_inv, p, L, H, I, k, plan, A2, err);
+        k_w16_gateup<COMPACT, CH><<<(unsigned)ctas, W16_WARPS * 32, SMEM, stream>>>(x16, x_inv, p, L, H, I, k, plan,
+                                                                                     A2, err);
         NVFP4MOE_CHECK_LAUNCH("w4a16 gate/up kernel");
     }
     if (mid_event) cudaEventRecord(mid_event, stream);
@@ -636,10 +722,24 @@ nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, bool c
     NVFP4MOE_CHECK_LAUNCH("w4a16 intermediate conversion");
     {
         const int64_t ctas = std::min<int64_t>(ceil_div(max_active * (H / 32), W16_WARPS), max_ctas);
-        down<<<(unsigned)ctas, W16_WARPS * 32, W16_SMEM, stream>>>(p, L, H, I, plan, a16, a_inv, Y, err);
+        k_w16_down<COMPACT, CH><<<(unsigned)ctas, W16_WARPS * 32, SMEM, stream>>>(p, L, H, I, plan, a16, a_inv, Y, err);
         NVFP4MOE_CHECK_LAUNCH("w4a16 down kernel");
     }
     return NVFP4MOE_OK;
+}
+
+nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, bool compact, int T, int H, int I,
+                                   int E, int k, const RoutingPlan& plan, uint16_t* A2, float* Y, void* scratch,
+                                   cudaStream_t stream, cudaEvent_t mid_event) {
+    const W16Layout L = w16_layout(E, H, I, compact);
+    const uint8_t* p = static_cast<const uint8_t*>(packed);
+    uint8_t* sc = static_cast<uint8_t*>(scratch);
+    const bool ch4 = w16_ch(H, I) == 4;
+    if (compact)
+        return ch4 ? run_w16<true, 4>(x, p, L, T, H, I, E, k, plan, A2, Y, sc, stream, mid_event)
+                   : run_w16<true, 2>(x, p, L, T, H, I, E, k, plan, A2, Y, sc, stream, mid_event);
+    return ch4 ? run_w16<false, 4>(x, p, L, T, H, I, E, k, plan, A2, Y, sc, stream, mid_event)
+               : run_w16<false, 2>(x, p, L, T, H, I, E, k, plan, A2, Y, sc, stream, mid_event);
 }
 
 }  // namespace nvfp4moe
