@@ -80,13 +80,6 @@ inline W16Layout w16_layout(int E, int H, int I, bool compact) {
 // 2^k as FP32 for k in [-126, 127]
 __device__ __forceinline__ float pow2f(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
 
-// A row exponent, loaded where it is written in the code: issued before the
-// weight stream so that its latency is not paid in the epilogue.
-__device__ __forceinline__ int ld_rexp(const int8_t* p) {
-    int v;
-    asm volatile("ld.global.nc.s8 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
-}
 
 // ---------------------------------------------------------------------------
 // pack: per 16-row tile and 64-column chunk, 512 bytes in fragment order (lane
@@ -399,36 +392,35 @@ __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* pair, int chu
                     sw[u] = *reinterpret_cast<const uint32_t*>(st + u * GB + CH * 512 + (cc >> 1) * 32 + g * 4);
 #pragma unroll
                 for (int blk = 0; blk < 2; ++blk) {
-                    float prod[2][NT][4];
+                    uint2 bw[2][NT];  // the block's two k16 steps
 #pragma unroll
-                    for (int s2 = 0; s2 < 2; ++s2) {
-                        const int stp = 2 * blk + s2;
-                        uint2 bw[NT];
+                    for (int s2 = 0; s2 < 2; ++s2)
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) bw[nt] = __ldg(bp[nt] + stp);
+                        for (int nt = 0; nt < NT; ++nt) bw[s2][nt] = __ldg(bp[nt] + 2 * blk + s2);
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
+                    for (int u = 0; u < 2; ++u) {
+                        float prod[NT][4];
+#pragma unroll
+                        for (int s2 = 0; s2 < 2; ++s2) {
+                            const int stp = 2 * blk + s2;
                             const uint32_t qw = stp == 0 ? q[u].x : stp == 1 ? q[u].y : stp == 2 ? q[u].z : q[u].w;
                             uint32_t a[4];
                             codes_step(qw, a);
 #pragma unroll
                             for (int nt = 0; nt < NT; ++nt) {
-                                if (s2 == 0) mma_f16_first(prod[u][nt], a, bw[nt].x, bw[nt].y);
-                                else mma_f16(prod[u][nt], a, bw[nt].x, bw[nt].y);
+                                if (s2 == 0) mma_f16_first(prod[nt], a, bw[s2][nt].x, bw[s2][nt].y);
+                                else mma_f16(prod[nt], a, bw[s2][nt].x, bw[s2][nt].y);
                             }
                         }
-                    }
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
                         const uint32_t nf = sw[u] >> (8 * (cc & 1) + 4 * blk);  // row g's field in bits 0..3, g + 8's in 16..19
                         const float s_g = __uint_as_float(0x46000000u - (nf & 15u) * 0x00800000u);
                         const float s_g8 = __uint_as_float(0x46000000u - ((nf >> 16) & 15u) * 0x00800000u);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
-                            acc[u][nt][0] = __fmaf_rn(prod[u][nt][0], s_g, acc[u][nt][0]);
-                            acc[u][nt][1] = __fmaf_rn(prod[u][nt][1], s_g, acc[u][nt][1]);
-                            acc[u][nt][2] = __fmaf_rn(prod[u][nt][2], s_g8, acc[u][nt][2]);
-                            acc[u][nt][3] = __fmaf_rn(prod[u][nt][3], s_g8, acc[u][nt][3]);
+                            acc[u][nt][0] = __fmaf_rn(prod[nt][0], s_g, acc[u][nt][0]);
+                            acc[u][nt][1] = __fmaf_rn(prod[nt][1], s_g, acc[u][nt][1]);
+                            acc[u][nt][2] = __fmaf_rn(prod[nt][2], s_g8, acc[u][nt][2]);
+                            acc[u][nt][3] = __fmaf_rn(prod[nt][3], s_g8, acc[u][nt][3]);
                         }
                     }
                 }
@@ -504,17 +496,6 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16Cfg<CH>::MIN_CTAS)
         const int n_e = plan.counts[e];
         const int row0 = plan.offsets[e];
         const float ag = glob[e * 3 + 0], au = glob[e * 3 + 1];
-        float ph[2][2] = {{1.0f, 1.0f}, {1.0f, 1.0f}};  // [gate, up][rows g, g + 8]: compact row factors
-        if (COMPACT) {
-            const int64_t r = (int64_t)e * I + ib * 16 + g;
-            const int8_t* rg = reinterpret_cast<const int8_t*>(packed + L.rexp_g);
-            const int8_t* ru = reinterpret_cast<const int8_t*>(packed + L.rexp_u);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                ph[0][h] = pow2f(ld_rexp(rg + r + 8 * h) - 13);
-                ph[1][h] = pow2f(ld_rexp(ru + r + 8 * h) - 13);
-            }
-        }
         const int64_t pair = (int64_t)e * iblocks + ib;  // tiles 2 pair (gate) and 2 pair + 1 (up)
         const uint8_t* tb = packed + L.gu + pair * (chunks / CH) * 2 * w16_group_bytes(COMPACT, CH);
         for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
@@ -529,6 +510,17 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16Cfg<CH>::MIN_CTAS)
             const bool ok = nt_count == 1 ? w16_stream<1, COMPACT, CH>(ring, tb, chunks, bptr, acc, err)
                                           : w16_stream<2, COMPACT, CH>(ring, tb, chunks, bptr, acc, err);
             if (!ok) return;
+            float ph[2][2] = {{1.0f, 1.0f}, {1.0f, 1.0f}};  // [gate, up][rows g, g + 8]: compact row factors
+            if (COMPACT) {
+                const int64_t r = (int64_t)e * I + ib * 16 + g;
+                const int8_t* rg = reinterpret_cast<const int8_t*>(packed + L.rexp_g);
+                const int8_t* ru = reinterpret_cast<const int8_t*>(packed + L.rexp_u);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    ph[0][h] = pow2f(rg[r + 8 * h] - 13);
+                    ph[1][h] = pow2f(ru[r + 8 * h] - 13);
+                }
+            }
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
                 if (nt >= nt_count) break;
@@ -573,14 +565,6 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16Cfg<CH>::MIN_CTAS)
         const int n_e = plan.counts[e];
         const int row0 = plan.offsets[e];
         const float ad = glob[e * 3 + 2];
-        float ph[2][2] = {{1.0f, 1.0f}, {1.0f, 1.0f}};  // [tile u][rows g, g + 8]: compact row factors
-        if (COMPACT) {
-            const int8_t* rd = reinterpret_cast<const int8_t*>(packed + L.rexp_d) + (int64_t)e * H + hb * 32 + g;
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) ph[u][h] = pow2f(ld_rexp(rd + u * 16 + 8 * h) - 13);
-        }
         const int64_t pair = (int64_t)e * (H / 32) + hb;  // 16-row tiles 2 pair, 2 pair + 1
         const uint8_t* tb = packed + L.d + pair * (chunks / CH) * 2 * w16_group_bytes(COMPACT, CH);
         for (int n0 = 0; n0 < n_e; n0 += 8 * W16_MAX_NT) {
@@ -595,6 +579,14 @@ __global__ void __launch_bounds__(W16_WARPS * 32, W16Cfg<CH>::MIN_CTAS)
             const bool ok = nt_count == 1 ? w16_stream<1, COMPACT, CH>(ring, tb, chunks, bptr, acc, err)
                                           : w16_stream<2, COMPACT, CH>(ring, tb, chunks, bptr, acc, err);
             if (!ok) return;
+            float ph[2][2] = {{1.0f, 1.0f}, {1.0f, 1.0f}};  // [tile u][rows g, g + 8]: compact row factors
+            if (COMPACT) {
+                const int8_t* rd = reinterpret_cast<const int8_t*>(packed + L.rexp_d) + (int64_t)e * H + hb * 32 + g;
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) ph[u][h] = pow2f(rd[u * 16 + 8 * h] - 13);
+            }
 #pragma unroll
             for (int nt = 0; nt < W16_MAX_NT; ++nt) {
                 if (nt >= nt_count) break;
