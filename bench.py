@@ -74,11 +74,17 @@ MODE_DTYPES = {0: "bf16 activations x fp4 e2m1 weights (e4m3 block scales), fp16
                2: "bf16 activations x fp4 e2m1 weights (compact power-of-two scales), fp16 mma -> f32",
                3: "fp8 e4m3 (e8m0 block scales) x fp4 e2m1 (e8m0 block scales) -> f32"}
 
-# DRAM bytes (read + write) of one k_w4a4_gemm<gate/up> launch, from ncu
-# (profiles/k_w4a4_gemm_prefill2k_e64.txt: 652.8 MB read + 22.6 MB written at
-# T=2048, E=64), scaled x4 to T=8192, E=256 (weights and activations both grow
-# 4x).  Valid for this kernel version and the default prefill workload only.
-GATEUP_TRAFFIC_T8192_E256 = 4 * (652.802560e6 + 22.621184e6)
+# DRAM bytes (read + write) per launch from ncu captures of smaller cases of
+# the same kernels (profiles/), valid for these kernel versions and workloads only:
+#  - k_w4a4_gemm gate/up, W4A4 (k_w4a4_gemm_prefill2k_e64.txt: 652.9 MB read +
+#    23.6 MB written at T=2048, E=64), scaled x4 to T=8192, E=256 (weights and
+#    activations both grow 4x);
+#  - the same for W4A8 (k_w4a8_gemm_prefill2k_e64.txt: 1202.4 MB + 39.4 MB);
+#  - k_w16_gateup + k_w16_down of one 16-token decode step at E=256 (the bench's
+#    own workload, captured at full size: k_w16_decode16.txt).
+GATEUP_TRAFFIC_T8192_E256 = 4 * (652.901632e6 + 23.571712e6)
+GATEUP_W4A8_TRAFFIC_T8192_E256 = 4 * (1202.429e6 + 39.362048e6)
+DECODE_TRAFFIC_T16_E256 = 1010.475e6 + 4.71296e6 + 505.455e6 + 5.101568e6
 
 
 class ClockSampler:
@@ -339,8 +345,8 @@ def run_ours(args, rank, world, local_rank):
         # sustained bf16 figure, scaled to FP4 (FP8 for W4A8) by the nominal dense ratio.
         ratio = FP4_OVER_BF16 if mode == moe.W4A4 else FP8_OVER_BF16
         peak = P["bf16_tflops_sustained"] * ratio
-        traffic = (GATEUP_TRAFFIC_T8192_E256 if mode == moe.W4A4 and (T, wl.E, wl.H, wl.I) == (8192, 256, 4096, 2048)
-                   else None)
+        full = (T, wl.E, wl.H, wl.I) == (8192, 256, 4096, 2048)
+        traffic = (GATEUP_TRAFFIC_T8192_E256 if mode == moe.W4A4 else GATEUP_W4A8_TRAFFIC_T8192_E256) if full else None
         roofline = {"bound": "tensor", "kernel": "k_w4a4_gemm<gate/up>", "achieved": round(achieved, 1),
                     "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                     "traffic": traffic, "traffic_unit": "bytes per launch (ncu dram read+write)",
@@ -361,7 +367,10 @@ def run_ours(args, rank, world, local_rank):
         t_kernel = (stage["gateup_gemm"] + stage["down_gemm"]) / 1e3
         achieved = wbytes / t_kernel / 1e9
         roofline = {"bound": "hbm", "kernel": "k_w16_gateup + k_w16_down", "achieved": round(achieved, 1),
-                    "peak": P["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / P["hbm_gbs"], 4), "traffic": None,
+                    "peak": P["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / P["hbm_gbs"], 4),
+                    "traffic": (DECODE_TRAFFIC_T16_E256 if mode == moe.W4A16 and wl.name == "decode" and T == 16
+                                and wl.E == 256 else None),
+                    "traffic_unit": "bytes per step of both GEMM launches (ncu dram read+write)",
                     "peak_src": f"{P['src']} copy bandwidth", "algorithmic_bytes_per_step": int(wbytes),
                     "active_experts": active}
 
@@ -456,7 +465,9 @@ def bench_decode(torch, moe, w, args, P, compact=False):
             **({"same_weights": same_weights} if same_weights else {}),
             "roofline": {"bound": "hbm", "kernel": "k_w16_gateup + k_w16_down", "achieved": round(achieved, 1),
                          "peak": P["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / P["hbm_gbs"], 4),
-                         "traffic": None, "algorithmic_bytes_per_step": int(wbytes)}}
+                         "traffic": None if compact else DECODE_TRAFFIC_T16_E256,
+                         "traffic_unit": "bytes per step of both GEMM launches (ncu dram read+write)",
+                         "algorithmic_bytes_per_step": int(wbytes)}}
 
 
 def bench_w4a8(torch, moe, args, P):
@@ -487,7 +498,9 @@ def bench_w4a8(torch, moe, args, P):
             "stages_ms": {k: round(v, 4) for k, v in stage.items()},
             "same_weights": {"mode": "W4A4", "ms_per_step": round(ms4, 4)},
             "roofline": {"bound": "tensor", "kernel": "k_w4a4_gemm<gate/up, FP8 x FP4>", "achieved": round(achieved, 1),
-                         "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                         "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                         "traffic": GATEUP_W4A8_TRAFFIC_T8192_E256,
+                         "traffic_unit": "bytes per launch (ncu dram read+write)",
                          "peak_src": f"{P['src']} bf16 sustained x {FP8_OVER_BF16:g} (nominal dense FP8:BF16)",
                          "algorithmic_flops_per_launch": flops}}
 
