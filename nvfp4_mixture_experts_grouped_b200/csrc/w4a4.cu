@@ -292,12 +292,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         tc::bulk_load(st + A_BYTES + B_BYTES, sfa, na * 512, &full[s]);
                     }
                     tc::tma_load_2d(st + A_BYTES, &tmB, ks * 128, (int32_t)(b_tile0 + BM * rank), &full[s]);
-#pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const uint8_t* sfb =
-                            p.sfb + ((b_tile0 / 128 + r) * atoms_per_row + ks * Cfg<KIND>::SFA_ATOMS) * 512;
-                        tc::bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES + r * SFA_BYTES, sfb, na * 512, &full[s]);
-                    }
+                    // the stage's scale atoms of all 256 N rows are stored together: one copy
+                    // (placed so that rows 128..255 start na atoms after rows 0..127)
+                    const uint8_t* sfb =
+                        p.sfb + ((b_tile0 / 256) * atoms_per_row * 2 + ks * Cfg<KIND>::SFA_ATOMS * 2) * 512;
+                    tc::bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES, sfb, 2 * na * 512, &full[s]);
                 }
             }
             // wait for the MMA's release of every slot still in use, so that no
@@ -392,12 +391,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const uint8_t* st = smem + s * STAGE_BYTES + A_BYTES + B_BYTES;
                 const uint32_t col = t_q + TM_SF + (uint32_t)s * TM_SF_STRIDE;
                 if (KIND == KIND_NVF4) {
+                    // B's atoms of N rows 128..255 follow the na atoms of rows 0..127 (na < 4
+                    // only in a last, partial stage; atoms past na are not read by the MMAs)
+                    const int na = min(4, ksub_total - ks * 4);
+                    const uint8_t* sb1 = st + SFA_BYTES + na * 512;
                     uint32_t v[48];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint4 a = *reinterpret_cast<const uint4*>(st + j * 512 + lane * 16);
                         const uint4 b0 = *reinterpret_cast<const uint4*>(st + SFA_BYTES + j * 512 + lane * 16);
-                        const uint4 b1 = *reinterpret_cast<const uint4*>(st + 2 * SFA_BYTES + j * 512 + lane * 16);
+                        const uint4 b1 = *reinterpret_cast<const uint4*>(sb1 + j * 512 + lane * 16);
                         v[4 * j + 0] = a.x, v[4 * j + 1] = a.y, v[4 * j + 2] = a.z, v[4 * j + 3] = a.w;
                         v[16 + 8 * j + 0] = b0.x, v[16 + 8 * j + 1] = b0.y, v[16 + 8 * j + 2] = b0.z,
                                        v[16 + 8 * j + 3] = b0.w;
@@ -564,6 +567,22 @@ done:
     }
 }
 
+// Byte offset of weight scale column kb of packed row r in the weights' scale
+// layout: the atom layout (128 rows x 4 columns per 512-byte atom), with the
+// atoms a K stage of a 256-row N tile needs stored together -- the stage's
+// atoms of rows 0..127 of the tile, then those of rows 128..255 -- so one bulk
+// copy fetches them.  n_kb: scale columns per row; stage_atoms: atoms per 128
+// rows in a full stage (4 for W4A4, 1 for W4A8); a last, partial stage holds
+// fewer of each.
+__host__ __device__ inline int64_t wsf_offset(int64_t r, int64_t kb, int64_t n_kb, int stage_atoms) {
+    const int64_t atoms_per_row = n_kb >> 2, katom = kb >> 2;
+    const int64_t ks = katom / stage_atoms;
+    const int64_t na = min((int64_t)stage_atoms, atoms_per_row - ks * stage_atoms);
+    return ((r >> 8) * atoms_per_row * 2 + ks * stage_atoms * 2 + ((r >> 7) & 1) * na + (katom - ks * stage_atoms)) *
+               512 +
+           (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);
+}
+
 // ---------------------------------------------------------------------------
 // pack: gate/up rows interleaved per 128 (a 256-row N-tile = 128 gate rows then
 // the same 128 intermediates' up rows), block scales into the atom layout.
@@ -601,8 +620,7 @@ __global__ void k_w4_pack_sf(const uint8_t* __restrict__ src0, const uint8_t* __
         src = w < 128 ? src0 : src1;
         srow = e * rows_per_expert_src + b * 128 + (w & 127);
     }
-    const int64_t off = ((prow >> 7) * (nkb >> 2) + (kb >> 2)) * 512 + (prow & 31) * 16 + ((prow >> 5) & 3) * 4 + (kb & 3);
-    dst[off] = src[srow * nkb + kb];
+    dst[wsf_offset(prow, kb, nkb, Cfg<KIND_NVF4>::SFA_ATOMS)] = src[srow * nkb + kb];
 }
 
 // W4A8 weights: codes in the padded form the FP8 x FP4 MMA reads (each 8 bytes
@@ -649,7 +667,7 @@ __global__ void k_w8_pack_sf(const uint8_t* __restrict__ src0, const uint8_t* __
     const uint8_t* s = src + srow * (2 * nkb32) + 2 * kb;
     int e = 0;
     const int kind = compact_block_kind(s[0], s[1], e);
-    dst[sf_atom_offset(prow, kb, nkb32)] = (uint8_t)(kind == 0 ? e + 127 : 127);
+    dst[wsf_offset(prow, kb, nkb32, Cfg<KIND_MXF8>::SFA_ATOMS)] = (uint8_t)(kind == 0 ? e + 127 : 127);
 }
 
 // ---------------------------------------------------------------------------
