@@ -281,27 +281,6 @@ __device__ __forceinline__ void dequant_step(uint32_t q, uint32_t m, uint32_t a[
     }
 }
 
-// 8 codes of one k16 step -> the four FP16x2 A-fragment registers, unscaled.
-__device__ __forceinline__ void codes_step(uint32_t q, uint32_t a[4]) {
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
-        : "r"(q));
-}
-
-// d = A B (no accumulator input)
-__device__ __forceinline__ void mma_f16_first(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%10,%10,%10};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
-}
-
 __device__ __forceinline__ void mma_f16(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -348,9 +327,9 @@ __device__ __forceinline__ void ring_issue(Ring& r, int stage, const uint8_t* pa
 // products with NT 8-token B tiles (FP16 rows in fragment order; every lane's
 // pointer is valid, lanes past the expert's tokens read a real row and their
 // results are dropped).  Returns false on a timeout.  COMPACT: the scales are
-// 4-bit fields n, one per 32 columns; the codes enter the MMA unscaled and each
-// 32-column block's FP32 product is added to the accumulator times 2^(13 - n)
-// (the row factor 2^(r - 13) is applied by the caller).
+// 4-bit fields n, one per 32 columns, and each weight is multiplied by 2^(13 - n)
+// in FP16 (exact); the row factor 2^(r - 13) is applied by the caller, an exact
+// power-of-two move, so the result equals the E4M3-scale form's bit for bit.
 template <int NT, bool COMPACT, int CH>
 __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* pair, int chunks, const __half* const bptr[W16_MAX_NT],
                                            float acc[2][W16_MAX_NT][4], int32_t* err) {
@@ -379,72 +358,37 @@ __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* pair, int chu
 #pragma unroll
             for (int u = 0; u < 2; ++u)
                 q[u] = *reinterpret_cast<const uint4*>(st + u * GB + cc * 512 + lane * 16);
-            if (COMPACT) {
-                // One power-of-two scale per 32 columns: the two k16 steps of a block
-                // accumulate unscaled codes into a block product, which joins the
-                // accumulator with one FP32 multiply-add per value:
-                // acc += product * 2^(13 - n) (the row factor 2^(r - 13) is applied
-                // at the end).  FP32 bits of 2^(13 - n): (140 - n) << 23.
-                static_assert(CH % 2 == 0, "a compact scale word covers two chunks");
-                uint32_t sw[2];  // the scale word of this chunk pair, each tile
+            uint32_t m[2][4];  // FP16x2 {scale g, scale g + 8} of each k16 step
 #pragma unroll
-                for (int u = 0; u < 2; ++u)
-                    sw[u] = *reinterpret_cast<const uint32_t*>(st + u * GB + CH * 512 + (cc >> 1) * 32 + g * 4);
-#pragma unroll
-                for (int blk = 0; blk < 2; ++blk) {
-                    uint2 bw[2][NT];  // the block's two k16 steps
-#pragma unroll
-                    for (int s2 = 0; s2 < 2; ++s2)
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) bw[s2][nt] = __ldg(bp[nt] + 2 * blk + s2);
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        float prod[NT][4];
-#pragma unroll
-                        for (int s2 = 0; s2 < 2; ++s2) {
-                            const int stp = 2 * blk + s2;
-                            const uint32_t qw = stp == 0 ? q[u].x : stp == 1 ? q[u].y : stp == 2 ? q[u].z : q[u].w;
-                            uint32_t a[4];
-                            codes_step(qw, a);
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) {
-                                if (s2 == 0) mma_f16_first(prod[nt], a, bw[s2][nt].x, bw[s2][nt].y);
-                                else mma_f16(prod[nt], a, bw[s2][nt].x, bw[s2][nt].y);
-                            }
-                        }
-                        const uint32_t nf = sw[u] >> (8 * (cc & 1) + 4 * blk);  // row g's field in bits 0..3, g + 8's in 16..19
-                        const float s_g = __uint_as_float(0x46000000u - (nf & 15u) * 0x00800000u);
-                        const float s_g8 = __uint_as_float(0x46000000u - ((nf >> 16) & 15u) * 0x00800000u);
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            acc[u][nt][0] = __fmaf_rn(prod[nt][0], s_g, acc[u][nt][0]);
-                            acc[u][nt][1] = __fmaf_rn(prod[nt][1], s_g, acc[u][nt][1]);
-                            acc[u][nt][2] = __fmaf_rn(prod[nt][2], s_g8, acc[u][nt][2]);
-                            acc[u][nt][3] = __fmaf_rn(prod[nt][3], s_g8, acc[u][nt][3]);
-                        }
-                    }
-                }
-            } else {
-                uint32_t m[2][4];  // FP16x2 {scale g, scale g + 8} of each k16 step
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < 2; ++u) {
+                if (COMPACT) {
+                    // the 4-bit fields n of rows g, g + 8 in the two halves of a word;
+                    // multiplier 2^(13 - n) = FP16 bits (28 - n) << 10 (the row factor
+                    // 2^(r - 13) is applied in the epilogue)
+                    static_assert(CH % 2 == 0, "a compact scale word covers two chunks");
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(st + u * GB + CH * 512 + (cc >> 1) * 32 + g * 4);
+                    const uint32_t n0 = (w >> (8 * (cc & 1))) & 0x000F000Fu;
+                    const uint32_t n1 = (w >> (8 * (cc & 1) + 4)) & 0x000F000Fu;
+                    m[u][0] = m[u][1] = 0x70007000u - n0 * 1024u;
+                    m[u][2] = m[u][3] = 0x70007000u - n1 * 1024u;
+                } else {
                     const uint2 sc = *reinterpret_cast<const uint2*>(st + u * GB + CH * 512 + cc * 64 + g * 8);
                     scales_f16x2x2(sc.x, m[u][0], m[u][1]);
                     scales_f16x2x2(sc.y, m[u][2], m[u][3]);
                 }
+            }
 #pragma unroll
-                for (int stp = 0; stp < 4; ++stp) {
-                    uint2 bw[NT];
+            for (int stp = 0; stp < 4; ++stp) {
+                uint2 bw[NT];
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) bw[nt] = __ldg(bp[nt] + stp);
+                for (int nt = 0; nt < NT; ++nt) bw[nt] = __ldg(bp[nt] + stp);
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const uint32_t qw = stp == 0 ? q[u].x : stp == 1 ? q[u].y : stp == 2 ? q[u].z : q[u].w;
-                        uint32_t a[4];
-                        dequant_step(qw, m[u][stp], a);
+                for (int u = 0; u < 2; ++u) {
+                    const uint32_t qw = stp == 0 ? q[u].x : stp == 1 ? q[u].y : stp == 2 ? q[u].z : q[u].w;
+                    uint32_t a[4];
+                    dequant_step(qw, m[u][stp], a);
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) mma_f16(acc[u][nt], a, bw[nt].x, bw[nt].y);
-                    }
+                    for (int nt = 0; nt < NT; ++nt) mma_f16(acc[u][nt], a, bw[nt].x, bw[nt].y);
                 }
             }
         }
