@@ -256,13 +256,19 @@ __global__ void __launch_bounds__(256)
     // every lane runs every iteration (the shuffles below need all 32); lanes past
     // the row's last block only skip their loads and stores.  The scatter form
     // needs nb % 4 == 0 (K % 64 == 0) so that a lane quad is all in or all out.
+    // the next iteration's loads are issued before this one's arithmetic and stores
+    uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+    if (lane < nb) {
+        n0 = __ldg(reinterpret_cast<const uint4*>(xr + lane * 16));
+        n1 = __ldg(reinterpret_cast<const uint4*>(xr + lane * 16 + 8));
+    }
     for (int64_t b0 = 0; b0 < nb; b0 += 32) {
         const int64_t b = b0 + lane;
         const bool active = b < nb;
-        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-        if (active) {
-            v0 = __ldg(reinterpret_cast<const uint4*>(xr + b * 16));
-            v1 = __ldg(reinterpret_cast<const uint4*>(xr + b * 16 + 8));
+        const uint4 v0 = n0, v1 = n1;
+        if (b + 32 < nb) {
+            n0 = __ldg(reinterpret_cast<const uint4*>(xr + (b + 32) * 16));
+            n1 = __ldg(reinterpret_cast<const uint4*>(xr + (b + 32) * 16 + 8));
         }
         float f[16];
         const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
@@ -328,11 +334,20 @@ __global__ void __launch_bounds__(256)
     const int64_t nb = K / 32;
     const uint16_t* xr = x + m * K;
     const int my_row = SCATTER && lane < k ? row_of_pair[m * k + lane] : 0;
+    // loads run two iterations ahead of the arithmetic and stores
+    uint4 nx[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int64_t b = 8 * i + (lane >> 2);
+        nx[i] = b < nb ? __ldg(reinterpret_cast<const uint4*>(xr + b * 32 + (lane & 3) * 8)) : make_uint4(0, 0, 0, 0);
+    }
     for (int64_t b0 = 0; b0 < nb; b0 += 8) {
         const int64_t b = b0 + (lane >> 2);  // this lane's block; it holds elements 8 (lane % 4) .. +7
         const bool active = b < nb;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (active) v = __ldg(reinterpret_cast<const uint4*>(xr + b * 32 + (lane & 3) * 8));
+        const uint4 v = nx[0];
+        nx[0] = nx[1];
+        nx[1] = b + 16 < nb ? __ldg(reinterpret_cast<const uint4*>(xr + (b + 16) * 32 + (lane & 3) * 8))
+                            : make_uint4(0, 0, 0, 0);
         float f[8];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
