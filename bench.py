@@ -192,8 +192,12 @@ def make_layer(torch, moe, mode, w, T, wl):
     return packed, ws
 
 
-def time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, steps, warmup, trace=True, on_start=None):
-    """Returns (ms per step, per-stage ms means) timed with CUDA events on the current stream."""
+def time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, steps, warmup, trace=True, on_start=None,
+               on_end=None):
+    """Returns (ms per step, per-stage ms means), both timed with CUDA events on the current
+    stream.  The step time comes from a pass without stage events (recording 7 events per
+    step costs a few microseconds, visible at decode sizes); the stage times from a second,
+    traced pass of the same steps."""
     H, I, E = wl.H, wl.I, wl.E
 
     def step():
@@ -203,30 +207,34 @@ def time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, steps, warmu
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    evs = []
-    if trace:
-        for _ in range(steps):
-            row = [torch.cuda.Event(enable_timing=True) for _ in range(N_TRACE)]
-            for e in row:
-                e.record()
-            evs.append(row)
-    torch.cuda.synchronize()
     if on_start:
         on_start()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
-    for i in range(steps):
-        if trace:
-            moe.nvfp4moe_set_trace_events(evs[i])
+    for _ in range(steps):
         step()
     t1.record()
     torch.cuda.synchronize()
-    moe.nvfp4moe_set_trace_events(None)
     moe.nvfp4moe_check_device_status()
     ms = t0.elapsed_time(t1) / steps
+    if on_end:
+        on_end()
     stage = None
     if trace:
+        evs = []
+        for _ in range(steps):
+            row = [torch.cuda.Event(enable_timing=True) for _ in range(N_TRACE)]
+            for e in row:
+                e.record()
+            evs.append(row)
+        torch.cuda.synchronize()
+        for i in range(steps):
+            moe.nvfp4moe_set_trace_events(evs[i])
+            step()
+        torch.cuda.synchronize()
+        moe.nvfp4moe_set_trace_events(None)
+        moe.nvfp4moe_check_device_status()
         stage = {}
         for s, name in enumerate(STAGES):
             stage[name] = float(np.mean([evs[i][s].elapsed_time(evs[i][s + 1]) for i in range(steps)]))
@@ -316,9 +324,15 @@ def run_ours(args, rank, world, local_rank):
     sampler = ClockSampler(local_rank) if rank == 0 else None
     if sampler:
         sampler.wait_ready()
+    held = {}
+
+    def end_of_region():
+        if sampler:
+            held["clocks"] = sampler.stop()
+
     ms, stage = time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, args.steps, args.warmup,
-                           on_start=sampler.mark if sampler else None)
-    clocks = sampler.stop() if sampler else None
+                           on_start=sampler.mark if sampler else None, on_end=end_of_region)
+    clocks = held.get("clocks")
     ms = max_over_ranks(torch, dist, ms, "cuda")
     if dist:
         dist.barrier()
