@@ -146,17 +146,6 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
 // ---------------------------------------------------------------------------
 // tcgen05
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
-                 "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -191,17 +180,6 @@ __device__ __forceinline__ uint64_t desc_sw128(const void* smem) {
     return d;
 }
 
-// Descriptor of a 32-row x 16-byte scale-factor block (no swizzle, 8-row core
-// matrices 128 bytes apart) for tcgen05.cp.
-__device__ __forceinline__ uint64_t desc_sf(const void* smem) {
-    const uint64_t addr = smem_u32(smem);
-    uint64_t d = 0;
-    d |= (addr >> 4) & 0x3FFFull;
-    d |= (uint64_t)(128 >> 4) << 32;  // stride byte offset between 8-row core matrices
-    d |= (uint64_t)1 << 46;
-    return d;
-}
-
 // Instruction descriptor of kind::mxf4nvf4 with E4M3 block scales (one per 16
 // elements, scale_vec::4X): A and B E2M1, K-major, FP32 accumulate.
 __host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int M, int N) {
@@ -210,17 +188,6 @@ __host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int M, int N) {
            | ((uint32_t)(N >> 3) << 17)  // N / 8
            | (0u << 23)                // scale format: UE4M3
            | ((uint32_t)(M >> 4) << 24);  // M / 16
-}
-
-__device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
-            d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-        : "memory");
 }
 
 // The pair form, issued by one thread of the even CTA: M = 256 rows, the first
@@ -263,19 +230,6 @@ __device__ __forceinline__ void mma_mxf8f6f4_pair(uint32_t d_tmem, uint64_t ades
             d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
-}
-
-// Copy a 32-row x 128-bit block from shared memory to TMEM, replicated into the
-// four 32-lane quadrants.
-__device__ __forceinline__ void tmem_cp_32x128_x4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
-// Arrive once on `bar` when all previously issued tcgen05 operations of this
-// thread have completed.
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
 }
 
 // Pair form: arrive once on the mbarrier at `bar`'s shared-memory offset in every

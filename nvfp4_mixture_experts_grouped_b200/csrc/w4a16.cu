@@ -80,7 +80,6 @@ inline W16Layout w16_layout(int E, int H, int I, bool compact) {
 // 2^k as FP32 for k in [-126, 127]
 __device__ __forceinline__ float pow2f(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
 
-
 // ---------------------------------------------------------------------------
 // pack: per 16-row tile and 64-column chunk, 512 bytes in fragment order (lane
 // l holds 16 bytes: one 32-bit word per k16 step); inside a word byte j holds
@@ -238,15 +237,6 @@ __global__ void __launch_bounds__(256)
         for (int q = 0; q < 4; ++q) d[wbase + q * 8] = o[q];
     }
     if (lane == 0) inv_scale[r] = ldexpf(1.0f, -sh);
-}
-
-// ---------------------------------------------------------------------------
-// dequantisation and MMA helpers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
 }
 
 // Four E4M3 scales (bytes 0..3 of `w`) -> two FP16x2 (exact): bytes 0, 1 and 2, 3.
