@@ -79,7 +79,7 @@ MODE_DTYPES = {0: "bf16 activations x fp4 e2m1 weights (e4m3 block scales), fp16
 #  - k_w4a4_gemm gate/up, W4A4 (k_w4a4_gemm_prefill2k_e64.txt: 652.9 MB read +
 #    23.6 MB written at T=2048, E=64), scaled x4 to T=8192, E=256 (weights and
 #    activations both grow 4x);
-#  - the same for W4A8 (k_w4a8_gemm_prefill2k_e64.txt: 1202.4 MB + 39.4 MB);
+#  - the same for W4A8 (k_w4a8_gemm_prefill2k_e64.txt), its weights read as packed 4-bit codes;
 #  - k_w16_gateup + k_w16_down of one 16-token decode step at E=256 (the bench's
 #    own workload, captured at full size: k_w16_decode16.txt).
 GATEUP_TRAFFIC_T8192_E256 = 4 * (652.901632e6 + 23.571712e6)

@@ -311,8 +311,8 @@ size_t moe_packed_weights_size(nvfp4moe_mode mode, int32_t E, int32_t H, int32_t
  * NVFP4MOE_W4A16C re-encodes the scales (nvfp4_compact_scales) and is
  * SYNCHRONOUS: it waits for `stream` and returns NVFP4MOE_ERR_NOT_REPRESENTABLE
  * when any weight row has no compact form (the packed buffer is then unusable).
- * NVFP4MOE_W4A8 stores each code in a byte-per-element padded form (twice the
- * code bytes) with E8M0 scales, and is SYNCHRONOUS in the same way: a row whose
+ * NVFP4MOE_W4A8 keeps the 4-bit codes and stores E8M0 scales per 32 (the MMA's
+ * scale type), and is SYNCHRONOUS in the same way: a row whose
  * 32-code blocks do not each have one power-of-two scale (or zero scale over
  * zero codes) makes it return NVFP4MOE_ERR_NOT_REPRESENTABLE.               */
 nvfp4moe_status moe_pack_weights(nvfp4moe_mode mode, const nvfp4moe_expert_weights* weights_host_struct,

@@ -109,16 +109,17 @@ struct W4Layout {
 inline int64_t a256(int64_t v) { return (v + 255) / 256 * 256; }
 
 // W4A4: codes 4 bits and an E4M3 scale per 16 elements (the checkpoint's bytes).
-// W4A8: codes in the padded form (16 codes in 8 bytes + 8 bytes of padding, so
-// one byte per element) and an E8M0 scale per 32; a status word for the pack.
+// W4A8: the same 4-bit codes (the tensor map unpacks them into the padded
+// shared-memory form the FP8 x FP4 MMA reads) and an E8M0 scale per 32; a
+// status word for the pack.
 W4Layout w4_layout(int E, int H, int I, bool mx8 = false) {
     const int64_t n = (int64_t)E * 3 * I * H;  // weights of the layer
     const int64_t gu = (int64_t)E * 2 * I * H;
     W4Layout L;
     L.gu_codes = 0;
-    L.gu_sf = a256(L.gu_codes + (mx8 ? gu : gu / 2));
+    L.gu_sf = a256(L.gu_codes + gu / 2);
     L.d_codes = a256(L.gu_sf + (mx8 ? gu / 32 : gu / 16));
-    L.d_sf = a256(L.d_codes + (mx8 ? (n - gu) : (n - gu) / 2));
+    L.d_sf = a256(L.d_codes + (n - gu) / 2);
     L.globals = a256(L.d_sf + (mx8 ? (n - gu) / 32 : (n - gu) / 16));
     L.status = a256(L.globals + (int64_t)E * 3 * 4);
     L.total = mx8 ? a256(L.status + 16) : L.status;
@@ -284,7 +285,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     // scale atoms of this stage per 128 rows (a partial last stage: W4A4 only)
                     const int na = KIND == KIND_NVF4 ? min(4, ksub_total - ks * 4) : 1;
                     uint8_t* st = smem + s * STAGE_BYTES;
-                    tc::mbar_arrive_expect_tx(&full[s], B_BYTES + 2 * na * 512 + (a_live ? A_BYTES + na * 512 : 0));
+                    // the unpacking copy of W4A8's B counts the packed bytes it reads (half of
+                    // what it writes to shared memory)
+                    constexpr int B_TX = KIND == KIND_MXF8 ? B_BYTES / 2 : B_BYTES;
+                    tc::mbar_arrive_expect_tx(&full[s], B_TX + 2 * na * 512 + (a_live ? A_BYTES + na * 512 : 0));
                     if (a_live) {
                         tc::tma_load_2d(st, &tmA, ks * 128, a_row, &full[s]);
                         const uint8_t* sfa =
@@ -623,29 +627,6 @@ __global__ void k_w4_pack_sf(const uint8_t* __restrict__ src0, const uint8_t* __
     dst[wsf_offset(prow, kb, nkb, Cfg<KIND_NVF4>::SFA_ATOMS)] = src[srow * nkb + kb];
 }
 
-// W4A8 weights: codes in the padded form the FP8 x FP4 MMA reads (each 8 bytes
-// of 16 codes followed by 8 zero bytes), rows interleaved as above.  One thread
-// per 8 source bytes.
-__global__ void k_w8_pack_codes(const uint8_t* __restrict__ src0, const uint8_t* __restrict__ src1, int64_t rows,
-                                int64_t row_bytes, int interleave, int64_t rows_per_expert_src,
-                                uint8_t* __restrict__ dst) {
-    const int64_t per_row = row_bytes / 8;
-    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= rows * per_row) return;
-    const int64_t prow = idx / per_row, v = idx - prow * per_row;
-    const uint8_t* src = src0;
-    int64_t srow = prow;
-    if (interleave) {
-        const int64_t per_e = 2 * rows_per_expert_src;
-        const int64_t e = prow / per_e, p = prow - e * per_e;
-        const int64_t b = p / 256, w = p % 256;
-        src = w < 128 ? src0 : src1;
-        srow = e * rows_per_expert_src + b * 128 + (w & 127);
-    }
-    const uint2 c = reinterpret_cast<const uint2*>(src + srow * row_bytes)[v];
-    reinterpret_cast<uint4*>(dst)[idx] = make_uint4(c.x, c.y, 0u, 0u);
-}
-
 // W4A8 weight scales: the E8M0 scale per 32 of each block whose two E4M3 scales
 // are one power of two 2^e (byte e + 127); a zero-scale block (all codes +-0)
 // takes 2^0.  Rows without that form are counted by the compact-form check
@@ -708,6 +689,31 @@ bool make_map(CUtensorMap* m, const void* base, int64_t row_bytes, int64_t rows,
     return true;
 }
 
+// 2-D map over 4-bit codes [rows, k_elems] (k_elems / 2 bytes per row) that the
+// copy unpacks into the padded shared-memory form (each 16 codes: 8 bytes, then
+// 8 bytes of gap): a box of 128 codes (128 bytes of shared memory) x box_rows,
+// 128-byte swizzle.  Coordinates are in codes.
+bool make_map_u4(CUtensorMap* m, const void* base, int64_t k_elems, int64_t rows, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) {
+        set_error("cuTensorMapEncodeTiled is not available from the driver");
+        return false;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)k_elems, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(k_elems / 2)};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d) for a [%lld x %lld] 4-bit map", (int)r, (long long)rows,
+                  (long long)k_elems);
+        return false;
+    }
+    return true;
+}
+
 // CTA pairs that fit on the device at once (1 CTA per SM), per device and kind, cached.
 template <int KIND>
 int max_resident_pairs() {
@@ -764,11 +770,11 @@ nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed,
                                 1 << 20)};
         for (nvfp4moe_status x : st)
             if (x != NVFP4MOE_OK) return x;
-        k_w8_pack_codes<<<(unsigned)ceil_div(gu_rows * (H / 16), 256), 256, 0, stream>>>(
+        k_w4_pack_codes<<<(unsigned)ceil_div(gu_rows * (H / 32), 256), 256, 0, stream>>>(
             w.gate_codes, w.up_codes, gu_rows, H / 2, 1, I, p + L.gu_codes);
         k_w8_pack_sf<<<(unsigned)ceil_div(gu_rows * (H / 32), 256), 256, 0, stream>>>(w.gate_sf, w.up_sf, gu_rows,
                                                                                        H / 32, 1, I, p + L.gu_sf);
-        k_w8_pack_codes<<<(unsigned)ceil_div(d_rows * (I / 16), 256), 256, 0, stream>>>(w.down_codes, nullptr, d_rows,
+        k_w4_pack_codes<<<(unsigned)ceil_div(d_rows * (I / 32), 256), 256, 0, stream>>>(w.down_codes, nullptr, d_rows,
                                                                                          I / 2, 0, H, p + L.d_codes);
         k_w8_pack_sf<<<(unsigned)ceil_div(d_rows * (I / 32), 256), 256, 0, stream>>>(w.down_sf, nullptr, d_rows, I / 32,
                                                                                        0, H, p + L.d_sf);
@@ -813,12 +819,18 @@ static nvfp4moe_status run_layer(const void* packed, int H, int I, int E, float 
         cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
     NVFP4MOE_CUDA(
         cudaFuncSetAttribute(k_w4a4_gemm<EPI_DOWN, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    // operand rows in bytes: FP4 two codes per byte; FP8 and padded FP4 one element per byte
+    // A rows in bytes: FP4 two codes per byte, FP8 one per byte.  B: W4A4 copies the
+    // packed codes as bytes; W4A8 copies them through a map that unpacks them into
+    // the padded form (coordinates in codes: a stage's 128 codes are 128 bytes of
+    // shared memory either way, so the x coordinate ks * 128 serves both)
     const int64_t hb = MX8 ? H : H / 2, ib = MX8 ? I : I / 2;
     CUtensorMap mA1, mGU, mA2, mD;
-    if (!make_map(&mA1, A1c, hb, rows_max, BM) || !make_map(&mGU, pk + L.gu_codes, hb, (int64_t)E * 2 * I, BN / 2) ||
-        !make_map(&mA2, A2c, ib, rows_max, BM) || !make_map(&mD, pk + L.d_codes, ib, (int64_t)E * H, BN / 2))
-        return NVFP4MOE_ERR_CUDA;
+    const bool ok = make_map(&mA1, A1c, hb, rows_max, BM) && make_map(&mA2, A2c, ib, rows_max, BM) &&
+                    (MX8 ? make_map_u4(&mGU, pk + L.gu_codes, H, (int64_t)E * 2 * I, BN / 2) &&
+                               make_map_u4(&mD, pk + L.d_codes, I, (int64_t)E * H, BN / 2)
+                         : make_map(&mGU, pk + L.gu_codes, H / 2, (int64_t)E * 2 * I, BN / 2) &&
+                               make_map(&mD, pk + L.d_codes, I / 2, (int64_t)E * H, BN / 2));
+    if (!ok) return NVFP4MOE_ERR_CUDA;
     const int pairs = max_resident_pairs<KIND>();
     if (pairs <= 0) return NVFP4MOE_ERR_CUDA;
     GemmParams g{};

@@ -45,8 +45,8 @@ def test_version_and_sizes():
     assert compact <= moe.moe_packed_weights_size(moe.W4A16C, E, H, I) <= compact + 2048
     bits = 8 * moe.moe_packed_weights_size(moe.W4A16C, E, H, I) / (E * 3 * I * H)
     assert 4.125 < bits < 4.13
-    # W4A8: codes one byte per element (padded form) + an E8M0 scale per 32 + globals + a status word
-    w8 = E * (2 * I * H + H * I) + E * (2 * I * H + H * I) // 32 + E * 3 * 4 + 16
+    # W4A8: the 4-bit codes + an E8M0 scale per 32 + globals + a status word
+    w8 = E * (2 * I * H + H * I) // 2 + E * (2 * I * H + H * I) // 32 + E * 3 * 4 + 16
     assert w8 <= moe.moe_packed_weights_size(moe.W4A8, E, H, I) <= w8 + 2048
     assert moe.moe_packed_weights_size(4, E, H, I) == 0  # unknown mode
     ws8 = moe.moe_forward_workspace_size(moe.W4A8, 8192, H, I, E, 8)
