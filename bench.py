@@ -151,6 +151,15 @@ def workload(args):
     return wl
 
 
+def config_of(wl, T, world):
+    """The workload description both arms print."""
+    weights_gb = wl.E * 3 * wl.H * wl.I * (0.5 + 1.0 / 16) / 1e9  # NVFP4 codes + E4M3 scales
+    return {"workload": f"{wl.name}: T={T} H={wl.H} I={wl.I} E={wl.E} groups={wl.n_group} keep={wl.topk_group} "
+                        f"top_k={wl.top_k} rsf={wl.rsf} {MODE_NAMES[wl.mode]}",
+            "global_batch": T * world, "tokens_per_gpu": T, "parallelism": f"replicas{world}",
+            "l2": f"inputs larger than L2 ({weights_gb:.2f} GB of expert weights per step)"}
+
+
 def layer_flops(T, H, I, k):
     return 6.0 * T * k * H * I
 
@@ -393,12 +402,7 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": MODE_DTYPES[mode],
         "data": "synthetic",
-        "config": {"workload": f"{wl.name}: T={T} H={wl.H} I={wl.I} E={wl.E} groups={wl.n_group} "
-                               f"keep={wl.topk_group} top_k={wl.top_k} rsf={wl.rsf} "
-                               f"{MODE_NAMES[mode]}",
-                   "global_batch": T * world, "tokens_per_gpu": T, "parallelism": f"replicas{world}",
-                   "l2": f"inputs larger than L2 ({moe.moe_packed_weights_size(mode, wl.E, wl.H, wl.I) / 1e9:.2f} GB "
-                         f"packed expert weights per step)"},
+        "config": config_of(wl, T, world),
         "roofline": roofline,
         "stages_ms": {k: round(v, 4) for k, v in stage.items()},
         "e2e": {"value": round(job_tokens_per_s(T, world, e2e_ms), 1), "unit": "tokens/s",
@@ -665,8 +669,7 @@ def run_reference(args, rank, world):
     out = {"impl": "reference", "metric": "MoE-layer tokens/s", "value": round(v, 3), "unit": "tokens/s",
            "n_gpus": world, "steps": len(vals), "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 1),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top_k={wl.top_k} "
-                                  f"{'W4A4' if wl.mode else 'W4A16'}"},
+           "config": config_of(wl, wl.T, world),
            "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "kind": "oracle", "cores": vals[0]["cores"],
                             "sample": vals[0]["sample"]},
            "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
