@@ -151,6 +151,16 @@ def workload(args):
     return wl
 
 
+def launches_per_step(mode, T, wl):
+    """Kernels one moe_forward launches (the library's dispatch): routing 1; the
+    permutation 1 fused kernel up to 8192 pairs with E <= 256, else 3; then W4A4 /
+    W4A8: quantise 1 + gate/up 1 + down 1; W4A16 (either scale form): two FP16
+    conversions + gate/up 1 + down 1; the combine 1."""
+    permute = 1 if (wl.E <= 256 and T * wl.top_k <= 8192) else 3
+    layer = 3 if mode in (1, 3) else 4
+    return 1 + permute + layer + 1
+
+
 def config_of(wl, T, world):
     """The workload description both arms print."""
     weights_gb = wl.E * 3 * wl.H * wl.I * (0.5 + 1.0 / 16) / 1e9  # NVFP4 codes + E4M3 scales
@@ -407,7 +417,7 @@ def run_ours(args, rank, world, local_rank):
         "stages_ms": {k: round(v, 4) for k, v in stage.items()},
         "e2e": {"value": round(job_tokens_per_s(T, world, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(d["x"].nbytes + d["logits"].nbytes), "d2h_bytes_per_step": int(T * wl.H * 2)},
-        "gpu_launches": 8 * args.steps,
+        "gpu_launches": launches_per_step(mode, T, wl) * args.steps,
         "clocks": clocks,
         "tflops": round(layer_flops(T, wl.H, wl.I, wl.top_k) / (ms / 1e3) / 1e12, 2),
     }
