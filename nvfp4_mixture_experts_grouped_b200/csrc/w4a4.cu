@@ -266,7 +266,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // [128 rank, +128); the scale factors of its A rows and of all 256 N rows.
         if (lane == 0) {
             // No L2 prefetch: every TMA instruction costs this thread ~85 cycles of
-            // issue (a prefetch ~270), and with five copies per stage the issue
+            // issue (a prefetch ~270), and with four copies per stage the issue
             // time, not the memory system, would bound the MMA rate.
             int it = 0;
             for (int tile = pair; tile < total; tile += n_pairs) {
