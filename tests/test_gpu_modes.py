@@ -84,3 +84,23 @@ def test_w4a8_bias_without_renormalisation():
     ri, rw = oracle.route(lg, bias, MID["ng"], MID["tg"], MID["k"], 2.827, False)
     assert np.array_equal(host(ids), ri) and np.array_equal(host(wts).view(np.uint32), rw.view(np.uint32))
     compare_layer(out_to_f64(out), oracle_mid(3, w, x, lg, bias=bias, renorm=False))
+
+
+@pytest.mark.parametrize("mode", [moe.W4A16, moe.W4A4, moe.W4A8])
+def test_single_expert_layer(mode):
+    # E = 1, top-1: every token on the one expert (several 256-row tiles and a ragged last one)
+    rng = np.random.default_rng(36)
+    E, H, I, T = 1, 512, 256, 300
+    gen = inputs.nvfp4_pow2_tensors
+    gc, gs, gg = gen(rng, E, I, H)
+    uc, us, ug = gen(rng, E, I, H)
+    dc, ds, dg = gen(rng, E, H, I)
+    w = dict(gate_codes=gc, gate_sf=gs, up_codes=uc, up_sf=us, down_codes=dc, down_sf=ds,
+             w_global=np.stack([gg, ug, dg], axis=1).astype(np.float32))
+    x = inputs.activations(rng, T, H)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    layer = GpuLayer(mode, w, T, 1, 1, 1)
+    out, ids, wts = layer.forward(bf16_tensor(x), dev(logits), out_fp32=True)
+    assert not host(ids).any()
+    ref = oracle.moe_layer(mode, x, logits, None, gc, gs, uc, us, dc, ds, w["w_global"], 1.0, 1, 1, 1, 2.827, True)
+    compare_layer(out_to_f64(out), ref)
