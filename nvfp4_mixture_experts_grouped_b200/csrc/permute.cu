@@ -69,10 +69,16 @@ __global__ void __launch_bounds__(1024)
     const int e = threadIdx.x;
     int cnt = 0;
     if (e < E) {
-        for (int c = 0; c < n_chunks; ++c) {
-            const int v = chunk_counts[(int64_t)c * E + e];
-            chunk_counts[(int64_t)c * E + e] = cnt;  // becomes the rank base of chunk c
-            cnt += v;
+        // 16 chunks' loads in flight before their stores: one L2 round trip per 16 chunks
+        for (int c0 = 0; c0 < n_chunks; c0 += 16) {
+            int v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = c0 + i < n_chunks ? chunk_counts[(int64_t)(c0 + i) * E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if (c0 + i < n_chunks) chunk_counts[(int64_t)(c0 + i) * E + e] = cnt;  // the rank base of chunk c0 + i
+                cnt += v[i];
+            }
         }
     }
     int total;
@@ -113,9 +119,11 @@ __global__ void __launch_bounds__(1024)
 __global__ void __launch_bounds__(PERM_CHUNK)
     k_scatter(const int32_t* __restrict__ ids, int T, int k, int E, const int32_t* __restrict__ chunk_base,
               RoutingPlan plan) {
-    extern __shared__ int s_wh[];  // [PERM_WARPS][E]
+    extern __shared__ int s_wh[];  // [PERM_WARPS][E] counters, then [E] padded expert offsets
+    int* s_poff = s_wh + PERM_WARPS * E;
     const int warp = warp_id(), lane = lane_id();
     for (int i = threadIdx.x; i < PERM_WARPS * E; i += blockDim.x) s_wh[i] = 0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_poff[e] = plan.pad_offsets[e];
     __syncthreads();
     const int t0 = blockIdx.x * PERM_CHUNK + warp * 32;
     {
@@ -134,15 +142,19 @@ __global__ void __launch_bounds__(PERM_CHUNK)
     }
     __syncthreads();
     // tokens of this warp in order; a token's k experts are distinct, so the
-    // k lanes never touch the same counter in one step
+    // k lanes never touch the same counter in one step.  Lane j < k holds slot
+    // j's expert of all 32 tokens, loaded before the serial part.
+    int eid[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) eid[i] = lane < k && t0 + i < T ? ids[(int64_t)(t0 + i) * k + lane] : 0;
+#pragma unroll
     for (int i = 0; i < 32; ++i) {
         const int t = t0 + i;
-        if (t >= T) break;
-        if (lane < k) {
+        if (lane < k && t < T) {
             const int64_t p = (int64_t)t * k + lane;
-            const int e = ids[p];
+            const int e = eid[i];
             const int r = s_wh[warp * E + e]++;
-            const int row = plan.pad_offsets[e] + r;
+            const int row = s_poff[e] + r;
             plan.row_of_pair[p] = row;
             plan.pair_of_row[row] = (int32_t)p;
         }
@@ -231,7 +243,7 @@ nvfp4moe_status launch_permute(const int32_t* ids, int T, int k, int E, int pad,
     NVFP4MOE_CHECK_LAUNCH("permute count kernel");
     k_scan_experts<<<1, 1024, 0, stream>>>(n_chunks, E, pad, plan.chunk_counts, plan);
     NVFP4MOE_CHECK_LAUNCH("permute scan kernel");
-    k_scatter<<<n_chunks, PERM_CHUNK, PERM_WARPS * E * sizeof(int), stream>>>(ids, T, k, E, plan.chunk_counts, plan);
+    k_scatter<<<n_chunks, PERM_CHUNK, (PERM_WARPS + 1) * E * sizeof(int), stream>>>(ids, T, k, E, plan.chunk_counts, plan);
     NVFP4MOE_CHECK_LAUNCH("permute scatter kernel");
     return NVFP4MOE_OK;
 }

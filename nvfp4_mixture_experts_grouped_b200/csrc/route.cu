@@ -16,8 +16,10 @@ __global__ void __launch_bounds__(RT_WARPS * 32)
                                     ids, wts, s_c[warp]);
 }
 
+// Up to 256 experts (NPL <= 8) the kernel fits 32 registers, 8 CTAs per SM:
+// 8192 tokens then run as one wave of 1024 CTAs instead of 888 + 136.
 template <int NPL>
-__global__ void __launch_bounds__(RT_WARPS * 32)
+__global__ void __launch_bounds__(RT_WARPS * 32, NPL <= 8 ? 8 : 1)
     k_route_rows(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int n_group,
                  int topk_group, int top_k, float rsf, int renorm, ExpSpecConsts kc, int32_t* __restrict__ ids,
                  float* __restrict__ wts) {
