@@ -100,11 +100,15 @@ uint8_t orc_e4m3_rne_satfinite(float x) {
 }
 
 /* Nearest E2M1 code to x, ties to the even mantissa bit, saturating to +-6; the
- * sign is kept, so a negative value that rounds to zero gives code 0x8. */
+ * sign is kept, so a negative value that rounds to zero gives code 0x8.  Every
+ * magnitude above 6 is the saturated code 7 outright: a nearest search alone
+ * loses it once |x| is so large (or infinite) that the distances to 4 and 6 are
+ * equal in double, where the even-code tie rule would pick 4. */
 uint8_t orc_e2m1_rne_sat(float x) {
     double a = fabs((double)x);
     int best = 0;
     double best_d = INFINITY;
+    if (a > 6.0) return (uint8_t)(signbit(x) ? 0xF : 0x7);
     for (int c = 0; c < 8; ++c) {
         double d = fabs(E2M1_MAGNITUDE[c] - a);
         if (d < best_d || (d == best_d && (c & 1) == 0)) {

@@ -412,6 +412,19 @@ def test_quantize_saturation_and_zero_block():
     assert oracle.e2m1_value(0xF) * oracle.e4m3_value(s[0, 0]) == -2688.0
 
 
+def test_e2m1_saturates_for_every_magnitude_above_six():
+    # "sat": any |x| > 6 is +-6 (code 7 / 0xF), however large, infinities included
+    for x in (6.0001, 7.0, 1e10, 2.0 ** 60, 1e30, 3.4e38, float("inf")):
+        assert oracle.e2m1_rne_sat(x) == 0x7, x
+        assert oracle.e2m1_rne_sat(-x) == 0xF, x
+    # a block whose amax saturates the scale at 448 and whose quotients are ~2^90
+    x = np.zeros((1, 16), np.float32)
+    x[0, :4] = [2.0 ** 100, 2.0 ** 99, -(2.0 ** 98), 1.0]
+    c, s = oracle.quantize_f32(x)
+    assert s[0, 0] == 0x7E
+    assert c[0, 0] == (0x7 | (0x7 << 4)) and c[0, 1] == 0xF  # codes 7, 7, 0xF, 0
+
+
 def test_quantize_roundtrip_of_representable_blocks():
     rng = np.random.default_rng(8)
     for _ in range(200):
