@@ -254,7 +254,7 @@ nvfp4moe_status launch_permute(const int32_t* ids, int T, int k, int E, int pad,
 // Linear layout (quantize_nvfp4): codes [M, K/2], scales [M, K/16].
 // Scatter layout (moe_forward W4A4): the token's codes go to the k permuted
 // rows of its pairs; scales go to the tcgen05 block-scale atom layout.
-template <bool SCATTER>
+template <bool SCATTER, bool BF16_UNIT>
 __global__ void __launch_bounds__(256)
     k_quantize(const uint16_t* __restrict__ x, int64_t M, int64_t K, float gs, uint8_t* __restrict__ codes,
                uint8_t* __restrict__ scales, const int32_t* __restrict__ row_of_pair, int k) {
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(256)
             f[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
         }
         uint32_t c0, c1;
-        const uint32_t sf = quantize_block16(f, gs, c0, c1);
+        const uint32_t sf = quantize_block16<BF16_UNIT>(f, gs, c0, c1);
         if (!SCATTER) {
             if (active) {
                 *reinterpret_cast<uint2*>(codes + m * (K / 2) + b * 8) = make_uint2(c0, c1);
@@ -316,7 +316,11 @@ __global__ void __launch_bounds__(256)
 nvfp4moe_status launch_quantize_linear(const uint16_t* x, int64_t M, int64_t K, float gs, uint8_t* codes,
                                        uint8_t* scales, cudaStream_t stream) {
     if (M == 0) return NVFP4MOE_OK;
-    k_quantize<false><<<(unsigned)ceil_div(M, 8), 256, 0, stream>>>(x, M, K, gs, codes, scales, nullptr, 1);
+    // gs == 1 (the unit global scale): the division-free form, same codes
+    if (gs == 1.0f)
+        k_quantize<false, true><<<(unsigned)ceil_div(M, 8), 256, 0, stream>>>(x, M, K, gs, codes, scales, nullptr, 1);
+    else
+        k_quantize<false, false><<<(unsigned)ceil_div(M, 8), 256, 0, stream>>>(x, M, K, gs, codes, scales, nullptr, 1);
     NVFP4MOE_CHECK_LAUNCH("quantize kernel");
     return NVFP4MOE_OK;
 }
@@ -324,7 +328,11 @@ nvfp4moe_status launch_quantize_linear(const uint16_t* x, int64_t M, int64_t K, 
 nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H, float gs, uint8_t* codes,
                                         uint8_t* scales, const int32_t* row_of_pair, int k, cudaStream_t stream) {
     if (T == 0) return NVFP4MOE_OK;
-    k_quantize<true><<<(unsigned)ceil_div(T, 8), 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k);
+    if (gs == 1.0f)
+        k_quantize<true, true><<<(unsigned)ceil_div(T, 8), 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k);
+    else
+        k_quantize<true, false><<<(unsigned)ceil_div(T, 8), 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair,
+                                                                             k);
     NVFP4MOE_CHECK_LAUNCH("quantize-scatter kernel");
     return NVFP4MOE_OK;
 }

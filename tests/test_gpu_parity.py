@@ -225,6 +225,40 @@ def test_quantize_exhaustive_bf16_ratios():
     assert np.array_equal(gsf, rs) and np.array_equal(gc, rc)
 
 
+def _blocks_below(anchor_bits, lo_bits, hi_bits):
+    """Blocks of 16 BF16 values: the anchor (the block's amax, which fixes its
+    scale) followed by every BF16 pattern in [lo_bits, hi_bits) with both signs,
+    fifteen per block (zeros pad the last)."""
+    mags = np.arange(lo_bits, hi_bits, dtype=np.uint32)
+    body = np.concatenate([mags, mags | 0x8000]).astype(np.uint16)
+    n = -(-len(body) // 15) * 15
+    body = np.concatenate([body, np.zeros(n - len(body), np.uint16)]).reshape(-1, 15)
+    return np.concatenate([np.full((body.shape[0], 1), anchor_bits, np.uint16), body], axis=1)
+
+
+def test_quantize_unit_global_every_scale_every_magnitude():
+    # gs == 1 takes the division-free quantiser; its codes must be the IEEE
+    # division's for every (x, scale) pair a block can hold.  Anchors: every
+    # positive BF16 amax from 2^-10 (scale 0 and the E4M3 subnormal scales) to
+    # 2^12 (past the 448 saturation), each with every BF16 magnitude in
+    # [amax/32, amax]; below that quotients are < 0.29 and fall to codes 0/0.5
+    # only through other anchors of the same scale.  Then a few anchors with every
+    # tiny BF16 value (FP32-subnormal range included) and huge anchors up to the
+    # BF16 maximum (saturated scale 448, codes 6).
+    parts = [_blocks_below(a, a - (5 << 7), a + 1) for a in range(117 << 7, (139 << 7) + 1)]
+    for a in (0x3A80, 0x3C00, 0x3F80, 0x4300, 0x4580):
+        parts.append(_blocks_below(a, 0x0001, 0x0A80))
+    for a in range(139 << 7, 0x7F80, 61):
+        parts.append(_blocks_below(a, a - (5 << 7), a + 1))
+    x = np.concatenate(parts)
+    pad = (-x.shape[0]) % 16
+    x = np.concatenate([x, np.zeros((pad, 16), np.uint16)]).reshape(-1, 256)
+    gc, gsf = _gpu_quant(x, 1.0)
+    rc, rs = oracle.quantize_bf16(x, 1.0)
+    assert np.array_equal(gsf, rs)
+    assert np.array_equal(gc, rc)
+
+
 # ---------------------------------------------------------------------------
 # the layer
 # ---------------------------------------------------------------------------
