@@ -1,9 +1,12 @@
 """B200 (sm_100a) routed-expert MoE layer with NVFP4 expert weights.
 
 Thin ctypes binding of ``libnvfp4moe.so`` (declared in ``include/nvfp4moe.h``).
-Every function takes ``torch`` tensors that already live on the GPU, checks
-nothing beyond what ctypes needs, and passes raw device pointers and sizes to
-the C ABI; all arithmetic runs in the library's CUDA kernels.  PyTorch is used
+Every function takes ``torch`` tensors that already live on the GPU and
+passes raw device pointers and sizes to the C ABI; all arithmetic runs in the
+library's CUDA kernels.  Before the call each tensor is checked for what a raw
+pointer cannot carry -- it is on a CUDA device, contiguous and at least as
+large as the header's layout for the given sizes -- so that a wrong argument
+raises here instead of becoming an out-of-bounds access on the GPU.  PyTorch is used
 for device memory and streams only.  There is no CPU fallback: if the shared
 library cannot be loaded every call raises.
 """
@@ -116,8 +119,25 @@ def load():
     return L
 
 
-def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+def _on_device(t) -> bool:
+    return t.is_cuda
+
+
+def _arg(t, name: str, nbytes: int | None = None, optional: bool = False):
+    """Device pointer of tensor ``t`` after the checks the C ABI cannot make: at
+    least ``nbytes`` bytes, contiguous, on a CUDA device.  ``None`` passes only
+    where the header allows NULL (``optional``)."""
+    if t is None:
+        if optional:
+            return None
+        raise NVFP4MoEError(1, f"{name} is required")
+    if nbytes is not None and t.numel() * t.element_size() < nbytes:
+        raise NVFP4MoEError(1, f"{name} holds {t.numel() * t.element_size()} bytes, needs {nbytes}")
+    if not t.is_contiguous():
+        raise NVFP4MoEError(1, f"{name} must be contiguous")
+    if not _on_device(t):
+        raise NVFP4MoEError(1, f"{name} must be a CUDA tensor (got {t.device})")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream):
@@ -147,10 +167,13 @@ def transcode_mxfp4_to_nvfp4(codes_in, e8m0_in, num_tensors, N, K, codes_out, e4
                              tensor_status_out, workspace, report: bool = True, stream=None, raise_on_error=False):
     """Returns (status, report dict or None).  With report=True the call is synchronous."""
     rep = TranscodeReport()
+    n = num_tensors * N * K
     st = load().transcode_mxfp4_to_nvfp4(
-        _ptr(codes_in), _ptr(e8m0_in), num_tensors, N, K, _ptr(codes_out), _ptr(e4m3_out), _ptr(global_scale_out),
-        _ptr(tensor_status_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
-        ctypes.byref(rep) if report else None, _stream(stream))
+        _arg(codes_in, "codes_in", n // 2), _arg(e8m0_in, "e8m0_in", n // 32), num_tensors, N, K,
+        _arg(codes_out, "codes_out", n // 2), _arg(e4m3_out, "e4m3_out", n // 16),
+        _arg(global_scale_out, "global_scale_out", 4 * num_tensors),
+        _arg(tensor_status_out, "tensor_status_out", 4 * num_tensors), _arg(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), ctypes.byref(rep) if report else None, _stream(stream))
     if st not in (0, 4, 5) or (raise_on_error and st != 0):
         _check(st)
     out = None
@@ -162,8 +185,10 @@ def transcode_mxfp4_to_nvfp4(codes_in, e8m0_in, num_tensors, N, K, codes_out, e4
 def moe_route(logits, bias, n_group, topk_group, top_k, routed_scaling_factor, renormalize, topk_ids, topk_weights,
               stream=None):
     T, E = logits.shape
-    _check(load().moe_route(_ptr(logits), _ptr(bias), T, E, n_group, topk_group, top_k, routed_scaling_factor,
-                            int(renormalize), _ptr(topk_ids), _ptr(topk_weights), _stream(stream)))
+    _check(load().moe_route(_arg(logits, "logits", 4 * T * E), _arg(bias, "bias", 4 * E, optional=True), T, E,
+                            n_group, topk_group, top_k, routed_scaling_factor, int(renormalize),
+                            _arg(topk_ids, "topk_ids", 4 * T * top_k), _arg(topk_weights, "topk_weights", 4 * T * top_k),
+                            _stream(stream)))
 
 
 def moe_router_topk_workspace_size(T) -> int:
@@ -174,19 +199,23 @@ def moe_router_topk(x_bf16, w_router, bias, n_group, topk_group, top_k, routed_s
                     logits_out, topk_ids, topk_weights, workspace, stream=None):
     T, H = x_bf16.shape
     E = w_router.shape[0]
-    _check(load().moe_router_topk(_ptr(x_bf16), _ptr(w_router), _ptr(bias), T, H, E, n_group, topk_group, top_k,
-                                  routed_scaling_factor, int(renormalize), _ptr(logits_out), _ptr(topk_ids),
-                                  _ptr(topk_weights), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                  _stream(stream)))
+    _check(load().moe_router_topk(_arg(x_bf16, "x_bf16", 2 * T * H), _arg(w_router, "w_router", 4 * E * H),
+                                  _arg(bias, "bias", 4 * E, optional=True), T, H, E, n_group, topk_group, top_k,
+                                  routed_scaling_factor, int(renormalize), _arg(logits_out, "logits_out", 4 * T * E),
+                                  _arg(topk_ids, "topk_ids", 4 * T * top_k),
+                                  _arg(topk_weights, "topk_weights", 4 * T * top_k), _arg(workspace, "workspace"),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def quantize_mxfp8(x, M, K, codes, e8m0_scales, stream=None):
-    _check(load().quantize_mxfp8(_ptr(x), M, K, _ptr(codes), _ptr(e8m0_scales), _stream(stream)))
+    _check(load().quantize_mxfp8(_arg(x, "x", 2 * M * K), M, K, _arg(codes, "codes", M * K),
+                                 _arg(e8m0_scales, "e8m0_scales", M * (K // 32)), _stream(stream)))
 
 
 def quantize_nvfp4(x_bf16, gs, codes, e4m3_scales, stream=None):
     M, K = x_bf16.shape
-    _check(load().quantize_nvfp4(_ptr(x_bf16), M, K, gs, _ptr(codes), _ptr(e4m3_scales), _stream(stream)))
+    _check(load().quantize_nvfp4(_arg(x_bf16, "x_bf16", 2 * M * K), M, K, gs, _arg(codes, "codes", M * K // 2),
+                                 _arg(e4m3_scales, "e4m3_scales", M * (K // 16)), _stream(stream)))
 
 
 def moe_permute_workspace_size(T, E, top_k, pad) -> int:
@@ -195,23 +224,29 @@ def moe_permute_workspace_size(T, E, top_k, pad) -> int:
 
 def moe_permute(topk_ids, E, pad, counts_out, pad_offsets_out, row_of_pair_out, workspace, stream=None):
     T, k = topk_ids.shape
-    _check(load().moe_permute(_ptr(topk_ids), T, E, k, pad, _ptr(counts_out), _ptr(pad_offsets_out),
-                              _ptr(row_of_pair_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                              _stream(stream)))
+    _check(load().moe_permute(_arg(topk_ids, "topk_ids", 4 * T * k), T, E, k, pad, _arg(counts_out, "counts_out", 4 * E),
+                              _arg(pad_offsets_out, "pad_offsets_out", 4 * (E + 1)),
+                              _arg(row_of_pair_out, "row_of_pair_out", 4 * T * k), _arg(workspace, "workspace"),
+                              workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def moe_permute_noalloc(topk_ids, E, pad, counts_out, pad_offsets_out, row_of_pair_out, stream=None):
     """moe_permute for callers that cannot allocate device memory: the scratch is
     a fixed 1 MiB device array inside the library (see include/nvfp4moe.h)."""
     T, k = topk_ids.shape
-    _check(load().moe_permute_noalloc(_ptr(topk_ids), T, E, k, pad, _ptr(counts_out), _ptr(pad_offsets_out),
-                                      _ptr(row_of_pair_out), _stream(stream)))
+    _check(load().moe_permute_noalloc(_arg(topk_ids, "topk_ids", 4 * T * k), T, E, k, pad,
+                                      _arg(counts_out, "counts_out", 4 * E),
+                                      _arg(pad_offsets_out, "pad_offsets_out", 4 * (E + 1)),
+                                      _arg(row_of_pair_out, "row_of_pair_out", 4 * T * k), _stream(stream)))
 
 
 def nvfp4_compact_scales(codes, e4m3_sf, rows, K, nib_out, row_exp_out, row_status_out, n_bad_out=None,
                          stream=None):
-    _check(load().nvfp4_compact_scales(_ptr(codes), _ptr(e4m3_sf), rows, K, _ptr(nib_out), _ptr(row_exp_out),
-                                       _ptr(row_status_out), _ptr(n_bad_out), _stream(stream)))
+    _check(load().nvfp4_compact_scales(_arg(codes, "codes", rows * K // 2), _arg(e4m3_sf, "e4m3_sf", rows * (K // 16)),
+                                       rows, K, _arg(nib_out, "nib_out", rows * (K // 64), optional=True),
+                                       _arg(row_exp_out, "row_exp_out", rows, optional=True),
+                                       _arg(row_status_out, "row_status_out", 4 * rows, optional=True),
+                                       _arg(n_bad_out, "n_bad_out", 4, optional=True), _stream(stream)))
 
 
 def moe_packed_weights_size(mode, E, H, I) -> int:
@@ -221,9 +256,21 @@ def moe_packed_weights_size(mode, E, H, I) -> int:
 def moe_pack_weights(mode, gate_codes, gate_sf, up_codes, up_sf, down_codes, down_sf, w_global, packed, stream=None):
     E, I = gate_codes.shape[0], gate_codes.shape[1]
     H = down_codes.shape[1]
-    w = ExpertWeights(gate_codes.data_ptr(), gate_sf.data_ptr(), up_codes.data_ptr(), up_sf.data_ptr(),
-                      down_codes.data_ptr(), down_sf.data_ptr(), w_global.data_ptr(), E, H, I)
-    _check(load().moe_pack_weights(mode, ctypes.byref(w), _ptr(packed), _stream(stream)))
+    n = E * I * H  # elements of each projection
+    ptrs = [_arg(gate_codes, "gate_codes", n // 2), _arg(gate_sf, "gate_sf", n // 16), _arg(up_codes, "up_codes", n // 2),
+            _arg(up_sf, "up_sf", n // 16), _arg(down_codes, "down_codes", n // 2), _arg(down_sf, "down_sf", n // 16),
+            _arg(w_global, "w_global", 4 * 3 * E)]
+    w = ExpertWeights(*[q.value for q in ptrs], E, H, I)
+    packed_ptr = _arg(packed, "packed", moe_packed_weights_size(mode, E, H, I))
+    _check(load().moe_pack_weights(mode, ctypes.byref(w), packed_ptr, _stream(stream)))
+
+
+def _layer_inputs(mode, x, router_logits, bias, packed_weights, T, H, I, E):
+    """Checked pointers of the layer's inputs: x [T, H] BF16, router_logits
+    [T, E] f32, bias [E] f32 or None, the packed weights of this mode."""
+    return (_arg(x, "x", 2 * T * H), _arg(router_logits, "router_logits", 4 * T * E),
+            _arg(bias, "bias", 4 * E, optional=True),
+            _arg(packed_weights, "packed_weights", moe_packed_weights_size(mode, E, H, I)))
 
 
 def moe_forward_workspace_size(mode, T, H, I, E, top_k) -> int:
@@ -235,11 +282,15 @@ def moe_forward(mode, x, router_logits, bias, packed_weights, act_global, T, H, 
                 stream=None):
     import torch
 
-    out_f32 = 1 if out.dtype == torch.float32 else 0
-    _check(load().moe_forward(mode, _ptr(x), _ptr(router_logits), _ptr(bias), _ptr(packed_weights), act_global, T, H,
-                              I, E, n_group, topk_group, top_k, routed_scaling_factor, int(renormalize),
-                              _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), out_f32,
-                              _ptr(topk_ids_out), _ptr(topk_weights_out), _stream(stream)))
+    out_f32 = 1 if out is not None and out.dtype == torch.float32 else 0
+    _check(load().moe_forward(mode, *_layer_inputs(mode, x, router_logits, bias, packed_weights, T, H, I, E),
+                              act_global, T, H, I, E, n_group, topk_group, top_k, routed_scaling_factor,
+                              int(renormalize), _arg(workspace, "workspace"),
+                              workspace.numel() * workspace.element_size(),
+                              _arg(out, "out", (4 if out_f32 else 2) * T * H), out_f32,
+                              _arg(topk_ids_out, "topk_ids_out", 4 * T * top_k, optional=True),
+                              _arg(topk_weights_out, "topk_weights_out", 4 * T * top_k, optional=True),
+                              _stream(stream)))
 
 
 def moe_forward_ex(mode, x, router_logits, bias, packed_weights, act_global_in, act_global_mid, T, H, I, E, n_group,
@@ -247,22 +298,28 @@ def moe_forward_ex(mode, x, router_logits, bias, packed_weights, act_global_in, 
                    topk_weights_out=None, stream=None):
     import torch
 
-    out_f32 = 1 if out.dtype == torch.float32 else 0
-    _check(load().moe_forward_ex(mode, _ptr(x), _ptr(router_logits), _ptr(bias), _ptr(packed_weights), act_global_in,
-                                 act_global_mid, T, H, I, E, n_group, topk_group, top_k, routed_scaling_factor,
-                                 int(renormalize), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                 _ptr(out), out_f32, _ptr(topk_ids_out), _ptr(topk_weights_out), _stream(stream)))
+    out_f32 = 1 if out is not None and out.dtype == torch.float32 else 0
+    _check(load().moe_forward_ex(mode, *_layer_inputs(mode, x, router_logits, bias, packed_weights, T, H, I, E),
+                                 act_global_in, act_global_mid, T, H, I, E, n_group, topk_group, top_k,
+                                 routed_scaling_factor, int(renormalize), _arg(workspace, "workspace"),
+                                 workspace.numel() * workspace.element_size(),
+                                 _arg(out, "out", (4 if out_f32 else 2) * T * H), out_f32,
+                                 _arg(topk_ids_out, "topk_ids_out", 4 * T * top_k, optional=True),
+                                 _arg(topk_weights_out, "topk_weights_out", 4 * T * top_k, optional=True),
+                                 _stream(stream)))
 
 
 def moe_forward_routed(mode, x, topk_ids, topk_weights, packed_weights, act_global, T, H, I, E, top_k, workspace, out,
                        stream=None):
     import torch
 
-    out_f32 = 1 if out.dtype == torch.float32 else 0
-    _check(load().moe_forward_routed(mode, _ptr(x), _ptr(topk_ids), _ptr(topk_weights), _ptr(packed_weights),
-                                     act_global, T, H, I, E, top_k, _ptr(workspace),
-                                     workspace.numel() * workspace.element_size(), _ptr(out), out_f32,
-                                     _stream(stream)))
+    out_f32 = 1 if out is not None and out.dtype == torch.float32 else 0
+    _check(load().moe_forward_routed(mode, _arg(x, "x", 2 * T * H), _arg(topk_ids, "topk_ids", 4 * T * top_k),
+                                     _arg(topk_weights, "topk_weights", 4 * T * top_k),
+                                     _arg(packed_weights, "packed_weights", moe_packed_weights_size(mode, E, H, I)),
+                                     act_global, T, H, I, E, top_k, _arg(workspace, "workspace"),
+                                     workspace.numel() * workspace.element_size(),
+                                     _arg(out, "out", (4 if out_f32 else 2) * T * H), out_f32, _stream(stream)))
 
 
 def nvfp4moe_set_trace_events(events) -> None:
