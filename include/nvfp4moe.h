@@ -192,7 +192,8 @@ nvfp4moe_status moe_router_topk(const uint16_t* x_bf16, const float* w_router, c
  *   topk_ids [T, top_k] i32 (each in [0, E), distinct within a row);
  *   counts_out [E] i32; pad_offsets_out [E+1] i32; row_of_pair_out [T*top_k]
  *   i32 (row of pair t*top_k + j); workspace of moe_permute_workspace_size().
- * Constraints: 1 <= E <= 1024, 1 <= top_k <= 32, pad in {1, 128}, T >= 0.     */
+ * Constraints: 1 <= E <= 1024, 1 <= top_k <= 32, pad in {1, 128}, T >= 0;
+ * T * top_k plus the padding rows fits int32 (else ERR_UNSUPPORTED_SHAPE).    */
 size_t moe_permute_workspace_size(int32_t T, int32_t E, int32_t top_k, int32_t pad);
 
 nvfp4moe_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t E, int32_t top_k, int32_t pad,
@@ -329,7 +330,9 @@ size_t moe_forward_workspace_size(nvfp4moe_mode mode, int32_t T, int32_t H, int3
  *   topk_ids_out [T, top_k] i32 and topk_weights_out [T, top_k] f32 are
  *   optional (NULL = not returned).
  * Constraints: as moe_route and moe_pack_weights; T >= 0 (0: no-op);
- * act_global finite and > 0; workspace_bytes >= moe_forward_workspace_size().
+ * act_global finite and > 0; workspace_bytes >= moe_forward_workspace_size();
+ * the permuted rows (T * top_k, plus up to 127 padding rows per expert in the
+ * tensor-core modes) fit int32 indices, else NVFP4MOE_ERR_UNSUPPORTED_SHAPE.
  * Device-side waits are bounded; a wait that gives up makes the call's next
  * synchronous status check return NVFP4MOE_ERR_TIMEOUT (see
  * nvfp4moe_check_device_status).                                              */

@@ -87,6 +87,15 @@ static nvfp4moe_status check_device() {
 // ---------------------------------------------------------------------------
 // workspace of moe_forward
 // ---------------------------------------------------------------------------
+// Permuted rows (pairs plus their padding) are addressed by int32 indices in
+// the routing plan (row_of_pair, pair_of_row): more than INT32_MAX of them is
+// refused up front (no device could hold their workspace anyway).
+static nvfp4moe_status check_row_count(int64_t rows) {
+    REQUIRE(rows <= INT32_MAX, NVFP4MOE_ERR_UNSUPPORTED_SHAPE,
+            "%lld permuted rows (T * top_k with padding) exceed the int32 row indices", (long long)rows);
+    return NVFP4MOE_OK;
+}
+
 struct ForwardLayout {
     int64_t P, rows_max, n_chunks, max_tiles;
     int pad;
@@ -330,6 +339,7 @@ nvfp4moe_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t E, int32
     REQUIRE(E >= 1 && E <= 1024, NVFP4MOE_ERR_UNSUPPORTED_SHAPE, "E=%d outside [1, 1024]", E);
     REQUIRE(top_k >= 1 && top_k <= 32 && top_k <= E, NVFP4MOE_ERR_UNSUPPORTED_SHAPE, "top_k=%d outside [1, 32]", top_k);
     REQUIRE(pad == 1 || pad == MTILE, NVFP4MOE_ERR_INVALID_ARG, "pad=%d must be 1 or %d", pad, MTILE);
+    RETURN_IF(check_row_count((int64_t)T * top_k + std::min<int64_t>(E, (int64_t)T * top_k) * (pad - 1)));
     REQUIRE(counts_out && pad_offsets_out && workspace, NVFP4MOE_ERR_INVALID_ARG, "null pointer");
     const size_t need = moe_permute_workspace_size(T, E, top_k, pad);
     REQUIRE(workspace_bytes >= need, NVFP4MOE_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes is below %zu",
@@ -429,6 +439,7 @@ static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, con
     const void* al16[] = {x, packed, workspace, out, logits, bias, ids_in, wts_in, ids_out, wts_out};
     for (const void* q : al16) REQUIRE(!q || aligned16(q), NVFP4MOE_ERR_ALIGNMENT, "a pointer is not 16-byte aligned");
     const ForwardLayout L = forward_layout(mode, T, H, I, E, top_k);
+    RETURN_IF(check_row_count(L.rows_max));
     REQUIRE(workspace_bytes >= (size_t)L.total, NVFP4MOE_ERR_WORKSPACE_TOO_SMALL,
             "workspace of %zu bytes is below the required %lld", workspace_bytes, (long long)L.total);
     RETURN_IF(check_device());

@@ -122,6 +122,27 @@ def test_forward_validation():
                            None, None, None) == 0
 
 
+def test_row_count_beyond_int32_indices_is_refused():
+    # permuted rows are int32 indices: T * top_k (+ padding) above INT32_MAX is
+    # refused before the workspace is looked at, however large it claims to be
+    lib = moe.load()
+    p = ctypes.c_void_p(4096)
+
+    def forward(mode, T, ws_bytes):
+        return lib.moe_forward(mode, p, p, None, p, 1.0, T, 4096, 2048, 256, 8, 4, 8, 2.827, 1, p, ws_bytes, p, 0,
+                               None, None, None)
+
+    big = (1 << 63) - 1
+    assert forward(1, 1 << 28, big) == 3  # W4A4: 2^31 pairs
+    assert forward(1, (1 << 28) - 64, big) == 3  # W4A4: below 2^31 pairs, above it with the 128-row padding
+    assert forward(0, 1 << 28, big) == 3  # W4A16: 2^31 pairs, no padding
+    assert forward(0, (1 << 28) - 1, 16) == 6  # 2^31 - 8 rows fit the indices: the small workspace is the error
+    # moe_permute: the same bound on pairs plus padding
+    assert lib.moe_permute(p, 1 << 28, 256, 8, 1, p, p, p, p, big, None) == 3
+    assert lib.moe_permute(p, (1 << 28) - 64, 256, 8, 128, p, p, p, p, big, None) == 3
+    assert lib.moe_permute(p, (1 << 28) - 1, 256, 8, 1, p, p, p, p, 16, None) == 6
+
+
 @pytest.mark.parametrize("g_in,g_mid", [(0.0, 1.0), (1.0, 0.0), (1.0, -2.0), (float("nan"), 1.0),
                                         (1.0, float("inf"))])
 def test_forward_ex_rejects_bad_activation_globals(g_in, g_mid):
