@@ -425,6 +425,22 @@ def test_e2m1_saturates_for_every_magnitude_above_six():
     assert c[0, 0] == (0x7 | (0x7 << 4)) and c[0, 1] == 0xF  # codes 7, 7, 0xF, 0
 
 
+def test_e2m1_keeps_the_sign_of_zero():
+    # reading: the sign survives rounding to zero (-0 and small negatives give
+    # code 0x8, as the hardware's satfinite conversion does); a block whose
+    # scale is zero is all 0x0
+    assert oracle.e2m1_rne_sat(0.0) == 0x0
+    assert oracle.e2m1_rne_sat(-0.0) == 0x8
+    assert oracle.e2m1_rne_sat(-0.2) == 0x8
+    x = np.zeros((2, 16), np.float32)
+    x[0, 0], x[0, 1], x[0, 2] = 6.0, -0.0, 0.0
+    x[1, :] = -0.0
+    c, s = oracle.quantize_f32(x)
+    assert s[0, 0] == 0x38  # E4M3 1.0
+    assert c[0, 0] == (0x7 | (0x8 << 4)) and c[0, 1] == 0x00
+    assert s[1, 0] == 0 and np.all(c[1] == 0)
+
+
 def test_quantize_roundtrip_of_representable_blocks():
     rng = np.random.default_rng(8)
     for _ in range(200):
@@ -446,6 +462,30 @@ def test_quantize_scale_against_torch_fp8():
     amax = np.abs(x.reshape(64, 16, 16)).max(-1)
     ref = torch.from_numpy((amax / np.float32(6)).astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert np.array_equal(s, ref)
+
+
+@pytest.mark.parametrize("gs", [0.37, 3.0, 1.0 / 64, 116.0])
+def test_quantize_scale_with_a_global_against_torch_fp8(gs):
+    # sf = E4M3((amax / 6) / gs): both divisions in IEEE FP32, the cast by torch
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((64, 256)) * np.exp(rng.uniform(-4, 4, (64, 1))) * gs).astype(np.float32)
+    c, s = oracle.quantize_f32(x, gs)
+    amax = np.abs(x.reshape(64, 16, 16)).max(-1)
+    v = (amax / np.float32(6)).astype(np.float32) / np.float32(gs)
+    assert np.all(v < 448)  # inside the cast's finite range
+    ref = torch.from_numpy(v.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(s, ref)
+
+
+@pytest.mark.parametrize("j", [-5, -1, 3, 7])
+def test_quantize_power_of_two_global_is_equivariant(j):
+    # scaling the block and the global by the same 2^j changes neither a scale
+    # byte nor a code: (amax 2^j / 6) / 2^j and x 2^j / (sf 2^j) are exact moves
+    rng = np.random.default_rng(6 + j)
+    x = (rng.standard_normal((32, 128)) * np.exp(rng.uniform(-3, 3, (32, 1)))).astype(np.float32)
+    c1, s1 = oracle.quantize_f32(x, 1.0)
+    cj, sj = oracle.quantize_f32(np.ldexp(x, j).astype(np.float32), 2.0 ** j)
+    assert np.array_equal(s1, sj) and np.array_equal(c1, cj)
 
 
 # ---------------------------------------------------------------------------
