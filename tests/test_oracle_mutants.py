@@ -55,6 +55,19 @@ MUTANTS = {
     "quantiser ignores the global": ("            v = v / gs;\n", ""),
     "router logits transposed operand": ("const double b = (double)w[(int64_t)e * H + h];",
                                          "const double b = (double)w[(int64_t)h * E + e];"),
+    "E8M0 bias": ("return ldexp(1.0, (int)byte - 127);", "return ldexp(1.0, (int)byte - 128);"),
+    "MXFP8 element scaling direction": ("orc_e4m3_rne_satfinite(ldexpf(xb[i], -X));", "orc_e4m3_rne_satfinite(ldexpf(xb[i], X));"),
+    "compact decode nibble order": ("const int n = (b & 1) ? (byte >> 4) : (byte & 15);",
+                                    "const int n = (b & 1) ? (byte & 15) : (byte >> 4);"),
+    "one group too few kept": ("for (int r = 0; r < topk_group; ++r) {", "for (int r = 0; r + 1 < topk_group; ++r) {"),
+    "renormalisation sum drops the last weight": ("for (int j = 0; j < top_k; ++j) S = S + s[",
+                                                  "for (int j = 0; j + 1 < top_k; ++j) S = S + s["),
+    "permutation offsets shifted": ("offsets[e + 1] = offsets[e] + counts[e];", "offsets[e + 1] = offsets[e] + counts[E - 1 - e];"),
+    "W4A16 intermediate not rounded to BF16": (
+        "for (int i = 0; i < I; ++i) a[i] = (double)orc_bf16_to_float(orc_float_to_bf16((float)a[i]));",
+        "for (int i = 0; i < I; ++i) a[i] = (double)(float)a[i];"),
+    "intermediate quantised with the input global": ("orc_quantize_f32(a32, 1, I, act_global_mid, aq, as);",
+                                                     "orc_quantize_f32(a32, 1, I, act_global, aq, as);"),
     "compact field sign": ("int lo = zero_of[2 * j] ? 15 : emax - e_of[2 * j];",
                            "int lo = zero_of[2 * j] ? 15 : e_of[2 * j] - emax;"),
 }
