@@ -1,5 +1,5 @@
 // tc_ptx.cuh -- inline-PTX wrappers for the sm_100a asynchronous machinery:
-// mbarriers (with bounded waits), TMA tiled and bulk copies (no multicast),
+// mbarriers (with bounded waits), TMA tiled and bulk copies (each to the issuing CTA only),
 // and the tcgen05 tensor-core / tensor-memory instructions.
 #pragma once
 
@@ -112,7 +112,7 @@ __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar_cluster_
 }
 
 // ---------------------------------------------------------------------------
-// TMA (cp.async.bulk), never with .multicast::cluster
+// TMA tiled and bulk copies, each into the issuing CTA's own shared memory
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int32_t x, int32_t y, uint64_t* bar) {
     asm volatile(

@@ -11,7 +11,7 @@
 // each CTA loads half of A's rows and half of B's rows, so a CTA moves 2/3 of the
 // operand bytes a single-CTA 128 x 256 tile needs for the same FLOPs.  Per CTA:
 //   warp 0      TMA producer: its A/B code half-tiles (SWIZZLE_128B tensor maps,
-//               never multicast) and block-scale atoms (1-D bulk copies) into a
+//               into its own CTA only) and block-scale atoms (1-D bulk copies) into a
 //               5-stage shared-memory ring guarded by mbarriers;
 //   warp 1      (even CTA) MMA issuer: four K=64 block-scaled M=256 x N=256 MMAs
 //               per stage into the pair's FP32 TMEM accumulators, nothing else
