@@ -644,12 +644,13 @@ def bench_transcode(torch, moe, args, P):
     return res
 
 
-def cpu_baseline(wl, d, args, steps=1):
-    """The oracle as it stands, on a bounded token sample of the same workload."""
+def cpu_baseline(wl, d, args, steps=1, per_thread=4):
+    """The oracle as it stands, on a bounded token sample of the same workload:
+    per_thread tokens for each host thread (4: ~10 s of oracle work)."""
     import oracle
 
     threads = oracle.num_threads()
-    n = args.cpu_sample_tokens or 4 * threads  # ~10 s of oracle work on a 16-thread host
+    n = args.cpu_sample_tokens or per_thread * threads
     toks = np.arange(n, dtype=np.int32)
     w = {k: d[k] for k in ("gate_codes", "gate_sf", "up_codes", "up_sf", "down_codes", "down_sf", "w_global")}
     t0 = time.perf_counter()
@@ -671,9 +672,12 @@ def run_reference(args, rank, world):
     import oracle
 
     oracle.build()
-    for _ in range(min(args.warmup, 1)):
-        cpu_baseline(wl, d, args)
-    vals = [cpu_baseline(wl, d, args) for _ in range(max(1, min(args.steps, 5)))]
+    # exactly W warm-up and K timed steps; past 6 steps in all each step samples
+    # one token per host thread (a few seconds), so the run stays within minutes
+    per_thread = 4 if args.warmup + args.steps <= 6 else 1
+    for _ in range(args.warmup):
+        cpu_baseline(wl, d, args, per_thread=per_thread)
+    vals = [cpu_baseline(wl, d, args, per_thread=per_thread) for _ in range(max(1, args.steps))]
     v = float(np.mean([r["value"] for r in vals]))
     dt = float(np.mean([r["seconds_per_step"] for r in vals]))
     out = {"impl": "reference", "metric": "MoE-layer tokens/s", "value": round(v, 3), "unit": "tokens/s",
