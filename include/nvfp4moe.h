@@ -305,7 +305,8 @@ typedef struct nvfp4moe_expert_weights {
 size_t moe_packed_weights_size(nvfp4moe_mode mode, int32_t E, int32_t H, int32_t I);
 
 /* One-time rearrangement of the checkpoint tensors into `packed` (device,
- * moe_packed_weights_size bytes, owned by the caller).  Values are unchanged:
+ * moe_packed_weights_size bytes, owned by the caller).  No counterpart on the
+ * pages: a layout step for the GEMMs below.  Values are unchanged:
  * the packed buffer holds the same codes, scales and globals, reordered (gate and
  * up rows interleaved, MMA scale-factor layout for W4A4, fragment order for
  * W4A16).  Constraints: H % 128 == 0, I % 128 == 0, E >= 1.
@@ -324,6 +325,13 @@ size_t moe_forward_workspace_size(nvfp4moe_mode mode, int32_t T, int32_t H, int3
 
 /* The whole layer: route -> permute -> (quantise) -> gate/up GEMM + SwiGLU
  * (+ requantise) -> down GEMM x routing weight -> weighted un-permute.
+ * Operation: out[t] = sum over the token's k routed experts j of
+ * g[t][j] * W_down,j (SiLU(W_gate,j x_t) * (W_up,j x_t)), the expert output and
+ * gate inside the saliency criterion of "patrickbdevaney/MiMo-V2.6-Flash-REAP50",
+ * "Pruning Method".  Mode NVFP4MOE_W4A4 quantises the activations to NVFP4 with
+ * a unit global (the default deployment); NVFP4MOE_W4A16 keeps them BF16 with
+ * the same FP4 weights ("AxionML / MiMo-V2.6-Flash-MOPD-NVFP4", "Usage",
+ * BF16-activation mode).
  *   x [T, H] BF16 bit patterns; router_logits [T, E] f32; bias [E] f32 or NULL;
  *   packed_weights from moe_pack_weights(mode, ...); out [T, H] BF16 bit
  *   patterns (out_is_fp32 == 0) or f32 (out_is_fp32 != 0).
@@ -343,7 +351,9 @@ nvfp4moe_status moe_forward(nvfp4moe_mode mode, const uint16_t* x, const float* 
                             int32_t out_is_fp32, int32_t* topk_ids_out, float* topk_weights_out, void* stream);
 
 /* Same layer from precomputed routing (topk_ids [T, top_k] i32, topk_weights
- * [T, top_k] f32, device): runs permute .. combine only. */
+ * [T, top_k] f32, device): runs permute .. combine only.  No counterpart on the
+ * pages: it lets the GEMM steps be driven without the router.  Arguments,
+ * constraints and errors as moe_forward's. */
 nvfp4moe_status moe_forward_routed(nvfp4moe_mode mode, const uint16_t* x, const int32_t* topk_ids,
                                    const float* topk_weights, const void* packed_weights, float act_global, int32_t T,
                                    int32_t H, int32_t I, int32_t E, int32_t top_k, void* workspace,
