@@ -317,6 +317,14 @@ def run_ours(args, rank, world, local_rank):
     import nvfp4_mixture_experts_grouped_b200 as moe
 
     torch.cuda.set_device(local_rank)
+    P = peaks()
+    wl = workload(args)
+    T = wl.T
+    # host-side input generation (about a minute at the 8K prefill) runs before
+    # the process group exists, so no collective waits on it
+    d = inputs.moe_inputs(wl)
+    w = {k: d[k] for k in ("gate_codes", "gate_sf", "up_codes", "up_sf", "down_codes", "down_sf", "w_global")}
+    d["x"], d["logits"] = rank_batch(wl, d, rank)
     dist = None
     if world > 1:
         import datetime
@@ -324,12 +332,6 @@ def run_ours(args, rank, world, local_rank):
         import torch.distributed as dist
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
-    P = peaks()
-    wl = workload(args)
-    T = wl.T
-    d = inputs.moe_inputs(wl)
-    w = {k: d[k] for k in ("gate_codes", "gate_sf", "up_codes", "up_sf", "down_codes", "down_sf", "w_global")}
-    d["x"], d["logits"] = rank_batch(wl, d, rank)
     mode = wl.mode
     packed, ws = make_layer(torch, moe, mode, w, T, wl)
     x = torch.from_numpy(d["x"].view(np.int16)).cuda().view(torch.bfloat16)
