@@ -148,7 +148,11 @@ nvfp4moe_status nvfp4_compact_scales(const uint8_t* codes, const uint8_t* e4m3_s
  *   topk_weights [T, top_k] f32.
  * Constraints: 1 <= E <= 1024, E % n_group == 0, 1 <= n_group <= 32,
  * 1 <= topk_group <= n_group, 1 <= top_k <= min(32, topk_group * E / n_group),
- * T >= 0 (0 is a no-op).  NaN logits give unspecified choices.               */
+ * T >= 0 (0 is a no-op).  NaN logits give unspecified choices.  Bias: a NaN
+ * entry makes that expert's c count as -inf (it ranks last), and a group whose
+ * score is NaN (biases of +inf and -inf in one group) scores -inf; infinite
+ * biases are otherwise ordinary values.  Whatever the bias, every id is in
+ * [0, E) and a token's ids are distinct.                                      */
 nvfp4moe_status moe_route(const float* logits, const float* bias, int32_t T, int32_t E, int32_t n_group,
                           int32_t topk_group, int32_t top_k, float routed_scaling_factor, int32_t renormalize,
                           int32_t* topk_ids, float* topk_weights, void* stream);
@@ -193,7 +197,9 @@ nvfp4moe_status moe_router_topk(const uint16_t* x_bf16, const float* w_router, c
  *   counts_out [E] i32; pad_offsets_out [E+1] i32; row_of_pair_out [T*top_k]
  *   i32 (row of pair t*top_k + j); workspace of moe_permute_workspace_size().
  * Constraints: 1 <= E <= 1024, 1 <= top_k <= 32, pad in {1, 128}, T >= 0;
- * T * top_k plus the padding rows fits int32 (else ERR_UNSUPPORTED_SHAPE).    */
+ * T * top_k plus the padding rows fits int32 (else ERR_UNSUPPORTED_SHAPE).
+ * An id outside [0, E) is skipped (not counted; its row_of_pair entry is left
+ * as it was); repeated ids within a row give unspecified rows.               */
 size_t moe_permute_workspace_size(int32_t T, int32_t E, int32_t top_k, int32_t pad);
 
 nvfp4moe_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t E, int32_t top_k, int32_t pad,
@@ -212,7 +218,9 @@ nvfp4moe_status moe_permute(const int32_t* topk_ids, int32_t T, int32_t E, int32
  *     with NVFP4MOE_ERR_UNSUPPORTED_SHAPE before anything is launched;
  *     T * top_k <= 65536 with E <= 256 always fits.
  *   - The first call on a device looks up the array's device address (with that
- *     device current); make that first call before any stream capture.
+ *     device current), and so does the first call in a new CUDA context of the
+ *     device (after cudaDeviceReset, say): make those calls before any stream
+ *     capture.
  *   - No call allocates or frees device memory.
  *   - All calls share the one array and it keeps the last call's contents:
  *     calls whose work overlaps on the GPU (other streams, other host threads)
@@ -353,7 +361,10 @@ nvfp4moe_status moe_forward(nvfp4moe_mode mode, const uint16_t* x, const float* 
 /* Same layer from precomputed routing (topk_ids [T, top_k] i32, topk_weights
  * [T, top_k] f32, device): runs permute .. combine only.  No counterpart on the
  * pages: it lets the GEMM steps be driven without the router.  Arguments,
- * constraints and errors as moe_forward's. */
+ * constraints and errors as moe_forward's.  A token's ids must lie in [0, E)
+ * and be distinct; the ids are device data, so this is checked on the device:
+ * a token that breaks the rule is computed with zero weights (its output row is
+ * 0) and the next nvfp4moe_check_device_status returns NVFP4MOE_ERR_INVALID_ARG. */
 nvfp4moe_status moe_forward_routed(nvfp4moe_mode mode, const uint16_t* x, const int32_t* topk_ids,
                                    const float* topk_weights, const void* packed_weights, float act_global, int32_t T,
                                    int32_t H, int32_t I, int32_t E, int32_t top_k, void* workspace,
@@ -391,8 +402,10 @@ nvfp4moe_status moe_forward_ex(nvfp4moe_mode mode, const uint16_t* x, const floa
 nvfp4moe_status nvfp4moe_set_trace_events(void* const* events, int32_t n_events);
 
 /* SYNCHRONOUS: waits for `stream`, then reads and clears the device error word
- * that bounded waits inside the GEMM kernels set when they give up.  Returns
- * NVFP4MOE_OK or NVFP4MOE_ERR_TIMEOUT. */
+ * that bounded waits inside the GEMM kernels set when they give up, and that
+ * moe_forward_routed sets for routing ids outside [0, E) or repeated within a
+ * token.  Returns NVFP4MOE_OK, NVFP4MOE_ERR_TIMEOUT (a wait gave up; reported
+ * first) or NVFP4MOE_ERR_INVALID_ARG (bad precomputed routing). */
 nvfp4moe_status nvfp4moe_check_device_status(void* stream);
 
 #ifdef __cplusplus

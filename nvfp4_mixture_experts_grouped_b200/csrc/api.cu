@@ -451,8 +451,7 @@ static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, con
     if (logits) {
         RETURN_IF(launch_route(logits, bias, T, E, n_group, topk_group, top_k, rsf, renorm, plan.ids, plan.wts, st));
     } else {
-        NVFP4MOE_CUDA(cudaMemcpyAsync(plan.ids, ids_in, (size_t)L.P * 4, cudaMemcpyDeviceToDevice, st));
-        NVFP4MOE_CUDA(cudaMemcpyAsync(plan.wts, wts_in, (size_t)L.P * 4, cudaMemcpyDeviceToDevice, st));
+        RETURN_IF(launch_check_routing(ids_in, wts_in, T, top_k, E, plan.ids, plan.wts, st));
     }
     trace(1, st);
     RETURN_IF(launch_permute(plan.ids, T, top_k, E, L.pad, plan, st));
@@ -540,7 +539,10 @@ nvfp4moe_status nvfp4moe_check_device_status(void* stream) {
     if (v != 0) {
         const int32_t zero = 0;
         NVFP4MOE_CUDA(cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice));
-        return fail(NVFP4MOE_ERR_TIMEOUT, "a bounded device-side wait gave up");
+        if (v & DEV_ERR_TIMEOUT) return fail(NVFP4MOE_ERR_TIMEOUT, "a bounded device-side wait gave up");
+        return fail(NVFP4MOE_ERR_INVALID_ARG,
+                    "precomputed routing named an expert outside [0, E) or one expert twice for a token; "
+                    "those tokens were computed with zero weights");
     }
     return NVFP4MOE_OK;
 }

@@ -36,8 +36,11 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 
-// Device error word set by bounded waits that give up (never trapped).
-enum : int32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1 };
+// Device error word, a set of bits (never trapped): DEV_ERR_TIMEOUT from bounded
+// waits that give up; DEV_ERR_BAD_ROUTING from precomputed routing that names an
+// expert outside [0, E) or one expert twice for a token.  Only the timeout bit
+// makes the other waits of a kernel give up too.
+enum : int32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_BAD_ROUTING = 2 };
 int32_t* device_error_word();  // device address of the word (current device)
 
 // Number of SMs of the current device (cached per device).

@@ -52,6 +52,10 @@ nvfp4moe_status launch_router_topk(const uint16_t* x, const float* w, const floa
 // permute.cu
 nvfp4moe_status launch_permute(const int32_t* ids, int T, int k, int E, int pad, RoutingPlan& plan,
                                cudaStream_t stream);
+// precomputed routing: copies ids / weights, replacing tokens with an id outside
+// [0, E) or a repeated id by experts 0..k-1 with weight 0 (DEV_ERR_BAD_ROUTING)
+nvfp4moe_status launch_check_routing(const int32_t* ids_in, const float* wts_in, int64_t T, int k, int E,
+                                     int32_t* ids, float* wts, cudaStream_t stream);
 nvfp4moe_status launch_quantize_linear(const uint16_t* x, int64_t M, int64_t K, float gs, uint8_t* codes,
                                        uint8_t* scales, cudaStream_t stream);
 nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H, float gs, uint8_t* codes,

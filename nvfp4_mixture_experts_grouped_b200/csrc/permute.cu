@@ -27,7 +27,10 @@ __global__ void __launch_bounds__(PERM_CHUNK)
     __syncthreads();
     const int t = blockIdx.x * PERM_CHUNK + threadIdx.x;
     if (t < T)
-        for (int j = 0; j < k; ++j) atomicAdd(&s_hist[ids[(int64_t)t * k + j]], 1);
+        for (int j = 0; j < k; ++j) {
+            const int e = ids[(int64_t)t * k + j];
+            if ((unsigned)e < (unsigned)E) atomicAdd(&s_hist[e], 1);  // ids outside [0, E) are skipped
+        }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[(int64_t)blockIdx.x * E + e] = s_hist[e];
 }
@@ -129,7 +132,10 @@ __global__ void __launch_bounds__(PERM_CHUNK)
     {
         const int t = t0 + lane;
         if (t < T)
-            for (int j = 0; j < k; ++j) atomicAdd(&s_wh[warp * E + ids[(int64_t)t * k + j]], 1);
+            for (int j = 0; j < k; ++j) {
+                const int e = ids[(int64_t)t * k + j];
+                if ((unsigned)e < (unsigned)E) atomicAdd(&s_wh[warp * E + e], 1);
+            }
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -150,7 +156,7 @@ __global__ void __launch_bounds__(PERM_CHUNK)
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         const int t = t0 + i;
-        if (lane < k && t < T) {
+        if (lane < k && t < T && (unsigned)eid[i] < (unsigned)E) {
             const int64_t p = (int64_t)t * k + lane;
             const int e = eid[i];
             const int r = s_wh[warp * E + e]++;
@@ -182,7 +188,10 @@ __global__ void __launch_bounds__(1024)
     const int p0 = min(P, warp * chunk), p1 = min(P, p0 + chunk);
     for (int i = tid; i < 32 * E; i += 1024) s_wc[i] = 0;
     __syncthreads();
-    for (int p = p0 + lane; p < p1; p += 32) atomicAdd(&s_wc[warp * E + ids[p]], 1);
+    for (int p = p0 + lane; p < p1; p += 32) {
+        const int e = ids[p];
+        if ((unsigned)e < (unsigned)E) atomicAdd(&s_wc[warp * E + e], 1);
+    }
     __syncthreads();
     int cnt = 0;
     if (tid < E) {
@@ -217,8 +226,9 @@ __global__ void __launch_bounds__(1024)
     __syncthreads();
     for (int b = p0; b < p1; b += 32) {
         const int p = b + lane;
-        const bool valid = p < p1;
-        const int e = valid ? ids[p] : -1 - lane;  // lanes past the chunk: keys of their own
+        const int id = p < p1 ? ids[p] : -1;
+        const bool valid = (unsigned)id < (unsigned)E;
+        const int e = valid ? id : -1 - lane;  // lanes past the chunk or with a bad id: keys of their own
         const unsigned same = __match_any_sync(0xffffffffu, e);
         if (valid) {
             const int row = s_poff[e] + s_wc[warp * E + e] + __popc(same & ((1u << lane) - 1u));
@@ -245,6 +255,46 @@ nvfp4moe_status launch_permute(const int32_t* ids, int T, int k, int E, int pad,
     NVFP4MOE_CHECK_LAUNCH("permute scan kernel");
     k_scatter<<<n_chunks, PERM_CHUNK, (PERM_WARPS + 1) * E * sizeof(int), stream>>>(ids, T, k, E, plan.chunk_counts, plan);
     NVFP4MOE_CHECK_LAUNCH("permute scatter kernel");
+    return NVFP4MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Precomputed routing (moe_forward_routed).  The permutation's counters and row
+// maps need every id in [0, E) and a token's ids distinct.  A token that breaks
+// either rule is replaced by experts 0..k-1 with weight 0 (its output row is 0)
+// and DEV_ERR_BAD_ROUTING is set in the device error word; the other tokens are
+// copied unchanged.  One thread per token.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    k_check_routing(const int32_t* __restrict__ ids_in, const float* __restrict__ wts_in, int64_t T, int k, int E,
+                    int32_t* __restrict__ ids, float* __restrict__ wts, int32_t* err) {
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T) return;
+    const int32_t* r = ids_in + t * k;
+    bool ok = true;
+    for (int j = 0; j < k; ++j) {
+        const int32_t e = r[j];
+        if (e < 0 || e >= E) ok = false;
+        for (int i = 0; i < j; ++i)
+            if (r[i] == e) ok = false;
+    }
+    for (int j = 0; j < k; ++j) {
+        ids[t * k + j] = ok ? r[j] : j;
+        wts[t * k + j] = ok ? wts_in[t * k + j] : 0.0f;
+    }
+    if (!ok) atomicOr(err, DEV_ERR_BAD_ROUTING);
+}
+
+nvfp4moe_status launch_check_routing(const int32_t* ids_in, const float* wts_in, int64_t T, int k, int E,
+                                     int32_t* ids, float* wts, cudaStream_t stream) {
+    if (T == 0) return NVFP4MOE_OK;
+    int32_t* err = device_error_word();
+    if (!err) {
+        set_error("device error word unavailable");
+        return NVFP4MOE_ERR_CUDA;
+    }
+    k_check_routing<<<(unsigned)ceil_div(T, 256), 256, 0, stream>>>(ids_in, wts_in, T, k, E, ids, wts, err);
+    NVFP4MOE_CHECK_LAUNCH("routing check kernel");
     return NVFP4MOE_OK;
 }
 

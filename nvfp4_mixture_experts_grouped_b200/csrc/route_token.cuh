@@ -52,6 +52,11 @@ __device__ __forceinline__ float sigmoid_spec(float x, const ExpSpecConsts& k) {
     return __fdiv_rn(e, __fadd_rn(1.0f, e));
 }
 
+// A NaN biased score (a NaN in the selection bias) or a NaN group score (an
+// infinite bias of each sign in one group) counts as -infinity, so every
+// comparison below is a total order and every chosen id is a real expert.
+__device__ __forceinline__ float nan_to_neg_inf(float v) { return v != v ? -INFINITY : v; }
+
 // (value desc, index asc) lexicographic "better than"
 __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
     return va > vb || (va == vb && ia < ib);
@@ -98,7 +103,7 @@ __device__ __forceinline__ void route_token_general(const float* __restrict__ lg
         const int e = lane + 32 * i;
         if (e < E) {
             s[i] = sigmoid_spec(s[i], kc);
-            c[i] = __fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f);
+            c[i] = nan_to_neg_inf(__fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f));
             const int g = e / gsz;
             s_c[g * (gsz + 1) + (e - g * gsz)] = c[i];
         } else {
@@ -117,7 +122,7 @@ __device__ __forceinline__ void route_token_general(const float* __restrict__ lg
         int i2 = -1;
         for (int j = 0; j < gsz; ++j)
             if (j != i1 && (i2 < 0 || gp[j] > gp[i2])) i2 = j;
-        score = i2 < 0 ? gp[i1] : __fadd_rn(gp[i1], gp[i2]);
+        score = nan_to_neg_inf(i2 < 0 ? gp[i1] : __fadd_rn(gp[i1], gp[i2]));
     }
     // keep topk_group groups
     uint32_t chosen = 0;
@@ -125,7 +130,7 @@ __device__ __forceinline__ void route_token_general(const float* __restrict__ lg
         float v = (lane < n_group && !((chosen >> lane) & 1u)) ? score : -INFINITY;
         int idx = (lane < n_group && !((chosen >> lane) & 1u)) ? lane : 0x7fffffff;
         warp_argmax(v, idx);
-        chosen |= 1u << idx;
+        if ((unsigned)idx < 32u) chosen |= 1u << idx;  // always: a group lane beats the -inf non-groups
     }
     // top_k experts inside the chosen groups
     uint32_t taken = 0;
@@ -143,6 +148,7 @@ __device__ __forceinline__ void route_token_general(const float* __restrict__ lg
             }
         }
         warp_argmax(v, idx);
+        idx = min(idx, E - 1);  // never taken: the kept groups hold >= top_k candidates, none NaN
         float sv = 0.0f;
         if ((idx & 31) == lane) {
             const int i = idx >> 5;
@@ -190,7 +196,7 @@ __device__ __forceinline__ void route_token_fast(const float* __restrict__ lg, c
         const int e = lane + 32 * i;
         if (e < E) {
             s[i] = sigmoid_spec(s[i], kc);
-            c[i] = __fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f);
+            c[i] = nan_to_neg_inf(__fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f));
             gbit[i] = 1u << (e / gsz);
         } else {
             s[i] = 0.0f;
@@ -210,7 +216,7 @@ __device__ __forceinline__ void route_token_fast(const float* __restrict__ lg, c
                 a = fmaxf(a, pa);
             }
             const int e = lane + 32 * i;
-            if ((lane & (gsz - 1)) == 0 && e < E) s_score[e / gsz] = __fadd_rn(a, b);
+            if ((lane & (gsz - 1)) == 0 && e < E) s_score[e / gsz] = nan_to_neg_inf(__fadd_rn(a, b));
         }
     } else {
         // per group: its rows, then the whole warp
@@ -230,7 +236,7 @@ __device__ __forceinline__ void route_token_fast(const float* __restrict__ lg, c
                 b = fmaxf(fminf(a, pa), fmaxf(b, pb));
                 a = fmaxf(a, pa);
             }
-            if (lane == 0) s_score[g] = __fadd_rn(a, b);
+            if (lane == 0) s_score[g] = nan_to_neg_inf(__fadd_rn(a, b));
         }
     }
     __syncwarp();
@@ -241,12 +247,14 @@ __device__ __forceinline__ void route_token_fast(const float* __restrict__ lg, c
         float v = (lane < n_group && !((chosen >> lane) & 1u)) ? score : -INFINITY;
         int idx = (lane < n_group && !((chosen >> lane) & 1u)) ? lane : 0x7fffffff;
         warp_argmax(v, idx);
-        chosen |= 1u << idx;
+        if ((unsigned)idx < 32u) chosen |= 1u << idx;  // always: a group lane beats the -inf non-groups
     }
-    // top_k experts inside the chosen groups
-    float cand[NPL];
+    // top_k experts inside the chosen groups; bit i of `cand`: register row i is
+    // still a candidate (a score of -inf is one too)
+    uint32_t cand = 0;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) cand[i] = (chosen & gbit[i]) ? c[i] : -INFINITY;
+    for (int i = 0; i < NPL; ++i)
+        if (chosen & gbit[i]) cand |= 1u << i;
     int my_id = 0;
     float my_s = 0.0f;
     for (int j = 0; j < top_k; ++j) {
@@ -255,12 +263,13 @@ __device__ __forceinline__ void route_token_fast(const float* __restrict__ lg, c
 #pragma unroll
         for (int i = 0; i < NPL; ++i) {
             const int e = lane + 32 * i;
-            if (cand[i] != -INFINITY && better(cand[i], e, v, idx)) {
-                v = cand[i];
+            if (((cand >> i) & 1u) && better(c[i], e, v, idx)) {
+                v = c[i];
                 idx = e;
             }
         }
         warp_argmax(v, idx);
+        idx = min(idx, E - 1);  // never taken: the kept groups hold >= top_k candidates, none NaN
         float sv = 0.0f;
         if ((idx & 31) == lane) {
             const int hit = idx >> 5;
@@ -268,7 +277,7 @@ __device__ __forceinline__ void route_token_fast(const float* __restrict__ lg, c
             for (int i = 0; i < NPL; ++i)
                 if (i == hit) {
                     sv = s[i];
-                    cand[i] = -INFINITY;
+                    cand &= ~(1u << i);
                 }
         }
         sv = __shfl_sync(0xffffffffu, sv, idx & 31);
@@ -286,7 +295,8 @@ __device__ __forceinline__ void route_token_fast(const float* __restrict__ lg, c
 }
 
 // Order-preserving int key of a float (larger float -> larger key; -0 and NaN
-// do not occur here: c = sigmoid + bias).  KEY_NONE is below every key.
+// do not occur here: c = sigmoid + bias with NaN taken as -inf).  KEY_NONE is
+// below every key, -inf's included.
 __device__ __forceinline__ int32_t okey(float v) {
     const int32_t b = __float_as_int(v);
     return b >= 0 ? b : b ^ 0x7FFFFFFF;
@@ -315,7 +325,7 @@ __device__ __forceinline__ void route_token_rows(const float* __restrict__ lg, c
         const int e = lane + 32 * i;
         if (e < E) {
             s[i] = sigmoid_spec(s[i], kc);
-            key[i] = okey(__fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f));
+            key[i] = okey(nan_to_neg_inf(__fadd_rn(s[i], bias ? __ldg(bias + e) : 0.0f)));
         } else {
             s[i] = 0.0f;
             key[i] = KEY_NONE;
@@ -333,7 +343,7 @@ __device__ __forceinline__ void route_token_rows(const float* __restrict__ lg, c
                 const int32_t m2 = __popc(holders) >= 2
                                        ? m1
                                        : __reduce_max_sync(0xffffffffu, (holders >> lane) & 1u ? KEY_NONE : key[g]);
-                if (lane == g) gkey = okey(__fadd_rn(okey_value(m1), okey_value(m2)));
+                if (lane == g) gkey = okey(nan_to_neg_inf(__fadd_rn(okey_value(m1), okey_value(m2))));
             }
     } else {
         for (int g = 0; g < n_group; ++g) {
@@ -352,7 +362,7 @@ __device__ __forceinline__ void route_token_rows(const float* __restrict__ lg, c
                 m2 = m1;
             else
                 m2 = __reduce_max_sync(0xffffffffu, (holders >> lane) & 1u ? b : a);
-            if (lane == g) gkey = okey(__fadd_rn(okey_value(m1), okey_value(m2)));
+            if (lane == g) gkey = okey(nan_to_neg_inf(__fadd_rn(okey_value(m1), okey_value(m2))));
         }
     }
     // keep topk_group groups: largest score, ties to the lower group
@@ -361,7 +371,7 @@ __device__ __forceinline__ void route_token_rows(const float* __restrict__ lg, c
         const bool elig = lane < n_group && !((chosen >> lane) & 1u);
         const int32_t m = __reduce_max_sync(0xffffffffu, elig ? gkey : KEY_NONE);
         const uint32_t g = __reduce_min_sync(0xffffffffu, elig && gkey == m ? (uint32_t)lane : 32u);
-        chosen |= 1u << g;
+        if (g < 32u) chosen |= 1u << g;  // always: every group's key is above KEY_NONE
     }
     // top_k experts inside the chosen groups: largest c, ties to the lower expert
 #pragma unroll
@@ -379,8 +389,9 @@ __device__ __forceinline__ void route_token_rows(const float* __restrict__ lg, c
                 li = i;
             }
         const int32_t m = __reduce_max_sync(0xffffffffu, lk);
-        const uint32_t idx =
+        uint32_t idx =
             __reduce_min_sync(0xffffffffu, lk == m && lk != KEY_NONE ? (uint32_t)(lane + 32 * li) : 0x7fffffffu);
+        idx = min(idx, (uint32_t)(E - 1));  // never taken: the kept groups hold >= top_k candidates
         float sv = 0.0f;
         if ((int)(idx & 31) == lane) {
             const int hit = (int)(idx >> 5);

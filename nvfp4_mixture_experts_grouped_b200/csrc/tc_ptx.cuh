@@ -64,7 +64,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity.  Gives up after about
-// `limit_cycles` SM clocks, records DEV_ERR_TIMEOUT in *err and returns false.
+// `limit_cycles` SM clocks, sets the timeout bit (1) of *err and returns false.
 template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err,
                                           long long limit_cycles = 4000000000LL) {
@@ -74,10 +74,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
         for (int i = 0; i < 256; ++i)
             if (mbar_try_wait<CLUSTER>(bar, parity)) return true;
         if (clock64() - t0 > limit_cycles) {
-            atomicExch(err, 1);
+            atomicOr(err, 1);
             return false;
         }
-        if (*(volatile int32_t*)err) return false;  // another thread already gave up
+        if (*(volatile int32_t*)err & 1) return false;  // another thread already gave up
     }
 }
 

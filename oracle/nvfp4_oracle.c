@@ -396,7 +396,9 @@ float orc_sigmoid_spec(float x) {
  * when absent) decides the selection; a group's score is the sum of its two
  * largest c (its largest when a group has one expert); groups and experts are
  * taken by descending value, ties to the lower index; the output order is the
- * selection order.  With renormalize: S = sum of the chosen s in output order
+ * selection order.  A NaN biased score, and a NaN group score (biases of +inf
+ * and -inf in one group), count as -inf, so the order is total and a selection
+ * always exists.  With renormalize: S = sum of the chosen s in output order
  * (sequential FP32 adds), w_j = (s_j / S) * rsf; without: w_j = s_j * rsf.   */
 void orc_route(const float* logits, const float* bias, int T, int E, int n_group, int topk_group, int top_k,
                float rsf, int renormalize, int32_t* topk_ids, float* topk_weights) {
@@ -411,6 +413,7 @@ void orc_route(const float* logits, const float* bias, int T, int E, int n_group
         for (int e = 0; e < E; ++e) {
             s[e] = orc_sigmoid_spec(lg[e]);
             c[e] = s[e] + (bias ? bias[e] : 0.0f);
+            if (isnan(c[e])) c[e] = -INFINITY; /* a NaN bias: the expert ranks last */
         }
         for (int g = 0; g < n_group; ++g) {
             int i1 = -1, i2 = -1;
@@ -419,6 +422,7 @@ void orc_route(const float* logits, const float* bias, int T, int E, int n_group
             for (int e = g * gsize; e < (g + 1) * gsize; ++e)
                 if (e != i1 && (i2 < 0 || c[e] > c[i2])) i2 = e;
             gscore[g] = (i2 < 0) ? c[i1] : c[i1] + c[i2];
+            if (isnan(gscore[g])) gscore[g] = -INFINITY; /* +inf and -inf biases in one group */
             gsel[g] = 0;
         }
         for (int r = 0; r < topk_group; ++r) {

@@ -143,6 +143,63 @@ def test_route_extreme_logits():
     assert np.array_equal(gi, ri) and np.array_equal(gw.view(np.uint32), rw.view(np.uint32))
 
 
+@pytest.mark.parametrize("E,ng,tg,k", [(256, 8, 4, 8), (128, 8, 4, 8), (16, 4, 2, 4), (96, 4, 2, 6), (60, 5, 2, 4)])
+def test_route_nan_and_infinite_bias(E, ng, tg, k):
+    # NaN bias entries rank their experts last (as -inf); +inf and -inf in one
+    # group give that group a -inf score.  Covers the row, segment and general
+    # per-token routines: ids, order and weight bits as the oracle, every id a
+    # distinct expert.
+    rng = np.random.default_rng(E + k)
+    T = 64
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    gsz = E // ng
+    for case in range(3):
+        bias = (rng.standard_normal(E) * 0.05).astype(np.float32)
+        if case == 0:
+            bias[rng.choice(E, E // 3, replace=False)] = np.nan
+        elif case == 1:
+            bias[:] = np.nan
+        else:
+            bias[0], bias[min(1, E - 1)] = np.inf, -np.inf
+            bias[gsz:2 * gsz] = np.nan
+        for kk in (k, min(32, tg * gsz)):
+            gi, gw = _gpu_route(logits, bias, ng, tg, kk, 2.827)
+            ri, rw = oracle.route(logits, bias, ng, tg, kk, 2.827)
+            assert np.array_equal(gi, ri)
+            assert np.array_equal(gw.view(np.uint32), rw.view(np.uint32))
+            assert gi.min() >= 0 and gi.max() < E
+            assert all(len(set(r)) == kk for r in gi.tolist())
+
+
+def test_routed_entry_point_reports_bad_ids():
+    # precomputed routing with an id outside [0, E), a negative id and a repeated
+    # id: those tokens come out as zero rows, the others exactly as with good
+    # routing, and the device status reports INVALID_ARG once, then clears
+    wl = inputs.WORKLOADS["tiny"]
+    d = inputs.moe_inputs(wl)
+    w = nvfp4_weights_from_inputs(d, False)
+    for mode in (moe.W4A4, moe.W4A16):
+        layer = GpuLayer(mode, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
+        x = bf16_tensor(d["x"])
+        good, ids, wts = layer.forward(x, dev(d["logits"]), out_fp32=True)
+        bad_ids = ids.clone()
+        bad_ids[3, 1] = wl.E
+        bad_ids[7, 2] = bad_ids[7, 0]
+        bad_ids[9, 0] = -1
+        out = torch.empty_like(good)
+        moe.moe_forward_routed(mode, x, bad_ids, wts, layer.packed, 1.0, wl.T, wl.H, wl.I, wl.E, wl.top_k, layer.ws,
+                               out)
+        with pytest.raises(moe.NVFP4MoEError) as ei:
+            moe.nvfp4moe_check_device_status()
+        assert ei.value.status == 1  # ERR_INVALID_ARG
+        moe.nvfp4moe_check_device_status()  # cleared
+        o, g = host(out), host(good)
+        bad = [3, 7, 9]
+        assert np.all(o[bad] == 0.0)
+        keep = [t for t in range(wl.T) if t not in bad]
+        assert np.array_equal(o[keep].view(np.uint32), g[keep].view(np.uint32))
+
+
 # ---------------------------------------------------------------------------
 # permutation
 # ---------------------------------------------------------------------------

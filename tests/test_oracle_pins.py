@@ -350,6 +350,39 @@ def test_route_bruteforce(E, ng, tg, k, ties):
         assert np.array_equal(w.view(np.uint32), rw.view(np.uint32))
 
 
+def test_route_nan_bias_ranks_like_minus_inf():
+    # The pages never make the selection bias NaN; the reading is that a NaN
+    # biased score counts as -inf.  -inf biases are ordinary values, which the
+    # brute force ranks directly, so NaN entries must give exactly the -inf
+    # routing, and a selection exists even when it has to take such experts.
+    rng = np.random.default_rng(5)
+    E, ng, tg = 16, 4, 2
+    logits = rng.standard_normal((40, E)).astype(np.float32)
+    bias = (rng.standard_normal(E) * 0.1).astype(np.float32)
+    bad = [1, 5, 6, 7, 12, 13, 14, 15]  # one whole group, most of another, one more
+    nan_b, inf_b = bias.copy(), bias.copy()
+    nan_b[bad], inf_b[bad] = np.nan, -np.inf
+    for k in (4, 8):  # k = 8: both kept groups whole, so -inf experts must be taken
+        ids, w = oracle.route(logits, nan_b, ng, tg, k, 2.827)
+        ids2, w2 = oracle.route(logits, inf_b, ng, tg, k, 2.827)
+        assert np.array_equal(ids, ids2) and np.array_equal(w.view(np.uint32), w2.view(np.uint32))
+        rid, rw = _route_bruteforce(logits, inf_b, ng, tg, k, 2.827, True)
+        assert np.array_equal(ids, rid) and np.array_equal(w.view(np.uint32), rw.view(np.uint32))
+        assert ids.min() >= 0 and ids.max() < E
+        assert all(len(set(r)) == k for r in ids.tolist())
+    # every bias NaN: all biased scores tie at -inf, so groups and experts go by index
+    ids, _ = oracle.route(logits, np.full(E, np.nan, np.float32), ng, tg, 4, 2.827)
+    assert np.array_equal(ids, np.tile(np.arange(4, dtype=np.int32), (40, 1)))
+    # +inf and -inf in one group: its score (inf + -inf) counts as -inf, so the
+    # group ranks as if both were -inf
+    pm, mm = bias.copy(), bias.copy()
+    pm[[0, 1]], mm[[0, 1]] = [np.inf, -np.inf], [-np.inf, -np.inf]
+    pm[2:4], mm[2:4] = -np.inf, -np.inf
+    a = oracle.route(logits, pm, ng, tg, 4, 2.827)[0]
+    b = oracle.route(logits, mm, ng, tg, 4, 2.827)[0]
+    assert not np.any(a // 4 == 0) and np.array_equal(a, b)
+
+
 def test_route_single_group_is_plain_topk_and_weights_sum():
     rng = np.random.default_rng(99)
     logits = rng.standard_normal((64, 32)).astype(np.float32)
