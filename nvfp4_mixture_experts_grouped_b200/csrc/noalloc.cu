@@ -5,8 +5,13 @@
 // workspace.  In host code `g_noalloc_permute_scratch` is only a host-side
 // stand-in for the device symbol, never a device address: handing it to a
 // kernel would fault, or silently touch the wrong memory where the GPU can reach
-// host memory.  The device address is therefore looked up once per device, with
-// that device current, through cudaGetSymbolAddress, and cached.
+// host memory.  The device address is therefore looked up with the device
+// current, through cudaGetSymbolAddress, and cached per device together with
+// the id of the CUDA context it belongs to: a new context on the device (after
+// cudaDeviceReset, for instance) holds the array at a new address, so a context
+// id that no longer matches makes the next call look the address up again.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -17,17 +22,47 @@ namespace nvfp4moe {
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) uint8_t g_noalloc_permute_scratch[NVFP4MOE_NOALLOC_SCRATCH_BYTES];
 
+// The driver's id of the calling thread's current context (unique for the
+// process's lifetime, unlike the context handle, which a new context can reuse);
+// 0 if there is none or the driver does not provide the calls.
+static unsigned long long current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
 static void* noalloc_scratch_address(nvfp4moe_status* st) {
     static std::mutex mu;
     static void* cache[64] = {};
+    static unsigned long long cache_ctx[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         set_error("moe_permute_noalloc: no usable current CUDA device");
         *st = NVFP4MOE_ERR_CUDA;
         return nullptr;
     }
+    const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lk(mu);
-    if (!cache[dev]) {
+    if (!cache[dev] || ctx == 0 || cache_ctx[dev] != ctx) {
+        // also makes the device's primary context current if no context was
         void* p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_permute_scratch);
         if (e != cudaSuccess || !p) {
@@ -37,6 +72,7 @@ static void* noalloc_scratch_address(nvfp4moe_status* st) {
             return nullptr;
         }
         cache[dev] = p;
+        cache_ctx[dev] = ctx != 0 ? ctx : current_context_id();
     }
     *st = NVFP4MOE_OK;
     return cache[dev];

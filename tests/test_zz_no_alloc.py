@@ -1,9 +1,9 @@
 """moe_permute_noalloc: the permutation for callers that cannot allocate device
 memory (a plugin handed only its inputs and outputs, or a path where cudaMalloc
 may not run).  Its scratch is a fixed device array inside the library, so it is
-checked through the C ABI against moe_permute with a caller workspace, on two
-calls in a row with different inputs (the array keeps the previous call's
-contents, which must not leak into the next result).  This file sorts last so
+checked through the C ABI against moe_permute with a caller workspace, on
+several calls in a row with different inputs (the array keeps the previous
+call's contents, which must not leak into the next result).  This file sorts last so
 that a run stopping at the first failure has already run every other test."""
 import numpy as np
 import pytest
@@ -39,9 +39,15 @@ def _no_alloc(ids, E, pad):
 
 def test_no_alloc_permute_matches_workspace_entry_point_twice():
     rng = np.random.default_rng(2024)
-    # first call: a large request; second call: a smaller one that reuses the
-    # same scratch array with stale contents from the first
-    for T, E, k, pad in ((8192, 256, 8, 128), (300, 64, 6, 1)):
+    # calls in a row on the one scratch array, each finding the previous call's
+    # contents there: a large request (the three-kernel path, which writes and
+    # reads back per-chunk counts), a small one (the one-CTA path), then two more
+    # large ones with other ids, expert counts and padding, so that the path that
+    # reads back scratch it wrote also runs on stale contents
+    cases = ((8192, 256, 8, 128), (300, 64, 6, 1), (4096, 256, 8, 128), (20000, 128, 3, 1))
+    for T, E, k, pad in cases:
+        assert moe.moe_permute_workspace_size(T, E, k, pad) <= (1 << 20)
+    for T, E, k, pad in cases:
         ids = _ids(rng, T, E, k)
         ref = _with_workspace(ids, E, pad)
         got = _no_alloc(ids, E, pad)
