@@ -178,8 +178,11 @@ int orc_transcode(const uint8_t* codes_in, const uint8_t* e8m0, int64_t num_tens
                   int64_t* report) {
     const int64_t blocks = N * K / 32;
     int worst = 0;
-    report[0] = report[1] = report[2] = report[3] = 0;
+    int64_t r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+    /* tensors are independent: one per thread, counts summed at the end */
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : r0, r1, r2, r3) reduction(max : worst)
     for (int64_t t = 0; t < num_tensors; ++t) {
+        int64_t zero_blocks = 0;
         const uint8_t* c = codes_in + t * blocks * 16;
         const uint8_t* s = e8m0 + t * blocks;
         uint8_t* so = e4m3_out + t * blocks * 2;
@@ -192,7 +195,7 @@ int orc_transcode(const uint8_t* codes_in, const uint8_t* e8m0, int64_t num_tens
             for (int i = 0; i < 32; ++i)
                 if (nibble(c + b * 16, i) & 7) zero = 0;
             if (zero) {
-                report[1]++;
+                zero_blocks++;
                 continue;
             }
             if (s[b] == 0xFF) {
@@ -204,7 +207,8 @@ int orc_transcode(const uint8_t* codes_in, const uint8_t* e8m0, int64_t num_tens
             if (!have || k > kmax) kmax = k;
             have = 1;
         }
-        report[0] += blocks;
+        r0 += blocks;
+        r1 += zero_blocks;
 
         int status = 0;
         if (nan_seen) status = 2;
@@ -213,7 +217,8 @@ int orc_transcode(const uint8_t* codes_in, const uint8_t* e8m0, int64_t num_tens
             memset(so, 0, (size_t)(blocks * 2));
             global_out[t] = 0.0f;
             tensor_status[t] = status;
-            report[status == 1 ? 2 : 3]++;
+            if (status == 1) r2++;
+            else r3++;
             if (status > worst) worst = status;
             continue;
         }
@@ -234,6 +239,7 @@ int orc_transcode(const uint8_t* codes_in, const uint8_t* e8m0, int64_t num_tens
         global_out[t] = ldexpf(1.0f, g);
         tensor_status[t] = 0;
     }
+    report[0] = r0, report[1] = r1, report[2] = r2, report[3] = r3;
     return worst;
 }
 
@@ -622,94 +628,189 @@ static void decode_row(const uint8_t* codes, const uint8_t* sf, double global, i
         out[k] = orc_e2m1_value(nibble(codes, k)) * orc_e4m3_value(sf[k / 16]) * global;
 }
 
+/* The layer input of one token as float64 values: its NVFP4 (mode 1) or MXFP8
+ * (mode 3) quantisation decoded, or its BF16 values (mode 0). */
+static void layer_input(int mode, const uint16_t* xt, int H, float act_global, double* xd) {
+    if (mode == 3) {
+        uint8_t* xq = (uint8_t*)malloc((size_t)H);
+        uint8_t* xs = (uint8_t*)malloc((size_t)H / 32);
+        orc_quantize_mxfp8_bf16(xt, 1, H, xq, xs);
+        for (int h = 0; h < H; ++h) xd[h] = mxfp8_value(xq, xs, h);
+        free(xq);
+        free(xs);
+    } else if (mode == 1) {
+        uint8_t* xq = (uint8_t*)malloc((size_t)H / 2);
+        uint8_t* xs = (uint8_t*)malloc((size_t)H / 16);
+        orc_quantize_bf16(xt, 1, H, act_global, xq, xs);
+        for (int h = 0; h < H; ++h)
+            xd[h] = orc_e2m1_value(nibble(xq, h)) * orc_e4m3_value(xs[h / 16]) * (double)act_global;
+        free(xq);
+        free(xs);
+    } else {
+        for (int h = 0; h < H; ++h) xd[h] = (double)orc_bf16_to_float(xt[h]);
+    }
+}
+
+/* The SwiGLU output a[I] of one (token, expert) pair as the down projection
+ * sees it: requantised to MXFP8 (mode 3) or NVFP4 with act_global_mid (mode 1),
+ * or rounded to BF16 (mode 0). */
+static void down_input(int mode, int I, float act_global_mid, double* a) {
+    float* a32 = (float*)malloc(sizeof(float) * (size_t)I);
+    if (mode == 3) {
+        uint8_t* mq = (uint8_t*)malloc((size_t)I);
+        uint8_t* ms = (uint8_t*)malloc((size_t)I / 32);
+        for (int i = 0; i < I; ++i) a32[i] = (float)a[i];
+        orc_quantize_mxfp8_f32(a32, 1, I, mq, ms);
+        for (int i = 0; i < I; ++i) a[i] = mxfp8_value(mq, ms, i);
+        free(mq);
+        free(ms);
+    } else if (mode == 1) {
+        uint8_t* aq = (uint8_t*)malloc((size_t)I / 2);
+        uint8_t* as = (uint8_t*)malloc((size_t)I / 16);
+        for (int i = 0; i < I; ++i) a32[i] = (float)a[i];
+        orc_quantize_f32(a32, 1, I, act_global_mid, aq, as);
+        for (int i = 0; i < I; ++i)
+            a[i] = orc_e2m1_value(nibble(aq, i)) * orc_e4m3_value(as[i / 16]) * (double)act_global_mid;
+        free(aq);
+        free(as);
+    } else {
+        for (int i = 0; i < I; ++i) a[i] = (double)orc_bf16_to_float(orc_float_to_bf16((float)a[i]));
+    }
+    free(a32);
+}
+
+/* Dot products of one decoded weight row w[K] with the rows v[q * ld .. + K) of
+ * n operands: out[q] = sum_k v[q][k] * w[k], each summed in k order (four
+ * operands at a time, so their sums proceed side by side).  */
+static void row_dots(const double* w, const double* const* v, int n, int64_t K, double* out) {
+    int q = 0;
+    for (; q + 4 <= n; q += 4) {
+        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+        const double *v0 = v[q], *v1 = v[q + 1], *v2 = v[q + 2], *v3 = v[q + 3];
+        for (int64_t k = 0; k < K; ++k) {
+            s0 += v0[k] * w[k];
+            s1 += v1[k] * w[k];
+            s2 += v2[k] * w[k];
+            s3 += v3[k] * w[k];
+        }
+        out[q] = s0, out[q + 1] = s1, out[q + 2] = s2, out[q + 3] = s3;
+    }
+    for (; q < n; ++q) {
+        double s0 = 0.0;
+        for (int64_t k = 0; k < K; ++k) s0 += v[q][k] * w[k];
+        out[q] = s0;
+    }
+}
+
 /* The layer with separate activation global scales for the layer input
  * (act_global) and the down-projection input (act_global_mid): [P1] "Why a unit
  * activation scale" compares calibrated per-layer scales, the down-projection
- * input's scale capped at 2688, and a unit scale everywhere. */
+ * input's scale capped at 2688, and a unit scale everywhere.
+ * Evaluation order: tokens are routed and their inputs quantised first; then,
+ * expert by expert, every weight row is decoded once and applied to all of the
+ * sample's pairs routed to that expert; each output element is the same float64
+ * sum, in the same k order, as a token-by-token evaluation would form.  The
+ * sample is processed in batches of at most 512 tokens (bounded memory). */
 void orc_moe_layer2(int mode, const uint16_t* x, const float* logits, const float* bias, const uint8_t* gate_codes,
                     const uint8_t* gate_sf, const uint8_t* up_codes, const uint8_t* up_sf, const uint8_t* down_codes,
                     const uint8_t* down_sf, const float* w_global, float act_global, float act_global_mid, int T,
                     int H, int I, int E, int n_group, int topk_group, int top_k, float rsf, int renormalize,
                     const int32_t* tokens, int n_tokens, double* out) {
     (void)T;
+    const int BATCH = 512;
+    int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)BATCH * top_k);
+    float* wts = (float*)malloc(sizeof(float) * (size_t)BATCH * top_k);
+    double* xd = (double*)malloc(sizeof(double) * (size_t)BATCH * H);
+    double* abuf = (double*)malloc(sizeof(double) * (size_t)BATCH * top_k * I);  /* per pair, SwiGLU output */
+    double* ybuf = (double*)malloc(sizeof(double) * (size_t)BATCH * top_k * H);  /* per pair, expert output */
+    int* pair_list = (int*)malloc(sizeof(int) * (size_t)BATCH * top_k);
+    int* first = (int*)malloc(sizeof(int) * (size_t)(E + 1));
+    for (int b0 = 0; b0 < n_tokens; b0 += BATCH) {
+        const int nb = n_tokens - b0 < BATCH ? n_tokens - b0 : BATCH;
+        const int np = nb * top_k;
 #pragma omp parallel for schedule(dynamic, 1)
-    for (int it = 0; it < n_tokens; ++it) {
-        const int t = tokens[it];
-        int32_t ids[64];
-        float wts[64];
-        orc_route(logits + (int64_t)t * E, bias, 1, E, n_group, topk_group, top_k, rsf, renormalize, ids, wts);
-
-        double* xd = (double*)malloc(sizeof(double) * (size_t)H);
-        double* wrow = (double*)malloc(sizeof(double) * (size_t)(H > I ? H : I));
-        double* a = (double*)malloc(sizeof(double) * (size_t)I);
-        float* a32 = (float*)malloc(sizeof(float) * (size_t)I);
-        uint8_t* aq = (uint8_t*)malloc((size_t)I / 2);
-        uint8_t* as = (uint8_t*)malloc((size_t)I / 16);
-        double* o = out + (int64_t)it * H;
-        for (int h = 0; h < H; ++h) o[h] = 0.0;
-
-        if (mode == 3) {
-            uint8_t* xq = (uint8_t*)malloc((size_t)H);
-            uint8_t* xs = (uint8_t*)malloc((size_t)H / 32);
-            orc_quantize_mxfp8_bf16(x + (int64_t)t * H, 1, H, xq, xs);
-            for (int h = 0; h < H; ++h) xd[h] = mxfp8_value(xq, xs, h);
-            free(xq);
-            free(xs);
-        } else if (mode == 1) {
-            uint8_t* xq = (uint8_t*)malloc((size_t)H / 2);
-            uint8_t* xs = (uint8_t*)malloc((size_t)H / 16);
-            orc_quantize_bf16(x + (int64_t)t * H, 1, H, act_global, xq, xs);
-            for (int h = 0; h < H; ++h)
-                xd[h] = orc_e2m1_value(nibble(xq, h)) * orc_e4m3_value(xs[h / 16]) * (double)act_global;
-            free(xq);
-            free(xs);
-        } else {
-            for (int h = 0; h < H; ++h) xd[h] = (double)orc_bf16_to_float(x[(int64_t)t * H + h]);
+        for (int it = 0; it < nb; ++it) {
+            const int t = tokens[b0 + it];
+            orc_route(logits + (int64_t)t * E, bias, 1, E, n_group, topk_group, top_k, rsf, renormalize,
+                      ids + (int64_t)it * top_k, wts + (int64_t)it * top_k);
+            layer_input(mode, x + (int64_t)t * H, H, act_global, xd + (int64_t)it * H);
         }
-
-        for (int j = 0; j < top_k; ++j) {
-            const int e = ids[j];
+        /* the batch's pairs (it * top_k + j) grouped by expert */
+        for (int e = 0; e <= E; ++e) first[e] = 0;
+        for (int q = 0; q < np; ++q) first[ids[q] + 1]++;
+        for (int e = 0; e < E; ++e) first[e + 1] += first[e];
+        {
+            int* fill = (int*)malloc(sizeof(int) * (size_t)E);
+            for (int e = 0; e < E; ++e) fill[e] = first[e];
+            for (int q = 0; q < np; ++q) pair_list[fill[ids[q]]++] = q;
+            free(fill);
+        }
+        for (int e = 0; e < E; ++e) {
+            const int n = first[e + 1] - first[e];
+            if (n == 0) continue;
+            const int* pl = pair_list + first[e];
             const double gg = w_global[e * 3 + 0], gu = w_global[e * 3 + 1], gd = w_global[e * 3 + 2];
-            for (int i = 0; i < I; ++i) {
-                const int64_t r = (int64_t)e * I + i;
-                double g = 0.0, u = 0.0;
-                decode_row(gate_codes + r * (H / 2), gate_sf + r * (H / 16), gg, H, wrow);
-                for (int h = 0; h < H; ++h) g += xd[h] * wrow[h];
-                decode_row(up_codes + r * (H / 2), up_sf + r * (H / 16), gu, H, wrow);
-                for (int h = 0; h < H; ++h) u += xd[h] * wrow[h];
-                a[i] = silu(g) * u;
+            const double** xv = (const double**)malloc(sizeof(double*) * (size_t)n);
+            const double** av = (const double**)malloc(sizeof(double*) * (size_t)n);
+            for (int q = 0; q < n; ++q) {
+                xv[q] = xd + (int64_t)(pl[q] / top_k) * H;
+                av[q] = abuf + (int64_t)pl[q] * I;
             }
-            if (mode == 3) {
-                uint8_t* mq = (uint8_t*)malloc((size_t)I);
-                uint8_t* ms = (uint8_t*)malloc((size_t)I / 32);
-                for (int i = 0; i < I; ++i) a32[i] = (float)a[i];
-                orc_quantize_mxfp8_f32(a32, 1, I, mq, ms);
-                for (int i = 0; i < I; ++i) a[i] = mxfp8_value(mq, ms, i);
-                free(mq);
-                free(ms);
-            } else if (mode == 1) {
-                for (int i = 0; i < I; ++i) a32[i] = (float)a[i];
-                orc_quantize_f32(a32, 1, I, act_global_mid, aq, as);
-                for (int i = 0; i < I; ++i)
-                    a[i] = orc_e2m1_value(nibble(aq, i)) * orc_e4m3_value(as[i / 16]) * (double)act_global_mid;
-            } else {
-                for (int i = 0; i < I; ++i) a[i] = (double)orc_bf16_to_float(orc_float_to_bf16((float)a[i]));
+#pragma omp parallel
+            {
+                double* wrow = (double*)malloc(sizeof(double) * (size_t)(H > I ? H : I));
+                double* gv = (double*)malloc(sizeof(double) * (size_t)n);
+                double* uv = (double*)malloc(sizeof(double) * (size_t)n);
+#pragma omp for schedule(dynamic, 16)
+                for (int i = 0; i < I; ++i) {
+                    const int64_t r = (int64_t)e * I + i;
+                    decode_row(gate_codes + r * (H / 2), gate_sf + r * (H / 16), gg, H, wrow);
+                    row_dots(wrow, xv, n, H, gv);
+                    decode_row(up_codes + r * (H / 2), up_sf + r * (H / 16), gu, H, wrow);
+                    row_dots(wrow, xv, n, H, uv);
+                    for (int q = 0; q < n; ++q) {
+                        double* a = abuf + (int64_t)pl[q] * I;
+                        const double g = gv[q], u = uv[q];
+                        a[i] = silu(g) * u;
+                    }
+                }
+#pragma omp for schedule(dynamic, 1)
+                for (int q = 0; q < n; ++q) down_input(mode, I, act_global_mid, abuf + (int64_t)pl[q] * I);
+#pragma omp for schedule(dynamic, 16)
+                for (int h = 0; h < H; ++h) {
+                    const int64_t r = (int64_t)e * H + h;
+                    decode_row(down_codes + r * (I / 2), down_sf + r * (I / 16), gd, I, wrow);
+                    row_dots(wrow, av, n, I, gv);
+                    for (int q = 0; q < n; ++q) ybuf[(int64_t)pl[q] * H + h] = gv[q];
+                }
+                free(wrow);
+                free(gv);
+                free(uv);
             }
-            for (int h = 0; h < H; ++h) {
-                const int64_t r = (int64_t)e * H + h;
-                decode_row(down_codes + r * (I / 2), down_sf + r * (I / 16), gd, I, wrow);
-                double y = 0.0;
-                for (int i = 0; i < I; ++i) y += a[i] * wrow[i];
-                o[h] += (double)wts[j] * y;
+            free(xv);
+            free(av);
+        }
+        /* out = sum_j g_{t,j} y_j, slot order */
+#pragma omp parallel for schedule(static)
+        for (int it = 0; it < nb; ++it) {
+            double* o = out + (int64_t)(b0 + it) * H;
+            for (int h = 0; h < H; ++h) o[h] = 0.0;
+            for (int j = 0; j < top_k; ++j) {
+                const int64_t q = (int64_t)it * top_k + j;
+                for (int h = 0; h < H; ++h) {
+                    const double y = ybuf[q * H + h];
+                    o[h] += (double)wts[q] * y;
+                }
             }
         }
-        free(xd);
-        free(wrow);
-        free(a);
-        free(a32);
-        free(aq);
-        free(as);
     }
+    free(ids);
+    free(wts);
+    free(xd);
+    free(abuf);
+    free(ybuf);
+    free(pair_list);
+    free(first);
 }
 
 /* One activation global scale for both quantisations (the pages' unit scale). */

@@ -39,7 +39,7 @@ MUTANTS = {
     "gate and up swapped": ("a[i] = silu(g) * u;", "a[i] = silu(u) * g;"),
     "down weight row index": ("const int64_t r = (int64_t)e * H + h;", "const int64_t r = (int64_t)e * H + (H - 1 - h);"),
     "block scale index": ("orc_e4m3_value(sf[k / 16]) * global;", "orc_e4m3_value(sf[k / 32]) * global;"),
-    "combine drops the routing weight": ("o[h] += (double)wts[j] * y;", "o[h] += y;"),
+    "combine drops the routing weight": ("o[h] += (double)wts[q] * y;", "o[h] += y;"),
     "permutation not stable": ("        for (int64_t p = 0; p < P; ++p)\n            if (topk_ids[p] == e) {",
                                "        for (int64_t p = P - 1; p >= 0; --p)\n            if (topk_ids[p] == e) {"),
     "MXFP8 scale exponent": ("X = ex - 1 - 8;", "X = ex - 1 - 7;"),
