@@ -6,8 +6,11 @@ permutation, NVFP4 activation quantisation (unit global), gate/up grouped GEMM
 + SwiGLU (+ requantisation), down grouped GEMM x routing weight, weighted
 un-permute.  Default workload: the 8192-token W4A4 prefill layer (H=4096,
 I=2048, 256 experts in 8 groups, keep 4, top-8, scaling 2.827).  At N=1 the
-run also measures the W4A16 decode layer (T=16) and the MXFP4->NVFP4
-transcode of one layer of expert weights, reported as nested objects.
+run also measures, as nested objects, the W4A16 decode layer (T=16, also with
+compact scales), the W4A8 prefill layer, the 65536-token skewed W4A4 layer on
+128 experts, the MXFP4->NVFP4 transcode of one layer of expert weights and the
+fused router.  Every timed step runs between its own CUDA events after an L2
+flush (256 MB written outside the events).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -67,6 +70,19 @@ def peaks():
 # nominal dense FP4 : BF16 and FP8 : BF16 tensor-core throughput on B200 (9 : 4.5 : 2.25 PFLOP/s)
 FP4_OVER_BF16 = 4.0
 FP8_OVER_BF16 = 2.0
+# B200 specification figures, for the second set of fractions
+SPEC_FP4_TFLOPS = 9000.0
+SPEC_FP8_TFLOPS = 4500.0
+SPEC_HBM_GBS = 8000.0
+# Rate of the block-scaled FP4 pair MMA (cta_group::2, M=256, N=256, K=64) that one
+# thread issuing back to back on resident operands reaches: one every 128 SM
+# cycles per CTA pair, i.e. 32,768 FLOP per cycle per SM (9.53 PFLOP/s at the
+# 1965 MHz maximum clock over 148 SMs).  Scaled by the SM clock sampled during
+# the timed region.
+MMA_FP4_FLOP_PER_CYCLE_PER_SM = 2 * 256 * 256 * 64 / 128 / 2
+N_SMS = 148
+# between timed steps this much memory is written, more than the 126 MB L2
+L2_FLUSH_BYTES = 256 << 20
 
 MODE_NAMES = {0: "W4A16", 1: "W4A4", 2: "W4A16 compact scales", 3: "W4A8 (MXFP8 x FP4)"}
 MODE_DTYPES = {0: "bf16 activations x fp4 e2m1 weights (e4m3 block scales), fp16 mma -> f32",
@@ -85,6 +101,8 @@ MODE_DTYPES = {0: "bf16 activations x fp4 e2m1 weights (e4m3 block scales), fp16
 GATEUP_TRAFFIC_T8192_E256 = 4 * (652.7936e6 + 21.404928e6)
 GATEUP_W4A8_TRAFFIC_T8192_E256 = 4 * (656.699392e6 + 35.003648e6)
 DECODE_TRAFFIC_T16_E256 = 1010.475e6 + 4.71296e6 + 505.455e6 + 5.101568e6
+# k_transcode of the bench's 768-tensor layer, out of place: not captured yet
+TRANSCODE_TRAFFIC = None
 
 
 class ClockSampler:
@@ -167,11 +185,48 @@ def config_of(wl, T, world):
     return {"workload": f"{wl.name}: T={T} H={wl.H} I={wl.I} E={wl.E} groups={wl.n_group} keep={wl.topk_group} "
                         f"top_k={wl.top_k} rsf={wl.rsf} {MODE_NAMES[wl.mode]}",
             "global_batch": T * world, "tokens_per_gpu": T, "parallelism": f"replicas{world}",
-            "l2": f"inputs larger than L2 ({weights_gb:.2f} GB of expert weights per step)"}
+            "l2": f"L2 flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB written, outside the step's events); "
+                  f"inputs larger than L2 too ({weights_gb:.2f} GB of expert weights per step)"}
 
 
 def layer_flops(T, H, I, k):
     return 6.0 * T * k * H * I
+
+
+def gemm_roofline(moe, mode, wl, T, gateup_ms, P, clocks, traffic):
+    """Roofline of the gate/up GEMM launch (the step's dominant kernel).  Peak:
+    the measured burst bf16 GEMM rate scaled by the nominal dense FP4:BF16 (FP8
+    for W4A8) ratio -- the kernel is timed in a region of tens of milliseconds,
+    too short for the power cap to lower the clock (the clocks sampled during it
+    are reported beside it).  Also: the fraction of the B200 specification
+    figure, of the pair MMA's own issue rate at the sampled clock, and the HBM
+    view (algorithmic bytes: the expert weights once, the input codes and scales
+    of every pair, the intermediate codes and scales written)."""
+    fp4 = mode == moe.W4A4
+    flops = 4.0 * T * wl.top_k * wl.H * wl.I  # padding excluded
+    t_kernel = gateup_ms / 1e3
+    achieved = flops / t_kernel / 1e12
+    ratio = FP4_OVER_BF16 if fp4 else FP8_OVER_BF16
+    peak = P["bf16_tflops"] * ratio
+    spec = SPEC_FP4_TFLOPS if fp4 else SPEC_FP8_TFLOPS
+    P_pairs = T * wl.top_k
+    act_b = 0.5 + 1.0 / 16 if fp4 else 1.0 + 1.0 / 32  # bytes per activation element with its scale
+    nbytes = wl.E * 2 * wl.I * wl.H * (0.5 + 1.0 / 16) + P_pairs * (wl.H + wl.I) * act_b
+    gbs = nbytes / t_kernel / 1e9
+    r = {"bound": "tensor", "kernel": "k_w4a4_gemm<gate/up>" + ("" if fp4 else ", FP8 x FP4"),
+         "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+         "traffic": traffic, "traffic_unit": "bytes per launch (ncu dram read+write)",
+         "peak_src": f"{P['src']} bf16 burst x {ratio:g} (nominal dense {'FP4' if fp4 else 'FP8'}:BF16)",
+         "algorithmic_flops_per_launch": flops,
+         "frac_of_spec": round(achieved / spec, 4), "spec_tflops": spec,
+         "hbm": {"algorithmic_bytes_per_launch": int(nbytes), "achieved_gbs": round(gbs, 1),
+                 "frac_of_measured": round(gbs / P["hbm_gbs"], 4), "frac_of_spec": round(gbs / SPEC_HBM_GBS, 4)}}
+    mhz = (clocks or {}).get("sm_mhz")
+    if fp4 and mhz:
+        pace = MMA_FP4_FLOP_PER_CYCLE_PER_SM * N_SMS * mhz * 1e6 / 1e12
+        r["frac_of_mma_pace"] = round(achieved / pace, 4)
+        r["mma_pace_tflops"] = round(pace, 1)
+    return r
 
 
 def max_over_ranks(torch, dist, ms, device):
@@ -211,32 +266,49 @@ def make_layer(torch, moe, mode, w, T, wl):
     return packed, ws
 
 
+class L2Flush:
+    """Writes L2_FLUSH_BYTES (more than the L2) on the current stream, between
+    timed steps and outside their events, so no step finds the previous step's
+    data in L2."""
+
+    def __init__(self, torch):
+        self.buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+        self.n = 0
+
+    def __call__(self):
+        self.n += 1
+        self.buf.fill_(self.n)
+
+
 def time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, steps, warmup, trace=True, on_start=None,
                on_end=None):
     """Returns (ms per step, per-stage ms means), both timed with CUDA events on the current
-    stream.  The step time comes from a pass without stage events (recording 7 events per
-    step costs a few microseconds, visible at decode sizes); the stage times from a second,
-    traced pass of the same steps."""
+    stream, each step between its own pair of events with an L2 flush before it.  The step
+    time comes from a pass without stage events (recording 7 events per step costs a few
+    microseconds, visible at decode sizes); the stage times from a second, traced pass of
+    the same steps."""
     H, I, E = wl.H, wl.I, wl.E
+    flush = L2Flush(torch)
 
     def step():
         moe.moe_forward(mode, x, logits, None, packed, 1.0, T, H, I, E, wl.n_group, wl.topk_group, wl.top_k, wl.rsf,
                         True, ws, out)
 
     for _ in range(warmup):
+        flush()
         step()
     torch.cuda.synchronize()
     if on_start:
         on_start()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(steps):
+    marks = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in marks:
+        flush()
+        a.record()
         step()
-    t1.record()
+        b.record()
     torch.cuda.synchronize()
     moe.nvfp4moe_check_device_status()
-    ms = t0.elapsed_time(t1) / steps
+    ms = float(np.sum([a.elapsed_time(b) for a, b in marks])) / steps
     if on_end:
         on_end()
     stage = None
@@ -249,6 +321,7 @@ def time_layer(torch, moe, mode, packed, ws, x, logits, out, wl, T, steps, warmu
             evs.append(row)
         torch.cuda.synchronize()
         for i in range(steps):
+            flush()
             moe.nvfp4moe_set_trace_events(evs[i])
             step()
         torch.cuda.synchronize()
@@ -372,23 +445,9 @@ def run_ours(args, rank, world, local_rank):
 
     # ----------------------------------------------------------------- roofline
     if mode in (moe.W4A4, moe.W4A8):
-        flops = 4.0 * T * wl.top_k * wl.H * wl.I  # gate/up GEMM, padding rows excluded
-        t_kernel = stage["gateup_gemm"] / 1e3
-        achieved = flops / t_kernel / 1e12
-        # The GEMM runs inside a long loop of steps and draws the board to its power
-        # cap (its SM clock falls to ~1.4-1.6 GHz), so the denominator is the
-        # sustained bf16 figure, scaled to FP4 (FP8 for W4A8) by the nominal dense ratio.
-        ratio = FP4_OVER_BF16 if mode == moe.W4A4 else FP8_OVER_BF16
-        peak = P["bf16_tflops_sustained"] * ratio
         full = (T, wl.E, wl.H, wl.I) == (8192, 256, 4096, 2048)
         traffic = (GATEUP_TRAFFIC_T8192_E256 if mode == moe.W4A4 else GATEUP_W4A8_TRAFFIC_T8192_E256) if full else None
-        roofline = {"bound": "tensor", "kernel": "k_w4a4_gemm<gate/up>", "achieved": round(achieved, 1),
-                    "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                    "traffic": traffic, "traffic_unit": "bytes per launch (ncu dram read+write)",
-                    "peak_src": f"{P['src']} bf16 sustained x {ratio:g} (nominal dense "
-                                f"{'FP4' if mode == moe.W4A4 else 'FP8'}:BF16); "
-                                f"burst would be {P['bf16_tflops'] * ratio:.0f}",
-                    "algorithmic_flops_per_launch": flops}
+        roofline = gemm_roofline(moe, mode, wl, T, stage["gateup_gemm"], P, clocks, traffic)
     else:
         # W4A16 weight stream: every active expert's codes + E4M3 scales read once
         ids_t = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
@@ -403,6 +462,7 @@ def run_ours(args, rank, world, local_rank):
         achieved = wbytes / t_kernel / 1e9
         roofline = {"bound": "hbm", "kernel": "k_w16_gateup + k_w16_down", "achieved": round(achieved, 1),
                     "peak": P["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / P["hbm_gbs"], 4),
+                    "frac_of_spec": round(achieved / SPEC_HBM_GBS, 4),
                     "traffic": (DECODE_TRAFFIC_T16_E256 if mode == moe.W4A16 and wl.name == "decode" and T == 16
                                 and wl.E == 256 else None),
                     "traffic_unit": "bytes per step of both GEMM launches (ncu dram read+write)",
@@ -431,6 +491,7 @@ def run_ours(args, rank, world, local_rank):
         del w
         res["decode_compact"] = bench_decode(torch, moe, None, args, P, compact=True)
         res["prefill_w4a8"] = bench_w4a8(torch, moe, args, P)
+        res["skewed"] = bench_skewed(torch, moe, args, P)
         res["transcode"] = bench_transcode(torch, moe, args, P)
         res["router"] = bench_router(torch, moe, args, P)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -472,8 +533,6 @@ def bench_decode(torch, moe, w, args, P, compact=False):
         torch.cuda.empty_cache()
     packed, ws = make_layer(torch, moe, mode, w, wl.T, wl)
     del w
-    # flush L2 between steps: the active experts' weights (~1.4 GB) exceed L2, but
-    # the same experts repeat every step, so rotate through a 256 MB buffer too
     ms, stage = time_layer(torch, moe, mode, packed, ws, xd, ld, out, wl, wl.T, max(args.steps, 20), args.warmup)
     ids = torch.empty((wl.T, wl.top_k), dtype=torch.int32, device="cuda")
     wts = torch.empty((wl.T, wl.top_k), dtype=torch.float32, device="cuda")
@@ -495,6 +554,8 @@ def bench_decode(torch, moe, w, args, P, compact=False):
             **({"same_weights": same_weights} if same_weights else {}),
             "roofline": {"bound": "hbm", "kernel": "k_w16_gateup + k_w16_down", "achieved": round(achieved, 1),
                          "peak": P["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / P["hbm_gbs"], 4),
+                         "frac_of_spec": round(achieved / SPEC_HBM_GBS, 4),
+                         "step_frac_of_spec": round(wbytes / (ms / 1e3) / 1e9 / SPEC_HBM_GBS, 4),
                          "traffic": None if compact else DECODE_TRAFFIC_T16_E256,
                          "traffic_unit": "bytes per step of both GEMM launches (ncu dram read+write)",
                          "algorithmic_bytes_per_step": int(wbytes)}}
@@ -520,19 +581,42 @@ def bench_w4a8(torch, moe, args, P):
     ms, stage = time_layer(torch, moe, moe.W4A8, packed, ws, xd, ld, out, wl, wl.T, args.steps, args.warmup)
     del packed, ws
     torch.cuda.empty_cache()
-    flops = 4.0 * wl.T * wl.top_k * wl.H * wl.I
-    achieved = flops / (stage["gateup_gemm"] / 1e3) / 1e12
-    peak = P["bf16_tflops_sustained"] * FP8_OVER_BF16
     return {"workload": f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top_k={wl.top_k} W4A8 (MXFP8 x FP4)",
             "value": round(wl.T / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
             "stages_ms": {k: round(v, 4) for k, v in stage.items()},
             "same_weights": {"mode": "W4A4", "ms_per_step": round(ms4, 4)},
-            "roofline": {"bound": "tensor", "kernel": "k_w4a4_gemm<gate/up, FP8 x FP4>", "achieved": round(achieved, 1),
-                         "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                         "traffic": GATEUP_W4A8_TRAFFIC_T8192_E256,
-                         "traffic_unit": "bytes per launch (ncu dram read+write)",
-                         "peak_src": f"{P['src']} bf16 sustained x {FP8_OVER_BF16:g} (nominal dense FP8:BF16)",
-                         "algorithmic_flops_per_launch": flops}}
+            "roofline": gemm_roofline(moe, moe.W4A8, wl, wl.T, stage["gateup_gemm"], P, None,
+                                      GATEUP_W4A8_TRAFFIC_T8192_E256)}
+
+
+def bench_skewed(torch, moe, args, P):
+    """The long skewed prefill: T=65536 on the 128-expert pruned layer (8 groups of
+    16), router logits with a Zipf(1.1) per-expert bias, W4A4.  Reports the
+    per-expert load (pairs routed to each expert) beside the stage times."""
+    wl = inputs.WORKLOADS["skewed"]
+    d = inputs.moe_inputs(wl)
+    w = {k: d[k] for k in ("gate_codes", "gate_sf", "up_codes", "up_sf", "down_codes", "down_sf", "w_global")}
+    xd = torch.from_numpy(d["x"].view(np.int16)).cuda().view(torch.bfloat16)
+    ld = torch.from_numpy(d["logits"]).cuda()
+    del d
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    packed, ws = make_layer(torch, moe, moe.W4A4, w, wl.T, wl)
+    del w
+    ms, stage = time_layer(torch, moe, moe.W4A4, packed, ws, xd, ld, out, wl, wl.T, args.steps, args.warmup)
+    ids = torch.empty((wl.T, wl.top_k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((wl.T, wl.top_k), dtype=torch.float32, device="cuda")
+    moe.moe_route(ld, None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf, True, ids, wts)
+    load = torch.bincount(ids.reshape(-1).long(), minlength=wl.E).cpu().numpy()
+    del packed, ws, xd, ld, out, ids, wts
+    torch.cuda.empty_cache()
+    return {"workload": f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} groups={wl.n_group} keep={wl.topk_group} "
+                        f"top_k={wl.top_k} rsf={wl.rsf} W4A4, logits + Zipf(1.1) expert bias",
+            "value": round(wl.T / (ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+            "tflops": round(layer_flops(wl.T, wl.H, wl.I, wl.top_k) / (ms / 1e3) / 1e12, 2),
+            "stages_ms": {k: round(v, 4) for k, v in stage.items()},
+            "expert_load": {"pairs_per_expert": [int(v) for v in load], "max": int(load.max()),
+                            "min": int(load.min()), "mean": round(float(load.mean()), 1)},
+            "roofline": gemm_roofline(moe, moe.W4A4, wl, wl.T, stage["gateup_gemm"], P, None, None)}
 
 
 def bench_router(torch, moe, args, P):
@@ -594,6 +678,7 @@ def bench_router(torch, moe, args, P):
             "higher_is_better": False, "eager_us_per_call": round(eager_us, 2),
             "roofline": {"bound": "hbm", "kernel": "k_router_topk", "achieved": round(gbs, 1), "peak": P["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / P["hbm_gbs"], 4), "traffic": None,
+                         "frac_of_spec": round(gbs / SPEC_HBM_GBS, 4),
                          "algorithmic_bytes_per_launch": int(nbytes)}}
 
 
@@ -630,7 +715,9 @@ def bench_transcode(torch, moe, args, P):
                        "out of place", "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
            "tensors_per_s": round(nt / (ms / 1e3), 1), "status": int(status), "report": rep,
            "roofline": {"bound": "hbm", "kernel": "k_transcode", "achieved": round(gbs, 1), "peak": P["hbm_gbs"],
-                        "unit": "GB/s", "frac": round(gbs / P["hbm_gbs"], 4), "traffic": None,
+                        "unit": "GB/s", "frac": round(gbs / P["hbm_gbs"], 4), "traffic": TRANSCODE_TRAFFIC,
+                        "traffic_unit": "bytes per launch (ncu dram read+write)",
+                        "frac_of_spec": round(gbs / SPEC_HBM_GBS, 4),
                         "algorithmic_bytes_per_launch": int(nbytes)}}
     # in place (codes aliased): scales only
     a.record()
