@@ -391,6 +391,25 @@ nvfp4moe_status moe_forward_ex(nvfp4moe_mode mode, const uint16_t* x, const floa
                                size_t workspace_bytes, void* out, int32_t out_is_fp32, int32_t* topk_ids_out,
                                float* topk_weights_out, void* stream);
 
+/* The down projection's input of the last moe_forward, moe_forward_ex or
+ * moe_forward_routed call made with `workspace` (same mode, T, H, I, E and
+ * top_k; nothing may have used the workspace since): for each listed pair
+ * p = t * top_k + j (pairs: device int32 [n_pairs]) the row of the requantised
+ * SwiGLU output, in the checkpoint layout.  No counterpart on the pages: it lets
+ * a caller (the parity checks) hold the gate/up half and the down half of the
+ * layer separately.
+ *   W4A4:   codes_out [n_pairs, I/2] NVFP4 (even element in the low nibble),
+ *           scales_out [n_pairs, I/16] E4M3;
+ *   W4A8:   codes_out [n_pairs, I] E4M3, scales_out [n_pairs, I/32] E8M0;
+ *   W4A16, W4A16C: codes_out [n_pairs, 2 I] (BF16 bit patterns), scales_out
+ *           unused (may be NULL).
+ * A pair index outside [0, T * top_k) leaves its output row untouched.
+ * Asynchronous on `stream`. */
+nvfp4moe_status moe_forward_intermediate(nvfp4moe_mode mode, int32_t T, int32_t H, int32_t I, int32_t E,
+                                         int32_t top_k, const void* workspace, size_t workspace_bytes,
+                                         const int32_t* pairs, int32_t n_pairs, uint8_t* codes_out,
+                                         uint8_t* scales_out, void* stream);
+
 /* Stage tracing.  When `events` is non-NULL, every later moe_forward /
  * moe_forward_routed call on this host thread records the cudaEvent_t handles
  * events[0..6] on its stream at its stage boundaries: [0] start, [1] after

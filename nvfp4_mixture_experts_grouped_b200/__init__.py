@@ -22,7 +22,7 @@ __all__ = [
     "moe_packed_weights_size", "moe_pack_weights", "moe_forward_workspace_size", "moe_forward",
     "moe_forward_ex", "moe_forward_routed", "nvfp4moe_check_device_status", "nvfp4moe_version", "moe_permute",
     "moe_permute_workspace_size", "nvfp4moe_set_trace_events", "moe_permute_noalloc", "W4A16C", "W4A8",
-    "nvfp4_compact_scales", "quantize_mxfp8",
+    "nvfp4_compact_scales", "quantize_mxfp8", "moe_forward_intermediate",
 ]
 
 W4A16 = 0
@@ -111,6 +111,8 @@ def load():
     L.moe_permute.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]
     L.moe_permute_noalloc.restype = ctypes.c_int
     L.moe_permute_noalloc.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
+    L.moe_forward_intermediate.restype = ctypes.c_int
+    L.moe_forward_intermediate.argtypes = [ctypes.c_int, i32, i32, i32, i32, i32, vp, sz, vp, i32, vp, vp, vp]
     L.nvfp4moe_set_trace_events.restype = ctypes.c_int
     L.nvfp4moe_set_trace_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     L.nvfp4moe_check_device_status.restype = ctypes.c_int
@@ -320,6 +322,20 @@ def moe_forward_routed(mode, x, topk_ids, topk_weights, packed_weights, act_glob
                                      act_global, T, H, I, E, top_k, _arg(workspace, "workspace"),
                                      workspace.numel() * workspace.element_size(),
                                      _arg(out, "out", (4 if out_f32 else 2) * T * H), out_f32, _stream(stream)))
+
+
+def moe_forward_intermediate(mode, T, H, I, E, top_k, workspace, pairs, codes_out, scales_out=None, stream=None):
+    """The down projection's input rows of `pairs` (int32 t * top_k + j) from the
+    last forward call made with `workspace`, in the checkpoint layout (see
+    include/nvfp4moe.h for the per-mode shapes)."""
+    n = pairs.numel()
+    row_bytes = I // 2 if mode == W4A4 else I if mode == W4A8 else 2 * I
+    scale_bytes = I // 16 if mode == W4A4 else I // 32 if mode == W4A8 else 0
+    _check(load().moe_forward_intermediate(mode, T, H, I, E, top_k, _arg(workspace, "workspace"),
+                                           workspace.numel() * workspace.element_size(), _arg(pairs, "pairs", 4 * n), n,
+                                           _arg(codes_out, "codes_out", n * row_bytes),
+                                           _arg(scales_out, "scales_out", n * scale_bytes, optional=scale_bytes == 0),
+                                           _stream(stream)))
 
 
 def nvfp4moe_set_trace_events(events) -> None:

@@ -16,7 +16,8 @@ ROOT = os.path.dirname(HERE)
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libnvfp4moe.so")
 
-SOURCES = ["api.cu", "transcode.cu", "route.cu", "router.cu", "permute.cu", "w4a16.cu", "w4a4.cu", "noalloc.cu", "compact.cu"]
+SOURCES = ["api.cu", "transcode.cu", "route.cu", "router.cu", "permute.cu", "w4a16.cu", "w4a4.cu", "noalloc.cu", "compact.cu",
+           "tmaps.cu"]
 # bit-exact steps: no FMA contraction anywhere the result decides an integer
 NO_FMAD = {"route.cu", "router.cu", "permute.cu", "transcode.cu"}
 

@@ -135,21 +135,25 @@ static ForwardLayout forward_layout(nvfp4moe_mode mode, int64_t T, int64_t H, in
     L.n_tiles = take(4);
     L.active = take(E * 4);
     L.n_active = take(4);
-    if (tc) {
-        // W4A4: NVFP4 codes + E4M3 per 16; W4A8: E4M3 elements + E8M0 per 32
-        const bool mx = mode == NVFP4MOE_W4A8;
-        L.a1c = take(mx ? L.rows_max * H : L.rows_max * H / 2);
-        L.a1s = take(L.rows_max * H / (mx ? 32 : 16));
-        L.a2c = take(mx ? L.rows_max * I : L.rows_max * I / 2);
-        L.a2s = take(L.rows_max * I / (mx ? 32 : 16));
+    if (mode == NVFP4MOE_W4A8) {
+        // E4M3 elements + E8M0 per 32 (atom layout); FP32 staged rows
+        L.a1c = take(L.rows_max * H);
+        L.a1s = take(L.rows_max * H / 32);
+        L.a2c = take(L.rows_max * I);
+        L.a2s = take(L.rows_max * I / 32);
         L.a2bf = -1;
-        if (mx) {
-            L.y = take(L.rows_max * H * 4);  // FP32 staged rows
-            L.ys = -1;
-        } else {
-            L.y = take(L.rows_max * H * 2);          // FP16 staged rows
-            L.ys = take(L.rows_max * (H / 64) * 4);  // their power-of-two scales
-        }
+        L.y = take(L.rows_max * H * 4);
+        L.ys = -1;
+    } else if (mode == NVFP4MOE_W4A4) {
+        // NVFP4 codes + E4M3 per 16 (atom layout); FP16 staged rows + their
+        // power-of-two scales per 64 columns
+        L.a1c = take(L.rows_max * H / 2);
+        L.a1s = take(L.rows_max * H / 16);
+        L.a2c = take(L.rows_max * I / 2);
+        L.a2s = take(L.rows_max * I / 16);
+        L.a2bf = -1;
+        L.y = take(L.rows_max * H * 2);
+        L.ys = take(L.rows_max * (H / 64) * 4);
     } else {
         L.a1c = L.a1s = L.a2c = L.a2s = L.ys = -1;
         L.a2bf = take(L.rows_max * I * 2);
@@ -462,14 +466,15 @@ static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, con
     if (tc) {
         uint8_t* a1c = ws + L.a1c;
         uint8_t* a1s = ws + L.a1s;
-        if (mode == NVFP4MOE_W4A8)
+        const bool mx8 = mode == NVFP4MOE_W4A8;
+        if (mx8)
             RETURN_IF(launch_quantize_mx8_scatter(x, T, H, a1c, a1s, plan.row_of_pair, top_k, st));
         else
             RETURN_IF(launch_quantize_scatter(x, T, H, act_global, a1c, a1s, plan.row_of_pair, top_k, st));
         trace(3, st);
-        RETURN_IF(launch_w4a4_layer(packed, mode == NVFP4MOE_W4A8, T, H, I, E, top_k, act_global, act_global_mid, L.rows_max, (int)L.max_tiles, plan, a1c,
-                                    a1s, ws + L.a2c, ws + L.a2s, static_cast<__half*>(Y), ys, st,
-                                    g_trace_on ? g_trace[4] : nullptr));
+        RETURN_IF(launch_w4a4_layer(packed, mx8, T, H, I, E, top_k, act_global, act_global_mid, L.rows_max,
+                                    (int)L.max_tiles, plan, a1c, a1s, ws + L.a2c, ws + L.a2s, static_cast<__half*>(Y),
+                                    mx8 ? nullptr : ys, st, g_trace_on ? g_trace[4] : nullptr));
     } else {
         trace(3, st);
         RETURN_IF(launch_w4a16_layer(x, packed, mode == NVFP4MOE_W4A16C, T, H, I, E, top_k, plan, reinterpret_cast<uint16_t*>(ws + L.a2bf),
@@ -513,6 +518,30 @@ nvfp4moe_status moe_forward_routed(nvfp4moe_mode mode, const uint16_t* x, const 
     if (T > 0 && (!topk_ids || !topk_weights)) return fail(NVFP4MOE_ERR_INVALID_ARG, "routing input is null");
     return forward_common(mode, x, nullptr, nullptr, topk_ids, topk_weights, packed_weights, act_global, act_global, T,
                           H, I, E, 1, 1, top_k, 1.0f, 0, workspace, workspace_bytes, out, out_is_fp32, nullptr, nullptr, stream);
+}
+
+nvfp4moe_status moe_forward_intermediate(nvfp4moe_mode mode, int32_t T, int32_t H, int32_t I, int32_t E,
+                                         int32_t top_k, const void* workspace, size_t workspace_bytes,
+                                         const int32_t* pairs, int32_t n_pairs, uint8_t* codes_out,
+                                         uint8_t* scales_out, void* stream) {
+    REQUIRE(valid_mode(mode), NVFP4MOE_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
+    REQUIRE(T >= 0 && n_pairs >= 0, NVFP4MOE_ERR_INVALID_ARG, "T=%d, n_pairs=%d", T, n_pairs);
+    RETURN_IF(validate_layer_shape(H, I, E));
+    REQUIRE(top_k >= 1 && top_k <= 32 && top_k <= E, NVFP4MOE_ERR_UNSUPPORTED_SHAPE, "top_k=%d outside [1, %d]", top_k,
+            std::min(32, (int)E));
+    if (T == 0 || n_pairs == 0) return NVFP4MOE_OK;
+    const bool scaled = mode == NVFP4MOE_W4A4 || mode == NVFP4MOE_W4A8;
+    REQUIRE(workspace && pairs && codes_out && (!scaled || scales_out), NVFP4MOE_ERR_INVALID_ARG, "null pointer");
+    const ForwardLayout L = forward_layout(mode, T, H, I, E, top_k);
+    REQUIRE(workspace_bytes >= (size_t)L.total, NVFP4MOE_ERR_WORKSPACE_TOO_SMALL,
+            "workspace of %zu bytes is below the required %lld", workspace_bytes, (long long)L.total);
+    RETURN_IF(check_device());
+    const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+    const int32_t* rop = reinterpret_cast<const int32_t*>(ws + L.row_of_pair);
+    const uint8_t* codes = ws + (scaled ? L.a2c : L.a2bf);
+    const uint8_t* scales = scaled ? ws + L.a2s : nullptr;
+    return launch_read_intermediate((int)mode, pairs, n_pairs, L.P, rop, codes, scales, I, codes_out, scales_out,
+                                    static_cast<cudaStream_t>(stream));
 }
 
 nvfp4moe_status nvfp4moe_set_trace_events(void* const* events, int32_t n_events) {

@@ -1,6 +1,7 @@
 // moe_internal.cuh -- declarations shared by the kernels and the C-ABI layer.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -11,8 +12,8 @@ namespace nvfp4moe {
 
 constexpr int PERM_CHUNK = 256;  // tokens per permutation chunk (one CTA)
 constexpr int PERM_WARPS = PERM_CHUNK / 32;
-constexpr int MTILE = 128;       // rows of one tcgen05 M-tile per CTA (the row padding of the W4A4 path)
-constexpr int PAIR_ROWS = 256;   // rows of one tile of a CTA pair (the tile list's unit)
+constexpr int MTILE = 128;       // rows of one tcgen05 M-tile per CTA (the row padding of the GEMM paths)
+constexpr int PAIR_ROWS = 256;   // rows of a pair tile (tokens as the MMA's M, 128 per CTA)
 
 __device__ __forceinline__ int64_t round_up_dev(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
@@ -56,8 +57,13 @@ nvfp4moe_status launch_permute(const int32_t* ids, int T, int k, int E, int pad,
 // [0, E) or a repeated id by experts 0..k-1 with weight 0 (DEV_ERR_BAD_ROUTING)
 nvfp4moe_status launch_check_routing(const int32_t* ids_in, const float* wts_in, int64_t T, int k, int E,
                                      int32_t* ids, float* wts, cudaStream_t stream);
+// the down projection's input rows of listed pairs in the checkpoint layout
+nvfp4moe_status launch_read_intermediate(int mode, const int32_t* pairs, int n_pairs, int64_t P,
+                                         const int32_t* row_of_pair, const uint8_t* codes, const uint8_t* scales,
+                                         int I, uint8_t* codes_out, uint8_t* scales_out, cudaStream_t stream);
 nvfp4moe_status launch_quantize_linear(const uint16_t* x, int64_t M, int64_t K, float gs, uint8_t* codes,
                                        uint8_t* scales, cudaStream_t stream);
+// scales in the atom layout of the W4A4 GEMMs (sf_atom_offset)
 nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H, float gs, uint8_t* codes,
                                         uint8_t* scales, const int32_t* row_of_pair, int k, cudaStream_t stream);
 // MXFP8 (E4M3 + E8M0 per 32): linear [M, K] codes / [M, K/32] scales, and the
@@ -67,7 +73,7 @@ nvfp4moe_status launch_quantize_mx8_linear(const uint16_t* x, int64_t M, int64_t
 nvfp4moe_status launch_quantize_mx8_scatter(const uint16_t* x, int64_t T, int64_t H, uint8_t* codes, uint8_t* scales,
                                             const int32_t* row_of_pair, int k, cudaStream_t stream);
 // Y staged as FP16 rows with a power-of-two scale per 64 columns (y_scale != nullptr,
-// W4A4) or as FP32 rows (y_scale == nullptr, W4A16).
+// W4A4) or as FP32 rows (y_scale == nullptr, W4A16 and W4A8).
 nvfp4moe_status launch_combine(const void* Y, const float* y_scale, const int32_t* row_of_pair, int64_t T, int H,
                                int k, void* out, bool out_f32, cudaStream_t stream);
 
@@ -88,6 +94,14 @@ size_t w4a16_scratch_size(int T, int H, int I, int k);  // FP16 copies of the ac
 nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, bool compact, int T, int H, int I,
                                    int E, int k, const RoutingPlan& plan, uint16_t* A2, float* Y, void* scratch,
                                    cudaStream_t stream, cudaEvent_t mid_event);
+
+// tmaps.cu: 2-D tensor maps of the TMA copies.  make_map: uint8 rows
+// [rows, row_bytes], a box of 128 bytes x box_rows, 128-byte swizzle; make_map_u4:
+// 4-bit codes [rows, k_elems] that the copy unpacks into the padded
+// shared-memory form (each 16 codes: 8 bytes, then 8 bytes of gap), a box of 128
+// codes x box_rows.  Both set the error string and return false on failure.
+bool make_map(CUtensorMap* m, const void* base, int64_t row_bytes, int64_t rows, int box_rows);
+bool make_map_u4(CUtensorMap* m, const void* base, int64_t k_elems, int64_t rows, int box_rows);
 
 // w4a4.cu: the tcgen05 pair GEMMs; mx8 selects W4A8 (MXFP8 activations x FP4
 // weights held in the padded form with E8M0 scales) instead of W4A4

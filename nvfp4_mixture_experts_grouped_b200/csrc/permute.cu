@@ -66,6 +66,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int& tota
     return before + x - v;
 }
 
+
 __global__ void __launch_bounds__(1024)
     k_scan_experts(int n_chunks, int E, int pad, int32_t* __restrict__ chunk_counts, RoutingPlan plan) {
     __shared__ int s_tmp[1024];
@@ -98,14 +99,8 @@ __global__ void __launch_bounds__(1024)
         plan.counts[e] = cnt;
         plan.offsets[e] = off;
         plan.pad_offsets[e] = poff;
-        for (int j = 0; j < tiles; ++j) {
-            int4 ti;
-            ti.x = e;
-            ti.y = poff + j * PAIR_ROWS;
-            ti.z = min(PAIR_ROWS, cnt - j * PAIR_ROWS);
-            ti.w = j;
-            plan.tiles[toff + j] = ti;
-        }
+        for (int j = 0; j < tiles; ++j)
+            plan.tiles[toff + j] = make_int4(e, poff + j * PAIR_ROWS, min(PAIR_ROWS, cnt - j * PAIR_ROWS), j);
         if (cnt > 0) plan.active[aoff] = e;
     }
     if (e == 0) {
@@ -299,6 +294,49 @@ nvfp4moe_status launch_check_routing(const int32_t* ids_in, const float* wts_in,
 }
 
 // ---------------------------------------------------------------------------
+// The down projection's input rows of listed pairs, back in the checkpoint layout
+// (moe_forward_intermediate).  One CTA per listed pair; a pair index outside
+// [0, P) is skipped.  W4A4: NVFP4 codes [I/2] + E4M3 scales [I/16]; W4A8: E4M3
+// [I] + E8M0 [I/32], both from the atom layout; W4A16: BF16 rows [I] (no scales).
+// ---------------------------------------------------------------------------
+template <int MODE>
+__global__ void __launch_bounds__(128)
+    k_read_intermediate(const int32_t* __restrict__ pairs, int64_t P, const int32_t* __restrict__ row_of_pair,
+                        const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales, int I,
+                        uint8_t* __restrict__ codes_out, uint8_t* __restrict__ scales_out) {
+    const int32_t p = pairs[blockIdx.x];
+    if (p < 0 || p >= P) return;
+    const int64_t row = row_of_pair[p];
+    const int row_bytes = MODE == NVFP4MOE_W4A4 ? I / 2 : MODE == NVFP4MOE_W4A8 ? I : 2 * I;
+    for (int i = threadIdx.x; i < row_bytes; i += blockDim.x)
+        codes_out[(int64_t)blockIdx.x * row_bytes + i] = codes[row * row_bytes + i];
+    if (MODE == NVFP4MOE_W4A4) {
+        for (int kb = threadIdx.x; kb < I / 16; kb += blockDim.x)
+            scales_out[(int64_t)blockIdx.x * (I / 16) + kb] = scales[sf_atom_offset(row, kb, I / 16)];
+    } else if (MODE == NVFP4MOE_W4A8) {
+        for (int kb = threadIdx.x; kb < I / 32; kb += blockDim.x)
+            scales_out[(int64_t)blockIdx.x * (I / 32) + kb] = scales[sf_atom_offset(row, kb, I / 32)];
+    }
+}
+
+nvfp4moe_status launch_read_intermediate(int mode, const int32_t* pairs, int n_pairs, int64_t P,
+                                         const int32_t* row_of_pair, const uint8_t* codes, const uint8_t* scales,
+                                         int I, uint8_t* codes_out, uint8_t* scales_out, cudaStream_t stream) {
+    if (n_pairs == 0) return NVFP4MOE_OK;
+    if (mode == NVFP4MOE_W4A4)
+        k_read_intermediate<NVFP4MOE_W4A4><<<n_pairs, 128, 0, stream>>>(pairs, P, row_of_pair, codes, scales, I,
+                                                                        codes_out, scales_out);
+    else if (mode == NVFP4MOE_W4A8)
+        k_read_intermediate<NVFP4MOE_W4A8><<<n_pairs, 128, 0, stream>>>(pairs, P, row_of_pair, codes, scales, I,
+                                                                        codes_out, scales_out);
+    else
+        k_read_intermediate<NVFP4MOE_W4A16><<<n_pairs, 128, 0, stream>>>(pairs, P, row_of_pair, codes, scales, I,
+                                                                         codes_out, scales_out);
+    NVFP4MOE_CHECK_LAUNCH("intermediate read-back kernel");
+    return NVFP4MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
 // 4. NVFP4 quantisation (one warp per row, a 16-element block per lane step)
 // ---------------------------------------------------------------------------
 // Linear layout (quantize_nvfp4): codes [M, K/2], scales [M, K/16].
@@ -476,7 +514,8 @@ nvfp4moe_status launch_quantize_mx8_scatter(const uint16_t* x, int64_t T, int64_
 // ---------------------------------------------------------------------------
 // 5. weighted un-permute: out[t] = sum_j Y[row_of_pair(t, j)] (routing weights
 //    already applied by the down GEMM), FP32 in slot order, one rounding.
-//    Y is FP16 with a power-of-two scale per 64 columns (W4A4) or FP32 (W4A16).
+//    Y is FP16 with a power-of-two scale per 64 columns (W4A4) or FP32 (W4A16,
+//    W4A8).
 // ---------------------------------------------------------------------------
 template <bool Y_F16, bool OUT_F32>
 __global__ void __launch_bounds__(256)

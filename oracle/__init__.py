@@ -261,3 +261,55 @@ def moe_layer(mode: int, x_bits, logits, bias, gate_codes, gate_sf, up_codes, up
                            ctypes.c_int(top_k), ctypes.c_float(rsf), ctypes.c_int(int(renormalize)), _p(tokens),
                            ctypes.c_int(len(tokens)), _p(out))
     return out
+
+
+def moe_intermediate(mode: int, x_bits, logits, bias, gate_codes, gate_sf, up_codes, up_sf, w_global,
+                     act_global: float, n_group: int, topk_group: int, top_k: int, rsf: float,
+                     renormalize: bool = True, tokens=None, acc_rel: float | None = None):
+    """The SwiGLU output before the intermediate quantisation, FP32 [n, top_k, I],
+    with the tokens' routing ids / weights [n, top_k] (float64 arithmetic as the
+    layer's, rounded once to FP32).  With acc_rel, also a bound [n, top_k, I] on
+    the distance of an FP32 evaluation whose gate/up dot products err by at most
+    acc_rel * sum |x w| (see orc_moe_intermediate)."""
+    x = np.ascontiguousarray(x_bits, np.uint16)
+    T, H = x.shape
+    E, I = gate_codes.shape[0], gate_codes.shape[1]
+    tokens = np.arange(T, dtype=np.int32) if tokens is None else np.ascontiguousarray(tokens, np.int32)
+    n = len(tokens)
+    a32 = np.empty((n, top_k, I), np.float32)
+    ids = np.empty((n, top_k), np.int32)
+    wts = np.empty((n, top_k), np.float32)
+    arrs = [np.ascontiguousarray(a, np.uint8) for a in (gate_codes, gate_sf, up_codes, up_sf)]
+    b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    err = None if acc_rel is None else np.empty((n, top_k, I), np.float32)
+    _load().orc_moe_intermediate(ctypes.c_int(mode), _p(x), _p(np.ascontiguousarray(logits, np.float32)),
+                                 None if b is None else _p(b), *[_p(a) for a in arrs],
+                                 _p(np.ascontiguousarray(w_global, np.float32)), ctypes.c_float(act_global),
+                                 ctypes.c_int(H), ctypes.c_int(I), ctypes.c_int(E), ctypes.c_int(n_group),
+                                 ctypes.c_int(topk_group), ctypes.c_int(top_k), ctypes.c_float(rsf),
+                                 ctypes.c_int(int(renormalize)), _p(tokens), ctypes.c_int(n), _p(a32), _p(ids),
+                                 _p(wts), ctypes.c_double(acc_rel or 0.0), None if err is None else _p(err))
+    return (a32, ids, wts) if err is None else (a32, ids, wts, err)
+
+
+def moe_down(a: np.ndarray, ids: np.ndarray, wts: np.ndarray, down_codes, down_sf, w_global) -> np.ndarray:
+    """float64 layer output [n, H] from down-projection inputs a [n, top_k, I]
+    (float64 values) and the tokens' routing ids / weights [n, top_k]."""
+    a = np.ascontiguousarray(a, np.float64)
+    n, k, I = a.shape
+    E, H = down_codes.shape[0], down_codes.shape[1]
+    out = np.empty((n, H), np.float64)
+    _load().orc_moe_down(_p(a), _p(np.ascontiguousarray(ids, np.int32)), _p(np.ascontiguousarray(wts, np.float32)),
+                         _p(np.ascontiguousarray(down_codes, np.uint8)), _p(np.ascontiguousarray(down_sf, np.uint8)),
+                         _p(np.ascontiguousarray(w_global, np.float32)), ctypes.c_int(H), ctypes.c_int(I),
+                         ctypes.c_int(E), ctypes.c_int(k), ctypes.c_int(n), _p(out))
+    return out
+
+
+def decode_mxfp8(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    M, K = codes.shape
+    out = np.empty((M, K), np.float64)
+    _load().orc_decode_mxfp8(_p(codes), _p(np.ascontiguousarray(scales, np.uint8)), ctypes.c_int64(M),
+                             ctypes.c_int64(K), _p(out))
+    return out

@@ -813,6 +813,153 @@ void orc_moe_layer2(int mode, const uint16_t* x, const float* logits, const floa
     free(first);
 }
 
+/* The layer split at the down projection's input, for checks that hold each
+ * half on its own.  orc_moe_intermediate: per sampled token its routing and,
+ * per slot j, the SwiGLU output a = SiLU(g) * u (float64, as orc_moe_layer2
+ * forms it) rounded to FP32 -- the values the intermediate quantisation takes
+ * in.  a32 [n_tokens, top_k, I], ids / wts [n_tokens, top_k].
+ * a_err (optional, same shape as a32): a bound on how far an FP32 evaluation of
+ * the same a may lie from it, for a GEMM whose dot products g and u carry an
+ * error of at most acc_rel * sum_h |x_h w_h| (the sum scaled like g and u):
+ *   |da| <= 1.1 * eg * (|u| + eu) + |SiLU(g)| * eu + 2^-20 |a|,
+ * with eg, eu those bounds, 1.1 the largest slope of SiLU and 2^-20 |a| the
+ * rounding of SiLU and the product in FP32. */
+static double silu_slope_bound(void) { return 1.1; }
+
+static void row_abs_dots(const double* w, const double* const* v, int n, int64_t K, double* out) {
+    for (int q = 0; q < n; ++q) {
+        double s0 = 0.0;
+        for (int64_t k = 0; k < K; ++k) s0 += fabs(v[q][k] * w[k]);
+        out[q] = s0;
+    }
+}
+
+void orc_moe_intermediate(int mode, const uint16_t* x, const float* logits, const float* bias,
+                          const uint8_t* gate_codes, const uint8_t* gate_sf, const uint8_t* up_codes,
+                          const uint8_t* up_sf, const float* w_global, float act_global, int H, int I, int E,
+                          int n_group, int topk_group, int top_k, float rsf, int renormalize, const int32_t* tokens,
+                          int n_tokens, float* a32, int32_t* ids, float* wts, double acc_rel, float* a_err) {
+    double* xd = (double*)malloc(sizeof(double) * (size_t)n_tokens * H);
+    const int np = n_tokens * top_k;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int it = 0; it < n_tokens; ++it) {
+        const int t = tokens[it];
+        orc_route(logits + (int64_t)t * E, bias, 1, E, n_group, topk_group, top_k, rsf, renormalize,
+                  ids + (int64_t)it * top_k, wts + (int64_t)it * top_k);
+        layer_input(mode, x + (int64_t)t * H, H, act_global, xd + (int64_t)it * H);
+    }
+    for (int e = 0; e < E; ++e) {
+        int n = 0;
+        for (int q = 0; q < np; ++q) n += ids[q] == e;
+        if (n == 0) continue;
+        int* pl = (int*)malloc(sizeof(int) * (size_t)n);
+        const double** xv = (const double**)malloc(sizeof(double*) * (size_t)n);
+        n = 0;
+        for (int q = 0; q < np; ++q)
+            if (ids[q] == e) {
+                pl[n] = q;
+                xv[n] = xd + (int64_t)(q / top_k) * H;
+                ++n;
+            }
+        const double gg = w_global[e * 3 + 0], gu = w_global[e * 3 + 1];
+#pragma omp parallel
+        {
+            double* wrow = (double*)malloc(sizeof(double) * (size_t)H);
+            double* gv = (double*)malloc(sizeof(double) * (size_t)n);
+            double* uv = (double*)malloc(sizeof(double) * (size_t)n);
+            double* ga = (double*)malloc(sizeof(double) * (size_t)n);
+            double* ua = (double*)malloc(sizeof(double) * (size_t)n);
+#pragma omp for schedule(dynamic, 16)
+            for (int i = 0; i < I; ++i) {
+                const int64_t r = (int64_t)e * I + i;
+                decode_row(gate_codes + r * (H / 2), gate_sf + r * (H / 16), gg, H, wrow);
+                row_dots(wrow, xv, n, H, gv);
+                if (a_err) row_abs_dots(wrow, xv, n, H, ga);
+                decode_row(up_codes + r * (H / 2), up_sf + r * (H / 16), gu, H, wrow);
+                row_dots(wrow, xv, n, H, uv);
+                if (a_err) row_abs_dots(wrow, xv, n, H, ua);
+                for (int q = 0; q < n; ++q) {
+                    const double a = silu(gv[q]) * uv[q];
+                    a32[(int64_t)pl[q] * I + i] = (float)a;
+                    if (a_err) {
+                        const double eg = acc_rel * ga[q], eu = acc_rel * ua[q];
+                        a_err[(int64_t)pl[q] * I + i] = (float)(silu_slope_bound() * eg * (fabs(uv[q]) + eu) +
+                                                                fabs(silu(gv[q])) * eu + ldexp(fabs(a), -20));
+                    }
+                }
+            }
+            free(wrow);
+            free(gv);
+            free(uv);
+            free(ga);
+            free(ua);
+        }
+        free(pl);
+        free(xv);
+    }
+    free(xd);
+}
+
+/* orc_moe_down: the layer output from given down-projection inputs a [n_tokens,
+ * top_k, I] (float64 values, already in the precision the mode uses) with the
+ * tokens' routing ids / wts [n_tokens, top_k]: out[t] = sum_j w_{t,j} *
+ * (W_down,e_j a_{t,j}) * global, in float64, slot order.  Fed the oracle's own
+ * requantised intermediate it reproduces orc_moe_layer2 exactly. */
+void orc_moe_down(const double* a, const int32_t* ids, const float* wts, const uint8_t* down_codes,
+                  const uint8_t* down_sf, const float* w_global, int H, int I, int E, int top_k, int n_tokens,
+                  double* out) {
+    const int np = n_tokens * top_k;
+    double* ybuf = (double*)malloc(sizeof(double) * (size_t)np * H);
+    for (int e = 0; e < E; ++e) {
+        int n = 0;
+        for (int q = 0; q < np; ++q) n += ids[q] == e;
+        if (n == 0) continue;
+        int* pl = (int*)malloc(sizeof(int) * (size_t)n);
+        const double** av = (const double**)malloc(sizeof(double*) * (size_t)n);
+        n = 0;
+        for (int q = 0; q < np; ++q)
+            if (ids[q] == e) {
+                pl[n] = q;
+                av[n] = a + (int64_t)q * I;
+                ++n;
+            }
+        const double gd = w_global[e * 3 + 2];
+#pragma omp parallel
+        {
+            double* wrow = (double*)malloc(sizeof(double) * (size_t)I);
+            double* yv = (double*)malloc(sizeof(double) * (size_t)n);
+#pragma omp for schedule(dynamic, 16)
+            for (int h = 0; h < H; ++h) {
+                const int64_t r = (int64_t)e * H + h;
+                decode_row(down_codes + r * (I / 2), down_sf + r * (I / 16), gd, I, wrow);
+                row_dots(wrow, av, n, I, yv);
+                for (int q = 0; q < n; ++q) ybuf[(int64_t)pl[q] * H + h] = yv[q];
+            }
+            free(wrow);
+            free(yv);
+        }
+        free(pl);
+        free(av);
+    }
+#pragma omp parallel for schedule(static)
+    for (int it = 0; it < n_tokens; ++it) {
+        double* o = out + (int64_t)it * H;
+        for (int h = 0; h < H; ++h) o[h] = 0.0;
+        for (int j = 0; j < top_k; ++j) {
+            const int64_t q = (int64_t)it * top_k + j;
+            for (int h = 0; h < H; ++h) o[h] += (double)wts[q] * ybuf[q * H + h];
+        }
+    }
+    free(ybuf);
+}
+
+/* Values of MXFP8 rows: E4M3 element x 2^(E8M0 - 127) per 32, codes [M, K],
+ * scales [M, K/32]. */
+void orc_decode_mxfp8(const uint8_t* codes, const uint8_t* scales, int64_t M, int64_t K, double* out) {
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) out[m * K + k] = mxfp8_value(codes + m * K, scales + m * (K / 32), k);
+}
+
 /* One activation global scale for both quantisations (the pages' unit scale). */
 void orc_moe_layer(int mode, const uint16_t* x, const float* logits, const float* bias, const uint8_t* gate_codes,
                    const uint8_t* gate_sf, const uint8_t* up_codes, const uint8_t* up_sf, const uint8_t* down_codes,

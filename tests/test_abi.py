@@ -215,3 +215,20 @@ def test_quantize_mxfp8_validation():
     assert lib.quantize_mxfp8(p, 4, 64, None, p, None) == 1
     assert lib.quantize_mxfp8(p, 4, 64, ctypes.c_void_p(4104), p, None) == 2
     assert lib.quantize_mxfp8(None, 0, 64, None, None, None) == 0
+
+
+def test_forward_intermediate_validation():
+    lib = moe.load()
+    p = ctypes.c_void_p(4096)
+
+    def call(mode=1, T=4, n=8, ws_bytes=1 << 40, ws=p, pairs=p, codes=p, scales=p):
+        return lib.moe_forward_intermediate(mode, T, 4096, 2048, 256, 8, ws, ws_bytes, pairs, n, codes, scales, None)
+
+    assert call(mode=4) == 1  # unknown mode
+    assert call(n=-1) == 1
+    assert call(ws=None) == 1
+    assert call(scales=None) == 1  # W4A4 has scales
+    assert call(ws_bytes=16) == 6
+    # T == 0 or no pairs: nothing to read
+    assert call(T=0, ws=None, pairs=None, codes=None, scales=None) == 0
+    assert call(n=0, ws=None, pairs=None, codes=None, scales=None) == 0

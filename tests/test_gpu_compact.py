@@ -135,5 +135,4 @@ def test_compact_decode_full_size_sampled():
     del ref16
     torch.cuda.empty_cache()
     assert torch.equal(out.view(torch.int32), base.view(torch.int32))
-    toks = np.array([0, 5, 11, wl.T - 1], np.int32)
-    compare_layer(out_to_f64(out)[toks], oracle_layer(moe.W4A16C, d, w, wl, tokens=toks))
+    compare_layer(out_to_f64(out), oracle_layer(moe.W4A16C, d, w, wl))  # all 16 tokens

@@ -11,8 +11,8 @@ import nvfp4_mixture_experts_grouped_b200 as moe
 import oracle
 from nvfp4_mixture_experts_grouped_b200 import inputs
 
-from helpers import (GpuLayer, bf16_tensor, compare_layer, dev, gpu_transcode, host, nvfp4_weights_from_inputs,
-                     oracle_layer, out_to_f64)
+from helpers import (GpuLayer, bf16_tensor, check_layer_split, compare_layer, covering_tokens, dev, gpu_transcode,
+                     host, nvfp4_weights_from_inputs, oracle_layer, out_to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -67,28 +67,36 @@ def test_transcode_large_tensor_uncached_path():
     _assert_transcode_equal(codes, e8)
 
 
-def test_transcode_full_layer_sampled():
-    """The full transcode workload (768 expert tensors + the adversarial one) on
-    the GPU; a seeded sample of tensors is checked against the oracle."""
+def test_transcode_full_layer_all_tensors():
+    """The full transcode workload on the GPU: 768 expert tensors of one layer
+    (gate and up [2048, 4096] out of place, down [4096, 2048] in place) plus the
+    adversarial tensor; every tensor's E4M3 scales, global and status equal the
+    oracle's, the codes are byte-identical and the report counts agree."""
     rng = np.random.default_rng(inputs.TRANSCODE_SEED)
     layer = inputs.transcode_layer(rng)
-    gate_c, gate_s = layer["gate"]
-    codes = np.concatenate([gate_c, layer["adversarial"][0]])
-    e8 = np.concatenate([gate_s, layer["adversarial"][1]])
-    gc, ge4, gg, gst, grep, gstatus = gpu_transcode(codes, e8)
-    assert gstatus == 5 and grep["nonrepresentable_tensors"] == 1 and gst[-1] == 1
-    assert np.all(gst[:-1] == 0)
-    pick = sorted(set(np.random.default_rng(1).choice(256, 6, replace=False).tolist()) | {0, 255, 256})
-    for t in pick:
-        rc, re4, rg, rst, _, _ = oracle.transcode(codes[t:t + 1], e8[t:t + 1], 1, 2048, 4096)
-        assert np.array_equal(ge4[t], re4[0]) and gg[t] == rg[0] and gst[t] == rst[0]
-    assert np.array_equal(gc, codes)
-    down_c, down_s = layer["down"]
-    gc2, ge42, gg2, gst2, _, st2 = gpu_transcode(down_c, down_s, in_place=True)
-    assert st2 == 0 and np.all(gst2 == 0)
-    for t in (0, 128, 255):
-        rc, re4, rg, _, _, _ = oracle.transcode(down_c[t:t + 1], down_s[t:t + 1], 1, 4096, 2048)
-        assert np.array_equal(ge42[t], re4[0]) and gg2[t] == rg[0]
+    batches = (("gate", 2048, 4096, False, True), ("up", 2048, 4096, False, False), ("down", 4096, 2048, True, False))
+    n_checked = 0
+    for name, N, K, in_place, with_adversarial in batches:
+        codes, e8 = layer[name]
+        if with_adversarial:
+            codes = np.concatenate([codes, layer["adversarial"][0]])
+            e8 = np.concatenate([e8, layer["adversarial"][1]])
+        nt = codes.shape[0]
+        gc, ge4, gg, gst, grep, gstatus = gpu_transcode(codes, e8, in_place=in_place)
+        rc, re4, rg, rst, rrep, _ = oracle.transcode(codes, e8, nt, N, K)
+        assert np.array_equal(gc, codes) and np.array_equal(rc.reshape(codes.shape), codes)
+        assert np.array_equal(ge4, re4)
+        assert np.array_equal(gg.view(np.uint32), rg.view(np.uint32))
+        assert np.array_equal(gst, rst)
+        assert [grep["blocks"], grep["zero_blocks"], grep["nonrepresentable_tensors"], grep["nan_scale_tensors"]] == \
+            rrep.tolist()
+        if with_adversarial:
+            assert gstatus == 5 and gst[-1] == 1 and np.all(gst[:-1] == 0)
+        else:
+            assert gstatus == 0 and np.all(gst == 0)
+        n_checked += nt
+        del codes, e8, gc, ge4, rc, re4
+    assert n_checked == 769
 
 
 # ---------------------------------------------------------------------------
@@ -336,6 +344,7 @@ def test_layer_tiny_all_tokens(mode):
     compare_layer(out_to_f64(out), ref, bf16_output=True)
     out32, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), out_fp32=True)
     compare_layer(out_to_f64(out32), ref)
+    check_layer_split(layer, d, w_ref, wl, np.arange(wl.T, dtype=np.int32), out32, out)
 
 
 def test_layer_decode_w4a16_full():
@@ -348,30 +357,30 @@ def test_layer_decode_w4a16_full():
     compare_layer(out_to_f64(out), ref)
     out16, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]))
     compare_layer(out_to_f64(out16), ref, bf16_output=True)
-
-
-def _sample_tokens(ids: np.ndarray, n: int, seed: int):
-    rng = np.random.default_rng(seed)
-    T = ids.shape[0]
-    heavy = np.bincount(ids.reshape(-1)).argmax()
-    on_heavy = np.where((ids == heavy).any(1))[0]
-    pick = set(rng.choice(T, n, replace=False).tolist()) | set(on_heavy[:2].tolist()) | {0, T - 1}
-    return np.array(sorted(pick), np.int32)
+    check_layer_split(layer, d, w, wl, np.arange(wl.T, dtype=np.int32), out, out16)
 
 
 @pytest.mark.parametrize("name", ["prefill", "skewed"])
 def test_layer_w4a4_full_size_sampled(name):
+    # full-size layers: at least 512 seeded tokens whose rows cover every
+    # 128-row run of every expert (tile halves, ragged last chunks, each
+    # expert's last row), held in two halves at the down projection's input:
+    # the intermediate codes against the oracle's up to boundary flips, the
+    # output against the oracle's down half of the GPU's intermediate at the bare
+    # bound (BF16 output with its own rounding allowed), and the whole layer
+    # (rel-L2 over all, max-abs over tokens without a flip)
     wl = inputs.WORKLOADS[name]
     d = inputs.moe_inputs(wl)
     w = nvfp4_weights_from_inputs(d, False)
     layer = GpuLayer(wl.mode, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
-    out, ids, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), out_fp32=True)
-    toks = _sample_tokens(host(ids), 12, wl.seed)
-    ref = oracle_layer(wl.mode, d, w, wl, tokens=toks)
-    compare_layer(out_to_f64(out)[toks], ref)
     out16, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]))
-    compare_layer(out_to_f64(out16)[toks], ref, bf16_output=True)
-    # also the W4A16 path on a decode-sized slice of the same weights
+    out, ids, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), out_fp32=True)
+    h_ids = host(ids)
+    ri, _ = oracle.route(d["logits"], None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf)
+    assert np.array_equal(h_ids, ri)
+    toks = covering_tokens(h_ids, wl.E, wl.seed)
+    assert len(toks) >= 512
+    check_layer_split(layer, d, w, wl, toks, out, out16)
     del layer
     torch.cuda.empty_cache()
 
@@ -470,10 +479,10 @@ def test_layer_prefill_calibrated_globals_sampled():
     amax = float(np.abs((d["x"].astype(np.uint32) << 16).view(np.float32)).max())
     g_in = float(np.float32(amax / 2688.0))
     layer = GpuLayer(moe.W4A4, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
+    out16, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), act_global=g_in, act_global_mid=0.5)
     out, ids, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), act_global=g_in, act_global_mid=0.5,
                                 out_fp32=True)
-    toks = _sample_tokens(host(ids), 8, wl.seed + 1)
-    ref = oracle_layer(moe.W4A4, d, w, wl, tokens=toks, act_global=g_in, act_global_mid=0.5)
-    compare_layer(out_to_f64(out)[toks], ref)
+    toks = covering_tokens(host(ids), wl.E, wl.seed + 1)
+    check_layer_split(layer, d, w, wl, toks, out, out16, act_global=g_in, act_global_mid=0.5)
     del layer
     torch.cuda.empty_cache()

@@ -12,7 +12,8 @@ import nvfp4_mixture_experts_grouped_b200 as moe
 import oracle
 from nvfp4_mixture_experts_grouped_b200 import inputs
 
-from helpers import GpuLayer, bf16_tensor, compare_layer, dev, host, nvfp4_weights_from_inputs, oracle_layer, out_to_f64
+from helpers import (GpuLayer, bf16_tensor, check_layer_split, compare_layer, covering_tokens, dev, host,
+                     nvfp4_weights_from_inputs, oracle_layer, out_to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -114,13 +115,11 @@ def test_w4a8_prefill_full_size_sampled():
     d = inputs.moe_inputs(wl)
     w = nvfp4_weights_from_inputs(d, False)
     layer = GpuLayer(moe.W4A8, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
+    out16, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]))
     out, ids, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), out_fp32=True)
-    h_ids = host(ids)
-    rng = np.random.default_rng(wl.seed)
-    heavy = np.bincount(h_ids.reshape(-1)).argmax()
-    toks = sorted(set(rng.choice(wl.T, 10, replace=False).tolist()) |
-                  set(np.where((h_ids == heavy).any(1))[0][:2].tolist()) | {0, wl.T - 1})
-    toks = np.array(toks, np.int32)
-    compare_layer(out_to_f64(out)[toks], oracle_layer(moe.W4A8, d, w, wl, tokens=toks))
+    # >= 512 seeded tokens covering every 128-row run of every expert, held in
+    # two halves at the down projection's input (see check_layer_split)
+    toks = covering_tokens(host(ids), wl.E, wl.seed)
+    check_layer_split(layer, d, w, wl, toks, out, out16)
     del layer
     torch.cuda.empty_cache()

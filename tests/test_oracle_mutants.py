@@ -37,7 +37,8 @@ MUTANTS = {
     "E2M1 drops the sign of zero": ("return (uint8_t)(signbit(x) ? (best | 8) : best);", "return (uint8_t)(x < 0 ? (best | 8) : best);"),
     "SiLU sign": ("return g / (1.0 + exp(-g));", "return g / (1.0 + exp(g));"),
     "gate and up swapped": ("a[i] = silu(g) * u;", "a[i] = silu(u) * g;"),
-    "down weight row index": ("const int64_t r = (int64_t)e * H + h;", "const int64_t r = (int64_t)e * H + (H - 1 - h);"),
+    "down weight row index": ("const int64_t r = (int64_t)e * H + h;", "const int64_t r = (int64_t)e * H + (H - 1 - h);",
+                              2),
     "block scale index": ("orc_e4m3_value(sf[k / 16]) * global;", "orc_e4m3_value(sf[k / 32]) * global;"),
     "combine drops the routing weight": ("o[h] += (double)wts[q] * y;", "o[h] += y;"),
     "permutation not stable": ("        for (int64_t p = 0; p < P; ++p)\n            if (topk_ids[p] == e) {",

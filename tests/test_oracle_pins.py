@@ -747,3 +747,89 @@ def test_router_logits_match_float64_matmul():
     # the only difference is the float64 summation order: at most one FP32 rounding apart
     ulp = np.spacing(np.abs(ref).astype(np.float32))
     assert np.all(np.abs(logits.astype(np.float64) - ref) <= ulp)
+
+
+# ---------------------------------------------------------------------------
+# the layer split at the down projection's input
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [0, 1, 3])
+def test_layer_split_at_the_intermediate_reproduces_the_layer(mode):
+    # The split oracle (SwiGLU output before the intermediate quantisation, then
+    # the down projection and combine from given down inputs) is what the GPU
+    # checks use to hold the two halves of the layer separately; requantising its
+    # FP32 intermediate with the oracle's own quantiser and feeding it back must
+    # give the whole-layer oracle bit for bit, in every mode.
+    wl = inputs.WORKLOADS["tiny"]
+    d = inputs.moe_inputs(wl, T=24)
+    w = {}
+    gl = []
+    for name in ("gate", "up", "down"):
+        c, e8 = d["mx"][name]
+        nt, N, kh = c.shape
+        c2, e4, g, st, _, _ = oracle.transcode(c, e8, nt, N, kh * 2)
+        w[name + "_codes"], w[name + "_sf"] = c2.reshape(c.shape), e4
+        gl.append(g)
+    w["w_global"] = np.stack(gl, 1).astype(np.float32)
+    g_in, g_mid = 0.75, 0.5
+    toks = np.array([3, 0, 23, 11, 11, 7], np.int32)
+    a32, ids, wts = oracle.moe_intermediate(mode, d["x"], d["logits"], None, w["gate_codes"], w["gate_sf"],
+                                            w["up_codes"], w["up_sf"], w["w_global"], g_in, wl.n_group,
+                                            wl.topk_group, wl.top_k, wl.rsf, True, toks)
+    ri, rw = oracle.route(d["logits"][toks], None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf)
+    assert np.array_equal(ids, ri) and np.array_equal(wts.view(np.uint32), rw.view(np.uint32))
+    n, k, I = a32.shape
+    flat = a32.reshape(n * k, I)
+    if mode == 1:
+        c, s = oracle.quantize_f32(flat, g_mid)
+        vals = oracle.decode_nvfp4(c, s, g_mid, n * k, I)
+    elif mode == 3:
+        c, s = oracle.quantize_mxfp8_f32(flat)
+        vals = oracle.decode_mxfp8(c, s)
+    else:
+        bits = np.array([oracle.float_to_bf16(float(v)) for v in flat.reshape(-1)], np.uint32)
+        vals = (bits << 16).view(np.float32).astype(np.float64).reshape(n * k, I)
+    out = oracle.moe_down(vals.reshape(n, k, I), ids, wts, w["down_codes"], w["down_sf"], w["w_global"])
+    ref = oracle.moe_layer(mode, d["x"], d["logits"], None, w["gate_codes"], w["gate_sf"], w["up_codes"],
+                           w["up_sf"], w["down_codes"], w["down_sf"], w["w_global"], g_in, wl.n_group,
+                           wl.topk_group, wl.top_k, wl.rsf, True, toks, act_global_mid=g_mid)
+    assert np.array_equal(out.view(np.uint64), ref.view(np.uint64))
+
+
+def test_intermediate_error_bound_covers_an_fp32_evaluation():
+    # The bound the split checks allow flips within must hold for an FP32
+    # evaluation of the same SwiGLU outputs: gate and up as float32 dot products
+    # of the decoded operands (a plain float32 matmul, its own summation order),
+    # SiLU and the product in float32.  At K = 256 a float32 sum errs by at most
+    # 256 * 2^-24 = 2^-16 of the sum of magnitudes, so 2^-16 is the bound's
+    # accumulation term here.
+    wl = inputs.WORKLOADS["tiny"]
+    d = inputs.moe_inputs(wl, T=16)
+    w = {}
+    gl = []
+    for name in ("gate", "up", "down"):
+        c, e8 = d["mx"][name]
+        nt, N, kh = c.shape
+        c2, e4, g, st, _, _ = oracle.transcode(c, e8, nt, N, kh * 2)
+        w[name + "_codes"], w[name + "_sf"] = c2.reshape(c.shape), e4
+        gl.append(g)
+    w["w_global"] = np.stack(gl, 1).astype(np.float32)
+    toks = np.arange(16, dtype=np.int32)
+    a32, ids, wts, err = oracle.moe_intermediate(0, d["x"], d["logits"], None, w["gate_codes"], w["gate_sf"],
+                                                 w["up_codes"], w["up_sf"], w["w_global"], 1.0, wl.n_group,
+                                                 wl.topk_group, wl.top_k, wl.rsf, True, toks, acc_rel=2.0 ** -16)
+    H, I = wl.H, wl.I
+    x = (d["x"][toks].astype(np.uint32) << 16).view(np.float32)
+    worst = 0.0
+    for t in range(16):
+        for j in range(wl.top_k):
+            e = ids[t, j]
+            wg = oracle.decode_nvfp4(w["gate_codes"][e], w["gate_sf"][e], w["w_global"][e, 0], I, H).astype(np.float32)
+            wu = oracle.decode_nvfp4(w["up_codes"][e], w["up_sf"][e], w["w_global"][e, 1], I, H).astype(np.float32)
+            g32 = wg @ x[t]
+            u32 = wu @ x[t]
+            a = (g32 / (np.float32(1) + np.exp(-g32))) * u32
+            dev = np.abs(a.astype(np.float64) - a32[t, j])
+            assert np.all(dev <= err[t, j]), (t, j, float((dev - err[t, j]).max()))
+            worst = max(worst, float((dev / err[t, j]).max()))
+    assert worst > 0.0
