@@ -54,6 +54,10 @@ def parse():
     ap.add_argument("--cpu-sample-tokens", type=int, default=0, help="oracle tokens per step (0 = host threads)")
     ap.add_argument("--tokens", type=int, default=0, help="override T (smaller cases for profiling)")
     ap.add_argument("--experts", type=int, default=0, help="override E (smaller cases for profiling)")
+    ap.add_argument("--transcode-only", action="store_true",
+                    help="run only the transcode sub-measurement and print its JSON (profiling)")
+    ap.add_argument("--transcode-experts", type=int, default=256,
+                    help="experts of the transcode sub-measurement's layer (smaller cases for profiling)")
     return ap.parse_args()
 
 
@@ -101,8 +105,9 @@ MODE_DTYPES = {0: "bf16 activations x fp4 e2m1 weights (e4m3 block scales), fp16
 GATEUP_TRAFFIC_T8192_E256 = 4 * (652.7936e6 + 21.404928e6)
 GATEUP_W4A8_TRAFFIC_T8192_E256 = 4 * (656.699392e6 + 35.003648e6)
 DECODE_TRAFFIC_T16_E256 = 1010.475e6 + 4.71296e6 + 505.455e6 + 5.101568e6
-# k_transcode of the bench's 768-tensor layer, out of place: not captured yet
-TRANSCODE_TRAFFIC = None
+#  - k_transcode out of place (k_transcode_layer96.txt: 427.9 MB read + 404.6 MB
+#    written for a 96-tensor layer), scaled x8 to the 768-tensor layer timed here.
+TRANSCODE_TRAFFIC_768 = 8 * (427850240 + 404599296)
 
 
 class ClockSampler:
@@ -391,6 +396,10 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     P = peaks()
+    if args.transcode_only:
+        if rank == 0:
+            print(json.dumps(bench_transcode(torch, moe, args, P)), flush=True)
+        return
     wl = workload(args)
     T = wl.T
     # host-side input generation (about a minute at the 8K prefill) runs before
@@ -683,11 +692,12 @@ def bench_router(torch, moe, args, P):
 
 
 def bench_transcode(torch, moe, args, P):
-    """MXFP4 -> NVFP4 transcode of one layer (768 expert tensors), out of place."""
+    """MXFP4 -> NVFP4 transcode of one layer (3 x E expert tensors, E = 256: 768), out of place."""
     rng = np.random.default_rng(inputs.TRANSCODE_SEED)
-    layer = inputs.transcode_layer(rng)
-    codes = np.concatenate([layer["gate"][0], layer["up"][0], layer["down"][0].reshape(256, 2048, 2048)])
-    e8 = np.concatenate([layer["gate"][1], layer["up"][1], layer["down"][1].reshape(256, 2048, 128)])
+    E = args.transcode_experts
+    layer = inputs.transcode_layer(rng, E=E)
+    codes = np.concatenate([layer["gate"][0], layer["up"][0], layer["down"][0].reshape(E, 2048, 2048)])
+    e8 = np.concatenate([layer["gate"][1], layer["up"][1], layer["down"][1].reshape(E, 2048, 128)])
     nt, N, K = codes.shape[0], 2048, 4096  # the down tensors [4096, 2048] have the same block count
     c = torch.from_numpy(codes).cuda()
     s = torch.from_numpy(e8).cuda()
@@ -711,11 +721,12 @@ def bench_transcode(torch, moe, args, P):
     ms = a.elapsed_time(b) / steps
     nbytes = c.numel() * 2 + s.numel() + e4.numel()  # read codes + e8m0, write codes + e4m3
     gbs = nbytes / (ms / 1e3) / 1e9
-    res = {"workload": "transcode: 768 MXFP4 expert tensors (256 experts x gate/up [2048,4096], down [4096,2048]), "
+    res = {"workload": f"transcode: {nt} MXFP4 expert tensors ({E} experts x gate/up [2048,4096], down [4096,2048]), "
                        "out of place", "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
            "tensors_per_s": round(nt / (ms / 1e3), 1), "status": int(status), "report": rep,
            "roofline": {"bound": "hbm", "kernel": "k_transcode", "achieved": round(gbs, 1), "peak": P["hbm_gbs"],
-                        "unit": "GB/s", "frac": round(gbs / P["hbm_gbs"], 4), "traffic": TRANSCODE_TRAFFIC,
+                        "unit": "GB/s", "frac": round(gbs / P["hbm_gbs"], 4),
+                        "traffic": TRANSCODE_TRAFFIC_768 if nt == 768 else None,
                         "traffic_unit": "bytes per launch (ncu dram read+write)",
                         "frac_of_spec": round(gbs / SPEC_HBM_GBS, 4),
                         "algorithmic_bytes_per_launch": int(nbytes)}}

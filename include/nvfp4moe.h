@@ -427,6 +427,23 @@ nvfp4moe_status nvfp4moe_set_trace_events(void* const* events, int32_t n_events)
  * first) or NVFP4MOE_ERR_INVALID_ARG (bad precomputed routing). */
 nvfp4moe_status nvfp4moe_check_device_status(void* stream);
 
+/* Test hooks for the error paths; both inject on the host's side and neither
+ * can fault the GPU.
+ * nvfp4moe_raise_device_error ORs `bits` (1 = timeout, 2 = bad routing; a
+ * non-empty subset, else NVFP4MOE_ERR_INVALID_ARG) into the device error word,
+ * ordered on `stream`.  While the timeout bit is set, every bounded wait of the
+ * GEMM kernels that is not satisfied within a few hundred polls gives up as if
+ * another thread had timed out: the kernels take their error paths (copies and
+ * MMAs already issued are drained before the CTA leaves), their outputs are
+ * undefined, and the next nvfp4moe_check_device_status reports
+ * NVFP4MOE_ERR_TIMEOUT and clears the word.
+ * nvfp4moe_selftest_wait_timeout launches one thread that waits, bounded by
+ * about `limit_cycles` SM clocks (0 .. 4e9), for a barrier nothing arrives on;
+ * when the bound runs out it sets the timeout bit.  Both asynchronous on
+ * `stream`; the context stays usable afterwards. */
+nvfp4moe_status nvfp4moe_raise_device_error(int32_t bits, void* stream);
+nvfp4moe_status nvfp4moe_selftest_wait_timeout(int64_t limit_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

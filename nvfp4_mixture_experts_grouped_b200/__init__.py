@@ -22,7 +22,8 @@ __all__ = [
     "moe_packed_weights_size", "moe_pack_weights", "moe_forward_workspace_size", "moe_forward",
     "moe_forward_ex", "moe_forward_routed", "nvfp4moe_check_device_status", "nvfp4moe_version", "moe_permute",
     "moe_permute_workspace_size", "nvfp4moe_set_trace_events", "moe_permute_noalloc", "W4A16C", "W4A8",
-    "nvfp4_compact_scales", "quantize_mxfp8", "moe_forward_intermediate",
+    "nvfp4_compact_scales", "quantize_mxfp8", "moe_forward_intermediate", "nvfp4moe_raise_device_error",
+    "nvfp4moe_selftest_wait_timeout",
 ]
 
 W4A16 = 0
@@ -117,6 +118,10 @@ def load():
     L.nvfp4moe_set_trace_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     L.nvfp4moe_check_device_status.restype = ctypes.c_int
     L.nvfp4moe_check_device_status.argtypes = [vp]
+    L.nvfp4moe_raise_device_error.restype = ctypes.c_int
+    L.nvfp4moe_raise_device_error.argtypes = [i32, vp]
+    L.nvfp4moe_selftest_wait_timeout.restype = ctypes.c_int
+    L.nvfp4moe_selftest_wait_timeout.argtypes = [ctypes.c_int64, vp]
     _lib = L
     return L
 
@@ -350,3 +355,13 @@ def nvfp4moe_set_trace_events(events) -> None:
 
 def nvfp4moe_check_device_status(stream=None):
     _check(load().nvfp4moe_check_device_status(_stream(stream)))
+
+
+def nvfp4moe_raise_device_error(bits: int, stream=None):
+    """Test hook: ORs `bits` into the device error word (see the header)."""
+    _check(load().nvfp4moe_raise_device_error(int(bits), _stream(stream)))
+
+
+def nvfp4moe_selftest_wait_timeout(limit_cycles: int, stream=None):
+    """Test hook: a bounded wait on a barrier nothing arrives on (see the header)."""
+    _check(load().nvfp4moe_selftest_wait_timeout(int(limit_cycles), _stream(stream)))

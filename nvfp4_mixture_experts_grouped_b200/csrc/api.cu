@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "moe_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace nvfp4moe {
 
@@ -28,16 +29,46 @@ void set_error(const char* fmt, ...) {
 
 __device__ int32_t g_device_error = 0;
 
+unsigned long long current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+
+// The word's device address, cached per device with the id of the context it
+// belongs to: a new context on the device (after cudaDeviceReset, for instance)
+// holds the word at a new address and makes the next call look it up again.
 int32_t* device_error_word() {
     int dev = 0;
-    cudaGetDevice(&dev);
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     static int32_t* cache[64] = {};
+    static unsigned long long cache_ctx[64] = {};
     static std::mutex mu;
+    const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lk(mu);
-    if (dev < 0 || dev >= 64) return nullptr;
-    if (!cache[dev]) {
+    if (!cache[dev] || ctx == 0 || cache_ctx[dev] != ctx) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) cache[dev] = static_cast<int32_t*>(p);
+        cache[dev] = cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess ? static_cast<int32_t*>(p) : nullptr;
+        cache_ctx[dev] = current_context_id();
     }
     return cache[dev];
 }
@@ -555,6 +586,43 @@ nvfp4moe_status nvfp4moe_set_trace_events(void* const* events, int32_t n_events)
         g_trace[i] = static_cast<cudaEvent_t>(events[i]);
     }
     g_trace_on = true;
+    return NVFP4MOE_OK;
+}
+
+// Test hooks for the error paths (host-side injection; nothing here faults).
+namespace {
+__global__ void k_raise_device_error(int32_t* w, int32_t bits) { atomicOr(w, bits); }
+// One thread waits for a phase of a barrier that nothing arrives on; its bounded
+// wait gives up after about limit_cycles and sets the timeout bit.
+__global__ void k_wait_nothing(int32_t* err, long long limit_cycles) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        nvfp4moe::tc::mbar_init(&bar, 1);
+        nvfp4moe::tc::fence_mbar_init();
+        (void)nvfp4moe::tc::mbar_wait(&bar, 0u, err, limit_cycles);
+    }
+}
+}  // namespace
+
+nvfp4moe_status nvfp4moe_raise_device_error(int32_t bits, void* stream) {
+    REQUIRE(bits > 0 && (bits & ~(DEV_ERR_TIMEOUT | DEV_ERR_BAD_ROUTING)) == 0, NVFP4MOE_ERR_INVALID_ARG,
+            "bits=%d must be a non-empty subset of %d", bits, DEV_ERR_TIMEOUT | DEV_ERR_BAD_ROUTING);
+    RETURN_IF(check_device());
+    int32_t* w = device_error_word();
+    if (!w) return fail(NVFP4MOE_ERR_CUDA, "device error word unavailable");
+    k_raise_device_error<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(w, bits);
+    NVFP4MOE_CHECK_LAUNCH("device error injection");
+    return NVFP4MOE_OK;
+}
+
+nvfp4moe_status nvfp4moe_selftest_wait_timeout(int64_t limit_cycles, void* stream) {
+    REQUIRE(limit_cycles >= 0 && limit_cycles <= 4000000000LL, NVFP4MOE_ERR_INVALID_ARG,
+            "limit_cycles=%lld outside [0, 4e9]", (long long)limit_cycles);
+    RETURN_IF(check_device());
+    int32_t* w = device_error_word();
+    if (!w) return fail(NVFP4MOE_ERR_CUDA, "device error word unavailable");
+    k_wait_nothing<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(w, (long long)limit_cycles);
+    NVFP4MOE_CHECK_LAUNCH("bounded-wait self-test");
     return NVFP4MOE_OK;
 }
 

@@ -41,7 +41,11 @@ inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 // expert outside [0, E) or one expert twice for a token.  Only the timeout bit
 // makes the other waits of a kernel give up too.
 enum : int32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_BAD_ROUTING = 2 };
-int32_t* device_error_word();  // device address of the word (current device)
+int32_t* device_error_word();  // device address of the word (current device and context)
+// The driver's id of the calling thread's current CUDA context (unique for the
+// process's lifetime, unlike the context handle, which a new context can reuse);
+// 0 if there is none or the driver does not provide the calls.
+unsigned long long current_context_id();
 
 // Number of SMs of the current device (cached per device).
 int num_sms();

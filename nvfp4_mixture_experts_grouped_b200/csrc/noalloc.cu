@@ -22,33 +22,6 @@ namespace nvfp4moe {
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) uint8_t g_noalloc_permute_scratch[NVFP4MOE_NOALLOC_SCRATCH_BYTES];
 
-// The driver's id of the calling thread's current context (unique for the
-// process's lifetime, unlike the context handle, which a new context can reuse);
-// 0 if there is none or the driver does not provide the calls.
-static unsigned long long current_context_id() {
-    using GetCurrent = CUresult (*)(CUcontext*);
-    using GetId = CUresult (*)(CUcontext, unsigned long long*);
-    static GetCurrent get_current = nullptr;
-    static GetId get_id = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_current = reinterpret_cast<GetCurrent>(p);
-        p = nullptr;
-        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_id = reinterpret_cast<GetId>(p);
-    });
-    CUcontext ctx = nullptr;
-    unsigned long long id = 0;
-    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
-        return 0;
-    return id;
-}
-
 static void* noalloc_scratch_address(nvfp4moe_status* st) {
     static std::mutex mu;
     static void* cache[64] = {};

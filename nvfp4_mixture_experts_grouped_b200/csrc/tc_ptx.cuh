@@ -81,6 +81,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
     }
 }
 
+// Drain wait of an error path: waits (bounded, ignoring the error word) for the
+// phase with the given parity, so that copies or MMAs already issued have landed
+// before the CTA frees what they write into.  Returns false if it gave up.
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, long long limit_cycles = 200000000LL) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait<CLUSTER>(bar, parity))
+        if (clock64() - t0 > limit_cycles) return false;
+    return true;
+}
+
 // ---------------------------------------------------------------------------
 // readiness flags: sequence numbers in shared memory, stored by the threads that
 // finished a piece of work and polled with plain loads by the thread that

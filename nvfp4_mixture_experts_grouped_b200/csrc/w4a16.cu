@@ -335,7 +335,14 @@ __device__ __forceinline__ bool w16_stream(Ring& r, const uint8_t* pair, int chu
     for (int grp = 0; grp < groups; ++grp) {
         const uint32_t n = base + grp;
         const int stage = n % STAGES;
-        if (!tc::mbar_wait(&r.bar[stage], (n / STAGES) & 1u, err)) return false;
+        if (!tc::mbar_wait(&r.bar[stage], (n / STAGES) & 1u, err)) {
+            // error path: the bulk copies already issued into this warp's ring land
+            // before the warp leaves
+            if (lane == 0)
+                for (int i = grp; i < min(grp + STAGES, groups); ++i)
+                    tc::mbar_drain(&r.bar[(base + i) % STAGES], ((base + i) / STAGES) & 1u);
+            return false;
+        }
         const uint8_t* st = r.buf + stage * W16Cfg<CH>::STAGE;
 #pragma unroll
         for (int cc = 0; cc < CH; ++cc) {

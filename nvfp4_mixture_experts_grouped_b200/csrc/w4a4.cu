@@ -178,7 +178,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint64_t* empty = sf_ready + STAGES;  // both CTAs: the even CTA's MMA commits
     uint64_t* acc_full = empty + STAGES;  // both CTAs: the even CTA's MMA commits
     uint64_t* acc_empty = acc_full + 1;   // even CTA only: both CTAs' epilogue warps
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+    uint64_t* drain = acc_empty + 1;      // even CTA only: the MMAs of an error path
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
     const uint32_t rank = tc::cluster_ctarank();  // 0: issues the MMAs of the pair
     const int warp = warp_id(), lane = lane_id();
@@ -190,6 +191,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         tc::mbar_init(acc_full, 1);
         tc::mbar_init(acc_empty, 2 * EPI_WARPS);
+        tc::mbar_init(drain, 1);
         tc::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -234,7 +236,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 for (int ks = 0; ks < ks_count; ++ks, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!tc::mbar_wait<true>(&empty[s], ph ^ 1u, p.err)) goto done;
+                    if (!tc::mbar_wait<true>(&empty[s], ph ^ 1u, p.err)) goto drain_loads;
                     // scale atoms of this stage per 128 rows (a partial last stage: W4A4 only)
                     const int na = KIND == KIND_NVF4 ? min(4, ksub_total - ks * 4) : 1;
                     uint8_t* st = smem + s * STAGE_BYTES;
@@ -259,7 +261,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             // wait for the MMA's release of every slot still in use, so that no
             // completion signal of the other CTA lands after this CTA has finished
             for (int i = it; i < it + STAGES; ++i)
-                if (!tc::mbar_wait<true>(&empty[i % STAGES], ((uint32_t)(i / STAGES) & 1u) ^ 1u, p.err)) goto done;
+                if (!tc::mbar_wait<true>(&empty[i % STAGES], ((uint32_t)(i / STAGES) & 1u) ^ 1u, p.err))
+                    goto drain_loads;
+            goto producer_done;
+        drain_loads:
+            // error path: the copies of the last STAGES issued stages land before the
+            // CTA leaves (a full barrier completes when its bytes have arrived)
+            for (int i = max(0, it - STAGES); i < it; ++i) tc::mbar_drain(&full[i % STAGES], (uint32_t)(i / STAGES) & 1u);
+        producer_done:;
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -321,13 +330,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 } else {
                     ++ks;
                 }
-                if (!ok) goto done;
+                if (!ok) goto drain_mma;
                 tc::tc_fence_after();
                 s = ns;
                 ph = nph;
                 adesc = ns == 0 ? adesc0 : adesc + STAGE_DESC;
                 sf_col = ns == 0 ? tmem + TM_SF : sf_col + TM_SF_STRIDE;
             }
+            goto mma_done;
+        drain_mma:
+            // error path: the MMAs already issued complete before TMEM is freed
+            tc::tc_commit_pair(drain, 0x1);
+            tc::mbar_drain(drain, 0u);
+        mma_done:;
         }
     } else if (warp >= 2 + EPI_WARPS) {
         // ------------------------------------------------------------ scale warps

@@ -5,7 +5,9 @@ after the call every margin byte is still 0xFF.  The workspace itself also start
 full of 0xFF (NaN patterns in every float view of it): the outputs must be
 bit-identical to those of a call on a zeroed workspace, so nothing the kernels
 read from the workspace can be a byte they did not write first.  The same for
-the transcode's outputs and workspace."""
+the transcode's outputs and workspace.  Then the error paths: a bounded wait
+that runs out reports a timeout, and GEMM kernels that give up mid-flight leave
+the context usable."""
 from __future__ import annotations
 
 import numpy as np
@@ -79,3 +81,50 @@ def test_transcode_writes_nothing_outside_its_buffers():
     for big in (co_big, e4_big, g_big, st_big, ws_big):
         assert margins_untouched(big)
     assert torch.equal(co.cpu(), c.view(torch.uint8).reshape(-1).cpu())
+
+
+# ---------------------------------------------------------------------------
+# error paths: a bounded wait that runs out, and GEMM kernels that give up
+# mid-flight; the failure is injected on the host's side and faults nothing
+# ---------------------------------------------------------------------------
+TIMEOUT = 8  # NVFP4MOE_ERR_TIMEOUT
+
+
+def test_bounded_wait_runs_out_and_reports_timeout():
+    moe.nvfp4moe_check_device_status()
+    moe.nvfp4moe_selftest_wait_timeout(2_000_000)  # ~1 ms of SM clocks, then the wait gives up
+    with pytest.raises(moe.NVFP4MoEError) as e:
+        moe.nvfp4moe_check_device_status()
+    assert e.value.status == TIMEOUT
+    moe.nvfp4moe_check_device_status()  # the word was cleared: OK again
+
+
+@pytest.mark.parametrize("mode", [moe.W4A4, moe.W4A8, moe.W4A16])
+def test_gemm_error_path_leaves_the_context_usable(mode):
+    # With the timeout bit raised before the call, every GEMM wait that is not
+    # satisfied at once gives up and the kernels leave through their error paths
+    # (draining the copies and MMAs they issued).  The status says so, and the
+    # next call on the same context gives the bits of a clean call.
+    wl = inputs.WORKLOADS["tiny"]
+    T = 300
+    d = inputs.moe_inputs(wl, T=T)
+    w = nvfp4_weights_from_inputs(d, False)
+    layer = GpuLayer(mode, w, T, wl.n_group, wl.topk_group, wl.top_k)
+    x, lg = bf16_tensor(d["x"]), dev(d["logits"])
+    ref, _, _ = layer.forward(x, lg, out_fp32=True)
+    ref = ref.clone()
+    moe.nvfp4moe_raise_device_error(1)
+    out = torch.empty_like(ref)
+    moe.moe_forward(mode, x, lg, None, layer.packed, 1.0, T, wl.H, wl.I, wl.E, wl.n_group, wl.topk_group, wl.top_k,
+                    wl.rsf, True, layer.ws, out)
+    with pytest.raises(moe.NVFP4MoEError) as e:
+        moe.nvfp4moe_check_device_status()
+    assert e.value.status == TIMEOUT
+    again, _, _ = layer.forward(x, lg, out_fp32=True)
+    assert torch.equal(again.view(torch.int32), ref.view(torch.int32))
+
+
+def test_raise_device_error_rejects_unknown_bits():
+    for bits in (0, 4, -1):
+        with pytest.raises(moe.NVFP4MoEError):
+            moe.nvfp4moe_raise_device_error(bits)
