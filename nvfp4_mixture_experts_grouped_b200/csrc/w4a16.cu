@@ -196,6 +196,10 @@ __global__ void k_w16_pack(const uint8_t* __restrict__ codes, const uint8_t* __r
 // t) are 32 consecutive bytes, so a lane fetches a step's B fragment (b0, b1)
 // with one 8-byte load.
 // ---------------------------------------------------------------------------
+// NCH > 0: rows of K = 256 * NCH elements, each lane's NCH 16-byte pieces loaded
+// once and held in registers (one memory round trip per row instead of two
+// passes of dependent loads); NCH == 0: any K (a multiple of 8), two passes.
+template <int NCH>
 __global__ void __launch_bounds__(256)
     k_rows_to_f16(const uint16_t* __restrict__ src, int64_t rows, int K, __half* __restrict__ dst,
                   float* __restrict__ inv_scale) {
@@ -203,9 +207,18 @@ __global__ void __launch_bounds__(256)
     if (r >= rows) return;
     const int lane = lane_id();
     const uint4* s = reinterpret_cast<const uint4*>(src + r * K);
+    // lane's pieces: i = lane + 32 c < K / 8
+    const int n_c = NCH > 0 ? NCH : (K / 8 - lane + 31) / 32;
+    constexpr int HELD = NCH > 0 ? NCH : 1;
+    uint4 held[HELD];
+    if (NCH > 0) {
+#pragma unroll
+        for (int c = 0; c < HELD; ++c) held[c] = s[lane + 32 * c];
+    }
     float amax = 0.0f;
-    for (int i = lane; i < K / 8; i += 32) {
-        const uint4 v = s[i];
+#pragma unroll
+    for (int c = 0; c < n_c; ++c) {
+        const uint4 v = NCH > 0 ? held[c < HELD ? c : 0] : s[lane + 32 * c];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q)
@@ -220,8 +233,10 @@ __global__ void __launch_bounds__(256)
         sh = 15 - e;       // amax * 2^sh in [2^14, 2^15)
     }
     uint32_t* d = reinterpret_cast<uint32_t*>(dst + r * K);
-    for (int i = lane; i < K / 8; i += 32) {
-        const uint4 v = s[i];
+#pragma unroll
+    for (int c = 0; c < n_c; ++c) {
+        const int i = lane + 32 * c;
+        const uint4 v = NCH > 0 ? held[c < HELD ? c : 0] : s[i];
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t o[4];
 #pragma unroll
@@ -237,6 +252,17 @@ __global__ void __launch_bounds__(256)
         for (int q = 0; q < 4; ++q) d[wbase + q * 8] = o[q];
     }
     if (lane == 0) inv_scale[r] = ldexpf(1.0f, -sh);
+}
+
+static void launch_rows_to_f16(const uint16_t* src, int64_t rows, int K, __half* dst, float* inv_scale,
+                               cudaStream_t stream) {
+    const unsigned grid = (unsigned)ceil_div(rows, 8);
+    if (K == 4096)
+        k_rows_to_f16<16><<<grid, 256, 0, stream>>>(src, rows, K, dst, inv_scale);
+    else if (K == 2048)
+        k_rows_to_f16<8><<<grid, 256, 0, stream>>>(src, rows, K, dst, inv_scale);
+    else
+        k_rows_to_f16<0><<<grid, 256, 0, stream>>>(src, rows, K, dst, inv_scale);
 }
 
 // Four E4M3 scales (bytes 0..3 of `w`) -> two FP16x2 (exact): bytes 0, 1 and 2, 3.
@@ -642,7 +668,7 @@ static nvfp4moe_status run_w16(const uint16_t* x, const uint8_t* p, const W16Lay
     int32_t* err = device_error_word();
     NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_gateup<COMPACT, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM));
     NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w16_down<COMPACT, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM));
-    k_rows_to_f16<<<(unsigned)ceil_div(T, 8), 256, 0, stream>>>(x, T, H, x16, x_inv);
+    launch_rows_to_f16(x, T, H, x16, x_inv, stream);
     NVFP4MOE_CHECK_LAUNCH("w4a16 activation conversion");
     {
         const int64_t ctas = std::min<int64_t>(ceil_div(max_active * (I / 16), W16_WARPS), max_ctas);
@@ -651,7 +677,7 @@ static nvfp4moe_status run_w16(const uint16_t* x, const uint8_t* p, const W16Lay
         NVFP4MOE_CHECK_LAUNCH("w4a16 gate/up kernel");
     }
     if (mid_event) cudaEventRecord(mid_event, stream);
-    k_rows_to_f16<<<(unsigned)ceil_div(P, 8), 256, 0, stream>>>(A2, P, I, a16, a_inv);
+    launch_rows_to_f16(A2, P, I, a16, a_inv, stream);
     NVFP4MOE_CHECK_LAUNCH("w4a16 intermediate conversion");
     {
         const int64_t ctas = std::min<int64_t>(ceil_div(max_active * (H / 32), W16_WARPS), max_ctas);

@@ -360,6 +360,43 @@ def test_layer_decode_w4a16_full():
     check_layer_split(layer, d, w, wl, np.arange(wl.T, dtype=np.int32), out, out16)
 
 
+def test_layer_w4a16_wide_dynamic_range_rows():
+    # W4A16 multiplies FP16 rows (each BF16 row scaled by a power of two so that
+    # its largest element sits just below 2^15) on FP16 tensor cores: elements
+    # far below their row's largest lose relative precision as FP16 subnormals.
+    # Rows spanning 2^36 (one element of 2^16 among N(0,1) x 2^-20 ones), a zero
+    # row and a row at 2^-60 (its SwiGLU products near 2^-110, still normal FP32)
+    # are held to the oracle token by token.
+    wl = inputs.WORKLOADS["decode"]
+    d = inputs.moe_inputs(wl)
+    rng = np.random.default_rng(77)
+    x = (rng.standard_normal((wl.T, wl.H)) * 2.0 ** -20).astype(np.float32)
+    cols = rng.integers(0, wl.H, size=wl.T)
+    x[np.arange(wl.T), cols] = np.where(rng.random(wl.T) < 0.5, -1.0, 1.0) * 2.0 ** 16
+    x[3] = 0.0
+    x[5] = rng.standard_normal(wl.H).astype(np.float32) * 2.0 ** -60
+    x[9] = rng.standard_normal(wl.H).astype(np.float32)  # an ordinary row beside them
+    d["x"] = inputs.bf16_bits(x)
+    w = nvfp4_weights_from_inputs(d, False)
+    layer = GpuLayer(moe.W4A16, w, wl.T, wl.n_group, wl.topk_group, wl.top_k)
+    out, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]), out_fp32=True)
+    ref = oracle_layer(moe.W4A16, d, w, wl)
+    got = out_to_f64(out)
+    assert np.all(got[3] == 0.0) and np.all(ref[3] == 0.0)
+    assert np.any(ref[5] != 0.0)
+    for t in range(wl.T):
+        if t != 3:
+            compare_layer(got[t:t + 1], ref[t:t + 1])
+    out16, _, _ = layer.forward(bf16_tensor(d["x"]), dev(d["logits"]))
+    for t in range(wl.T):
+        if t != 3:
+            compare_layer(out_to_f64(out16)[t:t + 1], ref[t:t + 1], bf16_output=True)
+    # (no split check here: its error model is the FP32 accumulation alone, and
+    # the intermediates these rows make through a zero weight at the outlier's
+    # column come from the FP16-subnormal elements only -- large relative error
+    # on values that are negligible in the output, which the bounds above hold)
+
+
 @pytest.mark.parametrize("name", ["prefill", "skewed"])
 def test_layer_w4a4_full_size_sampled(name):
     # full-size layers: at least 512 seeded tokens whose rows cover every
