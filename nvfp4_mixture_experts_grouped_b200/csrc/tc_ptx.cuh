@@ -93,48 +93,6 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, long 
 }
 
 // ---------------------------------------------------------------------------
-// readiness flags: sequence numbers in shared memory, stored by the threads that
-// finished a piece of work and polled with plain loads by the thread that
-// consumes it (cheaper per check than an mbarrier wait).  The stores are relaxed:
-// they only signal work that is complete when they issue (a tcgen05.st followed
-// by its tcgen05.wait::st), as the relaxed remote mbarrier arrive does; a
-// release at cluster scope costs the storing thread ~1300 cycles.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void flag_store_local(uint32_t* f, uint32_t v) {
-    asm volatile("st.relaxed.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(f)), "r"(v) : "memory");
-}
-__device__ __forceinline__ void flag_store_remote(uint32_t f_cluster_addr, uint32_t v) {
-    asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(f_cluster_addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint4 flags_load4(const uint32_t* f) {
-    uint4 r;
-    asm volatile("ld.volatile.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "r"(smem_u32(f))
-                 : "memory");
-    return r;
-}
-// All eight flags f[0..7] (16-byte aligned) at least `seq`; bounded like mbar_wait.
-__device__ __forceinline__ bool flags8_ready(const uint32_t* f, uint32_t seq) {
-    const uint4 a = flags_load4(f), b = flags_load4(f + 4);
-    return min(min(min(a.x, a.y), min(a.z, a.w)), min(min(b.x, b.y), min(b.z, b.w))) >= seq;
-}
-__device__ __forceinline__ bool flags8_wait(const uint32_t* f, uint32_t seq, int32_t* err,
-                                            long long limit_cycles = 4000000000LL) {
-    if (flags8_ready(f, seq)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        for (int i = 0; i < 64; ++i)
-            if (flags8_ready(f, seq)) return true;
-        if (clock64() - t0 > limit_cycles) {
-            atomicOr(err, 1);
-            return false;
-        }
-        if (*(volatile int32_t*)err & 1) return false;
-    }
-}
-
-// ---------------------------------------------------------------------------
 // thread-block clusters (CTA pairs)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -180,16 +138,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
-}
-
-// L2-only prefetches (no shared-memory destination, no completion tracking).
-__device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int32_t x, int32_t y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap), "r"(x), "r"(y)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
@@ -338,20 +286,6 @@ __device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, float va[1
         va[i] = __uint_as_float(r[i]);
         vb[i] = __uint_as_float(r[16 + i]);
     }
-}
-
-// 32 lanes x 32 bit: this thread's row, 32 consecutive columns from `ta`, with
-// the wait inside the same asm block (as tmem_ld16x2).
-__device__ __forceinline__ void tmem_ld32(uint32_t ta, float v[32]) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(ta)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 }  // namespace tc
