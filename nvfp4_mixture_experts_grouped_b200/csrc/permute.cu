@@ -413,14 +413,100 @@ nvfp4moe_status launch_quantize_linear(const uint16_t* x, int64_t M, int64_t K, 
     return NVFP4MOE_OK;
 }
 
+// Scatter form for rows of up to NG * 1024 elements: one warp per token; the
+// token's row is quantised once into registers -- lane l takes the two blocks
+// 64g + 2l, 64g + 2l + 1 of each 64-block group g (32 elements, all loads issued
+// before any arithmetic) -- and then written to each of its k permuted rows with
+// one 16-byte store per group (a warp store instruction covers 512 contiguous
+// bytes) and one scale word per lane pair (blocks 4q .. 4q + 3 of the atom row,
+// assembled by one shuffle).  The same block quantiser as k_quantize: the same
+// bytes, with the address arithmetic of a destination row done once per row
+// instead of once per block.  Needs K % 64 == 0 (so a lane pair is all in or all
+// out of the row).
+template <bool BF16_UNIT, int NG>
+__global__ void __launch_bounds__(256)
+    k_quantize_scatter(const uint16_t* __restrict__ x, int64_t M, int64_t K, float gs, uint8_t* __restrict__ codes,
+                       uint8_t* __restrict__ scales, const int32_t* __restrict__ row_of_pair, int k) {
+    const int64_t m = (int64_t)blockIdx.x * 8 + warp_id();
+    if (m >= M) return;
+    const int lane = lane_id();
+    const int64_t nb = K / 16;
+    const uint16_t* xr = x + m * K;
+    const int my_row = lane < k ? row_of_pair[m * k + lane] : 0;
+    uint4 v[NG][4];
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        const int64_t b = 64 * g + 2 * lane;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            v[g][i] = b < nb ? __ldg(reinterpret_cast<const uint4*>(xr + b * 16) + i) : make_uint4(0, 0, 0, 0);
+    }
+    uint4 cw[NG];      // codes of the lane's two blocks of group g
+    uint32_t sw[NG];   // even lanes: the scale word of blocks 64g + 2l .. + 3
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        uint32_t c[4], sf[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float f[16];
+            const uint32_t w[8] = {v[g][2 * h].x, v[g][2 * h].y, v[g][2 * h].z, v[g][2 * h].w,
+                                   v[g][2 * h + 1].x, v[g][2 * h + 1].y, v[g][2 * h + 1].z, v[g][2 * h + 1].w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                f[2 * i] = bf16_bits_to_float(w[i] & 0xFFFFu);
+                f[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+            }
+            sf[h] = quantize_block16<BF16_UNIT>(f, gs, c[2 * h], c[2 * h + 1]);
+        }
+        cw[g] = make_uint4(c[0], c[1], c[2], c[3]);
+        const uint32_t pair = sf[0] | (sf[1] << 8);
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, pair, 1);
+        sw[g] = pair | (other << 16);
+    }
+    for (int j = 0; j < k; ++j) {
+        const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
+        uint8_t* crow = codes + row * (K / 2);
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            const int64_t b = 64 * g + 2 * lane;
+            if (b < nb) {
+                *reinterpret_cast<uint4*>(crow + b * 8) = cw[g];
+                if ((lane & 1) == 0) *reinterpret_cast<uint32_t*>(scales + sf_atom_offset(row, b, nb)) = sw[g];
+            }
+        }
+    }
+}
+
+template <bool BF16_UNIT>
+static void launch_scatter_ng(int ng, const uint16_t* x, int64_t T, int64_t H, float gs, uint8_t* codes,
+                              uint8_t* scales, const int32_t* row_of_pair, int k, cudaStream_t stream) {
+    const unsigned grid = (unsigned)ceil_div(T, 8);
+    switch (ng) {
+        case 1: k_quantize_scatter<BF16_UNIT, 1><<<grid, 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k); break;
+        case 2: k_quantize_scatter<BF16_UNIT, 2><<<grid, 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k); break;
+        case 3: k_quantize_scatter<BF16_UNIT, 3><<<grid, 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k); break;
+        case 4: k_quantize_scatter<BF16_UNIT, 4><<<grid, 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k); break;
+        case 5: k_quantize_scatter<BF16_UNIT, 5><<<grid, 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k); break;
+        case 6: k_quantize_scatter<BF16_UNIT, 6><<<grid, 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k); break;
+        case 7: k_quantize_scatter<BF16_UNIT, 7><<<grid, 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k); break;
+        default: k_quantize_scatter<BF16_UNIT, 8><<<grid, 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k); break;
+    }
+}
+
 nvfp4moe_status launch_quantize_scatter(const uint16_t* x, int64_t T, int64_t H, float gs, uint8_t* codes,
                                         uint8_t* scales, const int32_t* row_of_pair, int k, cudaStream_t stream) {
     if (T == 0) return NVFP4MOE_OK;
-    if (gs == 1.0f)
+    const int64_t ng = (H / 16 + 63) / 64;  // 64-block groups per row
+    if (ng <= 8) {
+        // the row held in registers: one pass, 16-byte stores
+        if (gs == 1.0f) launch_scatter_ng<true>((int)ng, x, T, H, gs, codes, scales, row_of_pair, k, stream);
+        else launch_scatter_ng<false>((int)ng, x, T, H, gs, codes, scales, row_of_pair, k, stream);
+    } else if (gs == 1.0f) {
         k_quantize<true, true><<<(unsigned)ceil_div(T, 8), 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair, k);
-    else
+    } else {
         k_quantize<true, false><<<(unsigned)ceil_div(T, 8), 256, 0, stream>>>(x, T, H, gs, codes, scales, row_of_pair,
                                                                              k);
+    }
     NVFP4MOE_CHECK_LAUNCH("quantize-scatter kernel");
     return NVFP4MOE_OK;
 }
