@@ -58,6 +58,8 @@ def parse():
                     help="run only the transcode sub-measurement and print its JSON (profiling)")
     ap.add_argument("--transcode-experts", type=int, default=256,
                     help="experts of the transcode sub-measurement's layer (smaller cases for profiling)")
+    ap.add_argument("--router-only", action="store_true",
+                    help="run only the router sub-measurement and print its JSON (profiling)")
     return ap.parse_args()
 
 
@@ -396,9 +398,10 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     P = peaks()
-    if args.transcode_only:
+    if args.transcode_only or args.router_only:
         if rank == 0:
-            print(json.dumps(bench_transcode(torch, moe, args, P)), flush=True)
+            sub = bench_transcode if args.transcode_only else bench_router
+            print(json.dumps(sub(torch, moe, args, P)), flush=True)
         return
     wl = workload(args)
     T = wl.T
@@ -685,7 +688,8 @@ def bench_router(torch, moe, args, P):
                         f"FP32 router, {layers} layers' routers rotated (> L2)",
             "value": round(us, 2), "unit": "us per layer (CUDA graph of 47 layers' calls)",
             "higher_is_better": False, "eager_us_per_call": round(eager_us, 2),
-            "roofline": {"bound": "hbm", "kernel": "k_router_topk", "achieved": round(gbs, 1), "peak": P["hbm_gbs"],
+            "roofline": {"bound": "hbm", "kernel": "k_router_logits + k_route_rows", "achieved": round(gbs, 1),
+                         "peak": P["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / P["hbm_gbs"], 4), "traffic": None,
                          "frac_of_spec": round(gbs / SPEC_HBM_GBS, 4),
                          "algorithmic_bytes_per_launch": int(nbytes)}}

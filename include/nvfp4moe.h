@@ -158,7 +158,7 @@ nvfp4moe_status moe_route(const float* logits, const float* bias, int32_t T, int
                           int32_t* topk_ids, float* topk_weights, void* stream);
 
 /* ------------------------------------------------------------------------- */
-/* Router projection fused with the grouped top-k                             */
+/* Router projection followed by the grouped top-k                           */
 /* ------------------------------------------------------------------------- */
 /* Operation ("MiMo-V2.6-Flash-MOPD on one RTX PRO 6000", "Speed v6" and "What
  * makes it fast": the router's matmul followed by a fused top-k; routers kept
@@ -167,12 +167,12 @@ nvfp4moe_status moe_route(const float* logits, const float* bias, int32_t T, int
  * arithmetic (BF16 hidden rows, FP32 router rows; each logit summed in a fixed
  * order, so repeated calls give the same bits), written to logits_out, then
  * routed exactly as moe_route routes logits_out (same ids and weight bits).
- * One kernel launch (plus a 4-byte-per-16-tokens clear of the workspace).
+ * Two kernel launches: the projection, then moe_route's routing kernel.
  *   x_bf16 [T, H] bf16 bits; w_router [E, H] f32; bias [E] f32 or NULL;
  *   logits_out [T, E] f32; topk_ids [T, top_k] i32; topk_weights [T, top_k]
  *   f32 (caller-owned device memory); workspace: device, at least
- *   moe_router_topk_workspace_size(T) bytes, caller-owned, left all-zero on
- *   return; calls sharing one workspace must be ordered (one stream).
+ *   moe_router_topk_workspace_size(T) bytes, caller-owned; this version
+ *   neither reads nor writes it (the size is kept so callers need not change).
  * Constraints: as moe_route, plus H >= 256 with H % 256 == 0 and E % 4 == 0;
  * all pointers 16-byte aligned.  Meant for decode-sized T (the router is read
  * once per 16 tokens).                                                        */

@@ -70,7 +70,7 @@ def test_router_topk_matches_oracle(name):
     rid, rw = oracle.route(logits, bias, ng, tg, k, 2.827, True)
     assert np.array_equal(ids, rid)
     assert np.array_equal(wts.view(np.uint32), rw.view(np.uint32))
-    # the per-tile counters are left zero for the next call
+    # the workspace is not touched
     assert not ws.any()
 
 
