@@ -1,4 +1,4 @@
-"""GPU parity of the router projection fused with grouped top-k
+"""GPU parity of the router projection followed by grouped top-k
 (moe_router_topk) against the oracle.
 
 Logits: FP32 against the float64 oracle within the rounding bound of the
@@ -29,6 +29,9 @@ CASES = {
     "general_groups_ragged": (40, 512, 96, 4, 2, 6, True, 14),
     "many_tiles": (300, 1024, 256, 8, 4, 8, False, 15),
     "one_group": (20, 768, 64, 1, 1, 8, False, 16),
+    # hidden rows too long for the shared-memory tile (16 x 8192 BF16 = 256 KB):
+    # the projection reads them from global memory in its loop
+    "long_rows": (24, 8192, 64, 8, 4, 8, True, 17),
 }
 
 
