@@ -142,7 +142,7 @@ static int64_t al(int64_t v) { return (v + 255) / 256 * 256; }
 static ForwardLayout forward_layout(nvfp4moe_mode mode, int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
     ForwardLayout L{};
     L.P = T * k;
-    const bool tc = mode == NVFP4MOE_W4A4 || mode == NVFP4MOE_W4A8;  // tcgen05 GEMMs on 128-row tiles
+    const bool tc = mode == NVFP4MOE_W4A4 || mode == NVFP4MOE_W4A8;  // tcgen05 GEMMs, rows padded to 128
     L.pad = tc ? MTILE : 1;
     const int64_t occupied = std::min<int64_t>(E, L.P);
     L.rows_max = tc ? round_up(L.P + occupied * (MTILE - 1), MTILE) : std::max<int64_t>(L.P, 1);
@@ -489,6 +489,8 @@ static nvfp4moe_status forward_common(nvfp4moe_mode mode, const uint16_t* x, con
         RETURN_IF(launch_check_routing(ids_in, wts_in, T, top_k, E, plan.ids, plan.wts, st));
     }
     trace(1, st);
+    if (mode == NVFP4MOE_W4A4 || mode == NVFP4MOE_W4A8)
+        plan.tile_rows = w4a4_tile_rows(T, top_k, E);  // the GEMMs' tile form
     RETURN_IF(launch_permute(plan.ids, T, top_k, E, L.pad, plan, st));
     trace(2, st);
     void* Y = ws + L.y;

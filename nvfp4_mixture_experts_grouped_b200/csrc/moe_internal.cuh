@@ -12,8 +12,7 @@ namespace nvfp4moe {
 
 constexpr int PERM_CHUNK = 256;  // tokens per permutation chunk (one CTA)
 constexpr int PERM_WARPS = PERM_CHUNK / 32;
-constexpr int MTILE = 128;       // rows of one tcgen05 M-tile per CTA (the row padding of the GEMM paths)
-constexpr int PAIR_ROWS = 256;   // rows of a pair tile (tokens as the MMA's M, 128 per CTA)
+constexpr int MTILE = 128;       // rows of one tcgen05 M-tile (the row padding and tile size of the GEMM paths)
 
 __device__ __forceinline__ int64_t round_up_dev(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
@@ -27,10 +26,11 @@ struct RoutingPlan {
     int32_t* pad_offsets;   // [E+1] row offsets with every segment padded to `pad`
     int32_t* row_of_pair;   // [T*k]
     int32_t* pair_of_row;   // [rows_max]
-    int4* tiles;            // [max_tiles] {expert, first padded row, valid rows (<= 256), tile index in expert}
+    int4* tiles;            // [max_tiles] {expert, first padded row, valid rows (<= tile_rows), tile index in expert}
     int32_t* n_tiles;       // [1]
     int32_t* active;        // [E] experts with at least one row
     int32_t* n_active;      // [1]
+    int tile_rows = MTILE;  // rows per tile of the tile list: MTILE or 2 * MTILE (a CTA pair's tile)
 };
 
 // transcode.cu
@@ -103,7 +103,10 @@ nvfp4moe_status launch_w4a16_layer(const uint16_t* x, const void* packed, bool c
 bool make_map(CUtensorMap* m, const void* base, int64_t row_bytes, int64_t rows, int box_rows);
 bool make_map_u4(CUtensorMap* m, const void* base, int64_t k_elems, int64_t rows, int box_rows);
 
-// w4a4.cu: the tcgen05 pair GEMMs; mx8 selects W4A8 (MXFP8 activations x FP4
+// w4a4.cu: rows per tile of the tile list the W4A4 / W4A8 GEMMs are cut for at
+// this shape (MTILE: single-CTA tiles; 2 * MTILE: CTA-pair tiles)
+int w4a4_tile_rows(int64_t T, int k, int E);
+// w4a4.cu: the tcgen05 GEMMs; mx8 selects W4A8 (MXFP8 activations x FP4
 // weights held in the padded form with E8M0 scales) instead of W4A4
 size_t w4a4_packed_size(int E, int H, int I, bool mx8);
 nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed, bool mx8, cudaStream_t stream);

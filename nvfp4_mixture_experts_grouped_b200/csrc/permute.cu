@@ -90,7 +90,8 @@ __global__ void __launch_bounds__(1024)
     const int padded = e < E ? (int)round_up_dev(cnt, pad) : 0;
     int ptotal;
     const int poff = block_exclusive_scan(padded, s_tmp, ptotal);
-    const int tiles = e < E ? (cnt + PAIR_ROWS - 1) / PAIR_ROWS : 0;
+    const int tr = plan.tile_rows;
+    const int tiles = e < E ? (cnt + tr - 1) / tr : 0;
     int ttotal;
     const int toff = block_exclusive_scan(tiles, s_tmp, ttotal);
     int atotal;
@@ -100,7 +101,7 @@ __global__ void __launch_bounds__(1024)
         plan.offsets[e] = off;
         plan.pad_offsets[e] = poff;
         for (int j = 0; j < tiles; ++j)
-            plan.tiles[toff + j] = make_int4(e, poff + j * PAIR_ROWS, min(PAIR_ROWS, cnt - j * PAIR_ROWS), j);
+            plan.tiles[toff + j] = make_int4(e, poff + j * tr, min(tr, cnt - j * tr), j);
         if (cnt > 0) plan.active[aoff] = e;
     }
     if (e == 0) {
@@ -200,7 +201,8 @@ __global__ void __launch_bounds__(1024)
     const int off = block_exclusive_scan(cnt, s_tmp, total);
     const int padded = tid < E ? (int)round_up_dev(cnt, pad) : 0;
     const int poff = block_exclusive_scan(padded, s_tmp, ptotal);
-    const int tiles = tid < E ? (cnt + PAIR_ROWS - 1) / PAIR_ROWS : 0;
+    const int tr = plan.tile_rows;
+    const int tiles = tid < E ? (cnt + tr - 1) / tr : 0;
     const int toff = block_exclusive_scan(tiles, s_tmp, ttotal);
     const int aoff = block_exclusive_scan(tid < E && cnt > 0 ? 1 : 0, s_tmp, atotal);
     if (tid < E) {
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(1024)
         plan.pad_offsets[tid] = poff;
         s_poff[tid] = poff;
         for (int j = 0; j < tiles; ++j)
-            plan.tiles[toff + j] = make_int4(tid, poff + j * PAIR_ROWS, min(PAIR_ROWS, cnt - j * PAIR_ROWS), j);
+            plan.tiles[toff + j] = make_int4(tid, poff + j * tr, min(tr, cnt - j * tr), j);
         if (cnt > 0) plan.active[aoff] = tid;
     }
     if (tid == 0) {

@@ -6,18 +6,17 @@
 // W4A4 NVFP4 on native FP4 tensor cores) and "Why a unit activation scale".
 // Expert MLP: "MiMo-V2.6-Flash -- REAP-50", "Pruning Method" 1.
 //
-// One persistent kernel per projection.  CTA pairs (2-CTA clusters, one CTA per
-// SM) compute 256 x 256 output tiles with the pair form of the MMA (cta_group::2):
-// each CTA loads half of A's rows and half of B's rows, so a CTA moves 2/3 of the
-// operand bytes a single-CTA 128 x 256 tile needs for the same FLOPs.  Per CTA:
-//   warp 0      TMA producer: its A/B code half-tiles (SWIZZLE_128B tensor maps,
-//               into its own CTA only) and block-scale atoms (1-D bulk copies) into a
-//               5-stage shared-memory ring guarded by mbarriers;
-//   warp 1      (even CTA) MMA issuer: four K=64 block-scaled M=256 x N=256 MMAs
-//               per stage into the pair's FP32 TMEM accumulators, nothing else
-//               (a tcgen05.cp costs the tensor pipe ~60-80 cycles whatever its
-//               size, so twelve scale copies per stage would cost more than the
-//               stage's MMAs);
+// One persistent kernel per projection, one CTA per SM computing 128 x 256
+// output tiles (128 token rows of one expert x 256 weight rows) with the
+// single-CTA form of the MMA (cta_group::1).  Per CTA:
+//   warp 0      TMA producer: the tile's A rows and both 128-row halves of its B
+//               rows (SWIZZLE_128B tensor maps) and their block-scale atoms (1-D
+//               bulk copies) into a 4-stage shared-memory ring guarded by
+//               mbarriers;
+//   warp 1      MMA issuer: four K=64 block-scaled M=128 x N=256 MMAs per stage
+//               into the FP32 TMEM accumulator, nothing else (a tcgen05.cp costs
+//               the tensor pipe ~60-80 cycles whatever its size, so twelve scale
+//               copies per stage would cost more than the stage's MMAs);
 //   warps 18..21 scale warps: tcgen05.st of each stage's scale factors into the
 //               stage's TMEM scale columns, one warp per lane quadrant;
 //   warps 2..17 epilogue: tcgen05.ld of their 32-lane quadrant, then
@@ -26,9 +25,11 @@
 //                        block-scale layout);
 //               down:    x global scale x routing weight, per-pair rows staged
 //                        as FP16 with a power-of-two scale per 64 columns.
-// Rows of an expert are padded to 128 by the permutation and its rows are cut
-// into 256-row pair tiles, so a tile never straddles two experts; padding rows
-// are computed and never stored.
+// Rows of an expert are padded to 128 by the permutation and cut into 128-row
+// tiles, so a tile never straddles two experts; padding rows are computed and
+// never stored.  128-row tiles instead of the 256-row pair tiles of the CTA-pair
+// form cut the padded MMAs of the 8K prefill from 97,536 to ~82,000 rows, for a
+// B operand each CTA loads whole (twice the pair form's B bytes per CTA).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -45,8 +46,11 @@ namespace nvfp4moe {
 
 namespace {
 
-// A CTA pair computes a 256 x 256 tile: each CTA holds 128 rows of A, 128 rows
-// (N) of B, the scale factors of its A rows and of all 256 B rows.  Two operand
+// Two tile forms (CG): a CTA computes a 128 x 256 tile with single-CTA MMAs (CG =
+// 1: M = 128 token rows, N = 256 weight rows; it holds the tile's 128 rows of A,
+// all 256 rows of B and the scale factors of both), or a CTA pair computes a
+// 256 x 256 tile with the pair MMA (CG = 2: each CTA holds 128 rows of A, 128
+// rows of B, the scale factors of its A rows and of all 256 B rows).  Two operand
 // kinds share the kernel:
 //   KIND_NVF4  W4A4: A and B E2M1 with E4M3 scales per 16, kind::mxf4nvf4
 //              (scale_vec::4X, K=64 per MMA); a stage is 256 K elements.
@@ -55,7 +59,7 @@ namespace {
 //              (scale_vec::1X, K=32 per MMA); a stage is 128 K elements.
 // Either way an operand row of a stage is 128 bytes (one SWIZZLE_128B row) and a
 // stage holds four MMAs.
-constexpr int BM = 128, BN = 256;  // BM per CTA, BN per pair
+constexpr int BM = 128, BN = 256;  // rows of A per CTA; rows of B per tile
 enum { KIND_NVF4 = 0, KIND_MXF8 = 1 };
 
 template <int KIND>
@@ -63,7 +67,7 @@ struct Cfg;
 template <>
 struct Cfg<KIND_NVF4> {
     static constexpr int BK = 256;        // K elements per stage
-    static constexpr int STAGES = 5;
+    static constexpr int STAGES_1 = 4, STAGES_2 = 5;  // ring stages of the single-CTA and the pair form
     static constexpr int SF_ELEMS = 16;   // elements per scale
     static constexpr int SFA_ATOMS = 4;   // scale atoms (128 rows x 4 scales) per 128 rows per stage
     static constexpr uint32_t SF_STRIDE = 48;  // TMEM scale columns per ring slot: A 4 x 4, B 4 x 8
@@ -72,28 +76,33 @@ struct Cfg<KIND_NVF4> {
 template <>
 struct Cfg<KIND_MXF8> {
     static constexpr int BK = 128;
-    static constexpr int STAGES = 6;
+    static constexpr int STAGES_1 = 4, STAGES_2 = 6;
     static constexpr int SF_ELEMS = 32;
     static constexpr int SFA_ATOMS = 1;
     static constexpr uint32_t SF_STRIDE = 12;  // A 4, B 8 (one word per row holds the stage's four scales)
     static constexpr uint32_t SFB_COL = 4;
 };
 constexpr int A_BYTES = BM * 128;         // 128 rows x 128 bytes
-constexpr int B_BYTES = (BN / 2) * 128;
+template <int CG>  // B rows of a CTA x 128 bytes: all 256 (two 128-row copies), or its half of the pair's
+__host__ __device__ constexpr int b_bytes() { return (CG == 1 ? BN : BN / 2) * 128; }
+template <int KIND, int CG>
+__host__ __device__ constexpr int stages() { return CG == 1 ? Cfg<KIND>::STAGES_1 : Cfg<KIND>::STAGES_2; }
 template <int KIND>
 __host__ __device__ constexpr int sfa_bytes() { return Cfg<KIND>::SFA_ATOMS * 512; }
 template <int KIND>
 __host__ __device__ constexpr int sfb_bytes() { return 2 * Cfg<KIND>::SFA_ATOMS * 512; }
-template <int KIND>
+template <int KIND, int CG>
 __host__ __device__ constexpr int stage_bytes() {  // padded to the 1024-byte alignment of swizzled tiles
-    return (A_BYTES + B_BYTES + sfa_bytes<KIND>() + sfb_bytes<KIND>() + 1023) / 1024 * 1024;
+    return (A_BYTES + b_bytes<CG>() + sfa_bytes<KIND>() + sfb_bytes<KIND>() + 1023) / 1024 * 1024;
 }
-template <int KIND>
-__host__ __device__ constexpr int smem_bytes() { return Cfg<KIND>::STAGES * stage_bytes<KIND>() + 1024 + 256; }
-static_assert(smem_bytes<KIND_NVF4>() <= 232448 && smem_bytes<KIND_MXF8>() <= 232448,
+template <int KIND, int CG>
+__host__ __device__ constexpr int smem_bytes() { return stages<KIND, CG>() * stage_bytes<KIND, CG>() + 1024 + 256; }
+static_assert(smem_bytes<KIND_NVF4, 1>() <= 232448 && smem_bytes<KIND_MXF8, 1>() <= 232448 &&
+                  smem_bytes<KIND_NVF4, 2>() <= 232448 && smem_bytes<KIND_MXF8, 2>() <= 232448,
               "shared-memory ring above the 227 KB a CTA may use");
-static_assert(256 + Cfg<KIND_NVF4>::STAGES * Cfg<KIND_NVF4>::SF_STRIDE <= 512 &&
-                  256 + Cfg<KIND_MXF8>::STAGES * Cfg<KIND_MXF8>::SF_STRIDE <= 512,
+static_assert(256 + stages<KIND_NVF4, 1>() * Cfg<KIND_NVF4>::SF_STRIDE <= 512 &&
+                  256 + stages<KIND_NVF4, 2>() * Cfg<KIND_NVF4>::SF_STRIDE <= 512 &&
+                  256 + stages<KIND_MXF8, 2>() * Cfg<KIND_MXF8>::SF_STRIDE <= 512,
               "accumulator + per-slot scale columns must fit the TMEM allocation");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_SF = 256;  // scale-factor columns after the 256 accumulator columns
@@ -153,44 +162,52 @@ struct GemmParams {
 // One stage's MMA j (of four): K=64 block-scaled FP4 (four E4M3 scales per row
 // and MMA, own TMEM columns) or K=32 FP8 x FP4 (one E8M0 scale per row and MMA,
 // byte j of the stage's scale word).
-template <int KIND>
+template <int KIND, int CG>
 __device__ __forceinline__ void stage_mma(uint32_t tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t sf_col, int j, uint32_t accumulate) {
-    if (KIND == KIND_NVF4)
+    const uint32_t id8 = idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4);  // W4A8: scale byte j
+    if (KIND == KIND_NVF4 && CG == 1)
+        tc::mma_mxf4nvf4_1(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j, sf_col + 16 + 8 * j,
+                           accumulate);
+    else if (KIND == KIND_NVF4)
         tc::mma_mxf4nvf4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc, sf_col + 4 * j, sf_col + 16 + 8 * j,
                               accumulate);
+    else if (CG == 1)
+        tc::mma_mxf8f6f4_1(tmem, adesc + 2 * j, bdesc + 2 * j, id8, sf_col, sf_col + Cfg<KIND>::SFB_COL, accumulate);
     else
-        tc::mma_mxf8f6f4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, idesc | ((uint32_t)j << 29) | ((uint32_t)j << 4),
-                              sf_col, sf_col + Cfg<KIND>::SFB_COL, accumulate);
+        tc::mma_mxf8f6f4_pair(tmem, adesc + 2 * j, bdesc + 2 * j, id8, sf_col, sf_col + Cfg<KIND>::SFB_COL,
+                              accumulate);
 }
 
-template <int EPI, int KIND>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+template <int EPI, int KIND, int CG>
+__global__ void __cluster_dims__(CG, 1, 1) __launch_bounds__(THREADS, 1)
     k_w4a4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p) {
-    constexpr int STAGES = Cfg<KIND>::STAGES;
-    constexpr int STAGE_BYTES = stage_bytes<KIND>();
+    constexpr int STAGES = stages<KIND, CG>();
+    constexpr int STAGE_BYTES = stage_bytes<KIND, CG>();
+    constexpr int B_BYTES = b_bytes<CG>();
+    constexpr bool PAIR = CG == 2;  // barriers of the even CTA also see the odd CTA's arrivals
     constexpr int SFA_BYTES = sfa_bytes<KIND>();
     constexpr uint32_t TM_SF_STRIDE = Cfg<KIND>::SF_STRIDE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-    uint64_t* sf_ready = full + STAGES;   // even CTA only: both CTAs' scale warps
-    uint64_t* empty = sf_ready + STAGES;  // both CTAs: the even CTA's MMA commits
-    uint64_t* acc_full = empty + STAGES;  // both CTAs: the even CTA's MMA commits
-    uint64_t* acc_empty = acc_full + 1;   // even CTA only: both CTAs' epilogue warps
-    uint64_t* drain = acc_empty + 1;      // even CTA only: the MMAs of an error path
+    uint64_t* sf_ready = full + STAGES;   // the scale warps (pair: both CTAs', on the even CTA's)
+    uint64_t* empty = sf_ready + STAGES;  // the MMA thread's commits
+    uint64_t* acc_full = empty + STAGES;  // the MMA thread's commits
+    uint64_t* acc_empty = acc_full + 1;   // the epilogue warps (pair: both CTAs', on the even CTA's)
+    uint64_t* drain = acc_empty + 1;      // the MMAs of an error path
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
-    const uint32_t rank = tc::cluster_ctarank();  // 0: issues the MMAs of the pair
+    const uint32_t rank = PAIR ? tc::cluster_ctarank() : 0u;  // 0: issues the MMAs
     const int warp = warp_id(), lane = lane_id();
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             tc::mbar_init(&full[s], 1);
-            tc::mbar_init(&sf_ready[s], 2 * SF_WARPS);
+            tc::mbar_init(&sf_ready[s], CG * SF_WARPS);
             tc::mbar_init(&empty[s], 1);
         }
         tc::mbar_init(acc_full, 1);
-        tc::mbar_init(acc_empty, 2 * EPI_WARPS);
+        tc::mbar_init(acc_empty, CG * EPI_WARPS);
         tc::mbar_init(drain, 1);
         tc::fence_mbar_init();
     }
@@ -199,16 +216,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tc::prefetch_tmap(&tmB);
     }
     if (warp == 1) {
-        tc::tmem_alloc_pair(tmem_slot, TMEM_COLS);
-        tc::tmem_relinquish_pair();
+        if (PAIR) {
+            tc::tmem_alloc_pair(tmem_slot, TMEM_COLS);
+            tc::tmem_relinquish_pair();
+        } else {
+            tc::tmem_alloc_1(tmem_slot, TMEM_COLS);
+            tc::tmem_relinquish_1();
+        }
     }
-    // barriers initialised and TMEM allocated in both CTAs before either uses the other's
+    // barriers initialised and TMEM allocated (pair: in both CTAs) before any role uses them
     tc::tc_fence_before();
-    tc::cluster_sync();
+    if (PAIR) tc::cluster_sync();
+    else __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    // tile units: a CTA, or a CTA pair
+    const int cta = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int n_ctas = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
     const int total = p.n_tiles[0] * p.n_ntiles;
     // MMA steps (K=64 FP4 or K=32 FP8) and stages of four; scale atoms per 128 rows
     const int ksub_total = KIND == KIND_NVF4 ? p.K / 64 : p.K / 32;
@@ -217,14 +242,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        // This CTA's half of the pair tile: A rows [128 rank, +128) and B (N) rows
-        // [128 rank, +128); the scale factors of its A rows and of all 256 N rows.
+        // Single CTA: the tile's 128 rows of A, its 256 rows of B (two 128-row
+        // copies) and the scale factors of both.  Pair: this CTA's half of the pair
+        // tile, A rows [128 rank, +128) and B rows [128 rank, +128), the scale
+        // factors of its A rows and of all 256 B rows.
         if (lane == 0) {
             // No L2 prefetch: every TMA instruction costs this thread ~85 cycles of
-            // issue (a prefetch ~270), and with four copies per stage the issue
+            // issue (a prefetch ~270), and with five copies per stage the issue
             // time, not the memory system, would bound the MMA rate.
             int it = 0;
-            for (int tile = pair; tile < total; tile += n_pairs) {
+            for (int tile = cta; tile < total; tile += n_ctas) {
                 const int m = tile / p.n_ntiles, n = tile - m * p.n_ntiles;
                 const int4 ti = p.tiles[m];
                 // rows of this CTA's half that hold pairs; none in the odd half of an
@@ -236,7 +263,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 for (int ks = 0; ks < ks_count; ++ks, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!tc::mbar_wait<true>(&empty[s], ph ^ 1u, p.err)) goto drain_loads;
+                    if (!tc::mbar_wait<PAIR>(&empty[s], ph ^ 1u, p.err)) goto drain_loads;
                     // scale atoms of this stage per 128 rows (a partial last stage: W4A4 only)
                     const int na = KIND == KIND_NVF4 ? min(4, ksub_total - ks * 4) : 1;
                     uint8_t* st = smem + s * STAGE_BYTES;
@@ -250,7 +277,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                             p.sfa + ((int64_t)(a_row / 128) * atoms_per_row + ks * Cfg<KIND>::SFA_ATOMS) * 512;
                         tc::bulk_load(st + A_BYTES + B_BYTES, sfa, na * 512, &full[s]);
                     }
-                    tc::tma_load_2d(st + A_BYTES, &tmB, ks * 128, (int32_t)(b_tile0 + BM * rank), &full[s]);
+                    if (PAIR) {
+                        tc::tma_load_2d(st + A_BYTES, &tmB, ks * 128, (int32_t)(b_tile0 + BM * rank), &full[s]);
+                    } else {
+                        tc::tma_load_2d(st + A_BYTES, &tmB, ks * 128, (int32_t)b_tile0, &full[s]);
+                        tc::tma_load_2d(st + A_BYTES + B_BYTES / 2, &tmB, ks * 128, (int32_t)(b_tile0 + BM),
+                                        &full[s]);
+                    }
                     // the stage's scale atoms of all 256 N rows are stored together: one copy
                     // (placed so that rows 128..255 start na atoms after rows 0..127)
                     const uint8_t* sfb =
@@ -261,7 +294,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             // wait for the MMA's release of every slot still in use, so that no
             // completion signal of the other CTA lands after this CTA has finished
             for (int i = it; i < it + STAGES; ++i)
-                if (!tc::mbar_wait<true>(&empty[i % STAGES], ((uint32_t)(i / STAGES) & 1u) ^ 1u, p.err))
+                if (!tc::mbar_wait<PAIR>(&empty[i % STAGES], ((uint32_t)(i / STAGES) & 1u) ^ 1u, p.err))
                     goto drain_loads;
             goto producer_done;
         drain_loads:
@@ -272,8 +305,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // One thread of the even CTA issues the pair's M=256 x N=256 MMAs; scale
-        // factors are already in both CTAs' TMEM (the scale warps put them there).
+        // One thread (pair: of the even CTA) issues the tile's M=128 (pair: 256) x
+        // N=256 MMAs; the scale factors are already in TMEM (the scale warps put
+        // them there).
         // The tensor pipe accepts few MMAs ahead of the one it executes (an issue
         // returns ~140 cycles after the previous one), so whatever this thread does
         // between stages is pipe idle time.  The wait for the next stage is
@@ -282,15 +316,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // and scale column forward instead of recomputing them: its own
         // instructions are pipe idle time too.
         if (lane == 0 && rank == 0) {
-            const uint32_t idesc = KIND == KIND_NVF4 ? tc::idesc_mxf4nvf4(2 * BM, BN)
-                                                     : tc::idesc_mxf8f6f4_e4m3_e2m1(2 * BM, BN, 0);
-            const int n_tiles_mine = pair < total ? (total - pair + n_pairs - 1) / n_pairs : 0;
+            const uint32_t idesc = KIND == KIND_NVF4 ? tc::idesc_mxf4nvf4(CG * BM, BN)
+                                                     : tc::idesc_mxf8f6f4_e4m3_e2m1(CG * BM, BN, 0);
+            const int n_tiles_mine = cta < total ? (total - cta + n_ctas - 1) / n_ctas : 0;
             const int n_it = n_tiles_mine * ks_count;
             const uint64_t adesc0 = tc::desc_sw128(smem);
             constexpr uint64_t STAGE_DESC = STAGE_BYTES >> 4, B_DESC = A_BYTES >> 4;
             if (n_it > 0) {
-                if (!tc::mbar_wait<true>(acc_empty, 1u, p.err)) goto done;
-                if (!tc::mbar_wait<true>(&sf_ready[0], 0u, p.err)) goto done;
+                if (!tc::mbar_wait<PAIR>(acc_empty, 1u, p.err)) goto done;
+                if (!tc::mbar_wait<PAIR>(&sf_ready[0], 0u, p.err)) goto done;
                 tc::tc_fence_after();
             }
             int ks = 0, tl = 0, s = 0;
@@ -302,12 +336,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const uint64_t bdesc = adesc + B_DESC;
                 const uint32_t acc0 = ks != 0;
                 if (n64 == 4) {
-                    stage_mma<KIND>(tmem, adesc, bdesc, idesc, sf_col, 0, acc0);
-                    stage_mma<KIND>(tmem, adesc, bdesc, idesc, sf_col, 1, 1u);
-                    stage_mma<KIND>(tmem, adesc, bdesc, idesc, sf_col, 2, 1u);
+                    stage_mma<KIND, CG>(tmem, adesc, bdesc, idesc, sf_col, 0, acc0);
+                    stage_mma<KIND, CG>(tmem, adesc, bdesc, idesc, sf_col, 1, 1u);
+                    stage_mma<KIND, CG>(tmem, adesc, bdesc, idesc, sf_col, 2, 1u);
                 } else {
                     for (int j = 0; j < n64 - 1; ++j)
-                        stage_mma<KIND>(tmem, adesc, bdesc, idesc, sf_col, j, (ks | j) != 0);
+                        stage_mma<KIND, CG>(tmem, adesc, bdesc, idesc, sf_col, j, (ks | j) != 0);
                 }
                 const int ns = s + 1 == STAGES ? 0 : s + 1;
                 const uint32_t nph = ns == 0 ? ph ^ 1u : ph;
@@ -315,17 +349,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const bool more = it + 1 < n_it;
                 // next stage of the same tile: its scale factors (and so its operands)
                 bool ok = true;
-                if (more && !tile_end) ok = tc::mbar_wait<true>(&sf_ready[ns], nph, p.err);
-                stage_mma<KIND>(tmem, adesc, bdesc, idesc, sf_col, n64 - 1, (ks | (n64 - 1)) != 0);
-                tc::tc_commit_pair(&empty[s], 0x3);
+                if (more && !tile_end) ok = tc::mbar_wait<PAIR>(&sf_ready[ns], nph, p.err);
+                stage_mma<KIND, CG>(tmem, adesc, bdesc, idesc, sf_col, n64 - 1, (ks | (n64 - 1)) != 0);
+                if (PAIR) tc::tc_commit_pair(&empty[s], 0x3);
+                else tc::tc_commit_1(&empty[s]);
                 if (tile_end) {
-                    tc::tc_commit_pair(acc_full, 0x3);
+                    if (PAIR) tc::tc_commit_pair(acc_full, 0x3);
+                    else tc::tc_commit_1(acc_full);
                     ks = 0;
                     ++tl;
                     if (more) {
                         // the single accumulator: the epilogues must have read it
-                        ok = ok && tc::mbar_wait<true>(acc_empty, ((uint32_t)tl & 1u) ^ 1u, p.err);
-                        ok = ok && tc::mbar_wait<true>(&sf_ready[ns], nph, p.err);
+                        ok = ok && tc::mbar_wait<PAIR>(acc_empty, ((uint32_t)tl & 1u) ^ 1u, p.err);
+                        ok = ok && tc::mbar_wait<PAIR>(&sf_ready[ns], nph, p.err);
                     }
                 } else {
                     ++ks;
@@ -340,26 +376,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             goto mma_done;
         drain_mma:
             // error path: the MMAs already issued complete before TMEM is freed
-            tc::tc_commit_pair(drain, 0x1);
+            if (PAIR) tc::tc_commit_pair(drain, 0x1);
+            else tc::tc_commit_1(drain);
             tc::mbar_drain(drain, 0u);
         mma_done:;
         }
     } else if (warp >= 2 + EPI_WARPS) {
         // ------------------------------------------------------------ scale warps
         // Warp w writes the scale factors of every stage into TMEM lane quadrant
-        // w % 4 of its own CTA with tcgen05.st, in the replicated atom layout the
+        // w % 4 with tcgen05.st, in the replicated atom layout the
         // MMA reads: lane (32q + l), column c of an atom's 4 holds word c of the
         // atom's 16-byte row l.  Each ring slot has its own scale columns, rewritten
         // only after the slot's MMAs completed (the slot is refilled only after
-        // `empty`).  The even CTA's MMA thread waits for all eight scale warps.
+        // `empty`).  The MMA thread waits for all four (pair: eight) scale warps.
         const int q = warp & 3;
         const uint32_t t_q = tmem + ((uint32_t)(q * 32) << 16);
         int it = 0;
-        for (int tile = pair; tile < total; tile += n_pairs) {
+        for (int tile = cta; tile < total; tile += n_ctas) {
             for (int ks = 0; ks < ks_count; ++ks, ++it) {
                 const int s = it % STAGES;
                 const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                if (!tc::mbar_wait(&full[s], ph, p.err)) goto done;
+                if (!tc::mbar_wait(&full[s], ph, p.err)) goto done;  // completed by this CTA's copies
                 const uint8_t* st = smem + s * STAGE_BYTES + A_BYTES + B_BYTES;
                 const uint32_t col = t_q + TM_SF + (uint32_t)s * TM_SF_STRIDE;
                 if (KIND == KIND_NVF4) {
@@ -395,7 +432,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 tc::tmem_st_wait();
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive_remote_relaxed(tc::cluster_addr(&sf_ready[s], 0));
+                if (lane == 0) {
+                    if (PAIR) tc::mbar_arrive_remote_relaxed(tc::cluster_addr(&sf_ready[s], 0));
+                    else tc::mbar_arrive(&sf_ready[s]);
+                }
             }
         }
     } else {
@@ -406,17 +446,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int quarter = (warp - 2) >> 2;
         const int r_in = q * 32 + lane;
         const uint32_t t_row = tmem + ((uint32_t)(q * 32) << 16);
-        const uint32_t acc_empty_leader = tc::cluster_addr(acc_empty, 0);
+        const uint32_t acc_empty_leader = PAIR ? tc::cluster_addr(acc_empty, 0) : 0u;
         int tl = 0;
-        for (int tile = pair; tile < total; tile += n_pairs, ++tl) {
+        for (int tile = cta; tile < total; tile += n_ctas, ++tl) {
             const int m = tile / p.n_ntiles, n = tile - m * p.n_ntiles;
             const int4 ti = p.tiles[m];
-            // this CTA's 128 rows of the pair tile
+            // this CTA's 128 rows of the tile
             const int n_valid = ti.z - BM * (int)rank;
             const int64_t row0 = (int64_t)ti.y + BM * (int)rank;
             const bool valid = r_in < n_valid;
             const int64_t row = row0 + r_in;
-            if (!tc::mbar_wait<true>(acc_full, (uint32_t)tl & 1u, p.err)) goto done;
+            if (!tc::mbar_wait<PAIR>(acc_full, (uint32_t)tl & 1u, p.err)) goto done;
             tc::tc_fence_after();
             if (EPI == EPI_GATEUP) {
                 // columns [0,128) gate, [128,256) up, for intermediates n*128 .. n*128+127;
@@ -431,7 +471,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                                     uv + 16 * c);
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive_remote_relaxed(acc_empty_leader);
+                if (lane == 0) {
+                    if (PAIR) tc::mbar_arrive_remote_relaxed(acc_empty_leader);
+                    else tc::mbar_arrive(acc_empty);
+                }
                 if (valid) {
                     const float ag = p.globals[ti.x * 3 + 0] * p.act_global;
                     const float au = p.globals[ti.x * 3 + 1] * p.act_global;
@@ -477,7 +520,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 for (int c = 0; c < 2; ++c) tc::tmem_ld16x2(t_col + 32 * c, t_col + 32 * c + 16, v + 32 * c, v + 32 * c + 16);
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive_remote_relaxed(acc_empty_leader);
+                if (lane == 0) {
+                    if (PAIR) tc::mbar_arrive_remote_relaxed(acc_empty_leader);
+                    else tc::mbar_arrive(acc_empty);
+                }
                 // rows past the tile's valid count hold padding: weight 0, never stored
                 const float f = valid ? p.globals[ti.x * 3 + 2] * p.act_global * p.wts[p.pair_of_row[row]] : 0.0f;
                 const int c8 = lane & 7, g8 = lane >> 3;
@@ -529,13 +575,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
     }
 done:
-    // neither CTA frees its TMEM or exits while the other may still signal it
-    __syncthreads();
-    tc::tc_fence_before();
-    tc::cluster_sync();
+    // every role is done with TMEM before it is freed; pair: neither CTA frees its
+    // TMEM or exits while the other may still signal it
+    if (PAIR) {
+        __syncthreads();
+        tc::tc_fence_before();
+        tc::cluster_sync();
+    } else {
+        tc::tc_fence_before();
+        __syncthreads();
+    }
     if (warp == 1) {
         tc::tc_fence_after();
-        tc::tmem_dealloc_pair(tmem, TMEM_COLS);
+        if (PAIR) tc::tmem_dealloc_pair(tmem, TMEM_COLS);
+        else tc::tmem_dealloc_1(tmem, TMEM_COLS);
     }
 }
 
@@ -606,10 +659,11 @@ __global__ void k_w8_pack_sf(const uint8_t* __restrict__ src0, const uint8_t* __
 // ---------------------------------------------------------------------------
 // host: tensor maps and launches
 // ---------------------------------------------------------------------------
-// CTA pairs that fit on the device at once (1 CTA per SM), per device and kind, cached.
-template <int KIND>
-int max_resident_pairs() {
-    constexpr int SMEM_BYTES = smem_bytes<KIND>();
+// Tile units that fit on the device at once (1 CTA per SM): CTAs, or CTA pairs
+// (cluster occupancy), per device, kind and form, cached.
+template <int KIND, int CG>
+int max_resident_units() {
+    constexpr int SMEM_BYTES = smem_bytes<KIND, CG>();
     static std::mutex mu;
     static int cache[64] = {};
     int dev = 0;
@@ -619,21 +673,27 @@ int max_resident_pairs() {
     }
     std::lock_guard<std::mutex> lk(mu);
     if (cache[dev] == 0) {
-        if (cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SMEM_BYTES) !=
-            cudaSuccess) {
+        if (cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP, KIND, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM_BYTES) != cudaSuccess) {
             set_error("w4a4: cannot raise the shared-memory limit to %d bytes", SMEM_BYTES);
             return 0;
         }
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * 74, 1, 1);
-        cfg.blockDim = dim3(THREADS, 1, 1);
-        cfg.dynamicSmemBytes = SMEM_BYTES;
         int n = 0;
-        const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, k_w4a4_gemm<EPI_GATEUP, KIND>, &cfg);
+        cudaError_t e;
+        if (CG == 2) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2 * 74, 1, 1);
+            cfg.blockDim = dim3(THREADS, 1, 1);
+            cfg.dynamicSmemBytes = SMEM_BYTES;
+            e = cudaOccupancyMaxActiveClusters(&n, k_w4a4_gemm<EPI_GATEUP, KIND, CG>, &cfg);
+        } else {
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_w4a4_gemm<EPI_GATEUP, KIND, CG>, THREADS,
+                                                              SMEM_BYTES);
+            n *= num_sms();
+        }
         if (e != cudaSuccess || n <= 0) {
             (void)cudaGetLastError();
-            n = num_sms() / 2;  // one CTA per SM, two SMs per pair
+            n = num_sms() / CG;  // one CTA per SM
         }
         cache[dev] = n;
     }
@@ -698,19 +758,19 @@ nvfp4moe_status launch_w4a4_pack(const nvfp4moe_expert_weights& w, void* packed,
     return NVFP4MOE_OK;
 }
 
-template <int KIND>
+template <int KIND, int CG>
 static nvfp4moe_status run_layer(const void* packed, int H, int I, int E, float act_global_in, float act_global_mid,
                                  int64_t rows_max, int max_tiles, const RoutingPlan& plan, const uint8_t* A1c,
                                  const uint8_t* A1s, uint8_t* A2c, uint8_t* A2s, __half* Y, float* y_scale,
                                  cudaStream_t stream, cudaEvent_t mid_event) {
     constexpr bool MX8 = KIND == KIND_MXF8;
-    constexpr int SMEM_BYTES = smem_bytes<KIND>();
+    constexpr int SMEM_BYTES = smem_bytes<KIND, CG>();
     const W4Layout L = w4_layout(E, H, I, MX8);
     const uint8_t* pk = static_cast<const uint8_t*>(packed);
-    NVFP4MOE_CUDA(
-        cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    NVFP4MOE_CUDA(
-        cudaFuncSetAttribute(k_w4a4_gemm<EPI_DOWN, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w4a4_gemm<EPI_GATEUP, KIND, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SMEM_BYTES));
+    NVFP4MOE_CUDA(cudaFuncSetAttribute(k_w4a4_gemm<EPI_DOWN, KIND, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SMEM_BYTES));
     // A rows in bytes: FP4 two codes per byte, FP8 one per byte.  B: W4A4 copies the
     // packed codes as bytes; W4A8 copies them through a map that unpacks them into
     // the padded form (coordinates in codes: a stage's 128 codes are 128 bytes of
@@ -723,8 +783,8 @@ static nvfp4moe_status run_layer(const void* packed, int H, int I, int E, float 
                          : make_map(&mGU, pk + L.gu_codes, H / 2, (int64_t)E * 2 * I, BN / 2) &&
                                make_map(&mD, pk + L.d_codes, I / 2, (int64_t)E * H, BN / 2));
     if (!ok) return NVFP4MOE_ERR_CUDA;
-    const int pairs = max_resident_pairs<KIND>();
-    if (pairs <= 0) return NVFP4MOE_ERR_CUDA;
+    const int units = max_resident_units<KIND, CG>();
+    if (units <= 0) return NVFP4MOE_ERR_CUDA;
     GemmParams g{};
     g.tiles = plan.tiles;
     g.n_tiles = plan.n_tiles;
@@ -745,8 +805,8 @@ static nvfp4moe_status run_layer(const void* packed, int H, int I, int E, float 
     g.out_sf = A2s;
     g.out_k = I;
     {
-        const int grid = 2 * (int)std::min<int64_t>(pairs, (int64_t)max_tiles * g.n_ntiles);
-        k_w4a4_gemm<EPI_GATEUP, KIND><<<grid, THREADS, SMEM_BYTES, stream>>>(mA1, mGU, g);
+        const int grid = CG * (int)std::min<int64_t>(units, (int64_t)max_tiles * g.n_ntiles);
+        k_w4a4_gemm<EPI_GATEUP, KIND, CG><<<grid, THREADS, SMEM_BYTES, stream>>>(mA1, mGU, g);
         NVFP4MOE_CHECK_LAUNCH(MX8 ? "w4a8 gate/up kernel" : "w4a4 gate/up kernel");
     }
     if (mid_event) cudaEventRecord(mid_event, stream);
@@ -762,8 +822,8 @@ static nvfp4moe_status run_layer(const void* packed, int H, int I, int E, float 
     g.y_scale = y_scale;
     g.ldy = H;
     {
-        const int grid = 2 * (int)std::min<int64_t>(pairs, (int64_t)max_tiles * g.n_ntiles);
-        k_w4a4_gemm<EPI_DOWN, KIND><<<grid, THREADS, SMEM_BYTES, stream>>>(mA2, mD, g);
+        const int grid = CG * (int)std::min<int64_t>(units, (int64_t)max_tiles * g.n_ntiles);
+        k_w4a4_gemm<EPI_DOWN, KIND, CG><<<grid, THREADS, SMEM_BYTES, stream>>>(mA2, mD, g);
         NVFP4MOE_CHECK_LAUNCH(MX8 ? "w4a8 down kernel" : "w4a4 down kernel");
     }
     return NVFP4MOE_OK;
@@ -775,10 +835,22 @@ nvfp4moe_status launch_w4a4_layer(const void* packed, bool mx8, int T, int H, in
                                   uint8_t* A2s, __half* Y, float* y_scale, cudaStream_t stream, cudaEvent_t mid_event) {
     (void)T;
     (void)k;
-    return mx8 ? run_layer<KIND_MXF8>(packed, H, I, E, act_global_in, act_global_mid, rows_max, max_tiles, plan, A1c,
-                                      A1s, A2c, A2s, Y, y_scale, stream, mid_event)
-               : run_layer<KIND_NVF4>(packed, H, I, E, act_global_in, act_global_mid, rows_max, max_tiles, plan, A1c,
-                                      A1s, A2c, A2s, Y, y_scale, stream, mid_event);
+    // the tile form the plan's tile list was cut for
+#define W4_RUN(KD, CGV)                                                                                         \
+    run_layer<KD, CGV>(packed, H, I, E, act_global_in, act_global_mid, rows_max, max_tiles, plan, A1c, A1s, A2c, \
+                       A2s, Y, y_scale, stream, mid_event)
+    const bool pair = plan.tile_rows == 2 * MTILE;
+    if (mx8) return pair ? W4_RUN(KIND_MXF8, 2) : W4_RUN(KIND_MXF8, 1);
+    return pair ? W4_RUN(KIND_NVF4, 2) : W4_RUN(KIND_NVF4, 1);
+#undef W4_RUN
+}
+
+int w4a4_tile_rows(int64_t T, int k, int E) {
+    // CTA pairs (256-row tiles) when experts average 1024 rows or more (their
+    // tiles are mostly full, and the pair form loads half the B bytes per CTA
+    // and has a deeper ring); single CTAs (128-row tiles) below that, where
+    // halving the tile halves each expert's padding
+    return T * k >= 1024LL * E ? 2 * MTILE : MTILE;
 }
 
 }  // namespace nvfp4moe
