@@ -98,14 +98,14 @@ MODE_DTYPES = {0: "bf16 activations x fp4 e2m1 weights (e4m3 block scales), fp16
 
 # DRAM bytes (read + write) per launch from ncu captures of smaller cases of
 # the same kernels (profiles/), valid for these kernel versions and workloads only:
-#  - k_w4a4_gemm gate/up, W4A4 (k_w4a4_gemm_prefill2k_e64.txt: 652.8 MB read +
-#    21.4 MB written at T=2048, E=64), scaled x4 to T=8192, E=256 (weights and
-#    activations both grow 4x);
-#  - the same for W4A8 (k_w4a8_gemm_prefill2k_e64.txt: 656.7 MB + 35.0 MB);
+#  - k_w4a4_gemm gate/up, W4A4, single-CTA form (k_w4a4_gemm_traffic_prefill2k_e64.txt:
+#    653.8 MB read + 19.9 MB written at T=2048, E=64), scaled x4 to T=8192, E=256
+#    (weights and activations both grow 4x);
+#  - the same for W4A8 (same file: 656.7 MB + 33.4 MB);
 #  - k_w16_gateup + k_w16_down of one 16-token decode step at E=256 (the bench's
 #    own workload, captured at full size: k_w16_decode16.txt).
-GATEUP_TRAFFIC_T8192_E256 = 4 * (652.7936e6 + 21.404928e6)
-GATEUP_W4A8_TRAFFIC_T8192_E256 = 4 * (656.699392e6 + 35.003648e6)
+GATEUP_TRAFFIC_T8192_E256 = 4 * (653826816 + 19891200)
+GATEUP_W4A8_TRAFFIC_T8192_E256 = 4 * (656710656 + 33436160)
 DECODE_TRAFFIC_T16_E256 = 1010.475e6 + 4.71296e6 + 505.455e6 + 5.101568e6
 #  - k_transcode out of place (k_transcode_layer96.txt: 427.9 MB read + 404.6 MB
 #    written for a 96-tensor layer), scaled x8 to the 768-tensor layer timed here.

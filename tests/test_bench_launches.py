@@ -23,7 +23,7 @@ def _launches(name):
 
 
 @pytest.mark.parametrize("profile,workload,gemm", [
-    ("launches_prefill8k_w4a4.txt", "prefill", "k_w4a4_gemm<0, 0>"),
+    ("launches_prefill8k_w4a4.txt", "prefill", "k_w4a4_gemm<0, 0, 1>"),
     ("launches_decode16_w4a16.txt", "decode", "k_w16_gateup<0, 4>"),
 ])
 def test_launches_per_step_match_the_recorded_launch_list(profile, workload, gemm):
