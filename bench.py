@@ -684,7 +684,9 @@ def bench_router(torch, moe, args, P):
     gbs = nbytes / (us / 1e6) / 1e9
     del w
     torch.cuda.empty_cache()
-    return {"workload": f"router: T={T} H={H} E={E} groups={wl.n_group} keep={wl.topk_group} top_k={wl.top_k}, "
+    prefill = bench_router_prefill(torch, moe, args)
+    return {"prefill": prefill,
+            "workload": f"router: T={T} H={H} E={E} groups={wl.n_group} keep={wl.topk_group} top_k={wl.top_k}, "
                         f"FP32 router, {layers} layers' routers rotated (> L2)",
             "value": round(us, 2), "unit": "us per layer (CUDA graph of 47 layers' calls)",
             "higher_is_better": False, "eager_us_per_call": round(eager_us, 2),
@@ -693,6 +695,61 @@ def bench_router(torch, moe, args, P):
                          "unit": "GB/s", "frac": round(gbs / P["hbm_gbs"], 4), "traffic": None,
                          "frac_of_spec": round(gbs / SPEC_HBM_GBS, 4),
                          "algorithmic_bytes_per_launch": int(nbytes)}}
+
+
+# FP32 FMA peak of the CUDA cores, derived from unit counts and the clock: SMs x
+# 128 FP32 lanes x 2 FLOP x 1.965 GHz (the maximum SM clock), 74.4 TFLOP/s on 148 SMs
+FP32_LANES_PER_SM = 128
+MAX_SM_GHZ = 1.965
+
+
+def bench_router_prefill(torch, moe, args):
+    """Router projection + grouped top-k at the prefill shape, T=8192 (the
+    tiled FP32 projection).  Calls alternate between two hidden batches (134 MB
+    together, > L2) and four layers' routers."""
+    wl = inputs.WORKLOADS["prefill"]
+    T, H, E = wl.T, wl.H, wl.E
+    rng = np.random.default_rng(wl.seed + 101)
+    xs = [torch.from_numpy(inputs.bf16_bits(rng.standard_normal((T, H), dtype=np.float32)).view(np.int16)).cuda()
+          for _ in range(2)]
+    w = torch.empty((4, E, H), dtype=torch.float32, device="cuda")
+    for l in range(4):
+        w[l].copy_(torch.from_numpy(inputs.router_weights(rng, E, H)))
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    ids = torch.empty((T, wl.top_k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((T, wl.top_k), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(16, moe.moe_router_topk_workspace_size(T)), dtype=torch.uint8, device="cuda")
+
+    def call(i):
+        moe.moe_router_topk(xs[i % 2], w[i % 4], None, wl.n_group, wl.topk_group, wl.top_k, wl.rsf, True, logits,
+                            ids, wts, ws)
+
+    for i in range(max(args.warmup, 3)):
+        call(i)
+    torch.cuda.synchronize()
+    reps = max(args.steps, 20)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(reps):
+        call(i)
+    b.record()
+    torch.cuda.synchronize()
+    moe.nvfp4moe_check_device_status()
+    us = a.elapsed_time(b) / reps * 1e3
+    flops = 2.0 * T * H * E
+    tf = flops / (us / 1e6) / 1e12
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    peak = sms * FP32_LANES_PER_SM * 2 * MAX_SM_GHZ / 1e3
+    del xs, w
+    torch.cuda.empty_cache()
+    return {"workload": f"router: T={T} H={H} E={E} groups={wl.n_group} keep={wl.topk_group} top_k={wl.top_k}, "
+                        "FP32 router, two hidden batches x four routers rotated (> L2)",
+            "value": round(us, 2), "unit": "us per call (projection + routing)", "higher_is_better": False,
+            "roofline": {"bound": "alu", "kernel": "k_router_logits_tiled + k_route_rows", "achieved": round(tf, 2),
+                         "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(tf / peak, 4), "traffic": None,
+                         "peak_src": f"derived: {sms} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 FLOP x "
+                                     f"{MAX_SM_GHZ} GHz",
+                         "algorithmic_flops_per_call": int(flops)}}
 
 
 def bench_transcode(torch, moe, args, P):

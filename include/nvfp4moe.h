@@ -167,15 +167,22 @@ nvfp4moe_status moe_route(const float* logits, const float* bias, int32_t T, int
  * arithmetic (BF16 hidden rows, FP32 router rows; each logit summed in a fixed
  * order, so repeated calls give the same bits), written to logits_out, then
  * routed exactly as moe_route routes logits_out (same ids and weight bits).
- * Two kernel launches: the projection, then moe_route's routing kernel.
+ * Two kernel launches: the projection, then moe_route's routing kernel.  The
+ * projection has two forms.  Small T: each logit is the in-order sum of KS
+ * slice sums (KS = 8, 4 or 2 as H % 1024, % 512, % 256 allows), each a warp
+ * butterfly over 32 lane chains of H / (32 KS) FMAs; error at most
+ * (H/64 + 6) * 2^-24 * sum_h |x_h w_h|.  When ceil(T/128) * ceil(E/64) reaches
+ * the device's SM count: a tiled FP32 GEMM in which each logit is one FMA chain
+ * over h = 0 .. H-1; error at most gamma_H = H 2^-24 / (1 - H 2^-24) times the
+ * same sum.  The two forms may differ in the last bits of a logit, so the
+ * routing of one token can depend on how many tokens share the call.
  *   x_bf16 [T, H] bf16 bits; w_router [E, H] f32; bias [E] f32 or NULL;
  *   logits_out [T, E] f32; topk_ids [T, top_k] i32; topk_weights [T, top_k]
  *   f32 (caller-owned device memory); workspace: device, at least
  *   moe_router_topk_workspace_size(T) bytes, caller-owned; this version
  *   neither reads nor writes it (the size is kept so callers need not change).
- * Constraints: as moe_route, plus H >= 256 with H % 256 == 0 and E % 4 == 0;
- * all pointers 16-byte aligned.  Meant for decode-sized T (the router is read
- * once per 16 tokens).                                                        */
+ * Constraints: as moe_route, plus T <= 8,388,480 (65535 x 128), H >= 256
+ * with H % 256 == 0 and E % 4 == 0; all pointers 16-byte aligned.           */
 size_t moe_router_topk_workspace_size(int32_t T);
 nvfp4moe_status moe_router_topk(const uint16_t* x_bf16, const float* w_router, const float* bias, int32_t T,
                                 int32_t H, int32_t E, int32_t n_group, int32_t topk_group, int32_t top_k,

@@ -313,7 +313,8 @@ nvfp4moe_status moe_router_topk(const uint16_t* x_bf16, const float* w_router, c
                                 float routed_scaling_factor, int32_t renormalize, float* logits_out,
                                 int32_t* topk_ids, float* topk_weights, void* workspace, size_t workspace_bytes,
                                 void* stream) {
-    REQUIRE(T >= 0, NVFP4MOE_ERR_INVALID_ARG, "T=%d is negative", T);
+    REQUIRE(T >= 0 && T <= ROUTER_MAX_T, NVFP4MOE_ERR_INVALID_ARG, "T=%d is outside [0, %lld]", T,
+            (long long)ROUTER_MAX_T);
     RETURN_IF(validate_routing(E, n_group, topk_group, top_k));
     REQUIRE(E % 4 == 0, NVFP4MOE_ERR_UNSUPPORTED_SHAPE, "E=%d is not a multiple of 4", E);
     REQUIRE(H >= 256 && H % 256 == 0, NVFP4MOE_ERR_UNSUPPORTED_SHAPE, "H=%d must be a positive multiple of 256", H);

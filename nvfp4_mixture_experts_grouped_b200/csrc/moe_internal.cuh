@@ -46,6 +46,10 @@ nvfp4moe_status launch_route(const float* logits, const float* bias, int T, int 
 
 // router.cu
 size_t router_ws_size(int T);
+constexpr int64_t ROUTER_MAX_T = 65535LL * 128;  // the tiled projection's grid (128 tokens per CTA row)
+// the projection is the tiled FP32 GEMM (one FMA chain over H per logit) when
+// the token count fills at least one wave of its 128 x 64 tiles
+bool router_uses_tiled(int64_t T, int E);
 nvfp4moe_status launch_router_topk(const uint16_t* x, const float* w, const float* bias, int T, int H, int E,
                                    int n_group, int topk_group, int top_k, float rsf, int renorm, float* logits,
                                    int32_t* ids, float* wts, void* workspace, cudaStream_t stream);

@@ -17,9 +17,12 @@
 // bandwidth one (the router is 4 MB): each lane's router slice is loaded into
 // registers and the tile's 16 hidden rows are copied into shared memory by the
 // whole CTA, all loads issued before any arithmetic, so the kernel waits for one
-// memory round trip instead of one per 128 columns.  Then the routing, one warp
-// per token (route.cu).  CUDA-core FP32: large token counts re-read the router
-// per 16-token tile.  Built with -fmad=false; the dot products use explicit FMAs.
+// memory round trip instead of one per 128 columns.  When the token count fills
+// at least one wave of 128-token x 64-expert tiles (prefill sizes), the
+// projection is instead a register-tiled FP32 GEMM (k_router_logits_tiled), in
+// which each hidden row is read once per 64 experts and each router row once per
+// 128 tokens.  Then the routing, one warp per token (route.cu).  CUDA-core FP32
+// throughout.  Built with -fmad=false; the dot products use explicit FMAs.
 #include "moe_internal.cuh"
 #include "route_token.cuh"
 
@@ -134,7 +137,110 @@ __global__ void __launch_bounds__(RTR_WARPS * 32)
     }
 }
 
+// Prefill-size projection, a register-tiled FP32 GEMM.  CTA (bx, by) computes
+// the logits of experts 64bx .. 64bx+63 for tokens 128by .. 128by+127.  Thread
+// (ty, tx) = (tid / 8, tid % 8) holds 8 tokens {4ty .. 4ty+3, 64+4ty .. 64+4ty+3}
+// x 8 experts {4tx .. 4tx+3, 32+4tx .. 32+4tx+3} as 64 accumulators, so its four
+// shared-memory reads per h (one float4 each) are conflict-free across the warp.
+// H runs in chunks of 16 columns: every thread loads one hidden row's 16 BF16
+// (two 16-byte loads) and half of one router row's 16 FP32 (two 16-byte loads)
+// of the next chunk while it multiplies the current one, then stores them
+// transposed (h-major, hidden values widened to FP32) into the other of two
+// shared-memory buffers; one barrier per chunk.  Each logit is one FMA chain over
+// h = 0 .. H-1 in order: deterministic, and within gamma_H * sum_h |x_h w_h| of
+// the exact dot product.  Rows past T and experts past E load zeros and are not
+// stored.  E % 4 == 0, H % 16 == 0.
+constexpr int RTT_BM = 128;  // tokens per CTA
+constexpr int RTT_BN = 64;   // experts per CTA
+constexpr int RTT_BK = 16;   // columns of H per chunk
+constexpr int RTT_THREADS = (RTT_BM / 8) * (RTT_BN / 8);
+
+__global__ void __launch_bounds__(RTT_THREADS)
+    k_router_logits_tiled(const uint16_t* __restrict__ x, const float* __restrict__ w, int T, int H, int E,
+                          float* __restrict__ logits) {
+    __shared__ __align__(16) float s_x[2][RTT_BK][RTT_BM];
+    __shared__ __align__(16) float s_w[2][RTT_BK][RTT_BN];
+    const int tid = threadIdx.x;
+    const int e0 = blockIdx.x * RTT_BN;
+    const int64_t t0 = (int64_t)blockIdx.y * RTT_BM;
+    // loader roles: hidden row t0 + tid, all 16 columns of a chunk; router row
+    // e0 + tid % 64, columns 8 (tid / 64) .. + 7 of a chunk
+    const bool x_ok = t0 + tid < T;
+    const uint16_t* xrow = x + (x_ok ? t0 + tid : 0) * (int64_t)H;
+    const int we = tid % RTT_BN, wh = (tid / RTT_BN) * 8;
+    const bool w_ok = e0 + we < E;
+    const float* wrow = w + (int64_t)(w_ok ? e0 + we : 0) * H + wh;
+    uint4 xv[2];
+    float4 wv[2];
+    auto load = [&](int h0) {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        xv[0] = x_ok ? __ldg(reinterpret_cast<const uint4*>(xrow + h0)) : z;
+        xv[1] = x_ok ? __ldg(reinterpret_cast<const uint4*>(xrow + h0 + 8)) : z;
+        const float4 zf = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        wv[0] = w_ok ? __ldg(reinterpret_cast<const float4*>(wrow + h0)) : zf;
+        wv[1] = w_ok ? __ldg(reinterpret_cast<const float4*>(wrow + h0 + 4)) : zf;
+    };
+    auto store = [&](int buf) {
+        const uint32_t u[8] = {xv[0].x, xv[0].y, xv[0].z, xv[0].w, xv[1].x, xv[1].y, xv[1].z, xv[1].w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            s_x[buf][2 * i][tid] = bf16lo(u[i]);      // column 2i of the chunk
+            s_x[buf][2 * i + 1][tid] = bf16hi(u[i]);  // column 2i + 1
+        }
+        const float f[8] = {wv[0].x, wv[0].y, wv[0].z, wv[0].w, wv[1].x, wv[1].y, wv[1].z, wv[1].w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s_w[buf][wh + i][we] = f[i];
+    };
+    const int ty = tid / 8, tx = tid % 8;
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+    load(0);
+    store(0);
+    __syncthreads();
+    const int nk = H / RTT_BK;
+    for (int kc = 0; kc < nk; ++kc) {
+        const int buf = kc & 1;
+        const bool more = kc + 1 < nk;
+        if (more) load((kc + 1) * RTT_BK);  // in flight during this chunk's FMAs
+#pragma unroll
+        for (int kk = 0; kk < RTT_BK; ++kk) {
+            const float4 a0 = *reinterpret_cast<const float4*>(&s_x[buf][kk][4 * ty]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&s_x[buf][kk][64 + 4 * ty]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&s_w[buf][kk][4 * tx]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&s_w[buf][kk][32 + 4 * tx]);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = __fmaf_rn(a[i], b[j], acc[i][j]);
+        }
+        // the other buffer was last read in the previous chunk, before the barrier
+        if (more) store(buf ^ 1);
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t t = t0 + (i < 4 ? 4 * ty + i : 64 + 4 * ty + (i - 4));
+        if (t >= T) continue;
+#pragma unroll
+        for (int jh = 0; jh < 2; ++jh) {
+            const int e = e0 + 32 * jh + 4 * tx;  // e % 4 == 0 and E % 4 == 0: all four or none
+            if (e < E)
+                *reinterpret_cast<float4*>(logits + t * E + e) =
+                    make_float4(acc[i][4 * jh], acc[i][4 * jh + 1], acc[i][4 * jh + 2], acc[i][4 * jh + 3]);
+        }
+    }
+}
+
 }  // namespace
+
+bool router_uses_tiled(int64_t T, int E) {
+    return ceil_div(T, (int64_t)RTT_BM) * ceil_div((int64_t)E, (int64_t)RTT_BN) >= num_sms();
+}
 
 size_t router_ws_size(int T) { return (size_t)ceil_div((int64_t)T, RTR_TT) * sizeof(uint32_t); }
 
@@ -143,6 +249,13 @@ nvfp4moe_status launch_router_topk(const uint16_t* x, const float* w, const floa
                                    int32_t* ids, float* wts, void* workspace, cudaStream_t stream) {
     (void)workspace;  // no scratch: the routing is a second launch on logits
     if (T == 0) return NVFP4MOE_OK;
+    if (router_uses_tiled(T, E)) {
+        // at least one wave of 128 x 64 tiles
+        const dim3 tgrid((unsigned)ceil_div((int64_t)E, (int64_t)RTT_BN), (unsigned)ceil_div((int64_t)T, (int64_t)RTT_BM));
+        k_router_logits_tiled<<<tgrid, RTT_THREADS, 0, stream>>>(x, w, T, H, E, logits);
+        NVFP4MOE_CHECK_LAUNCH("router projection kernel");
+        return launch_route(logits, bias, T, E, n_group, topk_group, top_k, rsf, renorm, ids, wts, stream);
+    }
     const int ks = H % 1024 == 0 ? 8 : H % 512 == 0 ? 4 : 2;  // K slices per expert
     const dim3 grid((unsigned)(E / rtr_epb(ks)), (unsigned)ceil_div((int64_t)T, RTR_TT));
     // the tile's hidden rows in shared memory when they fit and a lane's router
