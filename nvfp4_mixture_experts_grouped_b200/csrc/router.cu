@@ -142,54 +142,72 @@ __global__ void __launch_bounds__(RTR_WARPS * 32)
 // (ty, tx) = (tid / 8, tid % 8) holds 8 tokens {4ty .. 4ty+3, 64+4ty .. 64+4ty+3}
 // x 8 experts {4tx .. 4tx+3, 32+4tx .. 32+4tx+3} as 64 accumulators, so its four
 // shared-memory reads per h (one float4 each) are conflict-free across the warp.
-// H runs in chunks of 16 columns: every thread loads one hidden row's 16 BF16
-// (two 16-byte loads) and half of one router row's 16 FP32 (two 16-byte loads)
-// of the next chunk while it multiplies the current one, then stores them
-// transposed (h-major, hidden values widened to FP32) into the other of two
-// shared-memory buffers; one barrier per chunk.  Each logit is one FMA chain over
-// h = 0 .. H-1 in order: deterministic, and within gamma_H * sum_h |x_h w_h| of
-// the exact dot product.  Rows past T and experts past E load zeros and are not
-// stored.  E % 4 == 0, H % 16 == 0.
-constexpr int RTT_BM = 128;  // tokens per CTA
-constexpr int RTT_BN = 64;   // experts per CTA
-constexpr int RTT_BK = 16;   // columns of H per chunk
+// H runs in chunks of 16 columns.  Every thread copies one hidden row's 16 BF16
+// and half of one router row's 16 FP32 of a chunk (four 16-byte cp.async, zero
+// fill past T or E) into its own slot of a three-deep staging ring, two chunks
+// ahead of the arithmetic; after a chunk's FMAs it waits for its own copies of
+// the next chunk and stores them transposed (h-major, hidden values widened to
+// FP32) into the other of two shared-memory buffers; one barrier per chunk.
+// Each logit is one FMA chain over h = 0 .. H-1 in order: deterministic, and
+// within gamma_H * sum_h |x_h w_h| of the exact dot product.  Rows past T and
+// experts past E are not stored.  E % 4 == 0, H % 16 == 0.
+constexpr int RTT_BM = 128;    // tokens per CTA
+constexpr int RTT_BN = 64;     // experts per CTA
+constexpr int RTT_BK = 16;     // columns of H per chunk
+constexpr int RTT_STAGES = 3;  // staging ring depth (copies run two chunks ahead)
 constexpr int RTT_THREADS = (RTT_BM / 8) * (RTT_BN / 8);
+
+__device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, bool valid) {
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    const uint32_t n = valid ? 16u : 0u;  // 0: nothing is read, the 16 bytes are zero-filled
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
 __global__ void __launch_bounds__(RTT_THREADS)
     k_router_logits_tiled(const uint16_t* __restrict__ x, const float* __restrict__ w, int T, int H, int E,
                           float* __restrict__ logits) {
     __shared__ __align__(16) float s_x[2][RTT_BK][RTT_BM];
     __shared__ __align__(16) float s_w[2][RTT_BK][RTT_BN];
+    __shared__ __align__(16) uint4 s_stage[RTT_STAGES][RTT_THREADS][4];  // per thread: 32 B hidden, 32 B router
     const int tid = threadIdx.x;
     const int e0 = blockIdx.x * RTT_BN;
     const int64_t t0 = (int64_t)blockIdx.y * RTT_BM;
-    // loader roles: hidden row t0 + tid, all 16 columns of a chunk; router row
+    // copy roles: hidden row t0 + tid, all 16 columns of a chunk; router row
     // e0 + tid % 64, columns 8 (tid / 64) .. + 7 of a chunk
     const bool x_ok = t0 + tid < T;
     const uint16_t* xrow = x + (x_ok ? t0 + tid : 0) * (int64_t)H;
     const int we = tid % RTT_BN, wh = (tid / RTT_BN) * 8;
     const bool w_ok = e0 + we < E;
     const float* wrow = w + (int64_t)(w_ok ? e0 + we : 0) * H + wh;
-    uint4 xv[2];
-    float4 wv[2];
-    auto load = [&](int h0) {
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        xv[0] = x_ok ? __ldg(reinterpret_cast<const uint4*>(xrow + h0)) : z;
-        xv[1] = x_ok ? __ldg(reinterpret_cast<const uint4*>(xrow + h0 + 8)) : z;
-        const float4 zf = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        wv[0] = w_ok ? __ldg(reinterpret_cast<const float4*>(wrow + h0)) : zf;
-        wv[1] = w_ok ? __ldg(reinterpret_cast<const float4*>(wrow + h0 + 4)) : zf;
+    const int nk = H / RTT_BK;
+    // chunk kc's copies into ring slot kc % 3, one commit group per chunk (an
+    // empty group past the last chunk keeps the group count uniform)
+    auto issue = [&](int kc) {
+        if (kc < nk) {
+            uint4* st = s_stage[kc % RTT_STAGES][tid];
+            const int h0 = kc * RTT_BK;
+            cp_async16_zfill(st + 0, xrow + h0, x_ok);
+            cp_async16_zfill(st + 1, xrow + h0 + 8, x_ok);
+            cp_async16_zfill(st + 2, wrow + h0, w_ok);
+            cp_async16_zfill(st + 3, wrow + h0 + 4, w_ok);
+        }
+        cp_async_commit();
     };
-    auto store = [&](int buf) {
-        const uint32_t u[8] = {xv[0].x, xv[0].y, xv[0].z, xv[0].w, xv[1].x, xv[1].y, xv[1].z, xv[1].w};
+    // this thread's staged chunk kc, transposed into buffer buf
+    auto transpose = [&](int kc, int buf) {
+        const uint4* st = s_stage[kc % RTT_STAGES][tid];
+        const uint4 x0 = st[0], x1 = st[1], w0 = st[2], w1 = st[3];
+        const uint32_t u[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             s_x[buf][2 * i][tid] = bf16lo(u[i]);      // column 2i of the chunk
             s_x[buf][2 * i + 1][tid] = bf16hi(u[i]);  // column 2i + 1
         }
-        const float f[8] = {wv[0].x, wv[0].y, wv[0].z, wv[0].w, wv[1].x, wv[1].y, wv[1].z, wv[1].w};
+        const uint32_t f[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) s_w[buf][wh + i][we] = f[i];
+        for (int i = 0; i < 8; ++i) s_w[buf][wh + i][we] = __uint_as_float(f[i]);
     };
     const int ty = tid / 8, tx = tid % 8;
     float acc[8][8];
@@ -197,14 +215,16 @@ __global__ void __launch_bounds__(RTT_THREADS)
     for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-    load(0);
-    store(0);
+    issue(0);
+    issue(1);
+    cp_async_wait_1();  // chunk 0 has landed (chunk 1 may be in flight)
+    transpose(0, 0);
     __syncthreads();
-    const int nk = H / RTT_BK;
     for (int kc = 0; kc < nk; ++kc) {
         const int buf = kc & 1;
-        const bool more = kc + 1 < nk;
-        if (more) load((kc + 1) * RTT_BK);  // in flight during this chunk's FMAs
+        // ring slot (kc + 2) % 3 was last read by this thread's transpose of
+        // chunk kc - 1, before the previous barrier
+        issue(kc + 2);
 #pragma unroll
         for (int kk = 0; kk < RTT_BK; ++kk) {
             const float4 a0 = *reinterpret_cast<const float4*>(&s_x[buf][kk][4 * ty]);
@@ -219,7 +239,10 @@ __global__ void __launch_bounds__(RTT_THREADS)
                 for (int j = 0; j < 8; ++j) acc[i][j] = __fmaf_rn(a[i], b[j], acc[i][j]);
         }
         // the other buffer was last read in the previous chunk, before the barrier
-        if (more) store(buf ^ 1);
+        if (kc + 1 < nk) {
+            cp_async_wait_1();  // chunk kc + 1 has landed (chunk kc + 2 may be in flight)
+            transpose(kc + 1, buf ^ 1);
+        }
         __syncthreads();
     }
 #pragma unroll
