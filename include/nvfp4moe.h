@@ -172,9 +172,10 @@ nvfp4moe_status moe_route(const float* logits, const float* bias, int32_t T, int
  * slice sums (KS = 8, 4 or 2 as H % 1024, % 512, % 256 allows), each a warp
  * butterfly over 32 lane chains of H / (32 KS) FMAs; error at most
  * (H/64 + 6) * 2^-24 * sum_h |x_h w_h|.  When ceil(T/128) * ceil(E/64) reaches
- * the device's SM count: a tiled FP32 GEMM in which each logit is one FMA chain
- * over h = 0 .. H-1; error at most gamma_H = H 2^-24 / (1 - H 2^-24) times the
- * same sum.  The two forms may differ in the last bits of a logit, so the
+ * the device's SM count: a tiled FP32 GEMM in which each logit is the FMA
+ * chain over the even 16-column chunks of H plus the chain over the odd ones;
+ * error at most gamma_(H/2+1) = n 2^-24 / (1 - n 2^-24), n = H/2 + 1, times
+ * the same sum.  The two forms may differ in the last bits of a logit, so the
  * routing of one token can depend on how many tokens share the call.
  *   x_bf16 [T, H] bf16 bits; w_router [E, H] f32; bias [E] f32 or NULL;
  *   logits_out [T, E] f32; topk_ids [T, top_k] i32; topk_weights [T, top_k]

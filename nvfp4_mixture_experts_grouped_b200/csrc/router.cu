@@ -138,24 +138,35 @@ __global__ void __launch_bounds__(RTR_WARPS * 32)
 }
 
 // Prefill-size projection, a register-tiled FP32 GEMM.  CTA (bx, by) computes
-// the logits of experts 64bx .. 64bx+63 for tokens 128by .. 128by+127.  Thread
-// (ty, tx) = (tid / 8, tid % 8) holds 8 tokens {4ty .. 4ty+3, 64+4ty .. 64+4ty+3}
-// x 8 experts {4tx .. 4tx+3, 32+4tx .. 32+4tx+3} as 64 accumulators, so its four
-// shared-memory reads per h (one float4 each) are conflict-free across the warp.
-// H runs in chunks of 16 columns.  Every thread copies one hidden row's 16 BF16
-// and half of one router row's 16 FP32 of a chunk (four 16-byte cp.async, zero
-// fill past T or E) into its own slot of a three-deep staging ring, two chunks
-// ahead of the arithmetic; after a chunk's FMAs it waits for its own copies of
-// the next chunk and stores them transposed (h-major, hidden values widened to
-// FP32) into the other of two shared-memory buffers; one barrier per chunk.
-// Each logit is one FMA chain over h = 0 .. H-1 in order: deterministic, and
-// within gamma_H * sum_h |x_h w_h| of the exact dot product.  Rows past T and
-// experts past E are not stored.  E % 4 == 0, H % 16 == 0.
+// the logits of experts 64bx .. 64bx+63 for tokens 128by .. 128by+127 with two
+// groups of 128 threads: group g takes the chunks of 16 columns of H with
+// index = g mod 2, so each SM runs twice the warps for the same tile.  In a
+// group, thread (ty, tx) = (l / 8, l % 8) holds 8 tokens {4ty .. 4ty+3,
+// 64+4ty .. 64+4ty+3} x 8 experts {4tx .. 4tx+3, 32+4tx .. 32+4tx+3} as 64
+// accumulators, so its four shared-memory reads per h (one float4 each) are
+// conflict-free across the warp.  Every thread copies one hidden row's 16 BF16
+// and half of one router row's 16 FP32 of its group's chunk (four 16-byte
+// cp.async, zero fill past T or E) into its own slot of a three-deep staging
+// ring, two chunks ahead of the arithmetic; after a chunk's FMAs it waits for
+// its own copies of the next one and stores them transposed (h-major, hidden
+// values widened to FP32) into the other of its group's two buffers; one
+// barrier per pair of chunks.  Each logit is the even-chunk FMA chain plus the
+// odd-chunk chain (columns in order within each), added once: deterministic,
+// and within gamma_(H/2+1) * sum_h |x_h w_h| of the exact dot product.  Rows
+// past T and experts past E are not stored.  E % 4 == 0, H % 32 == 0.
 constexpr int RTT_BM = 128;    // tokens per CTA
 constexpr int RTT_BN = 64;     // experts per CTA
 constexpr int RTT_BK = 16;     // columns of H per chunk
 constexpr int RTT_STAGES = 3;  // staging ring depth (copies run two chunks ahead)
-constexpr int RTT_THREADS = (RTT_BM / 8) * (RTT_BN / 8);
+constexpr int RTT_GROUP = (RTT_BM / 8) * (RTT_BN / 8);  // threads per K group
+constexpr int RTT_KG = 2;                                // K groups
+constexpr int RTT_THREADS = RTT_KG * RTT_GROUP;
+struct RttSmem {
+    float x[RTT_KG][2][RTT_BK][RTT_BM];
+    float w[RTT_KG][2][RTT_BK][RTT_BN];
+    uint4 stage[RTT_STAGES][RTT_THREADS][4];  // per thread: 32 B hidden, 32 B router
+};
+static_assert(sizeof(float) * RTT_BM * RTT_BN <= sizeof(RttSmem::x), "the final sum reuses the hidden buffers");
 
 __device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, bool valid) {
     const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
@@ -165,29 +176,29 @@ __device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, b
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
-__global__ void __launch_bounds__(RTT_THREADS)
+__global__ void __launch_bounds__(RTT_THREADS, 2)
     k_router_logits_tiled(const uint16_t* __restrict__ x, const float* __restrict__ w, int T, int H, int E,
                           float* __restrict__ logits) {
-    __shared__ __align__(16) float s_x[2][RTT_BK][RTT_BM];
-    __shared__ __align__(16) float s_w[2][RTT_BK][RTT_BN];
-    __shared__ __align__(16) uint4 s_stage[RTT_STAGES][RTT_THREADS][4];  // per thread: 32 B hidden, 32 B router
+    extern __shared__ __align__(16) unsigned char rtt_raw[];
+    RttSmem& sm = *reinterpret_cast<RttSmem*>(rtt_raw);
     const int tid = threadIdx.x;
+    const int g = tid / RTT_GROUP, l = tid % RTT_GROUP;
     const int e0 = blockIdx.x * RTT_BN;
     const int64_t t0 = (int64_t)blockIdx.y * RTT_BM;
-    // copy roles: hidden row t0 + tid, all 16 columns of a chunk; router row
-    // e0 + tid % 64, columns 8 (tid / 64) .. + 7 of a chunk
-    const bool x_ok = t0 + tid < T;
-    const uint16_t* xrow = x + (x_ok ? t0 + tid : 0) * (int64_t)H;
-    const int we = tid % RTT_BN, wh = (tid / RTT_BN) * 8;
+    // copy roles within the group: hidden row t0 + l, all 16 columns of a chunk;
+    // router row e0 + l % 64, columns 8 (l / 64) .. + 7 of a chunk
+    const bool x_ok = t0 + l < T;
+    const uint16_t* xrow = x + (x_ok ? t0 + l : 0) * (int64_t)H;
+    const int we = l % RTT_BN, wh = (l / RTT_BN) * 8;
     const bool w_ok = e0 + we < E;
     const float* wrow = w + (int64_t)(w_ok ? e0 + we : 0) * H + wh;
-    const int nk = H / RTT_BK;
-    // chunk kc's copies into ring slot kc % 3, one commit group per chunk (an
-    // empty group past the last chunk keeps the group count uniform)
-    auto issue = [&](int kc) {
-        if (kc < nk) {
-            uint4* st = s_stage[kc % RTT_STAGES][tid];
-            const int h0 = kc * RTT_BK;
+    const int nq = H / (RTT_KG * RTT_BK);  // chunks per group
+    // the group's chunk q (column chunk KG q + g) into ring slot q % 3, one
+    // commit group per chunk (an empty group past the last keeps the count uniform)
+    auto issue = [&](int q) {
+        if (q < nq) {
+            uint4* st = sm.stage[q % RTT_STAGES][tid];
+            const int h0 = (RTT_KG * q + g) * RTT_BK;
             cp_async16_zfill(st + 0, xrow + h0, x_ok);
             cp_async16_zfill(st + 1, xrow + h0 + 8, x_ok);
             cp_async16_zfill(st + 2, wrow + h0, w_ok);
@@ -195,21 +206,21 @@ __global__ void __launch_bounds__(RTT_THREADS)
         }
         cp_async_commit();
     };
-    // this thread's staged chunk kc, transposed into buffer buf
-    auto transpose = [&](int kc, int buf) {
-        const uint4* st = s_stage[kc % RTT_STAGES][tid];
+    // this thread's staged chunk q, transposed into its group's buffer buf
+    auto transpose = [&](int q, int buf) {
+        const uint4* st = sm.stage[q % RTT_STAGES][tid];
         const uint4 x0 = st[0], x1 = st[1], w0 = st[2], w1 = st[3];
         const uint32_t u[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            s_x[buf][2 * i][tid] = bf16lo(u[i]);      // column 2i of the chunk
-            s_x[buf][2 * i + 1][tid] = bf16hi(u[i]);  // column 2i + 1
+            sm.x[g][buf][2 * i][l] = bf16lo(u[i]);      // column 2i of the chunk
+            sm.x[g][buf][2 * i + 1][l] = bf16hi(u[i]);  // column 2i + 1
         }
         const uint32_t f[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) s_w[buf][wh + i][we] = __uint_as_float(f[i]);
+        for (int i = 0; i < 8; ++i) sm.w[g][buf][wh + i][we] = __uint_as_float(f[i]);
     };
-    const int ty = tid / 8, tx = tid % 8;
+    const int ty = l / 8, tx = l % 8;
     float acc[8][8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
@@ -220,17 +231,17 @@ __global__ void __launch_bounds__(RTT_THREADS)
     cp_async_wait_1();  // chunk 0 has landed (chunk 1 may be in flight)
     transpose(0, 0);
     __syncthreads();
-    for (int kc = 0; kc < nk; ++kc) {
-        const int buf = kc & 1;
-        // ring slot (kc + 2) % 3 was last read by this thread's transpose of
-        // chunk kc - 1, before the previous barrier
-        issue(kc + 2);
+    for (int q = 0; q < nq; ++q) {
+        const int buf = q & 1;
+        // ring slot (q + 2) % 3 was last read by this thread's transpose of
+        // chunk q - 1, before the previous barrier
+        issue(q + 2);
 #pragma unroll
         for (int kk = 0; kk < RTT_BK; ++kk) {
-            const float4 a0 = *reinterpret_cast<const float4*>(&s_x[buf][kk][4 * ty]);
-            const float4 a1 = *reinterpret_cast<const float4*>(&s_x[buf][kk][64 + 4 * ty]);
-            const float4 b0 = *reinterpret_cast<const float4*>(&s_w[buf][kk][4 * tx]);
-            const float4 b1 = *reinterpret_cast<const float4*>(&s_w[buf][kk][32 + 4 * tx]);
+            const float4 a0 = *reinterpret_cast<const float4*>(&sm.x[g][buf][kk][4 * ty]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&sm.x[g][buf][kk][64 + 4 * ty]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&sm.w[g][buf][kk][4 * tx]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&sm.w[g][buf][kk][32 + 4 * tx]);
             const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -239,12 +250,27 @@ __global__ void __launch_bounds__(RTT_THREADS)
                 for (int j = 0; j < 8; ++j) acc[i][j] = __fmaf_rn(a[i], b[j], acc[i][j]);
         }
         // the other buffer was last read in the previous chunk, before the barrier
-        if (kc + 1 < nk) {
-            cp_async_wait_1();  // chunk kc + 1 has landed (chunk kc + 2 may be in flight)
-            transpose(kc + 1, buf ^ 1);
+        if (q + 1 < nq) {
+            cp_async_wait_1();  // chunk q + 1 has landed (chunk q + 2 may be in flight)
+            transpose(q + 1, buf ^ 1);
         }
         __syncthreads();
     }
+    // the odd-chunk sums through shared memory (the hidden buffers, free after
+    // the last barrier), added to the even-chunk sums in that order
+    float* red = &sm.x[0][0][0][0];
+    if (g == 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) red[(i * 8 + j) * RTT_GROUP + l] = acc[i][j];
+    }
+    __syncthreads();
+    if (g == 1) return;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = __fadd_rn(acc[i][j], red[(i * 8 + j) * RTT_GROUP + l]);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t t = t0 + (i < 4 ? 4 * ty + i : 64 + 4 * ty + (i - 4));
@@ -275,7 +301,9 @@ nvfp4moe_status launch_router_topk(const uint16_t* x, const float* w, const floa
     if (router_uses_tiled(T, E)) {
         // at least one wave of 128 x 64 tiles
         const dim3 tgrid((unsigned)ceil_div((int64_t)E, (int64_t)RTT_BN), (unsigned)ceil_div((int64_t)T, (int64_t)RTT_BM));
-        k_router_logits_tiled<<<tgrid, RTT_THREADS, 0, stream>>>(x, w, T, H, E, logits);
+        NVFP4MOE_CUDA(cudaFuncSetAttribute(k_router_logits_tiled, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)sizeof(RttSmem)));
+        k_router_logits_tiled<<<tgrid, RTT_THREADS, sizeof(RttSmem), stream>>>(x, w, T, H, E, logits);
         NVFP4MOE_CHECK_LAUNCH("router projection kernel");
         return launch_route(logits, bias, T, E, n_group, topk_group, top_k, rsf, renorm, ids, wts, stream);
     }

@@ -5,9 +5,9 @@ Logits: FP32 against the float64 oracle within the rounding bound of the
 kernel's fixed summation order, plus the oracle's own one rounding to FP32.
 Small token counts: a chain of at most H/64 FMAs per lane, a 5-level butterfly
 and the in-order sum of the K slices, |err| <= (H/64 + 6) * 2^-24 * sum|x_h w_h|.
-Token counts that fill a wave of 128 x 64 tiles (the tiled projection): one FMA
-chain over all H columns, |err| <= gamma_H * sum|x_h w_h|, gamma_H =
-H 2^-24 / (1 - H 2^-24).  At those sizes the logits are compared on sampled
+Token counts that fill a wave of 128 x 64 tiles (the tiled projection): an FMA
+chain over the even 16-column chunks plus one over the odd chunks, added once,
+|err| <= gamma_n * sum|x_h w_h|, n = H/2 + 1, gamma_n = n 2^-24 / (1 - n 2^-24).  At those sizes the logits are compared on sampled
 tokens, at least eight from every 128-token tile, on all experts.  Routing:
 bit-exact against the oracle's routing of the kernel's own logits (ids, order,
 weight bits), which is also what moe_route gives on them."""
@@ -53,7 +53,8 @@ def logit_bound_units(T, H, E):
     """The kernel's error bound in units of 2^-24 * sum|x_h w_h|, plus one for
     the oracle's rounding of the float64 sum to FP32."""
     if uses_tiled(T, E):
-        return H / (1.0 - H * U) + 1.0
+        n = H / 2 + 1
+        return n / (1.0 - n * U) + 1.0
     return H / 64 + 7
 
 
