@@ -174,6 +174,7 @@ def test_error_string_is_text():
     ((16, 4096, 256, 7, 4, 8, 64), 3),   # E % n_group
     ((16, 4096, 256, 8, 4, 33, 64), 3),  # top_k > 32
     ((-2, 4096, 256, 8, 4, 8, 64), 1),   # negative T
+    ((65535 * 128 + 1, 4096, 256, 8, 4, 8, 1 << 30), 1),  # T above the tiled projection's grid
     ((33, 4096, 256, 8, 4, 8, 8), 6),    # workspace below 4 bytes per 16 tokens
 ])
 def test_router_topk_rejects_bad_arguments_before_launch(args, expect):
