@@ -36,8 +36,9 @@ __global__ void __launch_bounds__(PERM_CHUNK)
 }
 
 // ---------------------------------------------------------------------------
-// 2. per-expert scan over chunks, expert offsets, tile list (256-row pair tiles
-//    of the tcgen05 path), active list
+// 2. per-expert scan over chunks, expert offsets, tile list (tiles of
+//    plan.tile_rows rows: 128 for the single-CTA GEMM form, 256 for the CTA-pair
+//    form), active list
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp, int& total) {
     // blockDim.x == 1024: a shuffle scan inside each warp, then over the 32 warp totals

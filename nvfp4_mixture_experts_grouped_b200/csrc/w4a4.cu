@@ -6,9 +6,12 @@
 // W4A4 NVFP4 on native FP4 tensor cores) and "Why a unit activation scale".
 // Expert MLP: "MiMo-V2.6-Flash -- REAP-50", "Pruning Method" 1.
 //
-// One persistent kernel per projection, one CTA per SM computing 128 x 256
-// output tiles (128 token rows of one expert x 256 weight rows) with the
-// single-CTA form of the MMA (cta_group::1).  Per CTA:
+// One persistent kernel per projection in one of two tile forms, chosen per
+// call: one CTA per SM computing 128 x 256 output tiles (128 token rows of one
+// expert x 256 weight rows) with the single-CTA MMA (cta_group::1) when the
+// experts average fewer than 1024 rows, else CTA pairs computing 256 x 256
+// tiles with the pair MMA (cta_group::2), each CTA holding half of the tile's A
+// and B rows.  Described here for the single-CTA form; per CTA:
 //   warp 0      TMA producer: the tile's A rows and both 128-row halves of its B
 //               rows (SWIZZLE_128B tensor maps) and their block-scale atoms (1-D
 //               bulk copies) into a 4-stage shared-memory ring guarded by
